@@ -1,0 +1,507 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 WKV operator.
+
+One step = one pass of the whole hot path over one batch of each workload:
+    RWKV-4 forward            B=8,  T=1024, C=768            fp32
+    RWKV-6 bidirectional fwd  B=32, T=196,  H=12, N=64       fp32
+    RWKV-6 causal fwd         B=8,  T=4096, H=32, N=64       bf16 r/k/v/w, fp32 state/y
+    RWKV-6 bidirectional bwd  B=32, T=196,  H=12, N=64       fp32 (dr, dk, dv, dw, du)
+Metric: WKV tokens per second (sum of B*T over the four launches per step),
+whole job (all ranks).  Inputs are seeded synthetic data resident in HBM when
+the timed region starts; the step's working set (~1.2 GB) is far larger than
+the 126 MB L2, so every kernel starts cold.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+For N > 1 launch under torchrun; every rank runs the same per-GPU work on its
+own data (weak scaling, no collective on the data path) and the step time is
+the maximum over ranks.  `--impl reference` times the double-precision CPU
+oracle (the only reference this operator has) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "WKV tokens/sec/GPU and % of roofline (HBM GB/s or FP32/TC util) vs CPU oracle"
+UNIT = "tokens/s"
+WORKLOAD_NAME = ("wkv-hot-path step: wkv4_fwd B8xT1024xC768 f32 + wkv6_bidir_fwd B32xT196xH12 f32 + "
+                 "wkv6_fwd_bf16 B8xT4096xH32 + wkv6_bwd(bidir) B32xT196xH12 f32, N=64")
+STEP_WORKLOADS = ["wkv4_f32_b8t1024c768", "wkv6_bidir_f32_b32t196h12", "wkv6_causal_bf16_b8t4096h32",
+                  "wkv6_bidir_bwd_f32_b32t196h12"]
+N = 64
+L2_BYTES = 126 * 1024 * 1024
+FP32_LANES_PER_SM, SMS, SM_MAX_MHZ = 128, 148, 1965.0
+FP32_PEAK_TFLOPS = SMS * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12   # 74.4 (FMA = 2 flop)
+FALLBACK_HBM_GBS = 6650.0
+
+# Algorithmic work per unit (a unit is one token of one head for RWKV-6, one
+# (token, channel) for RWKV-4).  Bytes: inputs read once + outputs written once.
+# Flops: RWKV-6 forward 5 N^2 per direction (state update 3 N^2 + readout 2 N^2),
+# backward 14 N^2 per direction; RWKV-4 ~4 exp + 12 flop (HBM bound).
+ALG = {
+    "wkv4_f32_b8t1024c768": dict(bytes_per_unit=3 * 4, flops_per_unit=16, bound="hbm"),
+    "wkv6_bidir_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=10 * N * N, bound="alu"),
+    "wkv6_causal_bf16_b8t4096h32": dict(bytes_per_unit=4 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="alu"),
+    "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="alu"),
+}
+ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
+         "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd"}
+LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
+            "wkv6_bidir_bwd_f32_b32t196h12": 2}   # the backward adds a deterministic du reduction
+
+
+def units_of(name: str, x) -> int:
+    if name.startswith("wkv4"):
+        return x.B * x.T * x.C
+    return x.B * x.T * x.H
+
+
+def tokens_of(x) -> int:
+    return x.B * x.T
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_group(backend: str, world: int):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity for one rank)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, dist=None, device=None) -> float:
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(dist=None):
+    if dist is not None:
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- peaks, clocks, traffic
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    import glob
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_rnn_wkv6_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(name: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernels have not changed since."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    e = d.get("kernels", {}).get(name)
+    return None if e is None else float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples nvidia-smi during the timed region (SM clock, throttle reasons)."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- native (CUDA) arm
+
+class DeviceWorkload:
+    """Inputs resident in HBM, outputs and workspace preallocated; run() enqueues the ABI call."""
+
+    def __init__(self, name: str, seed: int):
+        import numpy as np
+        import torch
+        from linear_attention_rnn_wkv6_b200 import synth
+        self.name = name
+        self.kind, self.x = synth.make_workload(name, seed=seed)
+        x = self.x
+
+        def dev(a):
+            a = np.ascontiguousarray(a)
+            if a.dtype == np.uint16:
+                a = a.view(np.int16)
+            return torch.from_numpy(a).cuda()
+
+        self.host_inputs = {}
+        names = ("k", "v", "w", "u") if self.kind == "wkv4_fwd" else ("r", "k", "v", "w", "u") + (
+            ("dy",) if self.kind == "wkv6_bwd_bidir" else ())
+        self.inputs = {n: dev(getattr(x, n)) for n in names}
+        shape = (x.B, x.T, x.C)
+        if self.kind == "wkv6_bwd_bidir":
+            self.outputs = [torch.empty(shape, device="cuda") for _ in range(4)] + [torch.empty(x.C, device="cuda")]
+            import linear_attention_rnn_wkv6_b200 as wkv
+            self.ws_bytes = wkv.wkv6_bwd_workspace_bytes(x.B, x.T, x.C, x.H, 1)
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        else:
+            self.outputs = [torch.empty(shape, device="cuda")]
+        self.units = units_of(name, x)
+        self.tokens = tokens_of(x)
+
+    def run(self, stream, inputs=None, outputs=None):
+        import linear_attention_rnn_wkv6_b200 as wkv
+        x, i = self.x, (inputs or self.inputs)
+        o = outputs or self.outputs
+        s = stream.cuda_stream
+        if self.kind == "wkv4_fwd":
+            wkv.wkv4_fwd(x.B, x.T, x.C, i["k"], i["v"], i["w"], i["u"], o[0], s)
+        elif self.kind == "wkv6_bidir_fwd":
+            wkv.wkv6_bidir_fwd(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], o[0], s)
+        elif self.kind == "wkv6_fwd_bf16":
+            wkv.wkv6_fwd_bf16(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], o[0], s)
+        elif self.kind == "wkv6_bwd_bidir":
+            wkv.wkv6_bwd(x.B, x.T, x.C, x.H, 1, i["r"], i["k"], i["v"], i["w"], i["u"], i["dy"], *o,
+                         self.ws, self.ws_bytes, s)
+        else:
+            raise ValueError(self.kind)
+
+
+class HostSide:
+    """Pinned host copies of one workload's inputs and outputs for the end-to-end measurement."""
+
+    def __init__(self, dw: DeviceWorkload):
+        import torch
+        self.dw = dw
+        self.h_in = {n: t.cpu().pin_memory() for n, t in dw.inputs.items()}
+        self.d_in = {n: torch.empty_like(t) for n, t in dw.inputs.items()}
+        self.d_out = [torch.empty_like(t) for t in dw.outputs]
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dw.outputs]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def run(self, stream):
+        import torch
+        with torch.cuda.stream(stream):
+            for n, t in self.h_in.items():
+                self.d_in[n].copy_(t, non_blocking=True)
+            self.dw.run(stream, inputs=self.d_in, outputs=self.d_out)
+            for h, d in zip(self.h_out, self.d_out):
+                h.copy_(d, non_blocking=True)
+
+
+def run_native(args, rank, world, local):
+    import torch
+    import linear_attention_rnn_wkv6_b200 as wkv
+    torch.cuda.set_device(local)
+    dist = init_group("nccl", world)
+    dev = torch.device("cuda", local)
+    wkv.load()
+    seed = 1000 * rank
+    wls = [DeviceWorkload(n, seed) for n in STEP_WORKLOADS]
+    stream = torch.cuda.Stream()
+    tokens_per_step = sum(w.tokens for w in wls)
+
+    def step(evs=None):
+        for j, w in enumerate(wls):
+            if evs is not None:
+                evs[j][0].record(stream)
+            w.run(stream)
+            if evs is not None:
+                evs[j][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if wkv.wkv_take_device_faults() != 0:
+        raise RuntimeError("device fault word set during warm-up")
+
+    K = args.steps
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in wls]
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for k in range(K):
+            step(kev[k])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(dist)
+    elapsed_ms = t0.elapsed_time(t1)
+    per_kernel_ms = [sum(kev[k][j][0].elapsed_time(kev[k][j][1]) for k in range(K)) / K for j in range(len(wls))]
+    if wkv.wkv_take_device_faults() != 0:
+        raise RuntimeError("device fault word set during the timed region")
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
+    ms_per_step = elapsed_ms / K
+    value = tokens_per_step * world * K / (elapsed_ms / 1e3)
+
+    # end-to-end through the public API with host buffers (pinned), copies inside the timed region
+    hs = [HostSide(w) for w in wls]
+    for _ in range(max(1, min(args.warmup, 2))):
+        for h in hs:
+            h.run(stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Ke = max(1, min(K, 5))
+    barrier(dist)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Ke):
+        for h in hs:
+            h.run(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    e2e_value = tokens_per_step * world * Ke / (e2e_ms / 1e3)
+    h2d = sum(h.h2d for h in hs)
+    d2h = sum(h.d2h for h in hs)
+
+    if rank == 0:
+        hbm, hbm_src = load_peaks()
+        kernels = {}
+        for j, w in enumerate(wls):
+            a = ALG[w.name]
+            t_s = per_kernel_ms[j] / 1e3
+            alg_bytes = a["bytes_per_unit"] * w.units
+            alg_flops = a["flops_per_unit"] * w.units
+            if a["bound"] == "hbm":
+                achieved, peak, unit = alg_bytes / t_s / 1e9, hbm, "GB/s"
+                peak_src = f"{hbm_src} HBM copy bandwidth"
+            else:
+                achieved, peak, unit = alg_flops / t_s / 1e12, FP32_PEAK_TFLOPS, "TFLOP/s"
+                peak_src = "derived FP32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz"
+            kernels[w.name] = {
+                "entry": ENTRY[w.name], "launches": LAUNCHES[w.name], "ms": round(per_kernel_ms[j], 4),
+                "tokens_per_s": round(w.tokens / t_s, 1), "units": w.units,
+                "alg_bytes": alg_bytes, "alg_flops": alg_flops,
+                "hbm_gbs": round(alg_bytes / t_s / 1e9, 1), "fp32_tflops": round(alg_flops / t_s / 1e12, 2),
+                "bound": a["bound"], "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": unit,
+                "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                "share": round(per_kernel_ms[j] / sum(per_kernel_ms), 4),
+            }
+        dom = max(kernels, key=lambda n: kernels[n]["ms"])
+        d = kernels[dom]
+        traffic = recorded_traffic(dom)
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs on the causal workload)",
+            "data": "synthetic (seeded splitmix64 + Box-Muller, rank-dependent seed)",
+            "config": {"workload": WORKLOAD_NAME, "tokens_per_step_per_gpu": tokens_per_step,
+                       "l2": "inputs larger than L2: step working set ~1.2 GB > 126 MB L2, no explicit flush",
+                       "parallelism": f"replicated weak scaling x{world} (independent problems per rank)"},
+            "roofline": {"kernel": dom, "bound": "hbm" if d["bound"] == "hbm" else "alu",
+                         "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
+                         "traffic": traffic, "peak_source": d["peak_source"]},
+            "kernels": kernels,
+            "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": Ke,
+                    "note": "public C-ABI calls; pinned host inputs copied in and outputs copied out every step"},
+            "gpu_launches": K * sum(LAUNCHES[w.name] for w in wls),
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+def _oracle_unit_seconds(name: str, x, max_units: int, budget_s: float):
+    """Time the oracle on up to max_units units of workload `name` within ~budget_s.
+
+    Returns (seconds per unit, units timed, description)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    done, spent = 0, 0.0
+    if name.startswith("wkv4"):
+        # a unit is one (b, channel) series of T tokens; time contiguous channel blocks
+        blk = 16
+        for i in range(max_units // blk):
+            b, c0 = i % x.B, (i * blk) % x.C
+            k, v = x.k[b:b + 1, :, c0:c0 + blk], x.v[b:b + 1, :, c0:c0 + blk]
+            t = time.perf_counter()
+            oracle.wkv4_fwd(k, v, x.w[c0:c0 + blk], x.u[c0:c0 + blk])
+            spent += time.perf_counter() - t
+            done += blk
+            if spent > budget_s:
+                break
+        return spent / (done * x.T), done, f"{done} channels x T={x.T}"
+    sl_units = []
+    for i in range(max_units):
+        sl_units.append(((i * 7 + 3) % x.B, (i * 5 + 1) % x.H))
+    for b, h in sl_units:
+        sl = slice(h * N, (h + 1) * N)
+        r, k, v, w = (x.as_f64(n)[b:b + 1, :, sl] for n in ("r", "k", "v", "w"))
+        u = x.u[sl].astype(np.float64)
+        t = time.perf_counter()
+        if name == "wkv6_bidir_bwd_f32_b32t196h12":
+            oracle.wkv6_bwd(r, k, v, w, u, x.dy[b:b + 1, :, sl].astype(np.float64), H=1, bidirectional=True)
+        else:
+            oracle.wkv6_fwd(r, k, v, w, u, H=1, bidirectional="bidir" in name)
+        spent += time.perf_counter() - t
+        done += 1
+        if spent > budget_s:
+            break
+    # per-unit time: one (b, h) slice covers T token-heads
+    return spent / (done * x.T), done, f"{done} (b,h) slices x T={x.T}"
+
+
+def cpu_baseline(seconds_total: float = 12.0):
+    """The oracle, single-threaded, on a bounded sample of each workload, scaled to the full step."""
+    from linear_attention_rnn_wkv6_b200 import synth
+    est_step_s, samples = 0.0, []
+    tokens = 0
+    for name in STEP_WORKLOADS:
+        kind, x = synth.make_workload(name, seed=0)
+        per_unit_s, n, desc = _oracle_unit_seconds(name, x, max_units=4096, budget_s=seconds_total / 4)
+        units = units_of(name, x)
+        est_step_s += per_unit_s * units
+        tokens += tokens_of(x)
+        samples.append(f"{name}: {desc}")
+    return {"value": round(tokens / est_step_s, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "; ".join(samples) + "; time per unit scaled to the full step",
+            "est_step_s": round(est_step_s, 3)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    t_start = time.perf_counter()
+    from linear_attention_rnn_wkv6_b200 import synth
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = []
+    tokens = sum(tokens_of(synth.make_workload(n, 0)[1]) for n in STEP_WORKLOADS)
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(budget)
+        if i >= args.warmup:
+            per_step.append(cb["est_step_s"])
+    est = statistics.median(per_step)
+    value = tokens / est
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs)",
+        "config": {"workload": WORKLOAD_NAME,
+                   "note": "double-precision CPU oracle, single thread; each step times a bounded sample and "
+                           "scales it to the full workload"},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": round(time.perf_counter() - t_start, 1),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget of the cpu_baseline leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    if world != args.gpus and world == 1 and args.gpus > 1:
+        ap.error("for --gpus > 1 launch under torchrun (one process per GPU)")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_native(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * wkv.h -- C ABI of libwkv.so, the B200 (sm_100a) RWKV WKV operator.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers: CUDA device memory owned by the caller, contiguous, row-major,
+ *    16-byte aligned.  [B,T,C] arrays hold token t of batch b, channel c at
+ *    ((b*T + t)*C + c); channel c = h*N + i belongs to head h, row i.
+ *    u and du are [C] (= [H][N]).  Outputs are fully overwritten, never
+ *    accumulated into.  Inputs and outputs must not overlap.
+ *  - Head size N = C / H.  This build supports N == 64 (WKV_ERR_HEADSIZE otherwise).
+ *  - stream: a cudaStream_t (NULL = legacy default stream).  Every call only
+ *    enqueues work on that stream and returns; none synchronises, none
+ *    allocates device memory (scratch is passed in by the caller).
+ *  - Return value: WKV_OK (0) or a negative WKV_ERR_* code.  On an argument
+ *    error nothing is launched and no output is touched.  WKV_ERR_CUDA means
+ *    the launch itself failed (cudaGetLastError after the launch).
+ *  - Device-side waits (on TMA completion) are bounded by a one-second limit;
+ *    a wait that runs out makes the kernel stop early and records
+ *    WKV_FAULT_TIMEOUT in a device word that wkv_take_device_faults() reads.
+ *  - B == 0 or T == 0 is a valid empty problem: nothing is launched, except
+ *    that wkv6_bwd zeroes du when B*T == 0.
+ *
+ * RWKV-6 log-decay
+ * ----------------
+ * The decay argument w of the RWKV-6 entry points is the log-decay
+ * ew = -exp(w_raw) <= 0 that the reference's autograd wrapper hands its kernel
+ * ("How the WKV (Weighted Key Value) Mechanism in RWKV Processes Images",
+ * CUDA Wrapper (Image Side)); the kernel exponentiates it on the fly
+ * ("How Custom CUDA Kernels (wkv6_cuda.cu) Implement the WKV Operation",
+ * Kernel Architecture and Launch Configuration: w is "exponentiated
+ * on-the-fly"), so state row i of head h decays by d_t[i] = exp(ew_t[h*N+i]).
+ */
+#ifndef WKV_H_
+#define WKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *wkv_stream_t; /* identical to cudaStream_t */
+
+enum {
+    WKV_OK = 0,
+    WKV_ERR_ARG = -1,        /* B, T < 0; C, H < 1; C != H*N; a required pointer is NULL */
+    WKV_ERR_HEADSIZE = -2,   /* N = C/H is not a compiled head size (64) */
+    WKV_ERR_ALIGN = -3,      /* a pointer is not 16-byte aligned */
+    WKV_ERR_WORKSPACE = -4,  /* workspace NULL or smaller than the *_workspace_bytes query */
+    WKV_ERR_CUDA = -5,       /* a CUDA runtime call or the launch failed */
+    WKV_ERR_DEVICE = -6,     /* the current device is not sm_100 (B200) */
+    WKV_ERR_TOO_LARGE = -7   /* a size exceeds a documented limit (B*T*C >= 2^31 elements) */
+};
+
+/* Bits of the device fault word (see wkv_take_device_faults). */
+#define WKV_FAULT_TIMEOUT 0x1u   /* a bounded device-side wait ran out */
+
+/*
+ * wkv6_fwd -- causal RWKV-6 WKV forward, fp32 inputs, fp32 state and output.
+ *
+ * Operation ("RWKV Architecture: How Receptance Weighted Key Value Combines RNN
+ * Linear Inference with Transformer Parallel Training", RWKV-5 "Eagle" matrix
+ * state and RWKV-6 "Finch" dynamic decay; "How Custom CUDA Kernels
+ * (wkv6_cuda.cu) ...", Past-to-Future Pass, y += r*(u*x + s) with s = s*w + x):
+ * per (b, h), with S_{-1} = 0 (N x N),
+ *     y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),   S_t = diag(exp(w_t)) S_{t-1} + k_t^T v_t.
+ * Arguments follow the reference launcher cuda_forward(B, T, C, H, r, k, v, w, u, y)
+ * ("How Custom CUDA Kernels ...", Kernel Architecture and Launch Configuration).
+ *   r, k, v, w : [B,T,C] float, inputs (w = log-decay, see above)
+ *   u          : [C] float, bonus for the current token
+ *   y          : [B,T,C] float, output
+ */
+int wkv6_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v,
+             const float *w, const float *u, float *y, wkv_stream_t stream);
+
+/*
+ * wkv6_fwd_bf16 -- wkv6_fwd with bfloat16 r, k, v, w (raw IEEE bf16 bit patterns,
+ * uint16_t); u, the state and y stay fp32.  Same operation and layout.
+ */
+int wkv6_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t *k,
+                  const uint16_t *v, const uint16_t *w, const float *u, float *y, wkv_stream_t stream);
+
+/*
+ * wkv6_bidir_fwd -- bidirectional RWKV-6 WKV forward, fp32 ("How Custom CUDA
+ * Kernels (wkv6_cuda.cu) ...", Forward Pass Implementation: a future-to-past
+ * pass without the bonus, then a past-to-future pass that adds the bonus u):
+ *     y_t = r_t S^b_{t+1} + r_t (S_{t-1} + diag(u) k_t^T v_t),
+ *     S^b_t = diag(exp(w_t)) S^b_{t+1} + k_t^T v_t,  S^b_T = 0,
+ * i.e. every other token contributes once with the decay accumulated between
+ * the two positions and the current token once with u.  Same arguments as wkv6_fwd.
+ */
+int wkv6_bidir_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v,
+                   const float *w, const float *u, float *y, wkv_stream_t stream);
+
+/*
+ * wkv6_bwd -- gradients of L = sum(dy * y) for wkv6_fwd (bidirectional == 0) or
+ * wkv6_bidir_fwd (bidirectional != 0), fp32 ("How Custom CUDA Kernels
+ * (wkv6_cuda.cu) ...", Backward Pass Gradient Computation; arguments follow the
+ * reference backward(B, T, C, H, r, k, v, ew, u, gy, gr, gk, gv, gw, gu)).
+ *   r, k, v, w, dy     : [B,T,C] float, inputs
+ *   u                  : [C] float, input
+ *   dr, dk, dv, dw     : [B,T,C] float, outputs (dw is the gradient with respect
+ *                        to the log-decay w passed in)
+ *   du                 : [C] float, output, summed over B and T in a fixed
+ *                        order (bitwise reproducible run to run)
+ *   workspace          : device scratch of at least wkv6_bwd_workspace_bytes(...)
+ *                        bytes, 16-byte aligned, owned by the caller; its content
+ *                        on entry is ignored and on exit undefined.
+ */
+int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, const float *k,
+             const float *v, const float *w, const float *u, const float *dy, float *dr, float *dk,
+             float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes,
+             wkv_stream_t stream);
+
+/* Scratch bytes wkv6_bwd needs for these sizes (B*C floats of per-batch du partials). */
+size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional);
+
+/*
+ * wkv4_fwd -- RWKV-4 WKV forward, fp32 ("RWKV Architecture ...", The
+ * Fundamental Mathematical Duality and The Recurrent Inference Formulation):
+ *     y_t = (sum_{s<t} e^{-(t-1-s) w + k_s} v_s + e^{u + k_t} v_t)
+ *         / (sum_{s<t} e^{-(t-1-s) w + k_s}     + e^{u + k_t}),
+ * evaluated as the a/b recurrence carried in log space with a running maximum
+ * exponent (yarian.com RWKV overview, 3.2: log-space time decay).
+ *   k, v : [B,T,C] float inputs;  w : [C] float, w >= 0 (per-step decay e^{-w});
+ *   u    : [C] float bonus;       y : [B,T,C] float output.
+ * The receptance gate sigma(r) is applied outside the operator, as on the page.
+ */
+int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u,
+             float *y, wkv_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *wkv_status_string(int status);
+
+/*
+ * wkv_take_device_faults -- synchronise the current device, copy the device
+ * fault word (WKV_FAULT_* bits set by kernels whose bounded waits ran out) to
+ * *faults, and clear it.  Returns WKV_OK or WKV_ERR_CUDA.  Diagnostic call:
+ * unlike the entry points above it does synchronise.
+ */
+int wkv_take_device_faults(unsigned *faults);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int wkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_H_ */

@@ -1,0 +1,150 @@
+"""B200-native RWKV WKV operator: thin Python binding of libwkv.so.
+
+Every function here has the name and argument order of the C entry point it
+wraps (include/wkv.h) and only marshals arguments: torch tensors (or raw
+integer device addresses) become pointers, ``stream=None`` becomes the current
+torch CUDA stream, and a non-zero status raises :class:`WkvError`.  All of the
+operator's arithmetic runs in the CUDA kernels of libwkv.so; there is no CPU
+fallback.  If the library has not been built, importing the binding's entry
+points raises immediately.
+
+Build the library with ``python -m linear_attention_rnn_wkv6_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
+    "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
+    "EXPORTED_SYMBOLS", "HEAD_SIZE",
+]
+
+HEAD_SIZE = 64
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+# Every extern "C" symbol declared in include/wkv.h.
+EXPORTED_SYMBOLS = (
+    "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
+    "wkv_status_string", "wkv_take_device_faults", "wkv_version",
+)
+
+_I = ctypes.c_int
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+
+_SIGS = {
+    "wkv6_fwd": ([_I] * 4 + [_P] * 6 + [_P], _I),
+    "wkv6_fwd_bf16": ([_I] * 4 + [_P] * 6 + [_P], _I),
+    "wkv6_bidir_fwd": ([_I] * 4 + [_P] * 6 + [_P], _I),
+    "wkv6_bwd": ([_I] * 5 + [_P] * 11 + [_P, _SZ, _P], _I),
+    "wkv6_bwd_workspace_bytes": ([_I] * 5, _SZ),
+    "wkv4_fwd": ([_I] * 3 + [_P] * 5 + [_P], _I),
+    "wkv_status_string": ([_I], ctypes.c_char_p),
+    "wkv_take_device_faults": ([ctypes.POINTER(ctypes.c_uint)], _I),
+    "wkv_version": ([], _I),
+}
+
+
+class WkvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed with status {status}: {wkv_status_string(status)}")
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libwkv.so")
+
+
+def load():
+    """Load libwkv.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m linear_attention_rnn_wkv6_b200.build` "
+                               "(the WKV operator has no fallback implementation)")
+        lib = ctypes.CDLL(path)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = res
+        _LIB = lib
+    return _LIB
+
+
+def _ptr(x) -> int | None:
+    """Device address of a torch tensor (must be contiguous) or an integer address."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_contiguous():
+        raise ValueError("WKV tensors must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise WkvError(fn, status)
+
+
+def wkv6_fwd(B, T, C, H, r, k, v, w, u, y, stream=None) -> None:
+    """Causal RWKV-6 WKV forward (fp32).  See include/wkv.h."""
+    _check("wkv6_fwd", load().wkv6_fwd(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(y),
+                                       _stream(stream)))
+
+
+def wkv6_fwd_bf16(B, T, C, H, r, k, v, w, u, y, stream=None) -> None:
+    """Causal RWKV-6 WKV forward with bf16 r, k, v, w; fp32 u, state and y."""
+    _check("wkv6_fwd_bf16", load().wkv6_fwd_bf16(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
+                                                 _ptr(y), _stream(stream)))
+
+
+def wkv6_bidir_fwd(B, T, C, H, r, k, v, w, u, y, stream=None) -> None:
+    """Bidirectional RWKV-6 WKV forward (fp32)."""
+    _check("wkv6_bidir_fwd", load().wkv6_bidir_fwd(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
+                                                   _ptr(y), _stream(stream)))
+
+
+def wkv6_bwd_workspace_bytes(B, T, C, H, bidirectional) -> int:
+    return int(load().wkv6_bwd_workspace_bytes(B, T, C, H, int(bool(bidirectional))))
+
+
+def wkv6_bwd(B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, workspace, workspace_bytes,
+             stream=None) -> None:
+    """RWKV-6 WKV backward (fp32): dr, dk, dv, dw [B,T,C] and du [C]."""
+    _check("wkv6_bwd", load().wkv6_bwd(B, T, C, H, int(bool(bidirectional)), _ptr(r), _ptr(k), _ptr(v), _ptr(w),
+                                       _ptr(u), _ptr(dy), _ptr(dr), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du),
+                                       _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def wkv4_fwd(B, T, C, k, v, w, u, y, stream=None) -> None:
+    """RWKV-4 WKV forward (fp32)."""
+    _check("wkv4_fwd", load().wkv4_fwd(B, T, C, _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(y), _stream(stream)))
+
+
+def wkv_status_string(status: int) -> str:
+    return load().wkv_status_string(int(status)).decode()
+
+
+def wkv_take_device_faults() -> int:
+    """Synchronise the device and return (and clear) the WKV_FAULT_* bits."""
+    out = ctypes.c_uint(0)
+    _check("wkv_take_device_faults", load().wkv_take_device_faults(ctypes.byref(out)))
+    return int(out.value)
+
+
+def wkv_version() -> int:
+    return int(load().wkv_version())

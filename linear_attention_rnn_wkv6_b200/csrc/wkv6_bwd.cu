@@ -1,0 +1,421 @@
+// wkv6_bwd.cu -- RWKV-6 WKV backward (causal and bidirectional) for sm_100a.
+//
+// Gradients of L = sum_t dy_t . y_t for the forward in wkv6_fwd.cu ("How Custom
+// CUDA Kernels (wkv6_cuda.cu) ...", Backward Pass Gradient Computation: r, k, v,
+// u, and w in a backward-in-time and a forward-in-time part, no atomics).
+//
+// Four N x N matrices obey the same recurrence "before(next) = diag(d_t) before + outer_t":
+//   S  (causal state)      read at t as S_{t-1},    outer k_t^T v_t,   swept forward in time
+//   Gb (anti-causal adjoint) sum_{tau<t} P r dy^T, outer r_t^T dy_t,  swept forward in time
+//   G  (causal adjoint)    sum_{tau>t} P r dy^T,    outer r_t^T dy_t,  swept backward in time
+//   Sb (anti-causal state) read at t as S^b_{t+1}, outer k_t^T v_t,   swept backward in time
+// Readouts per token (primes: without the bonus):
+//   dr'_t = S dy_t (+ Sb dy_t),  dk'_t = G v_t (+ Gb v_t),  dv'_t = G^T k_t (+ Gb^T k_t)
+//   bonus: dr += u.k (v.dy), dk += u.r (v.dy), dv += (sum r u k) dy, du += r.k (v.dy)
+// Decay gradient without holding S and G together: with z_t = r_t.dr'^causal_t +
+// k_t.dk'^anti_t (forward sweep) and x_t = k_t.dk'^causal_t + r_t.dr'^anti_t
+// (backward sweep), for the log-decay ew_m
+//   dw_m = sum_{tau > m} z_tau - sum_{s >= m} x_s,
+// because each side sums r_t[i] k_s[i] P(s,t)[i] (v_s . dy_t) over the pairs
+// with m strictly between s and t (the totals of the anti-causal terms cancel).
+// The forward sweep parks z in dw; the backward sweep turns it into dw in place.
+//
+// Layout and scaled state as in wkv6_fwd.cu: one CTA per (b, h), 4 warps
+// splitting the 64 value columns, 32 registers per state per lane, TMA-staged
+// chunks of TC tokens, renorm steps bounding |L| by kTheta.
+#include "wkv_launch.cuh"
+
+namespace wkv {
+
+constexpr float kThetaB = 40.0f;
+
+template <int TC>
+struct BwdSmem {
+    float raw[2][5][TC][kHead];   // r, k, w, v, dy (TMA landing, 2 stages)
+    float Ap[TC][kHead];          // exp(L_p)
+    float ks[TC][kHead];          // k * exp(-L_{p+1})   (k on renorm steps)
+    float rs[TC][kHead];          // r * exp(-L_{p+1})   (r on renorm steps)
+    float kh[TC][kHead];          // k * exp(L_p)
+    float al[TC][kHead];          // exp(L_p + ew_p) on renorm steps
+    float vs[TC][kHead];
+    float dys[TC][kHead];
+    float pr[TC][4][kHead];       // per-warp partial sums over columns of S-type . dy
+    float pk[TC][4][kHead];       // per-warp partial sums over columns of G-type . v
+    float dvs[TC][kHead];         // dv' (complete over rows)
+    float vdy[TC];
+    float ruk[TC];
+    float u[kHead];
+    uint32_t renorm_mask;
+    alignas(8) uint64_t full[2];
+};
+
+enum { A_R = 0, A_K = 1, A_W = 2, A_V = 3, A_DY = 4 };
+
+// Reduce-scatter 8 row partials over the 4 column-group lanes (xor 16, xor 8).
+// Returns the two sums this lane keeps: rows q0 = 4*c1 + 2*c0 and q0 + 1.
+__device__ __forceinline__ void reduce_rows_over_cols(const float (&x)[8], bool c1, bool c0, float &o0,
+                                                      float &o1) {
+    float keep[4], send[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        keep[q] = c1 ? x[4 + q] : x[q];
+        send[q] = c1 ? x[q] : x[4 + q];
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) keep[q] += __shfl_xor_sync(0xffffffffu, send[q], 16);
+    float k2[2], s2[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        k2[q] = c0 ? keep[2 + q] : keep[q];
+        s2[q] = c0 ? keep[q] : keep[2 + q];
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) k2[q] += __shfl_xor_sync(0xffffffffu, s2[q], 8);
+    o0 = k2[0];
+    o1 = k2[1];
+}
+
+// Reduce-scatter 4 column partials over the 8 row-group lanes (xor 4, 2, 1);
+// the result (complete over the warp's 64 rows) is column (rg >> 1) & 3.
+__device__ __forceinline__ float reduce_cols_over_rows(const float (&yp)[4], bool b2, bool b1) {
+    float k0 = b2 ? yp[2] : yp[0];
+    float k1 = b2 ? yp[3] : yp[1];
+    const float s0 = b2 ? yp[0] : yp[2];
+    const float s1 = b2 ? yp[1] : yp[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
+    float kk = b1 ? k1 : k0;
+    const float s2 = b1 ? k0 : k1;
+    kk += __shfl_xor_sync(0xffffffffu, s2, 2);
+    kk += __shfl_xor_sync(0xffffffffu, kk, 1);
+    return kk;
+}
+
+template <int TC, bool BIDIR>
+__global__ void __launch_bounds__(128)
+wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
+                const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_v,
+                const __grid_constant__ CUtensorMap map_dy, BwdParams prm) {
+    using Smem = BwdSmem<TC>;
+    constexpr int NT = 128;
+    constexpr uint32_t kStageBytes = 5u * TC * kHead * sizeof(float);
+    extern __shared__ unsigned char smem_dyn[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~uintptr_t(127));
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = prm.T, C = prm.C, H = prm.H;
+    const int h = blockIdx.x % H;
+    const int b = blockIdx.x / H;
+    const int cbase = h * kHead;
+    const int nch = (T + TC - 1) / TC;
+    const int nchunks = 2 * nch;        // sweep A (forward in time), then sweep B
+
+    if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
+    if (tid == 0) {
+        prefetch_tensormap(&map_r);
+        prefetch_tensormap(&map_k);
+        prefetch_tensormap(&map_w);
+        prefetch_tensormap(&map_v);
+        prefetch_tensormap(&map_dy);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    auto t_lo_of = [&](int g) { return g < nch ? g * TC : T - (g - nch + 1) * TC; };
+    auto issue = [&](int g) {
+        const int s = g & 1, tl = t_lo_of(g);
+        mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+        tma_load_3d(&sm.raw[s][A_R][0][0], &map_r, cbase, tl, b, &sm.full[s]);
+        tma_load_3d(&sm.raw[s][A_K][0][0], &map_k, cbase, tl, b, &sm.full[s]);
+        tma_load_3d(&sm.raw[s][A_W][0][0], &map_w, cbase, tl, b, &sm.full[s]);
+        tma_load_3d(&sm.raw[s][A_V][0][0], &map_v, cbase, tl, b, &sm.full[s]);
+        tma_load_3d(&sm.raw[s][A_DY][0][0], &map_dy, cbase, tl, b, &sm.full[s]);
+    };
+    if (tid == 0) {
+        issue(0);
+        if (nchunks > 1) issue(1);
+    }
+
+    const int rg = lane & 7, cg = lane >> 3;
+    const int rowA = 4 * rg, rowB = 32 + 4 * rg;
+    const int jc = 16 * warp + 4 * cg;
+    const int jj = (rg >> 1) & 3;
+    const bool b2 = (rg & 4) != 0, b1 = (rg & 2) != 0;
+    const bool c1 = (cg & 2) != 0, c0 = (cg & 1) != 0;
+    const int q0 = 4 * (cg >> 1) + 2 * (cg & 1);   // rows kept by reduce_rows_over_cols: R(q0), R(q0+1)
+    auto rowq = [&](int q) { return q < 4 ? rowA + q : rowB + q - 4; };
+
+    float Ss[8][4], Gs[8][4];   // S-type and G-type states of the current sweep
+    float du_acc = 0.f;         // thread i < 64: sum_t r k (v.dy) for row i
+    float Rrun = 0.f;           // thread i < 64: running sum for dw (backward sweep)
+
+    for (int g = 0; g < nchunks; ++g) {
+        const int s = g & 1;
+        const bool sweepA = g < nch;
+        const int dir = sweepA ? 1 : -1;
+        const int tl = t_lo_of(g);
+        // sweep A: S-type always, G-type (Gb) when bidirectional;
+        // sweep B: G-type always, S-type (Sb) when bidirectional.
+        const bool hasS = sweepA || BIDIR;
+        const bool hasG = !sweepA || BIDIR;
+        if (g == 0 || g == nch) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) Ss[q][j] = Gs[q][j] = 0.f;
+        }
+        const bool ok = mbar_wait_bounded(&sm.full[s], (g >> 1) & 1);
+        if (!__syncthreads_and(ok)) {         // a bounded wait ran out: stop (fault recorded)
+            drain_two_stage(sm.full, g, nchunks);
+            return;
+        }
+
+        // ---- renorm flags ----
+        int bad = 0;
+        for (int e = tid; e < TC * kHead; e += NT) bad |= !(fabsf(sm.raw[s][A_W][e / kHead][e % kHead]) <= kThetaB / TC);
+        const int any_bad = __syncthreads_or(bad);
+        if (tid < 32) {
+            uint32_t mask = 1u << (TC - 1);
+            if (any_bad) {
+                for (int p = 0; p < TC - 1; ++p) {
+                    const int row = dir > 0 ? p : TC - 1 - p;
+                    const bool bb = !(fabsf(sm.raw[s][A_W][row][lane]) <= kThetaB / TC) ||
+                                    !(fabsf(sm.raw[s][A_W][row][lane + 32]) <= kThetaB / TC);
+                    if (__any_sync(0xffffffffu, bb)) mask |= 1u << p;
+                }
+            }
+            if (tid == 0) sm.renorm_mask = mask;
+        }
+        __syncthreads();
+        const uint32_t rmask = sm.renorm_mask;
+
+        // ---- transform (processing order p) ----
+        for (int i = tid; i < kHead; i += NT) {
+            float L = 0.f;
+            for (int p = 0; p < TC; ++p) {
+                const int row = dir > 0 ? p : TC - 1 - p;
+                const float ew = sm.raw[s][A_W][row][i];
+                const float rr = sm.raw[s][A_R][row][i];
+                const float kk = sm.raw[s][A_K][row][i];
+                const float eL = __expf(L);
+                sm.Ap[p][i] = eL;
+                sm.kh[p][i] = kk * eL;
+                if ((rmask >> p) & 1u) {
+                    sm.al[p][i] = __expf(L + ew);
+                    sm.ks[p][i] = kk;
+                    sm.rs[p][i] = rr;
+                    L = 0.f;
+                } else {
+                    L += ew;
+                    const float emL = __expf(-L);
+                    sm.ks[p][i] = kk * emL;
+                    sm.rs[p][i] = rr * emL;
+                }
+            }
+        }
+        for (int e = tid; e < TC * kHead; e += NT) {
+            const int p = e / kHead, j = e % kHead;
+            const int row = dir > 0 ? p : TC - 1 - p;
+            sm.vs[p][j] = sm.raw[s][A_V][row][j];
+            sm.dys[p][j] = sm.raw[s][A_DY][row][j];
+        }
+        for (int p = warp; p < TC; p += 4) {
+            const int row = dir > 0 ? p : TC - 1 - p;
+            float a = sm.raw[s][A_V][row][lane] * sm.raw[s][A_DY][row][lane] +
+                      sm.raw[s][A_V][row][lane + 32] * sm.raw[s][A_DY][row][lane + 32];
+            float c = sm.raw[s][A_R][row][lane] * sm.u[lane] * sm.raw[s][A_K][row][lane] +
+                      sm.raw[s][A_R][row][lane + 32] * sm.u[lane + 32] * sm.raw[s][A_K][row][lane + 32];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, o);
+                c += __shfl_xor_sync(0xffffffffu, c, o);
+            }
+            if (lane == 0) {
+                sm.vdy[p] = a;
+                sm.ruk[p] = c;
+            }
+        }
+        __syncthreads();
+
+        // ---- recurrences over the chunk ----
+        for (int p = 0; p < TC; ++p) {
+            const float4 va = *reinterpret_cast<const float4 *>(&sm.vs[p][jc]);
+            const float4 ga = *reinterpret_cast<const float4 *>(&sm.dys[p][jc]);
+            const float vc[4] = {va.x, va.y, va.z, va.w};
+            const float gc[4] = {ga.x, ga.y, ga.z, ga.w};
+            const bool ren = (rmask >> p) & 1u;
+            float al[8];
+            if (ren) {
+                const float4 x = *reinterpret_cast<const float4 *>(&sm.al[p][rowA]);
+                const float4 y = *reinterpret_cast<const float4 *>(&sm.al[p][rowB]);
+                al[0] = x.x; al[1] = x.y; al[2] = x.z; al[3] = x.w;
+                al[4] = y.x; al[5] = y.y; al[6] = y.z; al[7] = y.w;
+            }
+            if (hasS) {
+                // readout: S . dy over my columns, then update S += ks v^T
+                float part[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float a0 = Ss[q][0] * gc[0], a1 = Ss[q][1] * gc[1];
+                    a0 = fmaf(Ss[q][2], gc[2], a0);
+                    a1 = fmaf(Ss[q][3], gc[3], a1);
+                    part[q] = a0 + a1;
+                }
+                const float4 x = *reinterpret_cast<const float4 *>(&sm.ks[p][rowA]);
+                const float4 y = *reinterpret_cast<const float4 *>(&sm.ks[p][rowB]);
+                const float kr[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+                if (ren) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) Ss[q][j] = fmaf(Ss[q][j], al[q], kr[q] * vc[j]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) Ss[q][j] = fmaf(kr[q], vc[j], Ss[q][j]);
+                }
+                float o0, o1;
+                reduce_rows_over_cols(part, c1, c0, o0, o1);
+                sm.pr[p][warp][rowq(q0)] = o0;
+                sm.pr[p][warp][rowq(q0 + 1)] = o1;
+            }
+            if (hasG) {
+                // readouts: G . v over my columns, kh . G over my rows; update G += rs dy^T
+                float part[8], dvp[4];
+                const float4 x = *reinterpret_cast<const float4 *>(&sm.kh[p][rowA]);
+                const float4 y = *reinterpret_cast<const float4 *>(&sm.kh[p][rowB]);
+                const float khr[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float a0 = Gs[q][0] * vc[0], a1 = Gs[q][1] * vc[1];
+                    a0 = fmaf(Gs[q][2], vc[2], a0);
+                    a1 = fmaf(Gs[q][3], vc[3], a1);
+                    part[q] = a0 + a1;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float a0 = khr[0] * Gs[0][j], a1 = khr[1] * Gs[1][j];
+#pragma unroll
+                    for (int q = 2; q < 8; q += 2) {
+                        a0 = fmaf(khr[q], Gs[q][j], a0);
+                        a1 = fmaf(khr[q + 1], Gs[q + 1][j], a1);
+                    }
+                    dvp[j] = a0 + a1;
+                }
+                const float4 xr = *reinterpret_cast<const float4 *>(&sm.rs[p][rowA]);
+                const float4 yr = *reinterpret_cast<const float4 *>(&sm.rs[p][rowB]);
+                const float rr[8] = {xr.x, xr.y, xr.z, xr.w, yr.x, yr.y, yr.z, yr.w};
+                if (ren) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) Gs[q][j] = fmaf(Gs[q][j], al[q], rr[q] * gc[j]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) Gs[q][j] = fmaf(rr[q], gc[j], Gs[q][j]);
+                }
+                float o0, o1;
+                reduce_rows_over_cols(part, c1, c0, o0, o1);
+                sm.pk[p][warp][rowq(q0)] = o0;
+                sm.pk[p][warp][rowq(q0 + 1)] = o1;
+                const float dvj = reduce_cols_over_rows(dvp, b2, b1);
+                if ((rg & 1) == 0) sm.dvs[p][jc + jj] = dvj;
+            }
+        }
+        __syncthreads();
+
+        // ---- per-token outputs of the chunk ----
+        for (int e = tid; e < TC * kHead; e += NT) {
+            const int p = e / kHead, i = e % kHead;
+            const int t = dir > 0 ? tl + p : tl + TC - 1 - p;
+            if (t < 0 || t >= T) continue;
+            const size_t o = ((size_t)b * T + t) * C + cbase + i;
+            const float A = sm.Ap[p][i];
+            const float drs = hasS ? A * (sm.pr[p][0][i] + sm.pr[p][1][i] + sm.pr[p][2][i] + sm.pr[p][3][i]) : 0.f;
+            const float dks = hasG ? A * (sm.pk[p][0][i] + sm.pk[p][1][i] + sm.pk[p][2][i] + sm.pk[p][3][i]) : 0.f;
+            const float dvv = hasG ? sm.dvs[p][i] : 0.f;
+            const int row = dir > 0 ? p : TC - 1 - p;
+            const float rr = sm.raw[s][A_R][row][i], kk = sm.raw[s][A_K][row][i];
+            if (sweepA) {
+                const float vdy = sm.vdy[p];
+                prm.dr[o] = fmaf(sm.u[i] * kk, vdy, drs);
+                prm.dk[o] = fmaf(sm.u[i] * rr, vdy, dks);
+                prm.dv[o] = fmaf(sm.ruk[p], sm.dys[p][i], dvv);
+                prm.dw[o] = fmaf(rr, drs, kk * dks);           // z_t, parked in dw
+            } else {
+                prm.dr[o] += drs;
+                prm.dk[o] += dks;
+                prm.dv[o] += dvv;
+                sm.pr[p][0][i] = fmaf(kk, dks, rr * drs);      // x_t, for the dw scan below
+            }
+        }
+        if (sweepA) {
+            // du partial: thread i accumulates sum_t r k (v.dy) for row i
+            if (tid < kHead) {
+                for (int p = 0; p < TC; ++p) {
+                    const int t = tl + p;
+                    if (t < 0 || t >= T) continue;
+                    du_acc = fmaf(sm.raw[s][A_R][p][tid] * sm.raw[s][A_K][p][tid], sm.vdy[p], du_acc);
+                }
+            }
+        } else {
+            __syncthreads();
+            // dw scan in processing order (t decreasing): dw_t = R - x_t; R += z_t - x_t
+            if (tid < kHead) {
+                for (int p = 0; p < TC; ++p) {
+                    const int t = tl + TC - 1 - p;
+                    if (t < 0 || t >= T) continue;
+                    const size_t o = ((size_t)b * T + t) * C + cbase + tid;
+                    const float x = sm.pr[p][0][tid];
+                    const float z = prm.dw[o];
+                    prm.dw[o] = Rrun - x;
+                    Rrun += z - x;
+                }
+            }
+        }
+        __syncthreads();
+        // stage s is consumed: refill it with chunk g + 2
+        if (tid == 0 && g + 2 < nchunks) {
+            fence_proxy_async_smem();
+            issue(g + 2);
+        }
+    }
+    if (tid < kHead) prm.du_part[(size_t)b * C + cbase + tid] = du_acc;
+}
+
+// du[c] = sum_b du_part[b][c], in increasing b (deterministic).
+__global__ void wkv6_du_reduce_kernel(int B, int C, const float *__restrict__ part, float *__restrict__ du) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b) acc += part[(size_t)b * C + c];
+    du[c] = acc;
+}
+
+template <int TC, bool BIDIR>
+static cudaError_t launch_bwd(const CUtensorMap *maps, const BwdParams &prm, cudaStream_t stream) {
+    auto kern = wkv6_bwd_kernel<TC, BIDIR>;
+    const size_t smem = sizeof(BwdSmem<TC>) + 128;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(prm.B * prm.H), 128, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], prm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return cudaSuccess;
+}
+
+cudaError_t wkv6_bwd_launch(bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
+                            cudaStream_t stream) {
+    constexpr int TC = kBwdTC;
+    cudaError_t e = bidir ? launch_bwd<TC, true>(maps, prm, stream) : launch_bwd<TC, false>(maps, prm, stream);
+    if (e != cudaSuccess) return e;
+    wkv6_du_reduce_kernel<<<(prm.C + 255) / 256, 256, 0, stream>>>(prm.B, prm.C, prm.du_part, du);
+    return cudaGetLastError();
+}
+
+}  // namespace wkv

@@ -1,0 +1,332 @@
+// wkv6_fwd.cu -- RWKV-6 WKV forward (causal and bidirectional) for sm_100a.
+//
+// Operation (per batch b, head h; N = 64; d_t = exp(ew_t)):
+//   causal : y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),  S_t = diag(d_t) S_{t-1} + k_t^T v_t
+//   bidir  : adds r_t S^b_{t+1} with S^b_t = diag(d_t) S^b_{t+1} + k_t^T v_t (no bonus)
+// ("RWKV Architecture ...", RWKV-5 matrix state / RWKV-6 dynamic decay;
+//  "How Custom CUDA Kernels (wkv6_cuda.cu) ...", Forward Pass Implementation.)
+//
+// Design (B200-first; the pages' one-thread-per-column kernel is prior art only)
+// -----------------------------------------------------------------------------
+// * One CTA per (b, h, group of CW = 16*WARPS value columns).  Value columns j
+//   of S are independent (decay scales rows, x_t = k_t^T v_t is an outer
+//   product), so a head's 64 columns may be split over CTAs.
+// * Inputs are staged in chunks of TC tokens by TMA (3-D tensor maps over
+//   [B][T][C], boxes of TC x 64 for r, k, w and TC x CW for v) into a
+//   double-buffered shared-memory ring, one mbarrier per stage.  Rows outside
+//   [0, T) come back zero filled: zero r, k, v contribute nothing and a zero
+//   log-decay keeps the state, so ragged chunks need no masking except on the
+//   y store.
+// * Scaled state.  Inside a chunk (tokens in processing order p = 0..TC-1) the
+//   kernel keeps S' with S_before(p) = diag(exp(L_p)) S', where L_p is the sum
+//   of the log-decays of the chunk's tokens before p.  Then
+//       readout  y_p  = (r_p * exp(L_p)) . S'                   (1 FMA / element)
+//       update   S'  += (k_p * exp(-L_{p+1})) v_p^T               (1 FMA / element)
+//   instead of 3 operations per element for the plain recurrence.  A
+//   "renorm step" ends every run: S' <- diag(exp(L_p + ew_p)) S' + k_p v_p^T,
+//   after which L restarts at 0.  The last token of each chunk is always a
+//   renorm step, and so is any token whose |ew| exceeds kTheta / TC in some
+//   row, so |L| <= kTheta inside a run and exp(+-L) stays inside fp32.  For an
+//   arbitrary decay (down to exactly 0) the result is the plain recurrence's.
+// * Register state: warp w owns columns [16w, 16w+16) of the CTA's group;
+//   lane (rg = lane & 7, cg = lane >> 3) holds rows {4rg..4rg+3, 32+4rg..32+4rg+3}
+//   x columns {4cg..4cg+3}: 32 fp32 state registers.  The readout sums over
+//   rows with a 3-level butterfly reduce-scatter (4 shuffles).
+// * The bonus term (r_t . u . k_t) v_t is a per-token scalar c_t times v_t;
+//   c_t is formed once per token in the transform step.
+#include "wkv_launch.cuh"
+
+namespace wkv {
+
+constexpr float kTheta = 40.0f;  // bound on |L| inside a run (exp(40) ~ 2.4e17)
+
+template <typename Tin, int WARPS, int TC>
+struct FwdSmem {
+    static constexpr int CW = 16 * WARPS;
+    // raw TMA landing buffers (2 stages)
+    Tin raw_r[2][TC][kHead];
+    Tin raw_k[2][TC][kHead];
+    Tin raw_w[2][TC][kHead];
+    Tin raw_v[2][TC][CW];
+    // transformed chunk, processing order
+    float rs[TC][kHead];     // r_p * exp(L_p)
+    float ks[TC][kHead];     // k_p * exp(-L_{p+1})  (k_p on renorm steps)
+    float al[TC][kHead];     // exp(L_p + ew_p) on renorm steps
+    float vs[TC][CW];        // v_p (fp32), this CTA's columns
+    float ybuf[TC][CW];      // y_p, this CTA's columns
+    float c[TC];             // bonus scalar sum_i r_p u k_p
+    float u[kHead];
+    uint32_t renorm_mask;    // bit p set: token p is a renorm step
+    alignas(8) uint64_t full[2];
+};
+
+// Chunk g of the CTA's sweep sequence: pass 0 is anti-causal when bidirectional.
+struct ChunkPos {
+    int dir;     // +1 past->future, -1 future->past
+    int t_lo;    // first token (lowest t) of the TMA box; may be < 0 for dir -1
+    int pass;
+    int c;       // chunk index within the pass
+};
+
+__device__ __forceinline__ ChunkPos chunk_pos(int g, int nch, int T, int TC, bool bidir) {
+    ChunkPos cp;
+    cp.pass = bidir ? (g / nch) : 1;
+    cp.c = bidir ? (g % nch) : g;
+    cp.dir = (bidir && cp.pass == 0) ? -1 : +1;
+    cp.t_lo = (cp.dir > 0) ? cp.c * TC : (T - (cp.c + 1) * TC);
+    return cp;
+}
+
+template <typename Tin, int WARPS, int TC, bool BIDIR>
+__global__ void __launch_bounds__(32 * WARPS)
+wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
+                FwdParams prm) {
+    using Smem = FwdSmem<Tin, WARPS, TC>;
+    constexpr int CW = Smem::CW;
+    constexpr int NT = 32 * WARPS;
+    constexpr int GROUPS = kHead / CW;
+    constexpr uint32_t kStageBytes = (3 * TC * kHead + TC * CW) * sizeof(Tin);
+    extern __shared__ unsigned char smem_dyn[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~uintptr_t(127));
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int T = prm.T, C = prm.C, H = prm.H;
+    const int grp = blockIdx.x % GROUPS;
+    const int bh = blockIdx.x / GROUPS;
+    const int h = bh % H;
+    const int b = bh / H;
+    const int cbase = h * kHead;             // first channel of the head
+    const int col0 = grp * CW;               // first value column of this CTA (head-relative)
+    const int nch = (T + TC - 1) / TC;
+    const int nchunks = BIDIR ? 2 * nch : nch;
+
+    if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
+    if (tid == 0) {
+        prefetch_tensormap(&map_r);
+        prefetch_tensormap(&map_k);
+        prefetch_tensormap(&map_v);
+        prefetch_tensormap(&map_w);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](int g) {
+        const ChunkPos cp = chunk_pos(g, nch, T, TC, BIDIR);
+        const int s = g & 1;
+        mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+        tma_load_3d(&sm.raw_r[s][0][0], &map_r, cbase, cp.t_lo, b, &sm.full[s]);
+        tma_load_3d(&sm.raw_k[s][0][0], &map_k, cbase, cp.t_lo, b, &sm.full[s]);
+        tma_load_3d(&sm.raw_w[s][0][0], &map_w, cbase, cp.t_lo, b, &sm.full[s]);
+        tma_load_3d(&sm.raw_v[s][0][0], &map_v, cbase + col0, cp.t_lo, b, &sm.full[s]);
+    };
+    if (tid == 0) {
+        issue(0);
+        if (nchunks > 1) issue(1);
+    }
+
+    // register state: rows R(q) = (q < 4 ? 4*rg + q : 32 + 4*rg + q - 4), cols 4*cg + j
+    const int rg = lane & 7;
+    const int cg = lane >> 3;
+    const int rowA = 4 * rg;
+    const int rowB = 32 + 4 * rg;
+    const int jc = 16 * warp + 4 * cg;       // CTA-relative first column of this lane
+    const int jj = (rg >> 1) & 3;            // column (of the 4) this lane holds after the reduce
+    const bool b2 = (rg & 4) != 0, b1 = (rg & 2) != 0;
+    float S[8][4];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) S[q][j] = 0.f;
+
+    for (int g = 0; g < nchunks; ++g) {
+        const ChunkPos cp = chunk_pos(g, nch, T, TC, BIDIR);
+        const int s = g & 1;
+        const bool with_bonus = !(BIDIR && cp.pass == 0);
+        if (BIDIR && g == nch) {             // pass boundary: fresh state
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) S[q][j] = 0.f;
+        }
+        // ---- wait for the chunk ----
+        const bool ok = mbar_wait_bounded(&sm.full[s], (g >> 1) & 1);
+        if (!__syncthreads_and(ok)) {         // a bounded wait ran out: stop (fault recorded)
+            drain_two_stage(sm.full, g, nchunks);
+            return;
+        }
+
+        // ---- transform: renorm flags ----
+        // a token is a renorm step if some row has |ew| > kTheta / TC (or NaN)
+        int bad = 0;
+        for (int e = tid; e < TC * kHead; e += NT) {
+            const float ew = to_f32(sm.raw_w[s][e / kHead][e % kHead]);
+            bad |= !(fabsf(ew) <= kTheta / TC);
+        }
+        const int any_bad = __syncthreads_or(bad);
+        if (tid < 32) {
+            uint32_t mask = 1u << (TC - 1);
+            if (any_bad) {
+                for (int p = 0; p < TC - 1; ++p) {
+                    const int row = cp.dir > 0 ? p : TC - 1 - p;
+                    const float e0 = to_f32(sm.raw_w[s][row][lane]);
+                    const float e1 = to_f32(sm.raw_w[s][row][lane + 32]);
+                    const bool bad = !(fabsf(e0) <= kTheta / TC) || !(fabsf(e1) <= kTheta / TC);
+                    if (__any_sync(0xffffffffu, bad)) mask |= 1u << p;
+                }
+            }
+            if (tid == 0) sm.renorm_mask = mask;
+        }
+        __syncthreads();
+        const uint32_t rmask = sm.renorm_mask;
+        // ---- transform: scaled r, k per row (sequential over the chunk) ----
+        for (int i = tid; i < kHead; i += NT) {
+            float L = 0.f;
+#pragma unroll 4
+            for (int p = 0; p < TC; ++p) {
+                const int row = cp.dir > 0 ? p : TC - 1 - p;
+                const float ew = to_f32(sm.raw_w[s][row][i]);
+                const float rr = to_f32(sm.raw_r[s][row][i]);
+                const float kk = to_f32(sm.raw_k[s][row][i]);
+                sm.rs[p][i] = rr * __expf(L);
+                if ((rmask >> p) & 1u) {
+                    sm.al[p][i] = __expf(L + ew);
+                    sm.ks[p][i] = kk;
+                    L = 0.f;
+                } else {
+                    L += ew;
+                    sm.ks[p][i] = kk * __expf(-L);
+                }
+            }
+        }
+        // ---- transform: v (this CTA's columns) and the bonus scalar ----
+        for (int e = tid; e < TC * CW; e += NT) {
+            const int p = e / CW, j = e % CW;
+            const int row = cp.dir > 0 ? p : TC - 1 - p;
+            sm.vs[p][j] = to_f32(sm.raw_v[s][row][j]);
+        }
+        for (int p = warp; p < TC; p += WARPS) {
+            const int row = cp.dir > 0 ? p : TC - 1 - p;
+            float part = to_f32(sm.raw_r[s][row][lane]) * sm.u[lane] * to_f32(sm.raw_k[s][row][lane]) +
+                         to_f32(sm.raw_r[s][row][lane + 32]) * sm.u[lane + 32] *
+                             to_f32(sm.raw_k[s][row][lane + 32]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if (lane == 0) sm.c[p] = with_bonus ? part : 0.f;
+        }
+        __syncthreads();
+        // the raw stage is consumed: refill it with chunk g + 2
+        if (tid == 0 && g + 2 < nchunks) {
+            fence_proxy_async_smem();
+            issue(g + 2);
+        }
+
+        // ---- recurrence over the chunk ----
+#pragma unroll 2
+        for (int p = 0; p < TC; ++p) {
+            const float4 ra = *reinterpret_cast<const float4 *>(&sm.rs[p][rowA]);
+            const float4 rb = *reinterpret_cast<const float4 *>(&sm.rs[p][rowB]);
+            const float4 ka = *reinterpret_cast<const float4 *>(&sm.ks[p][rowA]);
+            const float4 kb = *reinterpret_cast<const float4 *>(&sm.ks[p][rowB]);
+            const float4 vv = *reinterpret_cast<const float4 *>(&sm.vs[p][jc]);
+            const float rr[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+            const float kr[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+            const float vc[4] = {vv.x, vv.y, vv.z, vv.w};
+            float yp[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float a0 = rr[0] * S[0][j], a1 = rr[1] * S[1][j];
+                a0 = fmaf(rr[2], S[2][j], a0);
+                a1 = fmaf(rr[3], S[3][j], a1);
+                a0 = fmaf(rr[4], S[4][j], a0);
+                a1 = fmaf(rr[5], S[5][j], a1);
+                a0 = fmaf(rr[6], S[6][j], a0);
+                a1 = fmaf(rr[7], S[7][j], a1);
+                yp[j] = a0 + a1;
+            }
+            if ((rmask >> p) & 1u) {
+                const float4 aa = *reinterpret_cast<const float4 *>(&sm.al[p][rowA]);
+                const float4 ab = *reinterpret_cast<const float4 *>(&sm.al[p][rowB]);
+                const float al[8] = {aa.x, aa.y, aa.z, aa.w, ab.x, ab.y, ab.z, ab.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) S[q][j] = fmaf(S[q][j], al[q], kr[q] * vc[j]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) S[q][j] = fmaf(kr[q], vc[j], S[q][j]);
+            }
+            // reduce-scatter the 4 column partials over the 8 row groups (lanes xor 4, 2, 1)
+            float k0 = b2 ? yp[2] : yp[0];
+            float k1 = b2 ? yp[3] : yp[1];
+            const float s0 = b2 ? yp[0] : yp[2];
+            const float s1 = b2 ? yp[1] : yp[3];
+            k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
+            k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
+            float kk = b1 ? k1 : k0;
+            const float s2 = b1 ? k0 : k1;
+            kk += __shfl_xor_sync(0xffffffffu, s2, 2);
+            kk += __shfl_xor_sync(0xffffffffu, kk, 1);
+            if ((rg & 1) == 0) {
+                const float vj = sm.vs[p][jc + jj];
+                sm.ybuf[p][jc + jj] = fmaf(sm.c[p], vj, kk);
+            }
+        }
+        __syncthreads();
+
+        // ---- write y for the chunk (float4, coalesced along channels) ----
+        constexpr int V4 = CW / 4;
+        for (int e = tid; e < TC * V4; e += NT) {
+            const int p = e / V4, j4 = (e % V4) * 4;
+            const int t = cp.dir > 0 ? cp.t_lo + p : cp.t_lo + TC - 1 - p;
+            if (t < 0 || t >= T) continue;
+            float4 *dst = reinterpret_cast<float4 *>(prm.y + ((size_t)b * T + t) * C + cbase + col0 + j4);
+            float4 val = *reinterpret_cast<const float4 *>(&sm.ybuf[p][j4]);
+            if (BIDIR && cp.pass == 1) {
+                const float4 old = *dst;    // anti-causal part written by pass 0 of this CTA
+                val.x += old.x;
+                val.y += old.y;
+                val.z += old.z;
+                val.w += old.w;
+            }
+            *dst = val;
+        }
+        if (BIDIR && g == nch - 1) __syncthreads();  // pass-0 y stores visible before pass-1 reads
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+
+template <typename Tin, int WARPS, int TC, bool BIDIR>
+static cudaError_t launch_fwd(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
+                              const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream) {
+    using Smem = FwdSmem<Tin, WARPS, TC>;
+    auto kern = wkv6_fwd_kernel<Tin, WARPS, TC, BIDIR>;
+    const size_t smem = sizeof(Smem) + 128;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int groups = kHead / Smem::CW;
+    const unsigned grid = (unsigned)(prm.B * prm.H * groups);
+    kern<<<grid, 32 * WARPS, smem, stream>>>(mr, mk, mv, mw, prm);
+    return cudaGetLastError();
+}
+
+cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const CUtensorMap &mk,
+                            const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
+                            cudaStream_t stream) {
+    constexpr int TC = kFwdTC;
+    if (bf16) {
+        return bidir ? launch_fwd<__nv_bfloat16, 4, TC, true>(mr, mk, mv, mw, prm, stream)
+                     : launch_fwd<__nv_bfloat16, 4, TC, false>(mr, mk, mv, mw, prm, stream);
+    }
+    return bidir ? launch_fwd<float, 4, TC, true>(mr, mk, mv, mw, prm, stream)
+                 : launch_fwd<float, 4, TC, false>(mr, mk, mv, mw, prm, stream);
+}
+
+}  // namespace wkv

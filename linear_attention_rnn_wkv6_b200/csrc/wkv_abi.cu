@@ -1,0 +1,193 @@
+// wkv_abi.cu -- the extern "C" entry points of libwkv.so (declared in include/wkv.h).
+//
+// Each entry point validates its arguments on the host (nothing is launched on
+// an error), builds the TMA tensor maps the kernel needs, and enqueues the
+// kernel(s) on the caller's stream.  No call allocates or synchronises.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "../../include/wkv.h"
+#include "wkv_launch.cuh"
+
+namespace wkv {
+
+__device__ unsigned int g_wkv_faults = 0;
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a [B][T][C] tensor; box = (box_c channels, box_t tokens, 1).
+bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int B, int T, int C, int box_c, int box_t) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t es = bf16 ? 2 : 4;
+    const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * (cuuint64_t)C * es};
+    const cuuint32_t box[3] = {(cuuint32_t)box_c, (cuuint32_t)box_t, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    std::memset(m, 0, sizeof(*m));
+    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                     const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// sm_100 check, cached per device.
+int check_device() {
+    static int cached[64];   // 0 unknown, 1 ok, 2 bad
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WKV_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && cached[dev] == 1) return WKV_OK;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    const bool ok = (major == 10 && minor == 0);
+    if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+    return ok ? WKV_OK : WKV_ERR_DEVICE;
+}
+
+// Shared checks of the RWKV-6 entry points.
+int check_wkv6(int B, int T, int C, int H, std::initializer_list<const void *> ptrs) {
+    if (B < 0 || T < 0 || C < 1 || H < 1 || C % H != 0) return WKV_ERR_ARG;
+    for (const void *p : ptrs)
+        if (p == nullptr) return WKV_ERR_ARG;
+    if (C / H != kHead) return WKV_ERR_HEADSIZE;
+    if ((long long)B * T * C >= (1ll << 31)) return WKV_ERR_TOO_LARGE;
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return WKV_ERR_ALIGN;
+    return WKV_OK;
+}
+
+int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r, const void *k, const void *v,
+               const void *w, const float *u, float *y, wkv_stream_t stream) {
+    int st = check_wkv6(B, T, C, H, {r, k, v, w, u, y});
+    if (st != WKV_OK) return st;
+    if (B == 0 || T == 0) return WKV_OK;
+    if ((st = check_device()) != WKV_OK) return st;
+    CUtensorMap mr, mk, mv, mw;
+    if (!make_map(&mr, r, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mk, k, bf16, B, T, C, kHead, kFwdTC) ||
+        !make_map(&mv, v, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mw, w, bf16, B, T, C, kHead, kFwdTC))
+        return WKV_ERR_CUDA;
+    FwdParams prm{B, T, C, H, u, y};
+    return wkv6_fwd_launch(bf16, bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? WKV_OK
+               : WKV_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace wkv
+
+using namespace wkv;
+
+extern "C" {
+
+int wkv6_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
+             const float *u, float *y, wkv_stream_t stream) {
+    return fwd_common(false, false, B, T, C, H, r, k, v, w, u, y, stream);
+}
+
+int wkv6_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                  const uint16_t *w, const float *u, float *y, wkv_stream_t stream) {
+    return fwd_common(true, false, B, T, C, H, r, k, v, w, u, y, stream);
+}
+
+int wkv6_bidir_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
+                   const float *u, float *y, wkv_stream_t stream) {
+    return fwd_common(false, true, B, T, C, H, r, k, v, w, u, y, stream);
+}
+
+size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional) {
+    (void)T;
+    (void)H;
+    (void)bidirectional;
+    if (B < 1 || C < 1) return 0;
+    return (size_t)B * (size_t)C * sizeof(float);
+}
+
+int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, const float *k, const float *v,
+             const float *w, const float *u, const float *dy, float *dr, float *dk, float *dv, float *dw,
+             float *du, void *workspace, size_t workspace_bytes, wkv_stream_t stream) {
+    int st = check_wkv6(B, T, C, H, {r, k, v, w, u, dy, dr, dk, dv, dw, du});
+    if (st != WKV_OK) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (B == 0 || T == 0) {
+        if ((st = check_device()) != WKV_OK) return st;
+        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    }
+    const size_t need = wkv6_bwd_workspace_bytes(B, T, C, H, bidirectional);
+    if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WKV_ERR_ALIGN;
+    if ((st = check_device()) != WKV_OK) return st;
+    CUtensorMap maps[5];
+    const void *src[5] = {r, k, w, v, dy};
+    for (int i = 0; i < 5; ++i)
+        if (!make_map(&maps[i], src[i], false, B, T, C, kHead, kBwdTC)) return WKV_ERR_CUDA;
+    BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, static_cast<float *>(workspace)};
+    return wkv6_bwd_launch(bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u, float *y,
+             wkv_stream_t stream) {
+    if (B < 0 || T < 0 || C < 1 || !k || !v || !w || !u || !y) return WKV_ERR_ARG;
+    if ((long long)B * T * C >= (1ll << 31)) return WKV_ERR_TOO_LARGE;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(w) || !aligned16(u) || !aligned16(y)) return WKV_ERR_ALIGN;
+    if (B == 0 || T == 0) return WKV_OK;
+    int st = check_device();
+    if (st != WKV_OK) return st;
+    return wkv4_fwd_launch(B, T, C, k, v, w, u, y, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? WKV_OK
+               : WKV_ERR_CUDA;
+}
+
+const char *wkv_status_string(int status) {
+    switch (status) {
+        case WKV_OK: return "ok";
+        case WKV_ERR_ARG: return "invalid argument (sizes < 0, C != H*N, or a NULL pointer)";
+        case WKV_ERR_HEADSIZE: return "unsupported head size (N = C/H must be 64)";
+        case WKV_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case WKV_ERR_WORKSPACE: return "workspace missing or too small";
+        case WKV_ERR_CUDA: return "CUDA runtime or launch error";
+        case WKV_ERR_DEVICE: return "current device is not sm_100 (B200)";
+        case WKV_ERR_TOO_LARGE: return "problem too large (B*T*C must be < 2^31)";
+        default: return "unknown status";
+    }
+}
+
+int wkv_take_device_faults(unsigned *faults) {
+    if (!faults) return WKV_ERR_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return WKV_ERR_CUDA;
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_wkv_faults, sizeof(v)) != cudaSuccess) return WKV_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_wkv_faults, &zero, sizeof(zero)) != cudaSuccess) return WKV_ERR_CUDA;
+    *faults = v;
+    return WKV_OK;
+}
+
+int wkv_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,32 @@
+// wkv_launch.cuh -- kernel parameter blocks and launcher prototypes (internal to libwkv.so).
+#pragma once
+
+#include "wkv_common.cuh"
+
+namespace wkv {
+
+struct FwdParams {
+    int B, T, C, H;
+    const float *u;
+    float *y;
+};
+
+struct BwdParams {
+    int B, T, C, H;
+    const float *u;
+    float *dr, *dk, *dv, *dw;
+    float *du_part;   // [B][C] per-batch du partials (caller's workspace)
+};
+
+constexpr int kFwdTC = 32;   // tokens per TMA chunk, forward kernels
+constexpr int kBwdTC = 16;   // tokens per TMA chunk, backward kernel
+
+cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const CUtensorMap &mk,
+                            const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
+                            cudaStream_t stream);
+cudaError_t wkv6_bwd_launch(bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
+                            cudaStream_t stream);
+cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,
+                            const float *u, float *y, cudaStream_t stream);
+
+}  // namespace wkv

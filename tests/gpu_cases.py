@@ -1,0 +1,91 @@
+"""Helpers for the GPU parity tests: run the C-ABI entry points on synthetic
+inputs and compute oracle references on the same (exact) input values."""
+from __future__ import annotations
+
+import numpy as np
+
+import linear_attention_rnn_wkv6_b200 as wkv
+from linear_attention_rnn_wkv6_b200 import synth
+
+TOL_F32_FWD = 1e-5     # relative L2, fp32 forward
+TOL_BF16_FWD = 2e-2    # relative L2, bf16 inputs, fp32 state and output
+TOL_F32_GRAD = 1e-4    # relative L2 per gradient tensor
+
+
+def torch():
+    import torch as _t
+    return _t
+
+
+def dev(a: np.ndarray):
+    t = torch()
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return t.from_numpy(a).cuda()
+
+
+def empty_nan(shape):
+    t = torch()
+    return t.full(shape, float("nan"), dtype=t.float32, device="cuda")
+
+
+def run_wkv6_fwd(x: synth.Wkv6Inputs, bidir: bool = False, sync: bool = True) -> np.ndarray:
+    r, k, v, w, u = (dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u"))
+    y = empty_nan((x.B, x.T, x.C))
+    if x.dtype == "bf16":
+        assert not bidir
+        wkv.wkv6_fwd_bf16(x.B, x.T, x.C, x.H, r, k, v, w, u, y)
+    elif bidir:
+        wkv.wkv6_bidir_fwd(x.B, x.T, x.C, x.H, r, k, v, w, u, y)
+    else:
+        wkv.wkv6_fwd(x.B, x.T, x.C, x.H, r, k, v, w, u, y)
+    assert wkv.wkv_take_device_faults() == 0
+    return y.cpu().numpy()
+
+
+def run_wkv6_bwd(x: synth.Wkv6Inputs, bidir: bool):
+    t = torch()
+    r, k, v, w, u, dy = (dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u", "dy"))
+    outs = [empty_nan((x.B, x.T, x.C)) for _ in range(4)] + [empty_nan((x.C,))]
+    nbytes = wkv.wkv6_bwd_workspace_bytes(x.B, x.T, x.C, x.H, bidir)
+    ws = t.empty(max(nbytes, 16), dtype=t.uint8, device="cuda")
+    wkv.wkv6_bwd(x.B, x.T, x.C, x.H, bidir, r, k, v, w, u, dy, *outs, ws, nbytes)
+    assert wkv.wkv_take_device_faults() == 0
+    return tuple(o.cpu().numpy() for o in outs)
+
+
+def run_wkv4(x: synth.Wkv4Inputs) -> np.ndarray:
+    k, v, w, u = (dev(getattr(x, n)) for n in ("k", "v", "w", "u"))
+    y = empty_nan((x.B, x.T, x.C))
+    wkv.wkv4_fwd(x.B, x.T, x.C, k, v, w, u, y)
+    assert wkv.wkv_take_device_faults() == 0
+    return y.cpu().numpy()
+
+
+def f64(x: synth.Wkv6Inputs):
+    return [x.as_f64(n) for n in ("r", "k", "v", "w")] + [x.u.astype(np.float64)]
+
+
+def unit_slice(x: synth.Wkv6Inputs, b: int, h: int):
+    """The oracle's inputs for one (b, h) unit, as a B=1, H=1 problem."""
+    N = x.C // x.H
+    sl = slice(h * N, (h + 1) * N)
+    r, k, v, w, u = f64(x)
+    out = [a[b:b + 1, :, sl] for a in (r, k, v, w)] + [u[sl]]
+    dy = x.dy[b:b + 1, :, sl].astype(np.float64) if x.dy is not None else None
+    return out, dy, sl
+
+
+def sample_units(B: int, H: int, n: int):
+    """n distinct (b, h) units spread over the batch and heads, deterministic."""
+    units, seen = [], set()
+    i = 0
+    while len(units) < min(n, B * H):
+        b = (i * 7 + 3) % B
+        h = (i * 13 + 5 * (i // B)) % H
+        if (b, h) not in seen:
+            seen.add((b, h))
+            units.append((b, h))
+        i += 1
+    return units

@@ -1,0 +1,226 @@
+"""Parity of the CUDA path (called through the C ABI) with the fp64 oracle.
+
+Small problems are compared element by element over the whole tensor; the
+five full-size workloads run in the launch configuration the benchmark times
+and are compared on sampled (b, h) units (every unit of a WKV6 problem is an
+independent problem) plus properties that hold at any size.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from linear_attention_rnn_wkv6_b200 import synth
+from tests import gpu_cases as gc
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    oracle.build()
+
+
+def _rel(a, b):
+    return oracle.rel_l2(a, b)
+
+
+# ------------------------------------------------------------------ forward, small and ragged
+
+FWD_SHAPES = [  # (B, T, H): several 32-token chunks, ragged tails, T < chunk, single token
+    (1, 1, 1), (1, 2, 1), (2, 31, 2), (1, 32, 1), (1, 33, 3), (2, 65, 2), (3, 100, 1), (1, 196, 4),
+]
+
+
+@pytest.mark.parametrize("B,T,H", FWD_SHAPES)
+@pytest.mark.parametrize("bidir", [False, True])
+def test_wkv6_fwd_f32_small(B, T, H, bidir):
+    x = synth.make_wkv6(B, T, H, seed=T * 10 + H)
+    y = gc.run_wkv6_fwd(x, bidir=bidir)
+    r, k, v, w, u = gc.f64(x)
+    ref = oracle.wkv6_fwd(r, k, v, w, u, H=H, bidirectional=bidir)
+    assert np.all(np.isfinite(y))
+    assert _rel(y, ref) <= gc.TOL_F32_FWD
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (2, 33, 2), (1, 97, 3), (2, 256, 2)])
+def test_wkv6_fwd_bf16_small(B, T, H):
+    x = synth.make_wkv6(B, T, H, seed=T + 7, wraw_lo=-8.0, dtype="bf16")
+    y = gc.run_wkv6_fwd(x)
+    r, k, v, w, u = gc.f64(x)
+    ref = oracle.wkv6_fwd(r, k, v, w, u, H=H)
+    err = _rel(y, ref)
+    assert err <= gc.TOL_BF16_FWD
+    assert err <= 1e-5   # the oracle sees the same rounded inputs: only fp32 rounding differs
+
+
+def _with_w(x, w):
+    x.w = w.astype(np.float32)
+    return x
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+@pytest.mark.parametrize("case", ["strong", "mixed", "zero_decay", "unit_decay", "long_memory"])
+def test_wkv6_fwd_decay_edge_cases(case, bidir):
+    B, T, H = 2, 70, 2
+    x = synth.make_wkv6(B, T, H, seed=11)
+    g = np.random.default_rng(5)
+    if case == "strong":          # every token forces a renorm step (|ew| up to e^3)
+        w = -np.exp(g.uniform(-1.0, 3.0, x.w.shape))
+    elif case == "mixed":         # a few tokens with huge or exactly-zero decay
+        w = x.w.astype(np.float64).copy()
+        w[:, 5, :] = -60.0
+        w[:, 40, 3] = -np.inf
+        w[1, 17, :] = -3.0
+    elif case == "zero_decay":    # decay exactly 0 everywhere: only the previous token survives
+        w = np.full(x.w.shape, -np.inf)
+    elif case == "unit_decay":    # decay exactly 1: plain causal / full linear attention
+        w = np.zeros(x.w.shape)
+    else:                         # very slow decay over a long sequence
+        x = synth.make_wkv6(1, 700, 2, seed=12)
+        w = -np.exp(np.random.default_rng(6).uniform(-9.0, -6.0, x.w.shape))
+    x = _with_w(x, w)
+    y = gc.run_wkv6_fwd(x, bidir=bidir)
+    r, k, v, ww, u = gc.f64(x)
+    ref = oracle.wkv6_fwd(r, k, v, ww, u, H=x.H, bidirectional=bidir)
+    assert np.all(np.isfinite(y))
+    assert _rel(y, ref) <= gc.TOL_F32_FWD
+
+
+def test_wkv6_fwd_output_fully_overwritten_and_deterministic():
+    x = synth.make_wkv6(2, 77, 3, seed=3)
+    y1 = gc.run_wkv6_fwd(x, bidir=True)   # outputs start as NaN inside run_wkv6_fwd
+    y2 = gc.run_wkv6_fwd(x, bidir=True)
+    assert np.all(np.isfinite(y1))
+    assert np.array_equal(y1, y2)
+
+
+def test_wkv6_fwd_slices_match_single_head_calls():
+    x = synth.make_wkv6(2, 50, 3, seed=4)
+    y = gc.run_wkv6_fwd(x)
+    for b in range(2):
+        for h in range(3):
+            sl = slice(64 * h, 64 * h + 64)
+            xs = synth.Wkv6Inputs(1, 50, 64, 1, *(np.ascontiguousarray(getattr(x, n)[b:b + 1, :, sl])
+                                                 for n in ("r", "k", "v", "w")), x.u[sl].copy())
+            assert np.array_equal(gc.run_wkv6_fwd(xs), y[b:b + 1, :, sl])
+
+
+# ------------------------------------------------------------------ backward, small and ragged
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (1, 2, 1), (2, 15, 2), (1, 16, 1), (2, 17, 1), (1, 50, 3),
+                                   (2, 96, 2)])
+@pytest.mark.parametrize("bidir", [False, True])
+def test_wkv6_bwd_small(B, T, H, bidir):
+    x = synth.make_wkv6(B, T, H, seed=100 + T, with_dy=True)
+    got = gc.run_wkv6_bwd(x, bidir)
+    r, k, v, w, u = gc.f64(x)
+    ref = oracle.wkv6_bwd(r, k, v, w, u, x.dy.astype(np.float64), H=H, bidirectional=bidir)
+    for name, g, e in zip(("dr", "dk", "dv", "dw", "du"), got, ref):
+        assert np.all(np.isfinite(g)), name
+        if name == "dw" and T <= 2:
+            assert np.max(np.abs(g)) <= 1e-6, name   # exactly zero in exact arithmetic
+            continue
+        assert _rel(g, e) <= gc.TOL_F32_GRAD, (name, _rel(g, e))
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_wkv6_bwd_strong_decay_and_determinism(bidir):
+    x = synth.make_wkv6(2, 45, 2, seed=7, with_dy=True)
+    w = -np.exp(np.random.default_rng(9).uniform(-2.0, 3.5, x.w.shape))
+    w[:, 10, :] = -np.inf
+    x = _with_w(x, w)
+    g1 = gc.run_wkv6_bwd(x, bidir)
+    g2 = gc.run_wkv6_bwd(x, bidir)
+    for a, b in zip(g1, g2):
+        assert np.array_equal(a, b)
+    r, k, v, ww, u = gc.f64(x)
+    ref = oracle.wkv6_bwd(r, k, v, ww, u, x.dy.astype(np.float64), H=2, bidirectional=bidir)
+    for name, g, e in zip(("dr", "dk", "dv", "dw", "du"), g1, ref):
+        assert _rel(g, e) <= gc.TOL_F32_GRAD, (name, _rel(g, e))
+
+
+# ------------------------------------------------------------------ RWKV-4
+
+@pytest.mark.parametrize("B,T,C", [(1, 1, 32), (2, 7, 40), (1, 100, 64), (2, 333, 96), (1, 1024, 32)])
+def test_wkv4_small(B, T, C):
+    x = synth.make_wkv4(B, T, C, seed=T)
+    y = gc.run_wkv4(x)
+    ref = oracle.wkv4_fwd(x.k, x.v, x.w, x.u)
+    assert np.all(np.isfinite(y))
+    assert _rel(y, ref) <= gc.TOL_F32_FWD
+
+
+def test_wkv4_large_keys():
+    x = synth.make_wkv4(2, 300, 64, seed=3, kv_std=1.0)
+    x.k = (x.k * 30.0).astype(np.float32)     # e^k overflows fp32 without the log-space state
+    y = gc.run_wkv4(x)
+    ref = oracle.wkv4_fwd(x.k, x.v, x.w, x.u)
+    assert np.all(np.isfinite(y))
+    assert _rel(y, ref) <= gc.TOL_F32_FWD
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def test_workload_causal_f32_small_config_full_tensor():
+    kind, x = synth.make_workload("wkv6_causal_f32_b1t196h4")
+    y = gc.run_wkv6_fwd(x)
+    r, k, v, w, u = gc.f64(x)
+    assert _rel(y, oracle.wkv6_fwd(r, k, v, w, u, H=x.H)) <= gc.TOL_F32_FWD
+
+
+def test_workload_wkv4_full_tensor():
+    kind, x = synth.make_workload("wkv4_f32_b8t1024c768")
+    y = gc.run_wkv4(x)
+    assert _rel(y, oracle.wkv4_fwd(x.k, x.v, x.w, x.u)) <= gc.TOL_F32_FWD
+
+
+def _sampled_fwd(x, bidir, n_units, tol):
+    y = gc.run_wkv6_fwd(x, bidir=bidir)
+    assert np.all(np.isfinite(y))
+    got, ref = [], []
+    for b, h in gc.sample_units(x.B, x.H, n_units):
+        (r, k, v, w, u), _, sl = gc.unit_slice(x, b, h)
+        ref.append(oracle.wkv6_fwd(r, k, v, w, u, H=1, bidirectional=bidir)[0])
+        got.append(y[b, :, sl])
+    err = _rel(np.stack(got), np.stack(ref))
+    assert err <= tol, err
+    return err
+
+
+def test_workload_bidir_f32_sampled():
+    kind, x = synth.make_workload("wkv6_bidir_f32_b32t196h12")
+    _sampled_fwd(x, True, 48, gc.TOL_F32_FWD)
+
+
+def test_workload_causal_bf16_long_sampled():
+    kind, x = synth.make_workload("wkv6_causal_bf16_b8t4096h32")
+    err = _sampled_fwd(x, False, 12, gc.TOL_BF16_FWD)
+    assert err <= 1e-5
+
+
+def test_workload_bidir_bwd_sampled():
+    kind, x = synth.make_workload("wkv6_bidir_bwd_f32_b32t196h12")
+    dr, dk, dv, dw, du = gc.run_wkv6_bwd(x, True)
+    units = gc.sample_units(x.B, x.H, 24)
+    got = {n: [] for n in ("dr", "dk", "dv", "dw")}
+    ref = {n: [] for n in ("dr", "dk", "dv", "dw")}
+    for b, h in units:
+        (r, k, v, w, u), dy, sl = gc.unit_slice(x, b, h)
+        e = oracle.wkv6_bwd(r, k, v, w, u, dy, H=1, bidirectional=True)
+        for n, gg, ee in zip(("dr", "dk", "dv", "dw"), (dr, dk, dv, dw), e[:4]):
+            got[n].append(gg[b, :, sl])
+            ref[n].append(ee[0])
+    for n in got:
+        err = _rel(np.stack(got[n]), np.stack(ref[n]))
+        assert err <= gc.TOL_F32_GRAD, (n, err)
+    # du sums over the whole batch: check every channel of the heads sampled, exactly defined
+    for h in sorted({h for _, h in units})[:3]:
+        sl = slice(64 * h, 64 * h + 64)
+        acc = np.zeros(64)
+        for b in range(x.B):
+            (r, k, v, w, u), dy, _ = gc.unit_slice(x, b, h)
+            acc += oracle.wkv6_bwd(r, k, v, w, u, dy, H=1, bidirectional=True)[4]
+        assert _rel(du[sl], acc) <= gc.TOL_F32_GRAD
