@@ -281,7 +281,7 @@ def run_native(args, rank, world, local):
     dev = torch.device("cuda", local)
     wkv.load()
     seed = 1000 * rank
-    wls = [DeviceWorkload(n, seed) for n in STEP_WORKLOADS]
+    wls = [DeviceWorkload(n, seed) for n in (args.only or STEP_WORKLOADS)]
     stream = torch.cuda.Stream()
     tokens_per_step = sum(w.tokens for w in wls)
 
@@ -321,7 +321,7 @@ def run_native(args, rank, world, local):
     value = tokens_per_step * world * K / (elapsed_ms / 1e3)
 
     # end-to-end through the public API with host buffers (pinned), copies inside the timed region
-    hs = [HostSide(w) for w in wls]
+    hs = [HostSide(w) for w in wls] if not args.no_e2e else []
     for _ in range(max(1, min(args.warmup, 2))):
         for h in hs:
             h.run(stream)
@@ -338,7 +338,7 @@ def run_native(args, rank, world, local):
     torch.cuda.synchronize()
     barrier(dist)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
-    e2e_value = tokens_per_step * world * Ke / (e2e_ms / 1e3)
+    e2e_value = tokens_per_step * world * Ke / (e2e_ms / 1e3) if hs else None
     h2d = sum(h.h2d for h in hs)
     d2h = sum(h.d2h for h in hs)
 
@@ -374,20 +374,21 @@ def run_native(args, rank, world, local):
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs on the causal workload)",
             "data": "synthetic (seeded splitmix64 + Box-Muller, rank-dependent seed)",
-            "config": {"workload": WORKLOAD_NAME, "tokens_per_step_per_gpu": tokens_per_step,
+            "config": {"workload": WORKLOAD_NAME if not args.only else " + ".join(args.only),
+                       "tokens_per_step_per_gpu": tokens_per_step,
                        "l2": "inputs larger than L2: step working set ~1.2 GB > 126 MB L2, no explicit flush",
                        "parallelism": f"replicated weak scaling x{world} (independent problems per rank)"},
             "roofline": {"kernel": dom, "bound": "hbm" if d["bound"] == "hbm" else "alu",
                          "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
                          "traffic": traffic, "peak_source": d["peak_source"]},
             "kernels": kernels,
-            "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": round(e2e_value, 1) if e2e_value else None, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": Ke,
                     "note": "public C-ABI calls; pinned host inputs copied in and outputs copied out every step"},
             "gpu_launches": K * sum(LAUNCHES[w.name] for w in wls),
             "clocks": clocks,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not args.only:
             line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -422,7 +423,7 @@ def _oracle_unit_seconds(name: str, x, max_units: int, budget_s: float):
         sl_units.append(((i * 7 + 3) % x.B, (i * 5 + 1) % x.H))
     for b, h in sl_units:
         sl = slice(h * N, (h + 1) * N)
-        r, k, v, w = (x.as_f64(n)[b:b + 1, :, sl] for n in ("r", "k", "v", "w"))
+        r, k, v, w = (x.as_f64(n, slice(b, b + 1), sl) for n in ("r", "k", "v", "w"))
         u = x.u[sl].astype(np.float64)
         t = time.perf_counter()
         if name == "wkv6_bidir_bwd_f32_b32t196h12":
@@ -486,11 +487,14 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget of the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--only", action="append", choices=STEP_WORKLOADS,
+                    help="run only these workloads (profiling); the default step runs all four")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

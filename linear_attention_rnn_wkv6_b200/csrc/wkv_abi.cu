@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -37,7 +38,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D map over a [B][T][C] tensor; box = (box_c channels, box_t tokens, 1).
-bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int B, int T, int C, int box_c, int box_t) {
+bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int B, int T, int C, int box_c, int box_t,
+              bool swizzle128 = false) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t es = bf16 ? 2 : 4;
@@ -48,7 +50,8 @@ bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int B, int T, int C, i
     std::memset(m, 0, sizeof(*m));
     CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                      const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -82,6 +85,14 @@ int check_wkv6(int B, int T, int C, int H, std::initializer_list<const void *> p
     return WKV_OK;
 }
 
+// Algorithm of the bf16 causal forward: the chunked tensor-core kernel (default)
+// or the token-by-token recurrence.  WKV6_BF16_PATH=recurrence selects the
+// latter (both compute the same operation; used to compare them).
+bool bf16_use_tensor_cores() {
+    const char *e = std::getenv("WKV6_BF16_PATH");
+    return !(e && std::strcmp(e, "recurrence") == 0);
+}
+
 int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r, const void *k, const void *v,
                const void *w, const float *u, float *y, wkv_stream_t stream) {
     int st = check_wkv6(B, T, C, H, {r, k, v, w, u, y});
@@ -89,6 +100,18 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
     if (B == 0 || T == 0) return WKV_OK;
     if ((st = check_device()) != WKV_OK) return st;
     CUtensorMap mr, mk, mv, mw;
+    if (bf16 && !bidir && bf16_use_tensor_cores()) {
+        constexpr int kTcChunk = 64;
+        if (!make_map(&mr, r, true, B, T, C, kHead, kTcChunk, true) ||
+            !make_map(&mk, k, true, B, T, C, kHead, kTcChunk, true) ||
+            !make_map(&mv, v, true, B, T, C, kHead, kTcChunk, true) ||
+            !make_map(&mw, w, true, B, T, C, kHead, kTcChunk, true))
+            return WKV_ERR_CUDA;
+        FwdParams prm{B, T, C, H, u, y};
+        return wkv6_fwd_tc_launch(mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                   ? WKV_OK
+                   : WKV_ERR_CUDA;
+    }
     if (!make_map(&mr, r, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mk, k, bf16, B, T, C, kHead, kFwdTC) ||
         !make_map(&mv, v, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mw, w, bf16, B, T, C, kHead, kFwdTC))
         return WKV_ERR_CUDA;

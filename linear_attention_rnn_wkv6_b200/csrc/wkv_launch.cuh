@@ -24,6 +24,8 @@ constexpr int kBwdTC = 16;   // tokens per TMA chunk, backward kernel
 cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const CUtensorMap &mk,
                             const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
                             cudaStream_t stream);
+cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
+                               const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream);
 cudaError_t wkv6_bwd_launch(bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
                             cudaStream_t stream);
 cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,

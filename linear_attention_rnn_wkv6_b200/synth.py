@@ -160,10 +160,14 @@ class Wkv6Inputs:
     dy: np.ndarray | None = None  # [B,T,C] float32 upstream gradient
     dtype: str = "f32"
 
-    def as_f64(self, name: str) -> np.ndarray:
+    def as_f64(self, name: str, b=slice(None), c=slice(None)) -> np.ndarray:
+        """Exact float64 copy of one input (optionally only batch slice b, channel slice c)."""
         a = getattr(self, name)
+        if name in ("u",):
+            return a[c].astype(np.float64)
+        a = a[b, :, c] if a.ndim == 3 else a
         if self.dtype == "bf16" and name in ("r", "k", "v", "w"):
-            return bf16_bits_to_f32(a).astype(np.float64)
+            return bf16_bits_to_f32(np.ascontiguousarray(a)).astype(np.float64)
         return a.astype(np.float64)
 
 

@@ -2,6 +2,8 @@
 inputs and compute oracle references on the same (exact) input values."""
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 import linear_attention_rnn_wkv6_b200 as wkv
@@ -71,21 +73,17 @@ def unit_slice(x: synth.Wkv6Inputs, b: int, h: int):
     """The oracle's inputs for one (b, h) unit, as a B=1, H=1 problem."""
     N = x.C // x.H
     sl = slice(h * N, (h + 1) * N)
-    r, k, v, w, u = f64(x)
-    out = [a[b:b + 1, :, sl] for a in (r, k, v, w)] + [u[sl]]
+    out = [x.as_f64(n, slice(b, b + 1), sl) for n in ("r", "k", "v", "w")] + [x.u[sl].astype(np.float64)]
     dy = x.dy[b:b + 1, :, sl].astype(np.float64) if x.dy is not None else None
     return out, dy, sl
 
 
 def sample_units(B: int, H: int, n: int):
-    """n distinct (b, h) units spread over the batch and heads, deterministic."""
-    units, seen = [], set()
-    i = 0
-    while len(units) < min(n, B * H):
-        b = (i * 7 + 3) % B
-        h = (i * 13 + 5 * (i // B)) % H
-        if (b, h) not in seen:
-            seen.add((b, h))
-            units.append((b, h))
-        i += 1
-    return units
+    """min(n, B*H) distinct (b, h) units spread over batch and heads, deterministic.
+
+    Walks the B*H units with a stride coprime to B*H, so it always terminates."""
+    total = B * H
+    n = min(n, total)
+    start = max(1, total // max(n, 1))
+    stride = next(s for s in range(start, start + total + 1) if math.gcd(s, total) == 1)
+    return [divmod((i * stride + 3) % total, H) for i in range(n)]
