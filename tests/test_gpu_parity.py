@@ -50,12 +50,9 @@ BF16_PATHS = ["tensor", "recurrence"]
 
 @pytest.fixture(params=BF16_PATHS)
 def bf16_path(request, monkeypatch):
-    """Run the bf16 causal forward through the chunked tensor-core kernel (default)
-    or the token-by-token recurrence kernel."""
-    if request.param == "recurrence":
-        monkeypatch.setenv("WKV6_BF16_PATH", "recurrence")
-    else:
-        monkeypatch.delenv("WKV6_BF16_PATH", raising=False)
+    """Run the bf16 causal forward through the chunked tensor-core kernel or the
+    token-by-token recurrence kernel."""
+    monkeypatch.setenv("WKV6_BF16_PATH", request.param)
     return request.param
 
 
