@@ -118,6 +118,32 @@ int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, cons
 size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional);
 
 /*
+ * wkv6_bwd_noalloc -- wkv6_bwd without a workspace argument, for callers that
+ * cannot allocate device memory: for example code that runs inside another
+ * framework's callback or plugin which hands it no scratch buffer, or a
+ * serving process that reserves all of its device memory at start-up and may
+ * not call cudaMalloc afterwards (cudaMalloc can synchronise the device and
+ * fragments a planned memory pool).  The source pages have no counterpart to
+ * this entry point; it exists for those callers.
+ *
+ * Same operation, arguments (minus workspace), layouts and results as wkv6_bwd.
+ * Its scratch is a fixed 1 MiB device array inside libwkv.so, which every GPU
+ * that loads the library holds until the process exits; the call itself
+ * allocates nothing.
+ *   Limit: B*C <= 262144, else WKV_ERR_TOO_LARGE and nothing is launched.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls share the one array: calls that may overlap on the GPU (on
+ *   different streams, or from several host threads) race and must be
+ *   serialised by the caller.  Nothing in the array needs clearing between
+ *   calls: each call writes every entry it later reads.
+ */
+int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, const float *r, const float *k,
+                     const float *v, const float *w, const float *u, const float *dy, float *dr, float *dk,
+                     float *dv, float *dw, float *du, wkv_stream_t stream);
+
+/*
  * wkv4_fwd -- RWKV-4 WKV forward, fp32 ("RWKV Architecture ...", The
  * Fundamental Mathematical Duality and The Recurrent Inference Formulation):
  *     y_t = (sum_{s<t} e^{-(t-1-s) w + k_s} v_s + e^{u + k_t} v_t)

@@ -18,7 +18,7 @@ import os
 __all__ = [
     "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
-    "EXPORTED_SYMBOLS", "HEAD_SIZE",
+    "wkv6_bwd_noalloc", "EXPORTED_SYMBOLS", "HEAD_SIZE",
 ]
 
 HEAD_SIZE = 64
@@ -28,7 +28,7 @@ _LIB = None
 # Every extern "C" symbol declared in include/wkv.h.
 EXPORTED_SYMBOLS = (
     "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
-    "wkv_status_string", "wkv_take_device_faults", "wkv_version",
+    "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc",
 )
 
 _I = ctypes.c_int
@@ -45,6 +45,7 @@ _SIGS = {
     "wkv_status_string": ([_I], ctypes.c_char_p),
     "wkv_take_device_faults": ([ctypes.POINTER(ctypes.c_uint)], _I),
     "wkv_version": ([], _I),
+    "wkv6_bwd_noalloc": ([_I] * 5 + [_P] * 11 + [_P], _I),
 }
 
 
@@ -128,6 +129,14 @@ def wkv6_bwd(B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, w
     _check("wkv6_bwd", load().wkv6_bwd(B, T, C, H, int(bool(bidirectional)), _ptr(r), _ptr(k), _ptr(v), _ptr(w),
                                        _ptr(u), _ptr(dy), _ptr(dr), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du),
                                        _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def wkv6_bwd_noalloc(B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, stream=None) -> None:
+    """wkv6_bwd without a workspace, for callers that cannot allocate device memory
+    (its scratch is a fixed array inside the library; B*C <= 262144)."""
+    _check("wkv6_bwd_noalloc", load().wkv6_bwd_noalloc(B, T, C, H, int(bool(bidirectional)), _ptr(r), _ptr(k), _ptr(v),
+                                                       _ptr(w), _ptr(u), _ptr(dy), _ptr(dr), _ptr(dk), _ptr(dv),
+                                                       _ptr(dw), _ptr(du), _stream(stream)))
 
 
 def wkv4_fwd(B, T, C, k, v, w, u, y, stream=None) -> None:

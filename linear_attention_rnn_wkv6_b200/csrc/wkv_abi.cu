@@ -214,3 +214,60 @@ int wkv_take_device_faults(unsigned *faults) {
 int wkv_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// wkv6_bwd_noalloc: wkv6_bwd for callers that cannot allocate device memory.
+//
+// The only scratch wkv6_bwd needs is B*C floats of per-batch du partials.  Here
+// they live in a fixed file-scope device array instead of a caller-supplied
+// workspace.  In host code the array's name is only a host-side stand-in, so
+// its device address is looked up with cudaGetSymbolAddress, once per device,
+// with that device current (the first call on each device does this).
+namespace wkv {
+namespace {
+
+constexpr size_t kNoAllocDuFloats = 262144;   // B*C limit: 1 MiB held by every device that loads the library
+static __device__ __align__(256) float g_noalloc_du_partials[kNoAllocDuFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device (looked up once per device).
+int noalloc_scratch(float **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_du_partials) != cudaSuccess || p == nullptr) return WKV_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return WKV_OK;
+}
+
+}  // namespace
+}  // namespace wkv
+
+extern "C" int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, const float *r, const float *k,
+                                const float *v, const float *w, const float *u, const float *dy, float *dr,
+                                float *dk, float *dv, float *dw, float *du, wkv_stream_t stream) {
+    int st = check_wkv6(B, T, C, H, {r, k, v, w, u, dy, dr, dk, dv, dw, du});
+    if (st != WKV_OK) return st;
+    if ((size_t)B * (size_t)C > kNoAllocDuFloats) return WKV_ERR_TOO_LARGE;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = check_device()) != WKV_OK) return st;
+    if (B == 0 || T == 0)
+        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    float *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != WKV_OK) return st;
+    CUtensorMap maps[5];
+    const void *src[5] = {r, k, w, v, dy};
+    for (int i = 0; i < 5; ++i)
+        if (!make_map(&maps[i], src[i], false, B, T, C, kHead, kBwdTC)) return WKV_ERR_CUDA;
+    // Every per-batch partial the reduction reads is written first by the
+    // backward kernel, so nothing left in the array by an earlier call leaks in.
+    BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, scratch};
+    return wkv6_bwd_launch(bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
