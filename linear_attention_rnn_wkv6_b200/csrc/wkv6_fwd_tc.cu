@@ -14,6 +14,9 @@
 //   M1  A  = Q Kt^T                       (TMEM cols [0,64))
 //   M2  Y  = Q S_in + tril_strict(A) V     (TMEM cols [64,128))
 //   M3  S += Kt^T V                        (TMEM cols [128,192)), then rows scaled by exp(Lam_L)
+// Every operand is staged K-major (the contraction index contiguous): TF32
+// operands in the transposed (MN-major) form produce no result on this
+// hardware, so Kt is kept in two layouts and V and S_in are stored transposed.
 // |Lam| <= 80 keeps exp(-Lam) inside fp32.  A chunk whose cumulative decay
 // leaves that range (fast-forgetting channels) is evaluated instead by the
 // exact token-by-token recurrence on the CUDA cores, starting from the state
@@ -35,11 +38,12 @@ constexpr int kLamPad = kHead + 4;     // padded row of the Lam table (bank spre
 
 struct TcSmem {
     __nv_bfloat16 raw[2][4][kL][kHead];   // r, k, v, w stages (TMA, 128B-swizzled), 64 KB
-    float Qs[16][kL][4];                  // Q   : unit over i, row p
-    float Ks[16][kL][4];                  // Kt  : unit over i, row s
-    float Vs[16][kL][4];                  // V   : unit over j, row s
-    float As[16][kL][4];                  // A   : unit over s, row p (masked)
-    float Ss[16][kHead][4];               // S_in: unit over j, row i
+    float Qs[16][kL][4];                  // Q    : unit over i, row p   (A of M1, M2)
+    float Ks[16][kL][4];                  // Kt   : unit over i, row s   (B of M1)
+    float KT[16][kHead][4];               // Kt^T : unit over s, row i   (A of M3)
+    float VT[16][kHead][4];               // V^T  : unit over s, row j   (B of M2, M3)
+    float As[16][kL][4];                  // A    : unit over s, row p, masked (A of M2)
+    float ST[16][kHead][4];               // S_in^T: unit over i, row j  (B of M2)
     float lam[kL + 1][kLamPad];           // exclusive cumulative log-decay, rows p = 0..64
     float dec[kHead];                     // exp(Lam_L)
     float c[kL];                          // bonus scalars
@@ -113,9 +117,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     bool failed = false;
     const int prow = 16 * warp + lane;       // accumulator row of this thread (valid for lane < 16)
     const bool rowlane = lane < 16;
-    constexpr uint32_t kIdK_K = tc::idesc_tf32(64, 64, false, false);   // A K-major, B K-major
-    constexpr uint32_t kIdK_MN = tc::idesc_tf32(64, 64, false, true);   // A K-major, B MN-major
-    constexpr uint32_t kIdMN_MN = tc::idesc_tf32(64, 64, true, true);   // A MN-major, B MN-major
+    constexpr uint32_t kIdK_K = tc::idesc_tf32(64, 64, false, false);   // A and B K-major
 
     for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
@@ -155,17 +157,30 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 const int p = (blk & 7) * 8 + pl;
                 const int u4 = (blk >> 3) * 4 + ul;
                 const int i0 = 4 * u4;
-                float q[4], kt[4], vv[4];
+                float q[4], kt[4];
 #pragma unroll
                 for (int e2 = 0; e2 < 4; ++e2) {
                     const int i = i0 + e2;
                     q[e2] = raw_at(sm.raw[s][R_], p, i) * __expf(sm.lam[p][i]);
                     kt[e2] = raw_at(sm.raw[s][K_], p, i) * __expf(-sm.lam[p + 1][i]);
-                    vv[e2] = raw_at(sm.raw[s][V_], p, i);
                 }
                 *reinterpret_cast<float4 *>(&sm.Qs[u4][p][0]) = make_float4(q[0], q[1], q[2], q[3]);
                 *reinterpret_cast<float4 *>(&sm.Ks[u4][p][0]) = make_float4(kt[0], kt[1], kt[2], kt[3]);
-                *reinterpret_cast<float4 *>(&sm.Vs[u4][p][0]) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+            }
+            // transposed tiles: 4 consecutive tokens of one channel per thread
+            for (int e = tid; e < kL * 16; e += 128) {
+                const int il = e & 7, sl = (e >> 3) & 3, blk = e >> 5;
+                const int i = (blk & 7) * 8 + il;
+                const int su = (blk >> 3) * 4 + sl;
+                float kt[4], vv[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const int tok = 4 * su + e2;
+                    kt[e2] = raw_at(sm.raw[s][K_], tok, i) * __expf(-sm.lam[tok + 1][i]);
+                    vv[e2] = raw_at(sm.raw[s][V_], tok, i);
+                }
+                *reinterpret_cast<float4 *>(&sm.KT[su][i][0]) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+                *reinterpret_cast<float4 *>(&sm.VT[su][i][0]) = make_float4(vv[0], vv[1], vv[2], vv[3]);
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
@@ -215,14 +230,14 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 if (c > 0) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        tc::mma_tf32(tY, tc::desc_kmajor(sm.Qs, k), tc::desc_mnmajor(sm.Ss, k), kIdK_MN, k > 0);
+                        tc::mma_tf32(tY, tc::desc_kmajor(sm.Qs, k), tc::desc_kmajor(sm.ST, k), kIdK_K, k > 0);
                 }
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    tc::mma_tf32(tY, tc::desc_kmajor(sm.As, k), tc::desc_mnmajor(sm.Vs, k), kIdK_MN, c > 0 || k > 0);
+                    tc::mma_tf32(tY, tc::desc_kmajor(sm.As, k), tc::desc_kmajor(sm.VT, k), kIdK_K, c > 0 || k > 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    tc::mma_tf32(tS, tc::desc_mnmajor(sm.Ks, k), tc::desc_mnmajor(sm.Vs, k), kIdMN_MN, c > 0 || k > 0);
+                    tc::mma_tf32(tS, tc::desc_kmajor(sm.KT, k), tc::desc_kmajor(sm.VT, k), kIdK_K, c > 0 || k > 0);
                 tc::mma_commit(&sm.mma_bar);
             }
             if (!mbar_wait_bounded(&sm.mma_bar, mma_phase)) failed = true;
@@ -238,13 +253,13 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 if (rowlane && t < T) {
                     float *dst = prm.y + ((size_t)b * T + t) * C + cbase;
                     const float cp = sm.c[prow];
+                    const float *vrow = &sm.VT[prow >> 2][0][prow & 3];   // v_p[j] at vrow[4 * j]
 #pragma unroll
                     for (int u4 = 0; u4 < 16; ++u4) {
-                        const float4 vv = *reinterpret_cast<const float4 *>(&sm.Vs[u4][prow][0]);
                         const float *src = u4 < 8 ? &y0[4 * u4] : &y1[4 * (u4 - 8)];
                         *reinterpret_cast<float4 *>(dst + 4 * u4) =
-                            make_float4(fmaf(cp, vv.x, src[0]), fmaf(cp, vv.y, src[1]), fmaf(cp, vv.z, src[2]),
-                                        fmaf(cp, vv.w, src[3]));
+                            make_float4(fmaf(cp, vrow[4 * (4 * u4)], src[0]), fmaf(cp, vrow[4 * (4 * u4 + 1)], src[1]),
+                                        fmaf(cp, vrow[4 * (4 * u4 + 2)], src[2]), fmaf(cp, vrow[4 * (4 * u4 + 3)], src[3]));
                     }
                 }
             }
@@ -263,10 +278,11 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 tc::tmem_st32(tS + lane_off, s0);
                 tc::tmem_st32(tS + lane_off + 32, s1);
                 if (rowlane) {
+                    float *dstT = &sm.ST[prow >> 2][0][prow & 3];         // S[i][j] at dstT[4 * j]
 #pragma unroll
-                    for (int u4 = 0; u4 < 16; ++u4) {
-                        const float *src = u4 < 8 ? &s0[4 * u4] : &s1[4 * (u4 - 8)];
-                        *reinterpret_cast<float4 *>(&sm.Ss[u4][prow][0]) = make_float4(src[0], src[1], src[2], src[3]);
+                    for (int j = 0; j < 32; ++j) {
+                        dstT[4 * j] = s0[j];
+                        dstT[4 * (32 + j)] = s1[j];
                     }
                 }
                 tc::tmem_wait_st();
@@ -326,10 +342,9 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 tc::tmem_st32(tS + lane_off, s0);
                 tc::tmem_st32(tS + lane_off + 32, s1);
                 if (rowlane) {
+                    float *dstT = &sm.ST[prow >> 2][0][prow & 3];
 #pragma unroll
-                    for (int u4 = 0; u4 < 16; ++u4)
-                        *reinterpret_cast<float4 *>(&sm.Ss[u4][prow][0]) =
-                            make_float4(Sr[4 * u4], Sr[4 * u4 + 1], Sr[4 * u4 + 2], Sr[4 * u4 + 3]);
+                    for (int j = 0; j < 64; ++j) dstT[4 * j] = Sr[j];
                 }
                 tc::tmem_wait_st();
             }

@@ -85,12 +85,12 @@ int check_wkv6(int B, int T, int C, int H, std::initializer_list<const void *> p
     return WKV_OK;
 }
 
-// Algorithm of the bf16 causal forward: the token-by-token recurrence (default)
-// or the chunked tensor-core kernel (WKV6_BF16_PATH=tensor).  Both compute the
-// same operation; the variable is read on every call.
+// Algorithm of the bf16 causal forward: the chunked tensor-core kernel (default)
+// or the token-by-token recurrence (WKV6_BF16_PATH=recurrence).  Both compute
+// the same operation; the variable is read on every call.
 bool bf16_use_tensor_cores() {
     const char *e = std::getenv("WKV6_BF16_PATH");
-    return e && std::strcmp(e, "tensor") == 0;
+    return !(e && std::strcmp(e, "recurrence") == 0);
 }
 
 int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r, const void *k, const void *v,
