@@ -8,23 +8,28 @@
 // 64 x 64 x 64 contractions on tcgen05 (kind::tf32, fp32 accumulators in TMEM).
 //
 // Chunk algebra.  With Lam_p = sum_{m<p} ew_m (per row i, exclusive, chunk-local),
-// Q_p = r_p * exp(Lam_p) and Kt_s = k_s * exp(-Lam_{s+1}):
-//   y_p   = Q_p S_in + sum_{s<p} (Q_p . Kt_s) v_s + c_p v_p        (c_p = sum_i r u k)
+// Q_p = r_p * exp(Lam_p), Kt_s = k_s * exp(-Lam_{s+1}) and c_p = sum_i r_p u k_p:
+//   y_p   = Q_p S_in + sum_{s<p} (Q_p . Kt_s) v_s + c_p v_p
 //   S_out = diag(exp(Lam_L)) (S_in + Kt^T V)
-//   M1  A  = Q Kt^T                       (TMEM cols [0,64))
-//   M2  Y  = Q S_in + tril_strict(A) V     (TMEM cols [64,128))
-//   M3  S += Kt^T V                        (TMEM cols [128,192)), then rows scaled by exp(Lam_L)
-// Every operand is staged K-major (the contraction index contiguous): TF32
-// operands in the transposed (MN-major) form produce no result on this
-// hardware, so Kt is kept in two layouts and V and S_in are stored transposed.
+//   M1  A  = Q Kt^T                                  (TMEM cols [0,64))
+//   M2  Y  = Q S_in + A' V,  A' = strict-lower(A) + diag(c)   (TMEM cols [64,128))
+//   M3  S += Kt^T V, then rows scaled by exp(Lam_L)  (TMEM cols [128,192))
+// All operands are K-major (TF32 operands in MN-major form give no result on
+// this hardware), staged in the 128-byte-swizzled canonical layout so both
+// row-wise and column-wise shared-memory writes are bank-conflict free; Kt is
+// kept in two orientations and V and S_in are stored transposed.
 // |Lam| <= 80 keeps exp(-Lam) inside fp32.  A chunk whose cumulative decay
 // leaves that range (fast-forgetting channels) is evaluated instead by the
 // exact token-by-token recurrence on the CUDA cores, starting from the state
-// held in TMEM, so any decay value down to exactly 0 stays exact.
+// held in TMEM, so any decay down to exactly 0 stays exact.
 //
-// One CTA (128 threads) per (b, h); thread 0 issues the MMAs; all threads do
-// the decay transform and the TMEM epilogues.  Inputs arrive by TMA with the
-// 128-byte swizzle (bank-conflict-free column reads of the bf16 tiles).
+// Warp roles (one CTA per (b, h), 13 warps):
+//   warp 0      TMA loads (2-stage ring) and, from one thread, all MMAs
+//   warps 1..8  transform: chunk operands for the MMAs, then the masked A'
+//   warps 9..12 epilogue: y out of TMEM, state rescale and its transposed copy
+// Operand sets are double buffered, so the transform of chunk c+1 overlaps the
+// MMAs and epilogue of chunk c.  Hand-offs are mbarriers; every wait is bounded
+// and a shared abort flag stops all roles after the first timeout.
 #include "wkv_launch.cuh"
 #include "wkv_tc.cuh"
 
@@ -34,42 +39,85 @@ namespace {
 
 constexpr int kL = 64;                 // tokens per chunk
 constexpr float kLamMax = 80.0f;       // |Lam| bound of the tensor-core path
-constexpr int kLamPad = kHead + 4;     // padded row of the Lam table (bank spread)
+constexpr int kTW = 8;                 // transform warps
+constexpr int kEW = 4;                 // epilogue warps
+constexpr int kThreads = 32 * (1 + kTW + kEW);
+constexpr int kTT = 32 * kTW;          // transform threads
+constexpr int kET = 32 * kEW;          // epilogue threads
+constexpr int kTokPerT = kL / (kTT / kHead);   // tokens per transform thread (16)
 
-struct TcSmem {
+struct Tc2Smem {
     __nv_bfloat16 raw[2][4][kL][kHead];   // r, k, v, w stages (TMA, 128B-swizzled), 64 KB
-    float Qs[16][kL][4];                  // Q    : unit over i, row p   (A of M1, M2)
-    float Ks[16][kL][4];                  // Kt   : unit over i, row s   (B of M1)
-    float KT[16][kHead][4];               // Kt^T : unit over s, row i   (A of M3)
-    float VT[16][kHead][4];               // V^T  : unit over s, row j   (B of M2, M3)
-    float As[16][kL][4];                  // A    : unit over s, row p, masked (A of M2)
-    float ST[16][kHead][4];               // S_in^T: unit over i, row j  (B of M2)
-    float lam[kL + 1][kLamPad];           // exclusive cumulative log-decay, rows p = 0..64
-    float dec[kHead];                     // exp(Lam_L)
-    float c[kL];                          // bonus scalars
+    float Q[2][kL * kHead];               // (row p, k = i)            A of M1, M2
+    float K[2][kL * kHead];               // (row s, k = i), B of M1; then A' (row p, k = s), A of M2
+    float KT[2][kHead * kL];              // (row i, k = s)            A of M3
+    float VT[2][kHead * kL];              // (row j, k = s)            B of M2, M3
+    float ST[kHead * kHead];              // S_in^T (row j, k = i)     B of M2
+    float dec[4][kHead];                  // exp(Lam_L) per row (ring of 4 chunks)
+    float cp[2][kL];                      // bonus scalars per token
+    float part_sum[kTW / 2][kHead];       // per-quarter log-decay sums (prefix exchange)
     float u[kHead];
+    int flag[4];                          // chunk c is flagged iff flag[c & 3] == c + 1
+    int abort_;
     uint32_t tmem_base;
-    int flag;
     alignas(8) uint64_t full[2];
-    alignas(8) uint64_t mma_bar;
+    alignas(8) uint64_t t_done, m1_done, a_done, mma_done, s_ready;
+    alignas(8) uint64_t set_free[2];
+    alignas(8) uint64_t final_bar;
 };
 
 enum { R_ = 0, K_ = 1, V_ = 2, W_ = 3 };
 
-// Element (row, col) of a 64 x 64 bf16 tile written by TMA with the 128-byte swizzle.
 __device__ __forceinline__ float raw_at(const __nv_bfloat16 (&t)[kL][kHead], int row, int col) {
     const int chunk = (col >> 3) ^ (row & 7);
     return __bfloat162float(t[row][chunk * 8 + (col & 7)]);
 }
 
+// Float index of element (row r, k) of a 64 x 64 tf32 K-major tile in the
+// 128-byte-swizzled canonical layout: two K-blocks of [64 rows][32 floats],
+// 16-byte chunk c of row r stored at chunk c ^ (r & 7).
+__device__ __forceinline__ int swz(int r, int k) {
+    return (k >> 5) * 2048 + r * 32 + ((((k & 31) >> 2) ^ (r & 7)) << 2) + (k & 3);
+}
+
+// Descriptor of the kstep-th group of 8 K values of such a tile.
+__device__ __forceinline__ uint64_t desc_sw(const float *tile, int kstep) {
+    const char *p = reinterpret_cast<const char *>(tile) + (kstep >> 2) * 8192 + (kstep & 3) * 32;
+    return tc::smem_desc(p, 16, 1024) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait that gives up at once when another thread has already aborted.
+__device__ __forceinline__ bool wait_or_abort(Tc2Smem &sm, uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*(volatile int *)&sm.abort_) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_wkv_faults, WKV_FAULT_TIMEOUT);
+            *(volatile int *)&sm.abort_ = 1;
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
                    FwdParams prm) {
     extern __shared__ unsigned char smem_dyn[];
-    TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    Tc2Smem &sm = *reinterpret_cast<Tc2Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = prm.T, C = prm.C, H = prm.H;
@@ -79,14 +127,23 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     constexpr uint32_t kStageBytes = 4u * kL * kHead * sizeof(__nv_bfloat16);
 
     if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
+    if (tid < 4) sm.flag[tid] = 0;
     if (tid == 0) {
+        sm.abort_ = 0;
         prefetch_tensormap(&map_r);
         prefetch_tensormap(&map_k);
         prefetch_tensormap(&map_v);
         prefetch_tensormap(&map_w);
         mbar_init(&sm.full[0], 1);
         mbar_init(&sm.full[1], 1);
-        mbar_init(&sm.mma_bar, 1);
+        mbar_init(&sm.t_done, kTT);
+        mbar_init(&sm.m1_done, 1);
+        mbar_init(&sm.a_done, kTT);
+        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.s_ready, kET);
+        mbar_init(&sm.set_free[0], 1);
+        mbar_init(&sm.set_free[1], 1);
+        mbar_init(&sm.final_bar, 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -98,7 +155,9 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     tc::fence_after_sync();
     const uint32_t tbase = sm.tmem_base;
     const uint32_t tA = tbase, tY = tbase + 64, tS = tbase + 128;
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;   // this warp's TMEM lane quarter
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lane quarter
+    const int qrow = 16 * (warp & 3) + lane;                          // accumulator row (lane < 16)
+    const bool rowlane = lane < 16;
 
     auto issue = [&](int c) {
         const int s = c & 1;
@@ -108,168 +167,285 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
         tma_load_3d(&sm.raw[s][V_][0][0], &map_v, cbase, c * kL, b, &sm.full[s]);
         tma_load_3d(&sm.raw[s][W_][0][0], &map_w, cbase, c * kL, b, &sm.full[s]);
     };
-    if (tid == 0) {
-        issue(0);
-        if (nch > 1) issue(1);
-    }
 
-    uint32_t mma_phase = 0;
-    bool failed = false;
-    const int prow = 16 * warp + lane;       // accumulator row of this thread (valid for lane < 16)
-    const bool rowlane = lane < 16;
-    constexpr uint32_t kIdK_K = tc::idesc_tf32(64, 64, false, false);   // A and B K-major
-
-    for (int c = 0; c < nch; ++c) {
-        const int s = c & 1;
-        const int t0 = c * kL;
-        const bool ok = mbar_wait_bounded(&sm.full[s], (c >> 1) & 1);
-        if (!__syncthreads_and(ok)) {
-            failed = true;
-            drain_two_stage(sm.full, c, nch);
-            break;
-        }
-        // ---- T1: cumulative log-decay per row (threads 0..63), bonus scalars (64..127)
-        int bad = 0;
-        if (tid < kHead) {
-            const int i = tid;
-            float L = 0.f, mx = 0.f;
-            for (int p = 0; p < kL; ++p) {
-                sm.lam[p][i] = L;
-                L += raw_at(sm.raw[s][W_], p, i);
-                mx = fmaxf(mx, fabsf(L));
+    if (warp == 0) {
+        // ===================== TMA + MMA issue (one thread) =====================
+        if (lane == 0) {
+            constexpr uint32_t kId = tc::idesc_tf32(64, 64, false, false);
+            int issued = 0;
+            issue(0);
+            ++issued;
+            if (nch > 1) {
+                issue(1);
+                ++issued;
             }
-            sm.lam[kL][i] = L;
-            sm.dec[i] = __expf(L);
-            bad = !(mx <= kLamMax);
-        } else {
-            const int p = tid - kHead;
-            float acc = 0.f;
-            for (int i = 0; i < kHead; ++i)
-                acc = fmaf(raw_at(sm.raw[s][R_], p, i) * sm.u[i], raw_at(sm.raw[s][K_], p, i), acc);
-            sm.c[p] = acc;
-        }
-        const bool flagged = __syncthreads_or(bad) != 0;
-
-        if (!flagged) {
-            // ---- T2: Q, Kt, V into the operand tiles (lane -> 8 rows x 4 units per quarter warp)
-            for (int e = tid; e < kL * 16; e += 128) {
-                const int pl = e & 7, ul = (e >> 3) & 3, blk = e >> 5;     // blk: 32 blocks of 8 rows x 4 units
-                const int p = (blk & 7) * 8 + pl;
-                const int u4 = (blk >> 3) * 4 + ul;
-                const int i0 = 4 * u4;
-                float q[4], kt[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    const int i = i0 + e2;
-                    q[e2] = raw_at(sm.raw[s][R_], p, i) * __expf(sm.lam[p][i]);
-                    kt[e2] = raw_at(sm.raw[s][K_], p, i) * __expf(-sm.lam[p + 1][i]);
-                }
-                *reinterpret_cast<float4 *>(&sm.Qs[u4][p][0]) = make_float4(q[0], q[1], q[2], q[3]);
-                *reinterpret_cast<float4 *>(&sm.Ks[u4][p][0]) = make_float4(kt[0], kt[1], kt[2], kt[3]);
-            }
-            // transposed tiles: 4 consecutive tokens of one channel per thread
-            for (int e = tid; e < kL * 16; e += 128) {
-                const int il = e & 7, sl = (e >> 3) & 3, blk = e >> 5;
-                const int i = (blk & 7) * 8 + il;
-                const int su = (blk >> 3) * 4 + sl;
-                float kt[4], vv[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    const int tok = 4 * su + e2;
-                    kt[e2] = raw_at(sm.raw[s][K_], tok, i) * __expf(-sm.lam[tok + 1][i]);
-                    vv[e2] = raw_at(sm.raw[s][V_], tok, i);
-                }
-                *reinterpret_cast<float4 *>(&sm.KT[su][i][0]) = make_float4(kt[0], kt[1], kt[2], kt[3]);
-                *reinterpret_cast<float4 *>(&sm.VT[su][i][0]) = make_float4(vv[0], vv[1], vv[2], vv[3]);
-            }
-            fence_proxy_async_smem();
-            tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
-            // the raw stage is consumed: refill it
-            if (tid == 0 && c + 2 < nch) {
-                fence_proxy_async_smem();
-                issue(c + 2);
-            }
-            // ---- M1: A = Q Kt^T
-            if (tid == 0) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc::mma_tf32(tA, tc::desc_kmajor(sm.Qs, k), tc::desc_kmajor(sm.Ks, k), kIdK_K, k > 0);
-                tc::mma_commit(&sm.mma_bar);
-            }
-            if (!mbar_wait_bounded(&sm.mma_bar, mma_phase)) failed = true;
-            mma_phase ^= 1;
-            tc::fence_after_sync();
-            // ---- E_A: strictly-lower mask, A -> As (unit over s, row p)
-            {
-                float a0[32], a1[32];
-                tc::tmem_ld32(tA + lane_off, a0);
-                tc::tmem_ld32(tA + lane_off + 32, a1);
-                tc::tmem_wait_ld();
-                if (rowlane) {
-#pragma unroll
-                    for (int u4 = 0; u4 < 16; ++u4) {
-                        float x[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int sc = 4 * u4 + e2;
-                            const float val = sc < 32 ? a0[sc] : a1[sc - 32];
-                            x[e2] = sc < prow ? val : 0.f;
-                        }
-                        *reinterpret_cast<float4 *>(&sm.As[u4][prow][0]) = make_float4(x[0], x[1], x[2], x[3]);
+            uint32_t ph_t = 0, ph_a = 0;
+            int s_seen = 0;   // s_ready phases observed
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                const int set = c & 1;
+                ok = wait_or_abort(sm, &sm.t_done, ph_t);
+                ph_t ^= 1;
+                if (!ok) break;
+                tc::fence_after_sync();
+                const bool flagged = *(volatile int *)&sm.flag[c & 3] == c + 1;
+                if (!flagged) {
+                    if (c + 2 < nch) {
+                        fence_proxy_async_smem();
+                        issue(c + 2);
+                        ++issued;
                     }
-                }
-            }
-            fence_proxy_async_smem();
-            tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
-            // ---- M2: Y = Q S_in + A V;  M3: S += Kt^T V
-            if (tid == 0) {
-                if (c > 0) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        tc::mma_tf32(tY, tc::desc_kmajor(sm.Qs, k), tc::desc_kmajor(sm.ST, k), kIdK_K, k > 0);
+                        tc::mma_tf32(tA, desc_sw(sm.Q[set], k), desc_sw(sm.K[set], k), kId, k > 0);
+                    tc::mma_commit(&sm.m1_done);
+                    ok = wait_or_abort(sm, &sm.a_done, ph_a);
+                    ph_a ^= 1;
+                    while (ok && s_seen <= c - 1) {
+                        ok = wait_or_abort(sm, &sm.s_ready, s_seen & 1);
+                        ++s_seen;
+                    }
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    if (c > 0) {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            tc::mma_tf32(tY, desc_sw(sm.Q[set], k), desc_sw(sm.ST, k), kId, k > 0);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        tc::mma_tf32(tY, desc_sw(sm.K[set], k), desc_sw(sm.VT[set], k), kId, c > 0 || k > 0);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        tc::mma_tf32(tS, desc_sw(sm.KT[set], k), desc_sw(sm.VT[set], k), kId, c > 0 || k > 0);
+                    tc::mma_commit(&sm.mma_done);
+                    tc::mma_commit(&sm.set_free[set]);
+                } else {
+                    // the transform warps evaluate this chunk exactly; they read the
+                    // raw stage until they publish the chunk's state
+                    while (ok && s_seen <= c) {
+                        ok = wait_or_abort(sm, &sm.s_ready, s_seen & 1);
+                        ++s_seen;
+                    }
+                    if (!ok) break;
+                    if (c + 2 < nch) {
+                        fence_proxy_async_smem();
+                        issue(c + 2);
+                        ++issued;
+                    }
+                    mbar_arrive(&sm.mma_done);
+                    mbar_arrive(&sm.set_free[set]);
                 }
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc::mma_tf32(tY, tc::desc_kmajor(sm.As, k), tc::desc_kmajor(sm.VT, k), kIdK_K, c > 0 || k > 0);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc::mma_tf32(tS, tc::desc_kmajor(sm.KT, k), tc::desc_kmajor(sm.VT, k), kIdK_K, c > 0 || k > 0);
-                tc::mma_commit(&sm.mma_bar);
             }
-            if (!mbar_wait_bounded(&sm.mma_bar, mma_phase)) failed = true;
-            mma_phase ^= 1;
+            // every MMA issued so far must finish before TMEM is released
+            tc::mma_commit(&sm.final_bar);
+            mbar_wait_bounded(&sm.final_bar, 0);
+            if (!ok) {
+                // let copies still in flight land before the CTA exits (bounded)
+                for (int cc = max(0, issued - 2); cc < issued; ++cc)
+                    mbar_wait_bounded(&sm.full[cc & 1], (cc >> 1) & 1);
+            }
+        }
+    } else if (warp <= kTW) {
+        // ===================== transform warps =====================
+        const int t = tid - 32;               // 0 .. kTT-1
+        const int i = t & (kHead - 1);        // channel (state row) of this thread
+        const int qtr = t >> 6;               // token range [kTokPerT*qtr, +kTokPerT)
+        const int p0 = kTokPerT * qtr;
+        const int tw = warp - 1;              // transform warp index
+        uint32_t ph_m1 = 0;
+        for (int c = 0; c < nch; ++c) {
+            const int set = c & 1, stg = c & 1;
+            const int t0 = c * kL;
+            // waits never make these threads leave early on their own: a timeout sets
+            // the shared abort flag, and all transform threads leave together at the
+            // first named barrier below, so none is left waiting at a barrier
+            bool ok = true;
+            if (c >= 2) ok = wait_or_abort(sm, &sm.set_free[set], ((c - 2) >> 1) & 1);
+            if (ok) ok = wait_or_abort(sm, &sm.full[stg], (c >> 1) & 1);
+            const auto &R = sm.raw[stg][R_];
+            const auto &Kr = sm.raw[stg][K_];
+            const auto &V = sm.raw[stg][V_];
+            const auto &W = sm.raw[stg][W_];
+            // ---- cumulative log-decay of this thread's tokens (exchange of quarter sums)
+            float ew[kTokPerT];
+            float local = 0.f;
+#pragma unroll
+            for (int e = 0; e < kTokPerT; ++e) {
+                ew[e] = raw_at(W, p0 + e, i);
+                local += ew[e];
+            }
+            sm.part_sum[qtr][i] = local;
+            named_sync(1, kTT);
+            if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
+            float L = 0.f;
+            for (int q = 0; q < qtr; ++q) L += sm.part_sum[q][i];
+            float lam[kTokPerT + 1];
+            float mx = fabsf(L);
+#pragma unroll
+            for (int e = 0; e < kTokPerT; ++e) {
+                lam[e] = L;
+                L += ew[e];
+                mx = fmaxf(mx, fabsf(L));
+            }
+            lam[kTokPerT] = L;
+            if (qtr == kTW / 2 - 1) sm.dec[c & 3][i] = __expf(L);
+            if (!(mx <= kLamMax)) atomicMax(&sm.flag[c & 3], c + 1);
+            // ---- bonus scalars c_p (warp reductions over the 64 channels)
+            for (int pp = 0; pp < kL / kTW; ++pp) {
+                const int p = tw * (kL / kTW) + pp;
+                float part = raw_at(R, p, lane) * sm.u[lane] * raw_at(Kr, p, lane) +
+                             raw_at(R, p, lane + 32) * sm.u[lane + 32] * raw_at(Kr, p, lane + 32);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                if (lane == 0) sm.cp[set][p] = part;
+            }
+            named_sync(1, kTT);
+            const bool flagged = *(volatile int *)&sm.flag[c & 3] == c + 1;
+            if (!flagged) {
+                // ---- chunk operands
+                float *Qs = sm.Q[set], *Ks = sm.K[set], *KT = sm.KT[set], *VT = sm.VT[set];
+#pragma unroll
+                for (int g = 0; g < kTokPerT / 4; ++g) {
+                    float kt4[4], v4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int p = p0 + 4 * g + e;
+                        const float q = raw_at(R, p, i) * __expf(lam[4 * g + e]);
+                        kt4[e] = raw_at(Kr, p, i) * __expf(-lam[4 * g + e + 1]);
+                        v4[e] = raw_at(V, p, i);
+                        Qs[swz(p, i)] = q;
+                        Ks[swz(p, i)] = kt4[e];
+                    }
+                    const int pb = p0 + 4 * g;
+                    *reinterpret_cast<float4 *>(&KT[swz(i, pb)]) = make_float4(kt4[0], kt4[1], kt4[2], kt4[3]);
+                    *reinterpret_cast<float4 *>(&VT[swz(i, pb)]) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.t_done);
+                // ---- masked A' = strict-lower(Q Kt^T) + diag(c) into the K buffer
+                wait_or_abort(sm, &sm.m1_done, ph_m1);   // on a timeout: garbage, then leave at the next barrier
+                ph_m1 ^= 1;
+                tc::fence_after_sync();
+                {
+                    const int col0 = 32 * (tw >> 2);        // warps 1..4 columns 0..31, warps 5..8 32..63
+                    float a[32];
+                    tc::tmem_ld32(tA + lane_off + col0, a);
+                    tc::tmem_wait_ld();
+                    if (rowlane) {
+                        const int p = qrow;
+                        const float cpp = sm.cp[set][p];
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            float x[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int s = col0 + 4 * g + e;
+                                x[e] = s < p ? a[4 * g + e] : (s == p ? cpp : 0.f);
+                            }
+                            *reinterpret_cast<float4 *>(&Ks[swz(p, col0 + 4 * g)]) = make_float4(x[0], x[1], x[2], x[3]);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc::fence_before_sync();
+                mbar_arrive(&sm.a_done);
+            } else {
+                mbar_arrive(&sm.t_done);
+                // ---- exact token-by-token evaluation of this chunk on the CUDA cores
+                if (c > 0) wait_or_abort(sm, &sm.s_ready, (c - 1) & 1);
+                tc::fence_after_sync();
+                const bool worker = tw < 4 && rowlane;   // warps 1..4 hold the 64 state rows
+                float Sr[64];
+                {
+                    float s0[32], s1[32];
+                    tc::tmem_ld32(tS + lane_off, s0);
+                    tc::tmem_ld32(tS + lane_off + 32, s1);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        Sr[j] = c > 0 ? s0[j] : 0.f;
+                        Sr[32 + j] = c > 0 ? s1[j] : 0.f;
+                    }
+                }
+                float *part = sm.Q[set];                  // [64 rows][64 cols] scratch
+                for (int p = 0; p < kL; ++p) {
+                    if (worker) {
+                        const float rr = raw_at(R, p, qrow);
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) part[qrow * 64 + j] = rr * Sr[j];
+                    }
+                    named_sync(1, kTT);
+                    if (t < kHead) {
+                        float acc = 0.f;
+                        for (int r = 0; r < kHead; ++r) acc += part[r * 64 + t];
+                        if (t0 + p < T)
+                            prm.y[((size_t)b * T + t0 + p) * C + cbase + t] = fmaf(sm.cp[set][p], raw_at(V, p, t), acc);
+                    }
+                    if (worker) {
+                        const float d = __expf(raw_at(W, p, qrow));
+                        const float kk = raw_at(Kr, p, qrow);
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) Sr[j] = fmaf(d, Sr[j], kk * raw_at(V, p, j));
+                    }
+                    named_sync(1, kTT);
+                }
+                {
+                    float s0[32], s1[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        s0[j] = Sr[j];
+                        s1[j] = Sr[32 + j];
+                    }
+                    if (tw < 4) {
+                        tc::tmem_st32(tS + lane_off, s0);
+                        tc::tmem_st32(tS + lane_off + 32, s1);
+                        tc::tmem_wait_st();
+                    }
+                    if (worker) {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) sm.ST[swz(j, qrow)] = Sr[j];
+                    }
+                }
+                fence_proxy_async_smem();
+                tc::fence_before_sync();
+                // the epilogue warps skip flagged chunks: the state hand-off is ours
+                for (int r = 0; r < kET / kTT + (t < kET % kTT ? 1 : 0); ++r) mbar_arrive(&sm.s_ready);
+            }
+        }
+    } else {
+        // ===================== epilogue warps =====================
+        const int e_t = tid - 32 * (1 + kTW);    // 0 .. kET-1
+        (void)e_t;
+        for (int c = 0; c < nch; ++c) {
+            const int set = c & 1;
+            const int t0 = c * kL;
+            if (!wait_or_abort(sm, &sm.mma_done, c & 1)) break;
             tc::fence_after_sync();
-            // ---- E_Y: y = Y + c_p v_p, straight to global
+            if (*(volatile int *)&sm.flag[c & 3] == c + 1) continue;
+            // ---- y = Y (the bonus is already on A's diagonal)
             {
                 float y0[32], y1[32];
                 tc::tmem_ld32(tY + lane_off, y0);
                 tc::tmem_ld32(tY + lane_off + 32, y1);
                 tc::tmem_wait_ld();
-                const int t = t0 + prow;
+                const int t = t0 + qrow;
                 if (rowlane && t < T) {
-                    float *dst = prm.y + ((size_t)b * T + t) * C + cbase;
-                    const float cp = sm.c[prow];
-                    const float *vrow = &sm.VT[prow >> 2][0][prow & 3];   // v_p[j] at vrow[4 * j]
+                    float4 *dst = reinterpret_cast<float4 *>(prm.y + ((size_t)b * T + t) * C + cbase);
 #pragma unroll
-                    for (int u4 = 0; u4 < 16; ++u4) {
-                        const float *src = u4 < 8 ? &y0[4 * u4] : &y1[4 * (u4 - 8)];
-                        *reinterpret_cast<float4 *>(dst + 4 * u4) =
-                            make_float4(fmaf(cp, vrow[4 * (4 * u4)], src[0]), fmaf(cp, vrow[4 * (4 * u4 + 1)], src[1]),
-                                        fmaf(cp, vrow[4 * (4 * u4 + 2)], src[2]), fmaf(cp, vrow[4 * (4 * u4 + 3)], src[3]));
-                    }
+                    for (int g = 0; g < 8; ++g) dst[g] = make_float4(y0[4 * g], y0[4 * g + 1], y0[4 * g + 2], y0[4 * g + 3]);
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        dst[8 + g] = make_float4(y1[4 * g], y1[4 * g + 1], y1[4 * g + 2], y1[4 * g + 3]);
                 }
             }
-            // ---- E_S: S rows scaled by exp(Lam_L); back to TMEM and to Ss for the next chunk
+            // ---- S rows scaled by exp(Lam_L); back to TMEM and transposed into ST
             {
                 float s0[32], s1[32];
                 tc::tmem_ld32(tS + lane_off, s0);
                 tc::tmem_ld32(tS + lane_off + 32, s1);
                 tc::tmem_wait_ld();
-                const float dsc = rowlane ? sm.dec[prow] : 0.f;
+                const float dsc = rowlane ? sm.dec[c & 3][qrow] : 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     s0[j] *= dsc;
@@ -278,86 +454,18 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 tc::tmem_st32(tS + lane_off, s0);
                 tc::tmem_st32(tS + lane_off + 32, s1);
                 if (rowlane) {
-                    float *dstT = &sm.ST[prow >> 2][0][prow & 3];         // S[i][j] at dstT[4 * j]
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        dstT[4 * j] = s0[j];
-                        dstT[4 * (32 + j)] = s1[j];
+                        sm.ST[swz(j, qrow)] = s0[j];
+                        sm.ST[swz(32 + j, qrow)] = s1[j];
                     }
                 }
                 tc::tmem_wait_st();
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
-        } else {
-            // ---- exact token-by-token fallback on the CUDA cores for this chunk
-            // state row i = prow (lane < 16) in registers; y via a shared-memory column sum
-            float Sr[64];
-            if (c > 0) {
-                float s0[32], s1[32];
-                tc::tmem_ld32(tS + lane_off, s0);
-                tc::tmem_ld32(tS + lane_off + 32, s1);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    Sr[j] = s0[j];
-                    Sr[32 + j] = s1[j];
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 64; ++j) Sr[j] = 0.f;
-            }
-            float (*part)[kHead] = reinterpret_cast<float (*)[kHead]>(&sm.As[0][0][0]);   // [64 rows][64 cols]
-            for (int p = 0; p < kL; ++p) {
-                if (rowlane) {
-                    const float rr = raw_at(sm.raw[s][R_], p, prow);
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) part[prow][j] = rr * Sr[j];
-                }
-                __syncthreads();
-                if (tid < kHead) {
-                    const int j = tid;
-                    float acc = 0.f;
-                    for (int i = 0; i < kHead; ++i) acc += part[i][j];
-                    const int t = t0 + p;
-                    if (t < T) prm.y[((size_t)b * T + t) * C + cbase + j] = fmaf(sm.c[p], raw_at(sm.raw[s][V_], p, j), acc);
-                }
-                if (rowlane) {
-                    const float d = __expf(raw_at(sm.raw[s][W_], p, prow));
-                    const float kk = raw_at(sm.raw[s][K_], p, prow);
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) Sr[j] = fmaf(d, Sr[j], kk * raw_at(sm.raw[s][V_], p, j));
-                }
-                __syncthreads();
-            }
-            {
-                float s0[32], s1[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    s0[j] = Sr[j];
-                    s1[j] = Sr[32 + j];
-                }
-                tc::tmem_st32(tS + lane_off, s0);
-                tc::tmem_st32(tS + lane_off + 32, s1);
-                if (rowlane) {
-                    float *dstT = &sm.ST[prow >> 2][0][prow & 3];
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) dstT[4 * j] = Sr[j];
-                }
-                tc::tmem_wait_st();
-            }
-            fence_proxy_async_smem();
-            tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
-            if (tid == 0 && c + 2 < nch) {
-                fence_proxy_async_smem();
-                issue(c + 2);
-            }
+            mbar_arrive(&sm.s_ready);
         }
-        if (failed) break;
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -367,10 +475,10 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
 
 cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
                                const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream) {
-    const size_t smem = sizeof(TcSmem) + 1024;
+    const size_t smem = sizeof(Tc2Smem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(wkv6_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    wkv6_fwd_tc_kernel<<<(unsigned)(prm.B * prm.H), 128, smem, stream>>>(mr, mk, mv, mw, prm);
+    wkv6_fwd_tc_kernel<<<(unsigned)(prm.B * prm.H), kThreads, smem, stream>>>(mr, mk, mv, mw, prm);
     return cudaGetLastError();
 }
 
