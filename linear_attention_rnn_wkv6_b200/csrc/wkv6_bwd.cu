@@ -92,7 +92,7 @@ __device__ __forceinline__ float reduce_cols_over_rows(const float (&yp)[4], boo
 }
 
 template <int TC, bool BIDIR>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 3)
 wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_v,
                 const __grid_constant__ CUtensorMap map_dy, BwdParams prm) {

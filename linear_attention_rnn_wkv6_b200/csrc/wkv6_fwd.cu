@@ -78,7 +78,7 @@ __device__ __forceinline__ ChunkPos chunk_pos(int g, int nch, int T, int TC, boo
 }
 
 template <typename Tin, int WARPS, int TC, bool BIDIR>
-__global__ void __launch_bounds__(32 * WARPS)
+__global__ void __launch_bounds__(32 * WARPS, 3)
 wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
                 FwdParams prm) {

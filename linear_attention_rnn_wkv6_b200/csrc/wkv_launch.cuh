@@ -18,8 +18,8 @@ struct BwdParams {
     float *du_part;   // [B][C] per-batch du partials (caller's workspace)
 };
 
-constexpr int kFwdTC = 32;   // tokens per TMA chunk, forward kernels
-constexpr int kBwdTC = 16;   // tokens per TMA chunk, backward kernel
+constexpr int kFwdTC = 16;   // tokens per TMA chunk, forward recurrence kernels
+constexpr int kBwdTC = 8;    // tokens per TMA chunk, backward kernel
 
 cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const CUtensorMap &mk,
                             const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
