@@ -44,7 +44,6 @@ constexpr int kEW = 4;                 // epilogue warps
 constexpr int kThreads = 32 * (1 + kTW + kEW);
 constexpr int kTT = 32 * kTW;          // transform threads
 constexpr int kET = 32 * kEW;          // epilogue threads
-constexpr int kTokPerT = kL / (kTT / kHead);   // tokens per transform thread (16)
 
 struct Tc2Smem {
     __nv_bfloat16 raw[2][4][kL][kHead];   // r, k, v, w stages (TMA, 128B-swizzled), 64 KB
@@ -55,7 +54,7 @@ struct Tc2Smem {
     float ST[kHead * kHead];              // S_in^T (row j, k = i)     B of M2
     float dec[4][kHead];                  // exp(Lam_L) per row (ring of 4 chunks)
     float cp[2][kL];                      // bonus scalars per token
-    float part_sum[kTW / 2][kHead];       // per-quarter log-decay sums (prefix exchange)
+    float part_sum[kTW][kHead];           // per-octet log2-decay sums (prefix exchange)
     float u[kHead];
     int flag[4];                          // chunk c is flagged iff flag[c & 3] == c + 1
     int abort_;
@@ -248,11 +247,15 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
         }
     } else if (warp <= kTW) {
         // ===================== transform warps =====================
+        // warp tw handles tokens [8 tw, 8 tw + 8) of the chunk; lane handles
+        // channels (2 lane, 2 lane + 1): bf16x2 loads, 8-byte Q / Kt stores and
+        // 16-byte stores of the transposed tiles, 8 independent tokens per thread.
         const int t = tid - 32;               // 0 .. kTT-1
-        const int i = t & (kHead - 1);        // channel (state row) of this thread
-        const int qtr = t >> 6;               // token range [kTokPerT*qtr, +kTokPerT)
-        const int p0 = kTokPerT * qtr;
-        const int tw = warp - 1;              // transform warp index
+        const int tw = warp - 1;              // transform warp index = token octet
+        const int ch = 2 * lane;              // first of this thread's two channels
+        const int p0 = 8 * tw;
+        const uint32_t raw_off = (uint32_t)(((lane & 3) << 2));   // byte offset inside the 16-byte chunk
+        const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
         uint32_t ph_m1 = 0;
         for (int c = 0; c < nch; ++c) {
             const int set = c & 1, stg = c & 1;
@@ -267,59 +270,104 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
             const auto &Kr = sm.raw[stg][K_];
             const auto &V = sm.raw[stg][V_];
             const auto &W = sm.raw[stg][W_];
-            // ---- cumulative log-decay of this thread's tokens (exchange of quarter sums)
-            float ew[kTokPerT];
-            float local = 0.f;
+            auto ld2 = [&](const __nv_bfloat16 (&tile)[kL][kHead], int e, float &a, float &b2) {
+                const int p = p0 + e;
+                const uint32_t off = (uint32_t)p * 128u + (((uint32_t)(lane >> 2) ^ (uint32_t)(e & 7)) << 4) + raw_off;
+                const uint32_t v = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(&tile[0][0]) + off);
+                a = __uint_as_float(v << 16);
+                b2 = __uint_as_float(v & 0xFFFF0000u);
+            };
+            // ---- cumulative log2-decay of this thread's 8 tokens, quarter exchange
+            float e0[8], e1[8];
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < kTokPerT; ++e) {
-                ew[e] = raw_at(W, p0 + e, i);
-                local += ew[e];
+            for (int e = 0; e < 8; ++e) {
+                ld2(W, e, e0[e], e1[e]);
+                e0[e] *= 1.4426950408889634f;
+                e1[e] *= 1.4426950408889634f;
+                s0 += e0[e];
+                s1 += e1[e];
             }
-            sm.part_sum[qtr][i] = local;
+            *reinterpret_cast<float2 *>(&sm.part_sum[tw][ch]) = make_float2(s0, s1);
             named_sync(1, kTT);
             if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
-            float L = 0.f;
-            for (int q = 0; q < qtr; ++q) L += sm.part_sum[q][i];
-            float lam[kTokPerT + 1];
-            float mx = fabsf(L);
-#pragma unroll
-            for (int e = 0; e < kTokPerT; ++e) {
-                lam[e] = L;
-                L += ew[e];
-                mx = fmaxf(mx, fabsf(L));
+            float L0 = 0.f, L1 = 0.f;
+            for (int q = 0; q < tw; ++q) {
+                const float2 ps = *reinterpret_cast<const float2 *>(&sm.part_sum[q][ch]);
+                L0 += ps.x;
+                L1 += ps.y;
             }
-            lam[kTokPerT] = L;
-            if (qtr == kTW / 2 - 1) sm.dec[c & 3][i] = __expf(L);
-            if (!(mx <= kLamMax)) atomicMax(&sm.flag[c & 3], c + 1);
-            // ---- bonus scalars c_p (warp reductions over the 64 channels)
-            for (int pp = 0; pp < kL / kTW; ++pp) {
-                const int p = tw * (kL / kTW) + pp;
-                float part = raw_at(R, p, lane) * sm.u[lane] * raw_at(Kr, p, lane) +
-                             raw_at(R, p, lane + 32) * sm.u[lane + 32] * raw_at(Kr, p, lane + 32);
+            float l0[9], l1[9];
+            float mx = fmaxf(fabsf(L0), fabsf(L1));
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-                if (lane == 0) sm.cp[set][p] = part;
+            for (int e = 0; e < 8; ++e) {
+                l0[e] = L0;
+                l1[e] = L1;
+                L0 += e0[e];
+                L1 += e1[e];
+                mx = fmaxf(mx, fmaxf(fabsf(L0), fabsf(L1)));
+            }
+            l0[8] = L0;
+            l1[8] = L1;
+            if (tw == kTW - 1) *reinterpret_cast<float2 *>(&sm.dec[c & 3][ch]) = make_float2(exp2f(L0), exp2f(L1));
+            if (!(mx <= kLamMax * 1.4426950408889634f)) atomicMax(&sm.flag[c & 3], c + 1);
+            // ---- r, k, v of the 8 tokens; bonus partials r u k
+            float r0[8], r1[8], k0[8], k1[8], v0[8], v1[8], bp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                ld2(R, e, r0[e], r1[e]);
+                ld2(Kr, e, k0[e], k1[e]);
+                ld2(V, e, v0[e], v1[e]);
+                bp[e] = fmaf(r0[e] * u0, k0[e], r1[e] * u1 * k1[e]);
+            }
+            // transpose-reduce the 8 partials over the 32 lanes: lane ends with token (lane >> 2)
+            {
+                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+                float a4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float keep = b4 ? bp[4 + q] : bp[q];
+                    const float send = b4 ? bp[q] : bp[4 + q];
+                    a4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+                float a2[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const float keep = b3 ? a4[2 + q] : a4[q];
+                    const float send = b3 ? a4[q] : a4[2 + q];
+                    a2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+                float a1 = (b2 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? a2[0] : a2[1], 4);
+                a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+                a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+                if ((lane & 3) == 0) sm.cp[set][p0 + (lane >> 2)] = a1;
             }
             named_sync(1, kTT);
             const bool flagged = *(volatile int *)&sm.flag[c & 3] == c + 1;
             if (!flagged) {
                 // ---- chunk operands
                 float *Qs = sm.Q[set], *Ks = sm.K[set], *KT = sm.KT[set], *VT = sm.VT[set];
+                float kt0[8], kt1[8];
 #pragma unroll
-                for (int g = 0; g < kTokPerT / 4; ++g) {
-                    float kt4[4], v4[4];
+                for (int e = 0; e < 8; ++e) {
+                    const int p = p0 + e;
+                    const float q0 = r0[e] * exp2f(l0[e]), q1 = r1[e] * exp2f(l1[e]);
+                    kt0[e] = k0[e] * exp2f(-l0[e + 1]);
+                    kt1[e] = k1[e] * exp2f(-l1[e + 1]);
+                    *reinterpret_cast<float2 *>(&Qs[swz(p, ch)]) = make_float2(q0, q1);
+                    *reinterpret_cast<float2 *>(&Ks[swz(p, ch)]) = make_float2(kt0[e], kt1[e]);
+                }
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int p = p0 + 4 * g + e;
-                        const float q = raw_at(R, p, i) * __expf(lam[4 * g + e]);
-                        kt4[e] = raw_at(Kr, p, i) * __expf(-lam[4 * g + e + 1]);
-                        v4[e] = raw_at(V, p, i);
-                        Qs[swz(p, i)] = q;
-                        Ks[swz(p, i)] = kt4[e];
-                    }
-                    const int pb = p0 + 4 * g;
-                    *reinterpret_cast<float4 *>(&KT[swz(i, pb)]) = make_float4(kt4[0], kt4[1], kt4[2], kt4[3]);
-                    *reinterpret_cast<float4 *>(&VT[swz(i, pb)]) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int pb = p0 + 4 * hh;
+                    *reinterpret_cast<float4 *>(&KT[swz(ch, pb)]) =
+                        make_float4(kt0[4 * hh], kt0[4 * hh + 1], kt0[4 * hh + 2], kt0[4 * hh + 3]);
+                    *reinterpret_cast<float4 *>(&KT[swz(ch + 1, pb)]) =
+                        make_float4(kt1[4 * hh], kt1[4 * hh + 1], kt1[4 * hh + 2], kt1[4 * hh + 3]);
+                    *reinterpret_cast<float4 *>(&VT[swz(ch, pb)]) =
+                        make_float4(v0[4 * hh], v0[4 * hh + 1], v0[4 * hh + 2], v0[4 * hh + 3]);
+                    *reinterpret_cast<float4 *>(&VT[swz(ch + 1, pb)]) =
+                        make_float4(v1[4 * hh], v1[4 * hh + 1], v1[4 * hh + 2], v1[4 * hh + 3]);
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.t_done);
@@ -418,7 +466,6 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
         const int e_t = tid - 32 * (1 + kTW);    // 0 .. kET-1
         (void)e_t;
         for (int c = 0; c < nch; ++c) {
-            const int set = c & 1;
             const int t0 = c * kL;
             if (!wait_or_abort(sm, &sm.mma_done, c & 1)) break;
             tc::fence_after_sync();
