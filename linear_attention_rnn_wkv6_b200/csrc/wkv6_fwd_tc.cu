@@ -4,32 +4,38 @@
 //   y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),   S_t = diag(d_t) S_{t-1} + k_t^T v_t.
 // The pages' parallel training form ("RWKV Architecture ...", The Parallel
 // Training Formulation) evaluates the decayed sums blockwise instead of token
-// by token; here a chunk of L = 64 tokens of one (b, h) is three dense
-// 64 x 64 x 64 contractions on tcgen05 (kind::tf32, fp32 accumulators in TMEM).
+// by token; here a chunk of L = 64 tokens of one (b, h) becomes three
+// tcgen05 contractions (kind::f16, bf16 operands, fp32 accumulators in tensor
+// memory; the state itself stays fp32 in tensor memory from chunk to chunk).
 //
 // Chunk algebra.  With Lam_p = sum_{m<p} ew_m (per row i, exclusive, chunk-local),
 // Q_p = r_p * exp(Lam_p), Kt_s = k_s * exp(-Lam_{s+1}) and c_p = sum_i r_p u k_p:
 //   y_p   = Q_p S_in + sum_{s<p} (Q_p . Kt_s) v_s + c_p v_p
 //   S_out = diag(exp(Lam_L)) (S_in + Kt^T V)
-//   M1  A  = Q Kt^T                                  (TMEM cols [0,64))
-//   M2  Y  = Q S_in + A' V,  A' = strict-lower(A) + diag(c)   (TMEM cols [64,128))
-//   M3  S += Kt^T V, then rows scaled by exp(Lam_L)  (TMEM cols [128,192))
-// All operands are K-major (TF32 operands in MN-major form give no result on
-// this hardware), staged in the 128-byte-swizzled canonical layout so both
-// row-wise and column-wise shared-memory writes are bank-conflict free; Kt is
-// kept in two orientations and V and S_in are stored transposed.
-// |Lam| <= 80 keeps exp(-Lam) inside fp32.  A chunk whose cumulative decay
-// leaves that range (fast-forgetting channels) is evaluated instead by the
-// exact token-by-token recurrence on the CUDA cores, starting from the state
-// held in TMEM, so any decay down to exactly 0 stays exact.
+// Every product is computed transposed, so that each operand is either a tile
+// exactly as the TMA wrote it or a tile a thread writes one contiguous row of:
+//   M1   A^T        = Kt Q^T                      (M = s, N = p, K = i; two TMEM buffers)
+//   P2   Y^T        = S_in^T Q^T                  (M = j, N = p, K = i)
+//   P34  [Y^T | S^T] += V^T [A'^T | Kt]           (M = j, N = 128, K = s; one instruction per K step)
+// where A' = strict-lower(A) + diag(c).  Q and Kt overwrite r and k in place in
+// the TMA stage (same 128-byte-swizzled row layout); V is used as loaded, as an
+// MN-major operand; Kt serves as K-major A of M1 and as MN-major half of P34's B.
+// After P34 the epilogue scales column i of S^T by exp(Lam_L[i]) in TMEM and
+// writes its bf16 copy S_in^T (K-major A of the next chunk's P2).
+// On this hardware a tcgen05.mma costs about the same issue time for any of
+// these shapes, so the kernel minimises the instruction count: 12 per chunk.
+// |Lam| <= 80 keeps exp(-Lam) inside fp32.  A chunk whose summed |ew| exceeds
+// that (fast-forgetting channels, decay down to exactly 0) is evaluated by the
+// exact token-by-token recurrence on the CUDA cores, from the state in TMEM.
 //
-// Warp roles (one CTA per (b, h), 13 warps):
-//   warp 0      TMA loads (2-stage ring) and, from one thread, all MMAs
-//   warps 1..8  transform: chunk operands for the MMAs, then the masked A'
-//   warps 9..12 epilogue: y out of TMEM, state rescale and its transposed copy
-// Operand sets are double buffered, so the transform of chunk c+1 overlaps the
-// MMAs and epilogue of chunk c.  Hand-offs are mbarriers; every wait is bounded
-// and a shared abort flag stops all roles after the first timeout.
+// Warp roles (one CTA per (b, h), 13 warps, two CTAs per SM):
+//   warp 0       TMA loads (2-stage ring) and, from one thread, all MMAs, issued
+//                as their inputs become ready
+//   warps 1..4   transform: Q, Kt, the bonus scalars c, exp(Lam_L), chunk flag
+//   warps 5..8   mask: A'^T from TMEM into shared memory
+//   warps 9..12  epilogue: y out of TMEM, state rescale, exact fallback chunks
+// Hand-offs are mbarriers; every wait is bounded and a shared abort flag stops
+// all roles after the first timeout.
 #include "wkv_launch.cuh"
 #include "wkv_tc.cuh"
 
@@ -37,60 +43,121 @@ namespace wkv {
 
 namespace {
 
-constexpr int kL = 64;                 // tokens per chunk
-constexpr float kLamMax = 80.0f;       // |Lam| bound of the tensor-core path
-constexpr int kTW = 8;                 // transform warps
-constexpr int kEW = 4;                 // epilogue warps
-constexpr int kThreads = 32 * (1 + kTW + kEW);
-constexpr int kTT = 32 * kTW;          // transform threads
-constexpr int kET = 32 * kEW;          // epilogue threads
-
-struct Tc2Smem {
-    __nv_bfloat16 raw[2][4][kL][kHead];   // r, k, v, w stages (TMA, 128B-swizzled), 64 KB
-    float Q[2][kL * kHead];               // (row p, k = i)            A of M1, M2
-    float K[2][kL * kHead];               // (row s, k = i), B of M1; then A' (row p, k = s), A of M2
-    float KT[2][kHead * kL];              // (row i, k = s)            A of M3
-    float VT[2][kHead * kL];              // (row j, k = s)            B of M2, M3
-    float ST[kHead * kHead];              // S_in^T (row j, k = i)     B of M2
-    float dec[4][kHead];                  // exp(Lam_L) per row (ring of 4 chunks)
-    float cp[2][kL];                      // bonus scalars per token
-    float part_sum[kTW][kHead];           // per-octet log2-decay sums (prefix exchange)
-    float u[kHead];
-    int flag[4];                          // chunk c is flagged iff flag[c & 3] == c + 1
-    int abort_;
-    uint32_t tmem_base;
-    alignas(8) uint64_t full[2];
-    alignas(8) uint64_t t_done, m1_done, a_done, mma_done, s_ready;
-    alignas(8) uint64_t set_free[2];
-    alignas(8) uint64_t final_bar;
-};
+constexpr int kL = 64;                       // tokens per chunk
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLamMax2 = 80.0f * kLog2e;   // |Lam| bound of the tensor-core path, log2 units
+constexpr int kTW = 4;                       // transform warps (16 tokens each)
+constexpr int kAW = 4;                       // mask warps
+constexpr int kEW = 4;                       // epilogue warps
+constexpr int kThreads = 32 * (1 + kTW + kAW + kEW);
+constexpr int kTT = 32 * kTW;
+constexpr int kAT = 32 * kAW;
+constexpr int kET = 32 * kEW;
+constexpr int kTokW = kL / kTW;              // tokens per transform warp
+constexpr int kTile = kL * kHead;            // bf16 elements of one 64 x 64 tile (8 KB)
 
 enum { R_ = 0, K_ = 1, V_ = 2, W_ = 3 };
 
-__device__ __forceinline__ float raw_at(const __nv_bfloat16 (&t)[kL][kHead], int row, int col) {
-    const int chunk = (col >> 3) ^ (row & 7);
-    return __bfloat162float(t[row][chunk * 8 + (col & 7)]);
+struct TcSmem {
+    __nv_bfloat16 Ap[2][kTile];          // A'^T (row s, p contiguous): first B atom of P34
+    __nv_bfloat16 SinT[kTile];           // bf16 S_in^T (row j, i contiguous): A of P2
+    __nv_bfloat16 raw[2][4][kTile];      // stages: r -> Q and k -> Kt in place, v, w (TMA, swizzled)
+    float dec[4][kHead];                 // exp(Lam_L) per row i (ring of 4 chunks)
+    float cp[4][kL];                     // bonus scalars per token (ring of 4 chunks)
+    float psum[2][kTW][kHead];           // per-warp log2-decay sums, by chunk parity
+    float pabs[2][kTW][kHead];           // per-warp sums of |log2-decay|
+    float u[kHead];
+    int flag[4];                         // chunk c is exact-evaluated iff flag[c & 3] == c + 1
+    int abort_;
+    uint32_t tmem_base;
+    alignas(8) uint64_t full[2];         // TMA stage landed
+    alignas(8) uint64_t t_done[2];       // transform of the stage's chunk done
+    alignas(8) uint64_t m1_done[2];      // per TMEM A buffer: A^T ready
+    alignas(8) uint64_t a_done[2];       // per TMEM A buffer: A'^T in shared memory, buffer read
+    alignas(8) uint64_t stage_free[2];   // every reader of the stage finished
+    alignas(8) uint64_t mma_done;        // Y^T and S^T of the chunk complete
+    alignas(8) uint64_t s_ready;         // y read out, state rescaled, S_in^T written
+    alignas(8) uint64_t final_bar;
+};
+
+// Byte offset of element (row, col) in a 64-row bf16 tile whose 128-byte rows
+// are 128B-swizzled (16-byte chunk g of row r stored at chunk g ^ (r & 7)).
+// This is the TMA's SWIZZLE_128B placement and, read through a descriptor, the
+// canonical K-major (rows along M/N) or MN-major (rows along K) layout.
+__device__ __forceinline__ uint32_t swz(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + ((col & 7) << 1));
 }
 
-// Float index of element (row r, k) of a 64 x 64 tf32 K-major tile in the
-// 128-byte-swizzled canonical layout: two K-blocks of [64 rows][32 floats],
-// 16-byte chunk c of row r stored at chunk c ^ (r & 7).
-__device__ __forceinline__ int swz(int r, int k) {
-    return (k >> 5) * 2048 + r * 32 + ((((k & 31) >> 2) ^ (r & 7)) << 2) + (k & 3);
+// K-major descriptor of the kstep-th group of 16 K values (32 bytes into each row).
+__device__ __forceinline__ uint64_t desc_k(const __nv_bfloat16 *tile, int kstep) {
+    return tc::smem_desc(reinterpret_cast<const char *>(tile) + kstep * 32, 16, 1024) | ((uint64_t)2 << 61);
+}
+// MN-major descriptor of the kstep-th group of 16 K rows; a second 64-wide MN
+// atom, if the instruction has one, starts lbo bytes after the first.
+__device__ __forceinline__ uint64_t desc_mn(const __nv_bfloat16 *tile, int kstep, uint32_t lbo) {
+    return tc::smem_desc(reinterpret_cast<const char *>(tile) + kstep * 2048, lbo, 1024) | ((uint64_t)2 << 61);
 }
 
-// Descriptor of the kstep-th group of 8 K values of such a tile.
-__device__ __forceinline__ uint64_t desc_sw(const float *tile, int kstep) {
-    const char *p = reinterpret_cast<const char *>(tile) + (kstep >> 2) * 8192 + (kstep & 3) * 32;
-    return tc::smem_desc(p, 16, 1024) | ((uint64_t)2 << 61);
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // .x = a (low half), .y = b
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ uint32_t ld_u32(const void *base, uint32_t off) {
+    return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(base) + off);
+}
+__device__ __forceinline__ void st_u32(void *base, uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(base) + off) = v;
+}
+__device__ __forceinline__ void st_u128(void *base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(base) + off) = v;
+}
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ float raw_at(const __nv_bfloat16 *tile, int row, int col) {
+    const uint32_t off = swz(row, col);
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(reinterpret_cast<const char *>(tile) + off));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Non-blocking: has the barrier phase with this parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Bounded wait that gives up at once when another thread has already aborted.
-__device__ __forceinline__ bool wait_or_abort(Tc2Smem &sm, uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool wait_or_abort(TcSmem &sm, uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
@@ -101,7 +168,7 @@ __device__ __forceinline__ bool wait_or_abort(Tc2Smem &sm, uint64_t *bar, uint32
             *(volatile int *)&sm.abort_ = 1;
             return false;
         }
-        __nanosleep(64);
+        __nanosleep(32);
     }
 }
 
@@ -109,21 +176,25 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+__device__ __forceinline__ bool is_flagged(const TcSmem &sm, int c) {
+    return *(const volatile int *)&sm.flag[c & 3] == c + 1;
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
                    FwdParams prm) {
     extern __shared__ unsigned char smem_dyn[];
-    Tc2Smem &sm = *reinterpret_cast<Tc2Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = prm.T, C = prm.C, H = prm.H;
     const int h = blockIdx.x % H, b = blockIdx.x / H;
     const int cbase = h * kHead;
     const int nch = (T + kL - 1) / kL;
-    constexpr uint32_t kStageBytes = 4u * kL * kHead * sizeof(__nv_bfloat16);
+    constexpr uint32_t kStageBytes = 4u * kTile * sizeof(__nv_bfloat16);
 
     if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
     if (tid < 4) sm.flag[tid] = 0;
@@ -133,15 +204,15 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
         prefetch_tensormap(&map_k);
         prefetch_tensormap(&map_v);
         prefetch_tensormap(&map_w);
-        mbar_init(&sm.full[0], 1);
-        mbar_init(&sm.full[1], 1);
-        mbar_init(&sm.t_done, kTT);
-        mbar_init(&sm.m1_done, 1);
-        mbar_init(&sm.a_done, kTT);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.t_done[i], kTT);
+            mbar_init(&sm.m1_done[i], 1);
+            mbar_init(&sm.a_done[i], kAT);
+            mbar_init(&sm.stage_free[i], 1);
+        }
         mbar_init(&sm.mma_done, 1);
         mbar_init(&sm.s_ready, kET);
-        mbar_init(&sm.set_free[0], 1);
-        mbar_init(&sm.set_free[1], 1);
         mbar_init(&sm.final_bar, 1);
         fence_barrier_init();
     }
@@ -152,362 +223,370 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    // TMEM columns: A^T buffers at 0 and 64, Y^T at 128, S^T at 192 (P34 writes 128..255)
     const uint32_t tbase = sm.tmem_base;
-    const uint32_t tA = tbase, tY = tbase + 64, tS = tbase + 128;
+    const uint32_t tY = tbase + 128, tS = tbase + 192;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lane quarter
-    const int qrow = 16 * (warp & 3) + lane;                          // accumulator row (lane < 16)
-    const bool rowlane = lane < 16;
-
-    auto issue = [&](int c) {
-        const int s = c & 1;
-        mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
-        tma_load_3d(&sm.raw[s][R_][0][0], &map_r, cbase, c * kL, b, &sm.full[s]);
-        tma_load_3d(&sm.raw[s][K_][0][0], &map_k, cbase, c * kL, b, &sm.full[s]);
-        tma_load_3d(&sm.raw[s][V_][0][0], &map_v, cbase, c * kL, b, &sm.full[s]);
-        tma_load_3d(&sm.raw[s][W_][0][0], &map_w, cbase, c * kL, b, &sm.full[s]);
-    };
+    const int qrow = 16 * (warp & 3) + (lane & 15);                 // accumulator row (M = 64 layout)
+    const bool rowlane = lane < 16;                                  // lanes 16..31 hold no row
 
     if (warp == 0) {
         // ===================== TMA + MMA issue (one thread) =====================
         if (lane == 0) {
-            constexpr uint32_t kId = tc::idesc_tf32(64, 64, false, false);
-            int issued = 0;
+            auto issue = [&](int c) {
+                const int s = c & 1;
+                mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+                tma_load_3d(sm.raw[s][R_], &map_r, cbase, c * kL, b, &sm.full[s]);
+                tma_load_3d(sm.raw[s][K_], &map_k, cbase, c * kL, b, &sm.full[s]);
+                tma_load_3d(sm.raw[s][V_], &map_v, cbase, c * kL, b, &sm.full[s]);
+                tma_load_3d(sm.raw[s][W_], &map_w, cbase, c * kL, b, &sm.full[s]);
+            };
+            constexpr uint32_t kIdKK = idesc_bf16(64, 64, false, false);
+            constexpr uint32_t kIdP34 = idesc_bf16(64, 128, true, true);
             issue(0);
-            ++issued;
-            if (nch > 1) {
-                issue(1);
-                ++issued;
-            }
-            uint32_t ph_t = 0, ph_a = 0;
-            int s_seen = 0;   // s_ready phases observed
+            if (nch > 1) issue(1);
+            int next_tma = nch > 1 ? 2 : 1;   // next chunk to load
+            int next_m1 = 0;                  // next chunk for M1
+            int next_p = 0;                   // next chunk for P2 / P34
+            bool p2_issued = false;           // P2 of chunk next_p issued, P34 pending
             bool ok = true;
-            for (int c = 0; c < nch && ok; ++c) {
-                const int set = c & 1;
-                ok = wait_or_abort(sm, &sm.t_done, ph_t);
-                ph_t ^= 1;
-                if (!ok) break;
-                tc::fence_after_sync();
-                const bool flagged = *(volatile int *)&sm.flag[c & 3] == c + 1;
-                if (!flagged) {
-                    if (c + 2 < nch) {
-                        fence_proxy_async_smem();
-                        issue(c + 2);
-                        ++issued;
-                    }
+            unsigned long long last = globaltimer_ns();
+            // Each step issues whatever has its inputs ready, the state chain
+            // (P34, then P2) first.  Invariants that keep every parity wait
+            // unambiguous: M1 runs at most one chunk ahead of P34, a stage is
+            // reloaded only after its chunk's last reader released it, and
+            // every chunk's a_done phase is observed before the chunk retires.
+            while (next_p < nch) {
+                bool progress = false;
+                if (p2_issued) {
+                    const int c = next_p, set = c & 1;
+                    if (mbar_test(&sm.a_done[set], (c >> 1) & 1)) {
+                        tc::fence_after_sync();
+                        const __nv_bfloat16 *V = sm.raw[set][V_];
+                        const uint32_t lbo = smem_u32(sm.raw[set][K_]) - smem_u32(sm.Ap[set]);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        tc::mma_tf32(tA, desc_sw(sm.Q[set], k), desc_sw(sm.K[set], k), kId, k > 0);
-                    tc::mma_commit(&sm.m1_done);
-                    ok = wait_or_abort(sm, &sm.a_done, ph_a);
-                    ph_a ^= 1;
-                    while (ok && s_seen <= c - 1) {
-                        ok = wait_or_abort(sm, &sm.s_ready, s_seen & 1);
-                        ++s_seen;
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(tY, desc_mn(V, k, 16), desc_mn(sm.Ap[set], k, lbo), kIdP34, true);
+                        tc::mma_commit(&sm.mma_done);
+                        tc::mma_commit(&sm.stage_free[set]);
+                        ++next_p;
+                        p2_issued = false;
+                        progress = true;
                     }
-                    if (!ok) break;
+                } else if (next_p < next_m1 && mbar_test(&sm.s_ready, next_p & 1)) {
+                    const int c = next_p, set = c & 1;
                     tc::fence_after_sync();
-                    if (c > 0) {
+                    if (!is_flagged(sm, c)) {
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            tc::mma_tf32(tY, desc_sw(sm.Q[set], k), desc_sw(sm.ST, k), kId, k > 0);
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(tY, desc_k(sm.SinT, k), desc_k(sm.raw[set][R_], k), kIdKK, k > 0);
+                        p2_issued = true;
+                        progress = true;
+                    } else if (mbar_test(&sm.a_done[set], (c >> 1) & 1)) {
+                        // the epilogue evaluates this chunk exactly and then releases its stage
+                        mbar_arrive(&sm.mma_done);
+                        ++next_p;
+                        progress = true;
                     }
+                }
+                if (next_m1 < nch && next_m1 <= next_p + 1) {
+                    const int c = next_m1, set = c & 1;
+                    if (mbar_test(&sm.t_done[set], (c >> 1) & 1)) {
+                        tc::fence_after_sync();
+                        if (!is_flagged(sm, c)) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        tc::mma_tf32(tY, desc_sw(sm.K[set], k), desc_sw(sm.VT[set], k), kId, c > 0 || k > 0);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        tc::mma_tf32(tS, desc_sw(sm.KT[set], k), desc_sw(sm.VT[set], k), kId, c > 0 || k > 0);
-                    tc::mma_commit(&sm.mma_done);
-                    tc::mma_commit(&sm.set_free[set]);
+                            for (int k = 0; k < 4; ++k)
+                                mma_bf16(tbase + 64 * set, desc_k(sm.raw[set][K_], k), desc_k(sm.raw[set][R_], k),
+                                         kIdKK, k > 0);
+                            tc::mma_commit(&sm.m1_done[set]);
+                        } else {
+                            mbar_arrive(&sm.m1_done[set]);   // the mask warps skip this chunk
+                        }
+                        ++next_m1;
+                        progress = true;
+                    }
+                }
+                if (next_tma < nch && mbar_test(&sm.stage_free[next_tma & 1], ((next_tma - 2) >> 1) & 1)) {
+                    fence_proxy_async_smem();
+                    issue(next_tma);
+                    ++next_tma;
+                    progress = true;
+                }
+                if (progress) {
+                    last = globaltimer_ns();
                 } else {
-                    // the transform warps evaluate this chunk exactly; they read the
-                    // raw stage until they publish the chunk's state
-                    while (ok && s_seen <= c) {
-                        ok = wait_or_abort(sm, &sm.s_ready, s_seen & 1);
-                        ++s_seen;
+                    if (*(volatile int *)&sm.abort_) {
+                        ok = false;
+                        break;
                     }
-                    if (!ok) break;
-                    if (c + 2 < nch) {
-                        fence_proxy_async_smem();
-                        issue(c + 2);
-                        ++issued;
+                    if (globaltimer_ns() - last > kWaitLimitNs) {
+                        atomicOr(&g_wkv_faults, WKV_FAULT_TIMEOUT);
+                        *(volatile int *)&sm.abort_ = 1;
+                        ok = false;
+                        break;
                     }
-                    mbar_arrive(&sm.mma_done);
-                    mbar_arrive(&sm.set_free[set]);
                 }
             }
             // every MMA issued so far must finish before TMEM is released
             tc::mma_commit(&sm.final_bar);
             mbar_wait_bounded(&sm.final_bar, 0);
             if (!ok) {
-                // let copies still in flight land before the CTA exits (bounded)
-                for (int cc = max(0, issued - 2); cc < issued; ++cc)
+                for (int cc = max(0, next_tma - 2); cc < next_tma; ++cc)
                     mbar_wait_bounded(&sm.full[cc & 1], (cc >> 1) & 1);
             }
         }
     } else if (warp <= kTW) {
         // ===================== transform warps =====================
-        // warp tw handles tokens [8 tw, 8 tw + 8) of the chunk; lane handles
-        // channels (2 lane, 2 lane + 1): bf16x2 loads, 8-byte Q / Kt stores and
-        // 16-byte stores of the transposed tiles, 8 independent tokens per thread.
-        const int t = tid - 32;               // 0 .. kTT-1
-        const int tw = warp - 1;              // transform warp index = token octet
-        const int ch = 2 * lane;              // first of this thread's two channels
-        const int p0 = 8 * tw;
-        const uint32_t raw_off = (uint32_t)(((lane & 3) << 2));   // byte offset inside the 16-byte chunk
+        // warp tw handles tokens [16 tw, 16 tw + 16) of the chunk; lane handles
+        // channels (2 lane, 2 lane + 1), i.e. 4 bytes of 16-byte chunk lane / 4
+        const int tw = warp - 1;
+        const int ch = 2 * lane;
+        const int p0 = kTokW * tw;
+        const uint32_t in_chunk = (uint32_t)(lane & 3) << 2;
+        const uint32_t chunk = (uint32_t)(lane >> 2);
         const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
-        uint32_t ph_m1 = 0;
         for (int c = 0; c < nch; ++c) {
-            const int set = c & 1, stg = c & 1;
-            const int t0 = c * kL;
-            // waits never make these threads leave early on their own: a timeout sets
-            // the shared abort flag, and all transform threads leave together at the
-            // first named barrier below, so none is left waiting at a barrier
-            bool ok = true;
-            if (c >= 2) ok = wait_or_abort(sm, &sm.set_free[set], ((c - 2) >> 1) & 1);
-            if (ok) ok = wait_or_abort(sm, &sm.full[stg], (c >> 1) & 1);
-            const auto &R = sm.raw[stg][R_];
-            const auto &Kr = sm.raw[stg][K_];
-            const auto &V = sm.raw[stg][V_];
-            const auto &W = sm.raw[stg][W_];
-            auto ld2 = [&](const __nv_bfloat16 (&tile)[kL][kHead], int e, float &a, float &b2) {
+            const int stg = c & 1, par = c & 1;
+            // a timeout sets the shared abort flag; all transform threads leave
+            // together after the named barrier below, so none is left waiting there
+            wait_or_abort(sm, &sm.full[stg], (c >> 1) & 1);
+            __nv_bfloat16 *Rb = sm.raw[stg][R_], *Kb = sm.raw[stg][K_];
+            const __nv_bfloat16 *Wb = sm.raw[stg][W_];
+            auto off = [&](int e) -> uint32_t {
                 const int p = p0 + e;
-                const uint32_t off = (uint32_t)p * 128u + (((uint32_t)(lane >> 2) ^ (uint32_t)(e & 7)) << 4) + raw_off;
-                const uint32_t v = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(&tile[0][0]) + off);
-                a = __uint_as_float(v << 16);
-                b2 = __uint_as_float(v & 0xFFFF0000u);
+                return (uint32_t)p * 128u + ((chunk ^ (uint32_t)(p & 7)) << 4) + in_chunk;
             };
-            // ---- cumulative log2-decay of this thread's 8 tokens, quarter exchange
-            float e0[8], e1[8];
-            float s0 = 0.f, s1 = 0.f;
+            // ---- log2-decay sums of this warp's 16 tokens (signed and absolute)
+            float s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                ld2(W, e, e0[e], e1[e]);
-                e0[e] *= 1.4426950408889634f;
-                e1[e] *= 1.4426950408889634f;
-                s0 += e0[e];
-                s1 += e1[e];
+            for (int e = 0; e < kTokW; ++e) {
+                const uint32_t wv = ld_u32(Wb, off(e));
+                const float x0 = bf_lo(wv) * kLog2e, x1 = bf_hi(wv) * kLog2e;
+                s0 += x0;
+                s1 += x1;
+                a0 += fabsf(x0);
+                a1 += fabsf(x1);
             }
-            *reinterpret_cast<float2 *>(&sm.part_sum[tw][ch]) = make_float2(s0, s1);
+            *reinterpret_cast<float2 *>(&sm.psum[par][tw][ch]) = make_float2(s0, s1);
+            *reinterpret_cast<float2 *>(&sm.pabs[par][tw][ch]) = make_float2(a0, a1);
             named_sync(1, kTT);
             if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
-            float L0 = 0.f, L1 = 0.f;
-            for (int q = 0; q < tw; ++q) {
-                const float2 ps = *reinterpret_cast<const float2 *>(&sm.part_sum[q][ch]);
-                L0 += ps.x;
-                L1 += ps.y;
-            }
-            float l0[9], l1[9];
-            float mx = fmaxf(fabsf(L0), fabsf(L1));
+            float L0 = 0.f, L1 = 0.f, tot0 = 0.f, tot1 = 0.f, ab0 = 0.f, ab1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                l0[e] = L0;
-                l1[e] = L1;
-                L0 += e0[e];
-                L1 += e1[e];
-                mx = fmaxf(mx, fmaxf(fabsf(L0), fabsf(L1)));
+            for (int q = 0; q < kTW; ++q) {
+                const float2 ps = *reinterpret_cast<const float2 *>(&sm.psum[par][q][ch]);
+                const float2 pa = *reinterpret_cast<const float2 *>(&sm.pabs[par][q][ch]);
+                if (q < tw) {
+                    L0 += ps.x;
+                    L1 += ps.y;
+                }
+                tot0 += ps.x;
+                tot1 += ps.y;
+                ab0 += pa.x;
+                ab1 += pa.y;
             }
-            l0[8] = L0;
-            l1[8] = L1;
-            if (tw == kTW - 1) *reinterpret_cast<float2 *>(&sm.dec[c & 3][ch]) = make_float2(exp2f(L0), exp2f(L1));
-            if (!(mx <= kLamMax * 1.4426950408889634f)) atomicMax(&sm.flag[c & 3], c + 1);
-            // ---- r, k, v of the 8 tokens; bonus partials r u k
-            float r0[8], r1[8], k0[8], k1[8], v0[8], v1[8], bp[8];
+            // sum |ew| bounds every |Lam_p| of the chunk; every warp reads the same
+            // sums in the same order, so all four reach the same verdict
+            const bool flagged = __any_sync(0xffffffffu, !(ab0 <= kLamMax2) || !(ab1 <= kLamMax2));
+            if (tw == 0) {
+                *reinterpret_cast<float2 *>(&sm.dec[c & 3][ch]) = make_float2(exp2f(tot0), exp2f(tot1));
+                if (lane == 0 && flagged) sm.flag[c & 3] = c + 1;
+            }
+            // ---- Q and Kt in place of r and k; bonus partials r u k
+            float bp[kTokW];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                ld2(R, e, r0[e], r1[e]);
-                ld2(Kr, e, k0[e], k1[e]);
-                ld2(V, e, v0[e], v1[e]);
-                bp[e] = fmaf(r0[e] * u0, k0[e], r1[e] * u1 * k1[e]);
+            for (int e = 0; e < kTokW; ++e) {
+                const uint32_t o = off(e);
+                const uint32_t rv = ld_u32(Rb, o), kv = ld_u32(Kb, o);
+                const float r0 = bf_lo(rv), r1 = bf_hi(rv), k0 = bf_lo(kv), k1 = bf_hi(kv);
+                bp[e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
+                if (!flagged) {
+                    const uint32_t wv = ld_u32(Wb, o);
+                    const float q0 = r0 * fast_exp2(L0), q1 = r1 * fast_exp2(L1);
+                    L0 += bf_lo(wv) * kLog2e;
+                    L1 += bf_hi(wv) * kLog2e;
+                    st_u32(Rb, o, pack_bf16(q0, q1));
+                    st_u32(Kb, o, pack_bf16(k0 * fast_exp2(-L0), k1 * fast_exp2(-L1)));
+                }
             }
-            // transpose-reduce the 8 partials over the 32 lanes: lane ends with token (lane >> 2)
+            // transpose-reduce the 16 partials over the 32 lanes: lanes 2m, 2m+1 end with token m
             {
-                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+                float a8[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float keep = b4 ? bp[8 + q] : bp[q];
+                    const float send = b4 ? bp[q] : bp[8 + q];
+                    a8[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
                 float a4[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float keep = b4 ? bp[4 + q] : bp[q];
-                    const float send = b4 ? bp[q] : bp[4 + q];
-                    a4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                    const float keep = b3 ? a8[4 + q] : a8[q];
+                    const float send = b3 ? a8[q] : a8[4 + q];
+                    a4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
                 }
                 float a2[2];
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
-                    const float keep = b3 ? a4[2 + q] : a4[q];
-                    const float send = b3 ? a4[q] : a4[2 + q];
-                    a2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                    const float keep = b2 ? a4[2 + q] : a4[q];
+                    const float send = b2 ? a4[q] : a4[2 + q];
+                    a2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
                 }
-                float a1 = (b2 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? a2[0] : a2[1], 4);
-                a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
-                a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
-                if ((lane & 3) == 0) sm.cp[set][p0 + (lane >> 2)] = a1;
+                float a1s = (b1 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? a2[0] : a2[1], 2);
+                a1s += __shfl_xor_sync(0xffffffffu, a1s, 1);
+                if ((lane & 1) == 0) sm.cp[c & 3][p0 + (lane >> 1)] = a1s;
             }
-            named_sync(1, kTT);
-            const bool flagged = *(volatile int *)&sm.flag[c & 3] == c + 1;
-            if (!flagged) {
-                // ---- chunk operands
-                float *Qs = sm.Q[set], *Ks = sm.K[set], *KT = sm.KT[set], *VT = sm.VT[set];
-                float kt0[8], kt1[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int p = p0 + e;
-                    const float q0 = r0[e] * exp2f(l0[e]), q1 = r1[e] * exp2f(l1[e]);
-                    kt0[e] = k0[e] * exp2f(-l0[e + 1]);
-                    kt1[e] = k1[e] * exp2f(-l1[e + 1]);
-                    *reinterpret_cast<float2 *>(&Qs[swz(p, ch)]) = make_float2(q0, q1);
-                    *reinterpret_cast<float2 *>(&Ks[swz(p, ch)]) = make_float2(kt0[e], kt1[e]);
-                }
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int pb = p0 + 4 * hh;
-                    *reinterpret_cast<float4 *>(&KT[swz(ch, pb)]) =
-                        make_float4(kt0[4 * hh], kt0[4 * hh + 1], kt0[4 * hh + 2], kt0[4 * hh + 3]);
-                    *reinterpret_cast<float4 *>(&KT[swz(ch + 1, pb)]) =
-                        make_float4(kt1[4 * hh], kt1[4 * hh + 1], kt1[4 * hh + 2], kt1[4 * hh + 3]);
-                    *reinterpret_cast<float4 *>(&VT[swz(ch, pb)]) =
-                        make_float4(v0[4 * hh], v0[4 * hh + 1], v0[4 * hh + 2], v0[4 * hh + 3]);
-                    *reinterpret_cast<float4 *>(&VT[swz(ch + 1, pb)]) =
-                        make_float4(v1[4 * hh], v1[4 * hh + 1], v1[4 * hh + 2], v1[4 * hh + 3]);
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&sm.t_done);
-                // ---- masked A' = strict-lower(Q Kt^T) + diag(c) into the K buffer
-                wait_or_abort(sm, &sm.m1_done, ph_m1);   // on a timeout: garbage, then leave at the next barrier
-                ph_m1 ^= 1;
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.t_done[stg]);
+        }
+    } else if (warp <= kTW + kAW) {
+        // ===================== mask warps: A'^T = strict-upper(A^T) + diag(c) =====================
+        const int s = qrow;
+        for (int c = 0; c < nch; ++c) {
+            const int set = c & 1;
+            if (!wait_or_abort(sm, &sm.m1_done[set], (c >> 1) & 1)) break;
+            if (!is_flagged(sm, c)) {
                 tc::fence_after_sync();
-                {
-                    const int col0 = 32 * (tw >> 2);        // warps 1..4 columns 0..31, warps 5..8 32..63
+                const float cps = sm.cp[c & 3][s];
+                __nv_bfloat16 *Ab = sm.Ap[set];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
                     float a[32];
-                    tc::tmem_ld32(tA + lane_off + col0, a);
+                    tc::tmem_ld32(tbase + 64 * set + lane_off + 32 * half, a);
                     tc::tmem_wait_ld();
                     if (rowlane) {
-                        const int p = qrow;
-                        const float cpp = sm.cp[set][p];
 #pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            float x[4];
+                        for (int g = 0; g < 4; ++g) {
+                            float x[8];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int s = col0 + 4 * g + e;
-                                x[e] = s < p ? a[4 * g + e] : (s == p ? cpp : 0.f);
+                            for (int e = 0; e < 8; ++e) {
+                                const int p = 32 * half + 8 * g + e;
+                                x[e] = p > s ? a[8 * g + e] : (p == s ? cps : 0.f);
                             }
-                            *reinterpret_cast<float4 *>(&Ks[swz(p, col0 + 4 * g)]) = make_float4(x[0], x[1], x[2], x[3]);
+                            st_u128(Ab, swz(s, 32 * half + 8 * g),
+                                    make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                               pack_bf16(x[6], x[7])));
                         }
                     }
                 }
                 fence_proxy_async_smem();
                 tc::fence_before_sync();
-                mbar_arrive(&sm.a_done);
-            } else {
-                mbar_arrive(&sm.t_done);
-                // ---- exact token-by-token evaluation of this chunk on the CUDA cores
-                if (c > 0) wait_or_abort(sm, &sm.s_ready, (c - 1) & 1);
-                tc::fence_after_sync();
-                const bool worker = tw < 4 && rowlane;   // warps 1..4 hold the 64 state rows
-                float Sr[64];
-                {
-                    float s0[32], s1[32];
-                    tc::tmem_ld32(tS + lane_off, s0);
-                    tc::tmem_ld32(tS + lane_off + 32, s1);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        Sr[j] = c > 0 ? s0[j] : 0.f;
-                        Sr[32 + j] = c > 0 ? s1[j] : 0.f;
-                    }
-                }
-                float *part = sm.Q[set];                  // [64 rows][64 cols] scratch
-                for (int p = 0; p < kL; ++p) {
-                    if (worker) {
-                        const float rr = raw_at(R, p, qrow);
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) part[qrow * 64 + j] = rr * Sr[j];
-                    }
-                    named_sync(1, kTT);
-                    if (t < kHead) {
-                        float acc = 0.f;
-                        for (int r = 0; r < kHead; ++r) acc += part[r * 64 + t];
-                        if (t0 + p < T)
-                            prm.y[((size_t)b * T + t0 + p) * C + cbase + t] = fmaf(sm.cp[set][p], raw_at(V, p, t), acc);
-                    }
-                    if (worker) {
-                        const float d = __expf(raw_at(W, p, qrow));
-                        const float kk = raw_at(Kr, p, qrow);
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) Sr[j] = fmaf(d, Sr[j], kk * raw_at(V, p, j));
-                    }
-                    named_sync(1, kTT);
-                }
-                {
-                    float s0[32], s1[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        s0[j] = Sr[j];
-                        s1[j] = Sr[32 + j];
-                    }
-                    if (tw < 4) {
-                        tc::tmem_st32(tS + lane_off, s0);
-                        tc::tmem_st32(tS + lane_off + 32, s1);
-                        tc::tmem_wait_st();
-                    }
-                    if (worker) {
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) sm.ST[swz(j, qrow)] = Sr[j];
-                    }
-                }
-                fence_proxy_async_smem();
-                tc::fence_before_sync();
-                // the epilogue warps skip flagged chunks: the state hand-off is ours
-                for (int r = 0; r < kET / kTT + (t < kET % kTT ? 1 : 0); ++r) mbar_arrive(&sm.s_ready);
             }
+            // every chunk arrives once, so the buffer's phase count stays chunk >> 1
+            mbar_arrive(&sm.a_done[set]);
         }
     } else {
         // ===================== epilogue warps =====================
-        const int e_t = tid - 32 * (1 + kTW);    // 0 .. kET-1
-        (void)e_t;
+        const int et = tid - 32 * (1 + kTW + kAW);   // 0 .. kET-1
+        const int j = qrow;                           // S^T / Y^T row served by this lane
+        // the state starts at zero: S^T in TMEM and its bf16 copy
+        {
+            float z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0.f;
+            tc::tmem_st32(tS + lane_off, z);
+            tc::tmem_st32(tS + lane_off + 32, z);
+            uint4 *st = reinterpret_cast<uint4 *>(sm.SinT);
+            for (int i = et; i < kTile * 2 / 16; i += kET) st[i] = make_uint4(0u, 0u, 0u, 0u);
+            tc::tmem_wait_st();
+            fence_proxy_async_smem();
+            tc::fence_before_sync();
+            mbar_arrive(&sm.s_ready);
+        }
         for (int c = 0; c < nch; ++c) {
-            const int t0 = c * kL;
-            if (!wait_or_abort(sm, &sm.mma_done, c & 1)) break;
+            const int t0 = c * kL, stg = c & 1;
+            const int pmax = min(kL, T - t0);
+            wait_or_abort(sm, &sm.mma_done, c & 1);
+            named_sync(2, kET);
+            if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
             tc::fence_after_sync();
-            if (*(volatile int *)&sm.flag[c & 3] == c + 1) continue;
-            // ---- y = Y (the bonus is already on A's diagonal)
-            {
-                float y0[32], y1[32];
-                tc::tmem_ld32(tY + lane_off, y0);
-                tc::tmem_ld32(tY + lane_off + 32, y1);
-                tc::tmem_wait_ld();
-                const int t = t0 + qrow;
-                if (rowlane && t < T) {
-                    float4 *dst = reinterpret_cast<float4 *>(prm.y + ((size_t)b * T + t) * C + cbase);
+            float *ycol = prm.y + ((size_t)b * T + t0) * C + cbase + j;
+            if (!is_flagged(sm, c)) {
+                // ---- y: row j of Y^T is channel j of the chunk's 64 outputs
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) dst[g] = make_float4(y0[4 * g], y0[4 * g + 1], y0[4 * g + 2], y0[4 * g + 3]);
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tc::tmem_ld32(tY + lane_off + 32 * half, v);
+                    tc::tmem_wait_ld();
+                    if (rowlane) {
 #pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        dst[8 + g] = make_float4(y1[4 * g], y1[4 * g + 1], y1[4 * g + 2], y1[4 * g + 3]);
+                        for (int e = 0; e < 32; ++e) {
+                            const int p = 32 * half + e;
+                            if (p < pmax) ycol[(size_t)p * C] = v[e];
+                        }
+                    }
                 }
-            }
-            // ---- S rows scaled by exp(Lam_L); back to TMEM and transposed into ST
-            {
-                float s0[32], s1[32];
-                tc::tmem_ld32(tS + lane_off, s0);
-                tc::tmem_ld32(tS + lane_off + 32, s1);
-                tc::tmem_wait_ld();
-                const float dsc = rowlane ? sm.dec[c & 3][qrow] : 0.f;
+                // ---- S^T columns scaled by exp(Lam_L), back to TMEM, bf16 copy into S_in^T
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    s0[j] *= dsc;
-                    s1[j] *= dsc;
-                }
-                tc::tmem_st32(tS + lane_off, s0);
-                tc::tmem_st32(tS + lane_off + 32, s1);
-                if (rowlane) {
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tc::tmem_ld32(tS + lane_off + 32 * half, v);
+                    tc::tmem_wait_ld();
+                    const float4 *dq = reinterpret_cast<const float4 *>(&sm.dec[c & 3][32 * half]);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        sm.ST[swz(j, qrow)] = s0[j];
-                        sm.ST[swz(32 + j, qrow)] = s1[j];
+                    for (int g = 0; g < 8; ++g) {
+                        const float4 d = dq[g];
+                        v[4 * g] *= d.x;
+                        v[4 * g + 1] *= d.y;
+                        v[4 * g + 2] *= d.z;
+                        v[4 * g + 3] *= d.w;
+                    }
+                    tc::tmem_st32(tS + lane_off + 32 * half, v);
+                    if (rowlane) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            st_u128(sm.SinT, swz(j, 32 * half + 8 * g),
+                                    make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]), pack_bf16(v[8 * g + 2], v[8 * g + 3]),
+                                               pack_bf16(v[8 * g + 4], v[8 * g + 5]),
+                                               pack_bf16(v[8 * g + 6], v[8 * g + 7])));
                     }
                 }
                 tc::tmem_wait_st();
+            } else {
+                // ---- exact token-by-token evaluation of this chunk on the CUDA cores:
+                // lane j owns column j of S (row j of S^T in TMEM)
+                const __nv_bfloat16 *R = sm.raw[stg][R_], *Kr = sm.raw[stg][K_];
+                const __nv_bfloat16 *V = sm.raw[stg][V_], *W = sm.raw[stg][W_];
+                for (int p = 0; p < kL; ++p) {
+                    const float vj = raw_at(V, p, j);
+                    float acc = 0.f;
+#pragma unroll 1
+                    for (int m = 0; m < 4; ++m) {
+                        float sv[16];
+                        tc::tmem_ld16(tS + lane_off + 16 * m, sv);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int i = 16 * m + e;
+                            acc = fmaf(raw_at(R, p, i), sv[e], acc);
+                            sv[e] = fmaf(__expf(raw_at(W, p, i)), sv[e], raw_at(Kr, p, i) * vj);
+                        }
+                        tc::tmem_st16(tS + lane_off + 16 * m, sv);
+                        tc::tmem_wait_st();
+                    }
+                    if (rowlane && p < pmax) ycol[(size_t)p * C] = fmaf(sm.cp[c & 3][p], vj, acc);
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tc::tmem_ld32(tS + lane_off + 32 * half, v);
+                    tc::tmem_wait_ld();
+                    if (rowlane) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            st_u128(sm.SinT, swz(j, 32 * half + 8 * g),
+                                    make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]), pack_bf16(v[8 * g + 2], v[8 * g + 3]),
+                                               pack_bf16(v[8 * g + 4], v[8 * g + 5]),
+                                               pack_bf16(v[8 * g + 6], v[8 * g + 7])));
+                    }
+                }
+                // every epilogue thread is done with the raw stage: release it
+                named_sync(2, kET);
+                if (et == 0) {
+                    fence_proxy_async_smem();
+                    mbar_arrive(&sm.stage_free[stg]);
+                }
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
@@ -522,8 +601,11 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
 
 cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
                                const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream) {
-    const size_t smem = sizeof(Tc2Smem) + 1024;
+    const size_t smem = sizeof(TcSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(wkv6_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(wkv6_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     wkv6_fwd_tc_kernel<<<(unsigned)(prm.B * prm.H), kThreads, smem, stream>>>(mr, mk, mv, mw, prm);
     return cudaGetLastError();

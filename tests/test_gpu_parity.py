@@ -58,8 +58,10 @@ def bf16_path(request, monkeypatch):
 
 def _bf16_bound(path):
     # the oracle sees the same rounded inputs: the recurrence differs only by fp32
-    # rounding; the tensor-core path rounds its chunk operands to tf32 (10-bit mantissa)
-    return 1e-5 if path == "recurrence" else 2e-3
+    # rounding; the tensor-core path rounds its chunk operands (decay-scaled r and k,
+    # the masked chunk matrix and the carried state) to bf16 for the MMAs, about
+    # 3e-3 relative L2, inside the 2e-2 tolerance of bf16 inputs
+    return 1e-5 if path == "recurrence" else 6e-3
 
 
 @pytest.mark.parametrize("B,T,H", [(1, 1, 1), (2, 33, 2), (1, 64, 1), (1, 65, 2), (1, 97, 3), (2, 256, 2)])
