@@ -12,16 +12,19 @@
 // Q_p = r_p * exp(Lam_p), Kt_s = k_s * exp(-Lam_{s+1}) and c_p = sum_i r_p u k_p:
 //   y_p   = Q_p S_in + sum_{s<p} (Q_p . Kt_s) v_s + c_p v_p
 //   S_out = diag(exp(Lam_L)) (S_in + Kt^T V)
-// Every product is computed transposed, so that each operand is either a tile
-// exactly as the TMA wrote it or a tile a thread writes one contiguous row of:
-//   M1   A^T        = Kt Q^T                      (M = s, N = p, K = i; two TMEM buffers)
-//   P2   Y^T        = S_in^T Q^T                  (M = j, N = p, K = i)
-//   P34  [Y^T | S^T] += V^T [A'^T | Kt]           (M = j, N = 128, K = s; one instruction per K step)
-// where A' = strict-lower(A) + diag(c).  Q and Kt overwrite r and k in place in
-// the TMA stage (same 128-byte-swizzled row layout); V is used as loaded, as an
-// MN-major operand; Kt serves as K-major A of M1 and as MN-major half of P34's B.
-// After P34 the epilogue scales column i of S^T by exp(Lam_L[i]) in TMEM and
-// writes its bf16 copy S_in^T (K-major A of the next chunk's P2).
+// The products are arranged so that every operand is either a tile exactly as
+// the TMA wrote it or a tile whose rows a thread writes contiguously:
+//   M1   A^T          = Kt Q^T                 (M = 64 (s), N = 64 (p), K = i; two TMEM buffers)
+//   P2   [Y ; S]     += [Q ; 0] S_in           (M = 128, N = 64 (j), K = i)
+//   P34  [Y ; S]     += [A' ; Kt^T] V          (M = 128, N = 64 (j), K = s)
+// where A' = strict-lower(A) + diag(c).  One M = 128 accumulator holds Y in
+// TMEM lanes 0..63 (row p) and the fp32 state S in lanes 64..127 (row i).
+// Q and Kt overwrite r and k in place in the TMA stage (same 128-byte-swizzled
+// rows); an all-zero tile follows Q so that [Q ; 0] is one K-major operand;
+// A'^T (written row s by row s) and Kt form the two 64-wide atoms of P34's
+// MN-major A, V is P34's MN-major B as loaded, and S_in (bf16, written row i
+// by row i) is P2's MN-major B.  After P34 the epilogue stores y, clears Y,
+// scales row i of S by exp(Lam_L[i]) in TMEM and writes the bf16 copy S_in.
 // On this hardware a tcgen05.mma costs about the same issue time for any of
 // these shapes, so the kernel minimises the instruction count: 12 per chunk.
 // |Lam| <= 80 keeps exp(-Lam) inside fp32.  A chunk whose summed |ew| exceeds
@@ -33,7 +36,8 @@
 //                as their inputs become ready
 //   warps 1..4   transform: Q, Kt, the bonus scalars c, exp(Lam_L), chunk flag
 //   warps 5..8   mask: A'^T from TMEM into shared memory
-//   warps 9..12  epilogue: y out of TMEM, state rescale, exact fallback chunks
+//   warps 9..12  epilogue: the two warps on TMEM lanes 0..63 store y, the two
+//                on lanes 64..127 rescale the state; all four run exact chunks
 // Hand-offs are mbarriers; every wait is bounded and a shared abort flag stops
 // all roles after the first timeout.
 #include "wkv_launch.cuh"
@@ -56,17 +60,18 @@ constexpr int kET = 32 * kEW;
 constexpr int kTokW = kL / kTW;              // tokens per transform warp
 constexpr int kTile = kL * kHead;            // bf16 elements of one 64 x 64 tile (8 KB)
 
-enum { R_ = 0, K_ = 1, V_ = 2, W_ = 3 };
+enum { R_ = 0, Z_ = 1, K_ = 2, V_ = 3, W_ = 4, kSlots = 5 };
 
 struct TcSmem {
-    __nv_bfloat16 Ap[2][kTile];          // A'^T (row s, p contiguous): first B atom of P34
-    __nv_bfloat16 SinT[kTile];           // bf16 S_in^T (row j, i contiguous): A of P2
-    __nv_bfloat16 raw[2][4][kTile];      // stages: r -> Q and k -> Kt in place, v, w (TMA, swizzled)
+    __nv_bfloat16 Ap[2][kTile];          // A'^T (row s, p contiguous): first A atom of P34
+    __nv_bfloat16 Sin[kTile];            // bf16 S_in (row i, j contiguous): B of P2
+    __nv_bfloat16 raw[2][kSlots][kTile]; // stages: r -> Q, zero tile, k -> Kt, v, w (TMA, swizzled)
     float dec[4][kHead];                 // exp(Lam_L) per row i (ring of 4 chunks)
     float cp[4][kL];                     // bonus scalars per token (ring of 4 chunks)
     float psum[2][kTW][kHead];           // per-warp log2-decay sums, by chunk parity
     float pabs[2][kTW][kHead];           // per-warp sums of |log2-decay|
     float u[kHead];
+    float ypart[2][2][kHead];            // exact chunks: per-warp column sums, by token parity
     int flag[4];                         // chunk c is exact-evaluated iff flag[c & 3] == c + 1
     int abort_;
     uint32_t tmem_base;
@@ -75,8 +80,8 @@ struct TcSmem {
     alignas(8) uint64_t m1_done[2];      // per TMEM A buffer: A^T ready
     alignas(8) uint64_t a_done[2];       // per TMEM A buffer: A'^T in shared memory, buffer read
     alignas(8) uint64_t stage_free[2];   // every reader of the stage finished
-    alignas(8) uint64_t mma_done;        // Y^T and S^T of the chunk complete
-    alignas(8) uint64_t s_ready;         // y read out, state rescaled, S_in^T written
+    alignas(8) uint64_t mma_done;        // Y and S of the chunk complete
+    alignas(8) uint64_t s_ready;         // y stored and Y cleared, state rescaled, S_in written
     alignas(8) uint64_t final_bar;
 };
 
@@ -176,6 +181,30 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Sum of v[m] over the 32 lanes of the warp, for m = 0..7, with lane l ending up
+// holding the sum for m = (l >> 2) & 7 (9 shuffles instead of 8 full reductions).
+__device__ __forceinline__ float transpose_reduce8(const float (&v)[8], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float a4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float keep = b4 ? v[4 + q] : v[q];
+        const float send = b4 ? v[q] : v[4 + q];
+        a4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float a2[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const float keep = b3 ? a4[2 + q] : a4[q];
+        const float send = b3 ? a4[q] : a4[2 + q];
+        a2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float a1 = (b2 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? a2[0] : a2[1], 4);
+    a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+    a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+    return a1;
+}
+
 __device__ __forceinline__ bool is_flagged(const TcSmem &sm, int c) {
     return *(const volatile int *)&sm.flag[c & 3] == c + 1;
 }
@@ -194,10 +223,15 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     const int h = blockIdx.x % H, b = blockIdx.x / H;
     const int cbase = h * kHead;
     const int nch = (T + kL - 1) / kL;
-    constexpr uint32_t kStageBytes = 4u * kTile * sizeof(__nv_bfloat16);
+    constexpr uint32_t kStageBytes = 4u * kTile * sizeof(__nv_bfloat16);   // r, k, v, w
 
     if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
     if (tid < 4) sm.flag[tid] = 0;
+    for (int i = tid; i < 2 * kTile * 2 / 16; i += kThreads) {   // the two zero tiles (never rewritten)
+        uint4 *z = reinterpret_cast<uint4 *>(sm.raw[i / (kTile * 2 / 16)][Z_]);
+        z[i % (kTile * 2 / 16)] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
     if (tid == 0) {
         sm.abort_ = 0;
         prefetch_tensormap(&map_r);
@@ -223,12 +257,10 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    // TMEM columns: A^T buffers at 0 and 64, Y^T at 128, S^T at 192 (P34 writes 128..255)
+    // TMEM columns: A^T buffers at 0 and 64 (M = 64 layout), [Y ; S] at 128 (M = 128: lane = row)
     const uint32_t tbase = sm.tmem_base;
-    const uint32_t tY = tbase + 128, tS = tbase + 192;
+    const uint32_t tD = tbase + 128;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lane quarter
-    const int qrow = 16 * (warp & 3) + (lane & 15);                 // accumulator row (M = 64 layout)
-    const bool rowlane = lane < 16;                                  // lanes 16..31 hold no row
 
     if (warp == 0) {
         // ===================== TMA + MMA issue (one thread) =====================
@@ -241,8 +273,9 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 tma_load_3d(sm.raw[s][V_], &map_v, cbase, c * kL, b, &sm.full[s]);
                 tma_load_3d(sm.raw[s][W_], &map_w, cbase, c * kL, b, &sm.full[s]);
             };
-            constexpr uint32_t kIdKK = idesc_bf16(64, 64, false, false);
-            constexpr uint32_t kIdP34 = idesc_bf16(64, 128, true, true);
+            constexpr uint32_t kIdM1 = idesc_bf16(64, 64, false, false);
+            constexpr uint32_t kIdP2 = idesc_bf16(128, 64, false, true);
+            constexpr uint32_t kIdP34 = idesc_bf16(128, 64, true, true);
             issue(0);
             if (nch > 1) issue(1);
             int next_tma = nch > 1 ? 2 : 1;   // next chunk to load
@@ -262,11 +295,10 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                     const int c = next_p, set = c & 1;
                     if (mbar_test(&sm.a_done[set], (c >> 1) & 1)) {
                         tc::fence_after_sync();
-                        const __nv_bfloat16 *V = sm.raw[set][V_];
                         const uint32_t lbo = smem_u32(sm.raw[set][K_]) - smem_u32(sm.Ap[set]);
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            mma_bf16(tY, desc_mn(V, k, 16), desc_mn(sm.Ap[set], k, lbo), kIdP34, true);
+                            mma_bf16(tD, desc_mn(sm.Ap[set], k, lbo), desc_mn(sm.raw[set][V_], k, 16), kIdP34, true);
                         tc::mma_commit(&sm.mma_done);
                         tc::mma_commit(&sm.stage_free[set]);
                         ++next_p;
@@ -277,9 +309,10 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                     const int c = next_p, set = c & 1;
                     tc::fence_after_sync();
                     if (!is_flagged(sm, c)) {
+                        // rows 64..127 of [Q ; 0] are the zero tile: S only accumulates 0
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            mma_bf16(tY, desc_k(sm.SinT, k), desc_k(sm.raw[set][R_], k), kIdKK, k > 0);
+                            mma_bf16(tD, desc_k(sm.raw[set][R_], k), desc_mn(sm.Sin, k, 16), kIdP2, true);
                         p2_issued = true;
                         progress = true;
                     } else if (mbar_test(&sm.a_done[set], (c >> 1) & 1)) {
@@ -297,7 +330,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
 #pragma unroll
                             for (int k = 0; k < 4; ++k)
                                 mma_bf16(tbase + 64 * set, desc_k(sm.raw[set][K_], k), desc_k(sm.raw[set][R_], k),
-                                         kIdKK, k > 0);
+                                         kIdM1, k > 0);
                             tc::mma_commit(&sm.m1_done[set]);
                         } else {
                             mbar_arrive(&sm.m1_done[set]);   // the mask warps skip this chunk
@@ -325,6 +358,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                         ok = false;
                         break;
                     }
+                    __nanosleep(20);   // leave the issue slots to the warps doing the work
                 }
             }
             // every MMA issued so far must finish before TMEM is released
@@ -392,57 +426,35 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 *reinterpret_cast<float2 *>(&sm.dec[c & 3][ch]) = make_float2(exp2f(tot0), exp2f(tot1));
                 if (lane == 0 && flagged) sm.flag[c & 3] = c + 1;
             }
-            // ---- Q and Kt in place of r and k; bonus partials r u k
-            float bp[kTokW];
+            // ---- Q and Kt in place of r and k; bonus scalars c_p, 8 tokens at a time
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float bp[8];
 #pragma unroll
-            for (int e = 0; e < kTokW; ++e) {
-                const uint32_t o = off(e);
-                const uint32_t rv = ld_u32(Rb, o), kv = ld_u32(Kb, o);
-                const float r0 = bf_lo(rv), r1 = bf_hi(rv), k0 = bf_lo(kv), k1 = bf_hi(kv);
-                bp[e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
-                if (!flagged) {
-                    const uint32_t wv = ld_u32(Wb, o);
-                    const float q0 = r0 * fast_exp2(L0), q1 = r1 * fast_exp2(L1);
-                    L0 += bf_lo(wv) * kLog2e;
-                    L1 += bf_hi(wv) * kLog2e;
-                    st_u32(Rb, o, pack_bf16(q0, q1));
-                    st_u32(Kb, o, pack_bf16(k0 * fast_exp2(-L0), k1 * fast_exp2(-L1)));
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t o = off(8 * half + e);
+                    const uint32_t rv = ld_u32(Rb, o), kv = ld_u32(Kb, o);
+                    const float r0 = bf_lo(rv), r1 = bf_hi(rv), k0 = bf_lo(kv), k1 = bf_hi(kv);
+                    bp[e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
+                    if (!flagged) {
+                        const uint32_t wv = ld_u32(Wb, o);
+                        const float q0 = r0 * fast_exp2(L0), q1 = r1 * fast_exp2(L1);
+                        L0 += bf_lo(wv) * kLog2e;
+                        L1 += bf_hi(wv) * kLog2e;
+                        st_u32(Rb, o, pack_bf16(q0, q1));
+                        st_u32(Kb, o, pack_bf16(k0 * fast_exp2(-L0), k1 * fast_exp2(-L1)));
+                    }
                 }
-            }
-            // transpose-reduce the 16 partials over the 32 lanes: lanes 2m, 2m+1 end with token m
-            {
-                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-                float a8[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float keep = b4 ? bp[8 + q] : bp[q];
-                    const float send = b4 ? bp[q] : bp[8 + q];
-                    a8[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-                }
-                float a4[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float keep = b3 ? a8[4 + q] : a8[q];
-                    const float send = b3 ? a8[q] : a8[4 + q];
-                    a4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-                }
-                float a2[2];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const float keep = b2 ? a4[2 + q] : a4[q];
-                    const float send = b2 ? a4[q] : a4[2 + q];
-                    a2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-                }
-                float a1s = (b1 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? a2[0] : a2[1], 2);
-                a1s += __shfl_xor_sync(0xffffffffu, a1s, 1);
-                if ((lane & 1) == 0) sm.cp[c & 3][p0 + (lane >> 1)] = a1s;
+                const float cpv = transpose_reduce8(bp, lane);
+                if ((lane & 3) == 0) sm.cp[c & 3][p0 + 8 * half + (lane >> 2)] = cpv;
             }
             fence_proxy_async_smem();
             mbar_arrive(&sm.t_done[stg]);
         }
     } else if (warp <= kTW + kAW) {
         // ===================== mask warps: A'^T = strict-upper(A^T) + diag(c) =====================
-        const int s = qrow;
+        const int s = 16 * (warp & 3) + (lane & 15);   // A^T row (M = 64 layout: lanes 0..15 of the quarter)
+        const bool rowlane = lane < 16;
         for (int c = 0; c < nch; ++c) {
             const int set = c & 1;
             if (!wait_or_abort(sm, &sm.m1_done[set], (c >> 1) & 1)) break;
@@ -479,15 +491,17 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     } else {
         // ===================== epilogue warps =====================
         const int et = tid - 32 * (1 + kTW + kAW);   // 0 .. kET-1
-        const int j = qrow;                           // S^T / Y^T row served by this lane
-        // the state starts at zero: S^T in TMEM and its bf16 copy
+        const int q = warp & 3;                       // TMEM lane quarter
+        const bool yrole = q < 2;                     // lanes 0..63: Y rows; lanes 64..127: S rows
+        const int row = 32 * (q & 1) + lane;          // p (Y) or i (S)
+        // everything starts at zero: Y, S and the bf16 copy S_in
         {
             float z[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) z[e] = 0.f;
-            tc::tmem_st32(tS + lane_off, z);
-            tc::tmem_st32(tS + lane_off + 32, z);
-            uint4 *st = reinterpret_cast<uint4 *>(sm.SinT);
+            tc::tmem_st32(tD + lane_off, z);
+            tc::tmem_st32(tD + lane_off + 32, z);
+            uint4 *st = reinterpret_cast<uint4 *>(sm.Sin);
             for (int i = et; i < kTile * 2 / 16; i += kET) st[i] = make_uint4(0u, 0u, 0u, 0u);
             tc::tmem_wait_st();
             fence_proxy_async_smem();
@@ -496,47 +510,43 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
         }
         for (int c = 0; c < nch; ++c) {
             const int t0 = c * kL, stg = c & 1;
-            const int pmax = min(kL, T - t0);
             wait_or_abort(sm, &sm.mma_done, c & 1);
             named_sync(2, kET);
             if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
             tc::fence_after_sync();
-            float *ycol = prm.y + ((size_t)b * T + t0) * C + cbase + j;
             if (!is_flagged(sm, c)) {
-                // ---- y: row j of Y^T is channel j of the chunk's 64 outputs
+                if (yrole) {
+                    // ---- y row p (64 channels, 256 contiguous bytes), then clear Y for the next chunk
+                    const bool live = t0 + row < T;
+                    float4 *dst = reinterpret_cast<float4 *>(prm.y + ((size_t)b * T + t0 + row) * C + cbase);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v[32];
-                    tc::tmem_ld32(tY + lane_off + 32 * half, v);
-                    tc::tmem_wait_ld();
-                    if (rowlane) {
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32];
+                        tc::tmem_ld32(tD + lane_off + 32 * half, v);
+                        tc::tmem_wait_ld();
+                        if (live) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int p = 32 * half + e;
-                            if (p < pmax) ycol[(size_t)p * C] = v[e];
+                            for (int g = 0; g < 8; ++g)
+                                dst[8 * half + g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
                         }
-                    }
-                }
-                // ---- S^T columns scaled by exp(Lam_L), back to TMEM, bf16 copy into S_in^T
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v[32];
-                    tc::tmem_ld32(tS + lane_off + 32 * half, v);
-                    tc::tmem_wait_ld();
-                    const float4 *dq = reinterpret_cast<const float4 *>(&sm.dec[c & 3][32 * half]);
-#pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        const float4 d = dq[g];
-                        v[4 * g] *= d.x;
-                        v[4 * g + 1] *= d.y;
-                        v[4 * g + 2] *= d.z;
-                        v[4 * g + 3] *= d.w;
+                        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                        tc::tmem_st32(tD + lane_off + 32 * half, v);
                     }
-                    tc::tmem_st32(tS + lane_off + 32 * half, v);
-                    if (rowlane) {
+                } else {
+                    // ---- S row i scaled by exp(Lam_L[i]), back to TMEM, bf16 copy into S_in
+                    const float dsc = sm.dec[c & 3][row];
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32];
+                        tc::tmem_ld32(tD + lane_off + 32 * half, v);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] *= dsc;
+                        tc::tmem_st32(tD + lane_off + 32 * half, v);
 #pragma unroll
                         for (int g = 0; g < 4; ++g)
-                            st_u128(sm.SinT, swz(j, 32 * half + 8 * g),
+                            st_u128(sm.Sin, swz(row, 32 * half + 8 * g),
                                     make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]), pack_bf16(v[8 * g + 2], v[8 * g + 3]),
                                                pack_bf16(v[8 * g + 4], v[8 * g + 5]),
                                                pack_bf16(v[8 * g + 6], v[8 * g + 7])));
@@ -544,38 +554,56 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 }
                 tc::tmem_wait_st();
             } else {
-                // ---- exact token-by-token evaluation of this chunk on the CUDA cores:
-                // lane j owns column j of S (row j of S^T in TMEM)
+                // ---- exact token-by-token evaluation of this chunk on the CUDA cores.
+                // The S warps own rows i of S and form per-warp column sums of
+                // r_p[i] S[i][j]; the Y warps add the two halves and the bonus and store y.
                 const __nv_bfloat16 *R = sm.raw[stg][R_], *Kr = sm.raw[stg][K_];
                 const __nv_bfloat16 *V = sm.raw[stg][V_], *W = sm.raw[stg][W_];
                 for (int p = 0; p < kL; ++p) {
-                    const float vj = raw_at(V, p, j);
-                    float acc = 0.f;
+                    if (!yrole) {
+                        const float rr = raw_at(R, p, row), dd = __expf(raw_at(W, p, row)), kk = raw_at(Kr, p, row);
 #pragma unroll 1
-                    for (int m = 0; m < 4; ++m) {
-                        float sv[16];
-                        tc::tmem_ld16(tS + lane_off + 16 * m, sv);
+                        for (int m = 0; m < 4; ++m) {
+                            float s16[16];
+                            tc::tmem_ld16(tD + lane_off + 16 * m, s16);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                float pr[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) pr[e] = rr * s16[8 * hh + e];
+                                const float colsum = transpose_reduce8(pr, lane);   // column 16 m + 8 hh + (lane >> 2)
+                                if ((lane & 3) == 0) sm.ypart[p & 1][q - 2][16 * m + 8 * hh + (lane >> 2)] = colsum;
+                            }
+                        }
+                        // update after every column sum of this token has read the old S
+#pragma unroll 1
+                        for (int m = 0; m < 4; ++m) {
+                            float s16[16];
+                            tc::tmem_ld16(tD + lane_off + 16 * m, s16);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) s16[e] = fmaf(dd, s16[e], kk * raw_at(V, p, 16 * m + e));
+                            tc::tmem_st16(tD + lane_off + 16 * m, s16);
+                            tc::tmem_wait_st();
+                        }
+                    }
+                    named_sync(2, kET);
+                    if (yrole && t0 + p < T) {
+                        const int jj = row;   // 0..63
+                        prm.y[((size_t)b * T + t0 + p) * C + cbase + jj] =
+                            sm.ypart[p & 1][0][jj] + sm.ypart[p & 1][1][jj] + sm.cp[c & 3][p] * raw_at(V, p, jj);
+                    }
+                }
+                if (!yrole) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32];
+                        tc::tmem_ld32(tD + lane_off + 32 * half, v);
                         tc::tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int i = 16 * m + e;
-                            acc = fmaf(raw_at(R, p, i), sv[e], acc);
-                            sv[e] = fmaf(__expf(raw_at(W, p, i)), sv[e], raw_at(Kr, p, i) * vj);
-                        }
-                        tc::tmem_st16(tS + lane_off + 16 * m, sv);
-                        tc::tmem_wait_st();
-                    }
-                    if (rowlane && p < pmax) ycol[(size_t)p * C] = fmaf(sm.cp[c & 3][p], vj, acc);
-                }
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v[32];
-                    tc::tmem_ld32(tS + lane_off + 32 * half, v);
-                    tc::tmem_wait_ld();
-                    if (rowlane) {
-#pragma unroll
                         for (int g = 0; g < 4; ++g)
-                            st_u128(sm.SinT, swz(j, 32 * half + 8 * g),
+                            st_u128(sm.Sin, swz(row, 32 * half + 8 * g),
                                     make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]), pack_bf16(v[8 * g + 2], v[8 * g + 3]),
                                                pack_bf16(v[8 * g + 4], v[8 * g + 5]),
                                                pack_bf16(v[8 * g + 6], v[8 * g + 7])));
