@@ -161,19 +161,34 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
+// try_wait with a suspend-time hint: the thread is parked by the hardware until
+// the phase completes or about `ns` nanoseconds pass, without issuing anything.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return done != 0;
+}
+
 // Bounded wait that gives up at once when another thread has already aborted.
+// Waiting threads stay parked in the barrier (20 us at a time) instead of
+// spinning, so they take no issue slots from the warps doing the work.
 __device__ __forceinline__ bool wait_or_abort(TcSmem &sm, uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_for(bar, parity, 20000u)) return true;
         if (*(volatile int *)&sm.abort_) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             atomicOr(&g_wkv_faults, WKV_FAULT_TIMEOUT);
             *(volatile int *)&sm.abort_ = 1;
             return false;
         }
-        __nanosleep(32);
     }
 }
 
@@ -272,6 +287,14 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 tma_load_3d(sm.raw[s][K_], &map_k, cbase, c * kL, b, &sm.full[s]);
                 tma_load_3d(sm.raw[s][V_], &map_v, cbase, c * kL, b, &sm.full[s]);
                 tma_load_3d(sm.raw[s][W_], &map_w, cbase, c * kL, b, &sm.full[s]);
+                // the load of chunk c + 2 waits for this stage's chunk to retire; start
+                // its HBM reads now so that it is served from L2
+                if (c + 2 < nch) {
+                    tma_prefetch_l2_3d(&map_r, cbase, (c + 2) * kL, b);
+                    tma_prefetch_l2_3d(&map_k, cbase, (c + 2) * kL, b);
+                    tma_prefetch_l2_3d(&map_v, cbase, (c + 2) * kL, b);
+                    tma_prefetch_l2_3d(&map_w, cbase, (c + 2) * kL, b);
+                }
             };
             constexpr uint32_t kIdM1 = idesc_bf16(64, 64, false, false);
             constexpr uint32_t kIdP2 = idesc_bf16(128, 64, false, true);
@@ -283,7 +306,8 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
             int next_p = 0;                   // next chunk for P2 / P34
             bool p2_issued = false;           // P2 of chunk next_p issued, P34 pending
             bool ok = true;
-            unsigned long long last = globaltimer_ns();
+            uint32_t idle = 0;                // idle polls since the last issue
+            unsigned long long idle_since = 0;
             // Each step issues whatever has its inputs ready, the state chain
             // (P34, then P2) first.  Invariants that keep every parity wait
             // unambiguous: M1 runs at most one chunk ahead of P34, a stage is
@@ -346,19 +370,24 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                     progress = true;
                 }
                 if (progress) {
-                    last = globaltimer_ns();
+                    idle = 0;
                 } else {
-                    if (*(volatile int *)&sm.abort_) {
-                        ok = false;
-                        break;
+                    // the clock and the abort flag are read every 64 idle polls only
+                    if ((++idle & 63) == 0) {
+                        if (*(volatile int *)&sm.abort_) {
+                            ok = false;
+                            break;
+                        }
+                        const unsigned long long now = globaltimer_ns();
+                        if (idle == 64) {
+                            idle_since = now;
+                        } else if (now - idle_since > kWaitLimitNs) {
+                            atomicOr(&g_wkv_faults, WKV_FAULT_TIMEOUT);
+                            *(volatile int *)&sm.abort_ = 1;
+                            ok = false;
+                            break;
+                        }
                     }
-                    if (globaltimer_ns() - last > kWaitLimitNs) {
-                        atomicOr(&g_wkv_faults, WKV_FAULT_TIMEOUT);
-                        *(volatile int *)&sm.abort_ = 1;
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(20);   // leave the issue slots to the warps doing the work
                 }
             }
             // every MMA issued so far must finish before TMEM is released
@@ -430,19 +459,36 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 float bp[8];
+                // flagged is warp-uniform: keeping the branch outside the token loop
+                // leaves one straight-line body whose loads and exponentials overlap
+                if (!flagged) {
+                    // all loads first: the in-place stores below may alias them as far as
+                    // the compiler can tell, so loads issued after a store would serialise
+                    uint32_t rv[8], kv[8], wv[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t o = off(8 * half + e);
-                    const uint32_t rv = ld_u32(Rb, o), kv = ld_u32(Kb, o);
-                    const float r0 = bf_lo(rv), r1 = bf_hi(rv), k0 = bf_lo(kv), k1 = bf_hi(kv);
-                    bp[e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
-                    if (!flagged) {
-                        const uint32_t wv = ld_u32(Wb, o);
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t o = off(8 * half + e);
+                        rv[e] = ld_u32(Rb, o);
+                        kv[e] = ld_u32(Kb, o);
+                        wv[e] = ld_u32(Wb, o);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t o = off(8 * half + e);
+                        const float r0 = bf_lo(rv[e]), r1 = bf_hi(rv[e]), k0 = bf_lo(kv[e]), k1 = bf_hi(kv[e]);
+                        bp[e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
                         const float q0 = r0 * fast_exp2(L0), q1 = r1 * fast_exp2(L1);
-                        L0 += bf_lo(wv) * kLog2e;
-                        L1 += bf_hi(wv) * kLog2e;
+                        L0 += bf_lo(wv[e]) * kLog2e;
+                        L1 += bf_hi(wv[e]) * kLog2e;
                         st_u32(Rb, o, pack_bf16(q0, q1));
                         st_u32(Kb, o, pack_bf16(k0 * fast_exp2(-L0), k1 * fast_exp2(-L1)));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t o = off(8 * half + e);
+                        const uint32_t rv = ld_u32(Rb, o), kv = ld_u32(Kb, o);
+                        bp[e] = fmaf(bf_lo(rv) * u0, bf_lo(kv), bf_hi(rv) * u1 * bf_hi(kv));
                     }
                 }
                 const float cpv = transpose_reduce8(bp, lane);

@@ -100,6 +100,14 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Prefetch one tile of a 3-D tensor map into L2 (no shared-memory destination,
+// no completion to wait for; out-of-range parts are ignored).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c, int t, int b) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c), "r"(t), "r"(b)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
