@@ -18,11 +18,14 @@
 //   dw_m = sum_{tau > m} z_tau - sum_{s >= m} x_s,
 // because each side sums r_t[i] k_s[i] P(s,t)[i] (v_s . dy_t) over the pairs
 // with m strictly between s and t (the totals of the anti-causal terms cancel).
-// The forward sweep parks z in dw; the backward sweep turns it into dw in place.
+// The forward sweep parks z in dw (and its dr, dk, dv parts in place); the backward
+// sweep loads them back by TMA one chunk ahead, adds its own parts and turns z into dw.
 //
 // Layout and scaled state as in wkv6_fwd.cu: one CTA per (b, h), 4 warps
 // splitting the 64 value columns, 32 registers per state per lane, TMA-staged
 // chunks of TC tokens, renorm steps bounding |L| by kTheta.
+#include <cstddef>
+
 #include "wkv_launch.cuh"
 
 namespace wkv {
@@ -31,7 +34,7 @@ constexpr float kThetaB = 40.0f;
 
 template <int TC>
 struct BwdSmem {
-    float raw[2][5][TC][kHead];   // r, k, w, v, dy (TMA landing, 2 stages)
+    alignas(128) float raw[2][5][TC][kHead];   // r, k, w, v, dy (TMA landing, 2 stages)
     float Ap[TC][kHead];          // exp(L_p)
     float ks[TC][kHead];          // k * exp(-L_{p+1})   (k on renorm steps)
     float rs[TC][kHead];          // r * exp(-L_{p+1})   (r on renorm steps)
@@ -45,9 +48,16 @@ struct BwdSmem {
     float vdy[TC];
     float ruk[TC];
     float u[kHead];
+    alignas(128) float part[2][4][TC][kHead];  // second sweep: the first sweep's dr, dk, dv, z (TMA, 2 stages)
     uint32_t renorm_mask;
     alignas(8) uint64_t full[2];
+    alignas(8) uint64_t pfull[2];
 };
+
+// TMA writes its tiles at 128-byte aligned shared-memory addresses only.
+static_assert(offsetof(BwdSmem<kBwdTC>, raw) % 128 == 0 && offsetof(BwdSmem<kBwdTC>, part) % 128 == 0 &&
+                  (kBwdTC * kHead * sizeof(float)) % 128 == 0,
+              "backward TMA destinations must be 128-byte aligned");
 
 enum { A_R = 0, A_K = 1, A_W = 2, A_V = 3, A_DY = 4 };
 
@@ -95,10 +105,13 @@ template <int TC, bool BIDIR>
 __global__ void __launch_bounds__(128, 3)
 wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_v,
-                const __grid_constant__ CUtensorMap map_dy, BwdParams prm) {
+                const __grid_constant__ CUtensorMap map_dy, const __grid_constant__ CUtensorMap map_dr,
+                const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
+                const __grid_constant__ CUtensorMap map_dw, BwdParams prm) {
     using Smem = BwdSmem<TC>;
     constexpr int NT = 128;
     constexpr uint32_t kStageBytes = 5u * TC * kHead * sizeof(float);
+    constexpr uint32_t kPartBytes = 4u * TC * kHead * sizeof(float);
     extern __shared__ unsigned char smem_dyn[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~uintptr_t(127));
 
@@ -119,6 +132,8 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         prefetch_tensormap(&map_dy);
         mbar_init(&sm.full[0], 1);
         mbar_init(&sm.full[1], 1);
+        mbar_init(&sm.pfull[0], 1);
+        mbar_init(&sm.pfull[1], 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -132,6 +147,17 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         tma_load_3d(&sm.raw[s][A_W][0][0], &map_w, cbase, tl, b, &sm.full[s]);
         tma_load_3d(&sm.raw[s][A_V][0][0], &map_v, cbase, tl, b, &sm.full[s]);
         tma_load_3d(&sm.raw[s][A_DY][0][0], &map_dy, cbase, tl, b, &sm.full[s]);
+    };
+    // second sweep, chunk g: what the first sweep stored for the same tokens.  It
+    // is loaded one chunk ahead, after the first sweep's stores of those tokens
+    // (the last first-sweep chunk stores the tokens of the first second-sweep chunk).
+    auto issue_part = [&](int g) {
+        const int s = g & 1, tl = t_lo_of(g);
+        mbar_arrive_expect_tx(&sm.pfull[s], kPartBytes);
+        tma_load_3d(&sm.part[s][0][0][0], &map_dr, cbase, tl, b, &sm.pfull[s]);
+        tma_load_3d(&sm.part[s][1][0][0], &map_dk, cbase, tl, b, &sm.pfull[s]);
+        tma_load_3d(&sm.part[s][2][0][0], &map_dv, cbase, tl, b, &sm.pfull[s]);
+        tma_load_3d(&sm.part[s][3][0][0], &map_dw, cbase, tl, b, &sm.pfull[s]);
     };
     if (tid == 0) {
         issue(0);
@@ -166,9 +192,11 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
 #pragma unroll
                 for (int j = 0; j < 4; ++j) Ss[q][j] = Gs[q][j] = 0.f;
         }
-        const bool ok = mbar_wait_bounded(&sm.full[s], (g >> 1) & 1);
+        bool ok = mbar_wait_bounded(&sm.full[s], (g >> 1) & 1);
+        if (!sweepA) ok = mbar_wait_bounded(&sm.pfull[s], ((g - nch) >> 1) & 1) && ok;
         if (!__syncthreads_and(ok)) {         // a bounded wait ran out: stop (fault recorded)
             drain_two_stage(sm.full, g, nchunks);
+            if (!sweepA) mbar_wait_bounded(&sm.pfull[s], ((g - nch) >> 1) & 1);
             return;
         }
 
@@ -348,12 +376,14 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                 prm.dv[o] = fmaf(sm.ruk[p], sm.dys[p][i], dvv);
                 prm.dw[o] = fmaf(rr, drs, kk * dks);           // z_t, parked in dw
             } else {
-                prm.dr[o] += drs;
-                prm.dk[o] += dks;
-                prm.dv[o] += dvv;
+                prm.dr[o] = sm.part[s][0][row][i] + drs;
+                prm.dk[o] = sm.part[s][1][row][i] + dks;
+                prm.dv[o] = sm.part[s][2][row][i] + dvv;
                 sm.pr[p][0][i] = fmaf(kk, dks, rr * drs);      // x_t, for the dw scan below
             }
         }
+        // the second sweep reads these stores back through the TMA (async proxy)
+        if (sweepA) asm volatile("fence.proxy.async.global;" ::: "memory");
         if (sweepA) {
             // du partial: thread i accumulates sum_t r k (v.dy) for row i
             if (tid < kHead) {
@@ -372,7 +402,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                     if (t < 0 || t >= T) continue;
                     const size_t o = ((size_t)b * T + t) * C + cbase + tid;
                     const float x = sm.pr[p][0][tid];
-                    const float z = prm.dw[o];
+                    const float z = sm.part[s][3][TC - 1 - p][tid];
                     prm.dw[o] = Rrun - x;
                     Rrun += z - x;
                 }
@@ -384,6 +414,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             fence_proxy_async_smem();
             issue(g + 2);
         }
+        if (tid == 0 && g + 1 >= nch && g + 1 < nchunks) issue_part(g + 1);
     }
     if (tid < kHead) prm.du_part[(size_t)b * C + cbase + tid] = du_acc;
 }
@@ -403,7 +434,8 @@ static cudaError_t launch_bwd(const CUtensorMap *maps, const BwdParams &prm, cud
     const size_t smem = sizeof(BwdSmem<TC>) + 128;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(prm.B * prm.H), 128, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], prm);
+    kern<<<(unsigned)(prm.B * prm.H), 128, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
+                                                            maps[6], maps[7], maps[8], prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return cudaSuccess;

@@ -88,6 +88,17 @@ int check_wkv6(int B, int T, int C, int H, std::initializer_list<const void *> p
 // Algorithm of the bf16 causal forward: the chunked tensor-core kernel (default)
 // or the token-by-token recurrence (WKV6_BF16_PATH=recurrence).  Both compute
 // the same operation; the variable is read on every call.
+// Tensor maps of the backward: inputs r, k, w, v, dy, then the outputs dr, dk,
+// dv, dw (the second sweep reads back what the first sweep stored there).
+bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], int B, int T, int C, const float *r, const float *k,
+                   const float *w, const float *v, const float *dy, const float *dr, const float *dk,
+                   const float *dv, const float *dw) {
+    const void *src[kBwdMaps] = {r, k, w, v, dy, dr, dk, dv, dw};
+    for (int i = 0; i < kBwdMaps; ++i)
+        if (!make_map(&maps[i], src[i], false, B, T, C, kHead, kBwdTC)) return false;
+    return true;
+}
+
 bool bf16_use_tensor_cores() {
     const char *e = std::getenv("WKV6_BF16_PATH");
     return !(e && std::strcmp(e, "recurrence") == 0);
@@ -166,10 +177,8 @@ int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, cons
     if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
     if ((st = check_device()) != WKV_OK) return st;
-    CUtensorMap maps[5];
-    const void *src[5] = {r, k, w, v, dy};
-    for (int i = 0; i < 5; ++i)
-        if (!make_map(&maps[i], src[i], false, B, T, C, kHead, kBwdTC)) return WKV_ERR_CUDA;
+    CUtensorMap maps[kBwdMaps];
+    if (!make_bwd_maps(maps, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, static_cast<float *>(workspace)};
     return wkv6_bwd_launch(bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
@@ -262,10 +271,8 @@ extern "C" int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, c
         return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
     float *scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != WKV_OK) return st;
-    CUtensorMap maps[5];
-    const void *src[5] = {r, k, w, v, dy};
-    for (int i = 0; i < 5; ++i)
-        if (!make_map(&maps[i], src[i], false, B, T, C, kHead, kBwdTC)) return WKV_ERR_CUDA;
+    CUtensorMap maps[kBwdMaps];
+    if (!make_bwd_maps(maps, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
     // Every per-batch partial the reduction reads is written first by the
     // backward kernel, so nothing left in the array by an earlier call leaks in.
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, scratch};

@@ -26,6 +26,8 @@ cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const 
                             cudaStream_t stream);
 cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
                                const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream);
+// maps: kBwdMaps tensor maps, in the order r, k, w, v, dy, dr, dk, dv, dw
+constexpr int kBwdMaps = 9;
 cudaError_t wkv6_bwd_launch(bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
                             cudaStream_t stream);
 cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,
