@@ -40,8 +40,6 @@ struct BwdSmem {
     float rs[TC][kHead];          // r * exp(-L_{p+1})   (r on renorm steps)
     float kh[TC][kHead];          // k * exp(L_p)
     float al[TC][kHead];          // exp(L_p + ew_p) on renorm steps
-    float vs[TC][kHead];
-    float dys[TC][kHead];
     float pr[TC][4][kHead];       // per-warp partial sums over columns of S-type . dy
     float pk[TC][4][kHead];       // per-warp partial sums over columns of G-type . v
     float dvs[TC][kHead];         // dv' (complete over rows)
@@ -99,6 +97,18 @@ __device__ __forceinline__ float reduce_cols_over_rows(const float (&yp)[4], boo
     kk += __shfl_xor_sync(0xffffffffu, s2, 2);
     kk += __shfl_xor_sync(0xffffffffu, kk, 1);
     return kk;
+}
+
+constexpr float2 kZero2 = {0.f, 0.f};
+
+// Row-pair operands (x[r], x[r+1]) for the rows r = rowA, rowA+2, rowB, rowB+2.
+__device__ __forceinline__ void load_pairs(const float *x, int rowA, int rowB, float2 (&o)[4]) {
+    const float4 a = *reinterpret_cast<const float4 *>(x + rowA);
+    const float4 b = *reinterpret_cast<const float4 *>(x + rowB);
+    o[0] = make_float2(a.x, a.y);
+    o[1] = make_float2(a.z, a.w);
+    o[2] = make_float2(b.x, b.y);
+    o[3] = make_float2(b.z, b.w);
 }
 
 template <int TC, bool BIDIR>
@@ -173,7 +183,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     const int q0 = 4 * (cg >> 1) + 2 * (cg & 1);   // rows kept by reduce_rows_over_cols: R(q0), R(q0+1)
     auto rowq = [&](int q) { return q < 4 ? rowA + q : rowB + q - 4; };
 
-    float Ss[8][4], Gs[8][4];   // S-type and G-type states of the current sweep
+    float2 S2[4][4], G2[4][4];  // S-type and G-type states of the current sweep (row pairs)
     float du_acc = 0.f;         // thread i < 64: sum_t r k (v.dy) for row i
     float Rrun = 0.f;           // thread i < 64: running sum for dw (backward sweep)
 
@@ -188,9 +198,9 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         const bool hasG = !sweepA || BIDIR;
         if (g == 0 || g == nch) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
+            for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) Ss[q][j] = Gs[q][j] = 0.f;
+                for (int j = 0; j < 4; ++j) S2[qq][j] = G2[qq][j] = kZero2;
         }
         bool ok = mbar_wait_bounded(&sm.full[s], (g >> 1) & 1);
         if (!sweepA) ok = mbar_wait_bounded(&sm.pfull[s], ((g - nch) >> 1) & 1) && ok;
@@ -219,35 +229,43 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         __syncthreads();
         const uint32_t rmask = sm.renorm_mask;
 
-        // ---- transform (processing order p) ----
-        for (int i = tid; i < kHead; i += NT) {
+        // ---- transform (processing order p): two threads per row i, each half of the
+        // chunk; the second one first sums the decays of the first half (with resets)
+        {
+            static_assert(NT == 2 * kHead && TC % 2 == 0, "transform split assumes 2 threads per row");
+            constexpr int TH = TC / 2;
+            const int i = tid & (kHead - 1), p0 = (tid >> 6) * TH;
             float L = 0.f;
-            for (int p = 0; p < TC; ++p) {
+            for (int p = 0; p < p0; ++p) {
                 const int row = dir > 0 ? p : TC - 1 - p;
-                const float ew = sm.raw[s][A_W][row][i];
-                const float rr = sm.raw[s][A_R][row][i];
-                const float kk = sm.raw[s][A_K][row][i];
+                L = ((rmask >> p) & 1u) ? 0.f : L + sm.raw[s][A_W][row][i];
+            }
+            float ew[TH], rr[TH], kk[TH];
+#pragma unroll
+            for (int e = 0; e < TH; ++e) {
+                const int p = p0 + e, row = dir > 0 ? p : TC - 1 - p;
+                ew[e] = sm.raw[s][A_W][row][i];
+                rr[e] = sm.raw[s][A_R][row][i];
+                kk[e] = sm.raw[s][A_K][row][i];
+            }
+#pragma unroll
+            for (int e = 0; e < TH; ++e) {
+                const int p = p0 + e;
                 const float eL = __expf(L);
                 sm.Ap[p][i] = eL;
-                sm.kh[p][i] = kk * eL;
+                sm.kh[p][i] = kk[e] * eL;
                 if ((rmask >> p) & 1u) {
-                    sm.al[p][i] = __expf(L + ew);
-                    sm.ks[p][i] = kk;
-                    sm.rs[p][i] = rr;
+                    sm.al[p][i] = __expf(L + ew[e]);
+                    sm.ks[p][i] = kk[e];
+                    sm.rs[p][i] = rr[e];
                     L = 0.f;
                 } else {
-                    L += ew;
+                    L += ew[e];
                     const float emL = __expf(-L);
-                    sm.ks[p][i] = kk * emL;
-                    sm.rs[p][i] = rr * emL;
+                    sm.ks[p][i] = kk[e] * emL;
+                    sm.rs[p][i] = rr[e] * emL;
                 }
             }
-        }
-        for (int e = tid; e < TC * kHead; e += NT) {
-            const int p = e / kHead, j = e % kHead;
-            const int row = dir > 0 ? p : TC - 1 - p;
-            sm.vs[p][j] = sm.raw[s][A_V][row][j];
-            sm.dys[p][j] = sm.raw[s][A_DY][row][j];
         }
         for (int p = warp; p < TC; p += 4) {
             const int row = dir > 0 ? p : TC - 1 - p;
@@ -268,42 +286,45 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         __syncthreads();
 
         // ---- recurrences over the chunk ----
+        // Packed fp32: each state is held as row pairs, S2[qq][j] = (S[row 2qq][j],
+        // S[row 2qq+1][j]) for the pairs (rowA, rowA+1), (rowA+2, rowA+3),
+        // (rowB, rowB+1), (rowB+2, rowB+3), so one __ffma2_rn does two
+        // multiply-adds; the per-row operands come as pairs from the float4 loads.
         for (int p = 0; p < TC; ++p) {
-            const float4 va = *reinterpret_cast<const float4 *>(&sm.vs[p][jc]);
-            const float4 ga = *reinterpret_cast<const float4 *>(&sm.dys[p][jc]);
-            const float vc[4] = {va.x, va.y, va.z, va.w};
-            const float gc[4] = {ga.x, ga.y, ga.z, ga.w};
+            const int prow = dir > 0 ? p : TC - 1 - p;
+            const float4 va = *reinterpret_cast<const float4 *>(&sm.raw[s][A_V][prow][jc]);
+            const float4 ga = *reinterpret_cast<const float4 *>(&sm.raw[s][A_DY][prow][jc]);
+            const float2 v2[4] = {make_float2(va.x, va.x), make_float2(va.y, va.y), make_float2(va.z, va.z),
+                                  make_float2(va.w, va.w)};
+            const float2 g2[4] = {make_float2(ga.x, ga.x), make_float2(ga.y, ga.y), make_float2(ga.z, ga.z),
+                                  make_float2(ga.w, ga.w)};
             const bool ren = (rmask >> p) & 1u;
-            float al[8];
-            if (ren) {
-                const float4 x = *reinterpret_cast<const float4 *>(&sm.al[p][rowA]);
-                const float4 y = *reinterpret_cast<const float4 *>(&sm.al[p][rowB]);
-                al[0] = x.x; al[1] = x.y; al[2] = x.z; al[3] = x.w;
-                al[4] = y.x; al[5] = y.y; al[6] = y.z; al[7] = y.w;
-            }
+            float2 al2[4];
+            if (ren) load_pairs(sm.al[p], rowA, rowB, al2);
             if (hasS) {
                 // readout: S . dy over my columns, then update S += ks v^T
                 float part[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    float a0 = Ss[q][0] * gc[0], a1 = Ss[q][1] * gc[1];
-                    a0 = fmaf(Ss[q][2], gc[2], a0);
-                    a1 = fmaf(Ss[q][3], gc[3], a1);
-                    part[q] = a0 + a1;
+                for (int qq = 0; qq < 4; ++qq) {
+                    float2 acc = __ffma2_rn(S2[qq][0], g2[0], kZero2);
+#pragma unroll
+                    for (int j = 1; j < 4; ++j) acc = __ffma2_rn(S2[qq][j], g2[j], acc);
+                    part[2 * qq] = acc.x;
+                    part[2 * qq + 1] = acc.y;
                 }
-                const float4 x = *reinterpret_cast<const float4 *>(&sm.ks[p][rowA]);
-                const float4 y = *reinterpret_cast<const float4 *>(&sm.ks[p][rowB]);
-                const float kr[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+                float2 kr2[4];
+                load_pairs(sm.ks[p], rowA, rowB, kr2);
                 if (ren) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
+                    for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) Ss[q][j] = fmaf(Ss[q][j], al[q], kr[q] * vc[j]);
+                        for (int j = 0; j < 4; ++j)
+                            S2[qq][j] = __ffma2_rn(S2[qq][j], al2[qq], __ffma2_rn(kr2[qq], v2[j], kZero2));
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
+                    for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) Ss[q][j] = fmaf(kr[q], vc[j], Ss[q][j]);
+                        for (int j = 0; j < 4; ++j) S2[qq][j] = __ffma2_rn(kr2[qq], v2[j], S2[qq][j]);
                 }
                 float o0, o1;
                 reduce_rows_over_cols(part, c1, c0, o0, o1);
@@ -313,39 +334,36 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             if (hasG) {
                 // readouts: G . v over my columns, kh . G over my rows; update G += rs dy^T
                 float part[8], dvp[4];
-                const float4 x = *reinterpret_cast<const float4 *>(&sm.kh[p][rowA]);
-                const float4 y = *reinterpret_cast<const float4 *>(&sm.kh[p][rowB]);
-                const float khr[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+                float2 kh2[4];
+                load_pairs(sm.kh[p], rowA, rowB, kh2);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    float a0 = Gs[q][0] * vc[0], a1 = Gs[q][1] * vc[1];
-                    a0 = fmaf(Gs[q][2], vc[2], a0);
-                    a1 = fmaf(Gs[q][3], vc[3], a1);
-                    part[q] = a0 + a1;
+                for (int qq = 0; qq < 4; ++qq) {
+                    float2 acc = __ffma2_rn(G2[qq][0], v2[0], kZero2);
+#pragma unroll
+                    for (int j = 1; j < 4; ++j) acc = __ffma2_rn(G2[qq][j], v2[j], acc);
+                    part[2 * qq] = acc.x;
+                    part[2 * qq + 1] = acc.y;
                 }
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    float a0 = khr[0] * Gs[0][j], a1 = khr[1] * Gs[1][j];
+                    float2 acc = __ffma2_rn(kh2[0], G2[0][j], kZero2);
 #pragma unroll
-                    for (int q = 2; q < 8; q += 2) {
-                        a0 = fmaf(khr[q], Gs[q][j], a0);
-                        a1 = fmaf(khr[q + 1], Gs[q + 1][j], a1);
-                    }
-                    dvp[j] = a0 + a1;
+                    for (int qq = 1; qq < 4; ++qq) acc = __ffma2_rn(kh2[qq], G2[qq][j], acc);
+                    dvp[j] = acc.x + acc.y;
                 }
-                const float4 xr = *reinterpret_cast<const float4 *>(&sm.rs[p][rowA]);
-                const float4 yr = *reinterpret_cast<const float4 *>(&sm.rs[p][rowB]);
-                const float rr[8] = {xr.x, xr.y, xr.z, xr.w, yr.x, yr.y, yr.z, yr.w};
+                float2 rr2[4];
+                load_pairs(sm.rs[p], rowA, rowB, rr2);
                 if (ren) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
+                    for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) Gs[q][j] = fmaf(Gs[q][j], al[q], rr[q] * gc[j]);
+                        for (int j = 0; j < 4; ++j)
+                            G2[qq][j] = __ffma2_rn(G2[qq][j], al2[qq], __ffma2_rn(rr2[qq], g2[j], kZero2));
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
+                    for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) Gs[q][j] = fmaf(rr[q], gc[j], Gs[q][j]);
+                        for (int j = 0; j < 4; ++j) G2[qq][j] = __ffma2_rn(rr2[qq], g2[j], G2[qq][j]);
                 }
                 float o0, o1;
                 reduce_rows_over_cols(part, c1, c0, o0, o1);
@@ -373,7 +391,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                 const float vdy = sm.vdy[p];
                 prm.dr[o] = fmaf(sm.u[i] * kk, vdy, drs);
                 prm.dk[o] = fmaf(sm.u[i] * rr, vdy, dks);
-                prm.dv[o] = fmaf(sm.ruk[p], sm.dys[p][i], dvv);
+                prm.dv[o] = fmaf(sm.ruk[p], sm.raw[s][A_DY][row][i], dvv);
                 prm.dw[o] = fmaf(rr, drs, kk * dks);           // z_t, parked in dw
             } else {
                 prm.dr[o] = sm.part[s][0][row][i] + drs;
