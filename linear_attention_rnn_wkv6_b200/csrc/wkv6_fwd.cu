@@ -137,11 +137,15 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     const int jc = 16 * warp + 4 * cg;       // CTA-relative first column of this lane
     const int jj = (rg >> 1) & 3;            // column (of the 4) this lane holds after the reduce
     const bool b2 = (rg & 4) != 0, b1 = (rg & 2) != 0;
-    float S[8][4];
+    // packed fp32: S2[qq][j] = (S[row 2qq][j], S[row 2qq+1][j]) for the row pairs
+    // (rowA, rowA+1), (rowA+2, rowA+3), (rowB, rowB+1), (rowB+2, rowB+3); one
+    // __ffma2_rn does two multiply-adds
+    constexpr float2 kZero2 = {0.f, 0.f};
+    float2 S2[4][4];
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
+    for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) S[q][j] = 0.f;
+        for (int j = 0; j < 4; ++j) S2[qq][j] = kZero2;
 
     for (int g = 0; g < nchunks; ++g) {
         const ChunkPos cp = chunk_pos(g, nch, T, TC, BIDIR);
@@ -149,9 +153,9 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         const bool with_bonus = !(BIDIR && cp.pass == 0);
         if (BIDIR && g == nch) {             // pass boundary: fresh state
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
+            for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) S[q][j] = 0.f;
+                for (int j = 0; j < 4; ++j) S2[qq][j] = kZero2;
         }
         // ---- wait for the chunk ----
         const bool ok = mbar_wait_bounded(&sm.full[s], (g >> 1) & 1);
@@ -184,22 +188,36 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         __syncthreads();
         const uint32_t rmask = sm.renorm_mask;
         // ---- transform: scaled r, k per row (sequential over the chunk) ----
-        for (int i = tid; i < kHead; i += NT) {
+        // two threads per row i, each half of the chunk; the second one first sums
+        // the decays of the first half (with the renorm resets)
+        {
+            static_assert(NT == 2 * kHead && TC % 2 == 0, "transform split assumes 2 threads per row");
+            constexpr int TH = TC / 2;
+            const int i = tid & (kHead - 1), p0 = (tid >> 6) * TH;
             float L = 0.f;
-#pragma unroll 4
-            for (int p = 0; p < TC; ++p) {
+            for (int p = 0; p < p0; ++p) {
                 const int row = cp.dir > 0 ? p : TC - 1 - p;
-                const float ew = to_f32(sm.raw_w[s][row][i]);
-                const float rr = to_f32(sm.raw_r[s][row][i]);
-                const float kk = to_f32(sm.raw_k[s][row][i]);
-                sm.rs[p][i] = rr * __expf(L);
+                L = ((rmask >> p) & 1u) ? 0.f : L + to_f32(sm.raw_w[s][row][i]);
+            }
+            float ew[TH], rr[TH], kk[TH];
+#pragma unroll
+            for (int e = 0; e < TH; ++e) {
+                const int p = p0 + e, row = cp.dir > 0 ? p : TC - 1 - p;
+                ew[e] = to_f32(sm.raw_w[s][row][i]);
+                rr[e] = to_f32(sm.raw_r[s][row][i]);
+                kk[e] = to_f32(sm.raw_k[s][row][i]);
+            }
+#pragma unroll
+            for (int e = 0; e < TH; ++e) {
+                const int p = p0 + e;
+                sm.rs[p][i] = rr[e] * __expf(L);
                 if ((rmask >> p) & 1u) {
-                    sm.al[p][i] = __expf(L + ew);
-                    sm.ks[p][i] = kk;
+                    sm.al[p][i] = __expf(L + ew[e]);
+                    sm.ks[p][i] = kk[e];
                     L = 0.f;
                 } else {
-                    L += ew;
-                    sm.ks[p][i] = kk * __expf(-L);
+                    L += ew[e];
+                    sm.ks[p][i] = kk[e] * __expf(-L);
                 }
             }
         }
@@ -233,34 +251,35 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             const float4 ka = *reinterpret_cast<const float4 *>(&sm.ks[p][rowA]);
             const float4 kb = *reinterpret_cast<const float4 *>(&sm.ks[p][rowB]);
             const float4 vv = *reinterpret_cast<const float4 *>(&sm.vs[p][jc]);
-            const float rr[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-            const float kr[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
-            const float vc[4] = {vv.x, vv.y, vv.z, vv.w};
+            const float2 rr2[4] = {make_float2(ra.x, ra.y), make_float2(ra.z, ra.w), make_float2(rb.x, rb.y),
+                                   make_float2(rb.z, rb.w)};
+            const float2 kr2[4] = {make_float2(ka.x, ka.y), make_float2(ka.z, ka.w), make_float2(kb.x, kb.y),
+                                   make_float2(kb.z, kb.w)};
+            const float2 v2[4] = {make_float2(vv.x, vv.x), make_float2(vv.y, vv.y), make_float2(vv.z, vv.z),
+                                  make_float2(vv.w, vv.w)};
             float yp[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                float a0 = rr[0] * S[0][j], a1 = rr[1] * S[1][j];
-                a0 = fmaf(rr[2], S[2][j], a0);
-                a1 = fmaf(rr[3], S[3][j], a1);
-                a0 = fmaf(rr[4], S[4][j], a0);
-                a1 = fmaf(rr[5], S[5][j], a1);
-                a0 = fmaf(rr[6], S[6][j], a0);
-                a1 = fmaf(rr[7], S[7][j], a1);
-                yp[j] = a0 + a1;
+                float2 acc = __ffma2_rn(rr2[0], S2[0][j], kZero2);
+#pragma unroll
+                for (int qq = 1; qq < 4; ++qq) acc = __ffma2_rn(rr2[qq], S2[qq][j], acc);
+                yp[j] = acc.x + acc.y;
             }
             if ((rmask >> p) & 1u) {
                 const float4 aa = *reinterpret_cast<const float4 *>(&sm.al[p][rowA]);
                 const float4 ab = *reinterpret_cast<const float4 *>(&sm.al[p][rowB]);
-                const float al[8] = {aa.x, aa.y, aa.z, aa.w, ab.x, ab.y, ab.z, ab.w};
+                const float2 al2[4] = {make_float2(aa.x, aa.y), make_float2(aa.z, aa.w), make_float2(ab.x, ab.y),
+                                       make_float2(ab.z, ab.w)};
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
+                for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) S[q][j] = fmaf(S[q][j], al[q], kr[q] * vc[j]);
+                    for (int j = 0; j < 4; ++j)
+                        S2[qq][j] = __ffma2_rn(S2[qq][j], al2[qq], __ffma2_rn(kr2[qq], v2[j], kZero2));
             } else {
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
+                for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) S[q][j] = fmaf(kr[q], vc[j], S[q][j]);
+                    for (int j = 0; j < 4; ++j) S2[qq][j] = __ffma2_rn(kr2[qq], v2[j], S2[qq][j]);
             }
             // reduce-scatter the 4 column partials over the 8 row groups (lanes xor 4, 2, 1)
             float k0 = b2 ? yp[2] : yp[0];
@@ -282,18 +301,33 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
 
         // ---- write y for the chunk (float4, coalesced along channels) ----
         constexpr int V4 = CW / 4;
-        for (int e = tid; e < TC * V4; e += NT) {
-            const int p = e / V4, j4 = (e % V4) * 4;
+        static_assert((TC * V4) % NT == 0, "y write-out assumes whole rounds of the block");
+        constexpr int kRounds = TC * V4 / NT;
+        // pass 1 adds the anti-causal part that pass 0 of this CTA stored: all of
+        // this thread's loads are issued before its stores, so their latencies overlap
+        float4 old[kRounds];
+        if (BIDIR && cp.pass == 1) {
+#pragma unroll
+            for (int m = 0; m < kRounds; ++m) {
+                const int e = tid + m * NT, p = e / V4, j4 = (e % V4) * 4;
+                const int t = cp.dir > 0 ? cp.t_lo + p : cp.t_lo + TC - 1 - p;
+                old[m] = (t >= 0 && t < T)
+                             ? *reinterpret_cast<const float4 *>(prm.y + ((size_t)b * T + t) * C + cbase + col0 + j4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < kRounds; ++m) {
+            const int e = tid + m * NT, p = e / V4, j4 = (e % V4) * 4;
             const int t = cp.dir > 0 ? cp.t_lo + p : cp.t_lo + TC - 1 - p;
             if (t < 0 || t >= T) continue;
             float4 *dst = reinterpret_cast<float4 *>(prm.y + ((size_t)b * T + t) * C + cbase + col0 + j4);
             float4 val = *reinterpret_cast<const float4 *>(&sm.ybuf[p][j4]);
             if (BIDIR && cp.pass == 1) {
-                const float4 old = *dst;    // anti-causal part written by pass 0 of this CTA
-                val.x += old.x;
-                val.y += old.y;
-                val.z += old.z;
-                val.w += old.w;
+                val.x += old[m].x;
+                val.y += old[m].y;
+                val.z += old[m].z;
+                val.w += old[m].w;
             }
             *dst = val;
         }
