@@ -1,0 +1,84 @@
+"""Run hot-path kernels a fixed number of times, for profilers.
+
+    python -m linear_attention_rnn_wkv6_b200.profile_cases [--case NAME[:B:T]] ... [--rounds R]
+
+Each case is one of the benchmark step's workloads (``synth.WORKLOADS``),
+optionally with its batch B and length T replaced, so that a profiler can
+capture a smaller instance of the same kernel.  Every round calls each case
+once, in the order given, through the C ABI (the backward adds its du
+reduction launch).  Inputs are the seeded synthetic ones of ``synth``; nothing
+here computes any part of the operator.
+"""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+
+from . import synth
+
+
+def _dev(a):
+    import torch
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def make_case(spec: str):
+    """Parse NAME[:B:T] and return (label, callable that launches the case once)."""
+    import torch
+    import linear_attention_rnn_wkv6_b200 as wkv
+
+    parts = spec.split(":")
+    name = parts[0]
+    kind, kw = synth.WORKLOADS[name]
+    kw = dict(kw)
+    if len(parts) == 3:
+        kw["B"], kw["T"] = int(parts[1]), int(parts[2])
+    if kind == "wkv4_fwd":
+        x = synth.make_wkv4(kw["B"], kw["T"], kw["C"], seed=0)
+        ins = [_dev(getattr(x, n)) for n in ("k", "v", "w", "u")]
+        y = torch.empty(x.B, x.T, x.C, device="cuda")
+        return f"{name} B={x.B} T={x.T}", lambda: wkv.wkv4_fwd(x.B, x.T, x.C, *ins, y)
+    args = {k: v for k, v in kw.items() if k not in ("B", "T", "H")}
+    x = synth.make_wkv6(kw["B"], kw["T"], kw["H"], seed=0, **args)
+    label = f"{name} B={x.B} T={x.T} H={x.H}"
+    if kind.startswith("wkv6_bwd"):
+        bidir = kind == "wkv6_bwd_bidir"
+        ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u", "dy")]
+        outs = [torch.empty(x.B, x.T, x.C, device="cuda") for _ in range(4)] + [torch.empty(x.C, device="cuda")]
+        nb = wkv.wkv6_bwd_workspace_bytes(x.B, x.T, x.C, x.H, bidir)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        return label, lambda: wkv.wkv6_bwd(x.B, x.T, x.C, x.H, bidir, *ins, *outs, ws, nb)
+    ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u")]
+    y = torch.empty(x.B, x.T, x.C, device="cuda")
+    fn = getattr(wkv, kind)
+    return label, lambda: fn(x.B, x.T, x.C, x.H, *ins, y)
+
+
+def main(argv=None) -> int:
+    import torch
+    import linear_attention_rnn_wkv6_b200 as wkv
+
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--case", action="append", required=True,
+                    help="workload name from synth.WORKLOADS, optionally NAME:B:T")
+    ap.add_argument("--rounds", type=int, default=2)
+    a = ap.parse_args(argv)
+    cases = [make_case(c) for c in a.case]
+    for _ in range(a.rounds):
+        for _, run in cases:
+            run()
+    torch.cuda.synchronize()
+    faults = wkv.wkv_take_device_faults()
+    for label, _ in cases:
+        print(label)
+    if faults:
+        print(f"device fault word {faults:#x}")
+        return 1
+    return 0
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())
