@@ -42,9 +42,10 @@ def build(force: bool = False) -> str:
 def _configure(lib):
     I = ctypes.c_int
     lib.oracle_wkv6_fwd.argtypes = [I, I, I, I, I] + [_DP] * 6
+    lib.oracle_wkv6_fwd_state.argtypes = [I, I, I, I] + [_DP] * 8
     lib.oracle_wkv6_bwd.argtypes = [I, I, I, I, I] + [_DP] * 11
     lib.oracle_wkv4_fwd.argtypes = [I, I, I] + [_DP] * 5
-    for f in (lib.oracle_wkv6_fwd, lib.oracle_wkv6_bwd, lib.oracle_wkv4_fwd):
+    for f in (lib.oracle_wkv6_fwd, lib.oracle_wkv6_fwd_state, lib.oracle_wkv6_bwd, lib.oracle_wkv4_fwd):
         f.restype = ctypes.c_int
     return lib
 
@@ -73,6 +74,25 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_wkv6_fwd failed ({rc})")
         return y
+
+    def wkv6_fwd_state(self, r, k, v, w, u, H: int, s0=None):
+        """Causal RWKV-6 forward from the initial state s0 ([B,H,N,N], None = zero).
+        Returns (y [B,T,C], sT [B,H,N,N] = the state after the last token)."""
+        r, k, v, w, u = map(_d, (r, k, v, w, u))
+        B, T, C = r.shape
+        N = C // H
+        y = np.zeros((B, T, C), dtype=np.float64)
+        sT = np.zeros((B, H, N, N), dtype=np.float64)
+        s0p = None
+        if s0 is not None:
+            s0 = _d(s0)
+            if s0.shape != (B, H, N, N):
+                raise ValueError(f"s0 must have shape {(B, H, N, N)}")
+            s0p = _p(s0)
+        rc = self._lib.oracle_wkv6_fwd_state(B, T, C, H, _p(r), _p(k), _p(v), _p(w), _p(u), s0p, _p(y), _p(sT))
+        if rc != 0:
+            raise ValueError(f"oracle_wkv6_fwd_state failed ({rc})")
+        return y, sT
 
     def wkv6_bwd(self, r, k, v, w, u, dy, H: int, bidirectional: bool = False):
         """RWKV-6 WKV backward -> (dr, dk, dv, dw, du); dw is w.r.t. the log-decay ew."""
@@ -105,6 +125,10 @@ def _default() -> Oracle:
 
 def wkv6_fwd(r, k, v, w, u, H: int, bidirectional: bool = False) -> np.ndarray:
     return _default().wkv6_fwd(r, k, v, w, u, H, bidirectional)
+
+
+def wkv6_fwd_state(r, k, v, w, u, H: int, s0=None):
+    return _default().wkv6_fwd_state(r, k, v, w, u, H, s0)
 
 
 def wkv6_bwd(r, k, v, w, u, dy, H: int, bidirectional: bool = False):

@@ -43,9 +43,12 @@
 /* ------------------------------------------------------------------------ */
 static void wkv6_head_sweep(int T, int C, int N, int b, int h, int reverse, int bonus,
                             const double *r, const double *k, const double *v,
-                            const double *w, const double *u, double *y, double *S, double *M)
+                            const double *w, const double *u, double *y, double *S, double *M,
+                            const double *s_init)
 {
-    memset(S, 0, sizeof(double) * (size_t)N * N);
+    /* S starts as s_init (N x N) or zero; on return it holds the state after the sweep */
+    if (s_init) memcpy(S, s_init, sizeof(double) * (size_t)N * N);
+    else memset(S, 0, sizeof(double) * (size_t)N * N);
     for (int step = 0; step < T; ++step) {
         const int t = reverse ? (T - 1 - step) : step;
         const double *rt = r + IDX(b, t, h * N);
@@ -86,8 +89,39 @@ int oracle_wkv6_fwd(int B, int T, int C, int H, int bidirectional,
     if (!S || !M) { free(S); free(M); return -2; }
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h) {
-            if (bidirectional) wkv6_head_sweep(T, C, N, b, h, 1, 0, r, k, v, w, u, y, S, M);
-            wkv6_head_sweep(T, C, N, b, h, 0, 1, r, k, v, w, u, y, S, M);
+            if (bidirectional) wkv6_head_sweep(T, C, N, b, h, 1, 0, r, k, v, w, u, y, S, M, NULL);
+            wkv6_head_sweep(T, C, N, b, h, 0, 1, r, k, v, w, u, y, S, M, NULL);
+        }
+    free(S);
+    free(M);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Causal RWKV-6 forward carrying the state across calls (RWKV Architecture   */
+/* page, Recurrent Inference Formulation: the N x N state is all that a step  */
+/* needs from the past, so a sequence may be processed in pieces).  The same */
+/* recurrence as above with S_{-1} = s0 instead of 0:                          */
+/*   s0 : [B][H][N][N] (row i = key channel, column j = value channel), or     */
+/*        NULL for the zero state;                                             */
+/*   sT : [B][H][N][N] receives S_{T-1} (s0 itself when T = 0), or NULL.       */
+/* ------------------------------------------------------------------------ */
+int oracle_wkv6_fwd_state(int B, int T, int C, int H, const double *r, const double *k,
+                          const double *v, const double *w, const double *u, const double *s0,
+                          double *y, double *sT)
+{
+    if (B < 0 || T < 0 || H < 1 || C % H != 0) return -1;
+    const int N = C / H;
+    const size_t NN = (size_t)N * N;
+    memset(y, 0, sizeof(double) * (size_t)B * T * C);
+    double *S = (double *)malloc(sizeof(double) * NN);
+    double *M = (double *)malloc(sizeof(double) * NN);
+    if (!S || !M) { free(S); free(M); return -2; }
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const size_t off = ((size_t)b * H + h) * NN;
+            wkv6_head_sweep(T, C, N, b, h, 0, 1, r, k, v, w, u, y, S, M, s0 ? s0 + off : NULL);
+            if (sT) memcpy(sT + off, S, sizeof(double) * NN);
         }
     free(S);
     free(M);

@@ -54,6 +54,25 @@ def wkv6(r, k, v, w, u, H, past=True, future=False, bonus=True):
     return y
 
 
+def wkv6_head_state(r, k, v, w, u, s0):
+    """Causal pair form started from the state s0 ([N,N], row i = key channel).
+
+    The initial state reaches y_t through the decays of tokens 0..t-1 and the
+    final state holds every pair decayed to the end:
+        y_t  = sum_s A_ts v_s + (r_t * exp(sum_{m<t} w_m)) . s0
+        S_T-1 = diag(exp(sum_m w_m)) s0 + sum_s diag(exp(sum_{m>s} w_m)) k_s^T v_s
+    """
+    r, k, v, w, u, s0 = (np.asarray(a, dtype=np.float64) for a in (r, k, v, w, u, s0))
+    T, N = r.shape
+    y = wkv6_head(r, k, v, w, u)
+    for t in range(T):
+        y[t] += (r[t] * np.exp(w[:t].sum(axis=0))) @ s0
+    sT = np.exp(w.sum(axis=0))[:, None] * s0
+    for s in range(T):
+        sT = sT + np.outer(k[s] * np.exp(w[s + 1:].sum(axis=0)), v[s])
+    return y, sT
+
+
 def wkv6_head_grads(r, k, v, w, u, dy, past=True, future=False):
     """Gradients of sum(dy * y) from the pair form (bonus always on).
 

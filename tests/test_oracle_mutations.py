@@ -37,6 +37,12 @@ MUTATIONS = [
       lambda o: pins.test_wkv6_backward_euler_identities(o, False)]),
     ("bwd_dk_drops_bonus", "dkt[i] += acck + u[h * N + i] * rt[i] * vdy;", "dkt[i] += acck;", 0,
      [lambda o: pins.test_wkv6_backward_matches_pair_form(o, False, 9, 4)]),
+    ("state_initial_transposed", "if (s_init) memcpy(S, s_init, sizeof(double) * (size_t)N * N);",
+     "if (s_init) { for (int i = 0; i < N; ++i) for (int j = 0; j < N; ++j) S[i * N + j] = s_init[j * N + i]; }",
+     0, [lambda o: pins.test_wkv6_state_matches_pair_form(o, 1, 7, 2, 8)]),
+    ("state_out_is_initial", "if (sT) memcpy(sT + off, S, sizeof(double) * NN);",
+     "if (sT) memcpy(sT + off, s0 ? s0 + off : S, sizeof(double) * NN);", 0,
+     [lambda o: pins.test_wkv6_state_matches_pair_form(o, 2, 3, 1, 4), lambda o: pins.test_wkv6_state_split_equals_whole(o, 13)]),
     ("wkv4_decay_sign", "e1 = exp(p - w[c] - q);", "e1 = exp(p + w[c] - q);", 0,
      [pins.test_wkv4_geometric_closed_form, pins.test_golden_wkv4_forward]),
     ("wkv4_missing_bonus", "e2 = exp(u[c] + kt - q);", "e2 = exp(kt - q);", 0,

@@ -254,6 +254,52 @@ def _wkv4_case(B, T, C, seed, kstd=1.0):
     return k, v, w, u
 
 
+# ---------------------------------------------------------------- state carried across calls
+
+@pytest.mark.parametrize("B,T,H,N", [(1, 1, 1, 4), (2, 3, 1, 4), (1, 7, 2, 8), (1, 33, 1, 8), (1, 5, 1, 64)])
+def test_wkv6_state_matches_pair_form(oracle_mod, B, T, H, N):
+    """y and the final state from an initial state s0 equal the pair sums with s0 decayed explicitly."""
+    r, k, v, w, u = _wkv6_case(B, T, H, N, seed=700 + 10 * T + N)
+    s0 = _rng(7 + T).normal(0, 1.0, (B, H, N, N))
+    y, sT = oracle_mod.wkv6_fwd_state(r, k, v, w, u, H, s0)
+    for b in range(B):
+        for h in range(H):
+            sl = slice(h * N, (h + 1) * N)
+            yb, sb = brute.wkv6_head_state(r[b, :, sl], k[b, :, sl], v[b, :, sl], w[b, :, sl], u[sl], s0[b, h])
+            assert np.max(np.abs(y[b, :, sl] - yb)) <= 1e-12 * max(1.0, np.max(np.abs(yb)))
+            assert np.max(np.abs(sT[b, h] - sb)) <= 1e-12 * max(1.0, np.max(np.abs(sb)))
+
+
+@pytest.mark.parametrize("cut", [0, 1, 13, 28, 29])
+def test_wkv6_state_split_equals_whole(oracle_mod, cut):
+    """Running tokens [0, cut) and then [cut, T) from the carried state reproduces the whole run."""
+    B, T, H, N = 2, 29, 2, 8
+    r, k, v, w, u = _wkv6_case(B, T, H, N, seed=901)
+    s0 = _rng(902).normal(0, 1.0, (B, H, N, N))
+    y, sT = oracle_mod.wkv6_fwd_state(r, k, v, w, u, H, s0)
+    a, z = slice(0, cut), slice(cut, T)
+    y1, s1 = oracle_mod.wkv6_fwd_state(r[:, a], k[:, a], v[:, a], w[:, a], u, H, s0)
+    y2, s2 = oracle_mod.wkv6_fwd_state(r[:, z], k[:, z], v[:, z], w[:, z], u, H, s1)
+    tol = 1e-12 * max(1.0, np.max(np.abs(y)))
+    assert np.max(np.abs(np.concatenate([y1, y2], axis=1) - y)) <= tol
+    assert np.max(np.abs(s2 - sT)) <= 1e-12 * max(1.0, np.max(np.abs(sT)))
+
+
+def test_wkv6_state_zero_is_the_plain_forward(oracle_mod):
+    B, T, H, N = 2, 11, 2, 4
+    r, k, v, w, u = _wkv6_case(B, T, H, N, seed=911)
+    y_plain = oracle_mod.wkv6_fwd(r, k, v, w, u, H=H)
+    y_none, s_none = oracle_mod.wkv6_fwd_state(r, k, v, w, u, H, None)
+    y_zero, s_zero = oracle_mod.wkv6_fwd_state(r, k, v, w, u, H, np.zeros((B, H, N, N)))
+    assert np.array_equal(y_none, y_plain) and np.array_equal(y_zero, y_plain)
+    assert np.array_equal(s_none, s_zero)
+    # no tokens: the state passes through unchanged
+    s0 = _rng(912).normal(0, 1.0, (B, H, N, N))
+    e = slice(0, 0)
+    y0, s_out = oracle_mod.wkv6_fwd_state(r[:, e], k[:, e], v[:, e], w[:, e], u, H, s0)
+    assert y0.shape == (B, 0, H * N) and np.array_equal(s_out, s0)
+
+
 @pytest.mark.parametrize("B,T,C", [(1, 1, 3), (2, 5, 3), (1, 40, 4)])
 def test_wkv4_recurrence_matches_ratio_of_sums(oracle_mod, B, T, C):
     k, v, w, u = _wkv4_case(B, T, C, seed=60 + T)
