@@ -95,6 +95,42 @@ int wkv6_bidir_fwd(int B, int T, int C, int H, const float *r, const float *k, c
                    const float *w, const float *u, float *y, wkv_stream_t stream);
 
 /*
+ * wkv6_fwd_state -- wkv6_fwd carrying the recurrent state across calls, so that a
+ * sequence can be processed in pieces (streaming, recurrent inference: "RWKV
+ * Architecture ...", Recurrent Inference Formulation -- the N x N state is all a
+ * step needs from the past).  Same operation with S_{-1} = s0 instead of 0:
+ *     y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),   S_t = diag(exp(w_t)) S_{t-1} + k_t^T v_t.
+ *   r, k, v, w, u, y : as in wkv6_fwd (fp32, causal)
+ *   s0 : [B,H,N,N] float, the initial state of each (b, h): element (i, j) at
+ *        ((b*H + h)*N + i)*N + j, row i = key channel, column j = value channel;
+ *        NULL means the zero state
+ *   sT : [B,H,N,N] float, output: the state S_{T-1} after the last token (s0, or
+ *        zero, when T == 0); NULL if not wanted.  s0 and sT may be the same buffer
+ *        (updated in place); neither may overlap the other arguments.
+ * Running wkv6_fwd_state on tokens [0, t) and then on [t, T) with the first
+ * call's sT as the second call's s0 gives the same y and final state as one call
+ * on [0, T) (up to fp32 rounding).  Errors: as wkv6_fwd, plus WKV_ERR_ALIGN for a
+ * misaligned s0 or sT and WKV_ERR_TOO_LARGE when B*H*N*N >= 2^31.
+ */
+int wkv6_fwd_state(int B, int T, int C, int H, const float *r, const float *k, const float *v,
+                   const float *w, const float *u, const float *s0, float *y, float *sT,
+                   wkv_stream_t stream);
+
+/*
+ * wkv6_decode -- one recurrent step for B independent sequences (token-by-token
+ * generation; the same recurrence as wkv6_fwd_state with T = 1, s0 = sT = state):
+ *     y_b = r_b (S_b + diag(u) k_b^T v_b),   S_b <- diag(exp(w_b)) S_b + k_b^T v_b.
+ *   r, k, v, w : [B,C] float, this step's token of each sequence (w = log-decay)
+ *   u          : [C] float
+ *   state      : [B,H,N,N] float, in/out, layout as s0 of wkv6_fwd_state
+ *   y          : [B,C] float, output
+ * Errors: WKV_ERR_ARG, WKV_ERR_HEADSIZE, WKV_ERR_ALIGN, WKV_ERR_TOO_LARGE
+ * (B*H*N*N >= 2^31), WKV_ERR_DEVICE, WKV_ERR_CUDA; B == 0 launches nothing.
+ */
+int wkv6_decode(int B, int C, int H, const float *r, const float *k, const float *v, const float *w,
+                const float *u, float *state, float *y, wkv_stream_t stream);
+
+/*
  * wkv6_bwd -- gradients of L = sum(dy * y) for wkv6_fwd (bidirectional == 0) or
  * wkv6_bidir_fwd (bidirectional != 0), fp32 ("How Custom CUDA Kernels
  * (wkv6_cuda.cu) ...", Backward Pass Gradient Computation; arguments follow the

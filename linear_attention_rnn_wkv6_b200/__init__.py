@@ -18,7 +18,7 @@ import os
 __all__ = [
     "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
-    "wkv6_bwd_noalloc", "EXPORTED_SYMBOLS", "HEAD_SIZE",
+    "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "EXPORTED_SYMBOLS", "HEAD_SIZE",
 ]
 
 HEAD_SIZE = 64
@@ -28,7 +28,8 @@ _LIB = None
 # Every extern "C" symbol declared in include/wkv.h.
 EXPORTED_SYMBOLS = (
     "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
-    "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc",
+    "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc", "wkv6_fwd_state",
+    "wkv6_decode",
 )
 
 _I = ctypes.c_int
@@ -46,6 +47,8 @@ _SIGS = {
     "wkv_take_device_faults": ([ctypes.POINTER(ctypes.c_uint)], _I),
     "wkv_version": ([], _I),
     "wkv6_bwd_noalloc": ([_I] * 5 + [_P] * 11 + [_P], _I),
+    "wkv6_fwd_state": ([_I] * 4 + [_P] * 8 + [_P], _I),
+    "wkv6_decode": ([_I] * 3 + [_P] * 7 + [_P], _I),
 }
 
 
@@ -117,6 +120,19 @@ def wkv6_bidir_fwd(B, T, C, H, r, k, v, w, u, y, stream=None) -> None:
     """Bidirectional RWKV-6 WKV forward (fp32)."""
     _check("wkv6_bidir_fwd", load().wkv6_bidir_fwd(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
                                                    _ptr(y), _stream(stream)))
+
+
+def wkv6_fwd_state(B, T, C, H, r, k, v, w, u, s0, y, sT, stream=None) -> None:
+    """Causal RWKV-6 forward (fp32) from the initial state s0 ([B,H,N,N] or None for zero);
+    writes the final state into sT ([B,H,N,N] or None)."""
+    _check("wkv6_fwd_state", load().wkv6_fwd_state(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
+                                                   _ptr(s0), _ptr(y), _ptr(sT), _stream(stream)))
+
+
+def wkv6_decode(B, C, H, r, k, v, w, u, state, y, stream=None) -> None:
+    """One recurrent step: r, k, v, w [B,C]; state [B,H,N,N] updated in place; y [B,C]."""
+    _check("wkv6_decode", load().wkv6_decode(B, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(state),
+                                             _ptr(y), _stream(stream)))
 
 
 def wkv6_bwd_workspace_bytes(B, T, C, H, bidirectional) -> int:

@@ -146,6 +146,21 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
         for (int j = 0; j < 4; ++j) S2[qq][j] = kZero2;
+    // state row of pair qq, half e (0: first row of the pair, 1: second)
+    auto prow = [&](int qq, int e) { return (qq < 2 ? rowA + 2 * qq : rowB + 2 * (qq - 2)) + e; };
+    const size_t state_off = ((size_t)b * H + h) * kHead * kHead + col0 + jc;
+    if (!BIDIR && prm.s0 != nullptr) {
+        // initial state: the scaled state equals the true state at a chunk start
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const float4 x0 = *reinterpret_cast<const float4 *>(prm.s0 + state_off + (size_t)prow(qq, 0) * kHead);
+            const float4 x1 = *reinterpret_cast<const float4 *>(prm.s0 + state_off + (size_t)prow(qq, 1) * kHead);
+            S2[qq][0] = make_float2(x0.x, x1.x);
+            S2[qq][1] = make_float2(x0.y, x1.y);
+            S2[qq][2] = make_float2(x0.z, x1.z);
+            S2[qq][3] = make_float2(x0.w, x1.w);
+        }
+    }
 
     for (int g = 0; g < nchunks; ++g) {
         const ChunkPos cp = chunk_pos(g, nch, T, TC, BIDIR);
@@ -332,6 +347,17 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             *dst = val;
         }
         if (BIDIR && g == nch - 1) __syncthreads();  // pass-0 y stores visible before pass-1 reads
+    }
+    if (!BIDIR && prm.sT != nullptr) {
+        // every chunk ends with a renorm step, so the scaled state is the true
+        // state S_{T-1} here (tokens past T were zero-filled: k = 0, ew = 0)
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            *reinterpret_cast<float4 *>(prm.sT + state_off + (size_t)prow(qq, 0) * kHead) =
+                make_float4(S2[qq][0].x, S2[qq][1].x, S2[qq][2].x, S2[qq][3].x);
+            *reinterpret_cast<float4 *>(prm.sT + state_off + (size_t)prow(qq, 1) * kHead) =
+                make_float4(S2[qq][0].y, S2[qq][1].y, S2[qq][2].y, S2[qq][3].y);
+        }
     }
 }
 

@@ -85,9 +85,6 @@ int check_wkv6(int B, int T, int C, int H, std::initializer_list<const void *> p
     return WKV_OK;
 }
 
-// Algorithm of the bf16 causal forward: the chunked tensor-core kernel (default)
-// or the token-by-token recurrence (WKV6_BF16_PATH=recurrence).  Both compute
-// the same operation; the variable is read on every call.
 // Tensor maps of the backward: inputs r, k, w, v, dy, then the outputs dr, dk,
 // dv, dw (the second sweep reads back what the first sweep stored there).
 bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], int B, int T, int C, const float *r, const float *k,
@@ -99,19 +96,23 @@ bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], int B, int T, int C, const flo
     return true;
 }
 
+// Algorithm of the bf16 causal forward: the chunked tensor-core kernel (default)
+// or the token-by-token recurrence (WKV6_BF16_PATH=recurrence).  Both compute
+// the same operation; the variable is read on every call.
 bool bf16_use_tensor_cores() {
     const char *e = std::getenv("WKV6_BF16_PATH");
     return !(e && std::strcmp(e, "recurrence") == 0);
 }
 
 int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r, const void *k, const void *v,
-               const void *w, const float *u, float *y, wkv_stream_t stream) {
+               const void *w, const float *u, float *y, wkv_stream_t stream, const float *s0 = nullptr,
+               float *sT = nullptr) {
     int st = check_wkv6(B, T, C, H, {r, k, v, w, u, y});
     if (st != WKV_OK) return st;
     if (B == 0 || T == 0) return WKV_OK;
     if ((st = check_device()) != WKV_OK) return st;
     CUtensorMap mr, mk, mv, mw;
-    if (bf16 && !bidir && bf16_use_tensor_cores()) {
+    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && bf16_use_tensor_cores()) {
         constexpr int kTcChunk = 64;
         if (!make_map(&mr, r, true, B, T, C, kHead, kTcChunk, true) ||
             !make_map(&mk, k, true, B, T, C, kHead, kTcChunk, true) ||
@@ -127,6 +128,8 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
         !make_map(&mv, v, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mw, w, bf16, B, T, C, kHead, kFwdTC))
         return WKV_ERR_CUDA;
     FwdParams prm{B, T, C, H, u, y};
+    prm.s0 = s0;
+    prm.sT = sT;
     return wkv6_fwd_launch(bf16, bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)) ==
                    cudaSuccess
                ? WKV_OK
@@ -153,6 +156,45 @@ int wkv6_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t 
 int wkv6_bidir_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
                    const float *u, float *y, wkv_stream_t stream) {
     return fwd_common(false, true, B, T, C, H, r, k, v, w, u, y, stream);
+}
+
+int wkv6_fwd_state(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
+                   const float *u, const float *s0, float *y, float *sT, wkv_stream_t stream) {
+    int st = check_wkv6(B, T, C, H, {r, k, v, w, u, y});
+    if (st != WKV_OK) return st;
+    if ((long long)B * H * kHead * kHead >= (1ll << 31)) return WKV_ERR_TOO_LARGE;
+    if ((s0 != nullptr && !aligned16(s0)) || (sT != nullptr && !aligned16(sT))) return WKV_ERR_ALIGN;
+    if (B == 0) return WKV_OK;
+    if (T == 0) {
+        // no tokens: the final state is the initial one
+        if (sT == nullptr) return WKV_OK;
+        if ((st = check_device()) != WKV_OK) return st;
+        const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+        const size_t bytes = sizeof(float) * (size_t)B * H * kHead * kHead;
+        if (s0 == sT) return WKV_OK;
+        const cudaError_t e = s0 != nullptr ? cudaMemcpyAsync(sT, s0, bytes, cudaMemcpyDeviceToDevice, cs)
+                                            : cudaMemsetAsync(sT, 0, bytes, cs);
+        return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    }
+    return fwd_common(false, false, B, T, C, H, r, k, v, w, u, y, stream, s0, sT);
+}
+
+int wkv6_decode(int B, int C, int H, const float *r, const float *k, const float *v, const float *w,
+                const float *u, float *state, float *y, wkv_stream_t stream) {
+    if (B < 0 || C < 1 || H < 1 || C % H != 0) return WKV_ERR_ARG;
+    if (!r || !k || !v || !w || !u || !state || !y) return WKV_ERR_ARG;
+    if (C / H != kHead) return WKV_ERR_HEADSIZE;
+    if ((long long)B * H * kHead * kHead >= (1ll << 31)) return WKV_ERR_TOO_LARGE;
+    for (const void *p : {(const void *)r, (const void *)k, (const void *)v, (const void *)w, (const void *)u,
+                          (const void *)state, (const void *)y})
+        if (!aligned16(p)) return WKV_ERR_ALIGN;
+    if (B == 0) return WKV_OK;
+    const int st = check_device();
+    if (st != WKV_OK) return st;
+    return wkv6_decode_launch(B, C, H, r, k, v, w, u, state, y, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? WKV_OK
+               : WKV_ERR_CUDA;
 }
 
 size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional) {

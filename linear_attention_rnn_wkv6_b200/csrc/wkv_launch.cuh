@@ -9,6 +9,10 @@ struct FwdParams {
     int B, T, C, H;
     const float *u;
     float *y;
+    // causal recurrence only: initial state S_{-1} and final state S_{T-1},
+    // [B][H][N][N] (row i = key channel, column j = value channel); null = none
+    const float *s0 = nullptr;
+    float *sT = nullptr;
 };
 
 struct BwdParams {
@@ -26,6 +30,9 @@ cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const 
                             cudaStream_t stream);
 cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
                                const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream);
+// One recurrent step for B sequences (state [B][H][N][N] updated in place).
+cudaError_t wkv6_decode_launch(int B, int C, int H, const float *r, const float *k, const float *v,
+                               const float *w, const float *u, float *state, float *y, cudaStream_t stream);
 // maps: kBwdMaps tensor maps, in the order r, k, w, v, dy, dr, dk, dv, dw
 constexpr int kBwdMaps = 9;
 cudaError_t wkv6_bwd_launch(bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,

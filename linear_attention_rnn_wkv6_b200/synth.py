@@ -12,7 +12,8 @@ Generator (counter based, independent of numpy/torch RNG versions):
   function of ``(seed, stream, i)``, so any slice can be regenerated alone.
 * uniform in [0, 1): top 53 bits of a draw times 2^-53.
 * normal: Box-Muller, one normal per pair of draws (2i, 2i+1), cosine branch.
-* every array has its own stream id (draw order r, k, v, w_raw, u, dy).
+* every array has its own stream id (draw order r, k, v, w_raw, u, dy, then
+  the initial recurrent state s0).
 
 The log-decay handed to the WKV6 entry points is ``ew = -exp(w_raw)``, computed
 here in float64 and then rounded to the input dtype: it is the input recipe of
@@ -33,7 +34,7 @@ _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-STREAM_R, STREAM_K, STREAM_V, STREAM_WRAW, STREAM_U, STREAM_DY = range(6)
+STREAM_R, STREAM_K, STREAM_V, STREAM_WRAW, STREAM_U, STREAM_DY, STREAM_S0 = range(7)
 
 _CHUNK = 1 << 16  # elements per block: scratch stays cache resident and is reused in place
 _SCALE53 = 1.0 / 9007199254740992.0
@@ -202,6 +203,11 @@ def make_wkv6(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, rkv_std: fl
     u = normal(seed, STREAM_U, C, u_std).astype(np.float32)
     dy = normal(seed, STREAM_DY, n, dy_std).astype(np.float32).reshape(shape) if with_dy else None
     return Wkv6Inputs(B, T, C, H, r, k, v, w, u, dy, dtype)
+
+
+def make_state(B: int, H: int, N: int = 64, *, seed: int = 0, std: float = 1.0) -> np.ndarray:
+    """An RWKV-6 recurrent state per (b, h): [B,H,N,N] float32 ~ N(0, std^2) (its own stream)."""
+    return normal(seed, STREAM_S0, B * H * N * N, std).astype(np.float32).reshape(B, H, N, N)
 
 
 def make_wkv4(B: int, T: int, C: int, *, seed: int = 0, kv_std: float = 1.0,

@@ -94,6 +94,32 @@ def test_wkv6_backward_argument_errors(lib):
     assert lib.wkv6_bwd(2, 8, 128, 2, 0, *q, FAKE, ws, None) == WKV_ERR_ALIGN
 
 
+def test_wkv6_state_argument_errors(lib):
+    f = lib.wkv6_fwd_state
+    p = [FAKE + 256 * i for i in range(5)]                     # r, k, v, w, u
+    s0, y, sT = FAKE + 4096, FAKE + 8192, FAKE + 12288
+    assert f(-1, 4, 64, 1, *p, s0, y, sT, None) == WKV_ERR_ARG
+    assert f(1, 4, 64, 2, *p, s0, y, sT, None) == WKV_ERR_HEADSIZE
+    assert f(1, 4, 64, 1, *p, s0, None, sT, None) == WKV_ERR_ARG    # y is required
+    assert f(1, 4, 64, 1, *p, s0 + 4, y, sT, None) == WKV_ERR_ALIGN
+    assert f(1, 4, 64, 1, *p, s0, y, sT + 8, None) == WKV_ERR_ALIGN
+    assert f(1 << 20, 1, 64 * 64, 64, *p, s0, y, sT, None) == -7    # too large
+    assert f(0, 4, 64, 1, *p, None, y, None, None) == WKV_OK        # states are optional
+
+
+def test_wkv6_decode_argument_errors(lib):
+    f = lib.wkv6_decode
+    p = [FAKE + 256 * i for i in range(5)]                     # r, k, v, w, u
+    st, y = FAKE + 4096, FAKE + 8192
+    assert f(-1, 64, 1, *p, st, y, None) == WKV_ERR_ARG
+    assert f(1, 100, 3, *p, st, y, None) == WKV_ERR_ARG               # C not divisible by H
+    assert f(1, 64, 2, *p, st, y, None) == WKV_ERR_HEADSIZE
+    assert f(1, 64, 1, *p, None, y, None) == WKV_ERR_ARG              # state is required
+    assert f(1, 64, 1, *p, st + 4, y, None) == WKV_ERR_ALIGN
+    assert f(1 << 20, 64 * 64, 64, *p, st, y, None) == -7             # B*H*N*N >= 2^31
+    assert f(0, 64, 1, *p, st, y, None) == WKV_OK
+
+
 def test_wkv4_argument_errors(lib):
     p = [FAKE + 256 * i for i in range(5)]
     assert lib.wkv4_fwd(-1, 4, 32, *p, None) == WKV_ERR_ARG
