@@ -36,6 +36,8 @@ METRIC = "WKV tokens/sec/GPU and % of roofline (HBM GB/s or FP32/TC util) vs CPU
 UNIT = "tokens/s"
 WORKLOAD_NAME = ("wkv-hot-path step: wkv4_fwd B8xT1024xC768 f32 + wkv6_bidir_fwd B32xT196xH12 f32 + "
                  "wkv6_fwd_bf16 B8xT4096xH32 + wkv6_bwd(bidir) B32xT196xH12 f32, N=64")
+# Workloads outside the step, measured on their own with --only.
+EXTRA_WORKLOADS = ["wkv6_decode_f32_b512h32"]
 STEP_WORKLOADS = ["wkv4_f32_b8t1024c768", "wkv6_bidir_f32_b32t196h12", "wkv6_causal_bf16_b8t4096h32",
                   "wkv6_bidir_bwd_f32_b32t196h12"]
 N = 64
@@ -55,11 +57,16 @@ ALG = {
     "wkv6_bidir_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=10 * N * N, bound="alu"),
     "wkv6_causal_bf16_b8t4096h32": dict(bytes_per_unit=4 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
     "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="alu"),
+    # decode: the state is read and written once per step (2 N^2 floats) next to 5 N floats of token data
+    "wkv6_decode_f32_b512h32": dict(bytes_per_unit=2 * N * N * 4 + 5 * N * 4, flops_per_unit=5 * N * N,
+                                    bound="hbm"),
 }
 ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
-         "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd"}
+         "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd",
+         "wkv6_decode_f32_b512h32": "wkv6_decode"}
 LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
-            "wkv6_bidir_bwd_f32_b32t196h12": 2}   # the backward adds a deterministic du reduction
+            "wkv6_bidir_bwd_f32_b32t196h12": 2,   # the backward adds a deterministic du reduction
+            "wkv6_decode_f32_b512h32": 1}
 
 
 def units_of(name: str, x) -> int:
@@ -163,7 +170,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -231,6 +238,9 @@ class DeviceWorkload:
             self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
         else:
             self.outputs = [torch.empty(shape, device="cuda")]
+        if self.kind == "wkv6_decode":
+            # the recurrent state stays resident on the device (updated in place every step)
+            self.state = dev(synth.make_state(x.B, x.H, seed=seed))
         self.units = units_of(name, x)
         self.tokens = tokens_of(x)
 
@@ -248,6 +258,9 @@ class DeviceWorkload:
         elif self.kind == "wkv6_bwd_bidir":
             wkv.wkv6_bwd(x.B, x.T, x.C, x.H, 1, i["r"], i["k"], i["v"], i["w"], i["u"], i["dy"], *o,
                          self.ws, self.ws_bytes, s)
+        elif self.kind == "wkv6_decode":
+            # [B,1,C] token tensors are the [B,C] arrays the step reads
+            wkv.wkv6_decode(x.B, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], self.state, o[0], s)
         else:
             raise ValueError(self.kind)
 
@@ -489,13 +502,13 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget of the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
-    ap.add_argument("--only", action="append", choices=STEP_WORKLOADS,
+    ap.add_argument("--only", action="append", choices=STEP_WORKLOADS + EXTRA_WORKLOADS,
                     help="run only these workloads (profiling); the default step runs all four")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -9,9 +9,10 @@
 // state.  The step reads and writes each 16 KB state once, so it is bound by
 // HBM (and, for small B*H, by launch latency).
 //
-// One CTA per (b, h), 256 threads: thread (q, j) owns value column j and the 16
-// state rows 16q .. 16q+15, so every row access is one coalesced 256-byte row
-// segment.  A thread issues all its state loads before its in-place stores.
+// One CTA per (b, h), 256 threads: thread (q, g) owns the 4 x 4 block of rows
+// 4q .. 4q+3 and columns 4g .. 4g+3, read and written as float4 (16 threads
+// cover a 256-byte row); all state loads are issued before the in-place
+// stores, and the column sums over the 16 row blocks go through shared memory.
 #include "wkv_launch.cuh"
 
 namespace wkv {
@@ -19,31 +20,32 @@ namespace wkv {
 namespace {
 
 constexpr int kDecThreads = 256;
-constexpr int kRowsPerThread = kHead / (kDecThreads / kHead);   // 16 state rows per thread
+constexpr int kColGroups = kHead / 4;                  // 16 float4 column groups per row
+constexpr int kRowBlocks = kDecThreads / kColGroups;   // 16 blocks of 4 rows
+static_assert(kRowBlocks * 4 == kHead, "thread layout covers the state");
 
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, 4)
 wkv6_decode_kernel(int H, int C, const float *__restrict__ r, const float *__restrict__ k,
                    const float *__restrict__ v, const float *__restrict__ w, const float *__restrict__ u,
                    float *__restrict__ state, float *__restrict__ y) {
-    static_assert(kRowsPerThread * (kDecThreads / kHead) == kHead, "thread layout covers the state");
-    __shared__ float rs[kHead], ks[kHead], ds[kHead], vs[kHead];
-    __shared__ float part[kDecThreads / kHead][kHead];
+    __shared__ __align__(16) float rs[kHead], ks[kHead], ds[kHead], vs[kHead];   // vs is read as float4
+    __shared__ float4 part[kRowBlocks][kColGroups];
     __shared__ float bonus;
     const int tid = threadIdx.x;
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const size_t io = (size_t)b * C + (size_t)h * kHead;   // this head's channels of token b
-    const int j = tid & (kHead - 1), q = tid >> 6;
+    const int g = tid % kColGroups, q = tid / kColGroups;
 
+    float4 *S = reinterpret_cast<float4 *>(state + (size_t)bh * kHead * kHead) + g;
+    float4 sv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sv[e] = S[(size_t)(4 * q + e) * kColGroups];
     if (tid < kHead) {
         rs[tid] = r[io + tid];
         ks[tid] = k[io + tid];
         vs[tid] = v[io + tid];
         ds[tid] = expf(w[io + tid]);
     }
-    float *S = state + (size_t)bh * kHead * kHead + j;
-    float sv[kRowsPerThread];
-#pragma unroll
-    for (int e = 0; e < kRowsPerThread; ++e) sv[e] = S[(size_t)(kRowsPerThread * q + e) * kHead];
     __syncthreads();
 
     // bonus scalar c = sum_i r_i u_i k_i (warp 0)
@@ -53,21 +55,28 @@ wkv6_decode_kernel(int H, int C, const float *__restrict__ r, const float *__res
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
         if (tid == 0) bonus = c;
     }
-    const float vj = vs[j];
-    float acc = 0.f;
+    const float4 vj = reinterpret_cast<const float4 *>(vs)[g];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int e = 0; e < kRowsPerThread; ++e) {
-        const int i = kRowsPerThread * q + e;
-        acc = fmaf(rs[i], sv[e], acc);
-        S[(size_t)i * kHead] = fmaf(ds[i], sv[e], ks[i] * vj);
+    for (int e = 0; e < 4; ++e) {
+        const int i = 4 * q + e;
+        const float ri = rs[i], di = ds[i], ki = ks[i];
+        acc.x = fmaf(ri, sv[e].x, acc.x);
+        acc.y = fmaf(ri, sv[e].y, acc.y);
+        acc.z = fmaf(ri, sv[e].z, acc.z);
+        acc.w = fmaf(ri, sv[e].w, acc.w);
+        S[(size_t)i * kColGroups] = make_float4(fmaf(di, sv[e].x, ki * vj.x), fmaf(di, sv[e].y, ki * vj.y),
+                                                fmaf(di, sv[e].z, ki * vj.z), fmaf(di, sv[e].w, ki * vj.w));
     }
-    part[q][j] = acc;
+    part[q][g] = acc;
     __syncthreads();
-    if (q == 0) {
-        float yj = bonus * vj;
+    if (tid < kHead) {
+        // y_j = c v_j + sum over the 16 row blocks of column j
+        const float *pf = reinterpret_cast<const float *>(part);
+        float yj = bonus * vs[tid];
 #pragma unroll
-        for (int qq = 0; qq < kDecThreads / kHead; ++qq) yj += part[qq][j];
-        y[io + j] = yj;
+        for (int qq = 0; qq < kRowBlocks; ++qq) yj += pf[qq * kHead + tid];
+        y[io + tid] = yj;
     }
 }
 

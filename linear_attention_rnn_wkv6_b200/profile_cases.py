@@ -2,7 +2,7 @@
 
     python -m linear_attention_rnn_wkv6_b200.profile_cases [--case NAME[:B:T]] ... [--rounds R]
 
-Each case is one of the benchmark step's workloads (``synth.WORKLOADS``),
+Each case is one of the benchmark's workloads (``synth.WORKLOADS``),
 optionally with its batch B and length T replaced, so that a profiler can
 capture a smaller instance of the same kernel.  Every round calls each case
 once, in the order given, through the C ABI (the backward adds its du
@@ -53,6 +53,9 @@ def make_case(spec: str):
         return label, lambda: wkv.wkv6_bwd(x.B, x.T, x.C, x.H, bidir, *ins, *outs, ws, nb)
     ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u")]
     y = torch.empty(x.B, x.T, x.C, device="cuda")
+    if kind == "wkv6_decode":
+        state = _dev(synth.make_state(x.B, x.H, seed=0))
+        return label, lambda: wkv.wkv6_decode(x.B, x.C, x.H, *ins, state, y)
     fn = getattr(wkv, kind)
     return label, lambda: fn(x.B, x.T, x.C, x.H, *ins, y)
 

@@ -222,7 +222,7 @@ def make_wkv4(B: int, T: int, C: int, *, seed: int = 0, kv_std: float = 1.0,
     return Wkv4Inputs(B, T, C, k, v, w, u)
 
 
-# The five workloads: name -> (kind, constructor kwargs).
+# The workloads: name -> (kind, constructor kwargs).
 WORKLOADS = {
     # causal RWKV-6 forward, fp32, small (oracle finishes in seconds)
     "wkv6_causal_f32_b1t196h4": ("wkv6_fwd", dict(B=1, T=196, H=4)),
@@ -234,6 +234,8 @@ WORKLOADS = {
     "wkv6_causal_bf16_b8t4096h32": ("wkv6_fwd_bf16", dict(B=8, T=4096, H=32, wraw_lo=-8.0, dtype="bf16")),
     # bidirectional RWKV-6 backward, fp32
     "wkv6_bidir_bwd_f32_b32t196h12": ("wkv6_bwd_bidir", dict(B=32, T=196, H=12, with_dy=True)),
+    # one recurrent decode step for 512 sequences of the long-text head layout (state from make_state)
+    "wkv6_decode_f32_b512h32": ("wkv6_decode", dict(B=512, T=1, H=32)),
 }
 
 
