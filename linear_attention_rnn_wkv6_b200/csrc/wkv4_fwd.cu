@@ -9,30 +9,48 @@
 // maximum exponent, so e^{k} never overflows and every exp has argument <= 0.
 //
 // The pages' parallel form computes the sums "via parallel associative prefix
-// scans": here the T axis of each channel is split into SEG segments, one warp
-// each (lane = channel, 32 consecutive channels per CTA for 128-byte loads):
-//   phase 1  every warp folds its segment from the empty state -> (a, b, p)
-//   phase 2  warp s combines the summaries of segments 0..s-1 (a segment of
-//            length L maps state X to e^{-L w} X (+) local, where (+) is the
-//            log-space sum) -> the state entering its segment
-//   phase 3  every warp reruns its segment from that state and writes y.
+// scans": here the T axis of each channel is split into SEG segments.  A CTA
+// covers CH = 16 consecutive channels of one batch row and all SEG segments;
+// a warp holds 16 channels x 2 segments (each load instruction reads two
+// 64-byte row pieces), so the grid has B * C/16 equal CTAs, enough to spread
+// evenly over the SMs.
+//   phase 1  every thread folds its segment from the empty state -> (a, b, p)
+//   phase 2  the thread of segment s combines the summaries of segments
+//            0..s-1 (a segment of length L maps state X to e^{-L w} X (+)
+//            local, where (+) is the log-space sum) -> the state entering it
+//   phase 3  every thread reruns its segment from that state and writes y.
 // Phase 3 re-reads k and v; the CTA's tile was read moments before, so the
 // re-read is served by L2 and HBM traffic stays at the algorithmic bytes.
+// Per element the work is a handful of FMAs and one ex2 per update or output
+// (the larger exponent's factor is exactly 1, so every argument is <= 0 and
+// the running denominator b stays >= 1, which the fast division relies on).
 #include "wkv_launch.cuh"
 
 namespace wkv {
 
+namespace {
+
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kCh = 16;     // channels per CTA
+constexpr int kSeg = 32;    // segments of T per channel
+constexpr int kU = 4;       // tokens loaded ahead per step
 
 struct Wkv4State {
     float a, b, p;   // p in log2 units; represents (a 2^p, b 2^p)
 };
 
+// 2^x for x <= 0 (x = -inf gives 0)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // One token of the recurrence (log2 domain).  k2 = k*log2e; w2 = w*log2e.
 __device__ __forceinline__ void wkv4_update(Wkv4State &s, float k2, float v, float w2) {
     const float pd = s.p - w2;              // decayed exponent
     const float d = pd - k2;
-    const float ex = exp2f(-fabsf(d));      // 0 when pd = -inf
+    const float ex = ex2(-fabsf(d));        // 0 when pd = -inf
     const bool keep = d >= 0.f;
     const float e1 = keep ? 1.f : ex;
     const float e2 = keep ? ex : 1.f;
@@ -42,59 +60,63 @@ __device__ __forceinline__ void wkv4_update(Wkv4State &s, float k2, float v, flo
 }
 
 __device__ __forceinline__ float wkv4_output(const Wkv4State &s, float k2, float v, float u2) {
-    const float uk = u2 + k2;
-    const float d = s.p - uk;
-    const float ex = exp2f(-fabsf(d));
+    const float d = s.p - (u2 + k2);
+    const float ex = ex2(-fabsf(d));
     const bool keep = d >= 0.f;
     const float e1 = keep ? 1.f : ex;
     const float e2 = keep ? ex : 1.f;
-    return __fdividef(fmaf(e1, s.a, e2 * v), fmaf(e1, s.b, e2));
+    return __fdividef(fmaf(e1, s.a, e2 * v), fmaf(e1, s.b, e2));   // denominator >= 1
 }
 
-template <int SEG, int U>
-__global__ void __launch_bounds__(32 * SEG)
-wkv4_fwd_kernel(int B, int T, int C, const float *__restrict__ k, const float *__restrict__ v,
+__global__ void __launch_bounds__(kCh * kSeg, 3)
+wkv4_fwd_kernel(int T, int C, const float *__restrict__ k, const float *__restrict__ v,
                 const float *__restrict__ w, const float *__restrict__ u, float *__restrict__ y) {
-    __shared__ Wkv4State summ[SEG][32];
-    const int lane = threadIdx.x & 31;
-    const int seg = threadIdx.x >> 5;
-    const int groups = (C + 31) / 32;
+    __shared__ Wkv4State summ[kSeg][kCh];
+    const int tid = threadIdx.x;
+    const int ch = tid & (kCh - 1);
+    const int seg = tid / kCh;
+    const int groups = (C + kCh - 1) / kCh;
     const int b = blockIdx.x / groups;
-    const int c = (blockIdx.x % groups) * 32 + lane;
+    const int c = (blockIdx.x % groups) * kCh + ch;
     const bool live = c < C;
-    const int seglen = (T + SEG - 1) / SEG;
-    const int t0 = seg * seglen;
+    const int seglen = (T + kSeg - 1) / kSeg;
+    const int t0 = min(T, seg * seglen);
     const int t1 = min(T, t0 + seglen);
     const float w2 = live ? w[c] * kLog2e : 0.f;
     const float u2 = live ? u[c] * kLog2e : 0.f;
-    const size_t base = (size_t)b * T * C + c;
+    // this batch row's arrays; offsets inside it fit in 32 bits (B*T*C < 2^31)
+    const size_t brow = (size_t)b * T * C;
+    const float *kr = k + brow, *vr = v + brow;
+    float *yr = y + brow;
 
     // ---- phase 1: segment summary from the empty state ----
     Wkv4State st{0.f, 0.f, -INFINITY};
-    for (int t = t0; t < t1; t += U) {
-        float kb[U], vb[U];
+    int off = t0 * C + c;
+    for (int t = t0; t < t1; t += kU) {
+        float kb[kU], vb[kU];
 #pragma unroll
-        for (int i = 0; i < U; ++i) {
+        for (int i = 0; i < kU; ++i) {
             const bool in = live && (t + i < t1);
-            kb[i] = in ? __ldg(k + base + (size_t)(t + i) * C) : 0.f;
-            vb[i] = in ? __ldg(v + base + (size_t)(t + i) * C) : 0.f;
+            kb[i] = in ? __ldg(kr + off + i * C) : 0.f;
+            vb[i] = in ? __ldg(vr + off + i * C) : 0.f;
         }
 #pragma unroll
-        for (int i = 0; i < U; ++i)
+        for (int i = 0; i < kU; ++i)
             if (t + i < t1) wkv4_update(st, kb[i] * kLog2e, vb[i], w2);
+        off += kU * C;
     }
-    summ[seg][lane] = st;
+    summ[seg][ch] = st;
     __syncthreads();
 
     // ---- phase 2: state entering this segment ----
     Wkv4State in{0.f, 0.f, -INFINITY};
     for (int j = 0; j < seg; ++j) {
-        const int L = min(T, (j + 1) * seglen) - j * seglen;
-        const Wkv4State loc = summ[j][lane];
+        const int L = min(T, (j + 1) * seglen) - min(T, j * seglen);
+        const Wkv4State loc = summ[j][ch];
         const float pd = in.p - (float)L * w2;   // decay the carried state over segment j
         const float q = fmaxf(pd, loc.p);
         if (q == -INFINITY) continue;            // both empty
-        const float e1 = exp2f(pd - q), e2 = exp2f(loc.p - q);
+        const float e1 = ex2(pd - q), e2 = ex2(loc.p - q);
         in.a = fmaf(e1, in.a, e2 * loc.a);
         in.b = fmaf(e1, in.b, e2 * loc.b);
         in.p = q;
@@ -102,30 +124,33 @@ wkv4_fwd_kernel(int B, int T, int C, const float *__restrict__ k, const float *_
 
     // ---- phase 3: rerun the segment, write y ----
     st = in;
-    for (int t = t0; t < t1; t += U) {
-        float kb[U], vb[U];
+    off = t0 * C + c;
+    for (int t = t0; t < t1; t += kU) {
+        float kb[kU], vb[kU];
 #pragma unroll
-        for (int i = 0; i < U; ++i) {
+        for (int i = 0; i < kU; ++i) {
             const bool in_ = live && (t + i < t1);
-            kb[i] = in_ ? __ldg(k + base + (size_t)(t + i) * C) : 0.f;
-            vb[i] = in_ ? __ldg(v + base + (size_t)(t + i) * C) : 0.f;
+            kb[i] = in_ ? __ldg(kr + off + i * C) : 0.f;
+            vb[i] = in_ ? __ldg(vr + off + i * C) : 0.f;
         }
 #pragma unroll
-        for (int i = 0; i < U; ++i) {
+        for (int i = 0; i < kU; ++i) {
             if (t + i < t1 && live) {
                 const float k2 = kb[i] * kLog2e;
-                y[base + (size_t)(t + i) * C] = wkv4_output(st, k2, vb[i], u2);
+                yr[off + i * C] = wkv4_output(st, k2, vb[i], u2);
                 wkv4_update(st, k2, vb[i], w2);
             }
         }
+        off += kU * C;
     }
 }
 
+}  // namespace
+
 cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,
                             const float *u, float *y, cudaStream_t stream) {
-    constexpr int SEG = 16, U = 8;
-    const int groups = (C + 31) / 32;
-    wkv4_fwd_kernel<SEG, U><<<(unsigned)(B * groups), 32 * SEG, 0, stream>>>(B, T, C, k, v, w, u, y);
+    const int groups = (C + kCh - 1) / kCh;
+    wkv4_fwd_kernel<<<(unsigned)(B * groups), kCh * kSeg, 0, stream>>>(T, C, k, v, w, u, y);
     return cudaGetLastError();
 }
 
