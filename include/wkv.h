@@ -150,6 +150,17 @@ int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, cons
              float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes,
              wkv_stream_t stream);
 
+/*
+ * wkv6_bwd_bf16 -- wkv6_bwd with bfloat16 r, k, v, w and dy (raw IEEE bf16 bit
+ * patterns, uint16_t) for bf16 training: the same gradients, computed in fp32
+ * from the bf16 values, with u and every gradient (dr, dk, dv, dw, du) in fp32.
+ * Same layouts, workspace (wkv6_bwd_workspace_bytes) and errors as wkv6_bwd.
+ */
+int wkv6_bwd_bf16(int B, int T, int C, int H, int bidirectional, const uint16_t *r, const uint16_t *k,
+                  const uint16_t *v, const uint16_t *w, const float *u, const uint16_t *dy, float *dr,
+                  float *dk, float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes,
+                  wkv_stream_t stream);
+
 /* Scratch bytes wkv6_bwd needs for these sizes (B*C floats of per-batch du partials). */
 size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional);
 

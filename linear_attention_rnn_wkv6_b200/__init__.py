@@ -18,7 +18,7 @@ import os
 __all__ = [
     "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
-    "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "EXPORTED_SYMBOLS", "HEAD_SIZE",
+    "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "EXPORTED_SYMBOLS", "HEAD_SIZE",
 ]
 
 HEAD_SIZE = 64
@@ -29,7 +29,7 @@ _LIB = None
 EXPORTED_SYMBOLS = (
     "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
     "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc", "wkv6_fwd_state",
-    "wkv6_decode",
+    "wkv6_decode", "wkv6_bwd_bf16",
 )
 
 _I = ctypes.c_int
@@ -49,6 +49,7 @@ _SIGS = {
     "wkv6_bwd_noalloc": ([_I] * 5 + [_P] * 11 + [_P], _I),
     "wkv6_fwd_state": ([_I] * 4 + [_P] * 8 + [_P], _I),
     "wkv6_decode": ([_I] * 3 + [_P] * 7 + [_P], _I),
+    "wkv6_bwd_bf16": ([_I] * 5 + [_P] * 11 + [_P, _SZ, _P], _I),
 }
 
 
@@ -145,6 +146,15 @@ def wkv6_bwd(B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, w
     _check("wkv6_bwd", load().wkv6_bwd(B, T, C, H, int(bool(bidirectional)), _ptr(r), _ptr(k), _ptr(v), _ptr(w),
                                        _ptr(u), _ptr(dy), _ptr(dr), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du),
                                        _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def wkv6_bwd_bf16(B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, workspace, workspace_bytes,
+                  stream=None) -> None:
+    """wkv6_bwd with bf16 r, k, v, w, dy (bit patterns); u and all gradients fp32."""
+    _check("wkv6_bwd_bf16", load().wkv6_bwd_bf16(B, T, C, H, int(bool(bidirectional)), _ptr(r), _ptr(k), _ptr(v),
+                                                 _ptr(w), _ptr(u), _ptr(dy), _ptr(dr), _ptr(dk), _ptr(dv),
+                                                 _ptr(dw), _ptr(du), _ptr(workspace), int(workspace_bytes),
+                                                 _stream(stream)))
 
 
 def wkv6_bwd_noalloc(B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, stream=None) -> None:

@@ -32,9 +32,9 @@ namespace wkv {
 
 constexpr float kThetaB = 40.0f;
 
-template <int TC>
+template <typename Tin, int TC>
 struct BwdSmem {
-    alignas(128) float raw[2][5][TC][kHead];   // r, k, w, v, dy (TMA landing, 2 stages)
+    alignas(128) Tin raw[2][5][TC][kHead];     // r, k, w, v, dy (TMA landing, 2 stages; fp32 or bf16)
     float Ap[TC][kHead];          // exp(L_p)
     float ks[TC][kHead];          // k * exp(-L_{p+1})   (k on renorm steps)
     float rs[TC][kHead];          // r * exp(-L_{p+1})   (r on renorm steps)
@@ -53,9 +53,19 @@ struct BwdSmem {
 };
 
 // TMA writes its tiles at 128-byte aligned shared-memory addresses only.
-static_assert(offsetof(BwdSmem<kBwdTC>, raw) % 128 == 0 && offsetof(BwdSmem<kBwdTC>, part) % 128 == 0 &&
-                  (kBwdTC * kHead * sizeof(float)) % 128 == 0,
+using BwdSmemF32 = BwdSmem<float, kBwdTC>;
+using BwdSmemBF16 = BwdSmem<__nv_bfloat16, kBwdTC>;
+static_assert(offsetof(BwdSmemF32, raw) % 128 == 0 && offsetof(BwdSmemF32, part) % 128 == 0 &&
+                  offsetof(BwdSmemBF16, part) % 128 == 0 && (kBwdTC * kHead * sizeof(__nv_bfloat16)) % 128 == 0,
               "backward TMA destinations must be 128-byte aligned");
+
+// Four consecutive inputs as fp32 (one 16-byte load for fp32, 8 bytes for bf16).
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    const uint2 x = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xFFFF0000u), __uint_as_float(x.y << 16),
+                       __uint_as_float(x.y & 0xFFFF0000u));
+}
 
 enum { A_R = 0, A_K = 1, A_W = 2, A_V = 3, A_DY = 4 };
 
@@ -111,16 +121,16 @@ __device__ __forceinline__ void load_pairs(const float *x, int rowA, int rowB, f
     o[3] = make_float2(b.z, b.w);
 }
 
-template <int TC, bool BIDIR>
+template <typename Tin, int TC, bool BIDIR>
 __global__ void __launch_bounds__(128, 3)
 wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_v,
                 const __grid_constant__ CUtensorMap map_dy, const __grid_constant__ CUtensorMap map_dr,
                 const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
                 const __grid_constant__ CUtensorMap map_dw, BwdParams prm) {
-    using Smem = BwdSmem<TC>;
+    using Smem = BwdSmem<Tin, TC>;
     constexpr int NT = 128;
-    constexpr uint32_t kStageBytes = 5u * TC * kHead * sizeof(float);
+    constexpr uint32_t kStageBytes = 5u * TC * kHead * sizeof(Tin);
     constexpr uint32_t kPartBytes = 4u * TC * kHead * sizeof(float);
     extern __shared__ unsigned char smem_dyn[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~uintptr_t(127));
@@ -212,15 +222,15 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
 
         // ---- renorm flags ----
         int bad = 0;
-        for (int e = tid; e < TC * kHead; e += NT) bad |= !(fabsf(sm.raw[s][A_W][e / kHead][e % kHead]) <= kThetaB / TC);
+        for (int e = tid; e < TC * kHead; e += NT) bad |= !(fabsf(to_f32(sm.raw[s][A_W][e / kHead][e % kHead])) <= kThetaB / TC);
         const int any_bad = __syncthreads_or(bad);
         if (tid < 32) {
             uint32_t mask = 1u << (TC - 1);
             if (any_bad) {
                 for (int p = 0; p < TC - 1; ++p) {
                     const int row = dir > 0 ? p : TC - 1 - p;
-                    const bool bb = !(fabsf(sm.raw[s][A_W][row][lane]) <= kThetaB / TC) ||
-                                    !(fabsf(sm.raw[s][A_W][row][lane + 32]) <= kThetaB / TC);
+                    const bool bb = !(fabsf(to_f32(sm.raw[s][A_W][row][lane])) <= kThetaB / TC) ||
+                                    !(fabsf(to_f32(sm.raw[s][A_W][row][lane + 32])) <= kThetaB / TC);
                     if (__any_sync(0xffffffffu, bb)) mask |= 1u << p;
                 }
             }
@@ -238,15 +248,15 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             float L = 0.f;
             for (int p = 0; p < p0; ++p) {
                 const int row = dir > 0 ? p : TC - 1 - p;
-                L = ((rmask >> p) & 1u) ? 0.f : L + sm.raw[s][A_W][row][i];
+                L = ((rmask >> p) & 1u) ? 0.f : L + to_f32(sm.raw[s][A_W][row][i]);
             }
             float ew[TH], rr[TH], kk[TH];
 #pragma unroll
             for (int e = 0; e < TH; ++e) {
                 const int p = p0 + e, row = dir > 0 ? p : TC - 1 - p;
-                ew[e] = sm.raw[s][A_W][row][i];
-                rr[e] = sm.raw[s][A_R][row][i];
-                kk[e] = sm.raw[s][A_K][row][i];
+                ew[e] = to_f32(sm.raw[s][A_W][row][i]);
+                rr[e] = to_f32(sm.raw[s][A_R][row][i]);
+                kk[e] = to_f32(sm.raw[s][A_K][row][i]);
             }
 #pragma unroll
             for (int e = 0; e < TH; ++e) {
@@ -269,10 +279,10 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         }
         for (int p = warp; p < TC; p += 4) {
             const int row = dir > 0 ? p : TC - 1 - p;
-            float a = sm.raw[s][A_V][row][lane] * sm.raw[s][A_DY][row][lane] +
-                      sm.raw[s][A_V][row][lane + 32] * sm.raw[s][A_DY][row][lane + 32];
-            float c = sm.raw[s][A_R][row][lane] * sm.u[lane] * sm.raw[s][A_K][row][lane] +
-                      sm.raw[s][A_R][row][lane + 32] * sm.u[lane + 32] * sm.raw[s][A_K][row][lane + 32];
+            float a = to_f32(sm.raw[s][A_V][row][lane]) * to_f32(sm.raw[s][A_DY][row][lane]) +
+                      to_f32(sm.raw[s][A_V][row][lane + 32]) * to_f32(sm.raw[s][A_DY][row][lane + 32]);
+            float c = to_f32(sm.raw[s][A_R][row][lane]) * sm.u[lane] * to_f32(sm.raw[s][A_K][row][lane]) +
+                      to_f32(sm.raw[s][A_R][row][lane + 32]) * sm.u[lane + 32] * to_f32(sm.raw[s][A_K][row][lane + 32]);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -292,8 +302,8 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         // multiply-adds; the per-row operands come as pairs from the float4 loads.
         for (int p = 0; p < TC; ++p) {
             const int prow = dir > 0 ? p : TC - 1 - p;
-            const float4 va = *reinterpret_cast<const float4 *>(&sm.raw[s][A_V][prow][jc]);
-            const float4 ga = *reinterpret_cast<const float4 *>(&sm.raw[s][A_DY][prow][jc]);
+            const float4 va = load4(&sm.raw[s][A_V][prow][jc]);
+            const float4 ga = load4(&sm.raw[s][A_DY][prow][jc]);
             const float2 v2[4] = {make_float2(va.x, va.x), make_float2(va.y, va.y), make_float2(va.z, va.z),
                                   make_float2(va.w, va.w)};
             const float2 g2[4] = {make_float2(ga.x, ga.x), make_float2(ga.y, ga.y), make_float2(ga.z, ga.z),
@@ -386,12 +396,12 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             const float dks = hasG ? A * (sm.pk[p][0][i] + sm.pk[p][1][i] + sm.pk[p][2][i] + sm.pk[p][3][i]) : 0.f;
             const float dvv = hasG ? sm.dvs[p][i] : 0.f;
             const int row = dir > 0 ? p : TC - 1 - p;
-            const float rr = sm.raw[s][A_R][row][i], kk = sm.raw[s][A_K][row][i];
+            const float rr = to_f32(sm.raw[s][A_R][row][i]), kk = to_f32(sm.raw[s][A_K][row][i]);
             if (sweepA) {
                 const float vdy = sm.vdy[p];
                 prm.dr[o] = fmaf(sm.u[i] * kk, vdy, drs);
                 prm.dk[o] = fmaf(sm.u[i] * rr, vdy, dks);
-                prm.dv[o] = fmaf(sm.ruk[p], sm.raw[s][A_DY][row][i], dvv);
+                prm.dv[o] = fmaf(sm.ruk[p], to_f32(sm.raw[s][A_DY][row][i]), dvv);
                 prm.dw[o] = fmaf(rr, drs, kk * dks);           // z_t, parked in dw
             } else {
                 prm.dr[o] = sm.part[s][0][row][i] + drs;
@@ -408,7 +418,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                 for (int p = 0; p < TC; ++p) {
                     const int t = tl + p;
                     if (t < 0 || t >= T) continue;
-                    du_acc = fmaf(sm.raw[s][A_R][p][tid] * sm.raw[s][A_K][p][tid], sm.vdy[p], du_acc);
+                    du_acc = fmaf(to_f32(sm.raw[s][A_R][p][tid]) * to_f32(sm.raw[s][A_K][p][tid]), sm.vdy[p], du_acc);
                 }
             }
         } else {
@@ -446,10 +456,10 @@ __global__ void wkv6_du_reduce_kernel(int B, int C, const float *__restrict__ pa
     du[c] = acc;
 }
 
-template <int TC, bool BIDIR>
+template <typename Tin, int TC, bool BIDIR>
 static cudaError_t launch_bwd(const CUtensorMap *maps, const BwdParams &prm, cudaStream_t stream) {
-    auto kern = wkv6_bwd_kernel<TC, BIDIR>;
-    const size_t smem = sizeof(BwdSmem<TC>) + 128;
+    auto kern = wkv6_bwd_kernel<Tin, TC, BIDIR>;
+    const size_t smem = sizeof(BwdSmem<Tin, TC>) + 128;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(prm.B * prm.H), 128, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
@@ -459,10 +469,13 @@ static cudaError_t launch_bwd(const CUtensorMap *maps, const BwdParams &prm, cud
     return cudaSuccess;
 }
 
-cudaError_t wkv6_bwd_launch(bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
+cudaError_t wkv6_bwd_launch(bool bf16, bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
                             cudaStream_t stream) {
     constexpr int TC = kBwdTC;
-    cudaError_t e = bidir ? launch_bwd<TC, true>(maps, prm, stream) : launch_bwd<TC, false>(maps, prm, stream);
+    using BF = __nv_bfloat16;
+    cudaError_t e = bf16 ? (bidir ? launch_bwd<BF, TC, true>(maps, prm, stream) : launch_bwd<BF, TC, false>(maps, prm, stream))
+                         : (bidir ? launch_bwd<float, TC, true>(maps, prm, stream)
+                                  : launch_bwd<float, TC, false>(maps, prm, stream));
     if (e != cudaSuccess) return e;
     wkv6_du_reduce_kernel<<<(prm.C + 255) / 256, 256, 0, stream>>>(prm.B, prm.C, prm.du_part, du);
     return cudaGetLastError();

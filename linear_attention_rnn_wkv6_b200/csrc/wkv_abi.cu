@@ -87,13 +87,34 @@ int check_wkv6(int B, int T, int C, int H, std::initializer_list<const void *> p
 
 // Tensor maps of the backward: inputs r, k, w, v, dy, then the outputs dr, dk,
 // dv, dw (the second sweep reads back what the first sweep stored there).
-bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], int B, int T, int C, const float *r, const float *k,
-                   const float *w, const float *v, const float *dy, const float *dr, const float *dk,
+bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], bool bf16, int B, int T, int C, const void *r, const void *k,
+                   const void *w, const void *v, const void *dy, const float *dr, const float *dk,
                    const float *dv, const float *dw) {
     const void *src[kBwdMaps] = {r, k, w, v, dy, dr, dk, dv, dw};
     for (int i = 0; i < kBwdMaps; ++i)
-        if (!make_map(&maps[i], src[i], false, B, T, C, kHead, kBwdTC)) return false;
+        if (!make_map(&maps[i], src[i], bf16 && i < 5, B, T, C, kHead, kBwdTC)) return false;
     return true;
+}
+
+// Shared by wkv6_bwd and wkv6_bwd_bf16 (inputs fp32 or bf16, gradients fp32).
+int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const void *r, const void *k,
+               const void *v, const void *w, const float *u, const void *dy, float *dr, float *dk, float *dv,
+               float *dw, float *du, void *workspace, size_t workspace_bytes, wkv_stream_t stream) {
+    int st = check_wkv6(B, T, C, H, {r, k, v, w, u, dy, dr, dk, dv, dw, du});
+    if (st != WKV_OK) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (B == 0 || T == 0) {
+        if ((st = check_device()) != WKV_OK) return st;
+        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    }
+    const size_t need = (size_t)B * (size_t)C * sizeof(float);
+    if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WKV_ERR_ALIGN;
+    if ((st = check_device()) != WKV_OK) return st;
+    CUtensorMap maps[kBwdMaps];
+    if (!make_bwd_maps(maps, bf16, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
+    BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, static_cast<float *>(workspace)};
+    return wkv6_bwd_launch(bf16, bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
 // Algorithm of the bf16 causal forward: the chunked tensor-core kernel (default)
@@ -208,21 +229,15 @@ size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional) {
 int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, const float *k, const float *v,
              const float *w, const float *u, const float *dy, float *dr, float *dk, float *dv, float *dw,
              float *du, void *workspace, size_t workspace_bytes, wkv_stream_t stream) {
-    int st = check_wkv6(B, T, C, H, {r, k, v, w, u, dy, dr, dk, dv, dw, du});
-    if (st != WKV_OK) return st;
-    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (B == 0 || T == 0) {
-        if ((st = check_device()) != WKV_OK) return st;
-        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
-    }
-    const size_t need = wkv6_bwd_workspace_bytes(B, T, C, H, bidirectional);
-    if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return WKV_ERR_ALIGN;
-    if ((st = check_device()) != WKV_OK) return st;
-    CUtensorMap maps[kBwdMaps];
-    if (!make_bwd_maps(maps, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
-    BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, static_cast<float *>(workspace)};
-    return wkv6_bwd_launch(bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return bwd_common(false, B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, workspace,
+                      workspace_bytes, stream);
+}
+
+int wkv6_bwd_bf16(int B, int T, int C, int H, int bidirectional, const uint16_t *r, const uint16_t *k,
+                  const uint16_t *v, const uint16_t *w, const float *u, const uint16_t *dy, float *dr, float *dk,
+                  float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes, wkv_stream_t stream) {
+    return bwd_common(true, B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, workspace,
+                      workspace_bytes, stream);
 }
 
 int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u, float *y,
@@ -314,9 +329,9 @@ extern "C" int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, c
     float *scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != WKV_OK) return st;
     CUtensorMap maps[kBwdMaps];
-    if (!make_bwd_maps(maps, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
+    if (!make_bwd_maps(maps, false, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
     // Every per-batch partial the reduction reads is written first by the
     // backward kernel, so nothing left in the array by an earlier call leaks in.
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, scratch};
-    return wkv6_bwd_launch(bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return wkv6_bwd_launch(false, bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }

@@ -35,7 +35,8 @@ cudaError_t wkv6_decode_launch(int B, int C, int H, const float *r, const float 
                                const float *w, const float *u, float *state, float *y, cudaStream_t stream);
 // maps: kBwdMaps tensor maps, in the order r, k, w, v, dy, dr, dk, dv, dw
 constexpr int kBwdMaps = 9;
-cudaError_t wkv6_bwd_launch(bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
+// bf16: r, k, w, v, dy are bf16 (their maps describe bf16 tensors); gradients stay fp32
+cudaError_t wkv6_bwd_launch(bool bf16, bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
                             cudaStream_t stream);
 cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,
                             const float *u, float *y, cudaStream_t stream);

@@ -234,6 +234,8 @@ WORKLOADS = {
     "wkv6_causal_bf16_b8t4096h32": ("wkv6_fwd_bf16", dict(B=8, T=4096, H=32, wraw_lo=-8.0, dtype="bf16")),
     # bidirectional RWKV-6 backward, fp32
     "wkv6_bidir_bwd_f32_b32t196h12": ("wkv6_bwd_bidir", dict(B=32, T=196, H=12, with_dy=True)),
+    # bidirectional RWKV-6 backward with bf16 inputs (fp32 gradients)
+    "wkv6_bidir_bwd_bf16_b32t196h12": ("wkv6_bwd_bidir", dict(B=32, T=196, H=12, with_dy=True, dtype="bf16")),
     # one recurrent decode step for 512 sequences of the long-text head layout (state from make_state)
     "wkv6_decode_f32_b512h32": ("wkv6_decode", dict(B=512, T=1, H=32)),
 }

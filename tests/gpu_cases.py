@@ -87,3 +87,19 @@ def sample_units(B: int, H: int, n: int):
     start = max(1, total // max(n, 1))
     stride = next(s for s in range(start, start + total + 1) if math.gcd(s, total) == 1)
     return [divmod((i * stride + 3) % total, H) for i in range(n)]
+
+
+def run_wkv6_bwd_bf16(x: synth.Wkv6Inputs, bidir: bool):
+    """wkv6_bwd_bf16 on bf16 inputs (x.dtype == "bf16"); dy is rounded to bf16 the same way.
+    Returns the fp32 gradients and the float64 dy the oracle must see."""
+    t = torch()
+    assert x.dtype == "bf16"
+    dy_bits = synth.to_bf16_bits(x.dy)
+    r, k, v, w, dy = (dev(a) for a in (x.r, x.k, x.v, x.w, dy_bits))
+    u = dev(x.u)
+    outs = [empty_nan((x.B, x.T, x.C)) for _ in range(4)] + [empty_nan((x.C,))]
+    nbytes = wkv.wkv6_bwd_workspace_bytes(x.B, x.T, x.C, x.H, bidir)
+    ws = t.empty(max(nbytes, 16), dtype=t.uint8, device="cuda")
+    wkv.wkv6_bwd_bf16(x.B, x.T, x.C, x.H, bidir, r, k, v, w, u, dy, *outs, ws, nbytes)
+    assert wkv.wkv_take_device_faults() == 0
+    return tuple(o.cpu().numpy() for o in outs), synth.bf16_bits_to_f32(dy_bits).astype(np.float64)

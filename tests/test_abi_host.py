@@ -94,6 +94,18 @@ def test_wkv6_backward_argument_errors(lib):
     assert lib.wkv6_bwd(2, 8, 128, 2, 0, *q, FAKE, ws, None) == WKV_ERR_ALIGN
 
 
+def test_wkv6_bwd_bf16_argument_errors(lib):
+    p = [FAKE + 256 * i for i in range(11)]
+    ws = wkv.wkv6_bwd_workspace_bytes(2, 8, 128, 2, 1)
+    f = lib.wkv6_bwd_bf16
+    assert f(-1, 8, 128, 2, 1, *p, FAKE, ws, None) == WKV_ERR_ARG
+    assert f(2, 8, 128, 4, 1, *p, FAKE, ws, None) == WKV_ERR_HEADSIZE
+    assert f(2, 8, 128, 2, 1, *p, None, ws, None) == WKV_ERR_WORKSPACE
+    q = list(p)
+    q[5] += 8                                                  # dy misaligned
+    assert f(2, 8, 128, 2, 1, *q, FAKE, ws, None) == WKV_ERR_ALIGN
+
+
 def test_wkv6_state_argument_errors(lib):
     f = lib.wkv6_fwd_state
     p = [FAKE + 256 * i for i in range(5)]                     # r, k, v, w, u

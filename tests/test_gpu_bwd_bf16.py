@@ -1,0 +1,70 @@
+"""GPU parity of wkv6_bwd_bf16 (bf16 r, k, v, w, dy; fp32 u and gradients) against
+the oracle's backward on the same bf16-rounded input values.
+
+The kernel computes in fp32 from exactly the values the oracle sees, so the fp32
+gradient tolerance applies (relative L2 per tensor).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from linear_attention_rnn_wkv6_b200 import synth
+from tests import gpu_cases as gc
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_attention_rnn_wkv6_b200 import build
+    build.build()
+
+
+def _check(x, bidir, got, dy64, H):
+    r, k, v, w, u = gc.f64(x)
+    ref = oracle.wkv6_bwd(r, k, v, w, u, dy64, H=H, bidirectional=bidir)
+    for name, g, e in zip(("dr", "dk", "dv", "dw", "du"), got, ref):
+        assert np.all(np.isfinite(g)), name
+        if name == "dw" and x.T <= 2:
+            assert np.max(np.abs(g)) <= 1e-6, name
+            continue
+        err = oracle.rel_l2(g, e)
+        assert err <= gc.TOL_F32_GRAD, (name, err)
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (2, 15, 2), (1, 16, 1), (2, 17, 1), (1, 50, 3), (2, 96, 2)])
+@pytest.mark.parametrize("bidir", [False, True])
+def test_bwd_bf16_small(B, T, H, bidir):
+    x = synth.make_wkv6(B, T, H, seed=400 + T, with_dy=True, dtype="bf16")
+    got, dy64 = gc.run_wkv6_bwd_bf16(x, bidir)
+    _check(x, bidir, got, dy64, H)
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_bwd_bf16_strong_decay(bidir):
+    x = synth.make_wkv6(2, 45, 2, seed=410, with_dy=True, dtype="bf16")
+    w = -np.exp(np.random.default_rng(411).uniform(-2.0, 3.5, x.w.shape)).astype(np.float32)
+    w[:, 10, :] = -np.inf
+    x.w = synth.to_bf16_bits(w)
+    got, dy64 = gc.run_wkv6_bwd_bf16(x, bidir)
+    _check(x, bidir, got, dy64, 2)
+
+
+def test_bwd_bf16_workload_sampled():
+    """The bidirectional backward workload's shape (B32 T196 H12) in bf16, on sampled (b, h) units."""
+    x = synth.make_wkv6(32, 196, 12, seed=0, with_dy=True, dtype="bf16")
+    (dr, dk, dv, dw, du), dy64 = gc.run_wkv6_bwd_bf16(x, True)
+    got = {n: [] for n in ("dr", "dk", "dv", "dw")}
+    ref = {n: [] for n in ("dr", "dk", "dv", "dw")}
+    for b, h in gc.sample_units(x.B, x.H, 16):
+        (r, k, v, w, u), _, sl = gc.unit_slice(x, b, h)
+        e = oracle.wkv6_bwd(r, k, v, w, u, dy64[b:b + 1, :, sl], H=1, bidirectional=True)
+        for n, gg, ee in zip(("dr", "dk", "dv", "dw"), (dr, dk, dv, dw), e[:4]):
+            got[n].append(gg[b, :, sl])
+            ref[n].append(ee[0])
+    for n in got:
+        err = oracle.rel_l2(np.stack(got[n]), np.stack(ref[n]))
+        assert err <= gc.TOL_F32_GRAD, (n, err)
