@@ -45,7 +45,9 @@ def _configure(lib):
     lib.oracle_wkv6_fwd_state.argtypes = [I, I, I, I] + [_DP] * 8
     lib.oracle_wkv6_bwd.argtypes = [I, I, I, I, I] + [_DP] * 11
     lib.oracle_wkv4_fwd.argtypes = [I, I, I] + [_DP] * 5
-    for f in (lib.oracle_wkv6_fwd, lib.oracle_wkv6_fwd_state, lib.oracle_wkv6_bwd, lib.oracle_wkv4_fwd):
+    lib.oracle_wkv4_bwd.argtypes = [I, I, I] + [_DP] * 9
+    for f in (lib.oracle_wkv6_fwd, lib.oracle_wkv6_fwd_state, lib.oracle_wkv6_bwd, lib.oracle_wkv4_fwd,
+              lib.oracle_wkv4_bwd):
         f.restype = ctypes.c_int
     return lib
 
@@ -115,6 +117,22 @@ class Oracle:
             raise ValueError(f"oracle_wkv4_fwd failed ({rc})")
         return y
 
+    def wkv4_bwd(self, k, v, w, u, dy):
+        """RWKV-4 backward -> (dk, dv [B,T,C], dw, du [C] summed over B and T)."""
+        k, v, w, u, dy = map(_d, (k, v, w, u, dy))
+        B, T, C = k.shape
+        dk = np.zeros((B, T, C), dtype=np.float64)
+        dv = np.zeros((B, T, C), dtype=np.float64)
+        dw = np.zeros(C, dtype=np.float64)
+        du = np.zeros(C, dtype=np.float64)
+        rc = self._lib.oracle_wkv4_bwd(B, T, C, _p(k), _p(v), _p(w), _p(u), _p(dy), _p(dk), _p(dv), _p(dw),
+                                       _p(du))
+        if rc != 0:
+            raise ValueError(f"oracle_wkv4_bwd failed ({rc})")
+        return dk, dv, dw, du
+
+
+
 
 def _default() -> Oracle:
     global _lib
@@ -137,6 +155,10 @@ def wkv6_bwd(r, k, v, w, u, dy, H: int, bidirectional: bool = False):
 
 def wkv4_fwd(k, v, w, u) -> np.ndarray:
     return _default().wkv4_fwd(k, v, w, u)
+
+
+def wkv4_bwd(k, v, w, u, dy):
+    return _default().wkv4_bwd(k, v, w, u, dy)
 
 
 def source() -> str:

@@ -298,3 +298,58 @@ int oracle_wkv4_fwd(int B, int T, int C, const double *k, const double *v, const
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-4 backward: gradients of L = sum_t dy_t . y_t for oracle_wkv4_fwd,     */
+/* written from the ratio-of-sums definition (RWKV Architecture page, The     */
+/* Fundamental Mathematical Duality: WKV_t = N_t / D_t with                   */
+/*   N_t = sum_{s<t} E_ts v_s + E_tt v_t,  D_t = sum_{s<t} E_ts + E_tt,        */
+/*   E_ts = e^{k_s - (t-1-s) w} for s < t,  E_tt = e^{u + k_t}).              */
+/* Differentiating the ratio, with g_t = dy_t / D_t:                          */
+/*   dv_s += g_t E_ts,   dk_s += g_t E_ts (v_s - y_t)         (s <= t)         */
+/*   du   += g_t E_tt (v_t - y_t)                                             */
+/*   dw   -= g_t (t-1-s) E_ts (v_s - y_t)                     (s < t)          */
+/* Every E_ts and D_t of step t is scaled by e^{-m_t}, m_t the largest exponent */
+/* of the step, which cancels in g_t E_ts (the log-space shift of the forward). */
+/* O(T^2) per channel: a plain evaluation of the definition.                  */
+/*   dk, dv : [B][T][C];  dw, du : [C], summed over B and T.                  */
+/* ------------------------------------------------------------------------ */
+int oracle_wkv4_bwd(int B, int T, int C, const double *k, const double *v, const double *w,
+                    const double *u, const double *dy, double *dk, double *dv, double *dw, double *du)
+{
+    if (B < 0 || T < 0 || C < 0) return -1;
+    memset(dk, 0, sizeof(double) * (size_t)B * T * C);
+    memset(dv, 0, sizeof(double) * (size_t)B * T * C);
+    memset(dw, 0, sizeof(double) * (size_t)C);
+    memset(du, 0, sizeof(double) * (size_t)C);
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < C; ++c)
+            for (int t = 0; t < T; ++t) {
+                const double kt = k[IDX(b, t, c)], vt = v[IDX(b, t, c)];
+                /* the step's largest exponent */
+                double m = u[c] + kt;
+                for (int s = 0; s < t; ++s) m = fmax(m, k[IDX(b, s, c)] - (t - 1 - s) * w[c]);
+                /* N_t, D_t (scaled by e^{-m}) and y_t */
+                const double ett = exp(u[c] + kt - m);
+                double D = ett, N = ett * vt;
+                for (int s = 0; s < t; ++s) {
+                    const double e = exp(k[IDX(b, s, c)] - (t - 1 - s) * w[c] - m);
+                    D += e;
+                    N += e * v[IDX(b, s, c)];
+                }
+                const double yt = N / D, g = dy[IDX(b, t, c)] / D;
+                /* the bonus term s = t */
+                dv[IDX(b, t, c)] += g * ett;
+                dk[IDX(b, t, c)] += g * ett * (vt - yt);
+                du[c] += g * ett * (vt - yt);
+                /* the decayed past s < t */
+                for (int s = 0; s < t; ++s) {
+                    const double vs = v[IDX(b, s, c)];
+                    const double e = exp(k[IDX(b, s, c)] - (t - 1 - s) * w[c] - m);
+                    dv[IDX(b, s, c)] += g * e;
+                    dk[IDX(b, s, c)] += g * e * (vs - yt);
+                    dw[c] -= (t - 1 - s) * g * e * (vs - yt);
+                }
+            }
+    return 0;
+}

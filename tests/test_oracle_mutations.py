@@ -43,6 +43,12 @@ MUTATIONS = [
     ("state_out_is_initial", "if (sT) memcpy(sT + off, S, sizeof(double) * NN);",
      "if (sT) memcpy(sT + off, s0 ? s0 + off : S, sizeof(double) * NN);", 0,
      [lambda o: pins.test_wkv6_state_matches_pair_form(o, 2, 3, 1, 4), lambda o: pins.test_wkv6_state_split_equals_whole(o, 13)]),
+    ("wkv4_bwd_dk_drops_y", "dk[IDX(b, s, c)] += g * e * (vs - yt);", "dk[IDX(b, s, c)] += g * e * vs;", 0,
+     [lambda o: pins.test_wkv4_backward_finite_differences(o, 2, 5, 3), pins.test_wkv4_backward_invariants]),
+    ("wkv4_bwd_dw_weight", "dw[c] -= (t - 1 - s) * g * e * (vs - yt);", "dw[c] -= (t - s) * g * e * (vs - yt);", 0,
+     [lambda o: pins.test_wkv4_backward_finite_differences(o, 2, 5, 3)]),
+    ("wkv4_bwd_bonus_dv_missing", "dv[IDX(b, t, c)] += g * ett;", "dv[IDX(b, t, c)] += 0.0 * ett;", 0,
+     [pins.test_wkv4_backward_invariants]),
     ("wkv4_decay_sign", "e1 = exp(p - w[c] - q);", "e1 = exp(p + w[c] - q);", 0,
      [pins.test_wkv4_geometric_closed_form, pins.test_golden_wkv4_forward]),
     ("wkv4_missing_bonus", "e2 = exp(u[c] + kt - q);", "e2 = exp(kt - q);", 0,

@@ -341,6 +341,68 @@ def test_wkv4_large_keys_stay_finite(oracle_mod):
     np.testing.assert_allclose(oracle_mod.wkv4_fwd(k2, v, w, u), y, rtol=1e-9, atol=1e-9)
 
 
+# ---------------------------------------------------------------- RWKV-4 backward
+
+def _wkv4_loss(oracle_mod, k, v, w, u, dy):
+    return float(np.sum(dy * oracle_mod.wkv4_fwd(k, v, w, u)))
+
+
+@pytest.mark.parametrize("B,T,C", [(1, 1, 2), (2, 5, 3), (1, 9, 2)])
+def test_wkv4_backward_finite_differences(oracle_mod, B, T, C):
+    """Central differences of the forward oracle (L = sum dy * y) reproduce every gradient."""
+    k, v, w, u = _wkv4_case(B, T, C, seed=500 + T)
+    dy = _rng(501 + T).normal(0, 1, (B, T, C))
+    dk, dv, dw, du = oracle_mod.wkv4_bwd(k, v, w, u, dy)
+    h = 1e-6
+
+    def fd(arr, idx):
+        a1, a2 = arr.copy(), arr.copy()
+        a1[idx] += h
+        a2[idx] -= h
+        return a1, a2
+
+    for name, grad, pos in (("dk", dk, 0), ("dv", dv, 1)):
+        for idx in np.ndindex(grad.shape):
+            args1, args2 = [k, v, w, u], [k, v, w, u]
+            args1[pos], args2[pos] = fd([k, v][pos], idx)
+            num = (_wkv4_loss(oracle_mod, *args1, dy) - _wkv4_loss(oracle_mod, *args2, dy)) / (2 * h)
+            assert abs(num - grad[idx]) <= 1e-6 * max(1.0, abs(num)), (name, idx, num, grad[idx])
+    for name, grad, pos in (("dw", dw, 2), ("du", du, 3)):
+        for c in range(C):
+            args1, args2 = [k, v, w, u], [k, v, w, u]
+            args1[pos], args2[pos] = fd([w, u][pos - 2], (c,))
+            num = (_wkv4_loss(oracle_mod, *args1, dy) - _wkv4_loss(oracle_mod, *args2, dy)) / (2 * h)
+            assert abs(num - grad[c]) <= 1e-6 * max(1.0, abs(num)), (name, c, num, grad[c])
+
+
+def test_wkv4_backward_invariants(oracle_mod):
+    """y is unchanged by a common shift of all k (so dk sums to 0 per sequence) and is
+    homogeneous of degree 1 in v (so <v, dv> = <dy, y> per sequence); T = 1 gives y = v."""
+    B, T, C = 2, 17, 4
+    k, v, w, u = _wkv4_case(B, T, C, seed=520)
+    dy = _rng(521).normal(0, 1, (B, T, C))
+    dk, dv, dw, du = oracle_mod.wkv4_bwd(k, v, w, u, dy)
+    y = oracle_mod.wkv4_fwd(k, v, w, u)
+    assert np.max(np.abs(dk.sum(axis=1))) <= 1e-12 * max(1.0, np.max(np.abs(dk)))
+    np.testing.assert_allclose(np.sum(v * dv, axis=1), np.sum(dy * y, axis=1), rtol=1e-12, atol=1e-12)
+    k1, v1, w1, u1 = _wkv4_case(2, 1, 3, seed=522)
+    dy1 = _rng(523).normal(0, 1, (2, 1, 3))
+    dk1, dv1, dw1, du1 = oracle_mod.wkv4_bwd(k1, v1, w1, u1, dy1)
+    assert np.allclose(dv1, dy1, rtol=0, atol=1e-15) and not np.any(dk1) and not np.any(dw1) and not np.any(du1)
+
+
+def test_wkv4_backward_large_keys_stay_finite(oracle_mod):
+    """k ~ N(0, 30^2): every exponent is shifted by the step's largest one, so nothing overflows;
+    the invariants still hold."""
+    k, v, w, u = _wkv4_case(1, 40, 3, seed=530, kstd=30.0)
+    dy = _rng(531).normal(0, 1, k.shape)
+    dk, dv, dw, du = oracle_mod.wkv4_bwd(k, v, w, u, dy)
+    for g in (dk, dv, dw, du):
+        assert np.all(np.isfinite(g))
+    y = oracle_mod.wkv4_fwd(k, v, w, u)
+    np.testing.assert_allclose(np.sum(v * dv, axis=1), np.sum(dy * y, axis=1), rtol=1e-10, atol=1e-10)
+
+
 # ---------------------------------------------------------------- planted mistakes are caught
 
 def test_pins_catch_a_planted_decay_index_error():
