@@ -37,7 +37,7 @@ UNIT = "tokens/s"
 WORKLOAD_NAME = ("wkv-hot-path step: wkv4_fwd B8xT1024xC768 f32 + wkv6_bidir_fwd B32xT196xH12 f32 + "
                  "wkv6_fwd_bf16 B8xT4096xH32 + wkv6_bwd(bidir) B32xT196xH12 f32, N=64")
 # Workloads outside the step, measured on their own with --only.
-EXTRA_WORKLOADS = ["wkv6_decode_f32_b512h32", "wkv6_bidir_bwd_bf16_b32t196h12"]
+EXTRA_WORKLOADS = ["wkv6_decode_f32_b512h32", "wkv6_bidir_bwd_bf16_b32t196h12", "wkv4_bwd_f32_b8t1024c768"]
 STEP_WORKLOADS = ["wkv4_f32_b8t1024c768", "wkv6_bidir_f32_b32t196h12", "wkv6_causal_bf16_b8t4096h32",
                   "wkv6_bidir_bwd_f32_b32t196h12"]
 N = 64
@@ -59,16 +59,20 @@ ALG = {
     "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="alu"),
     "wkv6_bidir_bwd_bf16_b32t196h12": dict(bytes_per_unit=5 * N * 2 + 4 * N * 4, flops_per_unit=28 * N * N,
                                            bound="alu"),
+    # RWKV-4 backward: k, v, dy in and dk, dv out per (token, channel)
+    "wkv4_bwd_f32_b8t1024c768": dict(bytes_per_unit=5 * 4, flops_per_unit=40, bound="hbm"),
     # decode: the state is read and written once per step (2 N^2 floats) next to 5 N floats of token data
     "wkv6_decode_f32_b512h32": dict(bytes_per_unit=2 * N * N * 4 + 5 * N * 4, flops_per_unit=5 * N * N,
                                     bound="hbm"),
 }
 ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
          "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd",
-         "wkv6_decode_f32_b512h32": "wkv6_decode", "wkv6_bidir_bwd_bf16_b32t196h12": "wkv6_bwd_bf16"}
+         "wkv6_decode_f32_b512h32": "wkv6_decode", "wkv6_bidir_bwd_bf16_b32t196h12": "wkv6_bwd_bf16",
+         "wkv4_bwd_f32_b8t1024c768": "wkv4_bwd"}
 LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
             "wkv6_bidir_bwd_f32_b32t196h12": 2,   # the backward adds a deterministic du reduction
-            "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 2}
+            "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 2,
+            "wkv4_bwd_f32_b8t1024c768": 2}
 
 
 def units_of(name: str, x) -> int:
@@ -229,16 +233,24 @@ class DeviceWorkload:
             return torch.from_numpy(a).cuda()
 
         self.host_inputs = {}
-        names = ("k", "v", "w", "u") if self.kind == "wkv4_fwd" else ("r", "k", "v", "w", "u") + (
-            ("dy",) if self.kind == "wkv6_bwd_bidir" else ())
+        if self.kind.startswith("wkv4"):
+            names = ("k", "v", "w", "u") + (("dy",) if self.kind == "wkv4_bwd" else ())
+        else:
+            names = ("r", "k", "v", "w", "u") + (("dy",) if self.kind == "wkv6_bwd_bidir" else ())
         self.inputs = {n: dev(getattr(x, n)) for n in names}
-        if x.dtype == "bf16" and "dy" in names:
+        if getattr(x, "dtype", "f32") == "bf16" and "dy" in names:
             self.inputs["dy"] = dev(synth.to_bf16_bits(x.dy))   # the bf16 backward takes dy in bf16 too
         shape = (x.B, x.T, x.C)
         if self.kind == "wkv6_bwd_bidir":
             self.outputs = [torch.empty(shape, device="cuda") for _ in range(4)] + [torch.empty(x.C, device="cuda")]
             import linear_attention_rnn_wkv6_b200 as wkv
             self.ws_bytes = wkv.wkv6_bwd_workspace_bytes(x.B, x.T, x.C, x.H, 1)
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        elif self.kind == "wkv4_bwd":
+            import linear_attention_rnn_wkv6_b200 as wkv
+            self.outputs = [torch.empty(shape, device="cuda") for _ in range(2)] + \
+                           [torch.empty(x.C, device="cuda") for _ in range(2)]
+            self.ws_bytes = wkv.wkv4_bwd_workspace_bytes(x.B, x.T, x.C)
             self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
         else:
             self.outputs = [torch.empty(shape, device="cuda")]
@@ -255,6 +267,8 @@ class DeviceWorkload:
         s = stream.cuda_stream
         if self.kind == "wkv4_fwd":
             wkv.wkv4_fwd(x.B, x.T, x.C, i["k"], i["v"], i["w"], i["u"], o[0], s)
+        elif self.kind == "wkv4_bwd":
+            wkv.wkv4_bwd(x.B, x.T, x.C, i["k"], i["v"], i["w"], i["u"], i["dy"], *o, self.ws, self.ws_bytes, s)
         elif self.kind == "wkv6_bidir_fwd":
             wkv.wkv6_bidir_fwd(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], o[0], s)
         elif self.kind == "wkv6_fwd_bf16":

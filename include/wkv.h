@@ -204,6 +204,27 @@ int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, const float 
 int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u,
              float *y, wkv_stream_t stream);
 
+/*
+ * wkv4_bwd -- gradients of L = sum(dy * y) for wkv4_fwd ("RWKV Architecture ...",
+ * The Fundamental Mathematical Duality: y_t = N_t / D_t, a ratio of decayed sums;
+ * its derivatives with respect to k_s, v_s, w and u).
+ *   k, v, dy   : [B,T,C] float inputs;  w (> 0), u : [C] float inputs
+ *   dk, dv     : [B,T,C] float outputs
+ *   dw, du     : [C] float outputs, summed over B and T in a fixed order
+ *                (bitwise reproducible run to run)
+ *   workspace  : device scratch of at least wkv4_bwd_workspace_bytes(B, T, C) bytes,
+ *                16-byte aligned, owned by the caller; content ignored on entry.
+ * dk and dv also serve as scratch during the call (they are fully written).
+ * Errors: WKV_ERR_ARG, WKV_ERR_ALIGN, WKV_ERR_WORKSPACE, WKV_ERR_TOO_LARGE
+ * (B*T*C >= 2^31), WKV_ERR_DEVICE, WKV_ERR_CUDA.  B == 0 or T == 0 zeroes dw, du.
+ */
+int wkv4_bwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u,
+             const float *dy, float *dk, float *dv, float *dw, float *du, void *workspace,
+             size_t workspace_bytes, wkv_stream_t stream);
+
+/* Scratch bytes wkv4_bwd needs: B*T*C floats (one per step) plus 2*B*C floats of partials. */
+size_t wkv4_bwd_workspace_bytes(int B, int T, int C);
+
 /* Static description of a status code (never NULL). */
 const char *wkv_status_string(int status);
 

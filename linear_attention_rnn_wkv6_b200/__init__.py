@@ -18,7 +18,8 @@ import os
 __all__ = [
     "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
-    "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "EXPORTED_SYMBOLS", "HEAD_SIZE",
+    "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
+    "EXPORTED_SYMBOLS", "HEAD_SIZE",
 ]
 
 HEAD_SIZE = 64
@@ -29,7 +30,7 @@ _LIB = None
 EXPORTED_SYMBOLS = (
     "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
     "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc", "wkv6_fwd_state",
-    "wkv6_decode", "wkv6_bwd_bf16",
+    "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
 )
 
 _I = ctypes.c_int
@@ -50,6 +51,8 @@ _SIGS = {
     "wkv6_fwd_state": ([_I] * 4 + [_P] * 8 + [_P], _I),
     "wkv6_decode": ([_I] * 3 + [_P] * 7 + [_P], _I),
     "wkv6_bwd_bf16": ([_I] * 5 + [_P] * 11 + [_P, _SZ, _P], _I),
+    "wkv4_bwd": ([_I] * 3 + [_P] * 9 + [_P, _SZ, _P], _I),
+    "wkv4_bwd_workspace_bytes": ([_I] * 3, _SZ),
 }
 
 
@@ -168,6 +171,16 @@ def wkv6_bwd_noalloc(B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, d
 def wkv4_fwd(B, T, C, k, v, w, u, y, stream=None) -> None:
     """RWKV-4 WKV forward (fp32)."""
     _check("wkv4_fwd", load().wkv4_fwd(B, T, C, _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(y), _stream(stream)))
+
+
+def wkv4_bwd_workspace_bytes(B, T, C) -> int:
+    return int(load().wkv4_bwd_workspace_bytes(B, T, C))
+
+
+def wkv4_bwd(B, T, C, k, v, w, u, dy, dk, dv, dw, du, workspace, workspace_bytes, stream=None) -> None:
+    """RWKV-4 WKV backward (fp32): dk, dv [B,T,C]; dw, du [C]."""
+    _check("wkv4_bwd", load().wkv4_bwd(B, T, C, _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(dy), _ptr(dk), _ptr(dv),
+                                       _ptr(dw), _ptr(du), _ptr(workspace), int(workspace_bytes), _stream(stream)))
 
 
 def wkv_status_string(status: int) -> str:

@@ -253,6 +253,35 @@ int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w
                : WKV_ERR_CUDA;
 }
 
+size_t wkv4_bwd_workspace_bytes(int B, int T, int C) {
+    if (B < 1 || T < 0 || C < 1) return 0;
+    return sizeof(float) * ((size_t)B * T * C + 2 * (size_t)B * C);
+}
+
+int wkv4_bwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u, const float *dy,
+             float *dk, float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes,
+             wkv_stream_t stream) {
+    if (B < 0 || T < 0 || C < 1 || !k || !v || !w || !u || !dy || !dk || !dv || !dw || !du) return WKV_ERR_ARG;
+    if ((long long)B * T * C >= (1ll << 31)) return WKV_ERR_TOO_LARGE;
+    for (const void *p : {(const void *)k, (const void *)v, (const void *)w, (const void *)u, (const void *)dy,
+                          (const void *)dk, (const void *)dv, (const void *)dw, (const void *)du})
+        if (!aligned16(p)) return WKV_ERR_ALIGN;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int st;
+    if (B == 0 || T == 0) {
+        if ((st = check_device()) != WKV_OK) return st;
+        if (cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)C, s) != cudaSuccess) return WKV_ERR_CUDA;
+        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    }
+    if (workspace == nullptr || workspace_bytes < wkv4_bwd_workspace_bytes(B, T, C)) return WKV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WKV_ERR_ALIGN;
+    if ((st = check_device()) != WKV_OK) return st;
+    return wkv4_bwd_launch(B, T, C, k, v, w, u, dy, dk, dv, dw, du, static_cast<float *>(workspace), s) ==
+                   cudaSuccess
+               ? WKV_OK
+               : WKV_ERR_CUDA;
+}
+
 const char *wkv_status_string(int status) {
     switch (status) {
         case WKV_OK: return "ok";

@@ -38,6 +38,10 @@ constexpr int kBwdMaps = 9;
 // bf16: r, k, w, v, dy are bf16 (their maps describe bf16 tensors); gradients stay fp32
 cudaError_t wkv6_bwd_launch(bool bf16, bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
                             cudaStream_t stream);
+// RWKV-4 backward; workspace: [B][T][C] + 2 [B][C] floats (see wkv4_bwd_workspace_bytes)
+cudaError_t wkv4_bwd_launch(int B, int T, int C, const float *k, const float *v, const float *w, const float *u,
+                            const float *dy, float *dk, float *dv, float *dw, float *du, float *workspace,
+                            cudaStream_t stream);
 cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,
                             const float *u, float *y, cudaStream_t stream);
 

@@ -181,6 +181,7 @@ class Wkv4Inputs:
     v: np.ndarray      # [B,T,C] float32
     w: np.ndarray      # [C] float32, > 0 (decay exp(-w) per step)
     u: np.ndarray      # [C] float32
+    dy: np.ndarray | None = None  # [B,T,C] float32 upstream gradient
 
 
 def make_wkv6(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, rkv_std: float = 0.5,
@@ -211,15 +212,17 @@ def make_state(B: int, H: int, N: int = 64, *, seed: int = 0, std: float = 1.0) 
 
 
 def make_wkv4(B: int, T: int, C: int, *, seed: int = 0, kv_std: float = 1.0,
-              logw_lo: float = -3.0, logw_hi: float = 1.0, u_std: float = 0.5) -> Wkv4Inputs:
+              logw_lo: float = -3.0, logw_hi: float = 1.0, u_std: float = 0.5,
+              with_dy: bool = False, dy_std: float = 1.0) -> Wkv4Inputs:
     """RWKV-4 inputs: k, v ~ N(0, kv_std^2); w = exp(U(logw_lo, logw_hi)) > 0 per channel;
-    u ~ N(0, u_std^2) per channel."""
+    u ~ N(0, u_std^2) per channel; dy ~ N(0, dy_std^2)."""
     n = B * T * C
     k = normal(seed, STREAM_K, n, kv_std).astype(np.float32).reshape(B, T, C)
     v = normal(seed, STREAM_V, n, kv_std).astype(np.float32).reshape(B, T, C)
     w = np.exp(uniform(seed, STREAM_WRAW, C, logw_lo, logw_hi)).astype(np.float32)
     u = normal(seed, STREAM_U, C, u_std).astype(np.float32)
-    return Wkv4Inputs(B, T, C, k, v, w, u)
+    dy = normal(seed, STREAM_DY, n, dy_std).astype(np.float32).reshape(B, T, C) if with_dy else None
+    return Wkv4Inputs(B, T, C, k, v, w, u, dy)
 
 
 # The workloads: name -> (kind, constructor kwargs).
@@ -236,6 +239,8 @@ WORKLOADS = {
     "wkv6_bidir_bwd_f32_b32t196h12": ("wkv6_bwd_bidir", dict(B=32, T=196, H=12, with_dy=True)),
     # bidirectional RWKV-6 backward with bf16 inputs (fp32 gradients)
     "wkv6_bidir_bwd_bf16_b32t196h12": ("wkv6_bwd_bidir", dict(B=32, T=196, H=12, with_dy=True, dtype="bf16")),
+    # RWKV-4 backward on the RWKV-4 forward's shape
+    "wkv4_bwd_f32_b8t1024c768": ("wkv4_bwd", dict(B=8, T=1024, C=768, with_dy=True)),
     # one recurrent decode step for 512 sequences of the long-text head layout (state from make_state)
     "wkv6_decode_f32_b512h32": ("wkv6_decode", dict(B=512, T=1, H=32)),
 }
@@ -243,6 +248,6 @@ WORKLOADS = {
 
 def make_workload(name: str, seed: int = 0):
     kind, kw = WORKLOADS[name]
-    if kind == "wkv4_fwd":
+    if kind in ("wkv4_fwd", "wkv4_bwd"):
         return kind, make_wkv4(seed=seed, **kw)
     return kind, make_wkv6(seed=seed, **kw)

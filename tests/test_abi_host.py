@@ -132,6 +132,21 @@ def test_wkv6_decode_argument_errors(lib):
     assert f(0, 64, 1, *p, st, y, None) == WKV_OK
 
 
+def test_wkv4_bwd_argument_errors(lib):
+    p = [FAKE + 256 * i for i in range(9)]                     # k, v, w, u, dy, dk, dv, dw, du
+    ws = wkv.wkv4_bwd_workspace_bytes(2, 8, 32)
+    assert ws == 4 * (2 * 8 * 32 + 2 * 2 * 32)
+    f = lib.wkv4_bwd
+    assert f(-1, 8, 32, *p, FAKE, ws, None) == WKV_ERR_ARG
+    assert f(2, 8, 0, *p, FAKE, ws, None) == WKV_ERR_ARG
+    assert f(2, 8, 32, *(p[:4] + [None] + p[5:]), FAKE, ws, None) == WKV_ERR_ARG      # dy missing
+    assert f(2, 8, 32, *p, None, ws, None) == WKV_ERR_WORKSPACE
+    assert f(2, 8, 32, *p, FAKE, ws - 4, None) == WKV_ERR_WORKSPACE
+    q = list(p)
+    q[6] += 4                                                  # dv misaligned
+    assert f(2, 8, 32, *q, FAKE, ws, None) == WKV_ERR_ALIGN
+
+
 def test_wkv4_argument_errors(lib):
     p = [FAKE + 256 * i for i in range(5)]
     assert lib.wkv4_fwd(-1, 4, 32, *p, None) == WKV_ERR_ARG
