@@ -32,12 +32,13 @@
 // exact token-by-token recurrence on the CUDA cores, from the state in TMEM.
 //
 // Warp roles (one CTA per (b, h), 13 warps, two CTAs per SM):
-//   warp 0       TMA loads (2-stage ring) and, from one thread, all MMAs, issued
-//                as their inputs become ready
+//   warp 0       TMA loads (3-stage r/k/v ring, 2-stage w ring) and, from one
+//                thread, all MMAs, in a fixed order
 //   warps 1..4   transform: Q, Kt, the bonus scalars c, exp(Lam_L), chunk flag
 //   warps 5..8   mask: A'^T from TMEM into shared memory
-//   warps 9..12  epilogue: the two warps on TMEM lanes 0..63 store y, the two
-//                on lanes 64..127 rescale the state; all four run exact chunks
+//   warps 9..12  epilogue: the two warps on TMEM lanes 0..63 stage y in the
+//                chunk's Q/Kt slots for a TMA store, the two on lanes 64..127
+//                rescale the state; all four run exact chunks
 // Hand-offs are mbarriers; every wait is bounded and a shared abort flag stops
 // all roles after the first timeout.
 #include "wkv_launch.cuh"
@@ -60,12 +61,15 @@ constexpr int kET = 32 * kEW;
 constexpr int kTokW = kL / kTW;              // tokens per transform warp
 constexpr int kTile = kL * kHead;            // bf16 elements of one 64 x 64 tile (8 KB)
 
-enum { R_ = 0, Z_ = 1, K_ = 2, V_ = 3, W_ = 4, kSlots = 5 };
+enum { R_ = 0, K_ = 1, V_ = 2, kSlots = 3 };
+constexpr int kStages = 3;                   // r, k, v ring (freed by P34)
+constexpr int kWStages = 2;                  // w ring (freed once the transform has read it)
 
 struct TcSmem {
-    __nv_bfloat16 Ap[2][kTile];          // A'^T (row s, p contiguous): first A atom of P34
+    __nv_bfloat16 Ap[kTile];             // A'^T (row s, p contiguous): first A atom of P34
     __nv_bfloat16 Sin[kTile];            // bf16 S_in (row i, j contiguous): B of P2
-    __nv_bfloat16 raw[2][kSlots][kTile]; // stages: r -> Q, zero tile, k -> Kt, v, w (TMA, swizzled)
+    __nv_bfloat16 raw[kStages][kSlots][kTile];   // stages: r -> Q, k -> Kt, v (TMA, swizzled)
+    __nv_bfloat16 wt[kWStages][kTile];   // log-decay tiles (TMA, swizzled)
     float dec[4][kHead];                 // exp(Lam_L) per row i (ring of 4 chunks)
     float cp[4][kL];                     // bonus scalars per token (ring of 4 chunks)
     float psum[2][kTW][kHead];           // per-warp log2-decay sums, by chunk parity
@@ -75,15 +79,21 @@ struct TcSmem {
     int flag[4];                         // chunk c is exact-evaluated iff flag[c & 3] == c + 1
     int abort_;
     uint32_t tmem_base;
-    alignas(8) uint64_t full[2];         // TMA stage landed
-    alignas(8) uint64_t t_done[2];       // transform of the stage's chunk done
+    alignas(8) uint64_t full[kStages];   // r, k, v of the stage landed
+    alignas(8) uint64_t wfull[kWStages]; // w of the w stage landed
+    alignas(8) uint64_t t_done[kStages]; // transform of the stage's chunk done
     alignas(8) uint64_t m1_done[2];      // per TMEM A buffer: A^T ready
     alignas(8) uint64_t a_done[2];       // per TMEM A buffer: A'^T in shared memory, buffer read
-    alignas(8) uint64_t stage_free[2];   // every reader of the stage finished
+    alignas(8) uint64_t ap_free;         // the A'^T buffer has been read (one phase per chunk)
+    alignas(8) uint64_t stage_free[kStages];   // every reader of the stage finished
     alignas(8) uint64_t mma_done;        // Y and S of the chunk complete
     alignas(8) uint64_t s_ready;         // y stored and Y cleared, state rescaled, S_in written
     alignas(8) uint64_t final_bar;
 };
+
+// Two CTAs per SM: 228 KB of shared memory less 1 KB reserved per CTA, with the
+// 1 KB alignment slack of the dynamic allocation.
+static_assert(sizeof(TcSmem) + 1024 <= 113 * 1024, "two CTAs per SM must fit");
 
 // Byte offset of element (row, col) in a 64-row bf16 tile whose 128-byte rows
 // are 128B-swizzled (16-byte chunk g of row r stored at chunk g ^ (r & 7)).
@@ -146,19 +156,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Non-blocking: has the barrier phase with this parity completed?
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
 }
 
 // try_wait with a suspend-time hint: the thread is parked by the hardware until
@@ -229,7 +226,7 @@ __device__ __forceinline__ bool is_flagged(const TcSmem &sm, int c) {
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
-                   FwdParams prm) {
+                   const __grid_constant__ CUtensorMap map_y, FwdParams prm) {
     extern __shared__ unsigned char smem_dyn[];
     TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
 
@@ -238,28 +235,29 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     const int h = blockIdx.x % H, b = blockIdx.x / H;
     const int cbase = h * kHead;
     const int nch = (T + kL - 1) / kL;
-    constexpr uint32_t kStageBytes = 4u * kTile * sizeof(__nv_bfloat16);   // r, k, v, w
+    constexpr uint32_t kStageBytes = 3u * kTile * sizeof(__nv_bfloat16);   // r, k, v
+    constexpr uint32_t kWBytes = kTile * sizeof(__nv_bfloat16);
 
     if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
     if (tid < 4) sm.flag[tid] = 0;
-    for (int i = tid; i < 2 * kTile * 2 / 16; i += kThreads) {   // the two zero tiles (never rewritten)
-        uint4 *z = reinterpret_cast<uint4 *>(sm.raw[i / (kTile * 2 / 16)][Z_]);
-        z[i % (kTile * 2 / 16)] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_proxy_async_smem();
     if (tid == 0) {
         sm.abort_ = 0;
         prefetch_tensormap(&map_r);
         prefetch_tensormap(&map_k);
         prefetch_tensormap(&map_v);
         prefetch_tensormap(&map_w);
-        for (int i = 0; i < 2; ++i) {
+        prefetch_tensormap(&map_y);
+        for (int i = 0; i < kStages; ++i) {
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.t_done[i], kTT);
-            mbar_init(&sm.m1_done[i], 1);
-            mbar_init(&sm.a_done[i], kAT);
             mbar_init(&sm.stage_free[i], 1);
         }
+        for (int i = 0; i < kWStages; ++i) mbar_init(&sm.wfull[i], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.m1_done[i], 1);
+            mbar_init(&sm.a_done[i], kAT);
+        }
+        mbar_init(&sm.ap_free, 1);
         mbar_init(&sm.mma_done, 1);
         mbar_init(&sm.s_ready, kET);
         mbar_init(&sm.final_bar, 1);
@@ -272,121 +270,130 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    // TMEM columns: A^T buffers at 0 and 64 (M = 64 layout), [Y ; S] at 128 (M = 128: lane = row)
+    // TMEM columns: A^T buffers at 0 and 64 (M = 64 layout); [Y ; S] at 128 and P2's
+    // Q S_in at 192 (M = 128: lane = row; only lanes 0..63 of the latter are read)
     const uint32_t tbase = sm.tmem_base;
-    const uint32_t tD = tbase + 128;
+    const uint32_t tD = tbase + 128, tD2 = tbase + 192;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lane quarter
 
     if (warp == 0) {
         // ===================== TMA + MMA issue (one thread) =====================
         if (lane == 0) {
             auto issue = [&](int c) {
-                const int s = c & 1;
+                const int s = c % kStages;
                 mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
                 tma_load_3d(sm.raw[s][R_], &map_r, cbase, c * kL, b, &sm.full[s]);
                 tma_load_3d(sm.raw[s][K_], &map_k, cbase, c * kL, b, &sm.full[s]);
                 tma_load_3d(sm.raw[s][V_], &map_v, cbase, c * kL, b, &sm.full[s]);
-                tma_load_3d(sm.raw[s][W_], &map_w, cbase, c * kL, b, &sm.full[s]);
-                // the load of chunk c + 2 waits for this stage's chunk to retire; start
-                // its HBM reads now so that it is served from L2
-                if (c + 2 < nch) {
-                    tma_prefetch_l2_3d(&map_r, cbase, (c + 2) * kL, b);
-                    tma_prefetch_l2_3d(&map_k, cbase, (c + 2) * kL, b);
-                    tma_prefetch_l2_3d(&map_v, cbase, (c + 2) * kL, b);
-                    tma_prefetch_l2_3d(&map_w, cbase, (c + 2) * kL, b);
+                // the load of chunk c + kStages waits for this stage's chunk to retire;
+                // start its HBM reads now so that it is served from L2
+                if (c + kStages < nch) {
+                    tma_prefetch_l2_3d(&map_r, cbase, (c + kStages) * kL, b);
+                    tma_prefetch_l2_3d(&map_k, cbase, (c + kStages) * kL, b);
+                    tma_prefetch_l2_3d(&map_v, cbase, (c + kStages) * kL, b);
                 }
+            };
+            // The thread's bookkeeping stays in scalars: an array indexed by a runtime
+            // value would live in local memory, one L2 round trip per access under load.
+            static_assert(kWStages == 2, "the w bookkeeping below has two stages");
+            int last_w0 = -1, last_w1 = -1;     // latest chunk loaded into each w stage (-1: none)
+            auto issue_w = [&](int c) {
+                const int s = c & 1;
+                if (s) last_w1 = c; else last_w0 = c;
+                mbar_arrive_expect_tx(&sm.wfull[s], kWBytes);
+                tma_load_3d(sm.wt[s], &map_w, cbase, c * kL, b, &sm.wfull[s]);
             };
             constexpr uint32_t kIdM1 = idesc_bf16(64, 64, false, false);
             constexpr uint32_t kIdP2 = idesc_bf16(128, 64, false, true);
             constexpr uint32_t kIdP34 = idesc_bf16(128, 64, true, true);
-            issue(0);
-            if (nch > 1) issue(1);
-            int next_tma = nch > 1 ? 2 : 1;   // next chunk to load
-            int next_m1 = 0;                  // next chunk for M1
-            int next_p = 0;                   // next chunk for P2 / P34
-            bool p2_issued = false;           // P2 of chunk next_p issued, P34 pending
+            for (int c = 0; c < kStages && c < nch; ++c) issue(c);
+            for (int c = 0; c < kWStages && c < nch; ++c) issue_w(c);
+            int next_tma = min(nch, kStages);   // next chunk to load (r, k, v)
+            // exact chunk whose w stage waits for its epilogue, per w stage (-1: none); a
+            // slot cannot be reused before it is resolved, since the chunk that would
+            // reuse it needs the pending load first
+            int w_pend0 = -1, w_pend1 = -1;
             bool ok = true;
-            uint32_t idle = 0;                // idle polls since the last issue
-            unsigned long long idle_since = 0;
-            // Each step issues whatever has its inputs ready, the state chain
-            // (P34, then P2) first.  Invariants that keep every parity wait
-            // unambiguous: M1 runs at most one chunk ahead of P34, a stage is
-            // reloaded only after its chunk's last reader released it, and
-            // every chunk's a_done phase is observed before the chunk retires.
-            while (next_p < nch) {
-                bool progress = false;
-                if (p2_issued) {
-                    const int c = next_p, set = c & 1;
-                    if (mbar_test(&sm.a_done[set], (c >> 1) & 1)) {
-                        tc::fence_after_sync();
-                        const uint32_t lbo = smem_u32(sm.raw[set][K_]) - smem_u32(sm.Ap[set]);
+            // A fixed issue order, waiting on one barrier at a time (the waiting thread
+            // is parked by the hardware and resumes as soon as the phase completes):
+            //   M1(0), P2(0), then for every chunk c:  P34(c), M1(c+1), P2(c+1), load c+3.
+            // Every input of a step comes from steps issued before it, so the order
+            // cannot deadlock; M1 runs at most one chunk ahead of P34, a stage is
+            // reloaded only after its chunk's last reader released it, and every parity
+            // wait is on the oldest phase not yet observed, so none is ambiguous.
+            auto step_m1 = [&](int c) -> bool {
+                const int set = c & 1, s = c % kStages;
+                if (!wait_or_abort(sm, &sm.t_done[s], (c / kStages) & 1)) return false;
+                tc::fence_after_sync();
+                if (!is_flagged(sm, c)) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_bf16(tD, desc_mn(sm.Ap[set], k, lbo), desc_mn(sm.raw[set][V_], k, 16), kIdP34, true);
-                        tc::mma_commit(&sm.mma_done);
-                        tc::mma_commit(&sm.stage_free[set]);
-                        ++next_p;
-                        p2_issued = false;
-                        progress = true;
-                    }
-                } else if (next_p < next_m1 && mbar_test(&sm.s_ready, next_p & 1)) {
-                    const int c = next_p, set = c & 1;
-                    tc::fence_after_sync();
-                    if (!is_flagged(sm, c)) {
-                        // rows 64..127 of [Q ; 0] are the zero tile: S only accumulates 0
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_bf16(tD, desc_k(sm.raw[set][R_], k), desc_mn(sm.Sin, k, 16), kIdP2, true);
-                        p2_issued = true;
-                        progress = true;
-                    } else if (mbar_test(&sm.a_done[set], (c >> 1) & 1)) {
-                        // the epilogue evaluates this chunk exactly and then releases its stage
-                        mbar_arrive(&sm.mma_done);
-                        ++next_p;
-                        progress = true;
-                    }
-                }
-                if (next_m1 < nch && next_m1 <= next_p + 1) {
-                    const int c = next_m1, set = c & 1;
-                    if (mbar_test(&sm.t_done[set], (c >> 1) & 1)) {
-                        tc::fence_after_sync();
-                        if (!is_flagged(sm, c)) {
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                mma_bf16(tbase + 64 * set, desc_k(sm.raw[set][K_], k), desc_k(sm.raw[set][R_], k),
-                                         kIdM1, k > 0);
-                            tc::mma_commit(&sm.m1_done[set]);
-                        } else {
-                            mbar_arrive(&sm.m1_done[set]);   // the mask warps skip this chunk
-                        }
-                        ++next_m1;
-                        progress = true;
-                    }
-                }
-                if (next_tma < nch && mbar_test(&sm.stage_free[next_tma & 1], ((next_tma - 2) >> 1) & 1)) {
-                    fence_proxy_async_smem();
-                    issue(next_tma);
-                    ++next_tma;
-                    progress = true;
-                }
-                if (progress) {
-                    idle = 0;
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tbase + 64 * set, desc_k(sm.raw[s][K_], k), desc_k(sm.raw[s][R_], k), kIdM1,
+                                 k > 0);
+                    tc::mma_commit(&sm.m1_done[set]);
+                    if (c + kWStages < nch) issue_w(c + kWStages);   // the transform is done with w
                 } else {
-                    // the clock and the abort flag are read every 64 idle polls only
-                    if ((++idle & 63) == 0) {
-                        if (*(volatile int *)&sm.abort_) {
-                            ok = false;
-                            break;
-                        }
-                        const unsigned long long now = globaltimer_ns();
-                        if (idle == 64) {
-                            idle_since = now;
-                        } else if (now - idle_since > kWaitLimitNs) {
-                            atomicOr(&g_wkv_faults, WKV_FAULT_TIMEOUT);
-                            *(volatile int *)&sm.abort_ = 1;
-                            ok = false;
-                            break;
-                        }
+                    mbar_arrive(&sm.m1_done[set]);   // the mask warps skip this chunk
+                    if (c & 1) w_pend1 = c; else w_pend0 = c;   // the exact evaluation still reads w
+                }
+                return true;
+            };
+            auto step_p2 = [&](int c) -> bool {
+                // the epilogue of chunk c - 1 is done (the initial phase stands for c = 0)
+                if (!wait_or_abort(sm, &sm.s_ready, c & 1)) return false;
+                tc::fence_after_sync();
+                // exact chunks up to c - 1 have released their w stage
+                if (w_pend0 >= 0 && w_pend0 <= c - 1) {
+                    if (w_pend0 + kWStages < nch) issue_w(w_pend0 + kWStages);
+                    w_pend0 = -1;
+                }
+                if (w_pend1 >= 0 && w_pend1 <= c - 1) {
+                    if (w_pend1 + kWStages < nch) issue_w(w_pend1 + kWStages);
+                    w_pend1 = -1;
+                }
+                if (!is_flagged(sm, c)) {
+                    const int s = c % kStages;
+                    // [Q ; next tile] S_in: rows 64..127 land in TMEM lanes that are never read
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tD2, desc_k(sm.raw[s][R_], k), desc_mn(sm.Sin, k, 16), kIdP2, k > 0);
+                }
+                return true;
+            };
+            auto step_p34 = [&](int c) -> bool {
+                const int set = c & 1, s = c % kStages;
+                if (!wait_or_abort(sm, &sm.a_done[set], (c >> 1) & 1)) return false;
+                tc::fence_after_sync();
+                if (!is_flagged(sm, c)) {
+                    const uint32_t lbo = smem_u32(sm.raw[s][K_]) - smem_u32(sm.Ap);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tD, desc_mn(sm.Ap, k, lbo), desc_mn(sm.raw[s][V_], k, 16), kIdP34, true);
+                    tc::mma_commit(&sm.mma_done);
+                    tc::mma_commit(&sm.ap_free);
+                } else {
+                    // the epilogue evaluates this chunk exactly and then releases its stage;
+                    // the A'^T buffer phase is completed by a commit, in order behind P34(c - 1)
+                    mbar_arrive(&sm.mma_done);
+                    tc::mma_commit(&sm.ap_free);
+                }
+                return true;
+            };
+            ok = step_m1(0) && step_p2(0);
+            for (int c = 0; c < nch && ok; ++c) {
+                ok = step_p34(c);
+                if (ok && c + 1 < nch) ok = step_m1(c + 1) && step_p2(c + 1);
+                if (ok && next_tma < nch) {
+                    // the stage of chunk next_tma - kStages (= c once the ring is full) is
+                    // released by the epilogue once its y store has read the staging tiles
+                    // (or its exact evaluation is done); P2(c + 1) already waited for the
+                    // rest of that epilogue, so this wait is short
+                    const int cc = next_tma - kStages;
+                    ok = wait_or_abort(sm, &sm.stage_free[cc % kStages], (cc / kStages) & 1);
+                    if (ok) {
+                        fence_proxy_async_smem();
+                        issue(next_tma);
+                        ++next_tma;
                     }
                 }
             }
@@ -394,8 +401,11 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
             tc::mma_commit(&sm.final_bar);
             mbar_wait_bounded(&sm.final_bar, 0);
             if (!ok) {
-                for (int cc = max(0, next_tma - 2); cc < next_tma; ++cc)
-                    mbar_wait_bounded(&sm.full[cc & 1], (cc >> 1) & 1);
+                // drain the loads still in flight (the last kStages r/k/v loads, the w loads)
+                for (int cc = max(0, next_tma - kStages); cc < next_tma; ++cc)
+                    mbar_wait_bounded(&sm.full[cc % kStages], (cc / kStages) & 1);
+                if (last_w0 >= 0) mbar_wait_bounded(&sm.wfull[0], (last_w0 / kWStages) & 1);
+                if (last_w1 >= 0) mbar_wait_bounded(&sm.wfull[1], (last_w1 / kWStages) & 1);
             }
         }
     } else if (warp <= kTW) {
@@ -409,12 +419,13 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
         const uint32_t chunk = (uint32_t)(lane >> 2);
         const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
         for (int c = 0; c < nch; ++c) {
-            const int stg = c & 1, par = c & 1;
+            const int stg = c % kStages, par = c & 1;
             // a timeout sets the shared abort flag; all transform threads leave
             // together after the named barrier below, so none is left waiting there
-            wait_or_abort(sm, &sm.full[stg], (c >> 1) & 1);
+            wait_or_abort(sm, &sm.full[stg], (c / kStages) & 1);
+            wait_or_abort(sm, &sm.wfull[c % kWStages], (c / kWStages) & 1);
             __nv_bfloat16 *Rb = sm.raw[stg][R_], *Kb = sm.raw[stg][K_];
-            const __nv_bfloat16 *Wb = sm.raw[stg][W_];
+            const __nv_bfloat16 *Wb = sm.wt[c % kWStages];
             auto off = [&](int e) -> uint32_t {
                 const int p = p0 + e;
                 return (uint32_t)p * 128u + ((chunk ^ (uint32_t)(p & 7)) << 4) + in_chunk;
@@ -462,26 +473,30 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 // flagged is warp-uniform: keeping the branch outside the token loop
                 // leaves one straight-line body whose loads and exponentials overlap
                 if (!flagged) {
-                    // all loads first: the in-place stores below may alias them as far as
-                    // the compiler can tell, so loads issued after a store would serialise
-                    uint32_t rv[8], kv[8], wv[8];
+                    // four tokens at a time, loads first: the in-place stores below may
+                    // alias them as far as the compiler can tell, so loads issued after a
+                    // store would serialise (batches of four keep the registers in bounds)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const uint32_t o = off(8 * half + e);
-                        rv[e] = ld_u32(Rb, o);
-                        kv[e] = ld_u32(Kb, o);
-                        wv[e] = ld_u32(Wb, o);
-                    }
+                    for (int sb = 0; sb < 2; ++sb) {
+                        uint32_t rv[4], kv[4], wv[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const uint32_t o = off(8 * half + e);
-                        const float r0 = bf_lo(rv[e]), r1 = bf_hi(rv[e]), k0 = bf_lo(kv[e]), k1 = bf_hi(kv[e]);
-                        bp[e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
-                        const float q0 = r0 * fast_exp2(L0), q1 = r1 * fast_exp2(L1);
-                        L0 += bf_lo(wv[e]) * kLog2e;
-                        L1 += bf_hi(wv[e]) * kLog2e;
-                        st_u32(Rb, o, pack_bf16(q0, q1));
-                        st_u32(Kb, o, pack_bf16(k0 * fast_exp2(-L0), k1 * fast_exp2(-L1)));
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t o = off(8 * half + 4 * sb + e);
+                            rv[e] = ld_u32(Rb, o);
+                            kv[e] = ld_u32(Kb, o);
+                            wv[e] = ld_u32(Wb, o);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t o = off(8 * half + 4 * sb + e);
+                            const float r0 = bf_lo(rv[e]), r1 = bf_hi(rv[e]), k0 = bf_lo(kv[e]), k1 = bf_hi(kv[e]);
+                            bp[4 * sb + e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
+                            const float q0 = r0 * fast_exp2(L0), q1 = r1 * fast_exp2(L1);
+                            L0 += bf_lo(wv[e]) * kLog2e;
+                            L1 += bf_hi(wv[e]) * kLog2e;
+                            st_u32(Rb, o, pack_bf16(q0, q1));
+                            st_u32(Kb, o, pack_bf16(k0 * fast_exp2(-L0), k1 * fast_exp2(-L1)));
+                        }
                     }
                 } else {
 #pragma unroll
@@ -505,9 +520,11 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
             const int set = c & 1;
             if (!wait_or_abort(sm, &sm.m1_done[set], (c >> 1) & 1)) break;
             if (!is_flagged(sm, c)) {
+                // the single A'^T buffer: P34 of the previous chunk must have read it
+                if (c > 0 && !wait_or_abort(sm, &sm.ap_free, (c - 1) & 1)) break;
                 tc::fence_after_sync();
                 const float cps = sm.cp[c & 3][s];
-                __nv_bfloat16 *Ab = sm.Ap[set];
+                __nv_bfloat16 *Ab = sm.Ap;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float a[32];
@@ -555,34 +572,42 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
             mbar_arrive(&sm.s_ready);
         }
         for (int c = 0; c < nch; ++c) {
-            const int t0 = c * kL, stg = c & 1;
+            const int t0 = c * kL, stg = c % kStages;
             wait_or_abort(sm, &sm.mma_done, c & 1);
             named_sync(2, kET);
             if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
             tc::fence_after_sync();
-            if (!is_flagged(sm, c)) {
+            const bool exact = is_flagged(sm, c);
+            if (!exact) {
                 if (yrole) {
-                    // ---- y row p (64 channels, 256 contiguous bytes), then clear Y for the next chunk
-                    const bool live = t0 + row < T;
-                    float4 *dst = reinterpret_cast<float4 *>(prm.y + ((size_t)b * T + t0 + row) * C + cbase);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float v[32];
-                        tc::tmem_ld32(tD + lane_off + 32 * half, v);
+                    // ---- y row p = (A' V) row p + (Q S_in) row p, then clear Y for the next
+                    // chunk.  The row goes to two 128B-swizzled fp32 staging tiles (columns
+                    // 0..31 and 32..63) in the Q and Kt slots of the chunk's stage, which no
+                    // MMA reads any more; one thread then stores them with the TMA, which
+                    // writes whole lines and leaves out the rows past T.
+#pragma unroll 1
+                    for (int qt = 0; qt < 4; ++qt) {   // 16 columns at a time keeps registers low
+                        float v[16], v2[16];
+                        tc::tmem_ld16(tD + lane_off + 16 * qt, v);
+                        tc::tmem_ld16(tD2 + lane_off + 16 * qt, v2);
                         tc::tmem_wait_ld();
-                        if (live) {
 #pragma unroll
-                            for (int g = 0; g < 8; ++g)
-                                dst[8 * half + g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+                        for (int e = 0; e < 16; ++e) v[e] += v2[e];
+                        char *box = reinterpret_cast<char *>(sm.raw[stg][R_ + (qt >> 1)]) + row * 128;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int j = 4 * (qt & 1) + g;   // 16-byte chunk of the 128-byte row
+                            *reinterpret_cast<float4 *>(box + ((j ^ (row & 7)) << 4)) =
+                                make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
                         }
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = 0.f;
-                        tc::tmem_st32(tD + lane_off + 32 * half, v);
+                        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                        tc::tmem_st16(tD + lane_off + 16 * qt, v);
                     }
                 } else {
                     // ---- S row i scaled by exp(Lam_L[i]), back to TMEM, bf16 copy into S_in
                     const float dsc = sm.dec[c & 3][row];
-#pragma unroll
+#pragma unroll 1
                     for (int half = 0; half < 2; ++half) {
                         float v[32];
                         tc::tmem_ld32(tD + lane_off + 32 * half, v);
@@ -604,7 +629,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 // The S warps own rows i of S and form per-warp column sums of
                 // r_p[i] S[i][j]; the Y warps add the two halves and the bonus and store y.
                 const __nv_bfloat16 *R = sm.raw[stg][R_], *Kr = sm.raw[stg][K_];
-                const __nv_bfloat16 *V = sm.raw[stg][V_], *W = sm.raw[stg][W_];
+                const __nv_bfloat16 *V = sm.raw[stg][V_], *W = sm.wt[c % kWStages];
                 for (int p = 0; p < kL; ++p) {
                     if (!yrole) {
                         const float rr = raw_at(R, p, row), dd = __expf(raw_at(W, p, row)), kk = raw_at(Kr, p, row);
@@ -665,7 +690,20 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
             fence_proxy_async_smem();
             tc::fence_before_sync();
             mbar_arrive(&sm.s_ready);
+            if (yrole && !exact) {
+                // every Y row is staged (and fenced for the async proxy): store the tiles,
+                // then release the stage once the TMA has read them
+                named_sync(3, kET / 2);
+                if (row == 0) {
+                    tma_store_3d(&map_y, sm.raw[stg][R_], cbase, t0, b);
+                    tma_store_3d(&map_y, sm.raw[stg][K_], cbase + kHead / 2, t0, b);
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                    mbar_arrive(&sm.stage_free[stg]);
+                }
+            }
         }
+        if (yrole && row == 0) bulk_wait_all();
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -674,14 +712,15 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
 }
 
 cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
-                               const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream) {
+                               const CUtensorMap &mw, const CUtensorMap &my, const FwdParams &prm,
+                               cudaStream_t stream) {
     const size_t smem = sizeof(TcSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(wkv6_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(wkv6_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    wkv6_fwd_tc_kernel<<<(unsigned)(prm.B * prm.H), kThreads, smem, stream>>>(mr, mk, mv, mw, prm);
+    wkv6_fwd_tc_kernel<<<(unsigned)(prm.B * prm.H), kThreads, smem, stream>>>(mr, mk, mv, mw, my, prm);
     return cudaGetLastError();
 }
 

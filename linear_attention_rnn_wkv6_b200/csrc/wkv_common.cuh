@@ -91,6 +91,20 @@ __device__ __forceinline__ void drain_two_stage(uint64_t *full, int g, int nchun
 // completion counted on `bar`.  Coordinates are (c, t, b); c must be a
 // multiple of 16 bytes / element size, t may be negative or past the end
 // (those rows are zero filled).
+// Tiled TMA store of a shared-memory box to a 3-D map; elements outside the
+// tensor are not written.  Completion is tracked with the bulk-group helpers.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c, int t, int b) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c), "r"(t), "r"(b), "r"(smem_u32(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The source shared memory of every committed store may be reused.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Every committed store has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c, int t, int b,
                                             uint64_t *bar) {
     asm volatile(

@@ -28,8 +28,10 @@ constexpr int kBwdTC = 8;    // tokens per TMA chunk, backward kernel
 cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const CUtensorMap &mk,
                             const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
                             cudaStream_t stream);
+// my: fp32 y map, box 32 channels x 64 tokens, 128-byte swizzle (TMA stores).
 cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
-                               const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream);
+                               const CUtensorMap &mw, const CUtensorMap &my, const FwdParams &prm,
+                               cudaStream_t stream);
 // One recurrent step for B sequences (state [B][H][N][N] updated in place).
 cudaError_t wkv6_decode_launch(int B, int C, int H, const float *r, const float *k, const float *v,
                                const float *w, const float *u, float *state, float *y, cudaStream_t stream);
