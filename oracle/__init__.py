@@ -46,8 +46,10 @@ def _configure(lib):
     lib.oracle_wkv6_bwd.argtypes = [I, I, I, I, I] + [_DP] * 11
     lib.oracle_wkv4_fwd.argtypes = [I, I, I] + [_DP] * 5
     lib.oracle_wkv4_bwd.argtypes = [I, I, I] + [_DP] * 9
+    lib.oracle_wkv5_fwd.argtypes = [I, I, I, I] + [_DP] * 6
+    lib.oracle_wkv5_bwd.argtypes = [I, I, I, I] + [_DP] * 11
     for f in (lib.oracle_wkv6_fwd, lib.oracle_wkv6_fwd_state, lib.oracle_wkv6_bwd, lib.oracle_wkv4_fwd,
-              lib.oracle_wkv4_bwd):
+              lib.oracle_wkv4_bwd, lib.oracle_wkv5_fwd, lib.oracle_wkv5_bwd):
         f.restype = ctypes.c_int
     return lib
 
@@ -131,7 +133,27 @@ class Oracle:
             raise ValueError(f"oracle_wkv4_bwd failed ({rc})")
         return dk, dv, dw, du
 
+    def wkv5_fwd(self, r, k, v, w, u, H: int) -> np.ndarray:
+        """RWKV-5 forward.  r,k,v: [B,T,C]; w (>= 0, static decay exp(-w)), u: [C] -> y [B,T,C]."""
+        r, k, v, w, u = map(_d, (r, k, v, w, u))
+        B, T, C = r.shape
+        y = np.zeros((B, T, C), dtype=np.float64)
+        rc = self._lib.oracle_wkv5_fwd(B, T, C, H, _p(r), _p(k), _p(v), _p(w), _p(u), _p(y))
+        if rc != 0:
+            raise ValueError(f"oracle_wkv5_fwd failed ({rc})")
+        return y
 
+    def wkv5_bwd(self, r, k, v, w, u, dy, H: int):
+        """RWKV-5 backward -> (dr, dk, dv [B,T,C], dw, du [C] summed over B and T)."""
+        r, k, v, w, u, dy = map(_d, (r, k, v, w, u, dy))
+        B, T, C = r.shape
+        outs = [np.zeros((B, T, C), dtype=np.float64) for _ in range(3)] + [np.zeros(C, dtype=np.float64)
+                                                                               for _ in range(2)]
+        rc = self._lib.oracle_wkv5_bwd(B, T, C, H, _p(r), _p(k), _p(v), _p(w), _p(u), _p(dy),
+                                       *[_p(o) for o in outs])
+        if rc != 0:
+            raise ValueError(f"oracle_wkv5_bwd failed ({rc})")
+        return tuple(outs)
 
 
 def _default() -> Oracle:
@@ -159,6 +181,14 @@ def wkv4_fwd(k, v, w, u) -> np.ndarray:
 
 def wkv4_bwd(k, v, w, u, dy):
     return _default().wkv4_bwd(k, v, w, u, dy)
+
+
+def wkv5_fwd(r, k, v, w, u, H: int) -> np.ndarray:
+    return _default().wkv5_fwd(r, k, v, w, u, H)
+
+
+def wkv5_bwd(r, k, v, w, u, dy, H: int):
+    return _default().wkv5_bwd(r, k, v, w, u, dy, H)
 
 
 def source() -> str:

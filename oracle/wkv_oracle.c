@@ -266,6 +266,111 @@ int oracle_wkv6_bwd(int B, int T, int C, int H, int bidirectional,
 }
 
 /* ------------------------------------------------------------------------ */
+/* RWKV-5 forward (RWKV Architecture page, RWKV-5 "Eagle": the matrix state   */
+/* decays by the static, per-channel factor exp(-w), S_t = exp(-w) . S_{t-1}  */
+/* + k_t^T v_t).  The readout is RWKV-6's with that constant decay:           */
+/*   y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),  S_{-1} = 0,                     */
+/* w : [C], w >= 0 (decay exp(-w) of state row i = channel h*N + i).         */
+/* ------------------------------------------------------------------------ */
+int oracle_wkv5_fwd(int B, int T, int C, int H, const double *r, const double *k, const double *v,
+                    const double *w, const double *u, double *y)
+{
+    if (B < 0 || T < 0 || H < 1 || C % H != 0) return -1;
+    const int N = C / H;
+    double *S = (double *)malloc(sizeof(double) * (size_t)N * N);
+    if (!S) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            memset(S, 0, sizeof(double) * (size_t)N * N);
+            for (int t = 0; t < T; ++t) {
+                const double *rt = r + IDX(b, t, h * N), *kt = k + IDX(b, t, h * N);
+                const double *vt = v + IDX(b, t, h * N);
+                double *yt = y + IDX(b, t, h * N);
+                for (int j = 0; j < N; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < N; ++i)
+                        acc += rt[i] * (S[i * N + j] + u[h * N + i] * kt[i] * vt[j]);
+                    yt[j] = acc;
+                }
+                for (int i = 0; i < N; ++i) {
+                    const double d = exp(-w[h * N + i]);
+                    for (int j = 0; j < N; ++j) S[i * N + j] = d * S[i * N + j] + kt[i] * vt[j];
+                }
+            }
+        }
+    free(S);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-5 backward: reverse-mode differentiation of oracle_wkv5_fwd, with    */
+/* every state stored.  The adjoint A_t = dL/dS_t obeys A_{T-1} = 0 and      */
+/* A_{t-1} = r_t dy_t^T + exp(-w) . A_t; per step                            */
+/*   dr_t = (S_{t-1} + diag(u) k_t^T v_t) dy_t                                */
+/*   dk_t = A_t v_t + u . r_t (v_t . dy_t)                                    */
+/*   dv_t = A_t^T k_t + (sum_i r_t u k_t) dy_t                                 */
+/*   du  += r_t . k_t (v_t . dy_t)                                            */
+/* and, since dS_t/dw = -exp(-w) . S_{t-1} row by row,                        */
+/*   dw  -= exp(-w) . sum_j S_{t-1}[i][j] A_t[i][j]   (summed over b and t).  */
+/* ------------------------------------------------------------------------ */
+int oracle_wkv5_bwd(int B, int T, int C, int H, const double *r, const double *k, const double *v,
+                    const double *w, const double *u, const double *dy,
+                    double *dr, double *dk, double *dv, double *dw, double *du)
+{
+    if (B < 0 || T < 0 || H < 1 || C % H != 0) return -1;
+    const int N = C / H;
+    const size_t NN = (size_t)N * N;
+    memset(dw, 0, sizeof(double) * (size_t)C);
+    memset(du, 0, sizeof(double) * (size_t)C);
+    if (T == 0) return 0;
+    double *states = (double *)malloc(sizeof(double) * NN * (size_t)(T + 1));
+    double *A = (double *)malloc(sizeof(double) * NN);
+    if (!states || !A) { free(states); free(A); return -2; }
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const double *uh = u + h * N, *wh = w + h * N;
+            memset(states, 0, sizeof(double) * NN);
+            for (int t = 0; t < T; ++t) {   /* states[t + 1] = S_t */
+                const double *kt = k + IDX(b, t, h * N), *vt = v + IDX(b, t, h * N);
+                for (int i = 0; i < N; ++i)
+                    for (int j = 0; j < N; ++j)
+                        states[NN * (t + 1) + i * N + j] = exp(-wh[i]) * states[NN * t + i * N + j] + kt[i] * vt[j];
+            }
+            memset(A, 0, sizeof(double) * NN);
+            for (int t = T - 1; t >= 0; --t) {
+                const double *rt = r + IDX(b, t, h * N), *kt = k + IDX(b, t, h * N);
+                const double *vt = v + IDX(b, t, h * N), *gt = dy + IDX(b, t, h * N);
+                const double *Sp = states + NN * t;
+                double vdy = 0.0, ruk = 0.0;
+                for (int j = 0; j < N; ++j) vdy += vt[j] * gt[j];
+                for (int i = 0; i < N; ++i) ruk += rt[i] * uh[i] * kt[i];
+                for (int i = 0; i < N; ++i) {
+                    double accr = 0.0, acck = 0.0, accw = 0.0;
+                    for (int j = 0; j < N; ++j) {
+                        accr += (Sp[i * N + j] + uh[i] * kt[i] * vt[j]) * gt[j];
+                        acck += A[i * N + j] * vt[j];
+                        accw += Sp[i * N + j] * A[i * N + j];
+                    }
+                    dr[IDX(b, t, h * N + i)] = accr;
+                    dk[IDX(b, t, h * N + i)] = acck + uh[i] * rt[i] * vdy;
+                    dw[h * N + i] -= exp(-wh[i]) * accw;
+                    du[h * N + i] += rt[i] * kt[i] * vdy;
+                }
+                for (int j = 0; j < N; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < N; ++i) acc += A[i * N + j] * kt[i];
+                    dv[IDX(b, t, h * N + j)] = acc + ruk * gt[j];
+                }
+                for (int i = 0; i < N; ++i)
+                    for (int j = 0; j < N; ++j) A[i * N + j] = rt[i] * gt[j] + exp(-wh[i]) * A[i * N + j];
+            }
+        }
+    free(states);
+    free(A);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* RWKV-4 forward (RWKV Architecture page, The Recurrent Inference            */
 /* Formulation):                                                             */
 /*   WKV_t = (a_{t-1} + e^{u+k_t} v_t) / (b_{t-1} + e^{u+k_t})                */

@@ -53,6 +53,14 @@ MUTATIONS = [
      [pins.test_wkv4_geometric_closed_form, pins.test_golden_wkv4_forward]),
     ("wkv4_missing_bonus", "e2 = exp(u[c] + kt - q);", "e2 = exp(kt - q);", 0,
      [pins.test_golden_wkv4_forward, lambda o: pins.test_wkv4_recurrence_matches_ratio_of_sums(o, 2, 5, 3)]),
+    ("wkv5_decay_sign", "const double d = exp(-w[h * N + i]);", "const double d = exp(w[h * N + i]);", 0,
+     [pins.test_wkv5_geometric_closed_form, lambda o: pins.test_wkv5_is_wkv6_with_constant_decay(o, 2, 7, 2, 4)]),
+    ("wkv5_readout_before_bonus", "acc += rt[i] * (S[i * N + j] + u[h * N + i] * kt[i] * vt[j]);",
+     "acc += rt[i] * S[i * N + j];", 0, [pins.test_wkv5_geometric_closed_form]),
+    ("wkv5_bwd_dw_sign", "dw[h * N + i] -= exp(-wh[i]) * accw;", "dw[h * N + i] += exp(-wh[i]) * accw;", 0,
+     [pins.test_wkv5_backward_finite_differences, pins.test_wkv5_backward_matches_summed_wkv6_pair_form]),
+    ("wkv5_bwd_adjoint_without_decay", "A[i * N + j] = rt[i] * gt[j] + exp(-wh[i]) * A[i * N + j];",
+     "A[i * N + j] = rt[i] * gt[j] + A[i * N + j];", 0, [pins.test_wkv5_backward_finite_differences]),
     ("wkv4_no_shift_update", "                p = q;\n", "", 0,
      [lambda o: pins.test_wkv4_recurrence_matches_ratio_of_sums(o, 1, 40, 4), pins.test_wkv4_large_keys_stay_finite]),
 ]

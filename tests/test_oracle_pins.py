@@ -417,3 +417,85 @@ def test_pins_catch_a_planted_decay_index_error():
         S = S + np.outer(K[t], V[t])
     yb = brute.wkv6_head(R, K, V, W, u)
     assert np.max(np.abs(y - yb)) > 1e-3
+
+
+# ---------------------------------------------------------------- RWKV-5 (static decay)
+
+def _wkv5_case(B, T, H, N, seed, wlo=-3.0, whi=1.0):
+    g = _rng(seed)
+    C = H * N
+    r, k, v = (g.normal(0, 0.7, (B, T, C)) for _ in range(3))
+    w = np.exp(g.uniform(wlo, whi, C))            # decay exp(-w) per channel
+    u = g.normal(0, 0.7, C)
+    return r, k, v, w, u
+
+
+@pytest.mark.parametrize("B,T,H,N", [(1, 1, 1, 4), (2, 7, 2, 4), (1, 33, 1, 8), (1, 5, 1, 64)])
+def test_wkv5_is_wkv6_with_constant_decay(oracle_mod, B, T, H, N):
+    """RWKV-5 is the static special case: the brute-force pair sums with ew_t = -w for every t."""
+    r, k, v, w, u = _wkv5_case(B, T, H, N, seed=60 + T)
+    y = oracle_mod.wkv5_fwd(r, k, v, w, u, H=H)
+    yb = brute.wkv6(r, k, v, np.broadcast_to(-w, r.shape).copy(), u, H)
+    assert np.max(np.abs(y - yb)) <= 1e-12 * max(1.0, np.max(np.abs(yb)))
+
+
+def test_wkv5_geometric_closed_form(oracle_mod):
+    """One live channel i with k = 1 and v = 1: y_t[j] = r_t[i] ((1 - d^t) / (1 - d) + u_i), d = e^{-w_i}."""
+    T, N, i = 12, 4, 2
+    r = np.zeros((1, T, N)); r[0, :, i] = _rng(61).normal(size=T)
+    k = np.zeros((1, T, N)); k[0, :, i] = 1.0
+    v = np.ones((1, T, N))
+    w = np.array([0.3, 1.1, 0.45, 2.0]); u = np.array([0.1, -0.2, 0.7, 0.4])
+    y = oracle_mod.wkv5_fwd(r, k, v, w, u, H=1)[0]
+    d = math.exp(-w[i])
+    for t in range(T):
+        exp = r[0, t, i] * ((1 - d ** t) / (1 - d) + u[i])
+        np.testing.assert_allclose(y[t], np.full(N, exp), rtol=1e-13, atol=1e-13)
+
+
+def test_wkv5_no_decay_is_masked_matmul(oracle_mod):
+    """w = 0 (decay 1), u = 1: y = tril(R K^T) V."""
+    T, N = 9, 8
+    g = _rng(62)
+    R, K, V = (g.normal(size=(T, N)) for _ in range(3))
+    y = oracle_mod.wkv5_fwd(R[None], K[None], V[None], np.zeros(N), np.ones(N), H=1)[0]
+    np.testing.assert_allclose(y, np.tril(R @ K.T) @ V, rtol=1e-12, atol=1e-12)
+
+
+def test_wkv5_backward_finite_differences(oracle_mod):
+    B, T, H, N = 2, 6, 2, 3
+    r, k, v, w, u = _wkv5_case(B, T, H, N, seed=63, wlo=-2.0, whi=0.5)
+    dy = _rng(64).normal(size=r.shape)
+    grads = oracle_mod.wkv5_bwd(r, k, v, w, u, dy, H=H)
+    loss = lambda a: float(np.sum(dy * oracle_mod.wkv5_fwd(a["r"], a["k"], a["v"], a["w"], a["u"], H=H)))
+    eps = 1e-6
+    for name, arr, g in zip(("r", "k", "v", "w", "u"), (r, k, v, w, u), grads):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            args = {"r": r, "k": k, "v": v, "w": w, "u": u}
+            hi = arr.copy(); hi[idx] += eps
+            lo = arr.copy(); lo[idx] -= eps
+            args[name] = hi
+            fp = loss(args)
+            args[name] = lo
+            fm = loss(args)
+            num[idx] = (fp - fm) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_wkv5_backward_matches_summed_wkv6_pair_form(oracle_mod):
+    """dr, dk, dv, du equal RWKV-6's at ew = -w; dw[c] is minus the per-token RWKV-6 dw summed over b, t."""
+    B, T, H, N = 2, 9, 1, 4
+    r, k, v, w, u = _wkv5_case(B, T, H, N, seed=65)
+    dy = _rng(66).normal(size=r.shape)
+    dr, dk, dv, dw, du = oracle_mod.wkv5_bwd(r, k, v, w, u, dy, H=H)
+    ew = np.broadcast_to(-w, r.shape[1:]).copy()
+    dw_sum = np.zeros(N); du_sum = np.zeros(N)
+    for b in range(B):
+        e = brute.wkv6_head_grads(r[b], k[b], v[b], ew, u, dy[b], past=True, future=False)
+        for name, got, ref in zip(("dr", "dk", "dv"), (dr[b], dk[b], dv[b]), e[:3]):
+            np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11, err_msg=name)
+        dw_sum -= e[3].sum(0)
+        du_sum += e[4]
+    np.testing.assert_allclose(dw, dw_sum, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(du, du_sum, rtol=1e-11, atol=1e-11)
