@@ -191,6 +191,41 @@ int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, const float 
                      float *dv, float *dw, float *du, wkv_stream_t stream);
 
 /*
+ * wkv5_fwd -- RWKV-5 WKV forward, fp32 ("RWKV Architecture ...", RWKV-5
+ * "Eagle": the matrix state decays by a static, per-channel factor):
+ *     S_t = diag(exp(-w)) S_{t-1} + k_t^T v_t,   y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),
+ * S_{-1} = 0; i.e. wkv6_fwd with the log-decay ew_t = -w at every token.
+ *   r, k, v, y : [B,T,C] float, y overwritten;  w, u : [C] float, w >= 0
+ *   (state row i of head h decays by exp(-w[h*N + i]) per token).
+ * Same sizes, pointer rules, stream semantics and errors as wkv6_fwd.
+ */
+int wkv5_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
+             const float *u, float *y, wkv_stream_t stream);
+
+/*
+ * wkv5_fwd_bf16 -- wkv5_fwd with bfloat16 r, k, v (raw IEEE bf16 bit patterns,
+ * uint16_t); w, u and y stay fp32, and the state is fp32.  Errors as wkv5_fwd.
+ */
+int wkv5_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                  const float *w, const float *u, float *y, wkv_stream_t stream);
+
+/*
+ * wkv5_bwd -- gradients of L = sum(dy * y) for wkv5_fwd (causal), fp32:
+ *   dr, dk, dv : [B,T,C] overwritten;  dw, du : [C] overwritten, summed over B
+ *   and T in a fixed order (deterministic).  dw is w.r.t. the decay rate w of
+ *   wkv5_fwd (dL/dw = -sum_{b,t} dL/d(ew_t)).
+ * workspace: at least wkv5_bwd_workspace_bytes(B,T,C,H) bytes of device memory,
+ * 16-byte aligned, caller-owned (the constant log-decay, its per-token gradient
+ * and the per-batch du partials).  Errors as wkv6_bwd.
+ */
+int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
+             const float *u, const float *dy, float *dr, float *dk, float *dv, float *dw, float *du,
+             void *workspace, size_t workspace_bytes, wkv_stream_t stream);
+
+/* Scratch bytes wkv5_bwd needs: 4 * (2*B*T*C + B*C). */
+size_t wkv5_bwd_workspace_bytes(int B, int T, int C, int H);
+
+/*
  * wkv4_fwd -- RWKV-4 WKV forward, fp32 ("RWKV Architecture ...", The
  * Fundamental Mathematical Duality and The Recurrent Inference Formulation):
  *     y_t = (sum_{s<t} e^{-(t-1-s) w + k_s} v_s + e^{u + k_t} v_t)

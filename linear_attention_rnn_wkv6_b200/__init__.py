@@ -19,7 +19,7 @@ __all__ = [
     "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
     "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
-    "EXPORTED_SYMBOLS", "HEAD_SIZE",
+    "wkv5_fwd", "wkv5_fwd_bf16", "wkv5_bwd", "wkv5_bwd_workspace_bytes", "EXPORTED_SYMBOLS", "HEAD_SIZE",
 ]
 
 HEAD_SIZE = 64
@@ -30,7 +30,8 @@ _LIB = None
 EXPORTED_SYMBOLS = (
     "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
     "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc", "wkv6_fwd_state",
-    "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
+    "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes", "wkv5_fwd", "wkv5_fwd_bf16",
+    "wkv5_bwd", "wkv5_bwd_workspace_bytes",
 )
 
 _I = ctypes.c_int
@@ -53,6 +54,10 @@ _SIGS = {
     "wkv6_bwd_bf16": ([_I] * 5 + [_P] * 11 + [_P, _SZ, _P], _I),
     "wkv4_bwd": ([_I] * 3 + [_P] * 9 + [_P, _SZ, _P], _I),
     "wkv4_bwd_workspace_bytes": ([_I] * 3, _SZ),
+    "wkv5_fwd": ([_I] * 4 + [_P] * 6 + [_P], _I),
+    "wkv5_fwd_bf16": ([_I] * 4 + [_P] * 6 + [_P], _I),
+    "wkv5_bwd": ([_I] * 4 + [_P] * 11 + [_P, _SZ, _P], _I),
+    "wkv5_bwd_workspace_bytes": ([_I] * 4, _SZ),
 }
 
 
@@ -181,6 +186,29 @@ def wkv4_bwd(B, T, C, k, v, w, u, dy, dk, dv, dw, du, workspace, workspace_bytes
     """RWKV-4 WKV backward (fp32): dk, dv [B,T,C]; dw, du [C]."""
     _check("wkv4_bwd", load().wkv4_bwd(B, T, C, _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(dy), _ptr(dk), _ptr(dv),
                                        _ptr(dw), _ptr(du), _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def wkv5_fwd(B, T, C, H, r, k, v, w, u, y, stream=None) -> None:
+    """RWKV-5 WKV forward (fp32): static per-channel decay exp(-w), w and u [C]."""
+    _check("wkv5_fwd", load().wkv5_fwd(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(y),
+                                       _stream(stream)))
+
+
+def wkv5_fwd_bf16(B, T, C, H, r, k, v, w, u, y, stream=None) -> None:
+    """RWKV-5 WKV forward with bf16 r, k, v (raw bf16 bits); w, u and y fp32."""
+    _check("wkv5_fwd_bf16", load().wkv5_fwd_bf16(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(y),
+                                                 _stream(stream)))
+
+
+def wkv5_bwd_workspace_bytes(B, T, C, H) -> int:
+    return int(load().wkv5_bwd_workspace_bytes(B, T, C, H))
+
+
+def wkv5_bwd(B, T, C, H, r, k, v, w, u, dy, dr, dk, dv, dw, du, workspace, workspace_bytes, stream=None) -> None:
+    """RWKV-5 WKV backward (fp32): dr, dk, dv [B,T,C]; dw, du [C]."""
+    _check("wkv5_bwd", load().wkv5_bwd(B, T, C, H, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(dy), _ptr(dr),
+                                       _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du), _ptr(workspace), int(workspace_bytes),
+                                       _stream(stream)))
 
 
 def wkv_status_string(status: int) -> str:

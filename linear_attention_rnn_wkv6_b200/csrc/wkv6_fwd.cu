@@ -34,6 +34,10 @@
 //   rows with a 3-level butterfly reduce-scatter (4 shuffles).
 // * The bonus term (r_t . u . k_t) v_t is a per-token scalar c_t times v_t;
 //   c_t is formed once per token in the transform step.
+// * RWKV-5 ("RWKV Architecture ...", RWKV-5 "Eagle": S_t = exp(-w) . S_{t-1} +
+//   k_t^T v_t with a static per-channel w) runs the same kernel with the
+//   log-decay -w of each channel in shared memory instead of the loaded w tile,
+//   so a stage carries r, k and v only.
 #include "wkv_launch.cuh"
 
 namespace wkv {
@@ -56,6 +60,7 @@ struct FwdSmem {
     float ybuf[TC][CW];      // y_p, this CTA's columns
     float c[TC];             // bonus scalar sum_i r_p u k_p
     float u[kHead];
+    float ew5[kHead];        // static log-decay -w5 (RWKV-5), unused otherwise
     uint32_t renorm_mask;    // bit p set: token p is a renorm step
     alignas(8) uint64_t full[2];
 };
@@ -87,6 +92,7 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     constexpr int NT = 32 * WARPS;
     constexpr int GROUPS = kHead / CW;
     constexpr uint32_t kStageBytes = (3 * TC * kHead + TC * CW) * sizeof(Tin);
+    constexpr uint32_t kWBytes = TC * kHead * sizeof(Tin);
     extern __shared__ unsigned char smem_dyn[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~uintptr_t(127));
 
@@ -103,7 +109,12 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     const int nch = (T + TC - 1) / TC;
     const int nchunks = BIDIR ? 2 * nch : nch;
 
-    if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
+    // RWKV-5: one log-decay per channel for every token; the w map is not read
+    const bool stat = prm.w5 != nullptr;
+    if (tid < kHead) {
+        sm.u[tid] = prm.u[cbase + tid];
+        sm.ew5[tid] = stat ? -prm.w5[cbase + tid] : 0.f;
+    }
     if (tid == 0) {
         prefetch_tensormap(&map_r);
         prefetch_tensormap(&map_k);
@@ -118,10 +129,10 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     auto issue = [&](int g) {
         const ChunkPos cp = chunk_pos(g, nch, T, TC, BIDIR);
         const int s = g & 1;
-        mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+        mbar_arrive_expect_tx(&sm.full[s], stat ? kStageBytes - kWBytes : kStageBytes);
         tma_load_3d(&sm.raw_r[s][0][0], &map_r, cbase, cp.t_lo, b, &sm.full[s]);
         tma_load_3d(&sm.raw_k[s][0][0], &map_k, cbase, cp.t_lo, b, &sm.full[s]);
-        tma_load_3d(&sm.raw_w[s][0][0], &map_w, cbase, cp.t_lo, b, &sm.full[s]);
+        if (!stat) tma_load_3d(&sm.raw_w[s][0][0], &map_w, cbase, cp.t_lo, b, &sm.full[s]);
         tma_load_3d(&sm.raw_v[s][0][0], &map_v, cbase + col0, cp.t_lo, b, &sm.full[s]);
     };
     if (tid == 0) {
@@ -179,11 +190,18 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             return;
         }
 
+        // log-decay of box row `row` (token cp.t_lo + row), channel i; a static decay
+        // applies to tokens inside [0, T) only, like the zero fill of the loaded w
+        auto ew_at = [&](int row, int i) -> float {
+            if (!stat) return to_f32(sm.raw_w[s][row][i]);
+            const int t = cp.t_lo + row;
+            return (t >= 0 && t < T) ? sm.ew5[i] : 0.f;
+        };
         // ---- transform: renorm flags ----
         // a token is a renorm step if some row has |ew| > kTheta / TC (or NaN)
         int bad = 0;
         for (int e = tid; e < TC * kHead; e += NT) {
-            const float ew = to_f32(sm.raw_w[s][e / kHead][e % kHead]);
+            const float ew = ew_at(e / kHead, e % kHead);
             bad |= !(fabsf(ew) <= kTheta / TC);
         }
         const int any_bad = __syncthreads_or(bad);
@@ -192,8 +210,8 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             if (any_bad) {
                 for (int p = 0; p < TC - 1; ++p) {
                     const int row = cp.dir > 0 ? p : TC - 1 - p;
-                    const float e0 = to_f32(sm.raw_w[s][row][lane]);
-                    const float e1 = to_f32(sm.raw_w[s][row][lane + 32]);
+                    const float e0 = ew_at(row, lane);
+                    const float e1 = ew_at(row, lane + 32);
                     const bool bad = !(fabsf(e0) <= kTheta / TC) || !(fabsf(e1) <= kTheta / TC);
                     if (__any_sync(0xffffffffu, bad)) mask |= 1u << p;
                 }
@@ -212,13 +230,13 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             float L = 0.f;
             for (int p = 0; p < p0; ++p) {
                 const int row = cp.dir > 0 ? p : TC - 1 - p;
-                L = ((rmask >> p) & 1u) ? 0.f : L + to_f32(sm.raw_w[s][row][i]);
+                L = ((rmask >> p) & 1u) ? 0.f : L + ew_at(row, i);
             }
             float ew[TH], rr[TH], kk[TH];
 #pragma unroll
             for (int e = 0; e < TH; ++e) {
                 const int p = p0 + e, row = cp.dir > 0 ? p : TC - 1 - p;
-                ew[e] = to_f32(sm.raw_w[s][row][i]);
+                ew[e] = ew_at(row, i);
                 rr[e] = to_f32(sm.raw_r[s][row][i]);
                 kk[e] = to_f32(sm.raw_k[s][row][i]);
             }

@@ -125,15 +125,17 @@ bool bf16_use_tensor_cores() {
     return !(e && std::strcmp(e, "recurrence") == 0);
 }
 
+// w5 (RWKV-5): static per-channel decay rate [C]; then w is ignored (pass w5 for
+// the argument checks) and the recurrence kernel runs with the constant log-decay.
 int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r, const void *k, const void *v,
                const void *w, const float *u, float *y, wkv_stream_t stream, const float *s0 = nullptr,
-               float *sT = nullptr) {
+               float *sT = nullptr, const float *w5 = nullptr) {
     int st = check_wkv6(B, T, C, H, {r, k, v, w, u, y});
     if (st != WKV_OK) return st;
     if (B == 0 || T == 0) return WKV_OK;
     if ((st = check_device()) != WKV_OK) return st;
     CUtensorMap mr, mk, mv, mw;
-    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && bf16_use_tensor_cores()) {
+    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && w5 == nullptr && bf16_use_tensor_cores()) {
         constexpr int kTcChunk = 64;
         CUtensorMap my;
         if (!make_map(&mr, r, true, B, T, C, kHead, kTcChunk, true) ||
@@ -147,12 +149,15 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
                    ? WKV_OK
                    : WKV_ERR_CUDA;
     }
+    // a static decay leaves the w map unread: it is built over r only to be well formed
     if (!make_map(&mr, r, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mk, k, bf16, B, T, C, kHead, kFwdTC) ||
-        !make_map(&mv, v, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mw, w, bf16, B, T, C, kHead, kFwdTC))
+        !make_map(&mv, v, bf16, B, T, C, kHead, kFwdTC) ||
+        !make_map(&mw, w5 != nullptr ? r : w, bf16, B, T, C, kHead, kFwdTC))
         return WKV_ERR_CUDA;
     FwdParams prm{B, T, C, H, u, y};
     prm.s0 = s0;
     prm.sT = sT;
+    prm.w5 = w5;
     return wkv6_fwd_launch(bf16, bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)) ==
                    cudaSuccess
                ? WKV_OK
@@ -240,6 +245,48 @@ int wkv6_bwd_bf16(int B, int T, int C, int H, int bidirectional, const uint16_t 
                   float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes, wkv_stream_t stream) {
     return bwd_common(true, B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, workspace,
                       workspace_bytes, stream);
+}
+
+int wkv5_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
+             const float *u, float *y, wkv_stream_t stream) {
+    return fwd_common(false, false, B, T, C, H, r, k, v, w, u, y, stream, nullptr, nullptr, w);
+}
+
+int wkv5_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                  const float *w, const float *u, float *y, wkv_stream_t stream) {
+    return fwd_common(true, false, B, T, C, H, r, k, v, w, u, y, stream, nullptr, nullptr, w);
+}
+
+size_t wkv5_bwd_workspace_bytes(int B, int T, int C, int H) {
+    (void)H;
+    if (B < 1 || T < 0 || C < 1) return 0;
+    return sizeof(float) * (2 * (size_t)B * T * C + (size_t)B * C);
+}
+
+int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
+             const float *u, const float *dy, float *dr, float *dk, float *dv, float *dw, float *du,
+             void *workspace, size_t workspace_bytes, wkv_stream_t stream) {
+    int st = check_wkv6(B, T, C, H, {r, k, v, w, u, dy, dr, dk, dv, dw, du});
+    if (st != WKV_OK) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (B == 0 || T == 0) {
+        if ((st = check_device()) != WKV_OK) return st;
+        if (cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)C, s) != cudaSuccess) return WKV_ERR_CUDA;
+        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    }
+    if (workspace == nullptr || workspace_bytes < wkv5_bwd_workspace_bytes(B, T, C, H)) return WKV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WKV_ERR_ALIGN;
+    if ((st = check_device()) != WKV_OK) return st;
+    // workspace: the constant log-decay [B][T][C], its per-token gradient [B][T][C],
+    // then the RWKV-6 backward's own [B][C]
+    float *ew = static_cast<float *>(workspace);
+    float *dwtok = ew + (size_t)B * T * C;
+    float *rest = dwtok + (size_t)B * T * C;
+    if (wkv5_expand_launch(B, T, C, w, ew, s) != cudaSuccess) return WKV_ERR_CUDA;
+    st = bwd_common(false, B, T, C, H, 0, r, k, v, ew, u, dy, dr, dk, dv, dwtok, du, rest,
+                    sizeof(float) * (size_t)B * C, stream);
+    if (st != WKV_OK) return st;
+    return wkv5_dw_reduce_launch(B * T, C, dwtok, dw, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
 int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u, float *y,

@@ -13,6 +13,9 @@ struct FwdParams {
     // [B][H][N][N] (row i = key channel, column j = value channel); null = none
     const float *s0 = nullptr;
     float *sT = nullptr;
+    // recurrence kernel only: RWKV-5 static decay rate w5[C] >= 0 (log-decay -w5 at
+    // every token); when set the w tensor map is not read
+    const float *w5 = nullptr;
 };
 
 struct BwdParams {
@@ -41,6 +44,9 @@ constexpr int kBwdMaps = 9;
 cudaError_t wkv6_bwd_launch(bool bf16, bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
                             cudaStream_t stream);
 // RWKV-4 backward; workspace: [B][T][C] + 2 [B][C] floats (see wkv4_bwd_workspace_bytes)
+// RWKV-5 backward helpers: ew[b][t][c] = -w[c]; dw[c] = -sum_rows dwtok[row][c].
+cudaError_t wkv5_expand_launch(int B, int T, int C, const float *w, float *ew, cudaStream_t stream);
+cudaError_t wkv5_dw_reduce_launch(int rows, int C, const float *dwtok, float *dw, cudaStream_t stream);
 cudaError_t wkv4_bwd_launch(int B, int T, int C, const float *k, const float *v, const float *w, const float *u,
                             const float *dy, float *dk, float *dv, float *dw, float *du, float *workspace,
                             cudaStream_t stream);

@@ -156,7 +156,7 @@ class Wkv6Inputs:
     r: np.ndarray      # [B,T,C] float32 (or bf16 bits, uint16)
     k: np.ndarray
     v: np.ndarray
-    w: np.ndarray      # log-decay ew = -exp(w_raw), [B,T,C]
+    w: np.ndarray      # log-decay ew = -exp(w_raw), [B,T,C]; RWKV-5: decay rate [C] float32 (decay exp(-w))
     u: np.ndarray      # [C] float32
     dy: np.ndarray | None = None  # [B,T,C] float32 upstream gradient
     dtype: str = "f32"
@@ -164,7 +164,7 @@ class Wkv6Inputs:
     def as_f64(self, name: str, b=slice(None), c=slice(None)) -> np.ndarray:
         """Exact float64 copy of one input (optionally only batch slice b, channel slice c)."""
         a = getattr(self, name)
-        if name in ("u",):
+        if name in ("u",) or a.ndim == 1:
             return a[c].astype(np.float64)
         a = a[b, :, c] if a.ndim == 3 else a
         if self.dtype == "bf16" and name in ("r", "k", "v", "w"):
@@ -206,6 +206,18 @@ def make_wkv6(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, rkv_std: fl
     return Wkv6Inputs(B, T, C, H, r, k, v, w, u, dy, dtype)
 
 
+def make_wkv5(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, rkv_std: float = 0.5,
+              wraw_lo: float = -6.0, wraw_hi: float = -0.5, u_std: float = 0.5,
+              with_dy: bool = False, dy_std: float = 1.0, dtype: str = "f32") -> Wkv6Inputs:
+    """RWKV-5 inputs: r, k, v, u, dy as make_wkv6 (same streams); the static decay rate
+    w = exp(w_raw) >= 0 per channel, w_raw ~ U(wraw_lo, wraw_hi) (the first C draws of the
+    w_raw stream), float32 also for bf16 r, k, v."""
+    x = make_wkv6(B, T, H, N, seed=seed, rkv_std=rkv_std, wraw_lo=wraw_lo, wraw_hi=wraw_hi, u_std=u_std,
+                  with_dy=with_dy, dy_std=dy_std, dtype=dtype)
+    x.w = np.exp(uniform(seed, STREAM_WRAW, H * N, wraw_lo, wraw_hi)).astype(np.float32)
+    return x
+
+
 def make_state(B: int, H: int, N: int = 64, *, seed: int = 0, std: float = 1.0) -> np.ndarray:
     """An RWKV-6 recurrent state per (b, h): [B,H,N,N] float32 ~ N(0, std^2) (its own stream)."""
     return normal(seed, STREAM_S0, B * H * N * N, std).astype(np.float32).reshape(B, H, N, N)
@@ -243,6 +255,10 @@ WORKLOADS = {
     "wkv4_bwd_f32_b8t1024c768": ("wkv4_bwd", dict(B=8, T=1024, C=768, with_dy=True)),
     # one recurrent decode step for 512 sequences of the long-text head layout (state from make_state)
     "wkv6_decode_f32_b512h32": ("wkv6_decode", dict(B=512, T=1, H=32)),
+    # RWKV-5 (static per-channel decay) forward on the long-text shape, bf16 r, k, v
+    "wkv5_causal_bf16_b8t4096h32": ("wkv5_fwd_bf16", dict(B=8, T=4096, H=32, wraw_lo=-8.0, dtype="bf16")),
+    # RWKV-5 backward, fp32, on the patch-sequence shape
+    "wkv5_bwd_f32_b32t196h12": ("wkv5_bwd", dict(B=32, T=196, H=12, with_dy=True)),
 }
 
 
@@ -250,4 +266,6 @@ def make_workload(name: str, seed: int = 0):
     kind, kw = WORKLOADS[name]
     if kind in ("wkv4_fwd", "wkv4_bwd"):
         return kind, make_wkv4(seed=seed, **kw)
+    if kind.startswith("wkv5"):
+        return kind, make_wkv5(seed=seed, **kw)
     return kind, make_wkv6(seed=seed, **kw)

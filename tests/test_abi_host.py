@@ -147,6 +147,28 @@ def test_wkv4_bwd_argument_errors(lib):
     assert f(2, 8, 32, *q, FAKE, ws, None) == WKV_ERR_ALIGN
 
 
+def test_wkv5_argument_errors(lib):
+    p = [FAKE + 256 * i for i in range(6)]                     # r, k, v, w, u, y
+    for f in (lib.wkv5_fwd, lib.wkv5_fwd_bf16):
+        assert f(-1, 4, 64, 1, *p, None) == WKV_ERR_ARG
+        assert f(1, 4, 64, 2, *p, None) == WKV_ERR_HEADSIZE
+        assert f(1, 4, 64, 1, *(p[:3] + [None] + p[4:]), None) == WKV_ERR_ARG   # w missing
+        q = list(p)
+        q[3] += 4                                              # w misaligned
+        assert f(1, 4, 64, 1, *q, None) == WKV_ERR_ALIGN
+        assert f(0, 4, 64, 1, *p, None) == WKV_OK
+    g = [FAKE + 256 * i for i in range(11)]                    # r, k, v, w, u, dy, dr, dk, dv, dw, du
+    ws = wkv.wkv5_bwd_workspace_bytes(2, 8, 128, 2)
+    assert ws == 4 * (2 * 2 * 8 * 128 + 2 * 128)
+    f = lib.wkv5_bwd
+    assert f(-1, 8, 128, 2, *g, FAKE, ws, None) == WKV_ERR_ARG
+    assert f(2, 8, 128, 4, *g, FAKE, ws, None) == WKV_ERR_HEADSIZE
+    assert f(2, 8, 128, 2, *(g[:9] + [None] + g[10:]), FAKE, ws, None) == WKV_ERR_ARG   # dw missing
+    assert f(2, 8, 128, 2, *g, None, ws, None) == WKV_ERR_WORKSPACE
+    assert f(2, 8, 128, 2, *g, FAKE, ws - 4, None) == WKV_ERR_WORKSPACE
+    assert f(2, 8, 128, 2, *g, FAKE + 4, ws, None) == WKV_ERR_ALIGN
+
+
 def test_wkv4_argument_errors(lib):
     p = [FAKE + 256 * i for i in range(5)]
     assert lib.wkv4_fwd(-1, 4, 32, *p, None) == WKV_ERR_ARG

@@ -1,0 +1,107 @@
+"""GPU parity of the RWKV-5 (static decay) entry points against the oracle's
+RWKV-5 forward and backward, through the C ABI on seeded inputs: fp32 forward
+(relative L2 <= 1e-5), bf16-input forward (<= 2e-2) and fp32 gradients
+(<= 1e-4 per tensor)."""
+import numpy as np
+import pytest
+
+import oracle
+from linear_attention_rnn_wkv6_b200 import synth
+from tests import gpu_cases as gc
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_attention_rnn_wkv6_b200 import build
+    build.build()
+
+
+def _fwd(x):
+    import linear_attention_rnn_wkv6_b200 as wkv
+    r, k, v, w, u = (gc.dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u"))
+    y = gc.empty_nan((x.B, x.T, x.C))
+    fn = wkv.wkv5_fwd_bf16 if x.dtype == "bf16" else wkv.wkv5_fwd
+    fn(x.B, x.T, x.C, x.H, r, k, v, w, u, y)
+    assert wkv.wkv_take_device_faults() == 0
+    return y.cpu().numpy()
+
+
+def _bwd(x):
+    import linear_attention_rnn_wkv6_b200 as wkv
+    t = gc.torch()
+    r, k, v, w, u, dy = (gc.dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u", "dy"))
+    outs = [gc.empty_nan((x.B, x.T, x.C)) for _ in range(3)] + [gc.empty_nan((x.C,)) for _ in range(2)]
+    nb = wkv.wkv5_bwd_workspace_bytes(x.B, x.T, x.C, x.H)
+    ws = t.empty(max(nb, 16), dtype=t.uint8, device="cuda")
+    wkv.wkv5_bwd(x.B, x.T, x.C, x.H, r, k, v, w, u, dy, *outs, ws, nb)
+    assert wkv.wkv_take_device_faults() == 0
+    return tuple(o.cpu().numpy() for o in outs)
+
+
+def _ref_fwd(x):
+    return oracle.wkv5_fwd(*[x.as_f64(n) for n in ("r", "k", "v", "w", "u")], H=x.H)
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (2, 17, 2), (1, 196, 4), (3, 77, 3), (1, 600, 2)])
+def test_wkv5_fwd_f32_matches_oracle(B, T, H):
+    x = synth.make_wkv5(B, T, H, seed=700 + T)
+    y = _fwd(x)
+    assert np.all(np.isfinite(y))
+    assert oracle.rel_l2(y, _ref_fwd(x)) <= gc.TOL_F32_FWD
+
+
+def test_wkv5_fwd_strong_and_zero_decay():
+    """Decay rates up to e^3 (renorm at every token) and exactly 0 (no decay at all)."""
+    x = synth.make_wkv5(2, 130, 2, seed=710, wraw_lo=-4.0, wraw_hi=3.0)
+    x.w[::7] = 0.0
+    assert oracle.rel_l2(_fwd(x), _ref_fwd(x)) <= gc.TOL_F32_FWD
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 5, 1), (2, 150, 2), (1, 1000, 3)])
+def test_wkv5_fwd_bf16_matches_oracle(B, T, H):
+    x = synth.make_wkv5(B, T, H, seed=720 + T, wraw_lo=-8.0, dtype="bf16")
+    y = _fwd(x)
+    assert np.all(np.isfinite(y))
+    assert oracle.rel_l2(y, _ref_fwd(x)) <= gc.TOL_BF16_FWD
+
+
+def test_wkv5_fwd_bf16_workload_sampled():
+    """The long-text shape (B8 T4096 H32, bf16 r, k, v), checked on 3 sampled (b, h) units."""
+    x = synth.make_wkv5(8, 4096, 32, seed=0, wraw_lo=-8.0, dtype="bf16")
+    y = _fwd(x)
+    for b, h in ((0, 0), (3, 17), (7, 31)):
+        sl = slice(64 * h, 64 * h + 64)
+        ref = oracle.wkv5_fwd(*[x.as_f64(n, slice(b, b + 1), sl) for n in ("r", "k", "v", "w", "u")], H=1)
+        assert oracle.rel_l2(y[b:b + 1, :, sl], ref) <= gc.TOL_BF16_FWD, (b, h)
+
+
+def _compare_grads(got, ref):
+    for name, g, e in zip(("dr", "dk", "dv", "dw", "du"), got, ref):
+        assert np.all(np.isfinite(g)), name
+        err = oracle.rel_l2(g, e)
+        assert err <= gc.TOL_F32_GRAD, (name, err)
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (2, 9, 2), (1, 150, 3), (3, 64, 1)])
+def test_wkv5_bwd_matches_oracle(B, T, H):
+    x = synth.make_wkv5(B, T, H, seed=730 + T, with_dy=True)
+    ref = oracle.wkv5_bwd(*[x.as_f64(n) for n in ("r", "k", "v", "w", "u")], x.dy.astype(np.float64), H=x.H)
+    _compare_grads(_bwd(x), ref)
+
+
+def test_wkv5_bwd_deterministic_and_workload_sampled():
+    """The patch-sequence shape (B32 T196 H12): dw and du repeat bit for bit; two heads checked."""
+    x = synth.make_wkv5(32, 196, 12, seed=0, with_dy=True)
+    g1, g2 = _bwd(x), _bwd(x)
+    for a, b in zip(g1, g2):
+        assert np.array_equal(a, b)
+    for h in (0, 11):
+        sl = slice(64 * h, 64 * h + 64)
+        ref = oracle.wkv5_bwd(*[x.as_f64(n, slice(None), sl) for n in ("r", "k", "v", "w", "u")],
+                              x.dy[:, :, sl].astype(np.float64), H=1)
+        _compare_grads(tuple(a[:, :, sl] for a in g1[:3]) + (g1[3][sl], g1[4][sl]), ref)
