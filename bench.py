@@ -37,7 +37,8 @@ UNIT = "tokens/s"
 WORKLOAD_NAME = ("wkv-hot-path step: wkv4_fwd B8xT1024xC768 f32 + wkv6_bidir_fwd B32xT196xH12 f32 + "
                  "wkv6_fwd_bf16 B8xT4096xH32 + wkv6_bwd(bidir) B32xT196xH12 f32, N=64")
 # Workloads outside the step, measured on their own with --only.
-EXTRA_WORKLOADS = ["wkv6_decode_f32_b512h32", "wkv6_bidir_bwd_bf16_b32t196h12", "wkv4_bwd_f32_b8t1024c768"]
+EXTRA_WORKLOADS = ["wkv6_decode_f32_b512h32", "wkv6_bidir_bwd_bf16_b32t196h12", "wkv4_bwd_f32_b8t1024c768",
+                   "wkv5_causal_bf16_b8t4096h32", "wkv5_bwd_f32_b32t196h12"]
 STEP_WORKLOADS = ["wkv4_f32_b8t1024c768", "wkv6_bidir_f32_b32t196h12", "wkv6_causal_bf16_b8t4096h32",
                   "wkv6_bidir_bwd_f32_b32t196h12"]
 N = 64
@@ -64,15 +65,22 @@ ALG = {
     # decode: the state is read and written once per step (2 N^2 floats) next to 5 N floats of token data
     "wkv6_decode_f32_b512h32": dict(bytes_per_unit=2 * N * N * 4 + 5 * N * 4, flops_per_unit=5 * N * N,
                                     bound="hbm"),
+    # RWKV-5: no per-token w; the forward (tensor-core chunked form, like the RWKV-6 bf16
+    # one, so bound by its bytes) reads bf16 r, k, v and writes fp32 y; the causal
+    # backward reads r, k, v, dy and writes dr, dk, dv (w, dw, u, du are per channel)
+    "wkv5_causal_bf16_b8t4096h32": dict(bytes_per_unit=3 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
+    "wkv5_bwd_f32_b32t196h12": dict(bytes_per_unit=7 * N * 4, flops_per_unit=14 * N * N, bound="alu"),
 }
 ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
          "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd",
          "wkv6_decode_f32_b512h32": "wkv6_decode", "wkv6_bidir_bwd_bf16_b32t196h12": "wkv6_bwd_bf16",
-         "wkv4_bwd_f32_b8t1024c768": "wkv4_bwd"}
+         "wkv4_bwd_f32_b8t1024c768": "wkv4_bwd", "wkv5_causal_bf16_b8t4096h32": "wkv5_fwd_bf16",
+         "wkv5_bwd_f32_b32t196h12": "wkv5_bwd"}
 LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
             "wkv6_bidir_bwd_f32_b32t196h12": 2,   # the backward adds a deterministic du reduction
             "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 2,
-            "wkv4_bwd_f32_b8t1024c768": 2}
+            "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
+            "wkv5_bwd_f32_b32t196h12": 4}   # decay expansion, backward, du and dw reductions
 
 
 def units_of(name: str, x) -> int:
@@ -236,7 +244,7 @@ class DeviceWorkload:
         if self.kind.startswith("wkv4"):
             names = ("k", "v", "w", "u") + (("dy",) if self.kind == "wkv4_bwd" else ())
         else:
-            names = ("r", "k", "v", "w", "u") + (("dy",) if self.kind == "wkv6_bwd_bidir" else ())
+            names = ("r", "k", "v", "w", "u") + (("dy",) if self.kind in ("wkv6_bwd_bidir", "wkv5_bwd") else ())
         self.inputs = {n: dev(getattr(x, n)) for n in names}
         if getattr(x, "dtype", "f32") == "bf16" and "dy" in names:
             self.inputs["dy"] = dev(synth.to_bf16_bits(x.dy))   # the bf16 backward takes dy in bf16 too
@@ -245,6 +253,12 @@ class DeviceWorkload:
             self.outputs = [torch.empty(shape, device="cuda") for _ in range(4)] + [torch.empty(x.C, device="cuda")]
             import linear_attention_rnn_wkv6_b200 as wkv
             self.ws_bytes = wkv.wkv6_bwd_workspace_bytes(x.B, x.T, x.C, x.H, 1)
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        elif self.kind == "wkv5_bwd":
+            import linear_attention_rnn_wkv6_b200 as wkv
+            self.outputs = [torch.empty(shape, device="cuda") for _ in range(3)] + \
+                           [torch.empty(x.C, device="cuda") for _ in range(2)]
+            self.ws_bytes = wkv.wkv5_bwd_workspace_bytes(x.B, x.T, x.C, x.H)
             self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
         elif self.kind == "wkv4_bwd":
             import linear_attention_rnn_wkv6_b200 as wkv
@@ -278,6 +292,11 @@ class DeviceWorkload:
                               self.ws, self.ws_bytes, s)
         elif self.kind == "wkv6_bwd_bidir":
             wkv.wkv6_bwd(x.B, x.T, x.C, x.H, 1, i["r"], i["k"], i["v"], i["w"], i["u"], i["dy"], *o,
+                         self.ws, self.ws_bytes, s)
+        elif self.kind == "wkv5_fwd_bf16":
+            wkv.wkv5_fwd_bf16(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], o[0], s)
+        elif self.kind == "wkv5_bwd":
+            wkv.wkv5_bwd(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], i["dy"], *o,
                          self.ws, self.ws_bytes, s)
         elif self.kind == "wkv6_decode":
             # [B,1,C] token tensors are the [B,C] arrays the step reads

@@ -75,6 +75,7 @@ struct TcSmem {
     float psum[2][kTW][kHead];           // per-warp log2-decay sums, by chunk parity
     float pabs[2][kTW][kHead];           // per-warp sums of |log2-decay|
     float u[kHead];
+    float ew5[kHead];                    // RWKV-5 static log-decay -w (natural log), unused otherwise
     float ypart[2][2][kHead];            // exact chunks: per-warp column sums, by token parity
     int flag[4];                         // chunk c is exact-evaluated iff flag[c & 3] == c + 1
     int abort_;
@@ -223,6 +224,7 @@ __device__ __forceinline__ bool is_flagged(const TcSmem &sm, int c) {
 
 }  // namespace
 
+template <bool STATIC>
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
@@ -238,7 +240,12 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
     constexpr uint32_t kStageBytes = 3u * kTile * sizeof(__nv_bfloat16);   // r, k, v
     constexpr uint32_t kWBytes = kTile * sizeof(__nv_bfloat16);
 
-    if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
+    // RWKV-5 (STATIC): a static decay exp(-w5) per channel replaces the loaded w tiles
+    constexpr bool stat = STATIC;
+    if (tid < kHead) {
+        sm.u[tid] = prm.u[cbase + tid];
+        sm.ew5[tid] = stat ? -prm.w5[cbase + tid] : 0.f;
+    }
     if (tid < 4) sm.flag[tid] = 0;
     if (tid == 0) {
         sm.abort_ = 0;
@@ -298,6 +305,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
             static_assert(kWStages == 2, "the w bookkeeping below has two stages");
             int last_w0 = -1, last_w1 = -1;     // latest chunk loaded into each w stage (-1: none)
             auto issue_w = [&](int c) {
+                if (stat) return;   // no w tiles with a static decay
                 const int s = c & 1;
                 if (s) last_w1 = c; else last_w0 = c;
                 mbar_arrive_expect_tx(&sm.wfull[s], kWBytes);
@@ -417,47 +425,60 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
         const int p0 = kTokW * tw;
         const uint32_t in_chunk = (uint32_t)(lane & 3) << 2;
         const uint32_t chunk = (uint32_t)(lane >> 2);
-        const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
         for (int c = 0; c < nch; ++c) {
             const int stg = c % kStages, par = c & 1;
             // a timeout sets the shared abort flag; all transform threads leave
             // together after the named barrier below, so none is left waiting there
             wait_or_abort(sm, &sm.full[stg], (c / kStages) & 1);
-            wait_or_abort(sm, &sm.wfull[c % kWStages], (c / kWStages) & 1);
+            if (!stat) wait_or_abort(sm, &sm.wfull[c % kWStages], (c / kWStages) & 1);
             __nv_bfloat16 *Rb = sm.raw[stg][R_], *Kb = sm.raw[stg][K_];
             const __nv_bfloat16 *Wb = sm.wt[c % kWStages];
             auto off = [&](int e) -> uint32_t {
                 const int p = p0 + e;
                 return (uint32_t)p * 128u + ((chunk ^ (uint32_t)(p & 7)) << 4) + in_chunk;
             };
-            // ---- log2-decay sums of this warp's 16 tokens (signed and absolute)
-            float s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
+            float L0, L1, tot0, tot1, ab0, ab1;
+            if (stat) {
+                const float st0 = sm.ew5[ch] * kLog2e, st1 = sm.ew5[ch + 1] * kLog2e;   // static log2-decay
+                // closed-form decay powers: Lam_p = p ew, the chunk total is L ew; no
+                // w tiles and no sums across the warps (each warp sees every channel)
+                if (*(volatile int *)&sm.abort_) break;
+                L0 = (float)p0 * st0;
+                L1 = (float)p0 * st1;
+                tot0 = (float)kL * st0;
+                tot1 = (float)kL * st1;
+                ab0 = fabsf(tot0);
+                ab1 = fabsf(tot1);
+            } else {
+                // ---- log2-decay sums of this warp's 16 tokens (signed and absolute)
+                float s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < kTokW; ++e) {
-                const uint32_t wv = ld_u32(Wb, off(e));
-                const float x0 = bf_lo(wv) * kLog2e, x1 = bf_hi(wv) * kLog2e;
-                s0 += x0;
-                s1 += x1;
-                a0 += fabsf(x0);
-                a1 += fabsf(x1);
-            }
-            *reinterpret_cast<float2 *>(&sm.psum[par][tw][ch]) = make_float2(s0, s1);
-            *reinterpret_cast<float2 *>(&sm.pabs[par][tw][ch]) = make_float2(a0, a1);
-            named_sync(1, kTT);
-            if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
-            float L0 = 0.f, L1 = 0.f, tot0 = 0.f, tot1 = 0.f, ab0 = 0.f, ab1 = 0.f;
-#pragma unroll
-            for (int q = 0; q < kTW; ++q) {
-                const float2 ps = *reinterpret_cast<const float2 *>(&sm.psum[par][q][ch]);
-                const float2 pa = *reinterpret_cast<const float2 *>(&sm.pabs[par][q][ch]);
-                if (q < tw) {
-                    L0 += ps.x;
-                    L1 += ps.y;
+                for (int e = 0; e < kTokW; ++e) {
+                    const uint32_t wv = ld_u32(Wb, off(e));
+                    const float x0 = bf_lo(wv) * kLog2e, x1 = bf_hi(wv) * kLog2e;
+                    s0 += x0;
+                    s1 += x1;
+                    a0 += fabsf(x0);
+                    a1 += fabsf(x1);
                 }
-                tot0 += ps.x;
-                tot1 += ps.y;
-                ab0 += pa.x;
-                ab1 += pa.y;
+                *reinterpret_cast<float2 *>(&sm.psum[par][tw][ch]) = make_float2(s0, s1);
+                *reinterpret_cast<float2 *>(&sm.pabs[par][tw][ch]) = make_float2(a0, a1);
+                named_sync(1, kTT);
+                if (*(volatile int *)&sm.abort_) break;        // uniform: every thread passed the barrier
+                L0 = 0.f, L1 = 0.f, tot0 = 0.f, tot1 = 0.f, ab0 = 0.f, ab1 = 0.f;
+#pragma unroll
+                for (int q = 0; q < kTW; ++q) {
+                    const float2 ps = *reinterpret_cast<const float2 *>(&sm.psum[par][q][ch]);
+                    const float2 pa = *reinterpret_cast<const float2 *>(&sm.pabs[par][q][ch]);
+                    if (q < tw) {
+                        L0 += ps.x;
+                        L1 += ps.y;
+                    }
+                    tot0 += ps.x;
+                    tot1 += ps.y;
+                    ab0 += pa.x;
+                    ab1 += pa.y;
+                }
             }
             // sum |ew| bounds every |Lam_p| of the chunk; every warp reads the same
             // sums in the same order, so all four reach the same verdict
@@ -472,7 +493,11 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 float bp[8];
                 // flagged is warp-uniform: keeping the branch outside the token loop
                 // leaves one straight-line body whose loads and exponentials overlap
+                // per-channel constants are re-read from shared memory here rather than
+                // held in registers across the chunk loop
+                const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
                 if (!flagged) {
+                    const float st0 = sm.ew5[ch] * kLog2e, st1 = sm.ew5[ch + 1] * kLog2e;
                     // four tokens at a time, loads first: the in-place stores below may
                     // alias them as far as the compiler can tell, so loads issued after a
                     // store would serialise (batches of four keep the registers in bounds)
@@ -484,7 +509,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                             const uint32_t o = off(8 * half + 4 * sb + e);
                             rv[e] = ld_u32(Rb, o);
                             kv[e] = ld_u32(Kb, o);
-                            wv[e] = ld_u32(Wb, o);
+                            wv[e] = stat ? 0u : ld_u32(Wb, o);
                         }
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -492,8 +517,8 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                             const float r0 = bf_lo(rv[e]), r1 = bf_hi(rv[e]), k0 = bf_lo(kv[e]), k1 = bf_hi(kv[e]);
                             bp[4 * sb + e] = fmaf(r0 * u0, k0, r1 * u1 * k1);
                             const float q0 = r0 * fast_exp2(L0), q1 = r1 * fast_exp2(L1);
-                            L0 += bf_lo(wv[e]) * kLog2e;
-                            L1 += bf_hi(wv[e]) * kLog2e;
+                            L0 += stat ? st0 : bf_lo(wv[e]) * kLog2e;
+                            L1 += stat ? st1 : bf_hi(wv[e]) * kLog2e;
                             st_u32(Rb, o, pack_bf16(q0, q1));
                             st_u32(Kb, o, pack_bf16(k0 * fast_exp2(-L0), k1 * fast_exp2(-L1)));
                         }
@@ -632,7 +657,8 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                 const __nv_bfloat16 *V = sm.raw[stg][V_], *W = sm.wt[c % kWStages];
                 for (int p = 0; p < kL; ++p) {
                     if (!yrole) {
-                        const float rr = raw_at(R, p, row), dd = __expf(raw_at(W, p, row)), kk = raw_at(Kr, p, row);
+                        const float rr = raw_at(R, p, row), kk = raw_at(Kr, p, row);
+                        const float dd = __expf(stat ? sm.ew5[row] : raw_at(W, p, row));
 #pragma unroll 1
                         for (int m = 0; m < 4; ++m) {
                             float s16[16];
@@ -715,12 +741,12 @@ cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, con
                                const CUtensorMap &mw, const CUtensorMap &my, const FwdParams &prm,
                                cudaStream_t stream) {
     const size_t smem = sizeof(TcSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(wkv6_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = prm.w5 != nullptr ? wkv6_fwd_tc_kernel<true> : wkv6_fwd_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(wkv6_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    wkv6_fwd_tc_kernel<<<(unsigned)(prm.B * prm.H), kThreads, smem, stream>>>(mr, mk, mv, mw, my, prm);
+    kern<<<(unsigned)(prm.B * prm.H), kThreads, smem, stream>>>(mr, mk, mv, mw, my, prm);
     return cudaGetLastError();
 }
 

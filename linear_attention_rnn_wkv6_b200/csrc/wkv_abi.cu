@@ -135,16 +135,17 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
     if (B == 0 || T == 0) return WKV_OK;
     if ((st = check_device()) != WKV_OK) return st;
     CUtensorMap mr, mk, mv, mw;
-    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && w5 == nullptr && bf16_use_tensor_cores()) {
+    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && bf16_use_tensor_cores()) {
         constexpr int kTcChunk = 64;
         CUtensorMap my;
         if (!make_map(&mr, r, true, B, T, C, kHead, kTcChunk, true) ||
             !make_map(&mk, k, true, B, T, C, kHead, kTcChunk, true) ||
             !make_map(&mv, v, true, B, T, C, kHead, kTcChunk, true) ||
-            !make_map(&mw, w, true, B, T, C, kHead, kTcChunk, true) ||
+            !make_map(&mw, w5 != nullptr ? r : w, true, B, T, C, kHead, kTcChunk, true) ||
             !make_map(&my, y, false, B, T, C, kHead / 2, kTcChunk, true))
             return WKV_ERR_CUDA;
         FwdParams prm{B, T, C, H, u, y};
+        prm.w5 = w5;
         return wkv6_fwd_tc_launch(mr, mk, mv, mw, my, prm, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                    ? WKV_OK
                    : WKV_ERR_CUDA;

@@ -13,8 +13,8 @@ struct FwdParams {
     // [B][H][N][N] (row i = key channel, column j = value channel); null = none
     const float *s0 = nullptr;
     float *sT = nullptr;
-    // recurrence kernel only: RWKV-5 static decay rate w5[C] >= 0 (log-decay -w5 at
-    // every token); when set the w tensor map is not read
+    // RWKV-5 static decay rate w5[C] >= 0 (log-decay -w5 at every token); when set
+    // the w tensor map is not read
     const float *w5 = nullptr;
 };
 

@@ -36,21 +36,41 @@ def make_case(spec: str):
     kw = dict(kw)
     if len(parts) == 3:
         kw["B"], kw["T"] = int(parts[1]), int(parts[2])
-    if kind == "wkv4_fwd":
-        x = synth.make_wkv4(kw["B"], kw["T"], kw["C"], seed=0)
-        ins = [_dev(getattr(x, n)) for n in ("k", "v", "w", "u")]
-        y = torch.empty(x.B, x.T, x.C, device="cuda")
-        return f"{name} B={x.B} T={x.T}", lambda: wkv.wkv4_fwd(x.B, x.T, x.C, *ins, y)
+    if kind in ("wkv4_fwd", "wkv4_bwd"):
+        x = synth.make_wkv4(kw["B"], kw["T"], kw["C"], seed=0, with_dy=kind == "wkv4_bwd")
+        label = f"{name} B={x.B} T={x.T}"
+        if kind == "wkv4_fwd":
+            ins = [_dev(getattr(x, n)) for n in ("k", "v", "w", "u")]
+            y = torch.empty(x.B, x.T, x.C, device="cuda")
+            return label, lambda: wkv.wkv4_fwd(x.B, x.T, x.C, *ins, y)
+        ins = [_dev(getattr(x, n)) for n in ("k", "v", "w", "u", "dy")]
+        outs = [torch.empty(x.B, x.T, x.C, device="cuda") for _ in range(2)] + \
+               [torch.empty(x.C, device="cuda") for _ in range(2)]
+        nb = wkv.wkv4_bwd_workspace_bytes(x.B, x.T, x.C)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        return label, lambda: wkv.wkv4_bwd(x.B, x.T, x.C, *ins, *outs, ws, nb)
     args = {k: v for k, v in kw.items() if k not in ("B", "T", "H")}
-    x = synth.make_wkv6(kw["B"], kw["T"], kw["H"], seed=0, **args)
+    make = synth.make_wkv5 if kind.startswith("wkv5") else synth.make_wkv6
+    x = make(kw["B"], kw["T"], kw["H"], seed=0, **args)
     label = f"{name} B={x.B} T={x.T} H={x.H}"
     if kind.startswith("wkv6_bwd"):
         bidir = kind == "wkv6_bwd_bidir"
-        ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u", "dy")]
+        ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u")]
         outs = [torch.empty(x.B, x.T, x.C, device="cuda") for _ in range(4)] + [torch.empty(x.C, device="cuda")]
         nb = wkv.wkv6_bwd_workspace_bytes(x.B, x.T, x.C, x.H, bidir)
         ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
-        return label, lambda: wkv.wkv6_bwd(x.B, x.T, x.C, x.H, bidir, *ins, *outs, ws, nb)
+        if x.dtype == "bf16":   # the bf16 backward takes dy in bf16 too
+            dy = _dev(synth.to_bf16_bits(x.dy))
+            return label, lambda: wkv.wkv6_bwd_bf16(x.B, x.T, x.C, x.H, bidir, *ins, dy, *outs, ws, nb)
+        dy = _dev(x.dy)
+        return label, lambda: wkv.wkv6_bwd(x.B, x.T, x.C, x.H, bidir, *ins, dy, *outs, ws, nb)
+    if kind == "wkv5_bwd":
+        ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u", "dy")]
+        outs = [torch.empty(x.B, x.T, x.C, device="cuda") for _ in range(3)] + \
+               [torch.empty(x.C, device="cuda") for _ in range(2)]
+        nb = wkv.wkv5_bwd_workspace_bytes(x.B, x.T, x.C, x.H)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        return label, lambda: wkv.wkv5_bwd(x.B, x.T, x.C, x.H, *ins, *outs, ws, nb)
     ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u")]
     y = torch.empty(x.B, x.T, x.C, device="cuda")
     if kind == "wkv6_decode":
