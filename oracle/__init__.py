@@ -48,8 +48,9 @@ def _configure(lib):
     lib.oracle_wkv4_bwd.argtypes = [I, I, I] + [_DP] * 9
     lib.oracle_wkv5_fwd.argtypes = [I, I, I, I] + [_DP] * 6
     lib.oracle_wkv5_bwd.argtypes = [I, I, I, I] + [_DP] * 11
+    lib.oracle_wkv6_fwd_fused.argtypes = [I, I, I, I, I] + [_DP] * 9 + [ctypes.c_double, _DP]
     for f in (lib.oracle_wkv6_fwd, lib.oracle_wkv6_fwd_state, lib.oracle_wkv6_bwd, lib.oracle_wkv4_fwd,
-              lib.oracle_wkv4_bwd, lib.oracle_wkv5_fwd, lib.oracle_wkv5_bwd):
+              lib.oracle_wkv4_bwd, lib.oracle_wkv5_fwd, lib.oracle_wkv5_bwd, lib.oracle_wkv6_fwd_fused):
         f.restype = ctypes.c_int
     return lib
 
@@ -155,6 +156,19 @@ class Oracle:
             raise ValueError(f"oracle_wkv5_bwd failed ({rc})")
         return tuple(outs)
 
+    def wkv6_fwd_fused(self, r, k, v, ww, w_base, u, g, gn_w, gn_b, eps: float, H: int,
+                       bidirectional: bool = False) -> np.ndarray:
+        """RWKV-6 forward at ew = -exp(w_base + ww), then per-head group norm (gn_w, gn_b, eps)
+        times the gate g.  r,k,v,ww,g: [B,T,C]; w_base,u,gn_w,gn_b: [C] -> out [B,T,C]."""
+        r, k, v, ww, w_base, u, g, gn_w, gn_b = map(_d, (r, k, v, ww, w_base, u, g, gn_w, gn_b))
+        B, T, C = r.shape
+        out = np.zeros((B, T, C), dtype=np.float64)
+        rc = self._lib.oracle_wkv6_fwd_fused(B, T, C, H, int(bidirectional), _p(r), _p(k), _p(v), _p(ww),
+                                             _p(w_base), _p(u), _p(g), _p(gn_w), _p(gn_b), float(eps), _p(out))
+        if rc != 0:
+            raise ValueError(f"oracle_wkv6_fwd_fused failed ({rc})")
+        return out
+
 
 def _default() -> Oracle:
     global _lib
@@ -189,6 +203,10 @@ def wkv5_fwd(r, k, v, w, u, H: int) -> np.ndarray:
 
 def wkv5_bwd(r, k, v, w, u, dy, H: int):
     return _default().wkv5_bwd(r, k, v, w, u, dy, H)
+
+
+def wkv6_fwd_fused(r, k, v, ww, w_base, u, g, gn_w, gn_b, eps: float, H: int, bidirectional: bool = False):
+    return _default().wkv6_fwd_fused(r, k, v, ww, w_base, u, g, gn_w, gn_b, eps, H, bidirectional)
 
 
 def source() -> str:

@@ -266,6 +266,51 @@ int oracle_wkv6_bwd(int B, int T, int C, int H, int bidirectional,
 }
 
 /* ------------------------------------------------------------------------ */
+/* RWKV-6 forward with its decay prologue and its norm/gate epilogue          */
+/* (RWKV Architecture page, RWKV-6 "Finch": w_t = w_base + tanh(x_t W1) W2;    */
+/* RWKV-5 "Eagle": group normalisation over each head, SiLU output gating;    */
+/* WKV processing-images page: the kernel is handed ew = -exp(w), and the     */
+/* block passes the WKV output and the gate g on to its output stage).        */
+/* The dense projections stay outside: the inputs are ww = tanh(x W1) W2 and  */
+/* g = silu(x W_g), both [B][T][C].  Per (b, t, head h), with y the RWKV-6     */
+/* output at ew = -exp(w_base + ww):                                          */
+/*   mu = mean_i y[h*N+i],  var = mean_i (y[h*N+i] - mu)^2                    */
+/*   out[c] = ((y[c] - mu) / sqrt(var + eps) * gn_w[c] + gn_b[c]) * g[c]      */
+/* ------------------------------------------------------------------------ */
+int oracle_wkv6_fwd_fused(int B, int T, int C, int H, int bidirectional,
+                          const double *r, const double *k, const double *v, const double *ww,
+                          const double *w_base, const double *u, const double *g,
+                          const double *gn_w, const double *gn_b, double eps, double *out)
+{
+    if (B < 0 || T < 0 || H < 1 || C % H != 0) return -1;
+    const int N = C / H;
+    const size_t n = (size_t)B * T * C;
+    double *ew = (double *)malloc(sizeof(double) * (n ? n : 1));
+    double *y = (double *)malloc(sizeof(double) * (n ? n : 1));
+    if (!ew || !y) { free(ew); free(y); return -2; }
+    for (size_t e = 0; e < n; ++e) ew[e] = -exp(w_base[e % C] + ww[e]);
+    int rc = oracle_wkv6_fwd(B, T, C, H, bidirectional, r, k, v, ew, u, y);
+    if (rc == 0)
+        for (size_t row = 0; row < (size_t)B * T; ++row)
+            for (int h = 0; h < H; ++h) {
+                const double *yh = y + row * C + (size_t)h * N;
+                double mu = 0.0, var = 0.0;
+                for (int i = 0; i < N; ++i) mu += yh[i];
+                mu /= N;
+                for (int i = 0; i < N; ++i) var += (yh[i] - mu) * (yh[i] - mu);
+                var /= N;
+                const double inv = 1.0 / sqrt(var + eps);
+                for (int i = 0; i < N; ++i) {
+                    const size_t c = (size_t)h * N + i;
+                    out[row * C + c] = ((yh[i] - mu) * inv * gn_w[c] + gn_b[c]) * g[row * C + c];
+                }
+            }
+    free(ew);
+    free(y);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
 /* RWKV-5 forward (RWKV Architecture page, RWKV-5 "Eagle": the matrix state   */
 /* decays by the static, per-channel factor exp(-w), S_t = exp(-w) . S_{t-1}  */
 /* + k_t^T v_t).  The readout is RWKV-6's with that constant decay:           */

@@ -61,6 +61,15 @@ MUTATIONS = [
      [pins.test_wkv5_backward_finite_differences, pins.test_wkv5_backward_matches_summed_wkv6_pair_form]),
     ("wkv5_bwd_adjoint_without_decay", "A[i * N + j] = rt[i] * gt[j] + exp(-wh[i]) * A[i * N + j];",
      "A[i * N + j] = rt[i] * gt[j] + A[i * N + j];", 0, [pins.test_wkv5_backward_finite_differences]),
+    ("fused_no_mean", "for (int i = 0; i < N; ++i) mu += yh[i];", "for (int i = 0; i < N; ++i) mu += 0.0 * yh[i];", 0,
+     [pins.test_fused_rows_are_normalised_per_head, lambda o: pins.test_fused_matches_library_group_norm(o, False)]),
+    ("fused_gate_before_bias", "out[row * C + c] = ((yh[i] - mu) * inv * gn_w[c] + gn_b[c]) * g[row * C + c];",
+     "out[row * C + c] = (yh[i] - mu) * inv * gn_w[c] * g[row * C + c] + gn_b[c];", 0,
+     [pins.test_fused_scale_invariance_and_affine_order]),
+    ("fused_decay_sign", "ew[e] = -exp(w_base[e % C] + ww[e]);", "ew[e] = -exp(w_base[e % C] - ww[e]);", 0,
+     [pins.test_fused_prologue_moves_constant_between_base_and_lora]),
+    ("fused_var_without_eps", "const double inv = 1.0 / sqrt(var + eps);", "const double inv = 1.0 / sqrt(var);", 0,
+     [lambda o: pins.test_fused_matches_library_group_norm(o, True)]),
     ("wkv4_no_shift_update", "                p = q;\n", "", 0,
      [lambda o: pins.test_wkv4_recurrence_matches_ratio_of_sums(o, 1, 40, 4), pins.test_wkv4_large_keys_stay_finite]),
 ]

@@ -499,3 +499,70 @@ def test_wkv5_backward_matches_summed_wkv6_pair_form(oracle_mod):
         du_sum += e[4]
     np.testing.assert_allclose(dw, dw_sum, rtol=1e-11, atol=1e-11)
     np.testing.assert_allclose(du, du_sum, rtol=1e-11, atol=1e-11)
+
+
+# ---------------------------------------------------------------- fused prologue / epilogue
+
+def _fused_case(B, T, H, N, seed):
+    g = _rng(seed)
+    C = H * N
+    r, k, v = (g.normal(0, 0.7, (B, T, C)) for _ in range(3))
+    ww = g.normal(0, 0.5, (B, T, C))                 # LoRA part of the decay pre-activation
+    wb = g.uniform(-4.0, -0.5, C)                    # w_base
+    u = g.normal(0, 0.7, C)
+    gate = g.normal(0, 1.0, (B, T, C))
+    gn_w, gn_b = g.normal(1.0, 0.3, C), g.normal(0, 0.3, C)
+    return r, k, v, ww, wb, u, gate, gn_w, gn_b
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_fused_matches_library_group_norm(oracle_mod, bidir):
+    """out = torch group_norm(y, H groups, gn_w, gn_b, eps) * g, with y the pinned RWKV-6
+    forward at ew = -exp(w_base + ww)."""
+    torch = pytest.importorskip("torch")
+    B, T, H, N = 2, 11, 3, 8
+    r, k, v, ww, wb, u, gate, gn_w, gn_b = _fused_case(B, T, H, N, seed=70 + bidir)
+    eps = 1e-3
+    out = oracle_mod.wkv6_fwd_fused(r, k, v, ww, wb, u, gate, gn_w, gn_b, eps, H=H, bidirectional=bidir)
+    y = oracle_mod.wkv6_fwd(r, k, v, -np.exp(wb + ww), u, H=H, bidirectional=bidir)
+    gn = torch.nn.functional.group_norm(torch.from_numpy(y.reshape(B * T, H * N)), H,
+                                        torch.from_numpy(gn_w), torch.from_numpy(gn_b), eps).numpy()
+    np.testing.assert_allclose(out, gn.reshape(B, T, H * N) * gate, rtol=1e-12, atol=1e-12)
+
+
+def test_fused_rows_are_normalised_per_head(oracle_mod):
+    """Unit affine and gate: every (token, head) row has mean 0 and mean square var / (var + eps)."""
+    B, T, H, N = 1, 9, 2, 16
+    r, k, v, ww, wb, u, _, _, _ = _fused_case(B, T, H, N, seed=72)
+    C = H * N
+    out = oracle_mod.wkv6_fwd_fused(r, k, v, ww, wb, u, np.ones((B, T, C)), np.ones(C), np.zeros(C), 1e-14, H=H)
+    rows = out.reshape(B * T, H, N)
+    assert np.max(np.abs(rows.mean(-1))) <= 1e-12
+    np.testing.assert_allclose((rows ** 2).mean(-1), 1.0, rtol=1e-9)
+
+
+def test_fused_scale_invariance_and_affine_order(oracle_mod):
+    """Scaling v by a > 0 scales y and leaves the normalised output unchanged (eps -> 0); the
+    affine map acts before the gate: out(gn_w, gn_b, g) = (out(1, 0, 1) * gn_w + gn_b) * g."""
+    B, T, H, N = 2, 7, 2, 8
+    r, k, v, ww, wb, u, gate, gn_w, gn_b = _fused_case(B, T, H, N, seed=73)
+    C = H * N
+    one, zero = np.ones(C), np.zeros(C)
+    base = oracle_mod.wkv6_fwd_fused(r, k, v, ww, wb, u, np.ones_like(gate), one, zero, 1e-14, H=H)
+    scaled = oracle_mod.wkv6_fwd_fused(r, k, 3.5 * v, ww, wb, u, np.ones_like(gate), one, zero, 1e-14, H=H)
+    np.testing.assert_allclose(scaled, base, rtol=1e-8, atol=1e-9)
+    full = oracle_mod.wkv6_fwd_fused(r, k, v, ww, wb, u, gate, gn_w, gn_b, 1e-14, H=H)
+    np.testing.assert_allclose(full, (base * gn_w + gn_b) * gate, rtol=1e-12, atol=1e-12)
+
+
+def test_fused_prologue_moves_constant_between_base_and_lora(oracle_mod):
+    """Only w_base + ww enters the decay: shifting a per-channel constant from one to the other
+    changes nothing, and a different sum changes the output."""
+    B, T, H, N = 1, 8, 2, 4
+    r, k, v, ww, wb, u, gate, gn_w, gn_b = _fused_case(B, T, H, N, seed=74)
+    shift = _rng(75).normal(size=H * N)
+    a = oracle_mod.wkv6_fwd_fused(r, k, v, ww, wb, u, gate, gn_w, gn_b, 1e-5, H=H)
+    b = oracle_mod.wkv6_fwd_fused(r, k, v, ww + shift, wb - shift, u, gate, gn_w, gn_b, 1e-5, H=H)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+    c = oracle_mod.wkv6_fwd_fused(r, k, v, ww + shift, wb, u, gate, gn_w, gn_b, 1e-5, H=H)
+    assert np.max(np.abs(c - a)) > 1e-3
