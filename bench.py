@@ -38,7 +38,7 @@ WORKLOAD_NAME = ("wkv-hot-path step: wkv4_fwd B8xT1024xC768 f32 + wkv6_bidir_fwd
                  "wkv6_fwd_bf16 B8xT4096xH32 + wkv6_bwd(bidir) B32xT196xH12 f32, N=64")
 # Workloads outside the step, measured on their own with --only.
 EXTRA_WORKLOADS = ["wkv6_decode_f32_b512h32", "wkv6_bidir_bwd_bf16_b32t196h12", "wkv4_bwd_f32_b8t1024c768",
-                   "wkv5_causal_bf16_b8t4096h32", "wkv5_bwd_f32_b32t196h12"]
+                   "wkv5_causal_bf16_b8t4096h32", "wkv5_bwd_f32_b32t196h12", "wkv6_bidir_fused_f32_b32t196h12"]
 STEP_WORKLOADS = ["wkv4_f32_b8t1024c768", "wkv6_bidir_f32_b32t196h12", "wkv6_causal_bf16_b8t4096h32",
                   "wkv6_bidir_bwd_f32_b32t196h12"]
 N = 64
@@ -70,17 +70,20 @@ ALG = {
     # backward reads r, k, v, dy and writes dr, dk, dv (w, dw, u, du are per channel)
     "wkv5_causal_bf16_b8t4096h32": dict(bytes_per_unit=3 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
     "wkv5_bwd_f32_b32t196h12": dict(bytes_per_unit=7 * N * 4, flops_per_unit=14 * N * N, bound="alu"),
+    # fused forward: r, k, v, ww and the gate in, the normalised and gated output out
+    "wkv6_bidir_fused_f32_b32t196h12": dict(bytes_per_unit=6 * N * 4, flops_per_unit=10 * N * N, bound="alu"),
 }
 ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
          "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd",
          "wkv6_decode_f32_b512h32": "wkv6_decode", "wkv6_bidir_bwd_bf16_b32t196h12": "wkv6_bwd_bf16",
          "wkv4_bwd_f32_b8t1024c768": "wkv4_bwd", "wkv5_causal_bf16_b8t4096h32": "wkv5_fwd_bf16",
-         "wkv5_bwd_f32_b32t196h12": "wkv5_bwd"}
+         "wkv5_bwd_f32_b32t196h12": "wkv5_bwd", "wkv6_bidir_fused_f32_b32t196h12": "wkv6_fwd_fused"}
 LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
             "wkv6_bidir_bwd_f32_b32t196h12": 2,   # the backward adds a deterministic du reduction
             "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 2,
             "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
-            "wkv5_bwd_f32_b32t196h12": 4}   # decay expansion, backward, du and dw reductions
+            "wkv5_bwd_f32_b32t196h12": 4,   # decay expansion, backward, du and dw reductions
+            "wkv6_bidir_fused_f32_b32t196h12": 1}
 
 
 def units_of(name: str, x) -> int:
@@ -243,6 +246,8 @@ class DeviceWorkload:
         self.host_inputs = {}
         if self.kind.startswith("wkv4"):
             names = ("k", "v", "w", "u") + (("dy",) if self.kind == "wkv4_bwd" else ())
+        elif self.kind == "wkv6_fwd_fused":
+            names = ("r", "k", "v", "ww", "w_base", "u", "g", "gn_w", "gn_b")
         else:
             names = ("r", "k", "v", "w", "u") + (("dy",) if self.kind in ("wkv6_bwd_bidir", "wkv5_bwd") else ())
         self.inputs = {n: dev(getattr(x, n)) for n in names}
@@ -293,6 +298,9 @@ class DeviceWorkload:
         elif self.kind == "wkv6_bwd_bidir":
             wkv.wkv6_bwd(x.B, x.T, x.C, x.H, 1, i["r"], i["k"], i["v"], i["w"], i["u"], i["dy"], *o,
                          self.ws, self.ws_bytes, s)
+        elif self.kind == "wkv6_fwd_fused":
+            wkv.wkv6_fwd_fused(x.B, x.T, x.C, x.H, x.bidir, *(i[n] for n in ("r", "k", "v", "ww", "w_base", "u", "g",
+                                                                            "gn_w", "gn_b")), x.eps, o[0], s)
         elif self.kind == "wkv5_fwd_bf16":
             wkv.wkv5_fwd_bf16(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], o[0], s)
         elif self.kind == "wkv5_bwd":

@@ -191,6 +191,33 @@ int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, const float 
                      float *dv, float *dw, float *du, wkv_stream_t stream);
 
 /*
+ * wkv6_fwd_fused -- RWKV-6 forward (causal, or bidirectional when
+ * bidirectional != 0) with its decay prologue and its output epilogue fused
+ * in, fp32.  RWKV-6 computes the decay pre-activation from a base and a
+ * low-rank term, w_t = w_base + tanh(x_t W1) W2 ("RWKV Architecture ...",
+ * RWKV-6 "Finch"), the kernel's log-decay is ew = -exp(w_t) ("How the WKV ...
+ * Processes Images", CUDA wrapper), and each head's output is group-normalised
+ * and multiplied by the SiLU gate (RWKV-5 "Eagle": multi-head normalisation and
+ * SiLU output gating; the spatial-mix block passes y and g on together).  The
+ * dense projections stay with the caller; this call takes their results:
+ *   r, k, v    : [B,T,C] float
+ *   ww         : [B,T,C] float, the low-rank term tanh(x W1) W2
+ *   w_base     : [C] float;   u : [C] float (bonus)
+ *   g          : [B,T,C] float, the gate (e.g. silu(x W_g))
+ *   gn_weight, gn_bias : [C] float;   eps : float > 0
+ *   out        : [B,T,C] float, overwritten with
+ *     out[b,t,c] = ((y[b,t,c] - mu) / sqrt(var + eps) * gn_weight[c] + gn_bias[c]) * g[b,t,c]
+ *   where y is wkv6_fwd (or wkv6_bidir_fwd) at w = -exp(w_base + ww), and mu and
+ *   var are the mean and the (biased) variance of y over the N channels of c's
+ *   head at (b, t).  Neither the log-decay nor y is written to memory.
+ * Same sizes, pointer rules and errors as wkv6_fwd; eps <= 0 or not finite gives
+ * WKV_ERR_ARG.
+ */
+int wkv6_fwd_fused(int B, int T, int C, int H, int bidirectional, const float *r, const float *k, const float *v,
+                   const float *ww, const float *w_base, const float *u, const float *g, const float *gn_weight,
+                   const float *gn_bias, float eps, float *out, wkv_stream_t stream);
+
+/*
  * wkv5_fwd -- RWKV-5 WKV forward, fp32 ("RWKV Architecture ...", RWKV-5
  * "Eagle": the matrix state decays by a static, per-channel factor):
  *     S_t = diag(exp(-w)) S_{t-1} + k_t^T v_t,   y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),

@@ -19,7 +19,8 @@ __all__ = [
     "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
     "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
-    "wkv5_fwd", "wkv5_fwd_bf16", "wkv5_bwd", "wkv5_bwd_workspace_bytes", "EXPORTED_SYMBOLS", "HEAD_SIZE",
+    "wkv5_fwd", "wkv5_fwd_bf16", "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused", "EXPORTED_SYMBOLS",
+    "HEAD_SIZE",
 ]
 
 HEAD_SIZE = 64
@@ -31,7 +32,7 @@ EXPORTED_SYMBOLS = (
     "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
     "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc", "wkv6_fwd_state",
     "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes", "wkv5_fwd", "wkv5_fwd_bf16",
-    "wkv5_bwd", "wkv5_bwd_workspace_bytes",
+    "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused",
 )
 
 _I = ctypes.c_int
@@ -58,6 +59,7 @@ _SIGS = {
     "wkv5_fwd_bf16": ([_I] * 4 + [_P] * 6 + [_P], _I),
     "wkv5_bwd": ([_I] * 4 + [_P] * 11 + [_P, _SZ, _P], _I),
     "wkv5_bwd_workspace_bytes": ([_I] * 4, _SZ),
+    "wkv6_fwd_fused": ([_I] * 5 + [_P] * 9 + [ctypes.c_float, _P, _P], _I),
 }
 
 
@@ -186,6 +188,14 @@ def wkv4_bwd(B, T, C, k, v, w, u, dy, dk, dv, dw, du, workspace, workspace_bytes
     """RWKV-4 WKV backward (fp32): dk, dv [B,T,C]; dw, du [C]."""
     _check("wkv4_bwd", load().wkv4_bwd(B, T, C, _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(dy), _ptr(dk), _ptr(dv),
                                        _ptr(dw), _ptr(du), _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def wkv6_fwd_fused(B, T, C, H, bidirectional, r, k, v, ww, w_base, u, g, gn_weight, gn_bias, eps, out,
+                   stream=None) -> None:
+    """RWKV-6 forward at ew = -exp(w_base + ww), then per-head group norm and the gate g (fp32)."""
+    _check("wkv6_fwd_fused", load().wkv6_fwd_fused(B, T, C, H, int(bool(bidirectional)), _ptr(r), _ptr(k), _ptr(v),
+                                                   _ptr(ww), _ptr(w_base), _ptr(u), _ptr(g), _ptr(gn_weight),
+                                                   _ptr(gn_bias), float(eps), _ptr(out), _stream(stream)))
 
 
 def wkv5_fwd(B, T, C, H, r, k, v, w, u, y, stream=None) -> None:

@@ -38,6 +38,17 @@
 //   k_t^T v_t with a static per-channel w) runs the same kernel with the
 //   log-decay -w of each channel in shared memory instead of the loaded w tile,
 //   so a stage carries r, k and v only.
+// * Fused prologue and epilogue (fp32).  RWKV-6 computes the decay from a base
+//   and a low-rank term, w_t = w_base + tanh(x_t W1) W2, and hands the kernel
+//   ew = -exp(w_t); a head's output is then group-normalised and gated
+//   ("RWKV Architecture ...", RWKV-6 "Finch" and RWKV-5 "Eagle"; the spatial-mix
+//   block of "How the WKV ... Processes Images").  With FwdParams::wb the loaded
+//   tile is ww = tanh(x W1) W2 and is turned into ew in shared memory; with
+//   FwdParams::gn_w each finished y row of a head (the 16 lanes of a half warp)
+//   is normalised, scaled, shifted and multiplied by the gate before its store.
+//   Neither w nor the un-normalised y makes a trip through HBM.
+#include <type_traits>
+
 #include "wkv_launch.cuh"
 
 namespace wkv {
@@ -61,6 +72,7 @@ struct FwdSmem {
     float c[TC];             // bonus scalar sum_i r_p u k_p
     float u[kHead];
     float ew5[kHead];        // static log-decay -w5 (RWKV-5), unused otherwise
+    float wbase[kHead];      // w_base of the decay prologue, unused otherwise
     uint32_t renorm_mask;    // bit p set: token p is a renorm step
     alignas(8) uint64_t full[2];
 };
@@ -111,9 +123,12 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
 
     // RWKV-5: one log-decay per channel for every token; the w map is not read
     const bool stat = prm.w5 != nullptr;
+    // decay prologue (fp32 only): the loaded tile is ww, turned into ew = -exp(w_base + ww)
+    const bool pro = std::is_same<Tin, float>::value && prm.wb != nullptr;
     if (tid < kHead) {
         sm.u[tid] = prm.u[cbase + tid];
         sm.ew5[tid] = stat ? -prm.w5[cbase + tid] : 0.f;
+        sm.wbase[tid] = pro ? prm.wb[cbase + tid] : 0.f;
     }
     if (tid == 0) {
         prefetch_tensormap(&map_r);
@@ -173,6 +188,16 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         }
     }
 
+    // group-norm weight and bias of the 4 output columns this thread writes (the same
+    // columns in every write-out round)
+    static_assert(NT % (CW / 4) == 0, "a thread writes the same columns in every round");
+    float4 gnw = make_float4(0.f, 0.f, 0.f, 0.f), gnb = gnw;
+    if (prm.gn_w != nullptr) {
+        const int j4 = (tid % (CW / 4)) * 4;
+        gnw = __ldg(reinterpret_cast<const float4 *>(prm.gn_w + cbase + col0 + j4));
+        gnb = __ldg(reinterpret_cast<const float4 *>(prm.gn_b + cbase + col0 + j4));
+    }
+
     for (int g = 0; g < nchunks; ++g) {
         const ChunkPos cp = chunk_pos(g, nch, T, TC, BIDIR);
         const int s = g & 1;
@@ -200,10 +225,23 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         // ---- transform: renorm flags ----
         // a token is a renorm step if some row has |ew| > kTheta / TC (or NaN)
         int bad = 0;
-        for (int e = tid; e < TC * kHead; e += NT) {
-            const float ew = ew_at(e / kHead, e % kHead);
-            bad |= !(fabsf(ew) <= kTheta / TC);
+        if constexpr (std::is_same<Tin, float>::value) {
+            if (pro) {
+                // decay prologue, in place: rows outside [0, T) keep the zero log-decay
+                for (int e = tid; e < TC * kHead; e += NT) {
+                    const int row = e / kHead, i = e % kHead, t = cp.t_lo + row;
+                    const float ew = (t >= 0 && t < T) ? -expf(sm.wbase[i] + sm.raw_w[s][row][i]) : 0.f;
+                    sm.raw_w[s][row][i] = ew;
+                    bad |= !(fabsf(ew) <= kTheta / TC);
+                }
+                fence_proxy_async_smem();   // the stage is reloaded by the TMA later
+            }
         }
+        if (!pro)
+            for (int e = tid; e < TC * kHead; e += NT) {
+                const float ew = ew_at(e / kHead, e % kHead);
+                bad |= !(fabsf(ew) <= kTheta / TC);
+            }
         const int any_bad = __syncthreads_or(bad);
         if (tid < 32) {
             uint32_t mask = 1u << (TC - 1);
@@ -349,12 +387,26 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                              : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
+        // norm/gate epilogue on the finished y (the causal sweep, or the second pass);
+        // the gate loads are issued first so that their latency overlaps the statistics
+        const bool epi = prm.gn_w != nullptr && (!BIDIR || cp.pass == 1);
+        float4 gate[kRounds];
+        if (epi) {
+#pragma unroll
+            for (int m = 0; m < kRounds; ++m) {
+                const int e = tid + m * NT, p = e / V4, j4 = (e % V4) * 4;
+                const int t = cp.dir > 0 ? cp.t_lo + p : cp.t_lo + TC - 1 - p;
+                gate[m] = (t >= 0 && t < T)
+                              ? __ldg(reinterpret_cast<const float4 *>(prm.g + ((size_t)b * T + t) * C + cbase +
+                                                                       col0 + j4))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
 #pragma unroll
         for (int m = 0; m < kRounds; ++m) {
             const int e = tid + m * NT, p = e / V4, j4 = (e % V4) * 4;
             const int t = cp.dir > 0 ? cp.t_lo + p : cp.t_lo + TC - 1 - p;
-            if (t < 0 || t >= T) continue;
-            float4 *dst = reinterpret_cast<float4 *>(prm.y + ((size_t)b * T + t) * C + cbase + col0 + j4);
+            const bool valid = t >= 0 && t < T;
             float4 val = *reinterpret_cast<const float4 *>(&sm.ybuf[p][j4]);
             if (BIDIR && cp.pass == 1) {
                 val.x += old[m].x;
@@ -362,7 +414,24 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                 val.z += old[m].z;
                 val.w += old[m].w;
             }
-            *dst = val;
+            const size_t off = ((size_t)b * T + t) * C + cbase + col0 + j4;
+            if (epi) {
+                static_assert(V4 == 16, "a head row is the 16 lanes of a half warp");
+                // mean and variance of the head's 64 outputs (two passes, exact order)
+                float sm1 = (val.x + val.y) + (val.z + val.w);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) sm1 += __shfl_xor_sync(0xffffffffu, sm1, o);
+                const float mu = sm1 * (1.f / kHead);
+                const float4 d = make_float4(val.x - mu, val.y - mu, val.z - mu, val.w - mu);
+                float q = (d.x * d.x + d.y * d.y) + (d.z * d.z + d.w * d.w);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+                const float rstd = rsqrtf(q * (1.f / kHead) + prm.gn_eps);
+                const float4 gg = gate[m];
+                val = make_float4(fmaf(d.x * rstd, gnw.x, gnb.x) * gg.x, fmaf(d.y * rstd, gnw.y, gnb.y) * gg.y,
+                                  fmaf(d.z * rstd, gnw.z, gnb.z) * gg.z, fmaf(d.w * rstd, gnw.w, gnb.w) * gg.w);
+            }
+            if (valid) *reinterpret_cast<float4 *>(prm.y + off) = val;
         }
         if (BIDIR && g == nch - 1) __syncthreads();  // pass-0 y stores visible before pass-1 reads
     }

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -127,15 +128,21 @@ bool bf16_use_tensor_cores() {
 
 // w5 (RWKV-5): static per-channel decay rate [C]; then w is ignored (pass w5 for
 // the argument checks) and the recurrence kernel runs with the constant log-decay.
+// fused (fp32 recurrence only): decay prologue and norm/gate epilogue of wkv6_fwd_fused.
+struct Fused {
+    const float *wb, *g, *gn_w, *gn_b;
+    float eps;
+};
+
 int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r, const void *k, const void *v,
                const void *w, const float *u, float *y, wkv_stream_t stream, const float *s0 = nullptr,
-               float *sT = nullptr, const float *w5 = nullptr) {
+               float *sT = nullptr, const float *w5 = nullptr, const Fused *fused = nullptr) {
     int st = check_wkv6(B, T, C, H, {r, k, v, w, u, y});
     if (st != WKV_OK) return st;
     if (B == 0 || T == 0) return WKV_OK;
     if ((st = check_device()) != WKV_OK) return st;
     CUtensorMap mr, mk, mv, mw;
-    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && bf16_use_tensor_cores()) {
+    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && fused == nullptr && bf16_use_tensor_cores()) {
         constexpr int kTcChunk = 64;
         CUtensorMap my;
         if (!make_map(&mr, r, true, B, T, C, kHead, kTcChunk, true) ||
@@ -159,6 +166,13 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
     prm.s0 = s0;
     prm.sT = sT;
     prm.w5 = w5;
+    if (fused != nullptr) {
+        prm.wb = fused->wb;
+        prm.g = fused->g;
+        prm.gn_w = fused->gn_w;
+        prm.gn_b = fused->gn_b;
+        prm.gn_eps = fused->eps;
+    }
     return wkv6_fwd_launch(bf16, bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)) ==
                    cudaSuccess
                ? WKV_OK
@@ -246,6 +260,17 @@ int wkv6_bwd_bf16(int B, int T, int C, int H, int bidirectional, const uint16_t 
                   float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes, wkv_stream_t stream) {
     return bwd_common(true, B, T, C, H, bidirectional, r, k, v, w, u, dy, dr, dk, dv, dw, du, workspace,
                       workspace_bytes, stream);
+}
+
+int wkv6_fwd_fused(int B, int T, int C, int H, int bidirectional, const float *r, const float *k, const float *v,
+                   const float *ww, const float *w_base, const float *u, const float *g, const float *gn_weight,
+                   const float *gn_bias, float eps, float *out, wkv_stream_t stream) {
+    if (!(eps > 0.f) || !std::isfinite(eps)) return WKV_ERR_ARG;
+    int st = check_wkv6(B, T, C, H, {w_base, g, gn_weight, gn_bias});
+    if (st != WKV_OK) return st;
+    const Fused f{w_base, g, gn_weight, gn_bias, eps};
+    return fwd_common(false, bidirectional != 0, B, T, C, H, r, k, v, ww, u, out, stream, nullptr, nullptr, nullptr,
+                      &f);
 }
 
 int wkv5_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,

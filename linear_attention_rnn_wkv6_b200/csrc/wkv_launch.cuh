@@ -16,6 +16,13 @@ struct FwdParams {
     // RWKV-5 static decay rate w5[C] >= 0 (log-decay -w5 at every token); when set
     // the w tensor map is not read
     const float *w5 = nullptr;
+    // fp32 recurrence kernel only.  Decay prologue: when wb (w_base [C]) is set, the
+    // w map holds ww [B][T][C] and the log-decay is ew = -exp(wb + ww).  Norm/gate
+    // epilogue: when gn_w is set, y receives (GroupNorm_head(y) * gn_w + gn_b) * g,
+    // with g [B][T][C], gn_w and gn_b [C] and the variance offset gn_eps.
+    const float *wb = nullptr;
+    const float *g = nullptr, *gn_w = nullptr, *gn_b = nullptr;
+    float gn_eps = 0.f;
 };
 
 struct BwdParams {

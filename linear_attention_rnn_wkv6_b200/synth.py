@@ -34,7 +34,7 @@ _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-STREAM_R, STREAM_K, STREAM_V, STREAM_WRAW, STREAM_U, STREAM_DY, STREAM_S0 = range(7)
+STREAM_R, STREAM_K, STREAM_V, STREAM_WRAW, STREAM_U, STREAM_DY, STREAM_S0, STREAM_WW, STREAM_G, STREAM_GN = range(10)
 
 _CHUNK = 1 << 16  # elements per block: scratch stays cache resident and is reused in place
 _SCALE53 = 1.0 / 9007199254740992.0
@@ -218,6 +218,49 @@ def make_wkv5(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, rkv_std: fl
     return x
 
 
+@dataclasses.dataclass
+class FusedInputs:
+    """Inputs of the RWKV-6 forward with the decay prologue and the norm/gate epilogue (fp32)."""
+    B: int
+    T: int
+    C: int
+    H: int
+    bidir: bool
+    r: np.ndarray      # [B,T,C]
+    k: np.ndarray
+    v: np.ndarray
+    ww: np.ndarray     # [B,T,C] low-rank decay term tanh(x W1) W2
+    w_base: np.ndarray # [C]
+    u: np.ndarray      # [C]
+    g: np.ndarray      # [B,T,C] gate
+    gn_w: np.ndarray   # [C]
+    gn_b: np.ndarray   # [C]
+    eps: float = 64e-5
+
+
+def make_fused(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, bidir: bool = False,
+               rkv_std: float = 0.5, base_lo: float = -6.0, base_hi: float = -1.0, ww_std: float = 0.5,
+               u_std: float = 0.5, eps: float = 64e-5) -> FusedInputs:
+    """r, k, v, u as make_wkv6 (same streams); w_base ~ U(base_lo, base_hi) per channel (the
+    first C draws of the w_raw stream), ww ~ N(0, ww_std^2), so that the decay pre-activation
+    w_base + ww spans the same range as make_wkv6's w_raw; the gate g ~ N(0, 1); the group
+    norm's weight ~ N(1, 0.1^2) and bias ~ N(0, 0.1^2) per channel."""
+    C = H * N
+    n = B * T * C
+    shape = (B, T, C)
+    f32 = lambda a: a.astype(np.float32)
+    r = f32(normal(seed, STREAM_R, n, rkv_std)).reshape(shape)
+    k = f32(normal(seed, STREAM_K, n, rkv_std)).reshape(shape)
+    v = f32(normal(seed, STREAM_V, n, rkv_std)).reshape(shape)
+    w_base = f32(uniform(seed, STREAM_WRAW, C, base_lo, base_hi))
+    u = f32(normal(seed, STREAM_U, C, u_std))
+    ww = f32(normal(seed, STREAM_WW, n, ww_std)).reshape(shape)
+    g = f32(normal(seed, STREAM_G, n, 1.0)).reshape(shape)
+    gn_w = f32(1.0 + normal(seed, STREAM_GN, C, 0.1))
+    gn_b = f32(normal(seed, STREAM_GN, C, 0.1, offset=C))
+    return FusedInputs(B, T, C, H, bidir, r, k, v, ww, w_base, u, g, gn_w, gn_b, eps)
+
+
 def make_state(B: int, H: int, N: int = 64, *, seed: int = 0, std: float = 1.0) -> np.ndarray:
     """An RWKV-6 recurrent state per (b, h): [B,H,N,N] float32 ~ N(0, std^2) (its own stream)."""
     return normal(seed, STREAM_S0, B * H * N * N, std).astype(np.float32).reshape(B, H, N, N)
@@ -259,6 +302,8 @@ WORKLOADS = {
     "wkv5_causal_bf16_b8t4096h32": ("wkv5_fwd_bf16", dict(B=8, T=4096, H=32, wraw_lo=-8.0, dtype="bf16")),
     # RWKV-5 backward, fp32, on the patch-sequence shape
     "wkv5_bwd_f32_b32t196h12": ("wkv5_bwd", dict(B=32, T=196, H=12, with_dy=True)),
+    # bidirectional RWKV-6 forward with the decay prologue and the group-norm/gate epilogue, fp32
+    "wkv6_bidir_fused_f32_b32t196h12": ("wkv6_fwd_fused", dict(B=32, T=196, H=12, bidir=True)),
 }
 
 
@@ -268,4 +313,6 @@ def make_workload(name: str, seed: int = 0):
         return kind, make_wkv4(seed=seed, **kw)
     if kind.startswith("wkv5"):
         return kind, make_wkv5(seed=seed, **kw)
+    if kind == "wkv6_fwd_fused":
+        return kind, make_fused(seed=seed, **kw)
     return kind, make_wkv6(seed=seed, **kw)

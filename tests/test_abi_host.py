@@ -169,6 +169,21 @@ def test_wkv5_argument_errors(lib):
     assert f(2, 8, 128, 2, *g, FAKE + 4, ws, None) == WKV_ERR_ALIGN
 
 
+def test_wkv6_fwd_fused_argument_errors(lib):
+    p = [FAKE + 256 * i for i in range(9)]                     # r, k, v, ww, w_base, u, g, gn_w, gn_b
+    out = FAKE + 4096
+    f = lib.wkv6_fwd_fused
+    assert f(-1, 4, 64, 1, 0, *p, 1e-5, out, None) == WKV_ERR_ARG
+    assert f(1, 4, 64, 2, 0, *p, 1e-5, out, None) == WKV_ERR_HEADSIZE
+    assert f(1, 4, 64, 1, 1, *(p[:6] + [None] + p[7:]), 1e-5, out, None) == WKV_ERR_ARG   # gate missing
+    assert f(1, 4, 64, 1, 0, *p, 0.0, out, None) == WKV_ERR_ARG                          # eps must be > 0
+    assert f(1, 4, 64, 1, 0, *p, float("nan"), out, None) == WKV_ERR_ARG
+    q = list(p)
+    q[8] += 4                                                  # gn_b misaligned
+    assert f(1, 4, 64, 1, 0, *q, 1e-5, out, None) == WKV_ERR_ALIGN
+    assert f(0, 4, 64, 1, 0, *p, 1e-5, out, None) == WKV_OK
+
+
 def test_wkv4_argument_errors(lib):
     p = [FAKE + 256 * i for i in range(5)]
     assert lib.wkv4_fwd(-1, 4, 32, *p, None) == WKV_ERR_ARG
