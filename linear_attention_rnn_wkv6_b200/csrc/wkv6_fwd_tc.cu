@@ -46,6 +46,8 @@
 
 namespace wkv {
 
+using namespace tc;
+
 namespace {
 
 constexpr int kL = 64;                       // tokens per chunk
@@ -96,69 +98,6 @@ struct TcSmem {
 // 1 KB alignment slack of the dynamic allocation.
 static_assert(sizeof(TcSmem) + 1024 <= 113 * 1024, "two CTAs per SM must fit");
 
-// Byte offset of element (row, col) in a 64-row bf16 tile whose 128-byte rows
-// are 128B-swizzled (16-byte chunk g of row r stored at chunk g ^ (r & 7)).
-// This is the TMA's SWIZZLE_128B placement and, read through a descriptor, the
-// canonical K-major (rows along M/N) or MN-major (rows along K) layout.
-__device__ __forceinline__ uint32_t swz(int row, int col) {
-    return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + ((col & 7) << 1));
-}
-
-// K-major descriptor of the kstep-th group of 16 K values (32 bytes into each row).
-__device__ __forceinline__ uint64_t desc_k(const __nv_bfloat16 *tile, int kstep) {
-    return tc::smem_desc(reinterpret_cast<const char *>(tile) + kstep * 32, 16, 1024) | ((uint64_t)2 << 61);
-}
-// MN-major descriptor of the kstep-th group of 16 K rows; a second 64-wide MN
-// atom, if the instruction has one, starts lbo bytes after the first.
-__device__ __forceinline__ uint64_t desc_mn(const __nv_bfloat16 *tile, int kstep, uint32_t lbo) {
-    return tc::smem_desc(reinterpret_cast<const char *>(tile) + kstep * 2048, lbo, 1024) | ((uint64_t)2 << 61);
-}
-
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         bool accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // .x = a (low half), .y = b
-    return *reinterpret_cast<const uint32_t *>(&h);
-}
-__device__ __forceinline__ uint32_t ld_u32(const void *base, uint32_t off) {
-    return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(base) + off);
-}
-__device__ __forceinline__ void st_u32(void *base, uint32_t off, uint32_t v) {
-    *reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(base) + off) = v;
-}
-__device__ __forceinline__ void st_u128(void *base, uint32_t off, uint4 v) {
-    *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(base) + off) = v;
-}
-__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-__device__ __forceinline__ float raw_at(const __nv_bfloat16 *tile, int row, int col) {
-    const uint32_t off = swz(row, col);
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(reinterpret_cast<const char *>(tile) + off));
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // try_wait with a suspend-time hint: the thread is parked by the hardware until
 // the phase completes or about `ns` nanoseconds pass, without issuing anything.
 __device__ __forceinline__ bool mbar_try_wait_for(uint64_t *bar, uint32_t parity, uint32_t ns) {
@@ -192,30 +131,6 @@ __device__ __forceinline__ bool wait_or_abort(TcSmem &sm, uint64_t *bar, uint32_
 
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Sum of v[m] over the 32 lanes of the warp, for m = 0..7, with lane l ending up
-// holding the sum for m = (l >> 2) & 7 (9 shuffles instead of 8 full reductions).
-__device__ __forceinline__ float transpose_reduce8(const float (&v)[8], int lane) {
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-    float a4[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float keep = b4 ? v[4 + q] : v[q];
-        const float send = b4 ? v[q] : v[4 + q];
-        a4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-    float a2[2];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const float keep = b3 ? a4[2 + q] : a4[q];
-        const float send = b3 ? a4[q] : a4[2 + q];
-        a2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    float a1 = (b2 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? a2[0] : a2[1], 4);
-    a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
-    a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
-    return a1;
 }
 
 __device__ __forceinline__ bool is_flagged(const TcSmem &sm, int c) {

@@ -126,6 +126,14 @@ bool bf16_use_tensor_cores() {
     return !(e && std::strcmp(e, "recurrence") == 0);
 }
 
+// Algorithm of the fp32 forward without state in/out, prologue or epilogue: the
+// chunked tensor-core kernel with split-bf16 operands (default) or the
+// token-by-token recurrence (WKV6_F32_PATH=recurrence).  Read on every call.
+bool f32_use_tensor_cores() {
+    const char *e = std::getenv("WKV6_F32_PATH");
+    return !(e && std::strcmp(e, "recurrence") == 0);
+}
+
 // w5 (RWKV-5): static per-channel decay rate [C]; then w is ignored (pass w5 for
 // the argument checks) and the recurrence kernel runs with the constant log-decay.
 // fused (fp32 recurrence only): decay prologue and norm/gate epilogue of wkv6_fwd_fused.
@@ -154,6 +162,14 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
         FwdParams prm{B, T, C, H, u, y};
         prm.w5 = w5;
         return wkv6_fwd_tc_launch(mr, mk, mv, mw, my, prm, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                   ? WKV_OK
+                   : WKV_ERR_CUDA;
+    }
+    if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && fused == nullptr && f32_use_tensor_cores()) {
+        FwdParams prm{B, T, C, H, u, y};
+        return wkv6_fwd_split_launch(bidir, static_cast<const float *>(r), static_cast<const float *>(k),
+                                     static_cast<const float *>(v), static_cast<const float *>(w), prm,
+                                     reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                    ? WKV_OK
                    : WKV_ERR_CUDA;
     }

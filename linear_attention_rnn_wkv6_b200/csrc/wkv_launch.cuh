@@ -42,6 +42,10 @@ cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const 
 cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
                                const CUtensorMap &mw, const CUtensorMap &my, const FwdParams &prm,
                                cudaStream_t stream);
+// fp32 causal or bidirectional forward on the tensor cores (split-bf16 operands);
+// r, k, v, w are [B][T][C] fp32 device pointers, 8-byte aligned.
+cudaError_t wkv6_fwd_split_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
+                                  const FwdParams &prm, cudaStream_t stream);
 // One recurrent step for B sequences (state [B][H][N][N] updated in place).
 cudaError_t wkv6_decode_launch(int B, int C, int H, const float *r, const float *k, const float *v,
                                const float *w, const float *u, float *state, float *y, cudaStream_t stream);

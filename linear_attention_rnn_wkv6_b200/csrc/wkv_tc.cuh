@@ -150,9 +150,150 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---- 16 lanes x 256 bits per repetition (.16x256b): all 32 threads of the warp
+// share 16 TMEM lanes.  Thread t holds, for repetition m (8 columns each),
+//   v[4m], v[4m+1]     lane (t / 4),     columns 8m + 2(t % 4) and 8m + 2(t % 4) + 1
+//   v[4m+2], v[4m+3]   lane (t / 4) + 8, the same two columns
+// (the placement of an mma.sync accumulator fragment; checked on this B200 by
+// writing lane * 100 + column with the 32x32b shape and reading it back).
+// The lane field of taddr is the first of the 16 lanes.
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr),
+          "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+          "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+          "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+          "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+          "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+          "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
 // TMEM address of (lane, column) relative to an allocation base.
 __device__ __forceinline__ uint32_t taddr(uint32_t base, uint32_t lane, uint32_t col) {
     return base + (lane << 16) + col;
+}
+
+
+// ---- bf16 operands (kind::f16) in 128-byte-swizzled tiles, and small device helpers
+
+// Byte offset of element (row, col) in a 64-row bf16 tile whose 128-byte rows
+// are 128B-swizzled (16-byte chunk g of row r stored at chunk g ^ (r & 7)).
+// This is the TMA's SWIZZLE_128B placement and, read through a descriptor, the
+// canonical K-major (rows along M/N) or MN-major (rows along K) layout.
+__device__ __forceinline__ uint32_t swz(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + ((col & 7) << 1));
+}
+
+// K-major descriptor of the kstep-th group of 16 K values (32 bytes into each row).
+__device__ __forceinline__ uint64_t desc_k(const __nv_bfloat16 *tile, int kstep) {
+    return smem_desc(reinterpret_cast<const char *>(tile) + kstep * 32, 16, 1024) | ((uint64_t)2 << 61);
+}
+// MN-major descriptor of the kstep-th group of 16 K rows; a second 64-wide MN
+// atom, if the instruction has one, starts lbo bytes after the first.
+__device__ __forceinline__ uint64_t desc_mn(const __nv_bfloat16 *tile, int kstep, uint32_t lbo) {
+    return smem_desc(reinterpret_cast<const char *>(tile) + kstep * 2048, lbo, 1024) | ((uint64_t)2 << 61);
+}
+
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // .x = a (low half), .y = b
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ uint32_t ld_u32(const void *base, uint32_t off) {
+    return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(base) + off);
+}
+__device__ __forceinline__ void st_u32(void *base, uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t *>(reinterpret_cast<char *>(base) + off) = v;
+}
+__device__ __forceinline__ void st_u128(void *base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(base) + off) = v;
+}
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ float raw_at(const __nv_bfloat16 *tile, int row, int col) {
+    const uint32_t off = swz(row, col);
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(reinterpret_cast<const char *>(tile) + off));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Sum of v[m] over the 32 lanes of the warp, for m = 0..7, with lane l ending up
+// holding the sum for m = (l >> 2) & 7 (9 shuffles instead of 8 full reductions).
+__device__ __forceinline__ float transpose_reduce8(const float (&v)[8], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float a4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float keep = b4 ? v[4 + q] : v[q];
+        const float send = b4 ? v[q] : v[4 + q];
+        a4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float a2[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const float keep = b3 ? a4[2 + q] : a4[q];
+        const float send = b3 ? a4[q] : a4[2 + q];
+        a2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float a1 = (b2 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? a2[0] : a2[1], 4);
+    a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+    a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+    return a1;
 }
 
 }  // namespace tc

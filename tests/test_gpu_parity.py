@@ -29,6 +29,17 @@ def _rel(a, b):
 
 # ------------------------------------------------------------------ forward, small and ragged
 
+F32_PATHS = ["tensor", "recurrence"]
+
+
+@pytest.fixture(params=F32_PATHS)
+def f32_path(request, monkeypatch):
+    """Run the fp32 forward (causal and bidirectional) through the chunked
+    tensor-core kernel with split-bf16 operands or the token-by-token recurrence."""
+    monkeypatch.setenv("WKV6_F32_PATH", request.param)
+    return request.param
+
+
 FWD_SHAPES = [  # (B, T, H): several 32-token chunks, ragged tails, T < chunk, single token
     (1, 1, 1), (1, 2, 1), (2, 31, 2), (1, 32, 1), (1, 33, 3), (2, 65, 2), (3, 100, 1), (1, 196, 4),
 ]
@@ -36,7 +47,7 @@ FWD_SHAPES = [  # (B, T, H): several 32-token chunks, ragged tails, T < chunk, s
 
 @pytest.mark.parametrize("B,T,H", FWD_SHAPES)
 @pytest.mark.parametrize("bidir", [False, True])
-def test_wkv6_fwd_f32_small(B, T, H, bidir):
+def test_wkv6_fwd_f32_small(B, T, H, bidir, f32_path):
     x = synth.make_wkv6(B, T, H, seed=T * 10 + H)
     y = gc.run_wkv6_fwd(x, bidir=bidir)
     r, k, v, w, u = gc.f64(x)
@@ -108,7 +119,7 @@ def _with_w(x, w):
 
 @pytest.mark.parametrize("bidir", [False, True])
 @pytest.mark.parametrize("case", ["strong", "mixed", "zero_decay", "unit_decay", "long_memory"])
-def test_wkv6_fwd_decay_edge_cases(case, bidir):
+def test_wkv6_fwd_decay_edge_cases(case, bidir, f32_path):
     B, T, H = 2, 70, 2
     x = synth.make_wkv6(B, T, H, seed=11)
     g = np.random.default_rng(5)
@@ -134,7 +145,7 @@ def test_wkv6_fwd_decay_edge_cases(case, bidir):
     assert _rel(y, ref) <= gc.TOL_F32_FWD
 
 
-def test_wkv6_fwd_output_fully_overwritten_and_deterministic():
+def test_wkv6_fwd_output_fully_overwritten_and_deterministic(f32_path):
     x = synth.make_wkv6(2, 77, 3, seed=3)
     y1 = gc.run_wkv6_fwd(x, bidir=True)   # outputs start as NaN inside run_wkv6_fwd
     y2 = gc.run_wkv6_fwd(x, bidir=True)
@@ -142,7 +153,7 @@ def test_wkv6_fwd_output_fully_overwritten_and_deterministic():
     assert np.array_equal(y1, y2)
 
 
-def test_wkv6_fwd_slices_match_single_head_calls():
+def test_wkv6_fwd_slices_match_single_head_calls(f32_path):
     x = synth.make_wkv6(2, 50, 3, seed=4)
     y = gc.run_wkv6_fwd(x)
     for b in range(2):
@@ -209,7 +220,7 @@ def test_wkv4_large_keys():
 
 # ------------------------------------------------------------------ full-size workloads
 
-def test_workload_causal_f32_small_config_full_tensor():
+def test_workload_causal_f32_small_config_full_tensor(f32_path):
     kind, x = synth.make_workload("wkv6_causal_f32_b1t196h4")
     y = gc.run_wkv6_fwd(x)
     r, k, v, w, u = gc.f64(x)
@@ -235,7 +246,7 @@ def _sampled_fwd(x, bidir, n_units, tol):
     return err
 
 
-def test_workload_bidir_f32_sampled():
+def test_workload_bidir_f32_sampled(f32_path):
     kind, x = synth.make_workload("wkv6_bidir_f32_b32t196h12")
     _sampled_fwd(x, True, 48, gc.TOL_F32_FWD)
 
