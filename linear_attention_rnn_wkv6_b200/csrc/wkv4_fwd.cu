@@ -145,11 +145,163 @@ wkv4_fwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
     }
 }
 
+// Four adjacent channels per thread (C % 4 == 0): one 16-byte load brings a token of
+// all four, and their chains are independent work for the same thread.  A CTA
+// covers 16 channels x kSegV segments (4 threads per token row), loads run one
+// batch of kUV tokens ahead of the updates, and full segments skip the per-token
+// bounds checks.  Phases as in wkv4_fwd_kernel, except that phase 2 is a
+// log-depth (Kogge-Stone) scan over the segments: an element covering a span of
+// n tokens is (a, b, p, n), and (left, right) combine to
+// (e^{-n_right w} left (+) right, n_left + n_right), which is associative.
+constexpr int kSegV = 32;                      // segments of T per channel
+constexpr int kUV = 4;                         // tokens per load batch (two batches in flight)
+
+constexpr int VEC = 4;                         // channels per thread (one float4); measured faster than 2
+constexpr int kThrV = (kCh / VEC) * kSegV;     // 128 threads
+using V = float4;
+__device__ __forceinline__ float comp(const float4 &x, int i) { return i == 0 ? x.x : i == 1 ? x.y : i == 2 ? x.z : x.w; }
+__device__ __forceinline__ float4 vmake(const float (&o)[4]) { return make_float4(o[0], o[1], o[2], o[3]); }
+
+__global__ void __launch_bounds__(kThrV, 3)
+wkv4_fwd_vec_kernel(int T, int C, const float *__restrict__ k, const float *__restrict__ v,
+                    const float *__restrict__ w, const float *__restrict__ u, float *__restrict__ y) {
+    constexpr int kQ = kCh / VEC;              // threads per token row of the CTA
+    __shared__ Wkv4State summ[kSegV][kCh];
+    __shared__ float sspan[kSegV][kQ];         // tokens covered by the scan element of each segment
+    const int tid = threadIdx.x;
+    const int cq = tid % kQ;                   // channel group within the CTA
+    const int seg = tid / kQ;
+    const int groups = (C + kCh - 1) / kCh;
+    const int b = blockIdx.x / groups;
+    const int c0 = (blockIdx.x % groups) * kCh + VEC * cq;
+    const bool live = c0 < C;                  // C % VEC == 0: the group is whole or absent
+    const int seglen = (T + kSegV - 1) / kSegV;
+    const int t0 = min(T, seg * seglen);
+    const int t1 = min(T, t0 + seglen);
+    float w2[VEC], u2[VEC];
+    {
+        const V wv = live ? *reinterpret_cast<const V *>(w + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const V uv = live ? *reinterpret_cast<const V *>(u + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            w2[i] = comp(wv, i) * kLog2e;
+            u2[i] = comp(uv, i) * kLog2e;
+        }
+    }
+    const size_t brow = (size_t)b * T * C;
+    const float *kr = k + brow + c0, *vr = v + brow + c0;
+    float *yr = y + brow + c0;
+    const bool full = live && (t1 - t0) == seglen && seglen % kUV == 0;
+    auto load = [&](int t, V (&kb)[kUV], V (&vb)[kUV]) {
+#pragma unroll
+        for (int e = 0; e < kUV; ++e) {
+            const bool in = live && t + e < t1;   // the look-ahead batch may pass the segment end
+            kb[e] = in ? __ldg(reinterpret_cast<const V *>(kr + (size_t)(t + e) * C)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            vb[e] = in ? __ldg(reinterpret_cast<const V *>(vr + (size_t)(t + e) * C)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+
+    // ---- phase 1: segment summaries from the empty state ----
+    Wkv4State st[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) st[i] = Wkv4State{0.f, 0.f, -INFINITY};
+    {
+        V kb[kUV], vb[kUV];
+        load(t0, kb, vb);
+        for (int t = t0; t < t1; t += kUV) {
+            V kn[kUV], vn[kUV];
+            load(t + kUV, kn, vn);             // past t1 every load is predicated off
+#pragma unroll
+            for (int e = 0; e < kUV; ++e)
+                if (full || t + e < t1) {
+#pragma unroll
+                    for (int i = 0; i < VEC; ++i) wkv4_update(st[i], comp(kb[e], i) * kLog2e, comp(vb[e], i), w2[i]);
+                }
+#pragma unroll
+            for (int e = 0; e < kUV; ++e) {
+                kb[e] = kn[e];
+                vb[e] = vn[e];
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) summ[seg][VEC * cq + i] = st[i];
+    sspan[seg][cq] = (float)(t1 - t0);
+    __syncthreads();
+
+    // ---- phase 2: inclusive scan over the segments, then the state entering this one ----
+    {
+        float span = (float)(t1 - t0);
+#pragma unroll 1
+        for (int o = 1; o < kSegV; o <<= 1) {
+            Wkv4State left[VEC];
+            float lspan = 0.f;
+            if (seg >= o) {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) left[i] = summ[seg - o][VEC * cq + i];
+                lspan = sspan[seg - o][cq];
+            }
+            __syncthreads();
+            if (seg >= o) {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) {
+                    const float pd = left[i].p - span * w2[i];   // the left span decays over this span
+                    const float q = fmaxf(pd, st[i].p);
+                    if (q == -INFINITY) continue;                // both empty
+                    const float e1 = ex2(pd - q), e2 = ex2(st[i].p - q);
+                    st[i].a = fmaf(e1, left[i].a, e2 * st[i].a);
+                    st[i].b = fmaf(e1, left[i].b, e2 * st[i].b);
+                    st[i].p = q;
+                }
+                span += lspan;
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) summ[seg][VEC * cq + i] = st[i];
+                sspan[seg][cq] = span;
+            }
+            __syncthreads();
+        }
+    }
+    // the state entering segment seg is the inclusive scan of segment seg - 1
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) st[i] = seg > 0 ? summ[seg - 1][VEC * cq + i] : Wkv4State{0.f, 0.f, -INFINITY};
+
+    // ---- phase 3: rerun the segment, write y ----
+    {
+        V kb[kUV], vb[kUV];
+        load(t0, kb, vb);
+        for (int t = t0; t < t1; t += kUV) {
+            V kn[kUV], vn[kUV];
+            load(t + kUV, kn, vn);
+#pragma unroll
+            for (int e = 0; e < kUV; ++e)
+                if (full || (live && t + e < t1)) {
+                    float o[VEC];
+#pragma unroll
+                    for (int i = 0; i < VEC; ++i) {
+                        const float k2 = comp(kb[e], i) * kLog2e, vv = comp(vb[e], i);
+                        o[i] = wkv4_output(st[i], k2, vv, u2[i]);
+                        wkv4_update(st[i], k2, vv, w2[i]);
+                    }
+                    *reinterpret_cast<V *>(yr + (size_t)(t + e) * C) = vmake(o);
+                }
+#pragma unroll
+            for (int e = 0; e < kUV; ++e) {
+                kb[e] = kn[e];
+                vb[e] = vn[e];
+            }
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,
                             const float *u, float *y, cudaStream_t stream) {
     const int groups = (C + kCh - 1) / kCh;
+    if (C % VEC == 0) {
+        wkv4_fwd_vec_kernel<<<(unsigned)(B * groups), kThrV, 0, stream>>>(T, C, k, v, w, u, y);
+        return cudaGetLastError();
+    }
     wkv4_fwd_kernel<<<(unsigned)(B * groups), kCh * kSeg, 0, stream>>>(T, C, k, v, w, u, y);
     return cudaGetLastError();
 }

@@ -138,6 +138,9 @@ __device__ __forceinline__ uint64_t desc_ap(const __nv_bfloat16 *tile, int ks) {
     return smem_desc(reinterpret_cast<const char *>(tile) + ks * 1024, 512, 128);
 }
 
+// A descriptor moved by `bytes` (a multiple of 16): the start address is the low field.
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity) {
     return mbar_wait_bounded(bar, parity);
 }
@@ -184,6 +187,10 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
     // TMEM: A (32 columns) and Y (64) share columns 0..63, S at 64..127 (M = 64 layouts)
     const uint32_t tY = sm.tmem_base, tS = sm.tmem_base + 64;
 
+    // base descriptors; every MMA below adds a compile-time offset (term tile, k-step)
+    constexpr uint32_t kTokB = kTokTile * 2, kApB = kApTile * 2, kStB = kStTile * 2;   // tile bytes
+    const uint64_t dQ = desc_k(sm.Q[0], 0), dKk = desc_k(sm.Kt[0], 0), dKm = desc_mn(sm.Kt[0], 0, 16);
+    const uint64_t dV = desc_mn(sm.V[0], 0, 16), dA = desc_ap(sm.Ap[0], 0), dS = desc_mn(sm.Sin[0], 0, 16);
     constexpr uint32_t kIdM1 = idesc_bf16(64, 32, false, false);
     constexpr uint32_t kIdAV = idesc_bf16(64, 64, false, true);
     constexpr uint32_t kIdQS = idesc_bf16(64, 64, false, true);
@@ -302,8 +309,8 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                     for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
                         for (int q = 0; q < kNP; ++q)
-                            mma_bf16(tY, desc_k(sm.Q[prod_a(q)], ks), desc_k(sm.Kt[prod_b(q)], ks), kIdM1,
-                                     ks > 0 || q > 0);
+                            mma_bf16(tY, dadd(dQ, prod_a(q) * kTokB + 32 * ks), dadd(dKk, prod_b(q) * kTokB + 32 * ks),
+                                     kIdM1, ks > 0 || q > 0);
                     mma_commit(&sm.bar_m1);
                 } else if (tid == 32) {
                     // S (rescaled by the previous epilogue, or zero) += Kt^T V
@@ -311,8 +318,8 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                     for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
                         for (int q = 0; q < kNP; ++q)
-                            mma_bf16(tS, desc_mn(sm.Kt[prod_a(q)], ks, 16), desc_mn(sm.V[prod_b(q)], ks, 16), kIdS,
-                                     true);
+                            mma_bf16(tS, dadd(dKm, prod_a(q) * kTokB + 2048 * ks), dadd(dV, prod_b(q) * kTokB + 2048 * ks),
+                                     kIdS, true);
                     mma_commit(&sm.bar_s);
                 }
                 ok = wait_bar(&sm.bar_m1, ph_m1);
@@ -360,15 +367,15 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                     for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
                         for (int q = 0; q < kNP; ++q)
-                            mma_bf16(tY, desc_ap(sm.Ap[prod_a(q)], ks), desc_mn(sm.V[prod_b(q)], ks, 16), kIdAV,
-                                     ks > 0 || q > 0);
+                            mma_bf16(tY, dadd(dA, prod_a(q) * kApB + 1024 * ks), dadd(dV, prod_b(q) * kTokB + 2048 * ks),
+                                     kIdAV, ks > 0 || q > 0);
                     if (c > 0) {
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
                             for (int q = 0; q < kNP; ++q)
-                                mma_bf16(tY, desc_k(sm.Q[prod_a(q)], ks), desc_mn(sm.Sin[prod_b(q)], ks, 16), kIdQS,
-                                         true);
+                                mma_bf16(tY, dadd(dQ, prod_a(q) * kTokB + 32 * ks),
+                                         dadd(dS, prod_b(q) * kStB + 2048 * ks), kIdQS, true);
                     }
                     mma_commit(&sm.bar_p);
                 }

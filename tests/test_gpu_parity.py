@@ -200,7 +200,8 @@ def test_wkv6_bwd_strong_decay_and_determinism(bidir):
 
 # ------------------------------------------------------------------ RWKV-4
 
-@pytest.mark.parametrize("B,T,C", [(1, 1, 32), (2, 7, 40), (1, 100, 64), (2, 333, 96), (1, 1024, 32)])
+@pytest.mark.parametrize("B,T,C", [(1, 1, 32), (2, 7, 40), (1, 100, 64), (2, 333, 96), (1, 1024, 32),
+                                   (2, 50, 30), (1, 65, 36), (3, 31, 20)])   # C % 4 != 0: per-channel kernel
 def test_wkv4_small(B, T, C):
     x = synth.make_wkv4(B, T, C, seed=T)
     y = gc.run_wkv4(x)
