@@ -51,11 +51,13 @@ FALLBACK_HBM_GBS = 6650.0
 # (token, channel) for RWKV-4).  Bytes: inputs read once + outputs written once.
 # Flops: RWKV-6 forward 5 N^2 per direction (state update 3 N^2 + readout 2 N^2),
 # backward 14 N^2 per direction; RWKV-4 ~4 exp + 12 flop (HBM bound).  The bf16
-# causal forward runs on the tensor cores (chunked form, about 40 N^2 tensor flops
-# per unit against a 2.25 PFLOP/s pipe), so its bound is the bytes it must move.
+# causal forward and the fp32 forward (causal and bidirectional) run on the tensor
+# cores (chunked form: about 40 N^2 tensor flops per unit and direction, six split
+# bf16 products each for fp32, against a 1.7 PFLOP/s pipe), so their bound is the
+# bytes they must move; the FP32-equivalent rate is reported next to it.
 ALG = {
     "wkv4_f32_b8t1024c768": dict(bytes_per_unit=3 * 4, flops_per_unit=16, bound="hbm"),
-    "wkv6_bidir_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=10 * N * N, bound="alu"),
+    "wkv6_bidir_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=10 * N * N, bound="hbm"),
     "wkv6_causal_bf16_b8t4096h32": dict(bytes_per_unit=4 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
     "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="alu"),
     "wkv6_bidir_bwd_bf16_b32t196h12": dict(bytes_per_unit=5 * N * 2 + 4 * N * 4, flops_per_unit=28 * N * N,
