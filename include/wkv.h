@@ -161,7 +161,9 @@ int wkv6_bwd_bf16(int B, int T, int C, int H, int bidirectional, const uint16_t 
                   float *dk, float *dv, float *dw, float *du, void *workspace, size_t workspace_bytes,
                   wkv_stream_t stream);
 
-/* Scratch bytes wkv6_bwd needs for these sizes (B*C floats of per-batch du partials). */
+/* Scratch bytes wkv6_bwd needs for these sizes: 2*B*C floats (per-batch du
+ * partials, and the per-channel totals that the tensor-core backward carries
+ * from its first kernel to its second). */
 size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional);
 
 /*

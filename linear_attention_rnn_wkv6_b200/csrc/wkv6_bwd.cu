@@ -456,6 +456,11 @@ __global__ void wkv6_du_reduce_kernel(int B, int C, const float *__restrict__ pa
     du[c] = acc;
 }
 
+cudaError_t wkv6_du_reduce_launch(int B, int C, const float *part, float *du, cudaStream_t stream) {
+    wkv6_du_reduce_kernel<<<(C + 255) / 256, 256, 0, stream>>>(B, C, part, du);
+    return cudaGetLastError();
+}
+
 template <typename Tin, int TC, bool BIDIR>
 static cudaError_t launch_bwd(const CUtensorMap *maps, const BwdParams &prm, cudaStream_t stream) {
     auto kern = wkv6_bwd_kernel<Tin, TC, BIDIR>;

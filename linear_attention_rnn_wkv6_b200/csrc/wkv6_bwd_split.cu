@@ -1,0 +1,979 @@
+// wkv6_bwd_split.cu -- RWKV-6 fp32 backward (causal and bidirectional) on the
+// 5th-generation tensor cores, operands split into two bf16 terms.
+//
+// Gradients of L = sum_t dy_t . y_t for the forward of wkv6_fwd.cu ("How Custom
+// CUDA Kernels (wkv6_cuda.cu) ...", Backward Pass Gradient Computation: a
+// forward-in-time part and a backward-in-time part, no atomics), evaluated in the
+// chunked form of the forward (wkv6_fwd_split.cu).  Per direction, in its
+// processing order p (time order for the causal sweep, reversed for the
+// anti-causal one), with S_{p-1} the state a token reads and
+// G_p = sum_{tau > p} diag(P(p, tau)) r_tau^T dy_tau the adjoint it sees:
+//   dr'_p = S_{p-1} dy_p,   dk'_p = G_p v_p,   dv'_p = G_p^T k_p        (no bonus)
+// In a chunk of L = 32 tokens with Lam_p = sum_{m<p} ew_m (chunk-local),
+// Q_p = r_p e^{Lam_p}, Kt_s = k_s e^{-Lam_{s+1}}, Gam = e^{Lam_L}:
+//   S kind (chunks in processing order, state S_in entering the chunk)
+//     dA = dY V^T (strict lower: s < p),   dQ = dA Kt + dY S_in^T,   dr'_p = e^{Lam_p} dQ_p
+//     S_out = diag(Gam) (S_in + Kt^T V)
+//   G kind (chunks in reverse order, adjoint G_out of the state leaving the chunk,
+//   Gt = diag(Gam) G_out)
+//     A^T = Kt Q^T,  dA^T = V dY^T (both strict: tau > s),  A' = A + diag(c) (causal bonus c)
+//     dKt = dA'^T Q + V Gt^T,   dk'_s = e^{-Lam_{s+1}} dKt_s
+//     dV  = A'^T dY + Kt Gt,    dv'_s = dV_s
+//     G_in = Gt + Q^T dY  (the adjoint leaving the previous chunk)
+// Bonus (causal only): dr += u k (v.dy), dk += u r (v.dy), dv += (sum r u k) dy,
+// du = sum r k (v.dy).  Decay gradient, without holding a state and an adjoint at
+// once: with z_t = r_t dr'^causal_t + k_t dk'^anti_t and x_t = k_t dk'^causal_t +
+// r_t dr'^anti_t,  dw_m = sum_{t > m} z_t - sum_{s >= m} x_s.  Each pass adds its
+// share as it runs: a pass forward in time subtracts the running prefix of its z
+// part, a pass backward in time subtracts the running suffix of its x part, and
+// the last pass adds the z totals.
+//
+// Precision: the gradient tolerance (1e-4 relative L2) allows two bf16 terms per
+// operand (x0 = bf16(x), x1 = bf16(x - x0), 16 significant bits) and three MMAs
+// per product (a0b0 + a0b1 + a1b0).
+//
+// Launches: the S kind (dr, du partials, the bonus parts of dk and dv, its dw share
+// and the z total per channel), then the G kind (dk, dv added, the rest of dw).
+// One CTA of 128 threads per (b, h) each, three CTAs per SM.  A chunk whose summed
+// |ew| exceeds 80 in some channel is evaluated token by token on the CUDA cores
+// from the state or adjoint held in tensor memory.
+#include "wkv_launch.cuh"
+#include "wkv_tc.cuh"
+
+namespace wkv {
+
+using namespace tc;
+
+namespace {
+
+constexpr int kBL = 32;                  // tokens per chunk
+constexpr int kBT = 2;                   // bf16 terms per operand
+constexpr int kBP = 3;                   // products per contraction: (0,0), (0,1), (1,0)
+constexpr int kBThr = 128;
+constexpr int kBTok = kBL * kHead;       // bf16 elements of a 32 x 64 token tile (4 KB)
+constexpr int kBAp = kBL * kBL;          // bf16 elements of a 32 x 32 chunk matrix (2 KB)
+constexpr int kBSt = kHead * kHead;      // bf16 elements of a 64 x 64 state tile (8 KB)
+constexpr int kBF = kBL * kHead;         // floats of a 32 x 64 fp32 tile (8 KB)
+constexpr float kLog2eB = 1.4426950408889634f;
+constexpr float kLamMaxB = 80.0f * kLog2eB;
+
+__device__ __forceinline__ constexpr int bprod_a(int q) { return q == 2 ? 1 : 0; }
+__device__ __forceinline__ constexpr int bprod_b(int q) { return q == 1 ? 1 : 0; }
+
+// Two-term split of a pair (a low, b high): packed first terms and packed second terms.
+__device__ __forceinline__ void split2_pair(float a, float b, uint32_t &t0, uint32_t &t1) {
+    t0 = pack_bf16(a, b);
+    const float ra = a - __uint_as_float(t0 << 16), rb = b - __uint_as_float(t0 & 0xFFFF0000u);
+    t1 = pack_bf16(ra, rb);
+}
+
+__device__ __forceinline__ void put_pair2(__nv_bfloat16 (*tiles)[kBTok], int row, int col, float a, float b) {
+    uint32_t t0, t1;
+    split2_pair(a, b, t0, t1);
+    const uint32_t o = swz(row, col);
+    st_u32(tiles[0], o, t0);
+    st_u32(tiles[1], o, t1);
+}
+
+// fp32 [32][64] tile, float pairs XOR-swizzled by row so that a row written by a
+// warp and an mma-fragment read (8 rows x 4 pairs) are both conflict-free.
+__device__ __forceinline__ int fidx(int p, int i) { return p * kHead + ((((i >> 1) ^ ((p & 7) << 2))) << 1) + (i & 1); }
+
+__device__ __forceinline__ uint64_t bdadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// no-swizzle K-major descriptor of a 32-row chunk matrix (units of 8 columns, 512 B apart)
+__device__ __forceinline__ uint64_t desc_cm(const __nv_bfloat16 *tile) { return smem_desc(tile, 512, 128); }
+
+struct BDecay {
+    float psum[4][kHead];
+    float pabs[4][kHead];
+};
+
+// Per-chunk decay prefix: quarter sums exchanged through `ds` (caller syncs between).
+// Returns the CTA-uniform exact-chunk verdict; L0, L1 = Lam at the thread's first token
+// (log2 units), tot = Lam_L.
+__device__ __forceinline__ void decay_sums(const float2 (&xw)[8], BDecay &ds, int warp, int ch, float &s0,
+                                           float &s1, float &a0, float &a1) {
+    s0 = s1 = a0 = a1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        s0 += xw[e].x * kLog2eB;
+        s1 += xw[e].y * kLog2eB;
+        a0 += fabsf(xw[e].x * kLog2eB);
+        a1 += fabsf(xw[e].y * kLog2eB);
+    }
+    *reinterpret_cast<float2 *>(&ds.psum[warp][ch]) = make_float2(s0, s1);
+    *reinterpret_cast<float2 *>(&ds.pabs[warp][ch]) = make_float2(a0, a1);
+}
+__device__ __forceinline__ bool decay_prefix(const BDecay &ds, int warp, int ch, float &L0, float &L1, float &tot0,
+                                             float &tot1) {
+    float ab0 = 0.f, ab1 = 0.f;
+    L0 = L1 = tot0 = tot1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 ps = *reinterpret_cast<const float2 *>(&ds.psum[q][ch]);
+        const float2 pa = *reinterpret_cast<const float2 *>(&ds.pabs[q][ch]);
+        if (q < warp) {
+            L0 += ps.x;
+            L1 += ps.y;
+        }
+        tot0 += ps.x;
+        tot1 += ps.y;
+        ab0 += pa.x;
+        ab1 += pa.y;
+    }
+    return __any_sync(0xffffffffu, !(ab0 <= kLamMaxB) || !(ab1 <= kLamMaxB));
+}
+
+// ======================================================================== S kind
+struct SSmem {
+    __nv_bfloat16 dY[kBT][kBTok];    // K-major A of dA and of dY S_in^T
+    __nv_bfloat16 V[kBT][kBTok];     // K-major B of dA; MN-major B of the state update
+    __nv_bfloat16 Kt[kBT][kBTok];    // MN-major B of dA Kt; MN-major A of the state update
+    __nv_bfloat16 dAp[kBT][kBAp];    // dA' (row p, s contiguous), no swizzle: K-major A of dA' Kt
+    __nv_bfloat16 Sin[kBT][kBSt];    // S_in (row i, j contiguous), 128B-swizzled: K-major B of dY S_in^T
+    float E[kBF];                    // e^{Lam_p} (fidx); after the epilogue: the chunk's z or x part
+    float R[kBF];                    // raw r (fidx)
+    float vdy[kBL], ruk[kBL];
+    float dec[kHead], u[kHead];
+    float dusum[4][kHead];
+    uint32_t tmem_base;
+    alignas(8) uint64_t bar_m1, bar_p, bar_s, bar_fin;
+};
+static_assert(sizeof(SSmem) + 1024 <= 74 * 1024, "three CTAs per SM must fit");
+static_assert(offsetof(SSmem, dY) % 1024 == 0 && offsetof(SSmem, V) % 1024 == 0 && offsetof(SSmem, Kt) % 1024 == 0 &&
+                  offsetof(SSmem, Sin) % 1024 == 0,
+              "swizzled tiles start on 1024-byte boundaries");
+struct SExact {   // exact chunks: raw k, v, ew in the dY, V, Kt tiles; dy in S_in[0]; R keeps r
+    float k[kBL][kHead], v[kBL][kHead], ew[kBL][kHead];
+};
+static_assert(sizeof(SExact) <= offsetof(SSmem, dAp) - offsetof(SSmem, dY), "exact-chunk inputs fit");
+static_assert(sizeof(float) * kBL * kHead <= sizeof(__nv_bfloat16) * kBSt, "exact-chunk dy fits in S_in[0]");
+
+}  // namespace
+
+// One pass per direction: causal first (forward in time), then, bidirectional,
+// the anti-causal pass (backward in time).
+template <bool BIDIR>
+__global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__restrict__ r,
+                                                              const float *__restrict__ k,
+                                                              const float *__restrict__ v,
+                                                              const float *__restrict__ w,
+                                                              const float *__restrict__ dy, BwdParams prm,
+                                                              float *__restrict__ ztot) {
+    extern __shared__ unsigned char smem_dyn[];
+    SSmem &sm = *reinterpret_cast<SSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    BDecay &ds = *reinterpret_cast<BDecay *>(&sm.dAp[0][0]);
+    SExact &xe = *reinterpret_cast<SExact *>(&sm.dY[0][0]);
+    float(*xdy)[kHead] = reinterpret_cast<float(*)[kHead]>(&sm.Sin[0][0]);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = prm.T, C = prm.C, H = prm.H;
+    const int h = blockIdx.x % H, b = blockIdx.x / H;
+    const int cbase = h * kHead;
+    const int nch = (T + kBL - 1) / kBL;
+    const int ch = 2 * lane, pq = 8 * warp;
+    const int q4 = lane & 3;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+
+    if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
+    if (tid == 0) {
+        mbar_init(&sm.bar_m1, 1);
+        mbar_init(&sm.bar_p, 1);
+        mbar_init(&sm.bar_s, 1);
+        mbar_init(&sm.bar_fin, 2);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 128);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tQ = sm.tmem_base, tS = sm.tmem_base + 64;   // dA (32 cols) then dQ (64) share 0..63
+
+    constexpr uint32_t kTokB = kBTok * 2, kApB = kBAp * 2, kStB = kBSt * 2;
+    const uint64_t dYk = desc_k(sm.dY[0], 0), dVk = desc_k(sm.V[0], 0), dVm = desc_mn(sm.V[0], 0, 16);
+    const uint64_t dKm = desc_mn(sm.Kt[0], 0, 16), dAp = desc_cm(sm.dAp[0]), dSk = desc_k(sm.Sin[0], 0);
+    constexpr uint32_t kIdDA = idesc_bf16(64, 32, false, false);    // dY (K-major) x V (K-major)
+    constexpr uint32_t kIdS = idesc_bf16(64, 64, true, true);       // Kt^T (MN) x V (MN)
+    constexpr uint32_t kIdQ1 = idesc_bf16(64, 64, false, true);     // dA' (K) x Kt (MN)
+    constexpr uint32_t kIdQ2 = idesc_bf16(64, 64, false, false);    // dY (K) x S_in (K-major, rows i)
+
+    float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    auto time_of = [&](int dir, int c, int p) { return dir > 0 ? c * kBL + p : T - 1 - (c * kBL + p); };
+    auto load_chunk = [&](int dir, int c) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int p = pq + e;
+            if (c * kBL + p < T) {
+                const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
+                xr_[e] = __ldg(reinterpret_cast<const float2 *>(r + o));
+                xk_[e] = __ldg(reinterpret_cast<const float2 *>(k + o));
+                xv_[e] = __ldg(reinterpret_cast<const float2 *>(v + o));
+                xw_[e] = __ldg(reinterpret_cast<const float2 *>(w + o));
+                xd_[e] = __ldg(reinterpret_cast<const float2 *>(dy + o));
+            } else {
+                xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
+            }
+        }
+    };
+
+    uint32_t ph = 0;
+    bool ok = true;
+    float du0 = 0.f, du1 = 0.f;      // sum over the causal pass of r k (v.dy), channels ch, ch + 1
+    float zrun = 0.f;                // thread i < 64: running prefix (causal) or suffix (anti) of the dw part
+    constexpr int npass = BIDIR ? 2 : 1;
+    load_chunk(1, 0);
+
+    for (int pass = 0; pass < npass && ok; ++pass) {
+        const int dir = pass == 0 ? 1 : -1;
+        const bool causal = dir > 0;
+        {   // S = 0 at the start of every pass
+            float z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0.f;
+            tmem_st32(tS + lane_off, z);
+            tmem_st32(tS + lane_off + 32, z);
+            tmem_wait_st();
+        }
+        for (int c = 0; c < nch; ++c) {
+            // ================= transform =================
+            float s0, s1, a0, a1;
+            decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
+            // v.dy and sum r u k per token (bonus scalars), reduced over the 64 channels
+            {
+                float pv[8], pr[8];
+                const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    pv[e] = fmaf(xv_[e].x, xd_[e].x, xv_[e].y * xd_[e].y);
+                    pr[e] = fmaf(xr_[e].x * u0, xk_[e].x, xr_[e].y * u1 * xk_[e].y);
+                }
+                const float vv = transpose_reduce8(pv, lane), rr = transpose_reduce8(pr, lane);
+                if ((lane & 3) == 0) {
+                    sm.vdy[pq + (lane >> 2)] = vv;
+                    sm.ruk[pq + (lane >> 2)] = rr;
+                }
+            }
+            __syncthreads();
+            float L0, L1, tot0, tot1;
+            const bool exact = decay_prefix(ds, warp, ch, L0, L1, tot0, tot1);
+            if (causal) {
+                // bonus parts: dr = u k (v.dy) is the base the epilogue adds to; dk, dv
+                // get theirs here (the G kind adds onto them); du partial sums
+                const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int p = pq + e;
+                    if (c * kBL + p >= T) continue;
+                    const float vd = sm.vdy[p], ruk = sm.ruk[p];
+                    const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
+                    *reinterpret_cast<float2 *>(prm.dr + o) = make_float2(u0 * xk_[e].x * vd, u1 * xk_[e].y * vd);
+                    *reinterpret_cast<float2 *>(prm.dk + o) = make_float2(u0 * xr_[e].x * vd, u1 * xr_[e].y * vd);
+                    *reinterpret_cast<float2 *>(prm.dv + o) = make_float2(ruk * xd_[e].x, ruk * xd_[e].y);
+                    du0 = fmaf(xr_[e].x * xk_[e].x, vd, du0);
+                    du1 = fmaf(xr_[e].y * xk_[e].y, vd, du1);
+                }
+            }
+            // raw r for the dw parts (both paths)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) *reinterpret_cast<float2 *>(&sm.R[fidx(pq + e, ch)]) = xr_[e];
+            if (!exact) {
+                if (warp == 0) *reinterpret_cast<float2 *>(&sm.dec[ch]) = make_float2(exp2f(tot0), exp2f(tot1));
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int p = pq + e;
+                    const float e0 = fast_exp2(L0), e1 = fast_exp2(L1);
+                    *reinterpret_cast<float2 *>(&sm.E[fidx(p, ch)]) = make_float2(e0, e1);
+                    L0 += xw_[e].x * kLog2eB;
+                    L1 += xw_[e].y * kLog2eB;
+                    put_pair2(sm.dY, p, ch, xd_[e].x, xd_[e].y);
+                    put_pair2(sm.V, p, ch, xv_[e].x, xv_[e].y);
+                    put_pair2(sm.Kt, p, ch, xk_[e].x * fast_exp2(-L0), xk_[e].y * fast_exp2(-L1));
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int p = pq + e;
+                    *reinterpret_cast<float2 *>(&xe.k[p][ch]) = xk_[e];
+                    *reinterpret_cast<float2 *>(&xe.v[p][ch]) = xv_[e];
+                    *reinterpret_cast<float2 *>(&xe.ew[p][ch]) = xw_[e];
+                    *reinterpret_cast<float2 *>(&xdy[p][ch]) = xd_[e];
+                }
+            }
+            if (c + 1 < nch) load_chunk(dir, c + 1);
+            else if (BIDIR && pass == 0) load_chunk(-1, 0);
+            fence_proxy_async_smem();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+
+            if (!exact) {
+                // ===== dA = dY V^T (warp 0), S += Kt^T V (warp 1) =====
+                if (tid == 0) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tQ, bdadd(dYk, bprod_a(q) * kTokB + 32 * ks), bdadd(dVk, bprod_b(q) * kTokB + 32 * ks),
+                                     kIdDA, ks > 0 || q > 0);
+                    mma_commit(&sm.bar_m1);
+                } else if (tid == 32) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tS, bdadd(dKm, bprod_a(q) * kTokB + 2048 * ks), bdadd(dVm, bprod_b(q) * kTokB + 2048 * ks),
+                                     kIdS, true);
+                    mma_commit(&sm.bar_s);
+                }
+                ok = mbar_wait_bounded(&sm.bar_m1, ph);
+                ok = __syncthreads_and(ok);
+                if (!ok) break;
+                fence_after_sync();
+                // ===== mask: dA' = strict-lower(dA) =====
+                if (warp < 2) {
+                    float a[16];
+                    tmem_ld_16x256b_x4(tQ + lane_off, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int p = 16 * warp + (lane >> 2) + 8 * hr;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const int s0_ = 8 * m + 2 * q4;
+                            const float x0 = s0_ < p ? a[4 * m + 2 * hr] : 0.f;
+                            const float x1 = s0_ + 1 < p ? a[4 * m + 2 * hr + 1] : 0.f;
+                            uint32_t t0, t1;
+                            split2_pair(x0, x1, t0, t1);
+                            const uint32_t o = (uint32_t)(m * 512 + p * 16 + 4 * q4);
+                            st_u32(sm.dAp[0], o, t0);
+                            st_u32(sm.dAp[1], o, t1);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                fence_before_sync();
+                __syncthreads();
+                fence_after_sync();
+                // ===== dQ = dA' Kt + dY S_in^T =====
+                if (tid == 0) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tQ, bdadd(dAp, bprod_a(q) * kApB + 1024 * ks), bdadd(dKm, bprod_b(q) * kTokB + 2048 * ks),
+                                     kIdQ1, ks > 0 || q > 0);
+                    if (c > 0) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                            for (int q = 0; q < kBP; ++q)
+                                mma_bf16(tQ, bdadd(dYk, bprod_a(q) * kTokB + 32 * ks), bdadd(dSk, bprod_b(q) * kStB + 32 * ks),
+                                         kIdQ2, true);
+                    }
+                    mma_commit(&sm.bar_p);
+                }
+                ok = mbar_wait_bounded(&sm.bar_p, ph) && mbar_wait_bounded(&sm.bar_s, ph);
+                ph ^= 1u;
+                ok = __syncthreads_and(ok);
+                if (!ok) break;
+                fence_after_sync();
+                // ===== epilogue: dr' = e^{Lam} dQ added to dr; its dw part into E; state =====
+                if (warp < 2) {
+                    float qv[32];
+                    tmem_ld_16x256b_x8(tQ + lane_off, qv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int p = 16 * warp + (lane >> 2) + 8 * hr;
+                        const bool valid = c * kBL + p < T;
+                        float2 *dst = reinterpret_cast<float2 *>(
+                            prm.dr + ((size_t)b * T + (valid ? time_of(dir, c, p) : 0)) * C + cbase + 2 * q4);
+                        float2 prev[8];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) prev[m] = valid ? dst[4 * m] : make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            const int i = 8 * m + 2 * q4;
+                            const float2 e2 = *reinterpret_cast<const float2 *>(&sm.E[fidx(p, i)]);
+                            const float2 r2 = *reinterpret_cast<const float2 *>(&sm.R[fidx(p, i)]);
+                            const float d0 = e2.x * qv[4 * m + 2 * hr], d1 = e2.y * qv[4 * m + 2 * hr + 1];
+                            if (valid) dst[4 * m] = make_float2(prev[m].x + d0, prev[m].y + d1);
+                            // the dw part of this token: z = r dr' (causal), x = r dr' (anti-causal)
+                            *reinterpret_cast<float2 *>(&sm.E[fidx(p, i)]) = make_float2(r2.x * d0, r2.y * d1);
+                        }
+                    }
+                }
+                {
+                    // S rows scaled by e^{Lam_L}, back to TMEM, two-term copy into S_in
+                    float sv[32];
+                    tmem_ld_16x256b_x8(tS + lane_off, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int i = 16 * warp + (lane >> 2) + 8 * hr;
+                        const float dsc = sm.dec[i];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            const float v0 = sv[4 * m + 2 * hr] * dsc, v1 = sv[4 * m + 2 * hr + 1] * dsc;
+                            sv[4 * m + 2 * hr] = v0;
+                            sv[4 * m + 2 * hr + 1] = v1;
+                            uint32_t t0, t1;
+                            split2_pair(v0, v1, t0, t1);
+                            const uint32_t o = swz(i, 8 * m + 2 * q4);
+                            st_u32(sm.Sin[0], o, t0);
+                            st_u32(sm.Sin[1], o, t1);
+                        }
+                    }
+                    tmem_st_16x256b_x8(tS + lane_off, sv);
+                    tmem_wait_st();
+                }
+            } else {
+                // ===== exact chunk: token by token from S in TMEM (rows i: lanes 0..15 of each
+                // quarter), 16 columns at a time so that no whole row is held in registers =====
+                const bool rl = lane < 16;
+                const int i = 16 * warp + (lane & 15);
+                for (int p = 0; p < kBL; ++p) {
+                    if (c * kBL + p >= T) break;   // uniform
+                    float acc = 0.f;
+#pragma unroll 1
+                    for (int qc = 0; qc < 4; ++qc) {
+                        float s16[16];
+                        tmem_ld16(tS + lane_off + 16 * qc, s16);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc = fmaf(s16[e], xdy[p][16 * qc + e], acc);
+                    }
+                    const float dd = rl ? __expf(xe.ew[p][i]) : 0.f, kk = rl ? xe.k[p][i] : 0.f;
+#pragma unroll 1
+                    for (int qc = 0; qc < 4; ++qc) {
+                        float s16[16];
+                        tmem_ld16(tS + lane_off + 16 * qc, s16);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) s16[e] = fmaf(dd, s16[e], kk * xe.v[p][16 * qc + e]);
+                        tmem_st16(tS + lane_off + 16 * qc, s16);
+                    }
+                    tmem_wait_st();
+                    if (rl) {
+                        const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + i;
+                        prm.dr[o] += acc;
+                        sm.E[fidx(p, i)] = sm.R[fidx(p, i)] * acc;
+                    }
+                }
+                __syncthreads();   // every row owner is done with the dy tile (in S_in[0])
+#pragma unroll 1
+                for (int qc = 0; qc < 4; ++qc) {
+                    float s16[16];
+                    tmem_ld16(tS + lane_off + 16 * qc, s16);
+                    tmem_wait_ld();
+                    if (rl) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            uint32_t t0, t1;
+                            split2_pair(s16[2 * m], s16[2 * m + 1], t0, t1);
+                            const uint32_t o = swz(i, 16 * qc + 2 * m);
+                            st_u32(sm.Sin[0], o, t0);
+                            st_u32(sm.Sin[1], o, t1);
+                        }
+                    }
+                }
+            }
+            // ===== dw part: causal pass dw = -(running prefix of z); anti-causal dw -= running suffix of x =====
+            __syncthreads();
+            if (tid < kHead) {
+                // the previous dw values of the chunk are loaded before any store (one L2
+                // round trip per chunk instead of one per token), 16 tokens at a time
+                const int i = tid;
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    float prev[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int p = 16 * hb + e;
+                        prev[e] = (!causal && c * kBL + p < T)
+                                      ? prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i]
+                                      : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int p = 16 * hb + e;
+                        if (c * kBL + p >= T) break;
+                        zrun += sm.E[fidx(p, i)];
+                        prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i] = prev[e] - zrun;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+        }
+        if (causal && tid < kHead) ztot[(size_t)b * C + cbase + tid] = zrun;   // z total of the S kind
+        zrun = 0.f;
+    }
+    // du partial of this (b, h): reduce the four token quarters
+    *reinterpret_cast<float2 *>(&sm.dusum[warp][ch]) = make_float2(du0, du1);
+    __syncthreads();
+    if (tid < kHead)
+        prm.du_part[(size_t)b * C + cbase + tid] = sm.dusum[0][tid] + sm.dusum[1][tid] + sm.dusum[2][tid] + sm.dusum[3][tid];
+    if (!ok && (tid == 0 || tid == 32)) {
+        mma_commit(&sm.bar_fin);
+        if (tid == 0) mbar_wait_bounded(&sm.bar_fin, 0);
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(sm.tmem_base, 128);
+}
+
+namespace {
+// ======================================================================== G kind
+struct GSmem {
+    __nv_bfloat16 Q[kBT][kBTok];     // K-major B of A^T; MN-major B of dA'^T Q; MN-major A of Q^T dY
+    __nv_bfloat16 Kt[kBT][kBTok];    // K-major A of A^T and of Kt Gt
+    __nv_bfloat16 V[kBT][kBTok];     // K-major A of dA^T and of V Gt^T
+    __nv_bfloat16 dY[kBT][kBTok];    // K-major B of dA^T; MN-major B of A'^T dY and of Q^T dY
+    __nv_bfloat16 Ap[kBT][kBAp];     // A'^T (row s, tau contiguous), no swizzle: K-major A of A'^T dY
+    __nv_bfloat16 dAp[kBT][kBAp];    // dA'^T likewise: K-major A of dA'^T Q
+    __nv_bfloat16 Gt[kBT][kBSt];     // Gt (row i, j contiguous), 128B-swizzled: K-major B of V Gt^T, MN-major B of Kt Gt
+    float F[kBF];                    // e^{-Lam_{s+1}} (fidx); after the first epilogue: the chunk's z or x part
+    float Kr[kBF];                   // raw k (fidx)
+    float dec[kHead];
+    uint32_t tmem_base;
+    alignas(8) uint64_t bar_m1, bar_k, bar_v, bar_g, bar_fin;
+};
+static_assert(sizeof(GSmem) + 1024 <= 74 * 1024, "three CTAs per SM must fit");
+static_assert(offsetof(GSmem, Q) % 1024 == 0 && offsetof(GSmem, Kt) % 1024 == 0 && offsetof(GSmem, V) % 1024 == 0 &&
+                  offsetof(GSmem, dY) % 1024 == 0 && offsetof(GSmem, Gt) % 1024 == 0,
+              "swizzled tiles start on 1024-byte boundaries");
+struct GExact {   // exact chunks: raw r, v, ew, dy in the Q, Kt, V, dY tiles (Kr keeps k)
+    float r[kBL][kHead], v[kBL][kHead], ew[kBL][kHead], dy[kBL][kHead];
+};
+static_assert(sizeof(GExact) <= offsetof(GSmem, Ap) - offsetof(GSmem, Q), "exact-chunk inputs fit");
+// exact chunks: k_p[i] G[i][j] partials, float4 groups XOR-swizzled by row (fits in Gt)
+__device__ __forceinline__ int pidx(int i, int j) { return i * kHead + ((((j >> 2) ^ (i & 15))) << 2) + (j & 3); }
+static_assert(sizeof(float) * kHead * kHead <= sizeof(__nv_bfloat16) * kBT * kBSt, "partials fit in Gt");
+}  // namespace
+
+// Passes: bidirectional, the anti-causal one first (its chunks in reverse processing
+// order run forward in time), then the causal one (backward in time); chunks of a
+// pass in reverse processing order, tokens of a chunk from the last to the first.
+template <bool BIDIR>
+__global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__restrict__ r,
+                                                              const float *__restrict__ k,
+                                                              const float *__restrict__ v,
+                                                              const float *__restrict__ w,
+                                                              const float *__restrict__ dy, BwdParams prm,
+                                                              const float *__restrict__ ztot) {
+    extern __shared__ unsigned char smem_dyn[];
+    GSmem &sm = *reinterpret_cast<GSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    BDecay &ds = *reinterpret_cast<BDecay *>(&sm.Ap[0][0]);
+    GExact &xe = *reinterpret_cast<GExact *>(&sm.Q[0][0]);
+    float *part = reinterpret_cast<float *>(&sm.Gt[0][0]);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = prm.T, C = prm.C, H = prm.H;
+    const int h = blockIdx.x % H, b = blockIdx.x / H;
+    const int cbase = h * kHead;
+    const int nch = (T + kBL - 1) / kBL;
+    const int ch = 2 * lane, pq = 8 * warp;
+    const int q4 = lane & 3;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+
+    if (tid == 0) {
+        mbar_init(&sm.bar_m1, 1);
+        mbar_init(&sm.bar_k, 1);
+        mbar_init(&sm.bar_v, 1);
+        mbar_init(&sm.bar_g, 1);
+        mbar_init(&sm.bar_fin, 2);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 128);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    // TMEM: A^T at 0..31 and dA^T at 32..63, then dKt, then dV, at 0..63; G at 64..127
+    const uint32_t tA = sm.tmem_base, tG = sm.tmem_base + 64;
+
+    constexpr uint32_t kTokB = kBTok * 2, kApB = kBAp * 2, kStB = kBSt * 2;
+    const uint64_t dQk = desc_k(sm.Q[0], 0), dQm = desc_mn(sm.Q[0], 0, 16), dKk = desc_k(sm.Kt[0], 0);
+    const uint64_t dVk = desc_k(sm.V[0], 0), dYk = desc_k(sm.dY[0], 0), dYm = desc_mn(sm.dY[0], 0, 16);
+    const uint64_t dAp = desc_cm(sm.Ap[0]), ddAp = desc_cm(sm.dAp[0]);
+    const uint64_t dGk = desc_k(sm.Gt[0], 0), dGm = desc_mn(sm.Gt[0], 0, 16);
+    constexpr uint32_t kIdAT = idesc_bf16(64, 32, false, false);   // Kt (K) x Q (K);  V (K) x dY (K)
+    constexpr uint32_t kIdG = idesc_bf16(64, 64, true, true);      // Q^T (MN) x dY (MN)
+    constexpr uint32_t kIdKM = idesc_bf16(64, 64, false, true);    // dA'^T (K) x Q (MN);  A'^T (K) x dY (MN);  Kt (K) x Gt (MN)
+    constexpr uint32_t kIdKK = idesc_bf16(64, 64, false, false);   // V (K) x Gt (K-major, rows i)
+
+    float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    auto time_of = [&](int dir, int c, int p) { return dir > 0 ? c * kBL + p : T - 1 - (c * kBL + p); };
+    auto load_chunk = [&](int dir, int c) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int p = pq + e;
+            if (c * kBL + p < T) {
+                const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
+                xr_[e] = __ldg(reinterpret_cast<const float2 *>(r + o));
+                xk_[e] = __ldg(reinterpret_cast<const float2 *>(k + o));
+                xv_[e] = __ldg(reinterpret_cast<const float2 *>(v + o));
+                xw_[e] = __ldg(reinterpret_cast<const float2 *>(w + o));
+                xd_[e] = __ldg(reinterpret_cast<const float2 *>(dy + o));
+            } else {
+                xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
+            }
+        }
+    };
+
+    uint32_t ph = 0;
+    bool ok = true;
+    float zrun = 0.f;     // thread i < 64: running prefix of z (anti-causal pass), then suffix of x (causal)
+    float zg_tot = 0.f;   // thread i < 64: z total of the anti-causal pass
+    constexpr int npass = BIDIR ? 2 : 1;
+    load_chunk(BIDIR ? -1 : 1, nch - 1);
+
+    for (int pass = 0; pass < npass && ok; ++pass) {
+        const int dir = (BIDIR && pass == 0) ? -1 : 1;
+        const bool last = pass == npass - 1;   // the causal pass: backward in time
+        {   // G = 0 at the start of every pass
+            float z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0.f;
+            tmem_st32(tG + lane_off, z);
+            tmem_st32(tG + lane_off + 32, z);
+            tmem_wait_st();
+        }
+        for (int c = nch - 1; c >= 0; --c) {
+            const bool first = c == nch - 1;   // no adjoint from later chunks yet
+            // ================= transform =================
+            float s0, s1, a0, a1;
+            decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
+            __syncthreads();
+            float L0, L1, tot0, tot1;
+            const bool exact = decay_prefix(ds, warp, ch, L0, L1, tot0, tot1);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) *reinterpret_cast<float2 *>(&sm.Kr[fidx(pq + e, ch)]) = xk_[e];
+            if (!exact) {
+                if (warp == 0) *reinterpret_cast<float2 *>(&sm.dec[ch]) = make_float2(exp2f(tot0), exp2f(tot1));
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int p = pq + e;
+                    put_pair2(sm.Q, p, ch, xr_[e].x * fast_exp2(L0), xr_[e].y * fast_exp2(L1));
+                    L0 += xw_[e].x * kLog2eB;
+                    L1 += xw_[e].y * kLog2eB;
+                    const float f0 = fast_exp2(-L0), f1 = fast_exp2(-L1);
+                    *reinterpret_cast<float2 *>(&sm.F[fidx(p, ch)]) = make_float2(f0, f1);
+                    put_pair2(sm.Kt, p, ch, xk_[e].x * f0, xk_[e].y * f1);
+                    put_pair2(sm.V, p, ch, xv_[e].x, xv_[e].y);
+                    put_pair2(sm.dY, p, ch, xd_[e].x, xd_[e].y);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int p = pq + e;
+                    *reinterpret_cast<float2 *>(&xe.r[p][ch]) = xr_[e];
+                    *reinterpret_cast<float2 *>(&xe.v[p][ch]) = xv_[e];
+                    *reinterpret_cast<float2 *>(&xe.ew[p][ch]) = xw_[e];
+                    *reinterpret_cast<float2 *>(&xe.dy[p][ch]) = xd_[e];
+                }
+            }
+            if (c > 0) load_chunk(dir, c - 1);
+            else if (BIDIR && pass == 0) load_chunk(1, nch - 1);
+            fence_proxy_async_smem();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+
+            if (!exact) {
+                // ===== Gt = diag(Gam) G_out in TMEM, and its two-term copy =====
+                if (!first) {
+                    float gv[32];
+                    tmem_ld_16x256b_x8(tG + lane_off, gv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int i = 16 * warp + (lane >> 2) + 8 * hr;
+                        const float dsc = sm.dec[i];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            const float g0 = gv[4 * m + 2 * hr] * dsc, g1 = gv[4 * m + 2 * hr + 1] * dsc;
+                            gv[4 * m + 2 * hr] = g0;
+                            gv[4 * m + 2 * hr + 1] = g1;
+                            uint32_t t0, t1;
+                            split2_pair(g0, g1, t0, t1);
+                            const uint32_t o = swz(i, 8 * m + 2 * q4);
+                            st_u32(sm.Gt[0], o, t0);
+                            st_u32(sm.Gt[1], o, t1);
+                        }
+                    }
+                    tmem_st_16x256b_x8(tG + lane_off, gv);
+                    tmem_wait_st();
+                    fence_proxy_async_smem();
+                    fence_before_sync();
+                    __syncthreads();
+                    fence_after_sync();
+                }
+                // ===== A^T = Kt Q^T, dA^T = V dY^T (warp 0);  G += Q^T dY (warp 1) =====
+                if (tid == 0) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q) {
+                            mma_bf16(tA, bdadd(dKk, bprod_a(q) * kTokB + 32 * ks), bdadd(dQk, bprod_b(q) * kTokB + 32 * ks),
+                                     kIdAT, ks > 0 || q > 0);
+                            mma_bf16(tA + 32, bdadd(dVk, bprod_a(q) * kTokB + 32 * ks),
+                                     bdadd(dYk, bprod_b(q) * kTokB + 32 * ks), kIdAT, ks > 0 || q > 0);
+                        }
+                    mma_commit(&sm.bar_m1);
+                } else if (tid == 32) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tG, bdadd(dQm, bprod_a(q) * kTokB + 2048 * ks), bdadd(dYm, bprod_b(q) * kTokB + 2048 * ks),
+                                     kIdG, true);
+                    mma_commit(&sm.bar_g);
+                }
+                ok = mbar_wait_bounded(&sm.bar_m1, ph);
+                ok = __syncthreads_and(ok);
+                if (!ok) break;
+                fence_after_sync();
+                // ===== masks: A'^T, dA'^T = strict-upper (tau > s) of A^T, dA^T =====
+                if (warp < 2) {
+                    float a[32];
+                    tmem_ld_16x256b_x8(tA + lane_off, a);   // columns 0..31 A^T, 32..63 dA^T
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int s_ = 16 * warp + (lane >> 2) + 8 * hr;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const int t0_ = 8 * m + 2 * q4;
+                            const bool k0 = t0_ > s_, k1 = t0_ + 1 > s_;
+                            uint32_t x0, x1;
+                            const uint32_t o = (uint32_t)(m * 512 + s_ * 16 + 4 * q4);
+                            split2_pair(k0 ? a[4 * m + 2 * hr] : 0.f, k1 ? a[4 * m + 2 * hr + 1] : 0.f, x0, x1);
+                            st_u32(sm.Ap[0], o, x0);
+                            st_u32(sm.Ap[1], o, x1);
+                            split2_pair(k0 ? a[16 + 4 * m + 2 * hr] : 0.f, k1 ? a[16 + 4 * m + 2 * hr + 1] : 0.f, x0, x1);
+                            st_u32(sm.dAp[0], o, x0);
+                            st_u32(sm.dAp[1], o, x1);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                fence_before_sync();
+                __syncthreads();
+                fence_after_sync();
+                // ===== dKt = dA'^T Q + V Gt^T =====
+                if (tid == 0) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tA, bdadd(ddAp, bprod_a(q) * kApB + 1024 * ks), bdadd(dQm, bprod_b(q) * kTokB + 2048 * ks),
+                                     kIdKM, ks > 0 || q > 0);
+                    if (!first) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                            for (int q = 0; q < kBP; ++q)
+                                mma_bf16(tA, bdadd(dVk, bprod_a(q) * kTokB + 32 * ks), bdadd(dGk, bprod_b(q) * kStB + 32 * ks),
+                                         kIdKK, true);
+                    }
+                    mma_commit(&sm.bar_k);
+                }
+                ok = mbar_wait_bounded(&sm.bar_k, ph);
+                ok = __syncthreads_and(ok);
+                if (!ok) break;
+                fence_after_sync();
+                // ===== epilogue 1: dk' = e^{-Lam_{s+1}} dKt added to dk; its dw part into F =====
+                if (warp < 2) {
+                    float kv[32];
+                    tmem_ld_16x256b_x8(tA + lane_off, kv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int s_ = 16 * warp + (lane >> 2) + 8 * hr;
+                        const bool valid = c * kBL + s_ < T;
+                        float2 *dst = reinterpret_cast<float2 *>(
+                            prm.dk + ((size_t)b * T + (valid ? time_of(dir, c, s_) : 0)) * C + cbase + 2 * q4);
+                        float2 prev[8];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) prev[m] = valid ? dst[4 * m] : make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            const int i = 8 * m + 2 * q4;
+                            const float2 f2 = *reinterpret_cast<const float2 *>(&sm.F[fidx(s_, i)]);
+                            const float2 k2 = *reinterpret_cast<const float2 *>(&sm.Kr[fidx(s_, i)]);
+                            const float d0 = f2.x * kv[4 * m + 2 * hr], d1 = f2.y * kv[4 * m + 2 * hr + 1];
+                            if (valid) dst[4 * m] = make_float2(prev[m].x + d0, prev[m].y + d1);
+                            *reinterpret_cast<float2 *>(&sm.F[fidx(s_, i)]) = make_float2(k2.x * d0, k2.y * d1);
+                        }
+                    }
+                }
+                tmem_wait_ld();
+                fence_before_sync();
+                __syncthreads();
+                fence_after_sync();
+                // ===== dV = A'^T dY + Kt Gt =====
+                if (tid == 0) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tA, bdadd(dAp, bprod_a(q) * kApB + 1024 * ks), bdadd(dYm, bprod_b(q) * kTokB + 2048 * ks),
+                                     kIdKM, ks > 0 || q > 0);
+                    if (!first) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                            for (int q = 0; q < kBP; ++q)
+                                mma_bf16(tA, bdadd(dKk, bprod_a(q) * kTokB + 32 * ks), bdadd(dGm, bprod_b(q) * kStB + 2048 * ks),
+                                         kIdKM, true);
+                    }
+                    mma_commit(&sm.bar_v);
+                }
+                ok = mbar_wait_bounded(&sm.bar_v, ph) && mbar_wait_bounded(&sm.bar_g, ph);
+                ph ^= 1u;
+                ok = __syncthreads_and(ok);
+                if (!ok) break;
+                fence_after_sync();
+                // ===== epilogue 2: dv' added to dv =====
+                if (warp < 2) {
+                    float vv[32];
+                    tmem_ld_16x256b_x8(tA + lane_off, vv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int s_ = 16 * warp + (lane >> 2) + 8 * hr;
+                        if (c * kBL + s_ >= T) continue;
+                        float2 *dst = reinterpret_cast<float2 *>(prm.dv + ((size_t)b * T + time_of(dir, c, s_)) * C +
+                                                                 cbase + 2 * q4);
+                        float2 prev[8];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) prev[m] = dst[4 * m];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m)
+                            dst[4 * m] = make_float2(prev[m].x + vv[4 * m + 2 * hr], prev[m].y + vv[4 * m + 2 * hr + 1]);
+                    }
+                }
+            } else {
+                // ===== exact chunk: token by token (last to first) from G in TMEM, 16 columns
+                // at a time (rows i: lanes 0..15 of each quarter) =====
+                const bool rl = lane < 16;
+                const int i = 16 * warp + (lane & 15);
+                for (int p = kBL - 1; p >= 0; --p) {
+                    if (c * kBL + p >= T) continue;   // uniform
+                    const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase;
+                    const float kk = rl ? sm.Kr[fidx(p, i)] : 0.f;
+                    float acc = 0.f;
+#pragma unroll 1
+                    for (int qc = 0; qc < 4; ++qc) {
+                        float g16[16];
+                        tmem_ld16(tG + lane_off + 16 * qc, g16);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc = fmaf(g16[e], xe.v[p][16 * qc + e], acc);
+                        if (rl) {
+#pragma unroll
+                            for (int g = 0; g < 4; ++g)
+                                *reinterpret_cast<float4 *>(&part[pidx(i, 16 * qc + 4 * g)]) =
+                                    make_float4(kk * g16[4 * g], kk * g16[4 * g + 1], kk * g16[4 * g + 2], kk * g16[4 * g + 3]);
+                        }
+                    }
+                    if (rl) {
+                        prm.dk[o + i] += acc;
+                        sm.F[fidx(p, i)] = kk * acc;
+                    }
+                    __syncthreads();
+                    if (tid < kHead) {
+                        float s = 0.f;
+                        for (int ii = 0; ii < kHead; ++ii) s += part[pidx(ii, tid)];
+                        prm.dv[o + tid] += s;
+                    }
+                    const float dd = rl ? __expf(xe.ew[p][i]) : 0.f, rr = rl ? xe.r[p][i] : 0.f;
+#pragma unroll 1
+                    for (int qc = 0; qc < 4; ++qc) {
+                        float g16[16];
+                        tmem_ld16(tG + lane_off + 16 * qc, g16);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) g16[e] = fmaf(dd, g16[e], rr * xe.dy[p][16 * qc + e]);
+                        tmem_st16(tG + lane_off + 16 * qc, g16);
+                    }
+                    tmem_wait_st();
+                    __syncthreads();
+                }
+            }
+            // ===== dw part: anti-causal pass dw -= running prefix of z (forward in time);
+            // causal pass dw += z totals - running suffix of x (backward in time) =====
+            __syncthreads();
+            if (tid < kHead) {
+                // previous dw values loaded before any store, 16 tokens at a time
+                const int i = tid;
+                const float ztot_all = last ? ztot[(size_t)b * C + cbase + i] + zg_tot : 0.f;
+#pragma unroll
+                for (int hb = 1; hb >= 0; --hb) {
+                    float prev[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int p = 16 * hb + e;
+                        prev[e] = c * kBL + p < T ? prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i] : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 15; e >= 0; --e) {
+                        const int p = 16 * hb + e;
+                        if (c * kBL + p >= T) continue;
+                        zrun += sm.F[fidx(p, i)];
+                        prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i] =
+                            prev[e] + (last ? ztot_all - zrun : -zrun);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+        }
+        if (!last) zg_tot = zrun;
+        zrun = 0.f;
+    }
+    if (!ok && (tid == 0 || tid == 32)) {
+        mma_commit(&sm.bar_fin);
+        if (tid == 0) mbar_wait_bounded(&sm.bar_fin, 0);
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(sm.tmem_base, 128);
+}
+
+cudaError_t wkv6_bwd_split_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
+                                  const float *dy, const BwdParams &prm, float *ztot, float *du,
+                                  cudaStream_t stream) {
+    const size_t smS = sizeof(SSmem) + 1024, smG = sizeof(GSmem) + 1024;
+    auto ks = bidir ? wkv6_bwd_s_kernel<true> : wkv6_bwd_s_kernel<false>;
+    auto kg = bidir ? wkv6_bwd_g_kernel<true> : wkv6_bwd_g_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smS);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smG);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ks, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kg, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(prm.B * prm.H);
+    ks<<<grid, kBThr, smS, stream>>>(r, k, v, w, dy, prm, ztot);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    kg<<<grid, kBThr, smG, stream>>>(r, k, v, w, dy, prm, ztot);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return wkv6_du_reduce_launch(prm.B, prm.C, prm.du_part, du, stream);
+}
+
+}  // namespace wkv

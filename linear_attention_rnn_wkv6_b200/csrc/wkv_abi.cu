@@ -97,6 +97,14 @@ bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], bool bf16, int B, int T, int C
     return true;
 }
 
+// Algorithm of the fp32 backward: the chunked tensor-core kernels with split-bf16
+// operands (default) or the two-sweep recurrence (WKV6_BWD_PATH=recurrence).
+// The bf16 backward always runs the recurrence.  Read on every call.
+bool bwd_use_tensor_cores() {
+    const char *e = std::getenv("WKV6_BWD_PATH");
+    return !(e && std::strcmp(e, "recurrence") == 0);
+}
+
 // Shared by wkv6_bwd and wkv6_bwd_bf16 (inputs fp32 or bf16, gradients fp32).
 int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const void *r, const void *k,
                const void *v, const void *w, const float *u, const void *dy, float *dr, float *dk, float *dv,
@@ -108,10 +116,20 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
         if ((st = check_device()) != WKV_OK) return st;
         return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
     }
-    const size_t need = (size_t)B * (size_t)C * sizeof(float);
+    const bool tensor = !bf16 && bwd_use_tensor_cores();
+    const size_t need = (tensor ? 2 : 1) * (size_t)B * (size_t)C * sizeof(float);
     if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
     if ((st = check_device()) != WKV_OK) return st;
+    if (tensor) {
+        float *ws = static_cast<float *>(workspace);
+        BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, ws};
+        return wkv6_bwd_split_launch(bidirectional != 0, static_cast<const float *>(r), static_cast<const float *>(k),
+                                     static_cast<const float *>(v), static_cast<const float *>(w),
+                                     static_cast<const float *>(dy), prm, ws + (size_t)B * C, du, s) == cudaSuccess
+                   ? WKV_OK
+                   : WKV_ERR_CUDA;
+    }
     CUtensorMap maps[kBwdMaps];
     if (!make_bwd_maps(maps, bf16, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, static_cast<float *>(workspace)};
@@ -261,7 +279,8 @@ size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional) {
     (void)H;
     (void)bidirectional;
     if (B < 1 || C < 1) return 0;
-    return (size_t)B * (size_t)C * sizeof(float);
+    // per-batch du partials, and per-channel z totals for the tensor-core kernels
+    return 2 * (size_t)B * (size_t)C * sizeof(float);
 }
 
 int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, const float *k, const float *v,

@@ -80,7 +80,7 @@ def test_wkv6_forward_argument_errors(lib, fn):
 def test_wkv6_backward_argument_errors(lib):
     p = [FAKE + 256 * i for i in range(11)]
     ws = wkv.wkv6_bwd_workspace_bytes(2, 8, 128, 2, 1)
-    assert ws == 2 * 128 * 4
+    assert ws == 2 * 2 * 128 * 4                               # du partials and z totals, B*C floats each
     assert lib.wkv6_bwd(-1, 8, 128, 2, 1, *p, FAKE, ws, None) == WKV_ERR_ARG
     assert lib.wkv6_bwd(2, 8, 128, 4, 1, *p, FAKE, ws, None) == WKV_ERR_HEADSIZE
     q = list(p)

@@ -166,10 +166,19 @@ def test_wkv6_fwd_slices_match_single_head_calls(f32_path):
 
 # ------------------------------------------------------------------ backward, small and ragged
 
-@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (1, 2, 1), (2, 15, 2), (1, 16, 1), (2, 17, 1), (1, 50, 3),
+@pytest.fixture(params=["tensor", "recurrence"])
+def bwd_path(request, monkeypatch):
+    """Run the fp32 backward through the chunked tensor-core kernels (split-bf16
+    operands) or the two-sweep recurrence kernel."""
+    monkeypatch.setenv("WKV6_BWD_PATH", request.param)
+    return request.param
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (1, 2, 1), (2, 15, 2), (1, 16, 1), (2, 17, 1), (1, 32, 1), (1, 33, 2),
+                                   (2, 65, 1), (1, 130, 2), (1, 50, 3),
                                    (2, 96, 2)])
 @pytest.mark.parametrize("bidir", [False, True])
-def test_wkv6_bwd_small(B, T, H, bidir):
+def test_wkv6_bwd_small(B, T, H, bidir, bwd_path):
     x = synth.make_wkv6(B, T, H, seed=100 + T, with_dy=True)
     got = gc.run_wkv6_bwd(x, bidir)
     r, k, v, w, u = gc.f64(x)
@@ -177,13 +186,20 @@ def test_wkv6_bwd_small(B, T, H, bidir):
     for name, g, e in zip(("dr", "dk", "dv", "dw", "du"), got, ref):
         assert np.all(np.isfinite(g)), name
         if name == "dw" and T <= 2:
-            assert np.max(np.abs(g)) <= 1e-6, name   # exactly zero in exact arithmetic
+            # exactly zero in exact arithmetic: the pair terms of r.dr and k.dk cancel.
+            # The recurrence computes both sides the same way (residue ~1e-7); the
+            # tensor-core kernels take them from two different chunk products with
+            # split-bf16 operands, so the residue is bounded by the gradient tolerance
+            # times the size of the cancelling terms.
+            scale = max(np.max(np.abs(r * ref[0])), np.max(np.abs(k * ref[1])))
+            bound = 1e-6 if bwd_path == "recurrence" else gc.TOL_F32_GRAD * scale
+            assert np.max(np.abs(g)) <= bound, (name, np.max(np.abs(g)), bound)
             continue
         assert _rel(g, e) <= gc.TOL_F32_GRAD, (name, _rel(g, e))
 
 
 @pytest.mark.parametrize("bidir", [False, True])
-def test_wkv6_bwd_strong_decay_and_determinism(bidir):
+def test_wkv6_bwd_strong_decay_and_determinism(bidir, bwd_path):
     x = synth.make_wkv6(2, 45, 2, seed=7, with_dy=True)
     w = -np.exp(np.random.default_rng(9).uniform(-2.0, 3.5, x.w.shape))
     w[:, 10, :] = -np.inf
@@ -258,7 +274,7 @@ def test_workload_causal_bf16_long_sampled(bf16_path):
     assert err <= _bf16_bound(bf16_path), err
 
 
-def test_workload_bidir_bwd_sampled():
+def test_workload_bidir_bwd_sampled(bwd_path):
     kind, x = synth.make_workload("wkv6_bidir_bwd_f32_b32t196h12")
     dr, dk, dv, dw, du = gc.run_wkv6_bwd(x, True)
     units = gc.sample_units(x.B, x.H, 24)
