@@ -59,7 +59,8 @@ ALG = {
     "wkv4_f32_b8t1024c768": dict(bytes_per_unit=3 * 4, flops_per_unit=16, bound="hbm"),
     "wkv6_bidir_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=10 * N * N, bound="hbm"),
     "wkv6_causal_bf16_b8t4096h32": dict(bytes_per_unit=4 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
-    "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="alu"),
+    # the fp32 backward's default path runs on the tensor cores (two-term split bf16 operands)
+    "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="hbm"),
     "wkv6_bidir_bwd_bf16_b32t196h12": dict(bytes_per_unit=5 * N * 2 + 4 * N * 4, flops_per_unit=28 * N * N,
                                            bound="alu"),
     # RWKV-4 backward: k, v, dy in and dk, dv out per (token, channel)
@@ -81,7 +82,7 @@ ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_
          "wkv4_bwd_f32_b8t1024c768": "wkv4_bwd", "wkv5_causal_bf16_b8t4096h32": "wkv5_fwd_bf16",
          "wkv5_bwd_f32_b32t196h12": "wkv5_bwd", "wkv6_bidir_fused_f32_b32t196h12": "wkv6_fwd_fused"}
 LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
-            "wkv6_bidir_bwd_f32_b32t196h12": 2,   # the backward adds a deterministic du reduction
+            "wkv6_bidir_bwd_f32_b32t196h12": 3,   # S-kind and G-kind tensor-core kernels and the deterministic du reduction
             "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 2,
             "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
             "wkv5_bwd_f32_b32t196h12": 4,   # decay expansion, backward, du and dw reductions
