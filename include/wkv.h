@@ -71,6 +71,10 @@ enum {
  *   r, k, v, w : [B,T,C] float, inputs (w = log-decay, see above)
  *   u          : [C] float, bonus for the current token
  *   y          : [B,T,C] float, output
+ * Algorithm: the chunked form ("RWKV Architecture ...", Parallel Training
+ * Formulation) on the tensor cores, every fp32 operand split exactly into three
+ * bf16 terms (relative L2 error about 2e-7); with the environment variable
+ * WKV6_F32_PATH=recurrence (read on every call), the token-by-token recurrence.
  */
 int wkv6_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v,
              const float *w, const float *u, float *y, wkv_stream_t stream);
@@ -144,6 +148,12 @@ int wkv6_decode(int B, int C, int H, const float *r, const float *k, const float
  *   workspace          : device scratch of at least wkv6_bwd_workspace_bytes(...)
  *                        bytes, 16-byte aligned, owned by the caller; its content
  *                        on entry is ignored and on exit undefined.
+ * Algorithm: the chunked form on the tensor cores in two kernels (one carrying
+ * the forward state, one the adjoint), operands split into two bf16 terms
+ * (relative L2 error about 1e-5 on every gradient); with the environment
+ * variable WKV6_BWD_PATH=recurrence (read on every call), the two-sweep
+ * recurrence.  Both write every output element; only the order of additions
+ * differs, and each is bitwise reproducible run to run.
  */
 int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, const float *k,
              const float *v, const float *w, const float *u, const float *dy, float *dr, float *dk,
@@ -175,7 +185,9 @@ size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional);
  * fragments a planned memory pool).  The source pages have no counterpart to
  * this entry point; it exists for those callers.
  *
- * Same operation, arguments (minus workspace), layouts and results as wkv6_bwd.
+ * Same operation, arguments (minus workspace) and layouts as wkv6_bwd, computed
+ * by the two-sweep recurrence kernel (the results agree with wkv6_bwd's within
+ * the fp32 gradient tolerance; wkv6_bwd runs the tensor-core kernels by default).
  * Its scratch is a fixed 1 MiB device array inside libwkv.so, which every GPU
  * that loads the library holds until the process exits; the call itself
  * allocates nothing.
@@ -245,7 +257,7 @@ int wkv5_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t 
  *   wkv5_fwd (dL/dw = -sum_{b,t} dL/d(ew_t)).
  * workspace: at least wkv5_bwd_workspace_bytes(B,T,C,H) bytes of device memory,
  * 16-byte aligned, caller-owned (the constant log-decay, its per-token gradient
- * and the per-batch du partials).  Errors as wkv6_bwd.
+ * and the RWKV-6 backward's scratch).  Errors as wkv6_bwd.
  */
 int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
              const float *u, const float *dy, float *dr, float *dk, float *dv, float *dw, float *du,

@@ -321,7 +321,7 @@ int wkv5_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t 
 size_t wkv5_bwd_workspace_bytes(int B, int T, int C, int H) {
     (void)H;
     if (B < 1 || T < 0 || C < 1) return 0;
-    return sizeof(float) * (2 * (size_t)B * T * C + (size_t)B * C);
+    return sizeof(float) * (2 * (size_t)B * T * C + 2 * (size_t)B * C);
 }
 
 int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
@@ -339,13 +339,13 @@ int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const f
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
     if ((st = check_device()) != WKV_OK) return st;
     // workspace: the constant log-decay [B][T][C], its per-token gradient [B][T][C],
-    // then the RWKV-6 backward's own [B][C]
+    // then the RWKV-6 backward's own 2 [B][C]
     float *ew = static_cast<float *>(workspace);
     float *dwtok = ew + (size_t)B * T * C;
     float *rest = dwtok + (size_t)B * T * C;
     if (wkv5_expand_launch(B, T, C, w, ew, s) != cudaSuccess) return WKV_ERR_CUDA;
     st = bwd_common(false, B, T, C, H, 0, r, k, v, ew, u, dy, dr, dk, dv, dwtok, du, rest,
-                    sizeof(float) * (size_t)B * C, stream);
+                    2 * sizeof(float) * (size_t)B * C, stream);
     if (st != WKV_OK) return st;
     return wkv5_dw_reduce_launch(B * T, C, dwtok, dw, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }

@@ -159,7 +159,7 @@ def test_wkv5_argument_errors(lib):
         assert f(0, 4, 64, 1, *p, None) == WKV_OK
     g = [FAKE + 256 * i for i in range(11)]                    # r, k, v, w, u, dy, dr, dk, dv, dw, du
     ws = wkv.wkv5_bwd_workspace_bytes(2, 8, 128, 2)
-    assert ws == 4 * (2 * 2 * 8 * 128 + 2 * 128)
+    assert ws == 4 * (2 * 2 * 8 * 128 + 2 * 2 * 128)
     f = lib.wkv5_bwd
     assert f(-1, 8, 128, 2, *g, FAKE, ws, None) == WKV_ERR_ARG
     assert f(2, 8, 128, 4, *g, FAKE, ws, None) == WKV_ERR_HEADSIZE

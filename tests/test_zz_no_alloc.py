@@ -4,9 +4,11 @@ Some callers cannot hand the library a workspace: code running inside another
 framework's plugin or callback that offers no scratch buffer, or a serving
 process that reserves its device memory at start-up and may not call cudaMalloc
 later.  wkv6_bwd_noalloc keeps its scratch in a fixed array inside libwkv.so
-instead.  These tests check, through the C ABI, that it returns exactly what
-the workspace-taking wkv6_bwd returns, call after call (the shared array keeps
-the previous call's contents), and that it refuses sizes past its fixed limit.
+instead.  These tests check, through the C ABI, that it returns the gradients
+the workspace-taking wkv6_bwd returns (within the gradient tolerance: it runs
+the recurrence kernel, wkv6_bwd the tensor-core kernels by default), call after
+call (the shared array keeps the previous call's contents), and that it
+refuses sizes past its fixed limit.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test; it also passes alone in a fresh process.
