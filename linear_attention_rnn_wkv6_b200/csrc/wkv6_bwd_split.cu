@@ -134,7 +134,8 @@ struct SSmem {
     __nv_bfloat16 Sin[kBT][kBSt];    // S_in (row i, j contiguous), 128B-swizzled: K-major B of dY S_in^T
     float E[kBF];                    // e^{Lam_p} (fidx); after the epilogue: the chunk's z or x part
     float R[kBF];                    // raw r (fidx)
-    float vdy[kBL], ruk[kBL];
+    float BR[kBF];                   // causal pass: the bonus part of dr, u k (v.dy) (fidx)
+    float vdy[kBL];
     float dec[kHead], u[kHead];
     float dusum[4][kHead];
     uint32_t tmem_base;
@@ -242,37 +243,26 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__res
             // ================= transform =================
             float s0, s1, a0, a1;
             decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
-            // v.dy and sum r u k per token (bonus scalars), reduced over the 64 channels
-            {
-                float pv[8], pr[8];
-                const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
+            // v.dy per token (the bonus scalar of dr, dk and du), reduced over the 64 channels
+            if (causal) {
+                float pv[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    pv[e] = fmaf(xv_[e].x, xd_[e].x, xv_[e].y * xd_[e].y);
-                    pr[e] = fmaf(xr_[e].x * u0, xk_[e].x, xr_[e].y * u1 * xk_[e].y);
-                }
-                const float vv = transpose_reduce8(pv, lane), rr = transpose_reduce8(pr, lane);
-                if ((lane & 3) == 0) {
-                    sm.vdy[pq + (lane >> 2)] = vv;
-                    sm.ruk[pq + (lane >> 2)] = rr;
-                }
+                for (int e = 0; e < 8; ++e) pv[e] = fmaf(xv_[e].x, xd_[e].x, xv_[e].y * xd_[e].y);
+                const float vv = transpose_reduce8(pv, lane);
+                if ((lane & 3) == 0) sm.vdy[pq + (lane >> 2)] = vv;
             }
             __syncthreads();
             float L0, L1, tot0, tot1;
             const bool exact = decay_prefix(ds, warp, ch, L0, L1, tot0, tot1);
             if (causal) {
-                // bonus parts: dr = u k (v.dy) is the base the epilogue adds to; dk, dv
-                // get theirs here (the G kind adds onto them); du partial sums
+                // the bonus part of dr (added by the epilogue, whose store is then plain) and
+                // the du partial sums; dk's and dv's bonus parts are the G kind's
                 const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int p = pq + e;
-                    if (c * kBL + p >= T) continue;
-                    const float vd = sm.vdy[p], ruk = sm.ruk[p];
-                    const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
-                    *reinterpret_cast<float2 *>(prm.dr + o) = make_float2(u0 * xk_[e].x * vd, u1 * xk_[e].y * vd);
-                    *reinterpret_cast<float2 *>(prm.dk + o) = make_float2(u0 * xr_[e].x * vd, u1 * xr_[e].y * vd);
-                    *reinterpret_cast<float2 *>(prm.dv + o) = make_float2(ruk * xd_[e].x, ruk * xd_[e].y);
+                    const float vd = c * kBL + p < T ? sm.vdy[p] : 0.f;
+                    *reinterpret_cast<float2 *>(&sm.BR[fidx(p, ch)]) = make_float2(u0 * xk_[e].x * vd, u1 * xk_[e].y * vd);
                     du0 = fmaf(xr_[e].x * xk_[e].x, vd, du0);
                     du1 = fmaf(xr_[e].y * xk_[e].y, vd, du1);
                 }
@@ -392,9 +382,12 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__res
                         const bool valid = c * kBL + p < T;
                         float2 *dst = reinterpret_cast<float2 *>(
                             prm.dr + ((size_t)b * T + (valid ? time_of(dir, c, p) : 0)) * C + cbase + 2 * q4);
+                        // causal pass: dr = bonus + dr' (plain store); anti-causal: dr += dr'
                         float2 prev[8];
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) prev[m] = valid ? dst[4 * m] : make_float2(0.f, 0.f);
+                        for (int m = 0; m < 8; ++m)
+                            prev[m] = causal ? *reinterpret_cast<const float2 *>(&sm.BR[fidx(p, 8 * m + 2 * q4)])
+                                             : (valid ? dst[4 * m] : make_float2(0.f, 0.f));
 #pragma unroll
                         for (int m = 0; m < 8; ++m) {
                             const int i = 8 * m + 2 * q4;
@@ -460,7 +453,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__res
                     tmem_wait_st();
                     if (rl) {
                         const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + i;
-                        prm.dr[o] += acc;
+                        prm.dr[o] = acc + (causal ? sm.BR[fidx(p, i)] : prm.dr[o]);
                         sm.E[fidx(p, i)] = sm.R[fidx(p, i)] * acc;
                     }
                 }
@@ -541,7 +534,8 @@ struct GSmem {
     __nv_bfloat16 dAp[kBT][kBAp];    // dA'^T likewise: K-major A of dA'^T Q
     __nv_bfloat16 Gt[kBT][kBSt];     // Gt (row i, j contiguous), 128B-swizzled: K-major B of V Gt^T, MN-major B of Kt Gt
     float F[kBF];                    // e^{-Lam_{s+1}} (fidx); after the first epilogue: the chunk's z or x part
-    float Kr[kBF];                   // raw k (fidx)
+    float BK[kBF];                   // first pass: the bonus part of dk, u r (v.dy) (fidx)
+    float vdy[kBL], cb[kBL];         // v.dy and the bonus scalar sum r u k per token
     float dec[kHead];
     uint32_t tmem_base;
     alignas(8) uint64_t bar_m1, bar_k, bar_v, bar_g, bar_fin;
@@ -550,7 +544,7 @@ static_assert(sizeof(GSmem) + 1024 <= 74 * 1024, "three CTAs per SM must fit");
 static_assert(offsetof(GSmem, Q) % 1024 == 0 && offsetof(GSmem, Kt) % 1024 == 0 && offsetof(GSmem, V) % 1024 == 0 &&
                   offsetof(GSmem, dY) % 1024 == 0 && offsetof(GSmem, Gt) % 1024 == 0,
               "swizzled tiles start on 1024-byte boundaries");
-struct GExact {   // exact chunks: raw r, v, ew, dy in the Q, Kt, V, dY tiles (Kr keeps k)
+struct GExact {   // exact chunks: raw r, v, ew, dy in the Q, Kt, V, dY tiles (F holds raw k)
     float r[kBL][kHead], v[kBL][kHead], ew[kBL][kHead], dy[kBL][kHead];
 };
 static_assert(sizeof(GExact) <= offsetof(GSmem, Ap) - offsetof(GSmem, Q), "exact-chunk inputs fit");
@@ -654,11 +648,33 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
             // ================= transform =================
             float s0, s1, a0, a1;
             decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
+            {   // v.dy and sum r u k per token, reduced over the 64 channels
+                const float u0 = prm.u[cbase + ch], u1 = prm.u[cbase + ch + 1];
+                float pv[8], pr[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    pv[e] = fmaf(xv_[e].x, xd_[e].x, xv_[e].y * xd_[e].y);
+                    pr[e] = fmaf(xr_[e].x * u0, xk_[e].x, xr_[e].y * u1 * xk_[e].y);
+                }
+                const float vv = transpose_reduce8(pv, lane), rr = transpose_reduce8(pr, lane);
+                if ((lane & 3) == 0) {
+                    sm.vdy[pq + (lane >> 2)] = vv;
+                    sm.cb[pq + (lane >> 2)] = rr;
+                }
+            }
             __syncthreads();
             float L0, L1, tot0, tot1;
             const bool exact = decay_prefix(ds, warp, ch, L0, L1, tot0, tot1);
+            if (pass == 0) {
+                // the bonus part of dk, added by the first pass's plain store
+                const float u0 = prm.u[cbase + ch], u1 = prm.u[cbase + ch + 1];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) *reinterpret_cast<float2 *>(&sm.Kr[fidx(pq + e, ch)]) = xk_[e];
+                for (int e = 0; e < 8; ++e) {
+                    const float vd = sm.vdy[pq + e];
+                    *reinterpret_cast<float2 *>(&sm.BK[fidx(pq + e, ch)]) =
+                        make_float2(u0 * xr_[e].x * vd, u1 * xr_[e].y * vd);
+                }
+            }
             if (!exact) {
                 if (warp == 0) *reinterpret_cast<float2 *>(&sm.dec[ch]) = make_float2(exp2f(tot0), exp2f(tot1));
 #pragma unroll
@@ -677,6 +693,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int p = pq + e;
+                    *reinterpret_cast<float2 *>(&sm.F[fidx(p, ch)]) = xk_[e];
                     *reinterpret_cast<float2 *>(&xe.r[p][ch]) = xr_[e];
                     *reinterpret_cast<float2 *>(&xe.v[p][ch]) = xv_[e];
                     *reinterpret_cast<float2 *>(&xe.ew[p][ch]) = xw_[e];
@@ -756,9 +773,12 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
                         for (int m = 0; m < 4; ++m) {
                             const int t0_ = 8 * m + 2 * q4;
                             const bool k0 = t0_ > s_, k1 = t0_ + 1 > s_;
+                            // causal pass: the diagonal carries dv's bonus part (sum r u k) dy
+                            const float dg = dir > 0 ? sm.cb[s_] : 0.f;
                             uint32_t x0, x1;
                             const uint32_t o = (uint32_t)(m * 512 + s_ * 16 + 4 * q4);
-                            split2_pair(k0 ? a[4 * m + 2 * hr] : 0.f, k1 ? a[4 * m + 2 * hr + 1] : 0.f, x0, x1);
+                            split2_pair(k0 ? a[4 * m + 2 * hr] : (t0_ == s_ ? dg : 0.f),
+                                        k1 ? a[4 * m + 2 * hr + 1] : (t0_ + 1 == s_ ? dg : 0.f), x0, x1);
                             st_u32(sm.Ap[0], o, x0);
                             st_u32(sm.Ap[1], o, x1);
                             split2_pair(k0 ? a[16 + 4 * m + 2 * hr] : 0.f, k1 ? a[16 + 4 * m + 2 * hr + 1] : 0.f, x0, x1);
@@ -793,7 +813,8 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
                 ok = __syncthreads_and(ok);
                 if (!ok) break;
                 fence_after_sync();
-                // ===== epilogue 1: dk' = e^{-Lam_{s+1}} dKt added to dk; its dw part into F =====
+                // ===== epilogue 1: dk' = e^{-Lam_{s+1}} dKt into dk (first pass: bonus + dk',
+                // a plain store; second: added); its dw part k dk' = Kt dKt into F =====
                 if (warp < 2) {
                     float kv[32];
                     tmem_ld_16x256b_x8(tA + lane_off, kv);
@@ -806,15 +827,19 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
                             prm.dk + ((size_t)b * T + (valid ? time_of(dir, c, s_) : 0)) * C + cbase + 2 * q4);
                         float2 prev[8];
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) prev[m] = valid ? dst[4 * m] : make_float2(0.f, 0.f);
+                        for (int m = 0; m < 8; ++m)
+                            prev[m] = pass == 0 ? *reinterpret_cast<const float2 *>(&sm.BK[fidx(s_, 8 * m + 2 * q4)])
+                                                : (valid ? dst[4 * m] : make_float2(0.f, 0.f));
 #pragma unroll
                         for (int m = 0; m < 8; ++m) {
                             const int i = 8 * m + 2 * q4;
                             const float2 f2 = *reinterpret_cast<const float2 *>(&sm.F[fidx(s_, i)]);
-                            const float2 k2 = *reinterpret_cast<const float2 *>(&sm.Kr[fidx(s_, i)]);
-                            const float d0 = f2.x * kv[4 * m + 2 * hr], d1 = f2.y * kv[4 * m + 2 * hr + 1];
+                            const uint32_t kt0 = ld_u32(sm.Kt[0], swz(s_, i)), kt1 = ld_u32(sm.Kt[1], swz(s_, i));
+                            const float g0 = kv[4 * m + 2 * hr], g1 = kv[4 * m + 2 * hr + 1];
+                            const float d0 = f2.x * g0, d1 = f2.y * g1;
                             if (valid) dst[4 * m] = make_float2(prev[m].x + d0, prev[m].y + d1);
-                            *reinterpret_cast<float2 *>(&sm.F[fidx(s_, i)]) = make_float2(k2.x * d0, k2.y * d1);
+                            *reinterpret_cast<float2 *>(&sm.F[fidx(s_, i)]) =
+                                make_float2((bf_lo(kt0) + bf_lo(kt1)) * g0, (bf_hi(kt0) + bf_hi(kt1)) * g1);
                         }
                     }
                 }
@@ -856,9 +881,10 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
                         if (c * kBL + s_ >= T) continue;
                         float2 *dst = reinterpret_cast<float2 *>(prm.dv + ((size_t)b * T + time_of(dir, c, s_)) * C +
                                                                  cbase + 2 * q4);
+                        // first pass: a plain store; second: added
                         float2 prev[8];
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) prev[m] = dst[4 * m];
+                        for (int m = 0; m < 8; ++m) prev[m] = pass == 0 ? make_float2(0.f, 0.f) : dst[4 * m];
 #pragma unroll
                         for (int m = 0; m < 8; ++m)
                             dst[4 * m] = make_float2(prev[m].x + vv[4 * m + 2 * hr], prev[m].y + vv[4 * m + 2 * hr + 1]);
@@ -872,7 +898,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
                 for (int p = kBL - 1; p >= 0; --p) {
                     if (c * kBL + p >= T) continue;   // uniform
                     const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase;
-                    const float kk = rl ? sm.Kr[fidx(p, i)] : 0.f;
+                    const float kk = rl ? sm.F[fidx(p, i)] : 0.f;   // raw k
                     float acc = 0.f;
 #pragma unroll 1
                     for (int qc = 0; qc < 4; ++qc) {
@@ -889,14 +915,15 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
                         }
                     }
                     if (rl) {
-                        prm.dk[o + i] += acc;
+                        prm.dk[o + i] = acc + (pass == 0 ? sm.BK[fidx(p, i)] : prm.dk[o + i]);
                         sm.F[fidx(p, i)] = kk * acc;
                     }
                     __syncthreads();
                     if (tid < kHead) {
-                        float s = 0.f;
+                        // the causal pass adds dv's bonus part (sum r u k) dy
+                        float s = dir > 0 ? sm.cb[p] * xe.dy[p][tid] : 0.f;
                         for (int ii = 0; ii < kHead; ++ii) s += part[pidx(ii, tid)];
-                        prm.dv[o + tid] += s;
+                        prm.dv[o + tid] = s + (pass == 0 ? 0.f : prm.dv[o + tid]);
                     }
                     const float dd = rl ? __expf(xe.ew[p][i]) : 0.f, rr = rl ? xe.r[p][i] : 0.f;
 #pragma unroll 1

@@ -105,6 +105,14 @@ bool bwd_use_tensor_cores() {
     return !(e && std::strcmp(e, "recurrence") == 0);
 }
 
+// Scratch of the tensor-core backward: per-batch du partials [B][C] and the S kind's
+// per-channel z totals [B][C].
+size_t bwd_tensor_workspace_floats(int B, int T, int C, bool bidir) {
+    (void)T;
+    (void)bidir;
+    return 2 * (size_t)B * C;
+}
+
 // Shared by wkv6_bwd and wkv6_bwd_bf16 (inputs fp32 or bf16, gradients fp32).
 int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const void *r, const void *k,
                const void *v, const void *w, const float *u, const void *dy, float *dr, float *dk, float *dv,
@@ -117,7 +125,8 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
         return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
     }
     const bool tensor = !bf16 && bwd_use_tensor_cores();
-    const size_t need = (tensor ? 2 : 1) * (size_t)B * (size_t)C * sizeof(float);
+    const size_t need = tensor ? bwd_tensor_workspace_floats(B, T, C, bidirectional != 0) * sizeof(float)
+                               : (size_t)B * (size_t)C * sizeof(float);
     if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
     if ((st = check_device()) != WKV_OK) return st;
@@ -275,12 +284,10 @@ int wkv6_decode(int B, int C, int H, const float *r, const float *k, const float
 }
 
 size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional) {
-    (void)T;
     (void)H;
-    (void)bidirectional;
-    if (B < 1 || C < 1) return 0;
-    // per-batch du partials, and per-channel z totals for the tensor-core kernels
-    return 2 * (size_t)B * (size_t)C * sizeof(float);
+    if (B < 1 || C < 1 || T < 0) return 0;
+    // the tensor-core kernels' scratch (the recurrence needs only the first B*C floats)
+    return bwd_tensor_workspace_floats(B, T, C, bidirectional != 0) * sizeof(float);
 }
 
 int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, const float *k, const float *v,
