@@ -81,8 +81,73 @@ __device__ __forceinline__ int fidx(int p, int i) { return p * kHead + ((((i >> 
 
 __device__ __forceinline__ uint64_t bdadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Ask L2 for the chunk's rows of `out` (32 tokens x this head's 256 bytes, two
+// 128-byte lines each) that a later phase of the chunk reads back and adds to;
+// threads 64 .. 127 issue one line each.
+__device__ __forceinline__ void prefetch_rows(const float *out, int b, int T, int C, int cbase, int c,
+                                              int tid, int dir) {
+    if (tid < 64) return;
+    const int p = (tid - 64) >> 1;
+    if (c * kBL + p >= T) return;
+    const int t = dir > 0 ? c * kBL + p : T - 1 - (c * kBL + p);
+    prefetch_l2(out + ((size_t)b * T + t) * C + cbase + 32 * (tid & 1));
+}
+
 // no-swizzle K-major descriptor of a 32-row chunk matrix (units of 8 columns, 512 B apart)
 __device__ __forceinline__ uint64_t desc_cm(const __nv_bfloat16 *tile) { return smem_desc(tile, 512, 128); }
+
+// One chunk of a dw scan, on all 128 threads: channel tid % 64, half tid / 64 of the
+// chunk (`order` 0: positions 0..15 come first in scan order, 1: 16..31 first).
+// part(p, i) is the token's z or x value; each thread adds its running sum (the
+// carry `run` from earlier chunks, the earlier half's total, its own prefix) times
+// `sign` to `base(p, i)` (`base_load`: the value in dw, else 0) and stores dw; `run`
+// ends as the carry after the chunk in every thread.  `xch` is 2 x 64 floats of
+// shared memory.  Loads of a thread's 16 tokens are issued before its stores.
+template <typename PartF, typename AddrF>
+__device__ __forceinline__ void dw_scan_chunk(int tid, int c, int T, int order, bool base_load, float sign,
+                                              float extra, float &run, float *xch, float *dw, PartF part,
+                                              AddrF addr) {
+    const int i = tid & (kHead - 1), h = tid >> 6;
+    const int p0 = 16 * h;
+    const bool first_half = (order == 0) == (h == 0);   // this half comes first in scan order
+    float prev[16], loc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const int p = p0 + e;
+        prev[e] = (base_load && c * kBL + p < T) ? dw[addr(p)] : 0.f;
+    }
+    float acc = 0.f;
+    if (order == 0) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int p = p0 + e;
+            acc += c * kBL + p < T ? part(p, i) : 0.f;
+            loc[e] = acc;
+        }
+    } else {
+#pragma unroll
+        for (int e = 15; e >= 0; --e) {
+            const int p = p0 + e;
+            acc += c * kBL + p < T ? part(p, i) : 0.f;
+            loc[e] = acc;
+        }
+    }
+    xch[h * kHead + i] = acc;
+    __syncthreads();
+    const float other = xch[(1 - h) * kHead + i];
+    const float carry = run + (first_half ? 0.f : other);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const int p = p0 + e;
+        if (c * kBL + p < T) dw[addr(p)] = prev[e] + extra + sign * (carry + loc[e]);
+    }
+    run += acc + other;
+    __syncthreads();   // xch is free again
+}
 
 struct BDecay {
     float psum[4][kHead];
@@ -138,6 +203,7 @@ struct SSmem {
     float vdy[kBL];
     float dec[kHead], u[kHead];
     float dusum[4][kHead];
+    float xch[2 * kHead];
     uint32_t tmem_base;
     alignas(8) uint64_t bar_m1, bar_p, bar_s, bar_fin;
 };
@@ -224,7 +290,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__res
     uint32_t ph = 0;
     bool ok = true;
     float du0 = 0.f, du1 = 0.f;      // sum over the causal pass of r k (v.dy), channels ch, ch + 1
-    float zrun = 0.f;                // thread i < 64: running prefix (causal) or suffix (anti) of the dw part
+    float zrun = 0.f;                // channel tid % 64: running prefix (causal) or suffix (anti) of the dw part
     constexpr int npass = BIDIR ? 2 : 1;
     load_chunk(1, 0);
 
@@ -240,6 +306,10 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__res
             tmem_wait_st();
         }
         for (int c = 0; c < nch; ++c) {
+            if (!causal) {   // this pass adds to dr and dw: start their reads from HBM now
+                prefetch_rows(prm.dr, b, T, C, cbase, c, tid, dir);
+                prefetch_rows(prm.dw, b, T, C, cbase, c, tid, dir);
+            }
             // ================= transform =================
             float s0, s1, a0, a1;
             decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
@@ -477,29 +547,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__res
             }
             // ===== dw part: causal pass dw = -(running prefix of z); anti-causal dw -= running suffix of x =====
             __syncthreads();
-            if (tid < kHead) {
-                // the previous dw values of the chunk are loaded before any store (one L2
-                // round trip per chunk instead of one per token), 16 tokens at a time
-                const int i = tid;
-#pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    float prev[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int p = 16 * hb + e;
-                        prev[e] = (!causal && c * kBL + p < T)
-                                      ? prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i]
-                                      : 0.f;
-                    }
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int p = 16 * hb + e;
-                        if (c * kBL + p >= T) break;
-                        zrun += sm.E[fidx(p, i)];
-                        prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i] = prev[e] - zrun;
-                    }
-                }
-            }
+            dw_scan_chunk(tid, c, T, 0, !causal, -1.f, 0.f, zrun, sm.xch, prm.dw,
+                          [&](int p, int i) { return sm.E[fidx(p, i)]; },
+                          [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
             fence_proxy_async_smem();
             fence_before_sync();
             __syncthreads();
@@ -627,8 +677,8 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
 
     uint32_t ph = 0;
     bool ok = true;
-    float zrun = 0.f;     // thread i < 64: running prefix of z (anti-causal pass), then suffix of x (causal)
-    float zg_tot = 0.f;   // thread i < 64: z total of the anti-causal pass
+    float zrun = 0.f;     // channel tid % 64: running prefix of z (anti-causal pass), then suffix of x (causal)
+    float zg_tot = 0.f;   // channel tid % 64: z total of the anti-causal pass
     constexpr int npass = BIDIR ? 2 : 1;
     load_chunk(BIDIR ? -1 : 1, nch - 1);
 
@@ -645,6 +695,12 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
         }
         for (int c = nch - 1; c >= 0; --c) {
             const bool first = c == nch - 1;   // no adjoint from later chunks yet
+            // rows this chunk reads back and adds to: start their reads from HBM now
+            prefetch_rows(prm.dw, b, T, C, cbase, c, tid, dir);
+            if (pass > 0) {
+                prefetch_rows(prm.dk, b, T, C, cbase, c, tid, dir);
+                prefetch_rows(prm.dv, b, T, C, cbase, c, tid, dir);
+            }
             // ================= transform =================
             float s0, s1, a0, a1;
             decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
@@ -942,27 +998,12 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
             // ===== dw part: anti-causal pass dw -= running prefix of z (forward in time);
             // causal pass dw += z totals - running suffix of x (backward in time) =====
             __syncthreads();
-            if (tid < kHead) {
-                // previous dw values loaded before any store, 16 tokens at a time
-                const int i = tid;
-                const float ztot_all = last ? ztot[(size_t)b * C + cbase + i] + zg_tot : 0.f;
-#pragma unroll
-                for (int hb = 1; hb >= 0; --hb) {
-                    float prev[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int p = 16 * hb + e;
-                        prev[e] = c * kBL + p < T ? prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i] : 0.f;
-                    }
-#pragma unroll
-                    for (int e = 15; e >= 0; --e) {
-                        const int p = 16 * hb + e;
-                        if (c * kBL + p >= T) continue;
-                        zrun += sm.F[fidx(p, i)];
-                        prm.dw[((size_t)b * T + time_of(dir, c, p)) * C + cbase + i] =
-                            prev[e] + (last ? ztot_all - zrun : -zrun);
-                    }
-                }
+            {
+                const float ztot_all = last ? ztot[(size_t)b * C + cbase + (tid & (kHead - 1))] + zg_tot : 0.f;
+                // the dA'^T tiles are free once dKt has read them: the scan's exchange buffer
+                dw_scan_chunk(tid, c, T, 1, true, -1.f, ztot_all, zrun, reinterpret_cast<float *>(&sm.dAp[0][0]), prm.dw,
+                              [&](int p, int i) { return sm.F[fidx(p, i)]; },
+                              [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
             }
             fence_proxy_async_smem();
             fence_before_sync();
