@@ -62,7 +62,7 @@ ALG = {
     # the fp32 backward's default path runs on the tensor cores (two-term split bf16 operands)
     "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="hbm"),
     "wkv6_bidir_bwd_bf16_b32t196h12": dict(bytes_per_unit=5 * N * 2 + 4 * N * 4, flops_per_unit=28 * N * N,
-                                           bound="alu"),
+                                           bound="hbm"),
     # RWKV-4 backward: k, v, dy in and dk, dv out per (token, channel)
     "wkv4_bwd_f32_b8t1024c768": dict(bytes_per_unit=5 * 4, flops_per_unit=40, bound="hbm"),
     # decode: the state is read and written once per step (2 N^2 floats) next to 5 N floats of token data
@@ -83,7 +83,7 @@ ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_
          "wkv5_bwd_f32_b32t196h12": "wkv5_bwd", "wkv6_bidir_fused_f32_b32t196h12": "wkv6_fwd_fused"}
 LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
             "wkv6_bidir_bwd_f32_b32t196h12": 3,   # S-kind and G-kind tensor-core kernels and the deterministic du reduction
-            "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 2,
+            "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 3,
             "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
             "wkv5_bwd_f32_b32t196h12": 4,   # decay expansion, backward, du and dw reductions
             "wkv6_bidir_fused_f32_b32t196h12": 1}

@@ -164,7 +164,8 @@ int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, cons
  * wkv6_bwd_bf16 -- wkv6_bwd with bfloat16 r, k, v, w and dy (raw IEEE bf16 bit
  * patterns, uint16_t) for bf16 training: the same gradients, computed in fp32
  * from the bf16 values, with u and every gradient (dr, dk, dv, dw, du) in fp32.
- * Same layouts, workspace (wkv6_bwd_workspace_bytes) and errors as wkv6_bwd.
+ * Same layouts, workspace (wkv6_bwd_workspace_bytes), algorithms (and
+ * WKV6_BWD_PATH switch) and errors as wkv6_bwd.
  */
 int wkv6_bwd_bf16(int B, int T, int C, int H, int bidirectional, const uint16_t *r, const uint16_t *k,
                   const uint16_t *v, const uint16_t *w, const float *u, const uint16_t *dy, float *dr,

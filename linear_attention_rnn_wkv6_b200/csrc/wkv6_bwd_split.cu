@@ -30,7 +30,8 @@
 //
 // Precision: the gradient tolerance (1e-4 relative L2) allows two bf16 terms per
 // operand (x0 = bf16(x), x1 = bf16(x - x0), 16 significant bits) and three MMAs
-// per product (a0b0 + a0b1 + a1b0).
+// per product (a0b0 + a0b1 + a1b0).  Inputs are fp32 or bf16 (widened exactly on
+// load); the arithmetic is the same.
 //
 // Launches: the S kind (dr, du partials, the bonus parts of dk and dv, its dw share
 // and the z total per channel), then the G kind (dk, dv added, the rest of dw).
@@ -80,6 +81,14 @@ __device__ __forceinline__ void put_pair2(__nv_bfloat16 (*tiles)[kBTok], int row
 __device__ __forceinline__ int fidx(int p, int i) { return p * kHead + ((((i >> 1) ^ ((p & 7) << 2))) << 1) + (i & 1); }
 
 __device__ __forceinline__ uint64_t bdadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// Two consecutive inputs (channels ch, ch + 1) as fp32: one 8-byte load for fp32
+// inputs, one 4-byte load of a bf16 pair (exact widening) for bf16 inputs.
+__device__ __forceinline__ float2 ld_pair(const float *p) { return __ldg(reinterpret_cast<const float2 *>(p)); }
+__device__ __forceinline__ float2 ld_pair(const __nv_bfloat16 *p) {
+    const uint32_t x = __ldg(reinterpret_cast<const unsigned int *>(p));
+    return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
+}
 
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -221,12 +230,12 @@ static_assert(sizeof(float) * kBL * kHead <= sizeof(__nv_bfloat16) * kBSt, "exac
 
 // One pass per direction: causal first (forward in time), then, bidirectional,
 // the anti-causal pass (backward in time).
-template <bool BIDIR>
-__global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__restrict__ r,
-                                                              const float *__restrict__ k,
-                                                              const float *__restrict__ v,
-                                                              const float *__restrict__ w,
-                                                              const float *__restrict__ dy, BwdParams prm,
+template <typename Tin, bool BIDIR>
+__global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restrict__ r,
+                                                              const Tin *__restrict__ k,
+                                                              const Tin *__restrict__ v,
+                                                              const Tin *__restrict__ w,
+                                                              const Tin *__restrict__ dy, BwdParams prm,
                                                               float *__restrict__ ztot) {
     extern __shared__ unsigned char smem_dyn[];
     SSmem &sm = *reinterpret_cast<SSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -276,11 +285,11 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const float *__res
             const int p = pq + e;
             if (c * kBL + p < T) {
                 const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
-                xr_[e] = __ldg(reinterpret_cast<const float2 *>(r + o));
-                xk_[e] = __ldg(reinterpret_cast<const float2 *>(k + o));
-                xv_[e] = __ldg(reinterpret_cast<const float2 *>(v + o));
-                xw_[e] = __ldg(reinterpret_cast<const float2 *>(w + o));
-                xd_[e] = __ldg(reinterpret_cast<const float2 *>(dy + o));
+                xr_[e] = ld_pair(r + o);
+                xk_[e] = ld_pair(k + o);
+                xv_[e] = ld_pair(v + o);
+                xw_[e] = ld_pair(w + o);
+                xd_[e] = ld_pair(dy + o);
             } else {
                 xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
             }
@@ -606,12 +615,12 @@ static_assert(sizeof(float) * kHead * kHead <= sizeof(__nv_bfloat16) * kBT * kBS
 // Passes: bidirectional, the anti-causal one first (its chunks in reverse processing
 // order run forward in time), then the causal one (backward in time); chunks of a
 // pass in reverse processing order, tokens of a chunk from the last to the first.
-template <bool BIDIR>
-__global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__restrict__ r,
-                                                              const float *__restrict__ k,
-                                                              const float *__restrict__ v,
-                                                              const float *__restrict__ w,
-                                                              const float *__restrict__ dy, BwdParams prm,
+template <typename Tin, bool BIDIR>
+__global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restrict__ r,
+                                                              const Tin *__restrict__ k,
+                                                              const Tin *__restrict__ v,
+                                                              const Tin *__restrict__ w,
+                                                              const Tin *__restrict__ dy, BwdParams prm,
                                                               const float *__restrict__ ztot) {
     extern __shared__ unsigned char smem_dyn[];
     GSmem &sm = *reinterpret_cast<GSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -664,11 +673,11 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
             const int p = pq + e;
             if (c * kBL + p < T) {
                 const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
-                xr_[e] = __ldg(reinterpret_cast<const float2 *>(r + o));
-                xk_[e] = __ldg(reinterpret_cast<const float2 *>(k + o));
-                xv_[e] = __ldg(reinterpret_cast<const float2 *>(v + o));
-                xw_[e] = __ldg(reinterpret_cast<const float2 *>(w + o));
-                xd_[e] = __ldg(reinterpret_cast<const float2 *>(dy + o));
+                xr_[e] = ld_pair(r + o);
+                xk_[e] = ld_pair(k + o);
+                xv_[e] = ld_pair(v + o);
+                xw_[e] = ld_pair(w + o);
+                xd_[e] = ld_pair(dy + o);
             } else {
                 xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
             }
@@ -1023,12 +1032,12 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const float *__res
     if (warp == 0) tmem_dealloc(sm.tmem_base, 128);
 }
 
-cudaError_t wkv6_bwd_split_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
-                                  const float *dy, const BwdParams &prm, float *ztot, float *du,
-                                  cudaStream_t stream) {
+template <typename Tin, bool BIDIR>
+static cudaError_t launch_split_bwd(const void *r, const void *k, const void *v, const void *w, const void *dy,
+                                   const BwdParams &prm, float *ztot, float *du, cudaStream_t stream) {
     const size_t smS = sizeof(SSmem) + 1024, smG = sizeof(GSmem) + 1024;
-    auto ks = bidir ? wkv6_bwd_s_kernel<true> : wkv6_bwd_s_kernel<false>;
-    auto kg = bidir ? wkv6_bwd_g_kernel<true> : wkv6_bwd_g_kernel<false>;
+    auto ks = wkv6_bwd_s_kernel<Tin, BIDIR>;
+    auto kg = wkv6_bwd_g_kernel<Tin, BIDIR>;
     cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smS);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smG);
     if (e == cudaSuccess)
@@ -1036,12 +1045,25 @@ cudaError_t wkv6_bwd_split_launch(bool bidir, const float *r, const float *k, co
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(kg, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
+    const Tin *r_ = static_cast<const Tin *>(r), *k_ = static_cast<const Tin *>(k), *v_ = static_cast<const Tin *>(v);
+    const Tin *w_ = static_cast<const Tin *>(w), *dy_ = static_cast<const Tin *>(dy);
     const unsigned grid = (unsigned)(prm.B * prm.H);
-    ks<<<grid, kBThr, smS, stream>>>(r, k, v, w, dy, prm, ztot);
+    ks<<<grid, kBThr, smS, stream>>>(r_, k_, v_, w_, dy_, prm, ztot);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    kg<<<grid, kBThr, smG, stream>>>(r, k, v, w, dy, prm, ztot);
+    kg<<<grid, kBThr, smG, stream>>>(r_, k_, v_, w_, dy_, prm, ztot);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return wkv6_du_reduce_launch(prm.B, prm.C, prm.du_part, du, stream);
+}
+
+cudaError_t wkv6_bwd_split_launch(bool bf16, bool bidir, const void *r, const void *k, const void *v, const void *w,
+                                  const void *dy, const BwdParams &prm, float *ztot, float *du,
+                                  cudaStream_t stream) {
+    using BF = __nv_bfloat16;
+    if (bf16)
+        return bidir ? launch_split_bwd<BF, true>(r, k, v, w, dy, prm, ztot, du, stream)
+                     : launch_split_bwd<BF, false>(r, k, v, w, dy, prm, ztot, du, stream);
+    return bidir ? launch_split_bwd<float, true>(r, k, v, w, dy, prm, ztot, du, stream)
+                 : launch_split_bwd<float, false>(r, k, v, w, dy, prm, ztot, du, stream);
 }
 
 }  // namespace wkv

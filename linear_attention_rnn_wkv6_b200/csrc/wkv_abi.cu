@@ -97,9 +97,9 @@ bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], bool bf16, int B, int T, int C
     return true;
 }
 
-// Algorithm of the fp32 backward: the chunked tensor-core kernels with split-bf16
-// operands (default) or the two-sweep recurrence (WKV6_BWD_PATH=recurrence).
-// The bf16 backward always runs the recurrence.  Read on every call.
+// Algorithm of the backward (fp32 or bf16 inputs): the chunked tensor-core kernels
+// with split-bf16 operands (default) or the two-sweep recurrence
+// (WKV6_BWD_PATH=recurrence).  Read on every call.
 bool bwd_use_tensor_cores() {
     const char *e = std::getenv("WKV6_BWD_PATH");
     return !(e && std::strcmp(e, "recurrence") == 0);
@@ -124,7 +124,7 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
         if ((st = check_device()) != WKV_OK) return st;
         return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
     }
-    const bool tensor = !bf16 && bwd_use_tensor_cores();
+    const bool tensor = bwd_use_tensor_cores();
     const size_t need = tensor ? bwd_tensor_workspace_floats(B, T, C, bidirectional != 0) * sizeof(float)
                                : (size_t)B * (size_t)C * sizeof(float);
     if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
@@ -133,9 +133,8 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
     if (tensor) {
         float *ws = static_cast<float *>(workspace);
         BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, ws};
-        return wkv6_bwd_split_launch(bidirectional != 0, static_cast<const float *>(r), static_cast<const float *>(k),
-                                     static_cast<const float *>(v), static_cast<const float *>(w),
-                                     static_cast<const float *>(dy), prm, ws + (size_t)B * C, du, s) == cudaSuccess
+        return wkv6_bwd_split_launch(bf16, bidirectional != 0, r, k, v, w, dy, prm, ws + (size_t)B * C, du, s) ==
+                       cudaSuccess
                    ? WKV_OK
                    : WKV_ERR_CUDA;
     }

@@ -56,10 +56,11 @@ cudaError_t wkv6_bwd_launch(bool bf16, bool bidir, const CUtensorMap *maps, cons
                             cudaStream_t stream);
 // du[c] = sum_b part[b][c] in increasing b.
 cudaError_t wkv6_du_reduce_launch(int B, int C, const float *part, float *du, cudaStream_t stream);
-// fp32 backward on the tensor cores (split-bf16 operands): an S-kind and a G-kind
-// launch and the du reduction; ztot is B*C floats of workspace (per-channel z totals).
-cudaError_t wkv6_bwd_split_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
-                                  const float *dy, const BwdParams &prm, float *ztot, float *du,
+// Backward on the tensor cores (split-bf16 operands; r, k, v, w, dy fp32 or, bf16,
+// bfloat16): an S-kind and a G-kind launch and the du reduction; ztot is B*C floats
+// of workspace (per-channel z totals).
+cudaError_t wkv6_bwd_split_launch(bool bf16, bool bidir, const void *r, const void *k, const void *v, const void *w,
+                                  const void *dy, const BwdParams &prm, float *ztot, float *du,
                                   cudaStream_t stream);
 // RWKV-4 backward; workspace: [B][T][C] + 2 [B][C] floats (see wkv4_bwd_workspace_bytes)
 // RWKV-5 backward helpers: ew[b][t][c] = -w[c]; dw[c] = -sum_rows dwtok[row][c].
