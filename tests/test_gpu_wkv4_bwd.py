@@ -43,7 +43,8 @@ def _compare(got, ref):
         assert err <= gc.TOL_F32_GRAD, (name, err)
 
 
-@pytest.mark.parametrize("B,T,C", [(1, 1, 16), (2, 7, 40), (1, 100, 64), (2, 333, 96), (1, 1024, 32)])
+@pytest.mark.parametrize("B,T,C", [(1, 1, 16), (2, 7, 40), (1, 100, 64), (2, 333, 96), (1, 1024, 32),
+                                   (2, 50, 30), (1, 65, 36), (3, 31, 20)])   # C not a multiple of 16 (or of 4)
 def test_wkv4_bwd_matches_oracle(B, T, C):
     x = synth.make_wkv4(B, T, C, seed=600 + T)
     dy = _dy(x, 601 + T)
