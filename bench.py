@@ -68,13 +68,14 @@ ALG = {
     # decode: the state is read and written once per step (2 N^2 floats) next to 5 N floats of token data
     "wkv6_decode_f32_b512h32": dict(bytes_per_unit=2 * N * N * 4 + 5 * N * 4, flops_per_unit=5 * N * N,
                                     bound="hbm"),
-    # RWKV-5: no per-token w; the forward (tensor-core chunked form, like the RWKV-6 bf16
-    # one, so bound by its bytes) reads bf16 r, k, v and writes fp32 y; the causal
-    # backward reads r, k, v, dy and writes dr, dk, dv (w, dw, u, du are per channel)
+    # RWKV-5: no per-token w; the forward and the causal backward run the tensor-core
+    # chunked forms, so both are bound by their bytes: the forward reads bf16 r, k, v and
+    # writes fp32 y; the backward reads r, k, v, dy and writes dr, dk, dv (w, dw, u, du
+    # are per channel)
     "wkv5_causal_bf16_b8t4096h32": dict(bytes_per_unit=3 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
-    "wkv5_bwd_f32_b32t196h12": dict(bytes_per_unit=7 * N * 4, flops_per_unit=14 * N * N, bound="alu"),
-    # fused forward: r, k, v, ww and the gate in, the normalised and gated output out
-    "wkv6_bidir_fused_f32_b32t196h12": dict(bytes_per_unit=6 * N * 4, flops_per_unit=10 * N * N, bound="alu"),
+    "wkv5_bwd_f32_b32t196h12": dict(bytes_per_unit=7 * N * 4, flops_per_unit=14 * N * N, bound="hbm"),
+    # fused forward (tensor-core kernel): r, k, v, ww and the gate in, the normalised and gated output out
+    "wkv6_bidir_fused_f32_b32t196h12": dict(bytes_per_unit=6 * N * 4, flops_per_unit=10 * N * N, bound="hbm"),
 }
 ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
          "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd",
@@ -85,7 +86,7 @@ LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_cau
             "wkv6_bidir_bwd_f32_b32t196h12": 3,   # S-kind and G-kind tensor-core kernels and the deterministic du reduction
             "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 3,
             "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
-            "wkv5_bwd_f32_b32t196h12": 4,   # decay expansion, backward, du and dw reductions
+            "wkv5_bwd_f32_b32t196h12": 5,   # decay expansion, S and G kinds, du and dw reductions
             "wkv6_bidir_fused_f32_b32t196h12": 1}
 
 

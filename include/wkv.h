@@ -225,8 +225,10 @@ int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, const float 
  *   where y is wkv6_fwd (or wkv6_bidir_fwd) at w = -exp(w_base + ww), and mu and
  *   var are the mean and the (biased) variance of y over the N channels of c's
  *   head at (b, t).  Neither the log-decay nor y is written to memory.
- * Same sizes, pointer rules and errors as wkv6_fwd; eps <= 0 or not finite gives
- * WKV_ERR_ARG.
+ * Same sizes, pointer rules, algorithm switch (WKV6_F32_PATH) and errors as
+ * wkv6_fwd; eps <= 0 or not finite gives WKV_ERR_ARG.  On the tensor-core path
+ * the prologue runs where the chunk is transformed and the norm and gate in the
+ * last sweep's epilogue.
  */
 int wkv6_fwd_fused(int B, int T, int C, int H, int bidirectional, const float *r, const float *k, const float *v,
                    const float *ww, const float *w_base, const float *u, const float *g, const float *gn_weight,

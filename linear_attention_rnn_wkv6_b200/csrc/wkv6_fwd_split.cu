@@ -30,6 +30,12 @@
 // decay exactly 0, NaN) is evaluated by the token-by-token recurrence on the CUDA
 // cores, from and back into the state in tensor memory.
 //
+// Fused form (wkv6_fwd_fused, "How the WKV ... Processes Images", the spatial-mix
+// block): the loaded w is ww and the log-decay is -exp(w_base + ww); the last sweep
+// replaces each finished y row of a head by (GroupNorm(y) * gn_w + gn_b) * g.  In
+// the tensor-core epilogue a row's 64 outputs are 16 values in each of 4 lanes of
+// one warp; in an exact chunk they are one value in each of threads 0..63.
+//
 // One CTA of 128 threads per (b, h), three CTAs per SM (70 KB of shared memory and
 // 128 TMEM columns each), so the phases of one CTA (transform, MMA, mask, MMA,
 // epilogue) overlap with those of the others.  Inputs are read with coalesced
@@ -68,6 +74,8 @@ struct SplitSmem {
     float dec[kHead];                   // exp(Lam_L) per channel
     float cp[kSL];                      // bonus scalars per token
     float u[kHead];
+    float gnw[kHead], gnb[kHead];       // fused epilogue: norm weight and bias of the head
+    float red[4];                       // fused epilogue of exact chunks: two-warp sums
     uint32_t tmem_base;
     alignas(8) uint64_t bar_m1;
     alignas(8) uint64_t bar_p;
@@ -145,9 +153,18 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity) {
     return mbar_wait_bounded(bar, parity);
 }
 
+// Barrier of warps 0 and 1 only (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void sync_warps01() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
 }  // namespace
 
-template <bool BIDIR>
+template <bool BIDIR, bool FUSED>
 __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__restrict__ r,
                                                                  const float *__restrict__ k,
                                                                  const float *__restrict__ v,
@@ -170,6 +187,11 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
 
     if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
+    if (FUSED && tid < kHead) {
+        sm.gnw[tid] = prm.gn_w[cbase + tid];
+        sm.gnb[tid] = prm.gn_b[cbase + tid];
+    }
+    const float2 wb = FUSED ? __ldg(reinterpret_cast<const float2 *>(prm.wb + cbase + ch)) : make_float2(0.f, 0.f);
     if (tid == 0) {
         mbar_init(&sm.bar_m1, 1);
         mbar_init(&sm.bar_p, 1);
@@ -224,6 +246,7 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
         const int dir = (BIDIR && di == 0) ? -1 : 1;   // bidirectional: anti-causal sweep first
         const bool bonus = dir > 0;
         const bool accumulate_y = BIDIR && di == 1;    // the causal sweep adds to y
+        const bool norm = FUSED && (!BIDIR || di == 1);  // the last sweep: norm/gate epilogue
         // S = 0 at the start of every sweep
         {
             float z[32];
@@ -235,6 +258,13 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
         }
         for (int c = 0; c < nch; ++c) {
             // ================= transform =================
+            if (FUSED) {
+                // decay prologue, here rather than at the load so that the load stays in flight
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (c * kSL + pq + e < T)
+                        xw_[e] = make_float2(-expf(wb.x + xw_[e].x), -expf(wb.y + xw_[e].y));
+            }
             float s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -379,6 +409,19 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                     }
                     mma_commit(&sm.bar_p);
                 }
+                // fused: the gate values of this chunk's rows are loaded while Y is computed
+                float2 gate[2][8];
+                if (norm && warp < 2) {
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int p = 16 * warp + (lane >> 2) + 8 * hr;
+                        const bool vd = c * kSL + p < T;
+                        const float2 *gs = reinterpret_cast<const float2 *>(
+                            prm.g + ((size_t)b * T + (vd ? time_of(dir, c, p) : 0)) * C + cbase + 2 * (lane & 3));
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) gate[hr][m] = vd ? __ldg(gs + 4 * m) : make_float2(0.f, 0.f);
+                    }
+                }
                 ok = wait_bar(&sm.bar_p, ph_p) && wait_bar(&sm.bar_s, ph_p);
                 ph_p ^= 1u;
                 ok = __syncthreads_and(ok);
@@ -405,14 +448,51 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                     float yv[32];
                     tmem_ld_16x256b_x8(tY + lane_off, yv);
                     tmem_wait_ld();
+                    if (norm) {
+                        // a row's 64 outputs: 16 here, the rest in the lanes differing in bits 0, 1
 #pragma unroll
-                    for (int hr = 0; hr < 2; ++hr)
-                        if (valid[hr]) {
+                        for (int hr = 0; hr < 2; ++hr) {
+                            float yr[16];
+                            float s1 = 0.f;
 #pragma unroll
-                            for (int m = 0; m < 8; ++m)
-                                dst[hr][4 * m] = make_float2(yv[4 * m + 2 * hr] + prev[hr][m].x,
-                                                             yv[4 * m + 2 * hr + 1] + prev[hr][m].y);
+                            for (int m = 0; m < 8; ++m) {
+                                yr[2 * m] = yv[4 * m + 2 * hr] + prev[hr][m].x;
+                                yr[2 * m + 1] = yv[4 * m + 2 * hr + 1] + prev[hr][m].y;
+                                s1 += yr[2 * m] + yr[2 * m + 1];
+                            }
+                            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+                            s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+                            const float mu = s1 * (1.f / kHead);
+                            float s2 = 0.f;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                yr[e] -= mu;
+                                s2 = fmaf(yr[e], yr[e], s2);
+                            }
+                            s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+                            s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+                            const float rstd = rsqrtf(s2 * (1.f / kHead) + prm.gn_eps);
+                            if (valid[hr]) {
+#pragma unroll
+                                for (int m = 0; m < 8; ++m) {
+                                    const int j = 8 * m + 2 * q4;
+                                    dst[hr][4 * m] =
+                                        make_float2(fmaf(yr[2 * m] * rstd, sm.gnw[j], sm.gnb[j]) * gate[hr][m].x,
+                                                    fmaf(yr[2 * m + 1] * rstd, sm.gnw[j + 1], sm.gnb[j + 1]) *
+                                                        gate[hr][m].y);
+                                }
+                            }
                         }
+                    } else {
+#pragma unroll
+                        for (int hr = 0; hr < 2; ++hr)
+                            if (valid[hr]) {
+#pragma unroll
+                                for (int m = 0; m < 8; ++m)
+                                    dst[hr][4 * m] = make_float2(yv[4 * m + 2 * hr] + prev[hr][m].x,
+                                                                 yv[4 * m + 2 * hr + 1] + prev[hr][m].y);
+                            }
+                    }
                 }
                 {
                     // S rows i scaled by exp(Lam_L[i]), back to TMEM, three-term copy into S_in
@@ -471,8 +551,24 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                         const int j = tid;
                         float acc = sm.cp[p] * xr.v[p][j];
                         for (int ii = 0; ii < kHead; ++ii) acc += part[ii * kPartStride + j];
-                        float *dst = prm.y + ((size_t)b * T + time_of(dir, c, p)) * C + cbase + j;
-                        *dst = accumulate_y ? *dst + acc : acc;
+                        const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + j;
+                        float *dst = prm.y + o;
+                        float yo = accumulate_y ? *dst + acc : acc;
+                        if (norm) {
+                            // the token's 64 outputs are one per thread of warps 0 and 1
+                            const float gt = __ldg(prm.g + o);
+                            float s1 = warp_sum(yo);
+                            if (lane == 0) sm.red[warp] = s1;
+                            sync_warps01();
+                            const float mu = (sm.red[0] + sm.red[1]) * (1.f / kHead);
+                            const float d = yo - mu;
+                            const float s2 = warp_sum(d * d);
+                            if (lane == 0) sm.red[2 + warp] = s2;
+                            sync_warps01();
+                            const float rstd = rsqrtf((sm.red[2] + sm.red[3]) * (1.f / kHead) + prm.gn_eps);
+                            yo = fmaf(d * rstd, sm.gnw[j], sm.gnb[j]) * gt;
+                        }
+                        *dst = yo;
                     }
                     if (row_lane) {
                         const float dd = __expf(xr.ew[p][i]), kk = xr.k[p][i];
@@ -524,7 +620,9 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
 cudaError_t wkv6_fwd_split_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
                                   const FwdParams &prm, cudaStream_t stream) {
     const size_t smem = sizeof(SplitSmem) + 1024;
-    auto kern = bidir ? wkv6_fwd_split_kernel<true> : wkv6_fwd_split_kernel<false>;
+    const bool fused = prm.gn_w != nullptr;
+    auto kern = bidir ? (fused ? wkv6_fwd_split_kernel<true, true> : wkv6_fwd_split_kernel<true, false>)
+                      : (fused ? wkv6_fwd_split_kernel<false, true> : wkv6_fwd_split_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);

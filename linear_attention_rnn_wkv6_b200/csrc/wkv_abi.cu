@@ -162,7 +162,7 @@ bool f32_use_tensor_cores() {
 
 // w5 (RWKV-5): static per-channel decay rate [C]; then w is ignored (pass w5 for
 // the argument checks) and the recurrence kernel runs with the constant log-decay.
-// fused (fp32 recurrence only): decay prologue and norm/gate epilogue of wkv6_fwd_fused.
+// fused: decay prologue and norm/gate epilogue of wkv6_fwd_fused (fp32 kernels).
 struct Fused {
     const float *wb, *g, *gn_w, *gn_b;
     float eps;
@@ -191,8 +191,15 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
                    ? WKV_OK
                    : WKV_ERR_CUDA;
     }
-    if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && fused == nullptr && f32_use_tensor_cores()) {
+    if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && f32_use_tensor_cores()) {
         FwdParams prm{B, T, C, H, u, y};
+        if (fused != nullptr) {
+            prm.wb = fused->wb;
+            prm.g = fused->g;
+            prm.gn_w = fused->gn_w;
+            prm.gn_b = fused->gn_b;
+            prm.gn_eps = fused->eps;
+        }
         return wkv6_fwd_split_launch(bidir, static_cast<const float *>(r), static_cast<const float *>(k),
                                      static_cast<const float *>(v), static_cast<const float *>(w), prm,
                                      reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess

@@ -16,7 +16,7 @@ struct FwdParams {
     // RWKV-5 static decay rate w5[C] >= 0 (log-decay -w5 at every token); when set
     // the w tensor map is not read
     const float *w5 = nullptr;
-    // fp32 recurrence kernel only.  Decay prologue: when wb (w_base [C]) is set, the
+    // fp32 kernels (recurrence and tensor-core).  Decay prologue: when wb (w_base [C]) is set, the
     // w map holds ww [B][T][C] and the log-decay is ew = -exp(wb + ww).  Norm/gate
     // epilogue: when gn_w is set, y receives (GroupNorm_head(y) * gn_w + gn_b) * g,
     // with g [B][T][C], gn_w and gn_b [C] and the variance offset gn_eps.

@@ -20,6 +20,14 @@ def _cuda():
     build.build()
 
 
+@pytest.fixture(params=["tensor", "recurrence"], autouse=True)
+def f32_path(request, monkeypatch):
+    """Both fp32 forward kernels: the chunked tensor-core one (split-bf16 operands; the norm
+    and gate in its epilogue) and the token-by-token recurrence."""
+    monkeypatch.setenv("WKV6_F32_PATH", request.param)
+    return request.param
+
+
 _NAMES = ("r", "k", "v", "ww", "w_base", "u", "g", "gn_w", "gn_b")
 
 
@@ -54,6 +62,17 @@ def test_fused_strong_decay_and_large_eps(bidir):
     and a variance offset comparable to the row variances."""
     x = synth.make_fused(2, 90, 2, seed=810, bidir=bidir, base_lo=-8.0, base_hi=2.0, ww_std=1.0, eps=0.05)
     assert oracle.rel_l2(_run(x), _ref(x)) <= gc.TOL_F32_FWD
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_fused_one_fast_forgetting_token(bidir):
+    """One token whose decay pre-activation is about 5 in a few channels (log-decay below -80):
+    the chunk holding it takes the exact token-by-token path, its neighbours the chunked one."""
+    x = synth.make_fused(2, 130, 2, seed=830, bidir=bidir)
+    x.ww[:, 40, 3:7] = 6.0
+    out = _run(x)
+    assert np.all(np.isfinite(out))
+    assert oracle.rel_l2(out, _ref(x)) <= gc.TOL_F32_FWD
 
 
 def test_fused_workload_sampled():
