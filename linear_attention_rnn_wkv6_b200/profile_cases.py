@@ -49,6 +49,12 @@ def make_case(spec: str):
         nb = wkv.wkv4_bwd_workspace_bytes(x.B, x.T, x.C)
         ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
         return label, lambda: wkv.wkv4_bwd(x.B, x.T, x.C, *ins, *outs, ws, nb)
+    if kind == "wkv6_fwd_fused":
+        x = synth.make_fused(kw["B"], kw["T"], kw["H"], seed=0, bidir=kw.get("bidir", False))
+        label = f"{name} B={x.B} T={x.T} H={x.H}"
+        ins = [_dev(getattr(x, n)) for n in ("r", "k", "v", "ww", "w_base", "u", "g", "gn_w", "gn_b")]
+        y = torch.empty(x.B, x.T, x.C, device="cuda")
+        return label, lambda: wkv.wkv6_fwd_fused(x.B, x.T, x.C, x.H, x.bidir, *ins, x.eps, y)
     args = {k: v for k, v in kw.items() if k not in ("B", "T", "H")}
     make = synth.make_wkv5 if kind.startswith("wkv5") else synth.make_wkv6
     x = make(kw["B"], kw["T"], kw["H"], seed=0, **args)
