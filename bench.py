@@ -330,14 +330,35 @@ class HostSide:
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
 
-    def run(self, stream):
+        self.comp_done = None   # the last call on d_in / d_out
+        self.out_done = None    # the last copy out of d_out
+
+    def run(self, s_in, s_comp, s_out):
+        """Copy this workload's inputs in (s_in), call it (s_comp), copy its outputs out
+        (s_out).  Events keep the order copy-in -> call -> copy-out, keep the next
+        copy-in behind the previous call (which reads d_in) and the next call behind
+        the previous copy-out (which reads d_out); the transfers of one workload then
+        overlap the calls and transfers of the others, in both directions of the link."""
         import torch
-        with torch.cuda.stream(stream):
+        if self.comp_done is not None:
+            s_in.wait_event(self.comp_done)
+        with torch.cuda.stream(s_in):
             for n, t in self.h_in.items():
                 self.d_in[n].copy_(t, non_blocking=True)
-            self.dw.run(stream, inputs=self.d_in, outputs=self.d_out)
+        in_done = torch.cuda.Event()
+        in_done.record(s_in)
+        s_comp.wait_event(in_done)
+        if self.out_done is not None:
+            s_comp.wait_event(self.out_done)
+        self.dw.run(s_comp, inputs=self.d_in, outputs=self.d_out)
+        self.comp_done = torch.cuda.Event()
+        self.comp_done.record(s_comp)
+        s_out.wait_event(self.comp_done)
+        with torch.cuda.stream(s_out):
             for h, d in zip(self.h_out, self.d_out):
                 h.copy_(d, non_blocking=True)
+        self.out_done = torch.cuda.Event()
+        self.out_done.record(s_out)
 
 
 def run_native(args, rank, world, local):
@@ -388,21 +409,33 @@ def run_native(args, rank, world, local):
     value = tokens_per_step * world * K / (elapsed_ms / 1e3)
 
     # end-to-end through the public API with host buffers (pinned), copies inside the timed region
+    # on three streams (copies in, calls, copies out): see HostSide.run
     hs = [HostSide(w) for w in wls] if not args.no_e2e else []
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     for _ in range(max(1, min(args.warmup, 2))):
         for h in hs:
-            h.run(stream)
+            h.run(s_in, stream, s_out)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     Ke = max(1, min(K, 5))
     barrier(dist)
     torch.cuda.synchronize()
     e0.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
     for _ in range(Ke):
         for h in hs:
-            h.run(stream)
+            h.run(s_in, stream, s_out)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
+    # the kernels are deterministic: what came back through the host must equal, bit for
+    # bit, what the device-timed calls on the same inputs left in their outputs
+    for h in hs:
+        for ho, do in zip(h.h_out, h.dw.outputs):
+            if not torch.equal(ho, do.cpu()):
+                raise RuntimeError(f"{h.dw.name}: end-to-end outputs differ from the device run's")
     barrier(dist)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     e2e_value = tokens_per_step * world * Ke / (e2e_ms / 1e3) if hs else None
@@ -451,7 +484,9 @@ def run_native(args, rank, world, local):
             "kernels": kernels,
             "e2e": {"value": round(e2e_value, 1) if e2e_value else None, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": Ke,
-                    "note": "public C-ABI calls; pinned host inputs copied in and outputs copied out every step"},
+                    "note": "public C-ABI calls; every step copies all inputs in from pinned host memory and all "
+                            "outputs out, on copy streams of their own, overlapped with the other workloads' "
+                            "calls and copies"},
             "gpu_launches": K * sum(LAUNCHES[w.name] for w in wls),
             "clocks": clocks,
         }
