@@ -23,23 +23,41 @@ __global__ void wkv5_expand_kernel(size_t n4, int C4, const float4 *__restrict__
     }
 }
 
-// dw[c] = -sum over rows (b, t) of dwtok[row][c], rows in increasing order.
-// A CTA of 32 x 8 threads covers 32 channels: each of the 8 row groups sums
-// every 8th row, then the 8 partials are added in a fixed order.
-__global__ void wkv5_dw_reduce_kernel(int rows, int C, const float *__restrict__ dwtok, float *__restrict__ dw) {
-    __shared__ float part[8][32];
+// dw[c] = -sum over rows (b, t) of dwtok[row][c], in two fixed-order stages so
+// that the result is deterministic and the rows are read by many CTAs at once.
+// Stage 1: a CTA of 32 x 8 threads takes 32 channels of one block of `blk` rows
+// (64, or more when the rows would need over 65535 blocks); row group y sums rows
+// y, y + 8, ... of the block, and the 8 group sums are added in order into
+// part[block][c].
+constexpr int kRowBlk = 64;
+__global__ void wkv5_dw_partial_kernel(int rows, int blk, int C, const float *__restrict__ dwtok,
+                                       float *__restrict__ part) {
+    __shared__ float grp[8][32];
     const int c = blockIdx.x * 32 + threadIdx.x;
+    const int r0 = blockIdx.y * blk, r1 = min(rows, r0 + blk);
     float acc = 0.f;
-    if (c < C)
-        for (int row = threadIdx.y; row < rows; row += 8) acc += dwtok[(size_t)row * C + c];
-    part[threadIdx.y][threadIdx.x] = acc;
+    if (c < C) {
+#pragma unroll 8
+        for (int row = r0 + threadIdx.y; row < r1; row += 8) acc += dwtok[(size_t)row * C + c];
+    }
+    grp[threadIdx.y][threadIdx.x] = acc;
     __syncthreads();
     if (threadIdx.y == 0 && c < C) {
         float s = 0.f;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) s += part[g][threadIdx.x];
-        dw[c] = -s;
+        for (int g = 0; g < 8; ++g) s += grp[g][threadIdx.x];
+        part[(size_t)blockIdx.y * C + c] = s;
     }
+}
+
+// Stage 2: dw[c] = -(sum of the blocks' partials in block order), one thread per channel.
+__global__ void wkv5_dw_final_kernel(int nblk, int C, const float *__restrict__ part, float *__restrict__ dw) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    float s = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < nblk; ++k) s += part[(size_t)k * C + c];
+    dw[c] = -s;
 }
 
 }  // namespace
@@ -52,8 +70,15 @@ cudaError_t wkv5_expand_launch(int B, int T, int C, const float *w, float *ew, c
     return cudaGetLastError();
 }
 
-cudaError_t wkv5_dw_reduce_launch(int rows, int C, const float *dwtok, float *dw, cudaStream_t stream) {
-    wkv5_dw_reduce_kernel<<<(unsigned)((C + 31) / 32), dim3(32, 8), 0, stream>>>(rows, C, dwtok, dw);
+cudaError_t wkv5_dw_reduce_launch(int rows, int C, const float *dwtok, float *part, float *dw,
+                                  cudaStream_t stream) {
+    const int blk = std::max(kRowBlk, (rows + 65534) / 65535);   // at most 65535 blocks (grid y)
+    const int nblk = (rows + blk - 1) / blk;
+    wkv5_dw_partial_kernel<<<dim3((unsigned)((C + 31) / 32), (unsigned)nblk), dim3(32, 8), 0, stream>>>(
+        rows, blk, C, dwtok, part);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    wkv5_dw_final_kernel<<<(unsigned)((C + 255) / 256), 256, 0, stream>>>(nblk, C, part, dw);
     return cudaGetLastError();
 }
 

@@ -360,7 +360,8 @@ int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const f
     st = bwd_common(false, B, T, C, H, 0, r, k, v, ew, u, dy, dr, dk, dv, dwtok, du, rest,
                     2 * sizeof(float) * (size_t)B * C, stream);
     if (st != WKV_OK) return st;
-    return wkv5_dw_reduce_launch(B * T, C, dwtok, dw, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    // the fold's per-block partials reuse the log-decay tensor, which the backward no longer reads
+    return wkv5_dw_reduce_launch(B * T, C, dwtok, ew, dw, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
 int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u, float *y,

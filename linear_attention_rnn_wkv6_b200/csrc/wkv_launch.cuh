@@ -65,7 +65,8 @@ cudaError_t wkv6_bwd_split_launch(bool bf16, bool bidir, const void *r, const vo
 // RWKV-4 backward; workspace: [B][T][C] + 2 [B][C] floats (see wkv4_bwd_workspace_bytes)
 // RWKV-5 backward helpers: ew[b][t][c] = -w[c]; dw[c] = -sum_rows dwtok[row][c].
 cudaError_t wkv5_expand_launch(int B, int T, int C, const float *w, float *ew, cudaStream_t stream);
-cudaError_t wkv5_dw_reduce_launch(int rows, int C, const float *dwtok, float *dw, cudaStream_t stream);
+// dw[c] = -sum over the rows of dwtok; `part` holds up to rows x C floats of scratch (ceil(rows / 64) x C in practice)
+cudaError_t wkv5_dw_reduce_launch(int rows, int C, const float *dwtok, float *part, float *dw, cudaStream_t stream);
 cudaError_t wkv4_bwd_launch(int B, int T, int C, const float *k, const float *v, const float *w, const float *u,
                             const float *dy, float *dk, float *dv, float *dw, float *du, float *workspace,
                             cudaStream_t stream);
