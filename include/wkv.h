@@ -318,6 +318,18 @@ int wkv_take_device_faults(unsigned *faults);
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int wkv_version(void);
 
+/*
+ * wkv_selftest_wait_timeout -- exercise the failure path of the bounded waits
+ * (the mbarrier waits every tensor-core and TMA kernel here uses, each limited
+ * to one second).  Launches one CTA on `stream` whose thread waits on an
+ * mbarrier that nothing arrives on; after the limit the wait gives up, sets
+ * WKV_FAULT_TIMEOUT in the device fault word and the kernel returns, so the
+ * context stays usable.  A caller then sees the bit through
+ * wkv_take_device_faults().  Takes about a second of GPU time; for tests and
+ * health checks only.  Returns WKV_OK, WKV_ERR_DEVICE or WKV_ERR_CUDA.
+ */
+int wkv_selftest_wait_timeout(wkv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,8 @@ __all__ = [
     "WkvError", "lib_path", "load", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd",
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
     "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
-    "wkv5_fwd", "wkv5_fwd_bf16", "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused", "EXPORTED_SYMBOLS",
+    "wkv5_fwd", "wkv5_fwd_bf16", "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused",
+    "wkv_selftest_wait_timeout", "WKV_FAULT_TIMEOUT", "EXPORTED_SYMBOLS",
     "HEAD_SIZE",
 ]
 
@@ -32,8 +33,9 @@ EXPORTED_SYMBOLS = (
     "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd", "wkv6_bwd_workspace_bytes", "wkv4_fwd",
     "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc", "wkv6_fwd_state",
     "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes", "wkv5_fwd", "wkv5_fwd_bf16",
-    "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused",
+    "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused", "wkv_selftest_wait_timeout",
 )
+WKV_FAULT_TIMEOUT = 0x1   # fault-word bit: a bounded device-side wait ran out
 
 _I = ctypes.c_int
 _P = ctypes.c_void_p
@@ -49,6 +51,7 @@ _SIGS = {
     "wkv_status_string": ([_I], ctypes.c_char_p),
     "wkv_take_device_faults": ([ctypes.POINTER(ctypes.c_uint)], _I),
     "wkv_version": ([], _I),
+    "wkv_selftest_wait_timeout": ([_P], _I),
     "wkv6_bwd_noalloc": ([_I] * 5 + [_P] * 11 + [_P], _I),
     "wkv6_fwd_state": ([_I] * 4 + [_P] * 8 + [_P], _I),
     "wkv6_decode": ([_I] * 3 + [_P] * 7 + [_P], _I),
@@ -230,6 +233,12 @@ def wkv_take_device_faults() -> int:
     out = ctypes.c_uint(0)
     _check("wkv_take_device_faults", load().wkv_take_device_faults(ctypes.byref(out)))
     return int(out.value)
+
+
+def wkv_selftest_wait_timeout(stream=None) -> None:
+    """Launch the one-CTA kernel whose bounded wait runs out (about a second); the fault
+    word then holds WKV_FAULT_TIMEOUT (read it with wkv_take_device_faults)."""
+    _check("wkv_selftest_wait_timeout", load().wkv_selftest_wait_timeout(_stream(stream)))
 
 
 def wkv_version() -> int:

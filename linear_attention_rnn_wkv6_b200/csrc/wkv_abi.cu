@@ -488,3 +488,30 @@ extern "C" int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, c
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, scratch};
     return wkv6_bwd_launch(false, bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// wkv_selftest_wait_timeout: exercises the failure path every kernel's bounded
+// waits share.  One thread waits on an mbarrier that nothing arrives on; the
+// wait gives up after its time limit, records WKV_FAULT_TIMEOUT in the fault
+// word and the kernel returns, so the context stays usable.
+
+namespace wkv {
+namespace {
+
+__global__ void wkv_wait_selftest_kernel() {
+    __shared__ alignas(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait_bounded(&bar, 0);   // phase 0 never completes: runs out after kWaitLimitNs
+}
+
+}  // namespace
+}  // namespace wkv
+
+extern "C" int wkv_selftest_wait_timeout(wkv_stream_t stream) {
+    int st = wkv::check_device();
+    if (st != WKV_OK) return st;
+    wkv::wkv_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
