@@ -129,3 +129,62 @@ def test_chunked_form_matches_oracle(T, L, bidirectional, shared):
     for got, ref in zip((y, dr, dk, dv, dw), (y_ref,) + tuple(a[0] for a in g_ref[:4])):
         assert np.allclose(got, ref, rtol=1e-9, atol=1e-10)
     assert np.allclose(du, g_ref[4], rtol=1e-9, atol=1e-10)
+
+
+def _anti_time_ordered(r, k, v, ew, dy, L):
+    """The anti-causal sweep on time-ordered chunk tiles: per chunk the log-decay sums run
+    over the later tokens (Lam^a_t = sum_{m>t} ew_m), Q^a_t = r_t e^{Lam^a_t},
+    Kt^a_s = k_s e^{-(ew_s + Lam^a_s)}, the masks are strict-upper, the state enters a chunk
+    from the later chunks and the adjoint from the earlier ones."""
+    T, N = r.shape
+    chunks = _partition(T, L, ragged_first=False)
+    nc = len(chunks)
+    loc = []
+    for idx in chunks:
+        suf = np.cumsum(ew[idx][::-1], axis=0)[::-1]          # sum_{m >= t}
+        lam = suf - ew[idx]                                     # sum_{m > t}
+        loc.append(dict(idx=idx, E=np.exp(lam), F=np.exp(-suf), gam=np.exp(suf[0]),
+                        Q=r[idx] * np.exp(lam), Kt=k[idx] * np.exp(-suf)))
+    S_in = [None] * nc
+    S_in[nc - 1] = np.zeros((N, N))
+    for j in range(nc - 2, -1, -1):
+        q = loc[j + 1]
+        S_in[j] = q["gam"][:, None] * (S_in[j + 1] + q["Kt"].T @ v[q["idx"]])
+    G = [None] * (nc + 1)          # G[j + 1] = dL/dS_in(j); G[0] = 0
+    G[0] = np.zeros((N, N))
+    for j in range(nc):
+        G[j + 1] = loc[j]["Q"].T @ dy[loc[j]["idx"]] + loc[j]["gam"][:, None] * G[j]
+    y, dr, dk, dv, z, x = (np.zeros((T, N)) for _ in range(6))
+    for j, q in enumerate(loc):
+        idx, Q, Kt, V, dY = q["idx"], q["Q"], q["Kt"], v[q["idx"]], dy[q["idx"]]
+        n = len(idx)
+        up = np.triu(np.ones((n, n)), 1)                      # s > t
+        A = (Q @ Kt.T) * up
+        dA = (dY @ V.T) * up
+        Gt = q["gam"][:, None] * G[j]
+        y[idx] = Q @ S_in[j] + A @ V
+        dQ = dA @ Kt + dY @ S_in[j].T
+        dKt = dA.T @ Q + V @ Gt.T
+        dr[idx], dk[idx], dv[idx] = q["E"] * dQ, q["F"] * dKt, A.T @ dY + Kt @ Gt
+        z[idx], x[idx] = Q * dQ, Kt * dKt
+    # dw_m = sum_{t<m} z_t - sum_{s<=m} x_s (the tokens processed after m come earlier in time)
+    zc = np.cumsum(z, axis=0) - z
+    xc = np.cumsum(x, axis=0)
+    return y, dr, dk, dv, zc - xc
+
+
+@pytest.mark.parametrize("T,L", [(7, 8), (37, 8), (50, 16), (33, 32)])
+def test_anti_causal_sweep_on_time_ordered_tiles(T, L):
+    """Causal part from the processing-order model plus the anti-causal part on time-ordered
+    tiles reproduce the oracle's bidirectional forward and gradients."""
+    N, H = 8, 1
+    r, k, v, ew, u, dy = _case(T, N, seed=7 * T + L)
+    (yc, drc, dkc, dvc, dwc), duc = _chunked(r, k, v, ew, u, dy, L, False, False)
+    ya, dra, dka, dva, dwa = _anti_time_ordered(r, k, v, ew, dy, L)
+    args = [a[None] for a in (r, k, v, ew)]
+    y_ref = oracle.wkv6_fwd(*args, u, H=H, bidirectional=True)[0]
+    g_ref = oracle.wkv6_bwd(*args, u, dy[None], H=H, bidirectional=True)
+    got = (yc + ya, drc + dra, dkc + dka, dvc + dva, dwc + dwa)
+    for a, ref in zip(got, (y_ref,) + tuple(g[0] for g in g_ref[:4])):
+        assert np.allclose(a, ref, rtol=1e-9, atol=1e-10)
+    assert np.allclose(duc, g_ref[4], rtol=1e-9, atol=1e-10)
