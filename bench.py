@@ -36,9 +36,12 @@ METRIC = "WKV tokens/sec/GPU and % of roofline (HBM GB/s or FP32/TC util) vs CPU
 UNIT = "tokens/s"
 WORKLOAD_NAME = ("wkv-hot-path step: wkv4_fwd B8xT1024xC768 f32 + wkv6_bidir_fwd B32xT196xH12 f32 + "
                  "wkv6_fwd_bf16 B8xT4096xH32 + wkv6_bwd(bidir) B32xT196xH12 f32, N=64")
-# Workloads outside the step, measured on their own with --only.
-EXTRA_WORKLOADS = ["wkv6_decode_f32_b512h32", "wkv6_bidir_bwd_bf16_b32t196h12", "wkv4_bwd_f32_b8t1024c768",
-                   "wkv5_causal_bf16_b8t4096h32", "wkv5_bwd_f32_b32t196h12", "wkv6_bidir_fused_f32_b32t196h12"]
+# Workloads outside the step, measured on their own with --only: the small causal fp32
+# forward (B1 T196 H4: four (b, h) units, bound by latency and launch, not by a roof),
+# the causal fp32 forward at the bidirectional workload's shape, and the NEXT rows.
+EXTRA_WORKLOADS = ["wkv6_causal_f32_b1t196h4", "wkv6_causal_f32_b32t196h12", "wkv6_decode_f32_b512h32",
+                   "wkv6_bidir_bwd_bf16_b32t196h12", "wkv4_bwd_f32_b8t1024c768", "wkv5_causal_bf16_b8t4096h32",
+                   "wkv5_bwd_f32_b32t196h12", "wkv6_bidir_fused_f32_b32t196h12"]
 STEP_WORKLOADS = ["wkv4_f32_b8t1024c768", "wkv6_bidir_f32_b32t196h12", "wkv6_causal_bf16_b8t4096h32",
                   "wkv6_bidir_bwd_f32_b32t196h12"]
 N = 64
@@ -46,45 +49,47 @@ L2_BYTES = 126 * 1024 * 1024
 FP32_LANES_PER_SM, SMS, SM_MAX_MHZ = 128, 148, 1965.0
 FP32_PEAK_TFLOPS = SMS * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12   # 74.4 (FMA = 2 flop)
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 # Algorithmic work per unit (a unit is one token of one head for RWKV-6, one
 # (token, channel) for RWKV-4).  Bytes: inputs read once + outputs written once.
 # Flops: RWKV-6 forward 5 N^2 per direction (state update 3 N^2 + readout 2 N^2),
-# backward 14 N^2 per direction; RWKV-4 ~4 exp + 12 flop (HBM bound).  The bf16
-# causal forward and the fp32 forward (causal and bidirectional) run on the tensor
-# cores (chunked form: about 40 N^2 tensor flops per unit and direction, six split
-# bf16 products each for fp32, against a 1.7 PFLOP/s pipe), so their bound is the
-# bytes they must move; the FP32-equivalent rate is reported next to it.
+# backward 14 N^2 per direction; RWKV-4 ~4 exp + 12 flop.  Each kernel's roofline
+# time is the slower of its bytes at HBM bandwidth and its flops at the peak of the
+# pipe it computes on (uses_tensor_cores): for the chunked tensor-core forms the
+# bytes bind, for the recurrence kernels of the test build the FP32 FMA pipe; both
+# fractions are reported per kernel.
 ALG = {
-    "wkv4_f32_b8t1024c768": dict(bytes_per_unit=3 * 4, flops_per_unit=16, bound="hbm"),
-    "wkv6_bidir_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=10 * N * N, bound="hbm"),
-    "wkv6_causal_bf16_b8t4096h32": dict(bytes_per_unit=4 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
+    "wkv4_f32_b8t1024c768": dict(bytes_per_unit=3 * 4, flops_per_unit=16),
+    "wkv6_causal_f32_b1t196h4": dict(bytes_per_unit=5 * N * 4, flops_per_unit=5 * N * N),
+    "wkv6_causal_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=5 * N * N),
+    "wkv6_bidir_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4, flops_per_unit=10 * N * N),
+    "wkv6_causal_bf16_b8t4096h32": dict(bytes_per_unit=4 * N * 2 + N * 4, flops_per_unit=5 * N * N),
     # the fp32 backward's default path runs on the tensor cores (two-term split bf16 operands)
-    "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N, bound="hbm"),
-    "wkv6_bidir_bwd_bf16_b32t196h12": dict(bytes_per_unit=5 * N * 2 + 4 * N * 4, flops_per_unit=28 * N * N,
-                                           bound="hbm"),
+    "wkv6_bidir_bwd_f32_b32t196h12": dict(bytes_per_unit=9 * N * 4, flops_per_unit=28 * N * N),
+    "wkv6_bidir_bwd_bf16_b32t196h12": dict(bytes_per_unit=5 * N * 2 + 4 * N * 4, flops_per_unit=28 * N * N),
     # RWKV-4 backward: k, v, dy in and dk, dv out per (token, channel)
-    "wkv4_bwd_f32_b8t1024c768": dict(bytes_per_unit=5 * 4, flops_per_unit=40, bound="hbm"),
+    "wkv4_bwd_f32_b8t1024c768": dict(bytes_per_unit=5 * 4, flops_per_unit=40),
     # decode: the state is read and written once per step (2 N^2 floats) next to 5 N floats of token data
-    "wkv6_decode_f32_b512h32": dict(bytes_per_unit=2 * N * N * 4 + 5 * N * 4, flops_per_unit=5 * N * N,
-                                    bound="hbm"),
+    "wkv6_decode_f32_b512h32": dict(bytes_per_unit=2 * N * N * 4 + 5 * N * 4, flops_per_unit=5 * N * N),
     # RWKV-5: no per-token w; the forward and the causal backward run the tensor-core
     # chunked forms, so both are bound by their bytes: the forward reads bf16 r, k, v and
     # writes fp32 y; the backward reads r, k, v, dy and writes dr, dk, dv (w, dw, u, du
     # are per channel)
-    "wkv5_causal_bf16_b8t4096h32": dict(bytes_per_unit=3 * N * 2 + N * 4, flops_per_unit=5 * N * N, bound="hbm"),
-    "wkv5_bwd_f32_b32t196h12": dict(bytes_per_unit=7 * N * 4, flops_per_unit=14 * N * N, bound="hbm"),
+    "wkv5_causal_bf16_b8t4096h32": dict(bytes_per_unit=3 * N * 2 + N * 4, flops_per_unit=5 * N * N),
+    "wkv5_bwd_f32_b32t196h12": dict(bytes_per_unit=7 * N * 4, flops_per_unit=14 * N * N),
     # fused forward (tensor-core kernel): r, k, v, ww and the gate in, the normalised and gated output out
-    "wkv6_bidir_fused_f32_b32t196h12": dict(bytes_per_unit=6 * N * 4, flops_per_unit=10 * N * N, bound="hbm"),
+    "wkv6_bidir_fused_f32_b32t196h12": dict(bytes_per_unit=6 * N * 4, flops_per_unit=10 * N * N),
 }
-ENTRY = {"wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
+ENTRY = {"wkv6_causal_f32_b1t196h4": "wkv6_fwd", "wkv6_causal_f32_b32t196h12": "wkv6_fwd",
+         "wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
          "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd",
          "wkv6_decode_f32_b512h32": "wkv6_decode", "wkv6_bidir_bwd_bf16_b32t196h12": "wkv6_bwd_bf16",
          "wkv4_bwd_f32_b8t1024c768": "wkv4_bwd", "wkv5_causal_bf16_b8t4096h32": "wkv5_fwd_bf16",
          "wkv5_bwd_f32_b32t196h12": "wkv5_bwd", "wkv6_bidir_fused_f32_b32t196h12": "wkv6_fwd_fused"}
 FLUSH_BYTES = 512 << 20   # an L2 flush write; working sets below this get one before every step
 
-LAUNCHES = {"wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
+LAUNCHES = {"wkv6_causal_f32_b1t196h4": 1, "wkv6_causal_f32_b32t196h12": 1, "wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
             "wkv6_bidir_bwd_f32_b32t196h12": 3,   # S-kind and G-kind tensor-core kernels and the deterministic du reduction
             "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 3,
             "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
@@ -156,6 +161,23 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def load_tensor_peak():
+    """Dense bf16 tensor throughput (TFLOP/s): the measured burst figure, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def uses_tensor_cores(name: str, library: str = "default") -> bool:
+    """Whether the workload's entry point runs a chunked tensor-core form in that build
+    (RWKV-4 and the decode step run on the CUDA cores in every build; the test build
+    runs every RWKV-6 and RWKV-5 entry point on its recurrence kernels)."""
+    return library == "default" and not name.startswith("wkv4") and "decode" not in name
+
+
 def kernel_source_hash() -> str:
     import glob
     h = hashlib.sha256()
@@ -181,26 +203,74 @@ def recorded_traffic(name: str):
 
 
 class ClockSampler:
-    """Samples nvidia-smi during the timed region (SM clock, throttle reasons)."""
+    """Samples the GPU's SM clock, power and throttle reasons every `period_s` during the
+    timed region, through NVML from a background thread (a timed region of a few ms
+    still gets samples); falls back to an `nvidia-smi -lms 50` child process when NVML
+    cannot be loaded."""
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.dev = device_index
+        self.period = period_s
+        self.samples = []     # (sm_mhz, sm_max_mhz, power_w, reason names)
+        self.source = None
         self.proc = None
+        self.thread = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            nv, h = self._nvml_handle()
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.stop = threading.Event()
+
+            def poll():
+                while True:
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, sm_max, pw, tuple(n for n, bit in bits.items() if rs & bit)))
+                    except Exception:
+                        pass
+                    if self.stop.wait(self.period):
+                        return
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = f"NVML every {self.period * 1e3:.0f} ms"
         except Exception:
-            self.proc = None
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                              "--format=csv,noheader,nounits", "-lms", "50"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi -lms 50"
+            except Exception:
+                self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -208,26 +278,26 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
                 out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            for ln in out.splitlines():
+                f = [x.strip() for x in ln.split(",")]
+                if len(f) < 8:
+                    continue
+                try:
+                    sm, mx = float(f[0]), float(f[1])
+                    pw = float(f[2]) if f[2].replace(".", "", 1).isdigit() else 0.0
+                except ValueError:
+                    continue
+                self.samples.append((sm, mx, pw, tuple(n for n, v in zip(self.NAMES, f[4:8])
+                                                      if v.lower().startswith("active"))))
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 8:
-                continue
-            try:
-                sm.append(float(f[0]))
-                mx = float(f[1])
-            except ValueError:
-                continue
-            for nm, val in zip(names, f[4:8]):
-                if val.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({n for x in self.samples for n in x[3]})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.samples[-1][1], "reasons": reasons,
+                "samples": len(sm), "power_w_max": round(max(x[2] for x in self.samples), 1),
+                "source": self.source}
 
 
 # ----------------------------------------------------------------------------- native (CUDA) arm
@@ -235,12 +305,23 @@ class ClockSampler:
 class DeviceWorkload:
     """Inputs resident in HBM, outputs and workspace preallocated; run() enqueues the ABI call."""
 
-    def __init__(self, name: str, seed: int):
+    def __init__(self, name: str, rank: int = 0, world: int = 1):
         import numpy as np
         import torch
         from linear_attention_rnn_wkv6_b200 import synth
+        from linear_attention_rnn_wkv6_b200.shard import batch_range
         self.name = name
-        self.kind, self.x = synth.make_workload(name, seed=seed)
+        # One seeded problem of world x B batches; this rank holds its window of
+        # batches.  Workloads without batch windows (static decay, fused, decode) run
+        # independent replicas with a rank-dependent seed instead.
+        self.split = world > 1 and synth.WORKLOADS[name][0] in (
+            "wkv4_fwd", "wkv4_bwd", "wkv6_fwd", "wkv6_fwd_bf16", "wkv6_bidir_fwd", "wkv6_bwd_bidir")
+        if self.split:
+            Bw = synth.WORKLOADS[name][1]["B"]
+            self.kind, self.x = synth.make_workload(name, seed=0, batch_scale=world,
+                                                    batches=batch_range(Bw * world, rank, world))
+        else:
+            self.kind, self.x = synth.make_workload(name, seed=1000 * rank)
         x = self.x
 
         def dev(a):
@@ -298,6 +379,8 @@ class DeviceWorkload:
         s = stream.cuda_stream
         if self.kind == "wkv4_fwd":
             wkv.wkv4_fwd(x.B, x.T, x.C, i["k"], i["v"], i["w"], i["u"], o[0], s)
+        elif self.kind == "wkv6_fwd":
+            wkv.wkv6_fwd(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], o[0], s)
         elif self.kind == "wkv4_bwd":
             wkv.wkv4_bwd(x.B, x.T, x.C, i["k"], i["v"], i["w"], i["u"], i["dy"], *o, self.ws, self.ws_bytes, s)
         elif self.kind == "wkv6_bidir_fwd":
@@ -323,6 +406,14 @@ class DeviceWorkload:
             wkv.wkv6_decode(x.B, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], self.state, o[0], s)
         else:
             raise ValueError(self.kind)
+        if self.split and self.kind in ("wkv6_bwd_bidir", "wkv4_bwd"):
+            # the batch-split backward's one exchange: the per-channel gradients summed
+            # over the batch (du; RWKV-4 also dw) are all-reduced over the ranks
+            import torch
+            from linear_attention_rnn_wkv6_b200.shard import allreduce_du
+            with torch.cuda.stream(stream):
+                for t in (o[4],) if self.kind == "wkv6_bwd_bidir" else (o[2], o[3]):
+                    allreduce_du(t)
 
 
 class HostSide:
@@ -375,9 +466,10 @@ def run_native(args, rank, world, local):
     torch.cuda.set_device(local)
     dist = init_group("nccl", world)
     dev = torch.device("cuda", local)
+    if args.library != "default":
+        wkv.use_library(args.library).__enter__()   # for the rest of this process
     wkv.load()
-    seed = 1000 * rank
-    wls = [DeviceWorkload(n, seed) for n in (args.only or STEP_WORKLOADS)]
+    wls = [DeviceWorkload(n, rank, world) for n in (args.only or STEP_WORKLOADS)]
     stream = torch.cuda.Stream()
     tokens_per_step = sum(w.tokens for w in wls)
     # A working set that fits in L2 several times over would stay cached from one step
@@ -463,25 +555,37 @@ def run_native(args, rank, world, local):
 
     if rank == 0:
         hbm, hbm_src = load_peaks()
+        tc_peak, tc_src = load_tensor_peak()
         kernels = {}
         for j, w in enumerate(wls):
             a = ALG[w.name]
             t_s = per_kernel_ms[j] / 1e3
             alg_bytes = a["bytes_per_unit"] * w.units
             alg_flops = a["flops_per_unit"] * w.units
-            if a["bound"] == "hbm":
-                achieved, peak, unit = alg_bytes / t_s / 1e9, hbm, "GB/s"
+            # roofline time = the slower of the bytes at HBM bandwidth and the flops at the
+            # peak of the pipe the kernel computes on (the tensor pipe for the chunked forms,
+            # the FP32 FMA pipe for the recurrences); frac = roofline time / measured time
+            pipe = "tensor" if uses_tensor_cores(w.name, args.library) else "fp32"
+            t_bytes = alg_bytes / (hbm * 1e9)
+            t_flops = alg_flops / ((tc_peak if pipe == "tensor" else FP32_PEAK_TFLOPS) * 1e12)
+            if t_bytes >= t_flops:
+                bound, achieved, peak, unit = "hbm", alg_bytes / t_s / 1e9, hbm, "GB/s"
                 peak_src = f"{hbm_src} HBM copy bandwidth"
+            elif pipe == "tensor":
+                bound, achieved, peak, unit = "tensor", alg_flops / t_s / 1e12, tc_peak, "TFLOP/s"
+                peak_src = f"{tc_src} bf16 tensor throughput"
             else:
-                achieved, peak, unit = alg_flops / t_s / 1e12, FP32_PEAK_TFLOPS, "TFLOP/s"
+                bound, achieved, peak, unit = "alu", alg_flops / t_s / 1e12, FP32_PEAK_TFLOPS, "TFLOP/s"
                 peak_src = "derived FP32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz"
             kernels[w.name] = {
                 "entry": ENTRY[w.name], "launches": LAUNCHES[w.name], "ms": round(per_kernel_ms[j], 4),
                 "tokens_per_s": round(w.tokens / t_s, 1), "units": w.units,
-                "alg_bytes": alg_bytes, "alg_flops": alg_flops,
+                "alg_bytes": alg_bytes, "alg_flops": alg_flops, "pipe": pipe,
                 "hbm_gbs": round(alg_bytes / t_s / 1e9, 1), "fp32_tflops": round(alg_flops / t_s / 1e12, 2),
-                "bound": a["bound"], "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": unit,
-                "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                "hbm_frac": round(alg_bytes / t_s / 1e9 / hbm, 4),
+                "fp32_frac": round(alg_flops / t_s / 1e12 / FP32_PEAK_TFLOPS, 4),
+                "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": unit,
+                "frac": round(max(t_bytes, t_flops) / t_s, 4), "peak_source": peak_src,
                 "share": round(per_kernel_ms[j] / sum(per_kernel_ms), 4),
             }
         dom = max(kernels, key=lambda n: kernels[n]["ms"])
@@ -492,7 +596,9 @@ def run_native(args, rank, world, local):
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs on the causal workload)",
-            "data": "synthetic (seeded splitmix64 + Box-Muller, rank-dependent seed)",
+            "data": ("synthetic (seeded splitmix64 + Box-Muller): one problem of N x B batches, each rank "
+                     "generating its own window of batches" if world > 1 else "synthetic (seeded splitmix64 + "
+                     "Box-Muller, seed 0)"),
             "config": {"workload": WORKLOAD_NAME if not args.only else " + ".join(args.only),
                        "tokens_per_step_per_gpu": tokens_per_step,
                        "l2": (f"working set {ws_bytes / 1e6:.0f} MB: L2 (126 MB) flushed before every step by a "
@@ -500,8 +606,12 @@ def run_native(args, rank, world, local):
                               "of the kernels' event times") if flush else
                              f"inputs larger than L2: step working set {ws_bytes / 1e9:.2f} GB > 126 MB L2, "
                              "no explicit flush",
-                       "parallelism": f"replicated weak scaling x{world} (independent problems per rank)"},
-            "roofline": {"kernel": dom, "bound": "hbm" if d["bound"] == "hbm" else "alu",
+                       "parallelism": (f"batch split x{world}: one problem of {world} x B batches, rank r "
+                                       "owning batches [rB, (r+1)B) (weak scaling: B per GPU fixed); the backward's "
+                                       "du all-reduced over the ranks (NCCL, C floats) inside every step"
+                                       if world > 1 else "single GPU"),
+                       "library": os.path.basename(wkv.lib_path())},
+            "roofline": {"kernel": dom, "bound": d["bound"],
                          "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
                          "traffic": traffic, "peak_source": d["peak_source"]},
             "kernels": kernels,
@@ -657,6 +767,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--only", action="append", choices=STEP_WORKLOADS + EXTRA_WORKLOADS,
                     help="run only these workloads (profiling); the default step runs all four")
+    ap.add_argument("--library", choices=["default", "recurrence"], default="default",
+                    help="the library build to time: the product (default) or the test build whose "
+                         "chunked-form entry points run the recurrence kernels (for comparison)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -21,6 +21,17 @@
  *  - B == 0 or T == 0 is a valid empty problem: nothing is launched, except
  *    that wkv6_bwd zeroes du when B*T == 0.
  *
+ * Library builds
+ * --------------
+ * libwkv.so runs one fixed algorithm per entry point: the chunked tensor-core
+ * forms where an entry point has one.  The same sources built with
+ * -DWKV_RECURRENCE_PATHS=1 give libwkv_recurrence.so, a test and comparison
+ * build with this same ABI in which wkv6_fwd, wkv6_fwd_bf16, wkv6_bidir_fwd,
+ * wkv6_fwd_fused, wkv5_fwd_bf16, wkv6_bwd, wkv6_bwd_bf16 and wkv5_bwd run the
+ * token-by-token recurrence kernels instead (the kernels wkv6_fwd_state,
+ * wkv5_fwd and wkv6_bwd_noalloc use in both builds).  Results agree within the
+ * tolerances stated below; nothing is selected at run time.
+ *
  * RWKV-6 log-decay
  * ----------------
  * The decay argument w of the RWKV-6 entry points is the log-decay
@@ -73,8 +84,8 @@ enum {
  *   y          : [B,T,C] float, output
  * Algorithm: the chunked form ("RWKV Architecture ...", Parallel Training
  * Formulation) on the tensor cores, every fp32 operand split exactly into three
- * bf16 terms (relative L2 error about 2e-7); with the environment variable
- * WKV6_F32_PATH=recurrence (read on every call), the token-by-token recurrence.
+ * bf16 terms (relative L2 error about 2e-7).  (In the test build, see "Library
+ * builds" above, the token-by-token recurrence.)
  */
 int wkv6_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v,
              const float *w, const float *u, float *y, wkv_stream_t stream);
@@ -150,10 +161,9 @@ int wkv6_decode(int B, int C, int H, const float *r, const float *k, const float
  *                        on entry is ignored and on exit undefined.
  * Algorithm: the chunked form on the tensor cores in two kernels (one carrying
  * the forward state, one the adjoint), operands split into two bf16 terms
- * (relative L2 error about 1e-5 on every gradient); with the environment
- * variable WKV6_BWD_PATH=recurrence (read on every call), the two-sweep
- * recurrence.  Both write every output element; only the order of additions
- * differs, and each is bitwise reproducible run to run.
+ * (relative L2 error about 1e-5 on every gradient); in the test build, the
+ * two-sweep recurrence.  Both write every output element; only the order of
+ * additions differs, and each is bitwise reproducible run to run.
  */
 int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, const float *k,
              const float *v, const float *w, const float *u, const float *dy, float *dr, float *dk,
@@ -164,8 +174,8 @@ int wkv6_bwd(int B, int T, int C, int H, int bidirectional, const float *r, cons
  * wkv6_bwd_bf16 -- wkv6_bwd with bfloat16 r, k, v, w and dy (raw IEEE bf16 bit
  * patterns, uint16_t) for bf16 training: the same gradients, computed in fp32
  * from the bf16 values, with u and every gradient (dr, dk, dv, dw, du) in fp32.
- * Same layouts, workspace (wkv6_bwd_workspace_bytes), algorithms (and
- * WKV6_BWD_PATH switch) and errors as wkv6_bwd.
+ * Same layouts, workspace (wkv6_bwd_workspace_bytes), algorithms and errors
+ * as wkv6_bwd.
  */
 int wkv6_bwd_bf16(int B, int T, int C, int H, int bidirectional, const uint16_t *r, const uint16_t *k,
                   const uint16_t *v, const uint16_t *w, const float *u, const uint16_t *dy, float *dr,
@@ -195,7 +205,10 @@ size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional);
  *   Limit: B*C <= 262144, else WKV_ERR_TOO_LARGE and nothing is launched.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept with the context it was
+ *   looked up in: after a cudaDeviceReset (a new context, into which the
+ *   library's device code is loaded anew) the next call looks it up again, so
+ *   that call too must come before any stream capture.
  *   All calls share the one array: calls that may overlap on the GPU (on
  *   different streams, or from several host threads) race and must be
  *   serialised by the caller.  Nothing in the array needs clearing between
@@ -225,8 +238,7 @@ int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, const float 
  *   where y is wkv6_fwd (or wkv6_bidir_fwd) at w = -exp(w_base + ww), and mu and
  *   var are the mean and the (biased) variance of y over the N channels of c's
  *   head at (b, t).  Neither the log-decay nor y is written to memory.
- * Same sizes, pointer rules, algorithm switch (WKV6_F32_PATH) and errors as
- * wkv6_fwd; eps <= 0 or not finite gives WKV_ERR_ARG.  On the tensor-core path
+ * Same sizes, pointer rules, algorithms and errors as wkv6_fwd; eps <= 0 or not finite gives WKV_ERR_ARG.  On the tensor-core path
  * the prologue runs where the chunk is transformed and the norm and gate in the
  * last sweep's epilogue.
  */

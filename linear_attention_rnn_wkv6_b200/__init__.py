@@ -12,6 +12,7 @@ Build the library with ``python -m linear_attention_rnn_wkv6_b200.build``.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -21,12 +22,16 @@ __all__ = [
     "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
     "wkv5_fwd", "wkv5_fwd_bf16", "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused",
     "wkv_selftest_wait_timeout", "WKV_FAULT_TIMEOUT", "EXPORTED_SYMBOLS",
-    "HEAD_SIZE",
+    "HEAD_SIZE", "LIBRARY_FILES", "use_library",
 ]
 
 HEAD_SIZE = 64
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB = None
+# The two builds of the library (same C ABI): the product, and the test build whose
+# chunked-form entry points run the token-by-token recurrence kernels.
+LIBRARY_FILES = {"default": "libwkv.so", "recurrence": "libwkv_recurrence.so"}
+_LIBS: dict = {}
+_ACTIVE = ["default"]
 
 # Every extern "C" symbol declared in include/wkv.h.
 EXPORTED_SYMBOLS = (
@@ -72,15 +77,17 @@ class WkvError(RuntimeError):
         super().__init__(f"{fn} failed with status {status}: {wkv_status_string(status)}")
 
 
-def lib_path() -> str:
-    return os.path.join(_HERE, "libwkv.so")
+def lib_path(variant: str | None = None) -> str:
+    return os.path.join(_HERE, LIBRARY_FILES[variant or _ACTIVE[0]])
 
 
-def load():
-    """Load libwkv.so (raises if it has not been built)."""
-    global _LIB
-    if _LIB is None:
-        path = lib_path()
+def load(variant: str | None = None):
+    """Load a build of the library (default: the one selected by use_library, normally
+    libwkv.so); raises if it has not been built."""
+    variant = variant or _ACTIVE[0]
+    lib = _LIBS.get(variant)
+    if lib is None:
+        path = lib_path(variant)
         if not os.path.exists(path):
             raise RuntimeError(f"{path} is missing: build it with `python -m linear_attention_rnn_wkv6_b200.build` "
                                "(the WKV operator has no fallback implementation)")
@@ -89,8 +96,22 @@ def load():
             f = getattr(lib, name)
             f.argtypes = args
             f.restype = res
-        _LIB = lib
-    return _LIB
+        _LIBS[variant] = lib
+    return lib
+
+
+@contextlib.contextmanager
+def use_library(variant: str):
+    """Route the wrappers below to another build of the library inside the block
+    ("recurrence": libwkv_recurrence.so, for tests and comparison timings)."""
+    if variant not in LIBRARY_FILES:
+        raise ValueError(f"unknown library build {variant!r}")
+    prev = _ACTIVE[0]
+    _ACTIVE[0] = variant
+    try:
+        yield load(variant)
+    finally:
+        _ACTIVE[0] = prev
 
 
 def _ptr(x) -> int | None:

@@ -477,10 +477,17 @@ static cudaError_t launch_bwd(const CUtensorMap *maps, const BwdParams &prm, cud
 cudaError_t wkv6_bwd_launch(bool bf16, bool bidir, const CUtensorMap *maps, const BwdParams &prm, float *du,
                             cudaStream_t stream) {
     constexpr int TC = kBwdTC;
+    // fp32 inputs serve wkv6_bwd_noalloc in every build; bf16 inputs are reached only in
+    // the library built with WKV_RECURRENCE_PATHS, whose wkv6_bwd_bf16 runs this kernel.
+#if WKV_RECURRENCE_PATHS
     using BF = __nv_bfloat16;
     cudaError_t e = bf16 ? (bidir ? launch_bwd<BF, TC, true>(maps, prm, stream) : launch_bwd<BF, TC, false>(maps, prm, stream))
                          : (bidir ? launch_bwd<float, TC, true>(maps, prm, stream)
                                   : launch_bwd<float, TC, false>(maps, prm, stream));
+#else
+    if (bf16) return cudaErrorNotSupported;
+    cudaError_t e = bidir ? launch_bwd<float, TC, true>(maps, prm, stream) : launch_bwd<float, TC, false>(maps, prm, stream);
+#endif
     if (e != cudaSuccess) return e;
     wkv6_du_reduce_kernel<<<(prm.C + 255) / 256, 256, 0, stream>>>(prm.B, prm.C, prm.du_part, du);
     return cudaGetLastError();

@@ -468,12 +468,16 @@ cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const 
                             const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
                             cudaStream_t stream) {
     constexpr int TC = kFwdTC;
-    if (bf16) {
-        return bidir ? launch_fwd<__nv_bfloat16, 4, TC, true>(mr, mk, mv, mw, prm, stream)
-                     : launch_fwd<__nv_bfloat16, 4, TC, false>(mr, mk, mv, mw, prm, stream);
-    }
-    return bidir ? launch_fwd<float, 4, TC, true>(mr, mk, mv, mw, prm, stream)
-                 : launch_fwd<float, 4, TC, false>(mr, mk, mv, mw, prm, stream);
+    // The fp32 causal form serves wkv6_fwd_state and wkv5_fwd in every build.  The
+    // bf16 causal and fp32 bidirectional forms are reached only in the library built
+    // with WKV_RECURRENCE_PATHS, whose chunked-form entry points run this kernel.
+#if WKV_RECURRENCE_PATHS
+    if (bf16) return bidir ? cudaErrorNotSupported : launch_fwd<__nv_bfloat16, 4, TC, false>(mr, mk, mv, mw, prm, stream);
+    if (bidir) return launch_fwd<float, 4, TC, true>(mr, mk, mv, mw, prm, stream);
+#else
+    if (bf16 || bidir) return cudaErrorNotSupported;
+#endif
+    return launch_fwd<float, 4, TC, false>(mr, mk, mv, mw, prm, stream);
 }
 
 }  // namespace wkv

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/wkv.h"
@@ -59,18 +60,18 @@ bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int B, int T, int C, i
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// sm_100 check, cached per device.
+// sm_100 check, cached per device (entry points may be called from several host threads).
 int check_device() {
-    static int cached[64];   // 0 unknown, 1 ok, 2 bad
+    static std::atomic<int> cached[64];   // 0 unknown, 1 ok, 2 bad
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WKV_ERR_CUDA;
-    if (dev >= 0 && dev < 64 && cached[dev] == 1) return WKV_OK;
+    if (dev >= 0 && dev < 64 && cached[dev].load(std::memory_order_relaxed) == 1) return WKV_OK;
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return WKV_ERR_CUDA;
     const bool ok = (major == 10 && minor == 0);
-    if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+    if (dev >= 0 && dev < 64) cached[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
     return ok ? WKV_OK : WKV_ERR_DEVICE;
 }
 
@@ -97,13 +98,15 @@ bool make_bwd_maps(CUtensorMap (&maps)[kBwdMaps], bool bf16, int B, int T, int C
     return true;
 }
 
-// Algorithm of the backward (fp32 or bf16 inputs): the chunked tensor-core kernels
-// with split-bf16 operands (default) or the two-sweep recurrence
-// (WKV6_BWD_PATH=recurrence).  Read on every call.
-bool bwd_use_tensor_cores() {
-    const char *e = std::getenv("WKV6_BWD_PATH");
-    return !(e && std::strcmp(e, "recurrence") == 0);
-}
+// Algorithm of every entry point that has a chunked tensor-core form (the fp32 and
+// bf16 forwards and backwards): fixed when the library is built.  The product
+// library (libwkv.so) runs the chunked forms; the test library built with
+// -DWKV_RECURRENCE_PATHS=1 (libwkv_recurrence.so) runs the token-by-token
+// recurrence kernels behind the same entry points.
+#ifndef WKV_RECURRENCE_PATHS
+#define WKV_RECURRENCE_PATHS 0
+#endif
+constexpr bool kTensorCorePaths = !WKV_RECURRENCE_PATHS;
 
 // Scratch of the tensor-core backward: per-batch du partials [B][C] and the S kind's
 // per-channel z totals [B][C].
@@ -124,9 +127,10 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
         if ((st = check_device()) != WKV_OK) return st;
         return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
     }
-    const bool tensor = bwd_use_tensor_cores();
-    const size_t need = tensor ? bwd_tensor_workspace_floats(B, T, C, bidirectional != 0) * sizeof(float)
-                               : (size_t)B * (size_t)C * sizeof(float);
+    const bool tensor = kTensorCorePaths;
+    // the documented requirement (wkv6_bwd_workspace_bytes) in both builds, although
+    // the recurrence uses only its first B*C floats
+    const size_t need = bwd_tensor_workspace_floats(B, T, C, bidirectional != 0) * sizeof(float);
     if (workspace == nullptr || workspace_bytes < need) return WKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
     if ((st = check_device()) != WKV_OK) return st;
@@ -142,22 +146,6 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
     if (!make_bwd_maps(maps, bf16, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, static_cast<float *>(workspace)};
     return wkv6_bwd_launch(bf16, bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
-}
-
-// Algorithm of the bf16 causal forward: the chunked tensor-core kernel (default)
-// or the token-by-token recurrence (WKV6_BF16_PATH=recurrence).  Both compute
-// the same operation; the variable is read on every call.
-bool bf16_use_tensor_cores() {
-    const char *e = std::getenv("WKV6_BF16_PATH");
-    return !(e && std::strcmp(e, "recurrence") == 0);
-}
-
-// Algorithm of the fp32 forward without state in/out, prologue or epilogue: the
-// chunked tensor-core kernel with split-bf16 operands (default) or the
-// token-by-token recurrence (WKV6_F32_PATH=recurrence).  Read on every call.
-bool f32_use_tensor_cores() {
-    const char *e = std::getenv("WKV6_F32_PATH");
-    return !(e && std::strcmp(e, "recurrence") == 0);
 }
 
 // w5 (RWKV-5): static per-channel decay rate [C]; then w is ignored (pass w5 for
@@ -176,7 +164,7 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
     if (B == 0 || T == 0) return WKV_OK;
     if ((st = check_device()) != WKV_OK) return st;
     CUtensorMap mr, mk, mv, mw;
-    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && fused == nullptr && bf16_use_tensor_cores()) {
+    if (bf16 && !bidir && s0 == nullptr && sT == nullptr && fused == nullptr && kTensorCorePaths) {
         constexpr int kTcChunk = 64;
         CUtensorMap my;
         if (!make_map(&mr, r, true, B, T, C, kHead, kTcChunk, true) ||
@@ -191,7 +179,7 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
                    ? WKV_OK
                    : WKV_ERR_CUDA;
     }
-    if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && f32_use_tensor_cores()) {
+    if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && kTensorCorePaths) {
         FwdParams prm{B, T, C, H, u, y};
         if (fused != nullptr) {
             prm.wb = fused->wb;
@@ -451,16 +439,40 @@ static __device__ __align__(256) float g_noalloc_du_partials[kNoAllocDuFloats];
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 float *g_noalloc_ptr[kMaxDevices];
+CUcontext g_noalloc_ctx[kMaxDevices];   // the context the address above belongs to
 
-// Device address of the scratch array on the current device (looked up once per device).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+// Device address of the scratch array on the current device.  It is looked up
+// (cudaGetSymbolAddress, with the device current) on the first call on each
+// device, and again whenever the device's context has changed since (after a
+// cudaDeviceReset the library's device code is loaded anew and the array may move).
 int noalloc_scratch(float **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx == nullptr) return WKV_ERR_CUDA;
+    CUcontext ctx = nullptr;   // null until the runtime has made the device's context current here
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return WKV_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void *p = nullptr;
+    if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || g_noalloc_ctx[dev] != ctx) {
+        void *p = nullptr;   // the lookup also makes the device's primary context current
         if (cudaGetSymbolAddress(&p, g_noalloc_du_partials) != cudaSuccess || p == nullptr) return WKV_ERR_CUDA;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return WKV_ERR_CUDA;
         g_noalloc_ptr[dev] = static_cast<float *>(p);
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_ptr[dev];
     return WKV_OK;

@@ -1,21 +1,17 @@
 // wkv_tc.cuh -- 5th-generation tensor-core (tcgen05) helpers for sm_100a.
 //
-// Operand tiles in shared memory use the no-swizzle canonical layout built
-// from 16-byte "units" (4 fp32 / tf32 values contiguous along one dimension):
-//     tile[unit][row][4]      (unit = contiguous-dimension index / 4)
-// with 64 rows per unit-slab (16 KB for a 64 x 64 fp32 tile).  Eight
-// consecutive rows of one unit form a 128-byte core matrix.  The same buffer
-// is a K-major operand when `unit` runs along K (rows along M/N) and an
-// MN-major operand when `unit` runs along M/N (rows along K); only the two
-// descriptor strides differ:
-//     K-major : SBO = 128 B (next 8 rows of M/N),  LBO = 64*16 B (next K unit)
-//     MN-major: SBO = 64*16 B (next M/N unit),     LBO = 128 B (next 8 rows of K)
-// One kind::tf32 MMA consumes K = 8: two K units (K-major, start advances by
-// 2*1024 B per step) or eight K rows (MN-major, start advances by 128 B).
+// Operands are bf16 tiles in shared memory (kind::f16, fp32 accumulators in
+// tensor memory).  A 64-row tile stores each row as 128 contiguous bytes
+// (64 bf16 values) with the 128-byte swizzle TMA applies (16-byte chunk g of row
+// r at chunk g ^ (r & 7)); read through a descriptor it is a K-major operand
+// (rows along M/N, K contiguous) or an MN-major one (rows along K), see desc_k
+// and desc_mn.  Small 32-row chunk matrices use the no-swizzle K-major layout
+// (units of 8 columns, 512 bytes apart; built by their kernels with smem_desc).
 //
 // Accumulators are fp32 in tensor memory.  With M = 64 (cta_group::1) row m of
 // D lives in TMEM lane (m % 16) + 32 * (m / 16), column n in column n, so warp
-// w reads rows 16w .. 16w+15 through its lanes 32w .. 32w+15.
+// w reads rows 16w .. 16w+15 through its lanes 32w .. 32w+15; with M = 128 row
+// m is lane m.
 #pragma once
 
 #include "wkv_common.cuh"
@@ -23,7 +19,8 @@
 namespace wkv {
 namespace tc {
 
-// ---- shared-memory matrix descriptor (tcgen05 format, version 1, no swizzle)
+// ---- shared-memory matrix descriptor (tcgen05 format, version 1); the layout
+// type (bits 61..63) is added by the callers that use a swizzled tile
 __device__ __forceinline__ uint64_t smem_desc(const void *base, uint32_t lbo_bytes, uint32_t sbo_bytes) {
     const uint32_t addr = smem_u32(base);
     uint64_t d = 0;
@@ -31,41 +28,7 @@ __device__ __forceinline__ uint64_t smem_desc(const void *base, uint32_t lbo_byt
     d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;    // bits [16,30) leading byte offset >> 4
     d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;    // bits [32,46) stride byte offset >> 4
     d |= (uint64_t)1 << 46;                               // bits [46,48) version = 1
-    // base offset 0, lbo mode 0, layout type 0 (no swizzle)
     return d;
-}
-
-constexpr uint32_t kUnitSlab = 64 * 16;   // bytes between units of a 64-row tile
-
-__device__ __forceinline__ uint64_t desc_kmajor(const void *tile, int kstep) {
-    // kstep-th group of 8 K values = 2 units
-    return smem_desc(static_cast<const char *>(tile) + 2 * kstep * kUnitSlab, kUnitSlab, 128);
-}
-__device__ __forceinline__ uint64_t desc_mnmajor(const void *tile, int kstep) {
-    // kstep-th group of 8 K rows = 128 bytes into every unit slab
-    return smem_desc(static_cast<const char *>(tile) + 128 * kstep, 128, kUnitSlab);
-}
-
-// ---- instruction descriptor: kind::tf32, D fp32, A/B tf32, M x N, majors
-__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn_major, bool b_mn_major) {
-    return (1u << 4)                          // D format f32
-         | (2u << 7)                          // A format tf32
-         | (2u << 10)                         // B format tf32
-         | ((a_mn_major ? 1u : 0u) << 15)
-         | ((b_mn_major ? 1u : 0u) << 16)
-         | ((uint32_t)(N >> 3) << 17)
-         | ((uint32_t)(M >> 4) << 24);
-}
-
-// ---- MMA issue (one thread), D[tmem] (+)= A[smem] * B[smem]
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         bool accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
-        : "memory");
 }
 
 // Arrive on `bar` once every MMA issued so far by this thread has completed.

@@ -184,26 +184,38 @@ class Wkv4Inputs:
     dy: np.ndarray | None = None  # [B,T,C] float32 upstream gradient
 
 
+def _batch_window(B: int, batches, T: int, C: int):
+    """(first batch, number of batches, flat offset) of the window `batches` = (lo, hi)
+    of a B-batch problem (None: all of it)."""
+    lo, hi = (0, B) if batches is None else batches
+    if not 0 <= lo <= hi <= B:
+        raise ValueError(f"batch window {batches} outside [0, {B}]")
+    return lo, hi - lo, lo * T * C
+
+
 def make_wkv6(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, rkv_std: float = 0.5,
               wraw_lo: float = -6.0, wraw_hi: float = -0.5, u_std: float = 0.5,
-              with_dy: bool = False, dy_std: float = 1.0, dtype: str = "f32") -> Wkv6Inputs:
+              with_dy: bool = False, dy_std: float = 1.0, dtype: str = "f32", batches=None) -> Wkv6Inputs:
     """RWKV-6 inputs: r,k,v ~ N(0, rkv_std^2), w_raw ~ U(wraw_lo, wraw_hi) per (t, channel),
-    ew = -exp(w_raw), u ~ N(0, u_std^2) per channel, dy ~ N(0, dy_std^2)."""
+    ew = -exp(w_raw), u ~ N(0, u_std^2) per channel, dy ~ N(0, dy_std^2).
+    batches=(lo, hi): only batches lo..hi-1 of the B-batch problem (bit-identical to the
+    same slice of the whole problem; B of the result is hi - lo)."""
     C = H * N
-    n = B * T * C
-    shape = (B, T, C)
+    _, Bl, off = _batch_window(B, batches, T, C)
+    n = Bl * T * C
+    shape = (Bl, T, C)
 
     def cast(x64: np.ndarray) -> np.ndarray:
         x32 = x64.astype(np.float32).reshape(shape)
         return to_bf16_bits(x32).reshape(shape) if dtype == "bf16" else x32
 
-    r = cast(normal(seed, STREAM_R, n, rkv_std))
-    k = cast(normal(seed, STREAM_K, n, rkv_std))
-    v = cast(normal(seed, STREAM_V, n, rkv_std))
-    w = cast(-np.exp(uniform(seed, STREAM_WRAW, n, wraw_lo, wraw_hi)))
+    r = cast(normal(seed, STREAM_R, n, rkv_std, offset=off))
+    k = cast(normal(seed, STREAM_K, n, rkv_std, offset=off))
+    v = cast(normal(seed, STREAM_V, n, rkv_std, offset=off))
+    w = cast(-np.exp(uniform(seed, STREAM_WRAW, n, wraw_lo, wraw_hi, offset=off)))
     u = normal(seed, STREAM_U, C, u_std).astype(np.float32)
-    dy = normal(seed, STREAM_DY, n, dy_std).astype(np.float32).reshape(shape) if with_dy else None
-    return Wkv6Inputs(B, T, C, H, r, k, v, w, u, dy, dtype)
+    dy = normal(seed, STREAM_DY, n, dy_std, offset=off).astype(np.float32).reshape(shape) if with_dy else None
+    return Wkv6Inputs(Bl, T, C, H, r, k, v, w, u, dy, dtype)
 
 
 def make_wkv5(B: int, T: int, H: int, N: int = 64, *, seed: int = 0, rkv_std: float = 0.5,
@@ -268,22 +280,25 @@ def make_state(B: int, H: int, N: int = 64, *, seed: int = 0, std: float = 1.0) 
 
 def make_wkv4(B: int, T: int, C: int, *, seed: int = 0, kv_std: float = 1.0,
               logw_lo: float = -3.0, logw_hi: float = 1.0, u_std: float = 0.5,
-              with_dy: bool = False, dy_std: float = 1.0) -> Wkv4Inputs:
+              with_dy: bool = False, dy_std: float = 1.0, batches=None) -> Wkv4Inputs:
     """RWKV-4 inputs: k, v ~ N(0, kv_std^2); w = exp(U(logw_lo, logw_hi)) > 0 per channel;
-    u ~ N(0, u_std^2) per channel; dy ~ N(0, dy_std^2)."""
-    n = B * T * C
-    k = normal(seed, STREAM_K, n, kv_std).astype(np.float32).reshape(B, T, C)
-    v = normal(seed, STREAM_V, n, kv_std).astype(np.float32).reshape(B, T, C)
+    u ~ N(0, u_std^2) per channel; dy ~ N(0, dy_std^2).  batches: as make_wkv6."""
+    _, Bl, off = _batch_window(B, batches, T, C)
+    n = Bl * T * C
+    k = normal(seed, STREAM_K, n, kv_std, offset=off).astype(np.float32).reshape(Bl, T, C)
+    v = normal(seed, STREAM_V, n, kv_std, offset=off).astype(np.float32).reshape(Bl, T, C)
     w = np.exp(uniform(seed, STREAM_WRAW, C, logw_lo, logw_hi)).astype(np.float32)
     u = normal(seed, STREAM_U, C, u_std).astype(np.float32)
-    dy = normal(seed, STREAM_DY, n, dy_std).astype(np.float32).reshape(B, T, C) if with_dy else None
-    return Wkv4Inputs(B, T, C, k, v, w, u, dy)
+    dy = normal(seed, STREAM_DY, n, dy_std, offset=off).astype(np.float32).reshape(Bl, T, C) if with_dy else None
+    return Wkv4Inputs(Bl, T, C, k, v, w, u, dy)
 
 
 # The workloads: name -> (kind, constructor kwargs).
 WORKLOADS = {
     # causal RWKV-6 forward, fp32, small (oracle finishes in seconds)
     "wkv6_causal_f32_b1t196h4": ("wkv6_fwd", dict(B=1, T=196, H=4)),
+    # causal RWKV-6 forward, fp32, on the patch-sequence shape of the bidirectional workload
+    "wkv6_causal_f32_b32t196h12": ("wkv6_fwd", dict(B=32, T=196, H=12)),
     # RWKV-4 scalar-state forward, fp32
     "wkv4_f32_b8t1024c768": ("wkv4_fwd", dict(B=8, T=1024, C=768)),
     # bidirectional RWKV-6 forward on 224px/16px patch sequences, fp32
@@ -307,8 +322,17 @@ WORKLOADS = {
 }
 
 
-def make_workload(name: str, seed: int = 0):
+def make_workload(name: str, seed: int = 0, batch_scale: int = 1, batches=None):
+    """The named workload's inputs.  batch_scale: a problem of batch_scale times the
+    workload's batch; batches=(lo, hi): only those batches of it (see make_wkv6)."""
     kind, kw = WORKLOADS[name]
+    kw = dict(kw, B=kw["B"] * batch_scale)
+    if batches is not None:
+        if kind in ("wkv4_fwd", "wkv4_bwd") or kind == "wkv6_fwd" or kind == "wkv6_fwd_bf16" or \
+                kind in ("wkv6_bidir_fwd", "wkv6_bwd_bidir"):
+            kw["batches"] = batches
+        else:
+            raise ValueError(f"{name}: no batch window for this workload kind")
     if kind in ("wkv4_fwd", "wkv4_bwd"):
         return kind, make_wkv4(seed=seed, **kw)
     if kind.startswith("wkv5"):

@@ -17,3 +17,15 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _guard_bands(request):
+    """After every GPU test: the guard bands around each device buffer the test handed
+    the library (tests/gpu_cases.py) must be intact."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    mod = sys.modules.get("tests.gpu_cases")
+    if mod is not None:
+        mod.check_guards()

@@ -1,4 +1,5 @@
-"""Host-side checks of libwkv.so (no GPU needed, no kernel launched).
+"""Host-side checks of libwkv.so and its test build libwkv_recurrence.so (no GPU
+needed, no kernel launched).
 
 The library must load, export every function include/wkv.h declares, and reject
 bad arguments on the host with the documented status codes before touching
@@ -19,11 +20,13 @@ HEADER = os.path.join(ROOT, "include", "wkv.h")
 WKV_OK, WKV_ERR_ARG, WKV_ERR_HEADSIZE, WKV_ERR_ALIGN, WKV_ERR_WORKSPACE = 0, -1, -2, -3, -4
 
 
-@pytest.fixture(scope="module")
-def lib():
+@pytest.fixture(scope="module", params=["default", "recurrence"])
+def lib(request):
+    """Both builds of the library (the product and the test build) carry the same ABI."""
     from linear_attention_rnn_wkv6_b200 import build
     build.build()
-    return wkv.load()
+    with wkv.use_library(request.param) as handle:
+        yield handle
 
 
 def _declared_functions():

@@ -25,9 +25,9 @@ def _cuda():
 
 
 @pytest.fixture(params=["tensor", "recurrence"], autouse=True)
-def bwd_path(request, monkeypatch):
-    monkeypatch.setenv("WKV6_BWD_PATH", request.param)
-    return request.param
+def bwd_path(request):
+    with gc.library_for(request.param):
+        yield request.param
 
 
 def _check(x, bidir, got, dy64, H, path):

@@ -21,11 +21,11 @@ def _cuda():
 
 
 @pytest.fixture(params=["tensor", "recurrence"], autouse=True)
-def f32_path(request, monkeypatch):
+def f32_path(request):
     """Both fp32 forward kernels: the chunked tensor-core one (split-bf16 operands; the norm
-    and gate in its epilogue) and the token-by-token recurrence."""
-    monkeypatch.setenv("WKV6_F32_PATH", request.param)
-    return request.param
+    and gate in its epilogue) and the token-by-token recurrence (the test build)."""
+    with gc.library_for(request.param):
+        yield request.param
 
 
 _NAMES = ("r", "k", "v", "ww", "w_base", "u", "g", "gn_w", "gn_b")

@@ -1,9 +1,8 @@
 """Parity of the CUDA path (called through the C ABI) with the fp64 oracle.
 
-Small problems are compared element by element over the whole tensor; the
-five full-size workloads run in the launch configuration the benchmark times
-and are compared on sampled (b, h) units (every unit of a WKV6 problem is an
-independent problem) plus properties that hold at any size.
+Small problems and the full-size workloads (in the launch configuration the
+benchmark times) are compared element by element over the whole tensor; the
+oracle runs one batch per host thread for the large ones.
 """
 import numpy as np
 import pytest
@@ -33,11 +32,12 @@ F32_PATHS = ["tensor", "recurrence"]
 
 
 @pytest.fixture(params=F32_PATHS)
-def f32_path(request, monkeypatch):
+def f32_path(request):
     """Run the fp32 forward (causal and bidirectional) through the chunked
-    tensor-core kernel with split-bf16 operands or the token-by-token recurrence."""
-    monkeypatch.setenv("WKV6_F32_PATH", request.param)
-    return request.param
+    tensor-core kernel with split-bf16 operands (libwkv.so) or the token-by-token
+    recurrence (the test build libwkv_recurrence.so)."""
+    with gc.library_for(request.param):
+        yield request.param
 
 
 FWD_SHAPES = [  # (B, T, H): several 32-token chunks, ragged tails, T < chunk, single token
@@ -60,11 +60,11 @@ BF16_PATHS = ["tensor", "recurrence"]
 
 
 @pytest.fixture(params=BF16_PATHS)
-def bf16_path(request, monkeypatch):
+def bf16_path(request):
     """Run the bf16 causal forward through the chunked tensor-core kernel or the
-    token-by-token recurrence kernel."""
-    monkeypatch.setenv("WKV6_BF16_PATH", request.param)
-    return request.param
+    token-by-token recurrence kernel (the test build)."""
+    with gc.library_for(request.param):
+        yield request.param
 
 
 def _bf16_bound(path):
@@ -167,11 +167,11 @@ def test_wkv6_fwd_slices_match_single_head_calls(f32_path):
 # ------------------------------------------------------------------ backward, small and ragged
 
 @pytest.fixture(params=["tensor", "recurrence"])
-def bwd_path(request, monkeypatch):
+def bwd_path(request):
     """Run the fp32 backward through the chunked tensor-core kernels (split-bf16
-    operands) or the two-sweep recurrence kernel."""
-    monkeypatch.setenv("WKV6_BWD_PATH", request.param)
-    return request.param
+    operands) or the two-sweep recurrence kernel (the test build)."""
+    with gc.library_for(request.param):
+        yield request.param
 
 
 @pytest.mark.parametrize("B,T,H", [(1, 1, 1), (1, 2, 1), (2, 15, 2), (1, 16, 1), (2, 17, 1), (1, 32, 1), (1, 33, 2),
@@ -250,50 +250,28 @@ def test_workload_wkv4_full_tensor():
     assert _rel(y, oracle.wkv4_fwd(x.k, x.v, x.w, x.u)) <= gc.TOL_F32_FWD
 
 
-def _sampled_fwd(x, bidir, n_units, tol):
-    y = gc.run_wkv6_fwd(x, bidir=bidir)
-    assert np.all(np.isfinite(y))
-    got, ref = [], []
-    for b, h in gc.sample_units(x.B, x.H, n_units):
-        (r, k, v, w, u), _, sl = gc.unit_slice(x, b, h)
-        ref.append(oracle.wkv6_fwd(r, k, v, w, u, H=1, bidirectional=bidir)[0])
-        got.append(y[b, :, sl])
-    err = _rel(np.stack(got), np.stack(ref))
-    assert err <= tol, err
-    return err
-
-
-def test_workload_bidir_f32_sampled(f32_path):
+def test_workload_bidir_f32_full_tensor(f32_path):
     kind, x = synth.make_workload("wkv6_bidir_f32_b32t196h12")
-    _sampled_fwd(x, True, 48, gc.TOL_F32_FWD)
+    y = gc.run_wkv6_fwd(x, bidir=True)
+    assert np.all(np.isfinite(y))
+    err = _rel(y, gc.oracle_fwd_full(x, True))
+    assert err <= gc.TOL_F32_FWD, err
 
 
-def test_workload_causal_bf16_long_sampled(bf16_path):
+def test_workload_causal_bf16_long_full_tensor(bf16_path):
     kind, x = synth.make_workload("wkv6_causal_bf16_b8t4096h32")
-    err = _sampled_fwd(x, False, 12, gc.TOL_BF16_FWD)
+    y = gc.run_wkv6_fwd(x)
+    assert np.all(np.isfinite(y))
+    err = _rel(y, gc.oracle_fwd_full(x, False))
+    assert err <= gc.TOL_BF16_FWD, err
     assert err <= _bf16_bound(bf16_path), err
 
 
-def test_workload_bidir_bwd_sampled(bwd_path):
+def test_workload_bidir_bwd_full_tensor(bwd_path):
     kind, x = synth.make_workload("wkv6_bidir_bwd_f32_b32t196h12")
-    dr, dk, dv, dw, du = gc.run_wkv6_bwd(x, True)
-    units = gc.sample_units(x.B, x.H, 24)
-    got = {n: [] for n in ("dr", "dk", "dv", "dw")}
-    ref = {n: [] for n in ("dr", "dk", "dv", "dw")}
-    for b, h in units:
-        (r, k, v, w, u), dy, sl = gc.unit_slice(x, b, h)
-        e = oracle.wkv6_bwd(r, k, v, w, u, dy, H=1, bidirectional=True)
-        for n, gg, ee in zip(("dr", "dk", "dv", "dw"), (dr, dk, dv, dw), e[:4]):
-            got[n].append(gg[b, :, sl])
-            ref[n].append(ee[0])
-    for n in got:
-        err = _rel(np.stack(got[n]), np.stack(ref[n]))
+    got = gc.run_wkv6_bwd(x, True)
+    ref = gc.oracle_bwd_full(x, True)
+    for n, g, e in zip(("dr", "dk", "dv", "dw", "du"), got, ref):
+        assert np.all(np.isfinite(g)), n
+        err = _rel(g, e)
         assert err <= gc.TOL_F32_GRAD, (n, err)
-    # du sums over the whole batch: check every channel of the heads sampled, exactly defined
-    for h in sorted({h for _, h in units})[:3]:
-        sl = slice(64 * h, 64 * h + 64)
-        acc = np.zeros(64)
-        for b in range(x.B):
-            (r, k, v, w, u), dy, _ = gc.unit_slice(x, b, h)
-            acc += oracle.wkv6_bwd(r, k, v, w, u, dy, H=1, bidirectional=True)[4]
-        assert _rel(du[sl], acc) <= gc.TOL_F32_GRAD

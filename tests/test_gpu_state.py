@@ -60,14 +60,13 @@ def test_fwd_state_matches_oracle(B, T, H, with_s0):
     assert _rel(sT, so) <= gc.TOL_F32_FWD, _rel(sT, so)
 
 
-def test_fwd_state_without_s0_equals_plain_forward(monkeypatch):
+def test_fwd_state_without_s0_equals_plain_forward():
     """No initial state is the zero state: bit-identical to the plain forward on the
     same (recurrence) kernel, and within the fp32 tolerance of the tensor-core path."""
     x = synth.make_wkv6(2, 150, 3, seed=310)
     y, _ = _run_state(x, None)
-    monkeypatch.setenv("WKV6_F32_PATH", "recurrence")
-    assert np.array_equal(y, gc.run_wkv6_fwd(x))
-    monkeypatch.setenv("WKV6_F32_PATH", "tensor")
+    with gc.library_for("recurrence"):
+        assert np.array_equal(y, gc.run_wkv6_fwd(x))
     assert _rel(y, gc.run_wkv6_fwd(x)) <= gc.TOL_F32_FWD
 
 

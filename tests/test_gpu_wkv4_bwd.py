@@ -30,7 +30,7 @@ def _run(x, dy):
     dk, dv = gc.empty_nan((x.B, x.T, x.C)), gc.empty_nan((x.B, x.T, x.C))
     dw, du = gc.empty_nan((x.C,)), gc.empty_nan((x.C,))
     nb = wkv.wkv4_bwd_workspace_bytes(x.B, x.T, x.C)
-    ws = t.empty(max(nb, 16), dtype=t.uint8, device="cuda")
+    ws = gc.workspace(nb)
     wkv.wkv4_bwd(x.B, x.T, x.C, k, v, w, u, g, dk, dv, dw, du, ws, nb)
     assert wkv.wkv_take_device_faults() == 0
     return tuple(a.cpu().numpy() for a in (dk, dv, dw, du))

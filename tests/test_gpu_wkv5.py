@@ -37,7 +37,7 @@ def _bwd(x):
     r, k, v, w, u, dy = (gc.dev(getattr(x, n)) for n in ("r", "k", "v", "w", "u", "dy"))
     outs = [gc.empty_nan((x.B, x.T, x.C)) for _ in range(3)] + [gc.empty_nan((x.C,)) for _ in range(2)]
     nb = wkv.wkv5_bwd_workspace_bytes(x.B, x.T, x.C, x.H)
-    ws = t.empty(max(nb, 16), dtype=t.uint8, device="cuda")
+    ws = gc.workspace(nb)
     wkv.wkv5_bwd(x.B, x.T, x.C, x.H, r, k, v, w, u, dy, *outs, ws, nb)
     assert wkv.wkv_take_device_faults() == 0
     return tuple(o.cpu().numpy() for o in outs)
@@ -63,10 +63,11 @@ def test_wkv5_fwd_strong_and_zero_decay():
 
 
 @pytest.fixture(params=["tensor_cores", "recurrence"])
-def bf16_path(request, monkeypatch):
-    """Both bf16 algorithms: the chunked tensor-core kernel (default) and the recurrence."""
-    monkeypatch.setenv("WKV6_BF16_PATH", request.param)
-    return request.param
+def bf16_path(request):
+    """Both bf16 algorithms: the chunked tensor-core kernel (default) and the recurrence
+    (the test build)."""
+    with gc.library_for(request.param):
+        yield request.param
 
 
 @pytest.mark.parametrize("B,T,H", [(1, 5, 1), (2, 150, 2), (1, 1000, 3)])
