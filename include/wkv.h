@@ -30,7 +30,12 @@
  * wkv6_fwd_fused, wkv5_fwd_bf16, wkv6_bwd, wkv6_bwd_bf16 and wkv5_bwd run the
  * token-by-token recurrence kernels instead (the kernels wkv6_fwd_state,
  * wkv5_fwd and wkv6_bwd_noalloc use in both builds).  Results agree within the
- * tolerances stated below; nothing is selected at run time.
+ * tolerances stated below; nothing is selected at run time.  A third build,
+ * libwkv_debug.so (-DWKV_DEVICE_CHECKS=1), is libwkv.so with an index check on
+ * every global store of every kernel: an index outside the array skips the store
+ * and records WKV_FAULT_INDEX (nothing traps), and every entry point then waits
+ * for its kernels and returns WKV_ERR_DEVICE_CHECK (or WKV_ERR_TIMEOUT for a
+ * bounded wait that ran out) instead of WKV_OK.
  *
  * RWKV-6 log-decay
  * ----------------
@@ -62,11 +67,14 @@ enum {
     WKV_ERR_WORKSPACE = -4,  /* workspace NULL or smaller than the *_workspace_bytes query */
     WKV_ERR_CUDA = -5,       /* a CUDA runtime call or the launch failed */
     WKV_ERR_DEVICE = -6,     /* the current device is not sm_100 (B200) */
-    WKV_ERR_TOO_LARGE = -7   /* a size exceeds a documented limit (B*T*C >= 2^31 elements) */
+    WKV_ERR_TOO_LARGE = -7,  /* a size exceeds a documented limit (B*T*C >= 2^31 elements) */
+    WKV_ERR_DEVICE_CHECK = -8, /* debug build: a kernel's index check failed (WKV_FAULT_INDEX) */
+    WKV_ERR_TIMEOUT = -9     /* debug build: a kernel's bounded wait ran out (WKV_FAULT_TIMEOUT) */
 };
 
 /* Bits of the device fault word (see wkv_take_device_faults). */
 #define WKV_FAULT_TIMEOUT 0x1u   /* a bounded device-side wait ran out */
+#define WKV_FAULT_INDEX 0x2u     /* debug build: a kernel's store index was out of range (store skipped) */
 
 /*
  * wkv6_fwd -- causal RWKV-6 WKV forward, fp32 inputs, fp32 state and output.
@@ -341,6 +349,16 @@ int wkv_version(void);
  * health checks only.  Returns WKV_OK, WKV_ERR_DEVICE or WKV_ERR_CUDA.
  */
 int wkv_selftest_wait_timeout(wkv_stream_t stream);
+
+/*
+ * wkv_selftest_index_check -- exercise the failure path of the kernels' index
+ * checks.  Launches one thread that attempts a store whose index equals the size
+ * of the array it targets; the check skips the store, records WKV_FAULT_INDEX in
+ * the device fault word and the kernel returns.  The product build returns WKV_OK
+ * (read the bit with wkv_take_device_faults); the debug build, which waits for
+ * its kernels, returns WKV_ERR_DEVICE_CHECK and clears the bit.  For tests only.
+ */
+int wkv_selftest_index_check(wkv_stream_t stream);
 
 #ifdef __cplusplus
 }

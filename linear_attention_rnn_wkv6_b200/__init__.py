@@ -21,15 +21,17 @@ __all__ = [
     "wkv6_bwd_workspace_bytes", "wkv4_fwd", "wkv_status_string", "wkv_take_device_faults", "wkv_version",
     "wkv6_bwd_noalloc", "wkv6_fwd_state", "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes",
     "wkv5_fwd", "wkv5_fwd_bf16", "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused",
-    "wkv_selftest_wait_timeout", "WKV_FAULT_TIMEOUT", "EXPORTED_SYMBOLS",
+    "wkv_selftest_wait_timeout", "wkv_selftest_index_check", "WKV_FAULT_TIMEOUT", "WKV_FAULT_INDEX",
+    "EXPORTED_SYMBOLS",
     "HEAD_SIZE", "LIBRARY_FILES", "use_library",
 ]
 
 HEAD_SIZE = 64
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# The two builds of the library (same C ABI): the product, and the test build whose
-# chunked-form entry points run the token-by-token recurrence kernels.
-LIBRARY_FILES = {"default": "libwkv.so", "recurrence": "libwkv_recurrence.so"}
+# The builds of the library (same C ABI): the product, the test build whose
+# chunked-form entry points run the token-by-token recurrence kernels, and the debug
+# build that checks every store index of every kernel.
+LIBRARY_FILES = {"default": "libwkv.so", "recurrence": "libwkv_recurrence.so", "debug": "libwkv_debug.so"}
 _LIBS: dict = {}
 _ACTIVE = ["default"]
 
@@ -39,8 +41,10 @@ EXPORTED_SYMBOLS = (
     "wkv_status_string", "wkv_take_device_faults", "wkv_version", "wkv6_bwd_noalloc", "wkv6_fwd_state",
     "wkv6_decode", "wkv6_bwd_bf16", "wkv4_bwd", "wkv4_bwd_workspace_bytes", "wkv5_fwd", "wkv5_fwd_bf16",
     "wkv5_bwd", "wkv5_bwd_workspace_bytes", "wkv6_fwd_fused", "wkv_selftest_wait_timeout",
+    "wkv_selftest_index_check",
 )
 WKV_FAULT_TIMEOUT = 0x1   # fault-word bit: a bounded device-side wait ran out
+WKV_FAULT_INDEX = 0x2     # fault-word bit: a kernel's store index was out of range (debug build)
 
 _I = ctypes.c_int
 _P = ctypes.c_void_p
@@ -57,6 +61,7 @@ _SIGS = {
     "wkv_take_device_faults": ([ctypes.POINTER(ctypes.c_uint)], _I),
     "wkv_version": ([], _I),
     "wkv_selftest_wait_timeout": ([_P], _I),
+    "wkv_selftest_index_check": ([_P], _I),
     "wkv6_bwd_noalloc": ([_I] * 5 + [_P] * 11 + [_P], _I),
     "wkv6_fwd_state": ([_I] * 4 + [_P] * 8 + [_P], _I),
     "wkv6_decode": ([_I] * 3 + [_P] * 7 + [_P], _I),
@@ -260,6 +265,13 @@ def wkv_selftest_wait_timeout(stream=None) -> None:
     """Launch the one-CTA kernel whose bounded wait runs out (about a second); the fault
     word then holds WKV_FAULT_TIMEOUT (read it with wkv_take_device_faults)."""
     _check("wkv_selftest_wait_timeout", load().wkv_selftest_wait_timeout(_stream(stream)))
+
+
+def wkv_selftest_index_check(stream=None) -> None:
+    """Launch the one-thread kernel whose store index equals its array's size: the check
+    skips the store and records WKV_FAULT_INDEX (the debug build raises WkvError with
+    WKV_ERR_DEVICE_CHECK, having waited for the kernel)."""
+    _check("wkv_selftest_index_check", load().wkv_selftest_index_check(_stream(stream)))
 
 
 def wkv_version() -> int:

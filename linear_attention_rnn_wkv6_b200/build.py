@@ -11,6 +11,10 @@ Variants (each a complete library with the same C ABI, include/wkv.h):
                                       the token-by-token recurrence kernels instead;
                                       for testing those kernels and timing the chunked
                                       forms against them
+  debug       libwkv_debug.so      -- built with -DWKV_DEVICE_CHECKS=1: the product
+                                      with an index check on every global store of
+                                      every kernel, and entry points that wait for
+                                      their kernels and report a failed check
 
 The libraries are written next to this file so that they travel with the source
 tree; the Python binding loads them from there.  Each .cu file is compiled to an
@@ -36,6 +40,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 VARIANTS = {
     "default": ("libwkv.so", []),
     "recurrence": ("libwkv_recurrence.so", ["-DWKV_RECURRENCE_PATHS=1"]),
+    "debug": ("libwkv_debug.so", ["-DWKV_DEVICE_CHECKS=1"]),
 }
 LIB = os.path.join(HERE, VARIANTS["default"][0])
 
@@ -95,8 +100,8 @@ def _build_variant(variant: str, verbose: bool) -> str:
     return out
 
 
-def build(force: bool = False, verbose: bool = False, variants=("default", "recurrence")) -> str:
-    """Build the requested variants (both by default) if their sources changed.
+def build(force: bool = False, verbose: bool = False, variants=("default", "recurrence", "debug")) -> str:
+    """Build the requested variants (all by default) if their sources changed.
     Returns the path of the default library."""
     todo = [v for v in variants if force or _stale(lib_file(v))]
     if todo:
@@ -111,7 +116,7 @@ def main() -> None:
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--variant", action="append", choices=sorted(VARIANTS))
     a = ap.parse_args()
-    variants = a.variant or ["default", "recurrence"]
+    variants = a.variant or ["default", "recurrence", "debug"]
     build(force=a.force, verbose=a.verbose, variants=variants)
     for v in variants:
         print(lib_file(v))

@@ -131,6 +131,7 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
     st = in;
     if (live)
         for (int t = t0, o = t0 * C + c; t < t1; ++t, o += C) {
+            if (!in_range((size_t)o, (size_t)T * C)) continue;   // y, g, m parked in this row of dv, dk, mwork
             const float k2 = kr[o] * kLog2e, vt = vr[o];
             const float uk = u2 + k2, d = st.p - uk;
             const float ex = ex2(-fabsf(d));
@@ -163,6 +164,7 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
     float dwa = 0.f, dua = 0.f;
     if (live)
         for (int t = t1 - 1, o = (t1 - 1) * C + c; t >= t0; --t, o -= C) {
+            if (!in_range((size_t)o, (size_t)T * C)) continue;   // dk, dv: this batch row
             const float gh = dkr[o], yt = dvr[o], m = mr[o];
             const float k2 = kr[o] * kLog2e, vt = vr[o];
             const float E = ex2(k2 + ri.q);            // e^{k_s} 2^q
@@ -185,8 +187,10 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
             sw += red[0][j][ch];
             su += red[1][j][ch];
         }
-        dw_part[(size_t)b * C + c] = sw;
-        du_part[(size_t)b * C + c] = su;
+        if (in_range((size_t)b * C + c, (size_t)(gridDim.x / groups) * C)) {
+            dw_part[(size_t)b * C + c] = sw;
+            du_part[(size_t)b * C + c] = su;
+        }
     }
 }
 

@@ -19,7 +19,7 @@ namespace {
 __global__ void wkv5_expand_kernel(size_t n4, int C4, const float4 *__restrict__ w, float4 *__restrict__ ew) {
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n4; e += (size_t)gridDim.x * blockDim.x) {
         const float4 x = w[e % C4];
-        ew[e] = make_float4(-x.x, -x.y, -x.z, -x.w);
+        if (in_range(e, n4)) ew[e] = make_float4(-x.x, -x.y, -x.z, -x.w);
     }
 }
 
@@ -46,7 +46,7 @@ __global__ void wkv5_dw_partial_kernel(int rows, int blk, int C, const float *__
         float s = 0.f;
 #pragma unroll
         for (int g = 0; g < 8; ++g) s += grp[g][threadIdx.x];
-        part[(size_t)blockIdx.y * C + c] = s;
+        if (in_range((size_t)blockIdx.y * C + c, (size_t)gridDim.y * C)) part[(size_t)blockIdx.y * C + c] = s;
     }
 }
 

@@ -391,6 +391,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
             const int t = dir > 0 ? tl + p : tl + TC - 1 - p;
             if (t < 0 || t >= T) continue;
             const size_t o = ((size_t)b * T + t) * C + cbase + i;
+            if (!in_range(o, (size_t)prm.B * T * C)) continue;   // dr, dk, dv, dw: [B][T][C]
             const float A = sm.Ap[p][i];
             const float drs = hasS ? A * (sm.pr[p][0][i] + sm.pr[p][1][i] + sm.pr[p][2][i] + sm.pr[p][3][i]) : 0.f;
             const float dks = hasG ? A * (sm.pk[p][0][i] + sm.pk[p][1][i] + sm.pk[p][2][i] + sm.pk[p][3][i]) : 0.f;
@@ -431,7 +432,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                     const size_t o = ((size_t)b * T + t) * C + cbase + tid;
                     const float x = sm.pr[p][0][tid];
                     const float z = sm.part[s][3][TC - 1 - p][tid];
-                    prm.dw[o] = Rrun - x;
+                    if (in_range(o, (size_t)prm.B * T * C)) prm.dw[o] = Rrun - x;
                     Rrun += z - x;
                 }
             }
@@ -444,7 +445,8 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         }
         if (tid == 0 && g + 1 >= nch && g + 1 < nchunks) issue_part(g + 1);
     }
-    if (tid < kHead) prm.du_part[(size_t)b * C + cbase + tid] = du_acc;
+    if (tid < kHead && in_range((size_t)b * C + cbase + tid, (size_t)prm.B * C))
+        prm.du_part[(size_t)b * C + cbase + tid] = du_acc;
 }
 
 // du[c] = sum_b du_part[b][c], in increasing b (deterministic).

@@ -111,15 +111,18 @@ __device__ __forceinline__ uint64_t desc_cm(const __nv_bfloat16 *tile) { return 
 
 // One chunk of a dw scan, on all 128 threads: channel tid % 64, half tid / 64 of the
 // chunk (`order` 0: positions 0..15 come first in scan order, 1: 16..31 first).
-// part(p, i) is the token's z or x value; each thread adds its running sum (the
-// carry `run` from earlier chunks, the earlier half's total, its own prefix) times
-// `sign` to `base(p, i)` (`base_load`: the value in dw, else 0) and stores dw; `run`
-// ends as the carry after the chunk in every thread.  `xch` is 2 x 64 floats of
-// shared memory.  Loads of a thread's 16 tokens are issued before its stores.
-template <typename PartF, typename AddrF>
+// part(p, i) is the token's scanned value; each thread stores
+//     base + extra(p) + sign * (running sum up to and including the token)
+// (`base`: the value in dw when `base_load`, else 0; the running sum is the carry
+// `run` from earlier chunks, the earlier half's total and the thread's own prefix),
+// or base + extra(p) alone where head(p) holds (the sequence's first token, whose
+// decay gradient takes the prefix form).  `run` ends as the carry after the chunk
+// in every thread.  `xch` is 2 x 64 floats of shared memory.  Loads of a thread's
+// 16 tokens are issued before its stores.
+template <typename PartF, typename ExtraF, typename HeadF, typename AddrF>
 __device__ __forceinline__ void dw_scan_chunk(int tid, int c, int T, int order, bool base_load, float sign,
-                                              float extra, float &run, float *xch, float *dw, PartF part,
-                                              AddrF addr) {
+                                              ExtraF extra, HeadF head, float &run, float *xch, float *dw,
+                                              size_t n, PartF part, AddrF addr) {
     const int i = tid & (kHead - 1), h = tid >> 6;
     const int p0 = 16 * h;
     const bool first_half = (order == 0) == (h == 0);   // this half comes first in scan order
@@ -127,7 +130,7 @@ __device__ __forceinline__ void dw_scan_chunk(int tid, int c, int T, int order, 
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const int p = p0 + e;
-        prev[e] = (base_load && c * kBL + p < T) ? dw[addr(p)] : 0.f;
+        prev[e] = (base_load && c * kBL + p < T && in_range(addr(p), n)) ? dw[addr(p)] : 0.f;
     }
     float acc = 0.f;
     if (order == 0) {
@@ -152,7 +155,8 @@ __device__ __forceinline__ void dw_scan_chunk(int tid, int c, int T, int order, 
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const int p = p0 + e;
-        if (c * kBL + p < T) dw[addr(p)] = prev[e] + extra + sign * (carry + loc[e]);
+        if (c * kBL + p < T && in_range(addr(p), n))
+            dw[addr(p)] = prev[e] + extra(p, i) + (head(p) ? 0.f : sign * (carry + loc[e]));
     }
     run += acc + other;
     __syncthreads();   // xch is free again
@@ -248,6 +252,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
     const int h = blockIdx.x % H, b = blockIdx.x / H;
     const int cbase = h * kHead;
     const int nch = (T + kBL - 1) / kBL;
+    const size_t nBTC = (size_t)prm.B * T * C;   // elements of a [B][T][C] array (store checks)
     const int ch = 2 * lane, pq = 8 * warp;
     const int q4 = lane & 3;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
@@ -322,8 +327,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
             // ================= transform =================
             float s0, s1, a0, a1;
             decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
-            // v.dy per token (the bonus scalar of dr, dk and du), reduced over the 64 channels
-            if (causal) {
+            // v.dy per token (the bonus scalar of dr, dk and du), reduced over the 64 channels;
+            // the anti-causal pass needs it too, to take dr's causal part back out of dr
+            if (causal || BIDIR) {
                 float pv[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) pv[e] = fmaf(xv_[e].x, xd_[e].x, xv_[e].y * xd_[e].y);
@@ -333,17 +339,20 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
             __syncthreads();
             float L0, L1, tot0, tot1;
             const bool exact = decay_prefix(ds, warp, ch, L0, L1, tot0, tot1);
-            if (causal) {
-                // the bonus part of dr (added by the epilogue, whose store is then plain) and
-                // the du partial sums; dk's and dv's bonus parts are the G kind's
+            if (causal || BIDIR) {
+                // the bonus part of dr (added by the causal epilogue, whose store is then
+                // plain; taken back out by the anti-causal one) and, causal pass, the du
+                // partial sums; dk's and dv's bonus parts are the G kind's
                 const float u0 = sm.u[ch], u1 = sm.u[ch + 1];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int p = pq + e;
                     const float vd = c * kBL + p < T ? sm.vdy[p] : 0.f;
                     *reinterpret_cast<float2 *>(&sm.BR[fidx(p, ch)]) = make_float2(u0 * xk_[e].x * vd, u1 * xk_[e].y * vd);
-                    du0 = fmaf(xr_[e].x * xk_[e].x, vd, du0);
-                    du1 = fmaf(xr_[e].y * xk_[e].y, vd, du1);
+                    if (causal) {
+                        du0 = fmaf(xr_[e].x * xk_[e].x, vd, du0);
+                        du1 = fmaf(xr_[e].y * xk_[e].y, vd, du1);
+                    }
                 }
             }
             // raw r for the dw parts (both paths)
@@ -458,7 +467,8 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
                         const int p = 16 * warp + (lane >> 2) + 8 * hr;
-                        const bool valid = c * kBL + p < T;
+                        const bool valid = c * kBL + p < T &&   // the head's 64 channels of the token
+                                           in_range_vec(((size_t)b * T + time_of(dir, c, p)) * C + cbase, kHead, nBTC);
                         float2 *dst = reinterpret_cast<float2 *>(
                             prm.dr + ((size_t)b * T + (valid ? time_of(dir, c, p) : 0)) * C + cbase + 2 * q4);
                         // causal pass: dr = bonus + dr' (plain store); anti-causal: dr += dr'
@@ -474,8 +484,18 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
                             const float2 r2 = *reinterpret_cast<const float2 *>(&sm.R[fidx(p, i)]);
                             const float d0 = e2.x * qv[4 * m + 2 * hr], d1 = e2.y * qv[4 * m + 2 * hr + 1];
                             if (valid) dst[4 * m] = make_float2(prev[m].x + d0, prev[m].y + d1);
-                            // the dw part of this token: z = r dr' (causal), x = r dr' (anti-causal)
-                            *reinterpret_cast<float2 *>(&sm.E[fidx(p, i)]) = make_float2(r2.x * d0, r2.y * d1);
+                            if (BIDIR && !causal) {
+                                // this token's dw terms: z = r dr'_causal (dr minus its bonus
+                                // part, as the causal pass stored it) and x = r dr'_anti; the
+                                // scan takes z - x and the per-token -z
+                                const float2 b2 = *reinterpret_cast<const float2 *>(&sm.BR[fidx(p, i)]);
+                                const float z0 = r2.x * (prev[m].x - b2.x), z1 = r2.y * (prev[m].y - b2.y);
+                                *reinterpret_cast<float2 *>(&sm.E[fidx(p, i)]) = make_float2(z0 - r2.x * d0, z1 - r2.y * d1);
+                                *reinterpret_cast<float2 *>(&sm.R[fidx(p, i)]) = make_float2(z0, z1);
+                            } else {
+                                // the dw part of this token: z = r dr' (causal pass)
+                                *reinterpret_cast<float2 *>(&sm.E[fidx(p, i)]) = make_float2(r2.x * d0, r2.y * d1);
+                            }
                         }
                     }
                 }
@@ -532,8 +552,17 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
                     tmem_wait_st();
                     if (rl) {
                         const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + i;
-                        prm.dr[o] = acc + (causal ? sm.BR[fidx(p, i)] : prm.dr[o]);
-                        sm.E[fidx(p, i)] = sm.R[fidx(p, i)] * acc;
+                        const bool ok = in_range(o, nBTC);
+                        const float old = causal ? sm.BR[fidx(p, i)] : (ok ? prm.dr[o] : 0.f);
+                        if (ok) prm.dr[o] = acc + old;
+                        const float rr = sm.R[fidx(p, i)];
+                        if (BIDIR && !causal) {   // z - x and z, as in the epilogue above
+                            const float z = rr * (old - sm.BR[fidx(p, i)]);
+                            sm.E[fidx(p, i)] = z - rr * acc;
+                            sm.R[fidx(p, i)] = z;
+                        } else {
+                            sm.E[fidx(p, i)] = rr * acc;
+                        }
                     }
                 }
                 __syncthreads();   // every row owner is done with the dy tile (in S_in[0])
@@ -554,23 +583,34 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
                     }
                 }
             }
-            // ===== dw part: causal pass dw = -(running prefix of z); anti-causal dw -= running suffix of x =====
+            // ===== dw part.  Causal only: dw = -(running prefix of z), the G kind adds the
+            // rest.  Bidirectional: nothing in the causal pass; the anti-causal pass (backward
+            // in time) stores this kind's share sum_{t>m} z_t - sum_{t>=m} x_t as the running
+            // suffix of z - x minus z_m, or -z_m (the prefix form) at the first token =====
             __syncthreads();
-            dw_scan_chunk(tid, c, T, 0, !causal, -1.f, 0.f, zrun, sm.xch, prm.dw,
-                          [&](int p, int i) { return sm.E[fidx(p, i)]; },
-                          [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
+            if (!BIDIR) {
+                dw_scan_chunk(tid, c, T, 0, false, -1.f, [](int, int) { return 0.f; }, [](int) { return false; }, zrun,
+                              sm.xch, prm.dw, nBTC, [&](int p, int i) { return sm.E[fidx(p, i)]; },
+                              [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
+            } else if (!causal) {
+                dw_scan_chunk(tid, c, T, 0, false, 1.f, [&](int p, int i) { return -sm.R[fidx(p, i)]; },
+                              [&](int p) { return time_of(dir, c, p) == 0; }, zrun, sm.xch, prm.dw, nBTC,
+                              [&](int p, int i) { return sm.E[fidx(p, i)]; },
+                              [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
+            }
             fence_proxy_async_smem();
             fence_before_sync();
             __syncthreads();
             fence_after_sync();
         }
-        if (causal && tid < kHead) ztot[(size_t)b * C + cbase + tid] = zrun;   // z total of the S kind
+        if (!BIDIR && tid < kHead && in_range((size_t)b * C + cbase + tid, (size_t)prm.B * C))
+            ztot[(size_t)b * C + cbase + tid] = zrun;   // z total of the S kind
         zrun = 0.f;
     }
     // du partial of this (b, h): reduce the four token quarters
     *reinterpret_cast<float2 *>(&sm.dusum[warp][ch]) = make_float2(du0, du1);
     __syncthreads();
-    if (tid < kHead)
+    if (tid < kHead && in_range((size_t)b * C + cbase + tid, (size_t)prm.B * C))
         prm.du_part[(size_t)b * C + cbase + tid] = sm.dusum[0][tid] + sm.dusum[1][tid] + sm.dusum[2][tid] + sm.dusum[3][tid];
     if (!ok && (tid == 0 || tid == 32)) {
         mma_commit(&sm.bar_fin);
@@ -633,6 +673,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
     const int h = blockIdx.x % H, b = blockIdx.x / H;
     const int cbase = h * kHead;
     const int nch = (T + kBL - 1) / kBL;
+    const size_t nBTC = (size_t)prm.B * T * C;   // elements of a [B][T][C] array (store checks)
     const int ch = 2 * lane, pq = 8 * warp;
     const int q4 = lane & 3;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
@@ -686,8 +727,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
 
     uint32_t ph = 0;
     bool ok = true;
-    float zrun = 0.f;     // channel tid % 64: running prefix of z (anti-causal pass), then suffix of x (causal)
-    float zg_tot = 0.f;   // channel tid % 64: z total of the anti-causal pass
+    float zrun = 0.f;     // channel tid % 64: the running suffix of the dw scan (causal pass)
     constexpr int npass = BIDIR ? 2 : 1;
     load_chunk(BIDIR ? -1 : 1, nch - 1);
 
@@ -730,8 +770,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
             __syncthreads();
             float L0, L1, tot0, tot1;
             const bool exact = decay_prefix(ds, warp, ch, L0, L1, tot0, tot1);
-            if (pass == 0) {
-                // the bonus part of dk, added by the first pass's plain store
+            if (pass == 0 || BIDIR) {
+                // the bonus part of dk, added by the first pass's plain store (and taken back
+                // out by the second, bidirectional)
                 const float u0 = prm.u[cbase + ch], u1 = prm.u[cbase + ch + 1];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -887,7 +928,8 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
                         const int s_ = 16 * warp + (lane >> 2) + 8 * hr;
-                        const bool valid = c * kBL + s_ < T;
+                        const bool valid = c * kBL + s_ < T &&   // the head's 64 channels of the token
+                                           in_range_vec(((size_t)b * T + time_of(dir, c, s_)) * C + cbase, kHead, nBTC);
                         float2 *dst = reinterpret_cast<float2 *>(
                             prm.dk + ((size_t)b * T + (valid ? time_of(dir, c, s_) : 0)) * C + cbase + 2 * q4);
                         float2 prev[8];
@@ -903,8 +945,18 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                             const float g0 = kv[4 * m + 2 * hr], g1 = kv[4 * m + 2 * hr + 1];
                             const float d0 = f2.x * g0, d1 = f2.y * g1;
                             if (valid) dst[4 * m] = make_float2(prev[m].x + d0, prev[m].y + d1);
-                            *reinterpret_cast<float2 *>(&sm.F[fidx(s_, i)]) =
-                                make_float2((bf_lo(kt0) + bf_lo(kt1)) * g0, (bf_hi(kt0) + bf_hi(kt1)) * g1);
+                            const float kt_0 = bf_lo(kt0) + bf_lo(kt1), kt_1 = bf_hi(kt0) + bf_hi(kt1);   // k e^{-Lam_{s+1}}
+                            if (BIDIR && pass > 0) {
+                                // this token's dw terms: z = k dk'_anti (dk minus its bonus part, as
+                                // the first pass stored it; k = Kt / e^{-Lam_{s+1}}) and x = k dk'_causal;
+                                // the scan takes z - x and the per-token -z
+                                const float2 b2 = *reinterpret_cast<const float2 *>(&sm.BK[fidx(s_, i)]);
+                                const float z0 = kt_0 / f2.x * (prev[m].x - b2.x), z1 = kt_1 / f2.y * (prev[m].y - b2.y);
+                                *reinterpret_cast<float2 *>(&sm.F[fidx(s_, i)]) = make_float2(z0 - kt_0 * g0, z1 - kt_1 * g1);
+                                *reinterpret_cast<float2 *>(&sm.BK[fidx(s_, i)]) = make_float2(z0, z1);
+                            } else {
+                                *reinterpret_cast<float2 *>(&sm.F[fidx(s_, i)]) = make_float2(kt_0 * g0, kt_1 * g1);
+                            }
                         }
                     }
                 }
@@ -943,7 +995,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
                         const int s_ = 16 * warp + (lane >> 2) + 8 * hr;
-                        if (c * kBL + s_ >= T) continue;
+                        if (c * kBL + s_ >= T ||
+                            !in_range_vec(((size_t)b * T + time_of(dir, c, s_)) * C + cbase, kHead, nBTC))
+                            continue;
                         float2 *dst = reinterpret_cast<float2 *>(prm.dv + ((size_t)b * T + time_of(dir, c, s_)) * C +
                                                                  cbase + 2 * q4);
                         // first pass: a plain store; second: added
@@ -980,15 +1034,23 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                         }
                     }
                     if (rl) {
-                        prm.dk[o + i] = acc + (pass == 0 ? sm.BK[fidx(p, i)] : prm.dk[o + i]);
-                        sm.F[fidx(p, i)] = kk * acc;
+                        const bool ok = in_range(o + i, nBTC);
+                        const float old = pass == 0 ? sm.BK[fidx(p, i)] : (ok ? prm.dk[o + i] : 0.f);
+                        if (ok) prm.dk[o + i] = acc + old;
+                        if (BIDIR && pass > 0) {   // z - x and z, as in the epilogue above
+                            const float z = kk * (old - sm.BK[fidx(p, i)]);
+                            sm.F[fidx(p, i)] = z - kk * acc;
+                            sm.BK[fidx(p, i)] = z;
+                        } else {
+                            sm.F[fidx(p, i)] = kk * acc;
+                        }
                     }
                     __syncthreads();
                     if (tid < kHead) {
                         // the causal pass adds dv's bonus part (sum r u k) dy
                         float s = dir > 0 ? sm.cb[p] * xe.dy[p][tid] : 0.f;
                         for (int ii = 0; ii < kHead; ++ii) s += part[pidx(ii, tid)];
-                        prm.dv[o + tid] = s + (pass == 0 ? 0.f : prm.dv[o + tid]);
+                        if (in_range(o + tid, nBTC)) prm.dv[o + tid] = s + (pass == 0 ? 0.f : prm.dv[o + tid]);
                     }
                     const float dd = rl ? __expf(xe.ew[p][i]) : 0.f, rr = rl ? xe.r[p][i] : 0.f;
 #pragma unroll 1
@@ -1004,14 +1066,22 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                     __syncthreads();
                 }
             }
-            // ===== dw part: anti-causal pass dw -= running prefix of z (forward in time);
-            // causal pass dw += z totals - running suffix of x (backward in time) =====
+            // ===== dw part (backward in time; the dA'^T tiles are free once dKt has read them:
+            // the scan's exchange buffer).  Causal only: dw += the S kind's z total - running
+            // suffix of x, except at the first token (dw there is the S kind's -z alone).
+            // Bidirectional: nothing in the first pass; the causal pass adds this kind's
+            // share, the running suffix of z - x minus z_m, or -z_m at the first token =====
             __syncthreads();
-            {
-                const float ztot_all = last ? ztot[(size_t)b * C + cbase + (tid & (kHead - 1))] + zg_tot : 0.f;
-                // the dA'^T tiles are free once dKt has read them: the scan's exchange buffer
-                dw_scan_chunk(tid, c, T, 1, true, -1.f, ztot_all, zrun, reinterpret_cast<float *>(&sm.dAp[0][0]), prm.dw,
-                              [&](int p, int i) { return sm.F[fidx(p, i)]; },
+            if (!BIDIR) {
+                const float zt = ztot[(size_t)b * C + cbase + (tid & (kHead - 1))];
+                dw_scan_chunk(tid, c, T, 1, true, -1.f, [&](int p, int) { return time_of(dir, c, p) == 0 ? 0.f : zt; },
+                              [&](int p) { return time_of(dir, c, p) == 0; }, zrun,
+                              reinterpret_cast<float *>(&sm.dAp[0][0]), prm.dw, nBTC, [&](int p, int i) { return sm.F[fidx(p, i)]; },
+                              [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
+            } else if (last) {
+                dw_scan_chunk(tid, c, T, 1, true, 1.f, [&](int p, int i) { return -sm.BK[fidx(p, i)]; },
+                              [&](int p) { return time_of(dir, c, p) == 0; }, zrun,
+                              reinterpret_cast<float *>(&sm.dAp[0][0]), prm.dw, nBTC, [&](int p, int i) { return sm.F[fidx(p, i)]; },
                               [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
             }
             fence_proxy_async_smem();
@@ -1019,7 +1089,6 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
             __syncthreads();
             fence_after_sync();
         }
-        if (!last) zg_tot = zrun;
         zrun = 0.f;
     }
     if (!ok && (tid == 0 || tid == 32)) {

@@ -65,8 +65,10 @@ wkv6_decode_kernel(int H, int C, const float *__restrict__ r, const float *__res
         acc.y = fmaf(ri, sv[e].y, acc.y);
         acc.z = fmaf(ri, sv[e].z, acc.z);
         acc.w = fmaf(ri, sv[e].w, acc.w);
-        S[(size_t)i * kColGroups] = make_float4(fmaf(di, sv[e].x, ki * vj.x), fmaf(di, sv[e].y, ki * vj.y),
-                                                fmaf(di, sv[e].z, ki * vj.z), fmaf(di, sv[e].w, ki * vj.w));
+        const size_t si = (size_t)bh * kHead * kHead + (size_t)i * kHead + 4 * g;   // element index in state
+        if (in_range_vec(si, 4, (size_t)gridDim.x * kHead * kHead))
+            S[(size_t)i * kColGroups] = make_float4(fmaf(di, sv[e].x, ki * vj.x), fmaf(di, sv[e].y, ki * vj.y),
+                                                    fmaf(di, sv[e].z, ki * vj.z), fmaf(di, sv[e].w, ki * vj.w));
     }
     part[q][g] = acc;
     __syncthreads();
@@ -76,7 +78,7 @@ wkv6_decode_kernel(int H, int C, const float *__restrict__ r, const float *__res
         float yj = bonus * vs[tid];
 #pragma unroll
         for (int qq = 0; qq < kRowBlocks; ++qq) yj += pf[qq * kHead + tid];
-        y[io + tid] = yj;
+        if (in_range(io + tid, (size_t)(gridDim.x / H) * C)) y[io + tid] = yj;
     }
 }
 

@@ -431,7 +431,7 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
                 val = make_float4(fmaf(d.x * rstd, gnw.x, gnb.x) * gg.x, fmaf(d.y * rstd, gnw.y, gnb.y) * gg.y,
                                   fmaf(d.z * rstd, gnw.z, gnb.z) * gg.z, fmaf(d.w * rstd, gnw.w, gnb.w) * gg.w);
             }
-            if (valid) *reinterpret_cast<float4 *>(prm.y + off) = val;
+            if (valid && in_range_vec(off, 4, (size_t)prm.B * T * C)) *reinterpret_cast<float4 *>(prm.y + off) = val;
         }
         if (BIDIR && g == nch - 1) __syncthreads();  // pass-0 y stores visible before pass-1 reads
     }
@@ -439,11 +439,14 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
         // every chunk ends with a renorm step, so the scaled state is the true
         // state S_{T-1} here (tokens past T were zero-filled: k = 0, ew = 0)
 #pragma unroll
+        const size_t nstate = (size_t)prm.B * H * kHead * kHead;
         for (int qq = 0; qq < 4; ++qq) {
-            *reinterpret_cast<float4 *>(prm.sT + state_off + (size_t)prow(qq, 0) * kHead) =
-                make_float4(S2[qq][0].x, S2[qq][1].x, S2[qq][2].x, S2[qq][3].x);
-            *reinterpret_cast<float4 *>(prm.sT + state_off + (size_t)prow(qq, 1) * kHead) =
-                make_float4(S2[qq][0].y, S2[qq][1].y, S2[qq][2].y, S2[qq][3].y);
+            if (in_range_vec(state_off + (size_t)prow(qq, 0) * kHead, 4, nstate))
+                *reinterpret_cast<float4 *>(prm.sT + state_off + (size_t)prow(qq, 0) * kHead) =
+                    make_float4(S2[qq][0].x, S2[qq][1].x, S2[qq][2].x, S2[qq][3].x);
+            if (in_range_vec(state_off + (size_t)prow(qq, 1) * kHead, 4, nstate))
+                *reinterpret_cast<float4 *>(prm.sT + state_off + (size_t)prow(qq, 1) * kHead) =
+                    make_float4(S2[qq][0].y, S2[qq][1].y, S2[qq][2].y, S2[qq][3].y);
         }
     }
 }

@@ -438,7 +438,9 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
                         const int p = 16 * warp + (lane >> 2) + 8 * hr;
-                        valid[hr] = c * kSL + p < T;
+                        valid[hr] = c * kSL + p < T &&   // the head's 64 channels of the token
+                                    in_range_vec(((size_t)b * T + time_of(dir, c, p)) * C + cbase, kHead,
+                                                 (size_t)prm.B * T * C);
                         dst[hr] = reinterpret_cast<float2 *>(
                             prm.y + ((size_t)b * T + (valid[hr] ? time_of(dir, c, p) : 0)) * C + cbase + 2 * q4);
 #pragma unroll
@@ -553,10 +555,11 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                         for (int ii = 0; ii < kHead; ++ii) acc += part[ii * kPartStride + j];
                         const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + j;
                         float *dst = prm.y + o;
-                        float yo = accumulate_y ? *dst + acc : acc;
+                        const bool ok = in_range(o, (size_t)prm.B * T * C);
+                        float yo = (accumulate_y && ok) ? *dst + acc : acc;
                         if (norm) {
                             // the token's 64 outputs are one per thread of warps 0 and 1
-                            const float gt = __ldg(prm.g + o);
+                            const float gt = ok ? __ldg(prm.g + o) : 0.f;
                             float s1 = warp_sum(yo);
                             if (lane == 0) sm.red[warp] = s1;
                             sync_warps01();
@@ -568,7 +571,7 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                             const float rstd = rsqrtf((sm.red[2] + sm.red[3]) * (1.f / kHead) + prm.gn_eps);
                             yo = fmaf(d * rstd, sm.gnw[j], sm.gnb[j]) * gt;
                         }
-                        *dst = yo;
+                        if (ok) *dst = yo;
                     }
                     if (row_lane) {
                         const float dd = __expf(xr.ew[p][i]), kk = xr.k[p][i];

@@ -601,7 +601,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                         }
                     }
                     named_sync(2, kET);
-                    if (yrole && t0 + p < T) {
+                    if (yrole && t0 + p < T && in_range(((size_t)b * T + t0 + p) * C + cbase + row, (size_t)prm.B * T * C)) {
                         const int jj = row;   // 0..63
                         prm.y[((size_t)b * T + t0 + p) * C + cbase + jj] =
                             sm.ypart[p & 1][0][jj] + sm.ypart[p & 1][1][jj] + sm.cp[c & 3][p] * raw_at(V, p, jj);

@@ -75,6 +75,24 @@ int check_device() {
     return ok ? WKV_OK : WKV_ERR_DEVICE;
 }
 
+// Result of an entry point that enqueued work (e: the runtime's status after the
+// launches).  In the debug build (-DWKV_DEVICE_CHECKS=1) the entry point also waits
+// for the device and reports what its kernels' checks recorded in the fault word
+// (then cleared): an index out of range as WKV_ERR_DEVICE_CHECK, a bounded wait
+// that ran out as WKV_ERR_TIMEOUT.  The other builds never wait.
+int launched(cudaError_t e) {
+    if (e != cudaSuccess) return WKV_ERR_CUDA;
+#if WKV_DEVICE_CHECKS
+    if (cudaDeviceSynchronize() != cudaSuccess) return WKV_ERR_CUDA;
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_wkv_faults, sizeof(v)) != cudaSuccess) return WKV_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(g_wkv_faults, &zero, sizeof(zero)) != cudaSuccess) return WKV_ERR_CUDA;
+    if (v & WKV_FAULT_INDEX) return WKV_ERR_DEVICE_CHECK;
+    if (v & WKV_FAULT_TIMEOUT) return WKV_ERR_TIMEOUT;
+#endif
+    return WKV_OK;
+}
+
 // Shared checks of the RWKV-6 entry points.
 int check_wkv6(int B, int T, int C, int H, std::initializer_list<const void *> ptrs) {
     if (B < 0 || T < 0 || C < 1 || H < 1 || C % H != 0) return WKV_ERR_ARG;
@@ -125,7 +143,7 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (B == 0 || T == 0) {
         if ((st = check_device()) != WKV_OK) return st;
-        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+        return launched(cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s));
     }
     const bool tensor = kTensorCorePaths;
     // the documented requirement (wkv6_bwd_workspace_bytes) in both builds, although
@@ -137,15 +155,12 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
     if (tensor) {
         float *ws = static_cast<float *>(workspace);
         BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, ws};
-        return wkv6_bwd_split_launch(bf16, bidirectional != 0, r, k, v, w, dy, prm, ws + (size_t)B * C, du, s) ==
-                       cudaSuccess
-                   ? WKV_OK
-                   : WKV_ERR_CUDA;
+        return launched(wkv6_bwd_split_launch(bf16, bidirectional != 0, r, k, v, w, dy, prm, ws + (size_t)B * C, du, s));
     }
     CUtensorMap maps[kBwdMaps];
     if (!make_bwd_maps(maps, bf16, B, T, C, r, k, w, v, dy, dr, dk, dv, dw)) return WKV_ERR_CUDA;
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, static_cast<float *>(workspace)};
-    return wkv6_bwd_launch(bf16, bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return launched(wkv6_bwd_launch(bf16, bidirectional != 0, maps, prm, du, s));
 }
 
 // w5 (RWKV-5): static per-channel decay rate [C]; then w is ignored (pass w5 for
@@ -175,9 +190,7 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
             return WKV_ERR_CUDA;
         FwdParams prm{B, T, C, H, u, y};
         prm.w5 = w5;
-        return wkv6_fwd_tc_launch(mr, mk, mv, mw, my, prm, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-                   ? WKV_OK
-                   : WKV_ERR_CUDA;
+        return launched(wkv6_fwd_tc_launch(mr, mk, mv, mw, my, prm, reinterpret_cast<cudaStream_t>(stream)));
     }
     if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && kTensorCorePaths) {
         FwdParams prm{B, T, C, H, u, y};
@@ -188,11 +201,9 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
             prm.gn_b = fused->gn_b;
             prm.gn_eps = fused->eps;
         }
-        return wkv6_fwd_split_launch(bidir, static_cast<const float *>(r), static_cast<const float *>(k),
+        return launched(wkv6_fwd_split_launch(bidir, static_cast<const float *>(r), static_cast<const float *>(k),
                                      static_cast<const float *>(v), static_cast<const float *>(w), prm,
-                                     reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-                   ? WKV_OK
-                   : WKV_ERR_CUDA;
+                                     reinterpret_cast<cudaStream_t>(stream)));
     }
     // a static decay leaves the w map unread: it is built over r only to be well formed
     if (!make_map(&mr, r, bf16, B, T, C, kHead, kFwdTC) || !make_map(&mk, k, bf16, B, T, C, kHead, kFwdTC) ||
@@ -210,10 +221,7 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
         prm.gn_b = fused->gn_b;
         prm.gn_eps = fused->eps;
     }
-    return wkv6_fwd_launch(bf16, bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)) ==
-                   cudaSuccess
-               ? WKV_OK
-               : WKV_ERR_CUDA;
+    return launched(wkv6_fwd_launch(bf16, bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace
@@ -254,7 +262,7 @@ int wkv6_fwd_state(int B, int T, int C, int H, const float *r, const float *k, c
         if (s0 == sT) return WKV_OK;
         const cudaError_t e = s0 != nullptr ? cudaMemcpyAsync(sT, s0, bytes, cudaMemcpyDeviceToDevice, cs)
                                             : cudaMemsetAsync(sT, 0, bytes, cs);
-        return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+        return launched(e);
     }
     return fwd_common(false, false, B, T, C, H, r, k, v, w, u, y, stream, s0, sT);
 }
@@ -271,10 +279,7 @@ int wkv6_decode(int B, int C, int H, const float *r, const float *k, const float
     if (B == 0) return WKV_OK;
     const int st = check_device();
     if (st != WKV_OK) return st;
-    return wkv6_decode_launch(B, C, H, r, k, v, w, u, state, y, reinterpret_cast<cudaStream_t>(stream)) ==
-                   cudaSuccess
-               ? WKV_OK
-               : WKV_ERR_CUDA;
+    return launched(wkv6_decode_launch(B, C, H, r, k, v, w, u, state, y, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t wkv6_bwd_workspace_bytes(int B, int T, int C, int H, int bidirectional) {
@@ -334,7 +339,7 @@ int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const f
     if (B == 0 || T == 0) {
         if ((st = check_device()) != WKV_OK) return st;
         if (cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)C, s) != cudaSuccess) return WKV_ERR_CUDA;
-        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+        return launched(cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s));
     }
     if (workspace == nullptr || workspace_bytes < wkv5_bwd_workspace_bytes(B, T, C, H)) return WKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
@@ -349,7 +354,7 @@ int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const f
                     2 * sizeof(float) * (size_t)B * C, stream);
     if (st != WKV_OK) return st;
     // the fold's per-block partials reuse the log-decay tensor, which the backward no longer reads
-    return wkv5_dw_reduce_launch(B * T, C, dwtok, ew, dw, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return launched(wkv5_dw_reduce_launch(B * T, C, dwtok, ew, dw, s));
 }
 
 int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u, float *y,
@@ -360,9 +365,7 @@ int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w
     if (B == 0 || T == 0) return WKV_OK;
     int st = check_device();
     if (st != WKV_OK) return st;
-    return wkv4_fwd_launch(B, T, C, k, v, w, u, y, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? WKV_OK
-               : WKV_ERR_CUDA;
+    return launched(wkv4_fwd_launch(B, T, C, k, v, w, u, y, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t wkv4_bwd_workspace_bytes(int B, int T, int C) {
@@ -383,15 +386,12 @@ int wkv4_bwd(int B, int T, int C, const float *k, const float *v, const float *w
     if (B == 0 || T == 0) {
         if ((st = check_device()) != WKV_OK) return st;
         if (cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)C, s) != cudaSuccess) return WKV_ERR_CUDA;
-        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+        return launched(cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s));
     }
     if (workspace == nullptr || workspace_bytes < wkv4_bwd_workspace_bytes(B, T, C)) return WKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
     if ((st = check_device()) != WKV_OK) return st;
-    return wkv4_bwd_launch(B, T, C, k, v, w, u, dy, dk, dv, dw, du, static_cast<float *>(workspace), s) ==
-                   cudaSuccess
-               ? WKV_OK
-               : WKV_ERR_CUDA;
+    return launched(wkv4_bwd_launch(B, T, C, k, v, w, u, dy, dk, dv, dw, du, static_cast<float *>(workspace), s));
 }
 
 const char *wkv_status_string(int status) {
@@ -404,6 +404,8 @@ const char *wkv_status_string(int status) {
         case WKV_ERR_CUDA: return "CUDA runtime or launch error";
         case WKV_ERR_DEVICE: return "current device is not sm_100 (B200)";
         case WKV_ERR_TOO_LARGE: return "problem too large (B*T*C must be < 2^31)";
+        case WKV_ERR_DEVICE_CHECK: return "a kernel's index check failed (debug build)";
+        case WKV_ERR_TIMEOUT: return "a kernel's bounded wait ran out (debug build)";
         default: return "unknown status";
     }
 }
@@ -490,7 +492,7 @@ extern "C" int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, c
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = check_device()) != WKV_OK) return st;
     if (B == 0 || T == 0)
-        return cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+        return launched(cudaMemsetAsync(du, 0, sizeof(float) * (size_t)C, s));
     float *scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != WKV_OK) return st;
     CUtensorMap maps[kBwdMaps];
@@ -498,7 +500,7 @@ extern "C" int wkv6_bwd_noalloc(int B, int T, int C, int H, int bidirectional, c
     // Every per-batch partial the reduction reads is written first by the
     // backward kernel, so nothing left in the array by an earlier call leaks in.
     BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, scratch};
-    return wkv6_bwd_launch(false, bidirectional != 0, maps, prm, du, s) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return launched(wkv6_bwd_launch(false, bidirectional != 0, maps, prm, du, s));
 }
 
 // ---------------------------------------------------------------------------
@@ -525,5 +527,30 @@ extern "C" int wkv_selftest_wait_timeout(wkv_stream_t stream) {
     int st = wkv::check_device();
     if (st != WKV_OK) return st;
     wkv::wkv_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
-    return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return launched(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// wkv_selftest_index_check: exercises the failure path of the index checks.  One
+// thread attempts a store whose index equals the size of the array it targets; the
+// check (the one every store of the debug build makes, applied here in every
+// build) skips the store and records WKV_FAULT_INDEX, and the kernel returns.
+
+namespace wkv {
+namespace {
+
+__device__ float g_selftest_sink[4];
+
+__global__ void wkv_index_selftest_kernel(size_t idx, size_t n) {
+    if (threadIdx.x == 0 && in_range_checked(idx, n)) g_selftest_sink[idx] = 1.f;
+}
+
+}  // namespace
+}  // namespace wkv
+
+extern "C" int wkv_selftest_index_check(wkv_stream_t stream) {
+    int st = wkv::check_device();
+    if (st != WKV_OK) return st;
+    wkv::wkv_index_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(4, 4);
+    return wkv::launched(cudaGetLastError());
 }

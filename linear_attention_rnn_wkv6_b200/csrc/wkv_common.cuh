@@ -133,6 +133,36 @@ __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// Index checks of the debug build.  Built with -DWKV_DEVICE_CHECKS=1
+// (libwkv_debug.so), every global store of the kernels first checks its element
+// index against the size of the array it writes; an index out of range skips the
+// store and records WKV_FAULT_INDEX in the fault word (the kernel goes on; nothing
+// traps).  In the other builds the check is the constant true and compiles away.
+#ifndef WKV_DEVICE_CHECKS
+#define WKV_DEVICE_CHECKS 0
+#endif
+// The check itself, in every build (the debug build's in_range, and the self-test).
+__device__ __forceinline__ bool in_range_checked(size_t idx, size_t n) {
+    if (idx >= n) {
+        atomicOr(&g_wkv_faults, WKV_FAULT_INDEX);
+        return false;
+    }
+    return true;
+}
+__device__ __forceinline__ bool in_range(size_t idx, size_t n) {
+#if WKV_DEVICE_CHECKS
+    return in_range_checked(idx, n);
+#else
+    (void)idx;
+    (void)n;
+    return true;
+#endif
+}
+// The same check for a vector store of `width` elements starting at idx.
+__device__ __forceinline__ bool in_range_vec(size_t idx, int width, size_t n) {
+    return in_range(idx, n) && in_range(idx + (size_t)(width - 1), n);
+}
+
 // exp(x) for the decay factorisation: exp2 of x*log2(e) on the SFU.
 __device__ __forceinline__ float fast_exp(float x) { return exp2f(x * 1.4426950408889634f); }
 

@@ -20,9 +20,9 @@ HEADER = os.path.join(ROOT, "include", "wkv.h")
 WKV_OK, WKV_ERR_ARG, WKV_ERR_HEADSIZE, WKV_ERR_ALIGN, WKV_ERR_WORKSPACE = 0, -1, -2, -3, -4
 
 
-@pytest.fixture(scope="module", params=["default", "recurrence"])
+@pytest.fixture(scope="module", params=["default", "recurrence", "debug"])
 def lib(request):
-    """Both builds of the library (the product and the test build) carry the same ABI."""
+    """Every build of the library (the product, the test build, the debug build) carries the same ABI."""
     from linear_attention_rnn_wkv6_b200 import build
     build.build()
     with wkv.use_library(request.param) as handle:

@@ -198,6 +198,27 @@ def test_wkv6_bwd_small(B, T, H, bidir, bwd_path):
         assert _rel(g, e) <= gc.TOL_F32_GRAD, (name, _rel(g, e))
 
 
+@pytest.mark.parametrize("B,T,H", [(2, 3, 1), (1, 31, 2), (2, 33, 1), (1, 65, 2), (2, 197, 2)])
+@pytest.mark.parametrize("bidir", [False, True])
+def test_wkv6_bwd_decay_gradient_vanishes_at_both_ends(B, T, H, bidir, bwd_path):
+    """The first token's decay scales the empty state and the last token's decay scales a
+    state no token reads (in both sweep directions), so dw[:, 0, :] and dw[:, T-1, :] are
+    exactly zero in exact arithmetic.  The chunked tensor-core backward evaluates the first
+    token's dw in prefix form and the last token's in suffix form, where every term is an
+    exact zero, so it returns exact zeros; the recurrence's ends are bounded by 1e-6 of the
+    largest |dw|."""
+    x = synth.make_wkv6(B, T, H, seed=900 + T, with_dy=True)
+    dr, dk, dv, dw, du = gc.run_wkv6_bwd(x, bidir)
+    ends = np.abs(dw[:, [0, T - 1], :])
+    if bwd_path == "recurrence":
+        assert ends.max() <= 1e-6 * np.abs(dw).max(), ends.max()
+    else:
+        assert np.all(ends == 0.0), ends.max()
+    r, k, v, w, u = gc.f64(x)
+    ref = oracle.wkv6_bwd(r, k, v, w, u, x.dy.astype(np.float64), H=H, bidirectional=bidir)
+    assert _rel(dw, ref[3]) <= gc.TOL_F32_GRAD
+
+
 @pytest.mark.parametrize("bidir", [False, True])
 def test_wkv6_bwd_strong_decay_and_determinism(bidir, bwd_path):
     x = synth.make_wkv6(2, 45, 2, seed=7, with_dy=True)
@@ -217,6 +238,8 @@ def test_wkv6_bwd_strong_decay_and_determinism(bidir, bwd_path):
 # ------------------------------------------------------------------ RWKV-4
 
 @pytest.mark.parametrize("B,T,C", [(1, 1, 32), (2, 7, 40), (1, 100, 64), (2, 333, 96), (1, 1024, 32),
+                                   (3, 9, 8), (1, 129, 36), (2, 1000, 100),   # T <= 1024: one cluster per row
+                                   (1, 1025, 32), (2, 2049, 48),              # longer: the two-pass kernel
                                    (2, 50, 30), (1, 65, 36), (3, 31, 20)])   # C % 4 != 0: per-channel kernel
 def test_wkv4_small(B, T, C):
     x = synth.make_wkv4(B, T, C, seed=T)
