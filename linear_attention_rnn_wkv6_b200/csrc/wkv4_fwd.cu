@@ -295,203 +295,10 @@ wkv4_fwd_vec_kernel(int T, int C, const float *__restrict__ k, const float *__re
     }
 }
 
-// ------------------------------------------------------------------ single pass, one cluster per row
-// For T <= kClMaxT the T axis of a 32-channel group is split over a cluster of
-// kCl CTAs; each CTA keeps its slice of k and v in registers, so the inputs are
-// read from HBM once and no pass re-reads them.  A CTA covers 32 channels (a
-// token row of the group is one 128-byte line: 8 threads x one float4) and 16
-// sub-segments of its slice (one per group of 8 threads), each thread at most
-// kClTok tokens.
-//   phase 1  every thread folds its sub-segment from the empty state
-//   phase 2  per channel, the CTA's 16 sub-segment summaries are combined in
-//            order (the state each sub-segment would enter with from the slice
-//            start, and the slice's own summary); the slice summaries are
-//            exchanged through distributed shared memory and every CTA folds
-//            those of the slices before its own -> the state entering its slice
-//   phase 3  every thread runs its sub-segment from its entering state, from the
-//            registers loaded in phase 1, and writes y.
-constexpr int kCl = 8;                         // CTAs per cluster, along T
-constexpr int kClCh = 32;                      // channels per CTA
-constexpr int kClQ = kClCh / VEC;              // threads per token row (8)
-constexpr int kClSub = 16;                     // sub-segments per CTA
-constexpr int kClTok = 8;                      // tokens per thread, at most
-constexpr int kClThr = kClQ * kClSub;          // 128 threads
-constexpr int kClMaxT = kCl * kClSub * kClTok; // 1024
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_barrier() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// A float in the shared memory of CTA `rank` of this cluster, at the address this
-// CTA's `local` has in its own shared memory.  Only read after a cluster barrier
-// that orders the owner's stores before it (the barrier's asm is the compiler
-// fence), so the loads themselves may be scheduled together.
-__device__ __forceinline__ float ld_dsmem(const float *local, uint32_t rank) {
-    uint32_t remote;
-    asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-    float x;
-    asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(remote));
-    return x;
-}
-
-// X <- (X decayed over n tokens) (+) L, in log space (w2 = w log2 e; n >= 0).
-__device__ __forceinline__ void wkv4_then(Wkv4State &X, float n, const Wkv4State &L, float w2) {
-    const float pd = X.p - n * w2;
-    const float q = fmaxf(pd, L.p);
-    if (q == -INFINITY) return;   // both empty: X stays empty
-    const float e1 = ex2(pd - q), e2 = ex2(L.p - q);
-    X.a = fmaf(e1, X.a, e2 * L.a);
-    X.b = fmaf(e1, X.b, e2 * L.b);
-    X.p = q;
-}
-
-__global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kClThr, 4)
-wkv4_fwd_cluster_kernel(int T, int C, const float *__restrict__ k, const float *__restrict__ v,
-                        const float *__restrict__ w, const float *__restrict__ u, float *__restrict__ y) {
-    __shared__ Wkv4State summ[kClSub][kClCh];   // phase 1 summaries, then the states entering each sub-segment
-    __shared__ float agg[3][kClCh];             // this slice's summary (a, b, p), read by the later slices
-    const int tid = threadIdx.x;
-    const int cq = tid % kClQ, sub = tid / kClQ;
-    const uint32_t slice = cluster_ctarank();
-    const int groups = (C + kClCh - 1) / kClCh;
-    const int row = blockIdx.x / kCl;            // (b, channel group) of the cluster
-    const int b = row / groups;
-    const int cg = (row % groups) * kClCh;       // first channel of the group
-    const int c0 = cg + VEC * cq;
-    const bool live = c0 < C;                    // C % VEC == 0: the float4 is whole or absent
-    const int sl = (T + kCl - 1) / kCl;          // tokens per slice
-    const int ss = (sl + kClSub - 1) / kClSub;   // tokens per sub-segment (<= kClTok when T <= kClMaxT)
-    const int s0 = min(T, (int)slice * sl), s1 = min(T, s0 + sl);
-    const int t0 = min(s1, s0 + sub * ss), t1 = min(s1, t0 + ss);
-    float w2[VEC], u2[VEC];
-    {
-        const V wv = live ? *reinterpret_cast<const V *>(w + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const V uv = live ? *reinterpret_cast<const V *>(u + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-            w2[i] = comp(wv, i) * kLog2e;
-            u2[i] = comp(uv, i) * kLog2e;
-        }
-    }
-    const size_t base = (size_t)b * T * C + c0;
-    // ---- the sub-segment's k and v, every load issued before any use ----
-    V kb[kClTok], vb[kClTok];
-#pragma unroll
-    for (int e = 0; e < kClTok; ++e) {
-        const bool in = live && t0 + e < t1;
-        kb[e] = in ? __ldg(reinterpret_cast<const V *>(k + base + (size_t)(t0 + e) * C)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        vb[e] = in ? __ldg(reinterpret_cast<const V *>(v + base + (size_t)(t0 + e) * C)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    // ---- phase 1: sub-segment summary from the empty state ----
-    Wkv4State st[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) st[i] = Wkv4State{0.f, 0.f, -INFINITY};
-#pragma unroll
-    for (int e = 0; e < kClTok; ++e)
-        if (t0 + e < t1) {
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) wkv4_update(st[i], comp(kb[e], i) * kLog2e, comp(vb[e], i), w2[i]);
-        }
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) summ[sub][VEC * cq + i] = st[i];
-    __syncthreads();
-    // ---- phase 2a: per channel, the state each sub-segment enters with, counted from
-    // the slice start (E_0 empty, E_{s+1} = E_s decayed over sub-segment s (+) its
-    // summary), and the slice summary E_16.  Thread (q, ch), q = tid / 32, first folds
-    // the four sub-segments 4q .. 4q+3 (their summary goes to gsum[q]); the quarters'
-    // entering states then come from gsum, and each thread finishes its four ----
-    __shared__ Wkv4State gsum[kClSub / 4][kClCh];
-    const int ch = tid % kClCh, qr = tid / kClCh;   // channel, quarter of the sub-segments
-    const float wch = cg + ch < C ? w[cg + ch] * kLog2e : 0.f;
-    auto sub_len = [&](int s) { const int a0 = min(s1, s0 + s * ss); return (float)(min(s1, a0 + ss) - a0); };
-    {
-        Wkv4State X{0.f, 0.f, -INFINITY};
-        for (int s = 4 * qr; s < 4 * qr + 4; ++s) wkv4_then(X, sub_len(s), summ[s][ch], wch);
-        gsum[qr][ch] = X;
-    }
-    __syncthreads();
-    {
-        Wkv4State X{0.f, 0.f, -INFINITY};   // entering quarter qr from the slice start
-        for (int g = 0; g < qr; ++g)
-            wkv4_then(X, sub_len(4 * g) + sub_len(4 * g + 1) + sub_len(4 * g + 2) + sub_len(4 * g + 3), gsum[g][ch], wch);
-        Wkv4State L[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) L[e] = summ[4 * qr + e][ch];
-        __syncthreads();   // every thread has read the phase 1 summaries it needs
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            summ[4 * qr + e][ch] = X;
-            wkv4_then(X, sub_len(4 * qr + e), L[e], wch);
-        }
-        if (qr == kClSub / 4 - 1) {   // X is now the slice summary E_16
-            agg[0][ch] = X.a;
-            agg[1][ch] = X.b;
-            agg[2][ch] = X.p;
-        }
-    }
-    cluster_barrier();   // every slice summary is published (and summ is complete in this CTA)
-    // ---- phase 2b: the state entering this slice, folded from the earlier slices'
-    // summaries (F_0 empty, F_{j+1} = F_j decayed over slice j (+) its summary), then the
-    // state entering each sub-segment: F decayed from the slice start (+) E_s ----
-    {
-        // every thread of channel ch folds the earlier slices (the four quarters redo the
-        // same fold; all of a thread's remote loads are issued before the first use)
-        float A[3][kCl];
-#pragma unroll
-        for (int j = 0; j < kCl; ++j)
-            if (j < (int)slice) {
-                A[0][j] = ld_dsmem(&agg[0][ch], j);
-                A[1][j] = ld_dsmem(&agg[1][ch], j);
-                A[2][j] = ld_dsmem(&agg[2][ch], j);
-            }
-        Wkv4State F{0.f, 0.f, -INFINITY};
-#pragma unroll
-        for (int j = 0; j < kCl; ++j)
-            if (j < (int)slice) {
-                const int j0 = min(T, j * sl), j1 = min(T, j0 + sl);
-                wkv4_then(F, (float)(j1 - j0), Wkv4State{A[0][j], A[1][j], A[2][j]}, wch);
-            }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int s = 4 * qr + e;
-            Wkv4State X = F;
-            wkv4_then(X, (float)(min(s1, s0 + s * ss) - s0), summ[s][ch], wch);
-            summ[s][ch] = X;
-        }
-    }
-    cluster_barrier();   // no CTA leaves while another may still read its summary; summ is final
-    // ---- phase 3: the sub-segment from its entering state, from registers; write y ----
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) st[i] = summ[sub][VEC * cq + i];
-#pragma unroll
-    for (int e = 0; e < kClTok; ++e)
-        if (live && t0 + e < t1) {
-            float o[VEC];
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) {
-                const float k2 = comp(kb[e], i) * kLog2e, vv = comp(vb[e], i);
-                o[i] = wkv4_output(st[i], k2, vv, u2[i]);
-                wkv4_update(st[i], k2, vv, w2[i]);
-            }
-            if (in_range_vec(base + (size_t)(t0 + e) * C, VEC, (size_t)(gridDim.x / kCl / groups) * T * C))
-                *reinterpret_cast<V *>(y + base + (size_t)(t0 + e) * C) = vmake(o);
-        }
-}
-
 }  // namespace
 
 cudaError_t wkv4_fwd_launch(int B, int T, int C, const float *k, const float *v, const float *w,
                             const float *u, float *y, cudaStream_t stream) {
-    if (C % VEC == 0 && T <= kClMaxT) {
-        // one cluster of kCl CTAs per (batch, 32-channel group)
-        const unsigned ctas = (unsigned)(B * ((C + kClCh - 1) / kClCh) * kCl);
-        wkv4_fwd_cluster_kernel<<<ctas, kClThr, 0, stream>>>(T, C, k, v, w, u, y);
-        return cudaGetLastError();
-    }
     const int groups = (C + kCh - 1) / kCh;
     if (C % VEC == 0) {
         wkv4_fwd_vec_kernel<<<(unsigned)(B * groups), kThrV, 0, stream>>>(T, C, k, v, w, u, y);

@@ -98,7 +98,7 @@ def test_debug_build_backward_bf16_and_noalloc(bidir, debug_build):
         assert oracle.rel_l2(g.cpu().numpy(), e) <= gc.TOL_F32_GRAD, name
 
 
-@pytest.mark.parametrize("B,T,C", [(2, 100, 64), (1, 1100, 32), (2, 30, 20)])   # cluster, two-pass, per-channel
+@pytest.mark.parametrize("B,T,C", [(2, 100, 64), (1, 1100, 32), (2, 30, 20)])   # four channels a thread, and one
 def test_debug_build_wkv4(B, T, C, debug_build):
     x = synth.make_wkv4(B, T, C, seed=540 + T, with_dy=True)
     y = gc.run_wkv4(x)

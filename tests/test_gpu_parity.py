@@ -238,8 +238,7 @@ def test_wkv6_bwd_strong_decay_and_determinism(bidir, bwd_path):
 # ------------------------------------------------------------------ RWKV-4
 
 @pytest.mark.parametrize("B,T,C", [(1, 1, 32), (2, 7, 40), (1, 100, 64), (2, 333, 96), (1, 1024, 32),
-                                   (3, 9, 8), (1, 129, 36), (2, 1000, 100),   # T <= 1024: one cluster per row
-                                   (1, 1025, 32), (2, 2049, 48),              # longer: the two-pass kernel
+                                   (3, 9, 8), (1, 129, 36), (2, 1000, 100), (1, 1025, 32), (2, 2049, 48),
                                    (2, 50, 30), (1, 65, 36), (3, 31, 20)])   # C % 4 != 0: per-channel kernel
 def test_wkv4_small(B, T, C):
     x = synth.make_wkv4(B, T, C, seed=T)
