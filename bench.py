@@ -93,7 +93,7 @@ LAUNCHES = {"wkv6_causal_f32_b1t196h4": 1, "wkv6_causal_f32_b32t196h12": 1, "wkv
             "wkv6_bidir_bwd_f32_b32t196h12": 3,   # S-kind and G-kind tensor-core kernels and the deterministic du reduction
             "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 3,
             "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
-            "wkv5_bwd_f32_b32t196h12": 6,   # decay expansion, S and G kinds, du reduction, two-stage dw fold
+            "wkv5_bwd_f32_b32t196h12": 4,   # S and G kinds with the static decay, du reduction, dw total
             "wkv6_bidir_fused_f32_b32t196h12": 1}
 
 

@@ -279,14 +279,19 @@ int wkv5_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t 
  *   and T in a fixed order (deterministic).  dw is w.r.t. the decay rate w of
  *   wkv5_fwd (dL/dw = -sum_{b,t} dL/d(ew_t)).
  * workspace: at least wkv5_bwd_workspace_bytes(B,T,C,H) bytes of device memory,
- * 16-byte aligned, caller-owned (the constant log-decay, its per-token gradient
- * and the RWKV-6 backward's scratch).  Errors as wkv6_bwd.
+ * 16-byte aligned, caller-owned.  Errors as wkv6_bwd.
+ * Algorithm: the chunked tensor-core backward of wkv6_bwd (causal) with the
+ * constant log-decay -w in place of loaded decays; each token's decay gradient is
+ * added into per-(b, c) totals in double instead of being stored, and dw is their
+ * sum over b.  (The test build runs the recurrence backward on a [B,T,C] copy of
+ * the log-decay and folds its per-token dw over b and t.)
  */
 int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
              const float *u, const float *dy, float *dr, float *dk, float *dv, float *dw, float *du,
              void *workspace, size_t workspace_bytes, wkv_stream_t stream);
 
-/* Scratch bytes wkv5_bwd needs: 4 * (2*B*T*C + B*C). */
+/* Scratch bytes wkv5_bwd needs: 24*B*C (product build; 4 * (2*B*T*C + 2*B*C) in
+ * the recurrence test build). */
 size_t wkv5_bwd_workspace_bytes(int B, int T, int C, int H);
 
 /*

@@ -1,9 +1,11 @@
-// wkv5.cu -- helpers of the RWKV-5 (static decay) backward.
+// wkv5.cu -- helpers of the RWKV-5 (static decay) backward in the recurrence test
+// build (libwkv_recurrence.so; the product build runs the tensor-core backward
+// with the static decay built in, wkv6_bwd_split.cu).
 //
 // RWKV-5 ("RWKV Architecture ...", RWKV-5 "Eagle") decays the matrix state by
 // the static per-channel factor exp(-w); it is RWKV-6 with the log-decay
-// ew_t = -w at every token.  Its backward therefore runs the RWKV-6 backward on
-// that constant log-decay and folds the per-token decay gradient into one value
+// ew_t = -w at every token.  Its backward can therefore run the RWKV-6 backward on
+// that constant log-decay and fold the per-token decay gradient into one value
 // per channel: dL/dw[c] = -sum_{b,t} dL/dew_t[b][c].  The two kernels here
 // write the constant log-decay tensor and do that fold (a fixed summation
 // order over b and t, so the result is deterministic).
@@ -11,6 +13,7 @@
 
 #include "wkv_launch.cuh"
 
+#if WKV_RECURRENCE_PATHS
 namespace wkv {
 
 namespace {
@@ -83,3 +86,4 @@ cudaError_t wkv5_dw_reduce_launch(int rows, int C, const float *dwtok, float *pa
 }
 
 }  // namespace wkv
+#endif  // WKV_RECURRENCE_PATHS

@@ -119,10 +119,11 @@ __device__ __forceinline__ uint64_t desc_cm(const __nv_bfloat16 *tile) { return 
 // decay gradient takes the prefix form).  `run` ends as the carry after the chunk
 // in every thread.  `xch` is 2 x 64 floats of shared memory.  Loads of a thread's
 // 16 tokens are issued before its stores.
-template <typename PartF, typename ExtraF, typename HeadF, typename AddrF>
+// ACC: add the values into `total` (one channel's running total, RWKV-5) instead of storing them.
+template <bool ACC = false, typename PartF, typename ExtraF, typename HeadF, typename AddrF>
 __device__ __forceinline__ void dw_scan_chunk(int tid, int c, int T, int order, bool base_load, float sign,
                                               ExtraF extra, HeadF head, float &run, float *xch, float *dw,
-                                              size_t n, PartF part, AddrF addr) {
+                                              size_t n, PartF part, AddrF addr, double *total = nullptr) {
     const int i = tid & (kHead - 1), h = tid >> 6;
     const int p0 = 16 * h;
     const bool first_half = (order == 0) == (h == 0);   // this half comes first in scan order
@@ -155,8 +156,11 @@ __device__ __forceinline__ void dw_scan_chunk(int tid, int c, int T, int order, 
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const int p = p0 + e;
-        if (c * kBL + p < T && in_range(addr(p), n))
-            dw[addr(p)] = prev[e] + extra(p, i) + (head(p) ? 0.f : sign * (carry + loc[e]));
+        if (c * kBL + p < T && (ACC || in_range(addr(p), n))) {
+            const float val = prev[e] + extra(p, i) + (head(p) ? 0.f : sign * (carry + loc[e]));
+            if (ACC) *total += (double)val;
+            else dw[addr(p)] = val;
+        }
     }
     run += acc + other;
     __syncthreads();   // xch is free again
@@ -234,7 +238,7 @@ static_assert(sizeof(float) * kBL * kHead <= sizeof(__nv_bfloat16) * kBSt, "exac
 
 // One pass per direction: causal first (forward in time), then, bidirectional,
 // the anti-causal pass (backward in time).
-template <typename Tin, bool BIDIR>
+template <typename Tin, bool BIDIR, bool STAT = false>
 __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restrict__ r,
                                                               const Tin *__restrict__ k,
                                                               const Tin *__restrict__ v,
@@ -283,6 +287,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
     constexpr uint32_t kIdQ2 = idesc_bf16(64, 64, false, false);    // dY (K) x S_in (K-major, rows i)
 
     float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    // RWKV-5: the static log-decay of channels ch, ch + 1 at every token
+    const float2 w5ew = STAT ? make_float2(-prm.w5[cbase + ch], -prm.w5[cbase + ch + 1]) : make_float2(0.f, 0.f);
+    double w5acc = 0.0;   // RWKV-5: this thread's channel's decay-gradient total
     auto time_of = [&](int dir, int c, int p) { return dir > 0 ? c * kBL + p : T - 1 - (c * kBL + p); };
     auto load_chunk = [&](int dir, int c) {
 #pragma unroll
@@ -293,7 +300,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
                 xr_[e] = ld_pair(r + o);
                 xk_[e] = ld_pair(k + o);
                 xv_[e] = ld_pair(v + o);
-                xw_[e] = ld_pair(w + o);
+                xw_[e] = STAT ? w5ew : ld_pair(w + o);
                 xd_[e] = ld_pair(dy + o);
             } else {
                 xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
@@ -589,9 +596,11 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
             // suffix of z - x minus z_m, or -z_m (the prefix form) at the first token =====
             __syncthreads();
             if (!BIDIR) {
-                dw_scan_chunk(tid, c, T, 0, false, -1.f, [](int, int) { return 0.f; }, [](int) { return false; }, zrun,
-                              sm.xch, prm.dw, nBTC, [&](int p, int i) { return sm.E[fidx(p, i)]; },
-                              [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
+                // (RWKV-5: the values are added into this thread's channel total instead)
+                dw_scan_chunk<STAT>(tid, c, T, 0, false, -1.f, [](int, int) { return 0.f; }, [](int) { return false; },
+                                    zrun, sm.xch, prm.dw, nBTC, [&](int p, int i) { return sm.E[fidx(p, i)]; },
+                                    [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); },
+                                    &w5acc);
             } else if (!causal) {
                 dw_scan_chunk(tid, c, T, 0, false, 1.f, [&](int p, int i) { return -sm.R[fidx(p, i)]; },
                               [&](int p) { return time_of(dir, c, p) == 0; }, zrun, sm.xch, prm.dw, nBTC,
@@ -612,6 +621,15 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
     __syncthreads();
     if (tid < kHead && in_range((size_t)b * C + cbase + tid, (size_t)prm.B * C))
         prm.du_part[(size_t)b * C + cbase + tid] = sm.dusum[0][tid] + sm.dusum[1][tid] + sm.dusum[2][tid] + sm.dusum[3][tid];
+    if (STAT) {
+        // RWKV-5: the two token halves' totals of each channel, then this kind's partial
+        __syncthreads();   // dusum is free again
+        double *wx = reinterpret_cast<double *>(&sm.dusum[0][0]);   // [half][channel]
+        wx[tid] = w5acc;
+        __syncthreads();
+        if (tid < kHead && in_range((size_t)b * C + cbase + tid, (size_t)prm.B * C))
+            prm.w5_part[(size_t)b * C + cbase + tid] = wx[tid] + wx[kHead + tid];
+    }
     if (!ok && (tid == 0 || tid == 32)) {
         mma_commit(&sm.bar_fin);
         if (tid == 0) mbar_wait_bounded(&sm.bar_fin, 0);
@@ -655,7 +673,7 @@ static_assert(sizeof(float) * kHead * kHead <= sizeof(__nv_bfloat16) * kBT * kBS
 // Passes: bidirectional, the anti-causal one first (its chunks in reverse processing
 // order run forward in time), then the causal one (backward in time); chunks of a
 // pass in reverse processing order, tokens of a chunk from the last to the first.
-template <typename Tin, bool BIDIR>
+template <typename Tin, bool BIDIR, bool STAT = false>
 __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restrict__ r,
                                                               const Tin *__restrict__ k,
                                                               const Tin *__restrict__ v,
@@ -707,6 +725,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
     constexpr uint32_t kIdKK = idesc_bf16(64, 64, false, false);   // V (K) x Gt (K-major, rows i)
 
     float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    // RWKV-5: the static log-decay of channels ch, ch + 1 at every token
+    const float2 w5ew = STAT ? make_float2(-prm.w5[cbase + ch], -prm.w5[cbase + ch + 1]) : make_float2(0.f, 0.f);
+    double w5acc = 0.0;   // RWKV-5: this thread's channel's decay-gradient total
     auto time_of = [&](int dir, int c, int p) { return dir > 0 ? c * kBL + p : T - 1 - (c * kBL + p); };
     auto load_chunk = [&](int dir, int c) {
 #pragma unroll
@@ -717,7 +738,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                 xr_[e] = ld_pair(r + o);
                 xk_[e] = ld_pair(k + o);
                 xv_[e] = ld_pair(v + o);
-                xw_[e] = ld_pair(w + o);
+                xw_[e] = STAT ? w5ew : ld_pair(w + o);
                 xd_[e] = ld_pair(dy + o);
             } else {
                 xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
@@ -1073,11 +1094,15 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
             // share, the running suffix of z - x minus z_m, or -z_m at the first token =====
             __syncthreads();
             if (!BIDIR) {
+                // (RWKV-5: nothing is read back; the values are added into this thread's channel total)
                 const float zt = ztot[(size_t)b * C + cbase + (tid & (kHead - 1))];
-                dw_scan_chunk(tid, c, T, 1, true, -1.f, [&](int p, int) { return time_of(dir, c, p) == 0 ? 0.f : zt; },
-                              [&](int p) { return time_of(dir, c, p) == 0; }, zrun,
-                              reinterpret_cast<float *>(&sm.dAp[0][0]), prm.dw, nBTC, [&](int p, int i) { return sm.F[fidx(p, i)]; },
-                              [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); });
+                dw_scan_chunk<STAT>(tid, c, T, 1, !STAT, -1.f,
+                                    [&](int p, int) { return time_of(dir, c, p) == 0 ? 0.f : zt; },
+                                    [&](int p) { return time_of(dir, c, p) == 0; }, zrun,
+                                    reinterpret_cast<float *>(&sm.dAp[0][0]), prm.dw, nBTC,
+                                    [&](int p, int i) { return sm.F[fidx(p, i)]; },
+                                    [&](int p) { return ((size_t)b * T + time_of(dir, c, p)) * C + cbase + (tid & (kHead - 1)); },
+                                    &w5acc);
             } else if (last) {
                 dw_scan_chunk(tid, c, T, 1, true, 1.f, [&](int p, int i) { return -sm.BK[fidx(p, i)]; },
                               [&](int p) { return time_of(dir, c, p) == 0; }, zrun,
@@ -1090,6 +1115,15 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
             fence_after_sync();
         }
         zrun = 0.f;
+    }
+    if (STAT) {
+        // RWKV-5: the two token halves' totals of each channel, then this kind's partial
+        __syncthreads();
+        double *wx = reinterpret_cast<double *>(&sm.dAp[0][0]);   // [half][channel]
+        wx[tid] = w5acc;
+        __syncthreads();
+        if (tid < kHead && in_range((size_t)b * C + cbase + tid, (size_t)prm.B * C))
+            prm.w5_part[((size_t)prm.B + b) * C + cbase + tid] = wx[tid] + wx[kHead + tid];
     }
     if (!ok && (tid == 0 || tid == 32)) {
         mma_commit(&sm.bar_fin);
@@ -1122,6 +1156,41 @@ static cudaError_t launch_split_bwd(const void *r, const void *k, const void *v,
     kg<<<grid, kBThr, smG, stream>>>(r_, k_, v_, w_, dy_, prm, ztot);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return wkv6_du_reduce_launch(prm.B, prm.C, prm.du_part, du, stream);
+}
+
+namespace {
+// dw[c] = -sum_b (part[0][b][c] + part[1][b][c]) in increasing b, in double (RWKV-5:
+// the gradient with respect to the decay rate w of the log-decay -w).
+__global__ void wkv5_dw_total_kernel(int B, int C, const double *__restrict__ part, float *__restrict__ dw) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    double acc = 0.0;
+    for (int b = 0; b < B; ++b) acc += part[(size_t)b * C + c] + part[((size_t)B + b) * C + c];
+    dw[c] = (float)(-acc);
+}
+}  // namespace
+
+cudaError_t wkv5_bwd_split_launch(const float *r, const float *k, const float *v, const float *dy,
+                                  const BwdParams &prm, float *ztot, float *du, cudaStream_t stream) {
+    const size_t smS = sizeof(SSmem) + 1024, smG = sizeof(GSmem) + 1024;
+    auto ks = wkv6_bwd_s_kernel<float, false, true>;
+    auto kg = wkv6_bwd_g_kernel<float, false, true>;
+    cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smS);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smG);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ks, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kg, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(prm.B * prm.H);
+    // the w argument is not read (the decay is prm.w5): r stands in for it
+    ks<<<grid, kBThr, smS, stream>>>(r, k, v, r, dy, prm, ztot);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    kg<<<grid, kBThr, smG, stream>>>(r, k, v, r, dy, prm, ztot);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = wkv6_du_reduce_launch(prm.B, prm.C, prm.du_part, du, stream)) != cudaSuccess) return e;
+    wkv5_dw_total_kernel<<<(prm.C + 255) / 256, 256, 0, stream>>>(prm.B, prm.C, prm.w5_part, prm.dw);
+    return cudaGetLastError();
 }
 
 cudaError_t wkv6_bwd_split_launch(bool bf16, bool bidir, const void *r, const void *k, const void *v, const void *w,

@@ -438,8 +438,8 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     if (!BIDIR && prm.sT != nullptr) {
         // every chunk ends with a renorm step, so the scaled state is the true
         // state S_{T-1} here (tokens past T were zero-filled: k = 0, ew = 0)
-#pragma unroll
         const size_t nstate = (size_t)prm.B * H * kHead * kHead;
+#pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
             if (in_range_vec(state_off + (size_t)prow(qq, 0) * kHead, 4, nstate))
                 *reinterpret_cast<float4 *>(prm.sT + state_off + (size_t)prow(qq, 0) * kHead) =

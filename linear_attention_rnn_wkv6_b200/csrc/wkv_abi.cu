@@ -192,6 +192,14 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
         prm.w5 = w5;
         return launched(wkv6_fwd_tc_launch(mr, mk, mv, mw, my, prm, reinterpret_cast<cudaStream_t>(stream)));
     }
+    if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && fused == nullptr && kTensorCorePaths &&
+        wkv6_fwd_cluster_fits(B, T, H)) {
+        // short sequence, few heads: every chunk of a (b, h) at once, in one cluster
+        FwdParams prm{B, T, C, H, u, y};
+        return launched(wkv6_fwd_cluster_launch(bidir, static_cast<const float *>(r), static_cast<const float *>(k),
+                                                static_cast<const float *>(v), static_cast<const float *>(w), prm,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+    }
     if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && kTensorCorePaths) {
         FwdParams prm{B, T, C, H, u, y};
         if (fused != nullptr) {
@@ -327,6 +335,8 @@ int wkv5_fwd_bf16(int B, int T, int C, int H, const uint16_t *r, const uint16_t 
 size_t wkv5_bwd_workspace_bytes(int B, int T, int C, int H) {
     (void)H;
     if (B < 1 || T < 0 || C < 1) return 0;
+    if (kTensorCorePaths)   // du partials and z totals (floats), two decay-gradient partials (doubles), [B][C] each
+        return (2 * sizeof(float) + 2 * sizeof(double)) * (size_t)B * C;
     return sizeof(float) * (2 * (size_t)B * T * C + 2 * (size_t)B * C);
 }
 
@@ -344,6 +354,15 @@ int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const f
     if (workspace == nullptr || workspace_bytes < wkv5_bwd_workspace_bytes(B, T, C, H)) return WKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WKV_ERR_ALIGN;
     if ((st = check_device()) != WKV_OK) return st;
+#if !WKV_RECURRENCE_PATHS
+    // the tensor-core backward with the static log-decay: workspace = du partials [B][C]
+    // and z totals [B][C] (floats), then the S and G kinds' decay-gradient partials [2][B][C]
+    float *ws = static_cast<float *>(workspace);
+    BwdParams prm{B, T, C, H, u, dr, dk, dv, dw, ws};
+    prm.w5 = w;
+    prm.w5_part = reinterpret_cast<double *>(ws + 2 * (size_t)B * C);
+    return launched(wkv5_bwd_split_launch(r, k, v, dy, prm, ws + (size_t)B * C, du, s));
+#else
     // workspace: the constant log-decay [B][T][C], its per-token gradient [B][T][C],
     // then the RWKV-6 backward's own 2 [B][C]
     float *ew = static_cast<float *>(workspace);
@@ -355,6 +374,7 @@ int wkv5_bwd(int B, int T, int C, int H, const float *r, const float *k, const f
     if (st != WKV_OK) return st;
     // the fold's per-block partials reuse the log-decay tensor, which the backward no longer reads
     return launched(wkv5_dw_reduce_launch(B * T, C, dwtok, ew, dw, s));
+#endif
 }
 
 int wkv4_fwd(int B, int T, int C, const float *k, const float *v, const float *w, const float *u, float *y,

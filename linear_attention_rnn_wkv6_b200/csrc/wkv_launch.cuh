@@ -30,6 +30,11 @@ struct BwdParams {
     const float *u;
     float *dr, *dk, *dv, *dw;
     float *du_part;   // [B][C] per-batch du partials (caller's workspace)
+    // RWKV-5 (tensor-core backward only): static decay rate w5[C] >= 0, the log-decay
+    // -w5 at every token (the w pointer is not read), and dw is not written: the
+    // kernels add each token's decay gradient into w5_part[2][B][C] (S kind, G kind)
+    const float *w5 = nullptr;
+    double *w5_part = nullptr;
 };
 
 constexpr int kFwdTC = 16;   // tokens per TMA chunk, forward recurrence kernels
@@ -46,6 +51,12 @@ cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, con
 // r, k, v, w are [B][T][C] fp32 device pointers, 8-byte aligned.
 cudaError_t wkv6_fwd_split_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
                                   const FwdParams &prm, cudaStream_t stream);
+// fp32 causal or bidirectional forward for short sequences and few heads: one
+// thread-block cluster per (b, h), one chunk per CTA, the chunk states exchanged
+// through distributed shared memory.  fits: whether (B, T, H) is such a problem.
+bool wkv6_fwd_cluster_fits(int B, int T, int H);
+cudaError_t wkv6_fwd_cluster_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
+                                    const FwdParams &prm, cudaStream_t stream);
 // One recurrent step for B sequences (state [B][H][N][N] updated in place).
 cudaError_t wkv6_decode_launch(int B, int C, int H, const float *r, const float *k, const float *v,
                                const float *w, const float *u, float *state, float *y, cudaStream_t stream);
@@ -62,6 +73,10 @@ cudaError_t wkv6_du_reduce_launch(int B, int C, const float *part, float *du, cu
 cudaError_t wkv6_bwd_split_launch(bool bf16, bool bidir, const void *r, const void *k, const void *v, const void *w,
                                   const void *dy, const BwdParams &prm, float *ztot, float *du,
                                   cudaStream_t stream);
+// RWKV-5 backward on the tensor cores: the causal S- and G-kind kernels with the static
+// log-decay -prm.w5, the du reduction, and dw[c] = -sum_b (w5_part[0][b][c] + w5_part[1][b][c]).
+cudaError_t wkv5_bwd_split_launch(const float *r, const float *k, const float *v, const float *dy,
+                                  const BwdParams &prm, float *ztot, float *du, cudaStream_t stream);
 // RWKV-4 backward; workspace: [B][T][C] + 2 [B][C] floats (see wkv4_bwd_workspace_bytes)
 // RWKV-5 backward helpers: ew[b][t][c] = -w[c]; dw[c] = -sum_rows dwtok[row][c].
 cudaError_t wkv5_expand_launch(int B, int T, int C, const float *w, float *ew, cudaStream_t stream);

@@ -162,7 +162,10 @@ def test_wkv5_argument_errors(lib):
         assert f(0, 4, 64, 1, *p, None) == WKV_OK
     g = [FAKE + 256 * i for i in range(11)]                    # r, k, v, w, u, dy, dr, dk, dv, dw, du
     ws = wkv.wkv5_bwd_workspace_bytes(2, 8, 128, 2)
-    assert ws == 4 * (2 * 2 * 8 * 128 + 2 * 2 * 128)
+    if wkv.lib_path().endswith("libwkv_recurrence.so"):
+        assert ws == 4 * (2 * 2 * 8 * 128 + 2 * 2 * 128)      # log-decay and per-token dw [B][T][C], 2 [B][C]
+    else:
+        assert ws == (2 * 4 + 2 * 8) * 2 * 128               # 2 [B][C] floats, 2 [B][C] doubles
     f = lib.wkv5_bwd
     assert f(-1, 8, 128, 2, *g, FAKE, ws, None) == WKV_ERR_ARG
     assert f(2, 8, 128, 4, *g, FAKE, ws, None) == WKV_ERR_HEADSIZE

@@ -56,6 +56,22 @@ def test_wkv6_fwd_f32_small(B, T, H, bidir, f32_path):
     assert _rel(y, ref) <= gc.TOL_F32_FWD
 
 
+# The product build runs problems with T <= 256 and at most 32 (b, h) units on the
+# cluster kernel (every chunk at once) and the rest on the chunk-chain kernel; these
+# shapes keep the chain kernel's small and ragged cases covered as well.
+CHAIN_SHAPES = [(5, 33, 7), (6, 100, 6), (1, 257, 2), (3, 31, 11)]
+
+
+@pytest.mark.parametrize("B,T,H", CHAIN_SHAPES)
+@pytest.mark.parametrize("bidir", [False, True])
+def test_wkv6_fwd_f32_chain_kernel_shapes(B, T, H, bidir, f32_path):
+    x = synth.make_wkv6(B, T, H, seed=T * 10 + H + 1)
+    y = gc.run_wkv6_fwd(x, bidir=bidir)
+    ref = gc.oracle_fwd_full(x, bidir)
+    assert np.all(np.isfinite(y))
+    assert _rel(y, ref) <= gc.TOL_F32_FWD
+
+
 BF16_PATHS = ["tensor", "recurrence"]
 
 
