@@ -13,10 +13,15 @@ the 126 MB L2, so every kernel starts cold.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
-For N > 1 launch under torchrun; every rank runs the same per-GPU work on its
-own data (weak scaling, no collective on the data path) and the step time is
-the maximum over ranks.  `--impl reference` times the double-precision CPU
-oracle (the only reference this operator has) on a bounded sample.
+For N > 1 launch under torchrun (NCCL): the step runs on one seeded problem of
+N x B batches, rank r generating and computing its window [rB, (r+1)B) of it
+(weak scaling: B per GPU fixed); the backward's du is all-reduced over the
+ranks inside every step (C floats), the one exchange the batch split needs; the
+step time is the maximum over ranks.  `--only NAME` times single workloads
+(also the ones outside the step), `--library recurrence` the test build of the
+library, and `--impl reference` the double-precision CPU oracle (the only
+reference this operator has) on a bounded sample.  SM clocks, power and
+throttle reasons are sampled through NVML every 2 ms during the timed region.
 """
 from __future__ import annotations
 

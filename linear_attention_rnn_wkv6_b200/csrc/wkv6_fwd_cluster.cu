@@ -22,8 +22,8 @@
 //      into the states entering its own chunk ("How Custom CUDA Kernels
 //      (wkv6_cuda.cu) ...", Forward Pass: the past-to-future state, and the
 //      future-to-past one of the bidirectional form):
-//        S_in  = fold over i = 0 .. j-1 of      F <- diag(Gam_i) F + X_i
-//        Sa_in = fold over i = n-1 .. j+1 of    F <- diag(Gam_i) F + Xa_i
+//        S_in  = sum_{i<j} diag(prod_{m=i+1}^{j-1} Gam_m) X_i
+//        Sa_in = sum_{i>j} diag(prod_{m=j+1}^{i-1} Gam_m) Xa_i
 //   3. Y = A' V + Q S_in + Qa Sa_in with A' = strict-lower(A) + strict-upper(Aa)
 //      + diag(c) (c_p = sum_i r_p u k_p, the bonus), one accumulator, one store.
 // No chunk waits for another chunk's result beyond the one exchange, so the
@@ -106,6 +106,39 @@ __device__ __forceinline__ float4 cl_ld4(uint32_t addr) {
     asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w) : "r"(addr));
     return x;
 }
+// Another CTA's shared memory, eight 16-byte loads at addr + 2048 e (e = 0..7), issued
+// back to back so that their latencies overlap: with addr = row r0 (of a 64 x 64
+// fp32 state), column 4 c4, they are rows r0 + 8 e, columns 4 c4 .. 4 c4 + 3.
+__device__ __forceinline__ void cl_ld_rows8(uint32_t addr, float (&x)[32]) {
+    asm volatile(
+        "ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%32];\n\t"
+        "ld.shared::cluster.v4.f32 {%4, %5, %6, %7}, [%32 + 2048];\n\t"
+        "ld.shared::cluster.v4.f32 {%8, %9, %10, %11}, [%32 + 4096];\n\t"
+        "ld.shared::cluster.v4.f32 {%12, %13, %14, %15}, [%32 + 6144];\n\t"
+        "ld.shared::cluster.v4.f32 {%16, %17, %18, %19}, [%32 + 8192];\n\t"
+        "ld.shared::cluster.v4.f32 {%20, %21, %22, %23}, [%32 + 10240];\n\t"
+        "ld.shared::cluster.v4.f32 {%24, %25, %26, %27}, [%32 + 12288];\n\t"
+        "ld.shared::cluster.v4.f32 {%28, %29, %30, %31}, [%32 + 14336];"
+        : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]), "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7]),
+          "=f"(x[8]), "=f"(x[9]), "=f"(x[10]), "=f"(x[11]), "=f"(x[12]), "=f"(x[13]), "=f"(x[14]), "=f"(x[15]),
+          "=f"(x[16]), "=f"(x[17]), "=f"(x[18]), "=f"(x[19]), "=f"(x[20]), "=f"(x[21]), "=f"(x[22]), "=f"(x[23]),
+          "=f"(x[24]), "=f"(x[25]), "=f"(x[26]), "=f"(x[27]), "=f"(x[28]), "=f"(x[29]), "=f"(x[30]), "=f"(x[31])
+        : "r"(addr));
+}
+// The decay totals of rows r0 + 8 e (e = 0..7) of another CTA, from addr = its gam[r0].
+__device__ __forceinline__ void cl_ld_gam8(uint32_t addr, float (&g)[8]) {
+    asm volatile(
+        "ld.shared::cluster.f32 %0, [%8];\n\t"
+        "ld.shared::cluster.f32 %1, [%8 + 32];\n\t"
+        "ld.shared::cluster.f32 %2, [%8 + 64];\n\t"
+        "ld.shared::cluster.f32 %3, [%8 + 96];\n\t"
+        "ld.shared::cluster.f32 %4, [%8 + 128];\n\t"
+        "ld.shared::cluster.f32 %5, [%8 + 160];\n\t"
+        "ld.shared::cluster.f32 %6, [%8 + 192];\n\t"
+        "ld.shared::cluster.f32 %7, [%8 + 224];"
+        : "=f"(g[0]), "=f"(g[1]), "=f"(g[2]), "=f"(g[3]), "=f"(g[4]), "=f"(g[5]), "=f"(g[6]), "=f"(g[7])
+        : "r"(addr));
+}
 __device__ __forceinline__ float cl_ld1(uint32_t addr) {
     float x;
     asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(addr));
@@ -174,6 +207,22 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     const size_t nBTC = (size_t)prm.B * T * C;
 
+    // ---- load the chunk first (tokens pq .. pq + 7 of this warp, channels ch, ch + 1): its
+    // latency overlaps the set-up below
+    float2 xr_[8], xk_[8], xv_[8], xw_[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int p = pq + e;
+        if (p < n) {
+            const size_t o = ((size_t)b * T + t0 + p) * C + cbase + ch;
+            xr_[e] = __ldg(reinterpret_cast<const float2 *>(r + o));
+            xk_[e] = __ldg(reinterpret_cast<const float2 *>(k + o));
+            xv_[e] = __ldg(reinterpret_cast<const float2 *>(v + o));
+            xw_[e] = __ldg(reinterpret_cast<const float2 *>(w + o));
+        } else {
+            xr_[e] = xk_[e] = xv_[e] = xw_[e] = make_float2(0.f, 0.f);
+        }
+    }
     if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
     if (tid == 0) {
         mbar_init(&sm.bar_a, 1);
@@ -192,21 +241,6 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
     const uint32_t tX = sm.tmem_base, tXa = sm.tmem_base + 64, tA = sm.tmem_base + 128, tAa = sm.tmem_base + 160,
                    tY = sm.tmem_base + 192;
 
-    // ---- load the chunk (tokens pq .. pq + 7 of this warp, channels ch, ch + 1)
-    float2 xr_[8], xk_[8], xv_[8], xw_[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const int p = pq + e;
-        if (p < n) {
-            const size_t o = ((size_t)b * T + t0 + p) * C + cbase + ch;
-            xr_[e] = __ldg(reinterpret_cast<const float2 *>(r + o));
-            xk_[e] = __ldg(reinterpret_cast<const float2 *>(k + o));
-            xv_[e] = __ldg(reinterpret_cast<const float2 *>(v + o));
-            xw_[e] = __ldg(reinterpret_cast<const float2 *>(w + o));
-        } else {
-            xr_[e] = xk_[e] = xv_[e] = xw_[e] = make_float2(0.f, 0.f);
-        }
-    }
     // ---- decay sums: this warp's quarter, then the prefix and the total per channel
     {
         float s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
@@ -417,74 +451,110 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
     }
     cl_barrier();   // every chunk's X, Xa and Gam are published
 
-    // ===== fold: the states entering this chunk, thread (row i, 32 columns) =====
-    {
-        const int i = tid >> 1, c0 = 32 * (tid & 1);
-        float f[32];
+    // ===== fold: the states entering this chunk,
+    //   S_in  = sum_{q<j} diag(prod_{m=q+1}^{j-1} Gam_m) X_q,
+    //   Sa_in = sum_{q>j} diag(prod_{m=j+1}^{q-1} Gam_m) Xa_q,
+    // taken from the nearest chunk outwards with the decay product kept per row, so
+    // that the CTAs' first remote reads go to different SMs.  Thread (warp w, lane l)
+    // holds rows r0 + 8 e (r0 = 2 w + l / 16, e = 0..7), columns 4 (l % 16) .. + 3, so
+    // that each remote load instruction of a warp reads 512 contiguous bytes (two rows;
+    // no bank conflicts).  The remote reads dominate, so two chunks' states are in
+    // flight per step: the next two causal predecessors, or (bidirectional) the next
+    // causal predecessor and the next anti-causal successor =====
+    if (live) {
+        const int r0 = 2 * warp + (lane >> 4), c4 = 4 * (lane & 15);
+        float fc[32], fa[32];   // [e][4]: row r0 + 8 e, columns c4 .. c4 + 3
+        float pc[8], pa[8];     // decay products between the next chunk read and this one, per row
 #pragma unroll
-        for (int e = 0; e < 32; ++e) f[e] = 0.f;
-        // causal: F <- diag(Gam_q) F + X_q for q = 0 .. j-1
-        for (int q = 0; q < (int)j; ++q) {
-            const float g = cl_ld1(cl_map(&sm.gam[i], q));
-            const uint32_t base = cl_map(&sm.X[i][c0], q);
+        for (int e = 0; e < 32; ++e) fc[e] = fa[e] = 0.f;
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                const float4 x = cl_ld4(base + 16 * e4);
-                f[4 * e4] = fmaf(g, f[4 * e4], x.x);
-                f[4 * e4 + 1] = fmaf(g, f[4 * e4 + 1], x.y);
-                f[4 * e4 + 2] = fmaf(g, f[4 * e4 + 2], x.z);
-                f[4 * e4 + 3] = fmaf(g, f[4 * e4 + 3], x.w);
+        for (int e = 0; e < 8; ++e) pc[e] = pa[e] = 1.f;
+        int qc = (int)j - 1, qa = (int)j + 1;   // next causal predecessor (down), anti-causal successor (up)
+        while (qc >= 0 || (BIDIR && qa < nch)) {
+            float x0[32], x1[32], g0[8], g1[8];
+            // first item: a causal predecessor if one is left, else an anti-causal successor
+            const bool first_c = qc >= 0;
+            const int q_first = first_c ? qc : qa;
+            // second item: bidirectional, the anti-causal successor (when the first was causal);
+            // causal only, the next causal predecessor
+            bool second = false, second_c = false;
+            int q_second = 0;
+            if (BIDIR) {
+                if (first_c && qa < nch) {
+                    second = true;
+                    q_second = qa;
+                }
+            } else if (qc - 1 >= 0) {
+                second = true;
+                second_c = true;
+                q_second = qc - 1;
+            }
+            cl_ld_rows8(cl_map(first_c ? &sm.X[r0][c4] : &sm.Xa[r0][c4], q_first), x0);
+            cl_ld_gam8(cl_map(&sm.gam[r0], q_first), g0);
+            if (second) {
+                cl_ld_rows8(cl_map(second_c ? &sm.X[r0][c4] : &sm.Xa[r0][c4], q_second), x1);
+                cl_ld_gam8(cl_map(&sm.gam[r0], q_second), g1);
+            }
+            // F += P X_q, then P *= Gam_q
+            if (first_c) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) fc[e] = fmaf(pc[e >> 2], x0[e], fc[e]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pc[e] *= g0[e];
+                --qc;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) fa[e] = fmaf(pa[e >> 2], x0[e], fa[e]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pa[e] *= g0[e];
+                ++qa;
+            }
+            if (second) {
+                if (second_c) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) fc[e] = fmaf(pc[e >> 2], x1[e], fc[e]);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) pc[e] *= g1[e];
+                    --qc;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) fa[e] = fmaf(pa[e >> 2], x1[e], fa[e]);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) pa[e] *= g1[e];
+                    ++qa;
+                }
             }
         }
         if (!exact) {
-            // three-term copy into the MN-major S_in tile (row i, columns c0 .. c0 + 31)
+            // three-term copies into the MN-major S_in tiles: 4 columns (8 bytes) per row and term
 #pragma unroll
-            for (int e8 = 0; e8 < 4; ++e8) {
-                uint32_t t[3][8];
+            for (int e = 0; e < 8; ++e) {
+                const int row = r0 + 8 * e;
+                const uint32_t o = swz(row, c4);
+                uint32_t t[3][4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) csplit3(f[8 * e8 + e], t[0][e], t[1][e], t[2][e]);
-                const uint32_t o = swz(i, c0 + 8 * e8);
+                for (int m = 0; m < 4; ++m) csplit3(fc[4 * e + m], t[0][m], t[1][m], t[2][m]);
 #pragma unroll
                 for (int q = 0; q < 3; ++q)
-                    st_u128(sm.Sin[q], o, make_uint4(cpack(t[q][0], t[q][1]), cpack(t[q][2], t[q][3]),
-                                                     cpack(t[q][4], t[q][5]), cpack(t[q][6], t[q][7])));
+                    *reinterpret_cast<uint2 *>(reinterpret_cast<char *>(sm.Sin[q]) + o) =
+                        make_uint2(cpack(t[q][0], t[q][1]), cpack(t[q][2], t[q][3]));
+                if (BIDIR) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) csplit3(fa[4 * e + m], t[0][m], t[1][m], t[2][m]);
+#pragma unroll
+                    for (int q = 0; q < 3; ++q)
+                        *reinterpret_cast<uint2 *>(reinterpret_cast<char *>(sm.Sain[q]) + o) =
+                            make_uint2(cpack(t[q][0], t[q][1]), cpack(t[q][2], t[q][3]));
+                }
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) xs.S[i][c0 + e] = f[e];
-        }
-        if (BIDIR) {
-            // anti-causal: F <- diag(Gam_q) F + Xa_q for q = nch-1 .. j+1
+            for (int e = 0; e < 8; ++e)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) f[e] = 0.f;
-            for (int q = nch - 1; q > (int)j; --q) {
-                const float g = cl_ld1(cl_map(&sm.gam[i], q));
-                const uint32_t base = cl_map(&sm.Xa[i][c0], q);
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 x = cl_ld4(base + 16 * e4);
-                    f[4 * e4] = fmaf(g, f[4 * e4], x.x);
-                    f[4 * e4 + 1] = fmaf(g, f[4 * e4 + 1], x.y);
-                    f[4 * e4 + 2] = fmaf(g, f[4 * e4 + 2], x.z);
-                    f[4 * e4 + 3] = fmaf(g, f[4 * e4 + 3], x.w);
+                for (int m = 0; m < 4; ++m) {
+                    xs.S[r0 + 8 * e][c4 + m] = fc[4 * e + m];
+                    if (BIDIR) xs.Sa[r0 + 8 * e][c4 + m] = fa[4 * e + m];
                 }
-            }
-            if (!exact) {
-#pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) {
-                    uint32_t t[3][8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) csplit3(f[8 * e8 + e], t[0][e], t[1][e], t[2][e]);
-                    const uint32_t o = swz(i, c0 + 8 * e8);
-#pragma unroll
-                    for (int q = 0; q < 3; ++q)
-                        st_u128(sm.Sain[q], o, make_uint4(cpack(t[q][0], t[q][1]), cpack(t[q][2], t[q][3]),
-                                                          cpack(t[q][4], t[q][5]), cpack(t[q][6], t[q][7])));
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) xs.Sa[i][c0 + e] = f[e];
-            }
         }
     }
     fence_proxy_async_smem();
