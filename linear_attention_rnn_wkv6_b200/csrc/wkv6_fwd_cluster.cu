@@ -162,7 +162,7 @@ struct ClusterSmem {
     float cp[kCL];                      // bonus scalars per token
     float u[kHead];
     uint32_t tmem_base;
-    alignas(8) uint64_t bar_a, bar_y, bar_fin;
+    alignas(8) uint64_t bar_a, bar_a2, bar_y, bar_y2, bar_fin;
 };
 static_assert(offsetof(ClusterSmem, Q) % 1024 == 0 && offsetof(ClusterSmem, Kt) % 1024 == 0 &&
                   offsetof(ClusterSmem, Qa) % 1024 == 0 && offsetof(ClusterSmem, Kta) % 1024 == 0 &&
@@ -226,8 +226,10 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
     if (tid < kHead) sm.u[tid] = prm.u[cbase + tid];
     if (tid == 0) {
         mbar_init(&sm.bar_a, 1);
+        mbar_init(&sm.bar_a2, 1);
         mbar_init(&sm.bar_y, 1);
-        mbar_init(&sm.bar_fin, 1);
+        mbar_init(&sm.bar_y2, 1);
+        mbar_init(&sm.bar_fin, 2);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -237,9 +239,10 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    // TMEM (M = 64 layouts): X at 0..63, Xa at 64..127, A at 128..159, Aa at 160..191, Y at 192..255
+    // TMEM (M = 64 layouts): X at 0..63, Xa at 64..127, A at 128..159, Aa at 160..191, Y at 192..255;
+    // the second Y accumulator (Q S_in) reuses X's columns once X is in shared memory
     const uint32_t tX = sm.tmem_base, tXa = sm.tmem_base + 64, tA = sm.tmem_base + 128, tAa = sm.tmem_base + 160,
-                   tY = sm.tmem_base + 192;
+                   tY = sm.tmem_base + 192, tY2 = sm.tmem_base;
 
     // ---- decay sums: this warp's quarter, then the prefix and the total per channel
     {
@@ -326,14 +329,11 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
     const uint64_t dS = desc_mn(sm.Sin[0], 0, 16), dSa = desc_mn(sm.Sain[0], 0, 16);
 
     if (!exact) {
-        // ===== X = Kt^T V, A = Q Kt^T (and Xa, Aa): one issuing thread =====
+        // ===== X = Kt^T V, A = Q Kt^T (and Xa, Aa): two issuing threads (one thread issues
+        // an MMA about every 47 cycles; a second issuer nearly halves the group's time).
+        // Causal: thread 0 issues A, thread 32 X.  Bidirectional: thread 0 A and X, thread
+        // 32 Aa and Xa =====
         if (tid == 0) {
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-                for (int q = 0; q < kCNP; ++q)
-                    mma_bf16(tX, cdadd(dKm, cprod_a(q) * kTokB + 2048 * ks), cdadd(dV, cprod_b(q) * kTokB + 2048 * ks),
-                             kIdX, ks > 0 || q > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
@@ -345,18 +345,35 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
                 for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
                     for (int q = 0; q < kCNP; ++q)
-                        mma_bf16(tXa, cdadd(dKam, cprod_a(q) * kTokB + 2048 * ks),
-                                 cdadd(dV, cprod_b(q) * kTokB + 2048 * ks), kIdX, ks > 0 || q > 0);
+                        mma_bf16(tX, cdadd(dKm, cprod_a(q) * kTokB + 2048 * ks), cdadd(dV, cprod_b(q) * kTokB + 2048 * ks),
+                                 kIdX, ks > 0 || q > 0);
+            }
+            mma_commit(&sm.bar_a);
+        } else if (tid == 32) {
+            if (BIDIR) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
                     for (int q = 0; q < kCNP; ++q)
                         mma_bf16(tAa, cdadd(dQa, cprod_a(q) * kTokB + 32 * ks),
                                  cdadd(dKak, cprod_b(q) * kTokB + 32 * ks), kIdA, ks > 0 || q > 0);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                    for (int q = 0; q < kCNP; ++q)
+                        mma_bf16(tXa, cdadd(dKam, cprod_a(q) * kTokB + 2048 * ks),
+                                 cdadd(dV, cprod_b(q) * kTokB + 2048 * ks), kIdX, ks > 0 || q > 0);
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                    for (int q = 0; q < kCNP; ++q)
+                        mma_bf16(tX, cdadd(dKm, cprod_a(q) * kTokB + 2048 * ks), cdadd(dV, cprod_b(q) * kTokB + 2048 * ks),
+                                 kIdX, ks > 0 || q > 0);
             }
-            mma_commit(&sm.bar_a);
+            mma_commit(&sm.bar_a2);
         }
-        ok = mbar_wait_bounded(&sm.bar_a, 0);
+        ok = mbar_wait_bounded(&sm.bar_a, 0) && mbar_wait_bounded(&sm.bar_a2, 0);
         ok = __syncthreads_and(ok);
         fence_after_sync();
         if (ok) {
@@ -563,7 +580,9 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
     fence_after_sync();
 
     if (!exact) {
-        // ===== Y = A' V + Q S_in + Qa Sa_in =====
+        // ===== Y = A' V + Qa Sa_in (thread 0, accumulator Y) and Q S_in (thread 32, accumulator
+        // Y2 in X's columns), summed in the epilogue =====
+        const bool has_s = j > 0, has_sa = BIDIR && (int)j < nch - 1;
         if (tid == 0 && ok) {
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks)
@@ -571,15 +590,7 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
                 for (int q = 0; q < kCNP; ++q)
                     mma_bf16(tY, cdadd(dAp, cprod_a(q) * kApB + 1024 * ks), cdadd(dV, cprod_b(q) * kTokB + 2048 * ks),
                              kIdAV, ks > 0 || q > 0);
-            if (j > 0) {
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-                    for (int q = 0; q < kCNP; ++q)
-                        mma_bf16(tY, cdadd(dQ, cprod_a(q) * kTokB + 32 * ks), cdadd(dS, cprod_b(q) * kStB + 2048 * ks),
-                                 kIdQS, true);
-            }
-            if (BIDIR && (int)j < nch - 1) {
+            if (has_sa) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
@@ -588,13 +599,28 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
                                  cdadd(dSa, cprod_b(q) * kStB + 2048 * ks), kIdQS, true);
             }
             mma_commit(&sm.bar_y);
+        } else if (tid == 32 && ok && has_s) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                for (int q = 0; q < kCNP; ++q)
+                    mma_bf16(tY2, cdadd(dQ, cprod_a(q) * kTokB + 32 * ks), cdadd(dS, cprod_b(q) * kStB + 2048 * ks),
+                             kIdQS, ks > 0 || q > 0);
+            mma_commit(&sm.bar_y2);
         }
-        if (ok) ok = mbar_wait_bounded(&sm.bar_y, 0);
+        if (ok) ok = mbar_wait_bounded(&sm.bar_y, 0) && (!has_s || mbar_wait_bounded(&sm.bar_y2, 0));
         ok = __syncthreads_and(ok);
         fence_after_sync();
         if (ok && warp < 2 && live) {
             float yv[32];
             tmem_ld_16x256b_x8(tY + lane_off, yv);
+            if (has_s) {
+                float y2[32];
+                tmem_ld_16x256b_x8(tY2 + lane_off, y2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) yv[e] += y2[e];
+            }
             tmem_wait_ld();
             const int q4 = lane & 3;
 #pragma unroll
@@ -655,10 +681,11 @@ wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k
             __syncthreads();
         }
     }
-    if (!ok && tid == 0) {
-        // a wait ran out: let every MMA issued so far finish before TMEM is released
+    if (!ok && (tid == 0 || tid == 32)) {
+        // a wait ran out: let every MMA issued so far (by both issuing threads) finish
+        // before TMEM is released
         mma_commit(&sm.bar_fin);
-        mbar_wait_bounded(&sm.bar_fin, 0);
+        if (tid == 0) mbar_wait_bounded(&sm.bar_fin, 0);
     }
     // no CTA leaves (or frees its shared memory) while another may still read it
     cl_barrier();
