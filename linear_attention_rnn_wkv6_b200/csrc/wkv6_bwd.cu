@@ -133,7 +133,7 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     constexpr uint32_t kStageBytes = 5u * TC * kHead * sizeof(Tin);
     constexpr uint32_t kPartBytes = 4u * TC * kHead * sizeof(float);
     extern __shared__ unsigned char smem_dyn[];
-    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~uintptr_t(127));
+    Smem &sm = *reinterpret_cast<Smem *>(smem_dyn + ((128u - (smem_u32(smem_dyn) & 127u)) & 127u));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = prm.T, C = prm.C, H = prm.H;

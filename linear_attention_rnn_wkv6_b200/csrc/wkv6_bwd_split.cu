@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
                                                               const Tin *__restrict__ dy, BwdParams prm,
                                                               float *__restrict__ ztot) {
     extern __shared__ unsigned char smem_dyn[];
-    SSmem &sm = *reinterpret_cast<SSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    SSmem &sm = *reinterpret_cast<SSmem *>(smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     BDecay &ds = *reinterpret_cast<BDecay *>(&sm.dAp[0][0]);
     SExact &xe = *reinterpret_cast<SExact *>(&sm.dY[0][0]);
     float(*xdy)[kHead] = reinterpret_cast<float(*)[kHead]>(&sm.Sin[0][0]);
@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                                                               const Tin *__restrict__ dy, BwdParams prm,
                                                               const float *__restrict__ ztot) {
     extern __shared__ unsigned char smem_dyn[];
-    GSmem &sm = *reinterpret_cast<GSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    GSmem &sm = *reinterpret_cast<GSmem *>(smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     BDecay &ds = *reinterpret_cast<BDecay *>(&sm.Ap[0][0]);
     GExact &xe = *reinterpret_cast<GExact *>(&sm.Q[0][0]);
     float *part = reinterpret_cast<float *>(&sm.Gt[0][0]);

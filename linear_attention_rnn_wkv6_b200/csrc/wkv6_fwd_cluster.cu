@@ -189,7 +189,7 @@ __global__ void __cluster_dims__(kCw, 1, 1) __launch_bounds__(kCThr, 1)
 wkv6_fwd_cluster_kernel(const float *__restrict__ r, const float *__restrict__ k, const float *__restrict__ v,
                         const float *__restrict__ w, FwdParams prm) {
     extern __shared__ unsigned char smem_dyn[];
-    ClusterSmem &sm = *reinterpret_cast<ClusterSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    ClusterSmem &sm = *reinterpret_cast<ClusterSmem *>(smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     ClusterExact &xr = *reinterpret_cast<ClusterExact *>(&sm.Q[0][0]);
     ClusterExactState &xs = *reinterpret_cast<ClusterExactState *>(&sm.Sin[0][0]);
 

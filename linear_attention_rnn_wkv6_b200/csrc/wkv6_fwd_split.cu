@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                                                                  const float *__restrict__ v,
                                                                  const float *__restrict__ w, FwdParams prm) {
     extern __shared__ unsigned char smem_dyn[];
-    SplitSmem &sm = *reinterpret_cast<SplitSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    SplitSmem &sm = *reinterpret_cast<SplitSmem *>(smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
     DecaySums &ds = *reinterpret_cast<DecaySums *>(&sm.Ap[0][0]);
     ExactRaw &xr = *reinterpret_cast<ExactRaw *>(&sm.Q[0][0]);
     float *part = reinterpret_cast<float *>(&sm.Sin[0][0]);

@@ -145,7 +145,7 @@ wkv6_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_const
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
                    const __grid_constant__ CUtensorMap map_y, FwdParams prm) {
     extern __shared__ unsigned char smem_dyn[];
-    TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    TcSmem &sm = *reinterpret_cast<TcSmem *>(smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = prm.T, C = prm.C, H = prm.H;
