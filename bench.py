@@ -471,9 +471,14 @@ def run_native(args, rank, world, local):
     torch.cuda.set_device(local)
     dist = init_group("nccl", world)
     dev = torch.device("cuda", local)
-    if args.library != "default":
-        wkv.use_library(args.library).__enter__()   # for the rest of this process
+    # the selected build for the rest of this process (the context manager is kept
+    # referenced: a generator context dropped after __enter__ would be closed, and its
+    # exit would restore the default build)
+    library_ctx = wkv.use_library(args.library)
+    library_ctx.__enter__()
     wkv.load()
+    if os.path.basename(wkv.lib_path()) != wkv.LIBRARY_FILES[args.library]:
+        raise RuntimeError(f"library {args.library!r} not selected")
     wls = [DeviceWorkload(n, rank, world) for n in (args.only or STEP_WORKLOADS)]
     stream = torch.cuda.Stream()
     tokens_per_step = sum(w.tokens for w in wls)

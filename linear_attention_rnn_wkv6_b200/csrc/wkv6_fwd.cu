@@ -106,7 +106,7 @@ wkv6_fwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
     constexpr uint32_t kStageBytes = (3 * TC * kHead + TC * CW) * sizeof(Tin);
     constexpr uint32_t kWBytes = TC * kHead * sizeof(Tin);
     extern __shared__ unsigned char smem_dyn[];
-    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~uintptr_t(127));
+    Smem &sm = *reinterpret_cast<Smem *>(smem_dyn + ((128u - (smem_u32(smem_dyn) & 127u)) & 127u));
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -471,16 +471,24 @@ cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const 
                             const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
                             cudaStream_t stream) {
     constexpr int TC = kFwdTC;
-    // The fp32 causal form serves wkv6_fwd_state and wkv5_fwd in every build.  The
-    // bf16 causal and fp32 bidirectional forms are reached only in the library built
-    // with WKV_RECURRENCE_PATHS, whose chunked-form entry points run this kernel.
+    // Reached only in the library built with WKV_RECURRENCE_PATHS: there the bf16
+    // causal forward and the fused fp32 forwards run this kernel (the other fp32
+    // forwards run the pipelined recurrence in every build).
 #if WKV_RECURRENCE_PATHS
     if (bf16) return bidir ? cudaErrorNotSupported : launch_fwd<__nv_bfloat16, 4, TC, false>(mr, mk, mv, mw, prm, stream);
     if (bidir) return launch_fwd<float, 4, TC, true>(mr, mk, mv, mw, prm, stream);
-#else
-    if (bf16 || bidir) return cudaErrorNotSupported;
-#endif
     return launch_fwd<float, 4, TC, false>(mr, mk, mv, mw, prm, stream);
+#else
+    (void)bf16;
+    (void)bidir;
+    (void)mr;
+    (void)mk;
+    (void)mv;
+    (void)mw;
+    (void)prm;
+    (void)stream;
+    return cudaErrorNotSupported;
+#endif
 }
 
 }  // namespace wkv

@@ -201,6 +201,8 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
                                                 reinterpret_cast<cudaStream_t>(stream)));
     }
     if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && kTensorCorePaths) {
+        // the chunked form (faster than the register recurrence at these sizes), with
+        // the decay prologue and norm/gate epilogue when fused
         FwdParams prm{B, T, C, H, u, y};
         if (fused != nullptr) {
             prm.wb = fused->wb;
@@ -222,6 +224,11 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
     prm.s0 = s0;
     prm.sT = sT;
     prm.w5 = w5;
+    if (!bf16 && fused == nullptr)
+        // fp32 without the fused prologue/epilogue: the register recurrence fed by a
+        // transform warp (in the product build only with an initial or final state or
+        // a static decay, which the chunked forms do not take)
+        return launched(wkv6_fwd_pipe_launch(bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)));
     if (fused != nullptr) {
         prm.wb = fused->wb;
         prm.g = fused->g;

@@ -57,6 +57,11 @@ cudaError_t wkv6_fwd_split_launch(bool bidir, const float *r, const float *k, co
 bool wkv6_fwd_cluster_fits(int B, int T, int H);
 cudaError_t wkv6_fwd_cluster_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
                                     const FwdParams &prm, cudaStream_t stream);
+// fp32 causal or bidirectional forward as a register recurrence: four warps hold a
+// head's state, a fifth stages and transforms the inputs (maps: fp32, box 64
+// channels x kFwdTC tokens); supports s0/sT (causal) and w5, not the fused forms.
+cudaError_t wkv6_fwd_pipe_launch(bool bidir, const CUtensorMap &mr, const CUtensorMap &mk, const CUtensorMap &mv,
+                                 const CUtensorMap &mw, const FwdParams &prm, cudaStream_t stream);
 // One recurrent step for B sequences (state [B][H][N][N] updated in place).
 cudaError_t wkv6_decode_launch(int B, int C, int H, const float *r, const float *k, const float *v,
                                const float *w, const float *u, float *state, float *y, cudaStream_t stream);

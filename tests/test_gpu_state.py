@@ -60,16 +60,34 @@ def test_fwd_state_matches_oracle(B, T, H, with_s0):
     assert _rel(sT, so) <= gc.TOL_F32_FWD, _rel(sT, so)
 
 
-def test_fwd_state_without_s0_equals_plain_forward():
-    """No initial state is the zero state: bit-identical to the plain forward on the
-    same (recurrence) kernel, and within the fp32 tolerance of the tensor-core path."""
+@pytest.mark.parametrize("library", ["default", "recurrence"])
+def test_fwd_state_without_s0_is_the_zero_state(library):
+    """No initial state is the zero state: the same bits as an explicit zero s0 (both
+    builds run the state form on the register recurrence)."""
     x = synth.make_wkv6(2, 150, 3, seed=310)
-    y, _ = _run_state(x, None)
+    with gc.library_for(library):
+        y, sT = _run_state(x, None)
+        yz, sTz = _run_state(x, np.zeros((x.B, x.H, 64, 64), np.float32))
+    assert np.array_equal(y, yz) and np.array_equal(sT, sTz)
+
+
+def test_fwd_state_without_s0_equals_plain_forward_on_the_same_kernel():
+    """In the test build the plain forward runs the same register recurrence as the
+    state form: bit-identical outputs."""
+    x = synth.make_wkv6(2, 300, 3, seed=311)
     with gc.library_for("recurrence"):
+        y, _ = _run_state(x, None)
         assert np.array_equal(y, gc.run_wkv6_fwd(x))
+
+
+@pytest.mark.parametrize("T", [150, 300])
+def test_fwd_state_without_s0_near_chunked_forward(T):
+    """Product build: the plain forward takes a chunked form (the cluster form at
+    T = 150, the chunk chain at T = 300), the state form the register recurrence;
+    both within the fp32 tolerance of each other."""
+    x = synth.make_wkv6(2, T, 3, seed=312)
+    y, _ = _run_state(x, None)
     assert _rel(y, gc.run_wkv6_fwd(x)) <= gc.TOL_F32_FWD
-
-
 @pytest.mark.parametrize("cut", [1, 16, 77, 199])
 def test_fwd_state_split_sequence(cut):
     """Two calls over [0, cut) and [cut, T) with the carried state match one call and the oracle."""
