@@ -100,13 +100,8 @@ __device__ __forceinline__ uint32_t cl_map(const void *local, uint32_t rank) {
     asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
     return remote;
 }
-// Loads from another CTA's shared memory, after a cluster barrier that ordered its stores.
-__device__ __forceinline__ float4 cl_ld4(uint32_t addr) {
-    float4 x;
-    asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w) : "r"(addr));
-    return x;
-}
-// Another CTA's shared memory, eight 16-byte loads at addr + 2048 e (e = 0..7), issued
+// Loads from another CTA's shared memory, after a cluster barrier that ordered its
+// stores.  Eight 16-byte loads at addr + 2048 e (e = 0..7), issued
 // back to back so that their latencies overlap: with addr = row r0 (of a 64 x 64
 // fp32 state), column 4 c4, they are rows r0 + 8 e, columns 4 c4 .. 4 c4 + 3.
 __device__ __forceinline__ void cl_ld_rows8(uint32_t addr, float (&x)[32]) {
@@ -139,12 +134,6 @@ __device__ __forceinline__ void cl_ld_gam8(uint32_t addr, float (&g)[8]) {
         : "=f"(g[0]), "=f"(g[1]), "=f"(g[2]), "=f"(g[3]), "=f"(g[4]), "=f"(g[5]), "=f"(g[6]), "=f"(g[7])
         : "r"(addr));
 }
-__device__ __forceinline__ float cl_ld1(uint32_t addr) {
-    float x;
-    asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(addr));
-    return x;
-}
-
 struct ClusterSmem {
     // token tiles (32 rows of 64 bf16, 128B-swizzled), time order
     __nv_bfloat16 Q[kCNT][kCTok];       // K-major A of A = Q Kt^T and of Y += Q S_in
