@@ -367,7 +367,7 @@ class DeviceWorkload:
             self.outputs = [torch.empty(shape, device="cuda")]
         if self.kind == "wkv6_decode":
             # the recurrent state stays resident on the device (updated in place every step)
-            self.state = dev(synth.make_state(x.B, x.H, seed=seed))
+            self.state = dev(synth.make_state(x.B, x.H, seed=1000 * rank + 1))
         self.units = units_of(name, x)
         self.tokens = tokens_of(x)
 

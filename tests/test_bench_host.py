@@ -49,3 +49,22 @@ def test_default_step_is_not_flushed_and_small_workloads_are():
     assert step > bench.FLUSH_BYTES          # the step's kernels start cold without a flush
     assert _bytes_of("wkv4_f32_b8t1024c768") < bench.FLUSH_BYTES       # alone it would stay in L2
     assert _bytes_of("wkv6_bidir_f32_b32t196h12") < bench.FLUSH_BYTES
+
+
+def test_every_workload_constructs_on_the_host(monkeypatch):
+    """Each workload bench.py can time builds its inputs, outputs, workspace and state
+    (device copies redirected to host tensors), alone and as rank 1 of 2; the batch
+    window of a split workload has the rank's share of the units."""
+    monkeypatch.setattr(torch.Tensor, "cuda", lambda self, *a, **k: self)
+    empty = torch.empty
+
+    def host_empty(*a, **k):
+        k.pop("device", None)
+        return empty(*a, **k)
+
+    monkeypatch.setattr(torch, "empty", host_empty)
+    for name in bench.STEP_WORKLOADS + bench.EXTRA_WORKLOADS:
+        one = bench.DeviceWorkload(name, 0, 1)
+        two = bench.DeviceWorkload(name, 1, 2)
+        assert one.units > 0 and one.tokens > 0 and one.footprint() > 0, name
+        assert two.units == one.units and two.tokens == one.tokens, name   # weak scaling: B per rank fixed
