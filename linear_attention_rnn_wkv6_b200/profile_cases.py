@@ -1,6 +1,6 @@
 """Run hot-path kernels a fixed number of times, for profilers.
 
-    python -m linear_attention_rnn_wkv6_b200.profile_cases [--case NAME[:B:T]] ... [--rounds R]
+    python -m linear_attention_rnn_wkv6_b200.profile_cases [--case NAME[:B:T]] ... [--rounds R] [--library L]
 
 Each case is one of the benchmark's workloads (``synth.WORKLOADS``),
 optionally with its batch B and length T replaced, so that a profiler can
@@ -94,13 +94,16 @@ def main(argv=None) -> int:
     ap.add_argument("--case", action="append", required=True,
                     help="workload name from synth.WORKLOADS, optionally NAME:B:T")
     ap.add_argument("--rounds", type=int, default=2)
+    ap.add_argument("--library", choices=sorted(wkv.LIBRARY_FILES), default="default",
+                    help="the library build whose kernels run (recurrence: the test build)")
     a = ap.parse_args(argv)
-    cases = [make_case(c) for c in a.case]
-    for _ in range(a.rounds):
-        for _, run in cases:
-            run()
-    torch.cuda.synchronize()
-    faults = wkv.wkv_take_device_faults()
+    with wkv.use_library(a.library):
+        cases = [make_case(c) for c in a.case]
+        for _ in range(a.rounds):
+            for _, run in cases:
+                run()
+        torch.cuda.synchronize()
+        faults = wkv.wkv_take_device_faults()
     for label, _ in cases:
         print(label)
     if faults:
