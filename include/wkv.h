@@ -32,10 +32,11 @@
  * wkv5_fwd and wkv6_bwd_noalloc use in both builds).  Results agree within the
  * tolerances stated below; nothing is selected at run time.  A third build,
  * libwkv_debug.so (-DWKV_DEVICE_CHECKS=1), is libwkv.so with an index check on
- * every global store of every kernel: an index outside the array skips the store
- * and records WKV_FAULT_INDEX (nothing traps), and every entry point then waits
- * for its kernels and returns WKV_ERR_DEVICE_CHECK (or WKV_ERR_TIMEOUT for a
- * bounded wait that ran out) instead of WKV_OK.
+ * every global store of every kernel (and every L2 prefetch of an output row):
+ * an index outside the array skips the access and records WKV_FAULT_INDEX
+ * (nothing traps), and every entry point then waits for its kernels and returns
+ * WKV_ERR_DEVICE_CHECK (or WKV_ERR_TIMEOUT for a bounded wait that ran out)
+ * instead of WKV_OK.
  *
  * RWKV-6 log-decay
  * ----------------

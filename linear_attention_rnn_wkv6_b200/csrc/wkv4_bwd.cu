@@ -200,13 +200,30 @@ __global__ void wkv4_bwd_reduce_kernel(int B, int C, const float *__restrict__ d
                                        float *__restrict__ du) {
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= C) return;
+    // eight batches' loads in flight at a time; the additions stay in increasing b
     float sw = 0.f, su = 0.f;
-    for (int b = 0; b < B; ++b) {
+    int b = 0;
+    for (; b + 8 <= B; b += 8) {
+        float xw[8], xu[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            xw[e] = dw_part[(size_t)(b + e) * C + c];
+            xu[e] = du_part[(size_t)(b + e) * C + c];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            sw += xw[e];
+            su += xu[e];
+        }
+    }
+    for (; b < B; ++b) {
         sw += dw_part[(size_t)b * C + c];
         su += du_part[(size_t)b * C + c];
     }
-    dw[c] = sw;
-    du[c] = su;
+    if (in_range(c, (size_t)C)) {
+        dw[c] = sw;
+        du[c] = su;
+    }
 }
 
 }  // namespace

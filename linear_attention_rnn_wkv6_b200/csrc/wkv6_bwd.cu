@@ -453,9 +453,18 @@ wkv6_bwd_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant
 __global__ void wkv6_du_reduce_kernel(int B, int C, const float *__restrict__ part, float *__restrict__ du) {
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= C) return;
+    // eight loads in flight at a time; the additions stay in increasing b
     float acc = 0.f;
-    for (int b = 0; b < B; ++b) acc += part[(size_t)b * C + c];
-    du[c] = acc;
+    int b = 0;
+    for (; b + 8 <= B; b += 8) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = part[(size_t)(b + e) * C + c];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc += x[e];
+    }
+    for (; b < B; ++b) acc += part[(size_t)b * C + c];
+    if (in_range(c, (size_t)C)) du[c] = acc;
 }
 
 cudaError_t wkv6_du_reduce_launch(int B, int C, const float *part, float *du, cudaStream_t stream) {

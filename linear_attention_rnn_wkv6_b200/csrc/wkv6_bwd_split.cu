@@ -96,14 +96,16 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
 
 // Ask L2 for the chunk's rows of `out` (32 tokens x this head's 256 bytes, two
 // 128-byte lines each) that a later phase of the chunk reads back and adds to;
-// threads 64 .. 127 issue one line each.
+// threads 64 .. 127 issue one line each.  `out` holds n = B*T*C floats; the debug
+// build checks the line's index against it like a store.
 __device__ __forceinline__ void prefetch_rows(const float *out, int b, int T, int C, int cbase, int c,
-                                              int tid, int dir) {
+                                              int tid, int dir, size_t n) {
     if (tid < 64) return;
     const int p = (tid - 64) >> 1;
     if (c * kBL + p >= T) return;
     const int t = dir > 0 ? c * kBL + p : T - 1 - (c * kBL + p);
-    prefetch_l2(out + ((size_t)b * T + t) * C + cbase + 32 * (tid & 1));
+    const size_t off = ((size_t)b * T + t) * C + cbase + 32 * (tid & 1);
+    if (in_range_vec(off, 32, n)) prefetch_l2(out + off);
 }
 
 // no-swizzle K-major descriptor of a 32-row chunk matrix (units of 8 columns, 512 B apart)
@@ -328,8 +330,8 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
         }
         for (int c = 0; c < nch; ++c) {
             if (!causal) {   // this pass adds to dr and dw: start their reads from HBM now
-                prefetch_rows(prm.dr, b, T, C, cbase, c, tid, dir);
-                prefetch_rows(prm.dw, b, T, C, cbase, c, tid, dir);
+                prefetch_rows(prm.dr, b, T, C, cbase, c, tid, dir, nBTC);
+                prefetch_rows(prm.dw, b, T, C, cbase, c, tid, dir, nBTC);
             }
             // ================= transform =================
             float s0, s1, a0, a1;
@@ -766,10 +768,11 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
         for (int c = nch - 1; c >= 0; --c) {
             const bool first = c == nch - 1;   // no adjoint from later chunks yet
             // rows this chunk reads back and adds to: start their reads from HBM now
-            prefetch_rows(prm.dw, b, T, C, cbase, c, tid, dir);
+            // (RWKV-5 reads no dw back: there dw is the [C] result of the last kernel)
+            if (!STAT) prefetch_rows(prm.dw, b, T, C, cbase, c, tid, dir, nBTC);
             if (pass > 0) {
-                prefetch_rows(prm.dk, b, T, C, cbase, c, tid, dir);
-                prefetch_rows(prm.dv, b, T, C, cbase, c, tid, dir);
+                prefetch_rows(prm.dk, b, T, C, cbase, c, tid, dir, nBTC);
+                prefetch_rows(prm.dv, b, T, C, cbase, c, tid, dir, nBTC);
             }
             // ================= transform =================
             float s0, s1, a0, a1;
@@ -1164,9 +1167,21 @@ namespace {
 __global__ void wkv5_dw_total_kernel(int B, int C, const double *__restrict__ part, float *__restrict__ dw) {
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= C) return;
+    // eight batches' loads in flight at a time; the additions stay in increasing b
     double acc = 0.0;
-    for (int b = 0; b < B; ++b) acc += part[(size_t)b * C + c] + part[((size_t)B + b) * C + c];
-    dw[c] = (float)(-acc);
+    int b = 0;
+    for (; b + 8 <= B; b += 8) {
+        double x[8], z[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            x[e] = part[(size_t)(b + e) * C + c];
+            z[e] = part[((size_t)B + b + e) * C + c];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc += x[e] + z[e];
+    }
+    for (; b < B; ++b) acc += part[(size_t)b * C + c] + part[((size_t)B + b) * C + c];
+    if (in_range(c, (size_t)C)) dw[c] = (float)(-acc);
 }
 }  // namespace
 

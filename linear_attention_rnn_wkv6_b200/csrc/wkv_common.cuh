@@ -134,9 +134,9 @@ template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // Index checks of the debug build.  Built with -DWKV_DEVICE_CHECKS=1
-// (libwkv_debug.so), every global store of the kernels first checks its element
-// index against the size of the array it writes; an index out of range skips the
-// store and records WKV_FAULT_INDEX in the fault word (the kernel goes on; nothing
+// (libwkv_debug.so), every global store of the kernels (and every L2 prefetch of
+// an output row) first checks its element index against the size of the array it
+// writes; an index out of range skips the access and records WKV_FAULT_INDEX in the fault word (the kernel goes on; nothing
 // traps).  In the other builds the check is the constant true and compiles away.
 #ifndef WKV_DEVICE_CHECKS
 #define WKV_DEVICE_CHECKS 0

@@ -1,5 +1,6 @@
 """The debug build (libwkv_debug.so, -DWKV_DEVICE_CHECKS=1): every global store of
-every kernel checks its index against the size of the array it writes, and every
+every kernel (and every L2 prefetch of an output row) checks its index against the
+size of the array it writes, and every
 entry point waits for its kernels and returns WKV_ERR_DEVICE_CHECK when a check
 failed (the store is skipped; nothing traps).  compute-sanitizer is not available
 on this pool; these checks and the tests' guard bands take its place.
