@@ -40,8 +40,10 @@ def f32_path(request):
         yield request.param
 
 
-FWD_SHAPES = [  # (B, T, H): several 32-token chunks, ragged tails, T < chunk, single token
-    (1, 1, 1), (1, 2, 1), (2, 31, 2), (1, 32, 1), (1, 33, 3), (2, 65, 2), (3, 100, 1), (1, 196, 4),
+FWD_SHAPES = [  # (B, T, H): several 32-token chunks, ragged tails, T < chunk, single token; 16, 17
+    # and 48 sit on the register recurrence's 16-token stage boundaries
+    (1, 1, 1), (1, 2, 1), (1, 16, 1), (2, 17, 2), (2, 31, 2), (1, 32, 1), (1, 33, 3), (1, 48, 1), (2, 65, 2),
+    (3, 100, 1), (1, 196, 4),
 ]
 
 
