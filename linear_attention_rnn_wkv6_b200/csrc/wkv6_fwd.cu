@@ -1,4 +1,7 @@
-// wkv6_fwd.cu -- RWKV-6 WKV forward (causal and bidirectional) for sm_100a.
+// wkv6_fwd.cu -- RWKV-6 WKV forward (causal and bidirectional) for sm_100a: the
+// first register-recurrence kernel, which the test build (WKV_RECURRENCE_PATHS)
+// runs for the bf16 causal forward and the fused fp32 forwards; every other
+// recurrence-form forward runs the pipelined kernel of wkv6_fwd_pipe.cu.
 //
 // Operation (per batch b, head h; N = 64; d_t = exp(ew_t)):
 //   causal : y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),  S_t = diag(d_t) S_{t-1} + k_t^T v_t

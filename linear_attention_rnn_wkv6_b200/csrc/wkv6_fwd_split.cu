@@ -1,7 +1,7 @@
 // wkv6_fwd_split.cu -- RWKV-6 fp32 forward (causal and bidirectional) on the
 // 5th-generation tensor cores, with every operand split into three bf16 terms.
 //
-// Same operation as the fp32 recurrence in wkv6_fwd.cu:
+// Same operation as the fp32 register recurrences (wkv6_fwd_pipe.cu, wkv6_fwd.cu):
 //   y_t = r_t (S_{t-1} + diag(u) k_t^T v_t),   S_t = diag(d_t) S_{t-1} + k_t^T v_t,
 // and, bidirectional ("How Custom CUDA Kernels (wkv6_cuda.cu) ...", Future-to-Past
 // Pass), the same sweep run from the last token back to the first with no bonus,

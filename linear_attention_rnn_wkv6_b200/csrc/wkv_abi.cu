@@ -164,7 +164,7 @@ int bwd_common(bool bf16, int B, int T, int C, int H, int bidirectional, const v
 }
 
 // w5 (RWKV-5): static per-channel decay rate [C]; then w is ignored (pass w5 for
-// the argument checks) and the recurrence kernel runs with the constant log-decay.
+// the argument checks) and the register recurrence runs with the constant log-decay.
 // fused: decay prologue and norm/gate epilogue of wkv6_fwd_fused (fp32 kernels).
 struct Fused {
     const float *wb, *g, *gn_w, *gn_b;
