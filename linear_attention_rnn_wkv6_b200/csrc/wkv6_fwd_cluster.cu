@@ -44,7 +44,11 @@ using namespace tc;
 namespace {
 
 constexpr int kCw = 8;                   // CTAs (chunks) per cluster
-constexpr int kClusterMaxHeads = 32;     // at most this many (b, h) units: one cluster each
+// at most this many (b, h) units, one cluster each (measured crossover with the chunk
+// chain at T = 196: causal 24 units 34.8 against 36.9 us, 32 units 47.2 against 36.9 us;
+// bidirectional 36 units 59.4 against 69.6 us, 48 units 75.8 against 70.6 us)
+constexpr int kClusterMaxUnitsCausal = 24;
+constexpr int kClusterMaxUnitsBidir = 36;
 constexpr int kCL = 32;                  // tokens per chunk
 constexpr int kCNT = 3;                  // bf16 terms per operand
 constexpr int kCNP = 6;                  // products per contraction
@@ -697,10 +701,10 @@ cudaError_t launch_cluster(const float *r, const float *k, const float *v, const
 }
 }  // namespace
 
-bool wkv6_fwd_cluster_fits(int B, int T, int H) {
+bool wkv6_fwd_cluster_fits(int B, int T, int H, bool bidir) {
     // every chunk in one cluster, and few enough (b, h) that one CTA per SM and chunk
     // beats carrying the state chunk by chunk (the chain of wkv6_fwd_split.cu)
-    return T <= kCw * kCL && (long long)B * H <= kClusterMaxHeads;
+    return T <= kCw * kCL && (long long)B * H <= (bidir ? kClusterMaxUnitsBidir : kClusterMaxUnitsCausal);
 }
 
 cudaError_t wkv6_fwd_cluster_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,

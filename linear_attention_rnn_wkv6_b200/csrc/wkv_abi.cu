@@ -193,7 +193,7 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
         return launched(wkv6_fwd_tc_launch(mr, mk, mv, mw, my, prm, reinterpret_cast<cudaStream_t>(stream)));
     }
     if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && fused == nullptr && kTensorCorePaths &&
-        wkv6_fwd_cluster_fits(B, T, H)) {
+        wkv6_fwd_cluster_fits(B, T, H, bidir)) {
         // short sequence, few heads: every chunk of a (b, h) at once, in one cluster
         FwdParams prm{B, T, C, H, u, y};
         return launched(wkv6_fwd_cluster_launch(bidir, static_cast<const float *>(r), static_cast<const float *>(k),

@@ -53,8 +53,9 @@ cudaError_t wkv6_fwd_split_launch(bool bidir, const float *r, const float *k, co
                                   const FwdParams &prm, cudaStream_t stream);
 // fp32 causal or bidirectional forward for short sequences and few heads: one
 // thread-block cluster per (b, h), one chunk per CTA, the chunk states exchanged
-// through distributed shared memory.  fits: whether (B, T, H) is such a problem.
-bool wkv6_fwd_cluster_fits(int B, int T, int H);
+// through distributed shared memory.  fits: whether (B, T, H) is such a problem for
+// the causal or the bidirectional form.
+bool wkv6_fwd_cluster_fits(int B, int T, int H, bool bidir);
 cudaError_t wkv6_fwd_cluster_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
                                     const FwdParams &prm, cudaStream_t stream);
 // fp32 causal or bidirectional forward as a register recurrence: four warps hold a

@@ -58,10 +58,11 @@ def test_wkv6_fwd_f32_small(B, T, H, bidir, f32_path):
     assert _rel(y, ref) <= gc.TOL_F32_FWD
 
 
-# The product build runs problems with T <= 256 and at most 32 (b, h) units on the
-# cluster kernel (every chunk at once) and the rest on the chunk-chain kernel; these
-# shapes keep the chain kernel's small and ragged cases covered as well.
-CHAIN_SHAPES = [(5, 33, 7), (6, 100, 6), (1, 257, 2), (3, 31, 11)]
+# The product build runs problems with T <= 256 and at most 24 (causal) or 36
+# (bidirectional) (b, h) units on the cluster kernel (every chunk at once) and the rest
+# on the chunk-chain kernel; these shapes keep the chain kernel's small and ragged
+# cases covered as well, and the cluster kernel's largest unit counts.
+CHAIN_SHAPES = [(5, 33, 7), (6, 100, 6), (1, 257, 2), (3, 31, 11), (6, 196, 4), (9, 70, 4)]
 
 
 @pytest.mark.parametrize("B,T,H", CHAIN_SHAPES)
