@@ -46,7 +46,8 @@ WORKLOAD_NAME = ("wkv-hot-path step: wkv4_fwd B8xT1024xC768 f32 + wkv6_bidir_fwd
 # the causal fp32 forward at the bidirectional workload's shape, and the NEXT rows.
 EXTRA_WORKLOADS = ["wkv6_causal_f32_b1t196h4", "wkv6_causal_f32_b32t196h12", "wkv6_decode_f32_b512h32",
                    "wkv6_bidir_bwd_bf16_b32t196h12", "wkv4_bwd_f32_b8t1024c768", "wkv5_causal_bf16_b8t4096h32",
-                   "wkv5_bwd_f32_b32t196h12", "wkv6_bidir_fused_f32_b32t196h12"]
+                   "wkv5_bwd_f32_b32t196h12", "wkv6_bidir_fused_f32_b32t196h12", "wkv6_state_f32_b32t196h12",
+                   "wkv5_causal_f32_b32t196h12"]
 STEP_WORKLOADS = ["wkv4_f32_b8t1024c768", "wkv6_bidir_f32_b32t196h12", "wkv6_causal_bf16_b8t4096h32",
                   "wkv6_bidir_bwd_f32_b32t196h12"]
 N = 64
@@ -85,6 +86,10 @@ ALG = {
     "wkv5_bwd_f32_b32t196h12": dict(bytes_per_unit=7 * N * 4, flops_per_unit=14 * N * N),
     # fused forward (tensor-core kernel): r, k, v, ww and the gate in, the normalised and gated output out
     "wkv6_bidir_fused_f32_b32t196h12": dict(bytes_per_unit=6 * N * 4, flops_per_unit=10 * N * N),
+    # state in/out: the two N x N states of a (b, h) spread over its T = 196 tokens
+    "wkv6_state_f32_b32t196h12": dict(bytes_per_unit=5 * N * 4 + 2 * N * N * 4 / 196, flops_per_unit=5 * N * N),
+    # RWKV-5 fp32: r, k, v in, y out (w is [C])
+    "wkv5_causal_f32_b32t196h12": dict(bytes_per_unit=4 * N * 4, flops_per_unit=5 * N * N),
 }
 ENTRY = {"wkv6_causal_f32_b1t196h4": "wkv6_fwd", "wkv6_causal_f32_b32t196h12": "wkv6_fwd",
          "wkv4_f32_b8t1024c768": "wkv4_fwd", "wkv6_bidir_f32_b32t196h12": "wkv6_bidir_fwd",
@@ -180,7 +185,9 @@ def uses_tensor_cores(name: str, library: str = "default") -> bool:
     """Whether the workload's entry point runs a chunked tensor-core form in that build
     (RWKV-4 and the decode step run on the CUDA cores in every build; the test build
     runs every RWKV-6 and RWKV-5 entry point on its recurrence kernels)."""
-    return library == "default" and not name.startswith("wkv4") and "decode" not in name
+    # the fp32 forwards with a state or a static decay run the register recurrence in every build
+    register_recurrence = name.startswith("wkv6_state") or name.startswith("wkv5_causal_f32")
+    return library == "default" and not name.startswith("wkv4") and "decode" not in name and not register_recurrence
 
 
 def kernel_source_hash() -> str:
@@ -368,6 +375,10 @@ class DeviceWorkload:
         if self.kind == "wkv6_decode":
             # the recurrent state stays resident on the device (updated in place every step)
             self.state = dev(synth.make_state(x.B, x.H, seed=1000 * rank + 1))
+        if self.kind == "wkv6_fwd_state":
+            # the initial state is an input resident on the device; the final state an output
+            self.state = dev(synth.make_state(x.B, x.H, seed=1000 * rank + 1))
+            self.outputs.append(torch.empty((x.B, x.H, 64, 64), device="cuda"))
         self.units = units_of(name, x)
         self.tokens = tokens_of(x)
 
@@ -409,6 +420,10 @@ class DeviceWorkload:
         elif self.kind == "wkv6_decode":
             # [B,1,C] token tensors are the [B,C] arrays the step reads
             wkv.wkv6_decode(x.B, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], self.state, o[0], s)
+        elif self.kind == "wkv6_fwd_state":
+            wkv.wkv6_fwd_state(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], self.state, o[0], o[1], s)
+        elif self.kind == "wkv5_fwd":
+            wkv.wkv5_fwd(x.B, x.T, x.C, x.H, i["r"], i["k"], i["v"], i["w"], i["u"], o[0], s)
         else:
             raise ValueError(self.kind)
         if self.split and self.kind in ("wkv6_bwd_bidir", "wkv4_bwd"):

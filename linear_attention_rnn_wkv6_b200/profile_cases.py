@@ -82,6 +82,10 @@ def make_case(spec: str):
     if kind == "wkv6_decode":
         state = _dev(synth.make_state(x.B, x.H, seed=0))
         return label, lambda: wkv.wkv6_decode(x.B, x.C, x.H, *ins, state, y)
+    if kind == "wkv6_fwd_state":
+        s0 = _dev(synth.make_state(x.B, x.H, seed=0))
+        sT = torch.empty(x.B, x.H, 64, 64, device="cuda")
+        return label, lambda: wkv.wkv6_fwd_state(x.B, x.T, x.C, x.H, *ins, s0, y, sT)
     fn = getattr(wkv, kind)
     return label, lambda: fn(x.B, x.T, x.C, x.H, *ins, y)
 

@@ -319,6 +319,10 @@ WORKLOADS = {
     "wkv5_bwd_f32_b32t196h12": ("wkv5_bwd", dict(B=32, T=196, H=12, with_dy=True)),
     # bidirectional RWKV-6 forward with the decay prologue and the group-norm/gate epilogue, fp32
     "wkv6_bidir_fused_f32_b32t196h12": ("wkv6_fwd_fused", dict(B=32, T=196, H=12, bidir=True)),
+    # causal RWKV-6 forward from an initial state (make_state), final state out, fp32
+    "wkv6_state_f32_b32t196h12": ("wkv6_fwd_state", dict(B=32, T=196, H=12)),
+    # RWKV-5 (static per-channel decay) forward, fp32, on the patch-sequence shape
+    "wkv5_causal_f32_b32t196h12": ("wkv5_fwd", dict(B=32, T=196, H=12)),
 }
 
 
