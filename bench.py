@@ -96,7 +96,8 @@ ENTRY = {"wkv6_causal_f32_b1t196h4": "wkv6_fwd", "wkv6_causal_f32_b32t196h12": "
          "wkv6_causal_bf16_b8t4096h32": "wkv6_fwd_bf16", "wkv6_bidir_bwd_f32_b32t196h12": "wkv6_bwd",
          "wkv6_decode_f32_b512h32": "wkv6_decode", "wkv6_bidir_bwd_bf16_b32t196h12": "wkv6_bwd_bf16",
          "wkv4_bwd_f32_b8t1024c768": "wkv4_bwd", "wkv5_causal_bf16_b8t4096h32": "wkv5_fwd_bf16",
-         "wkv5_bwd_f32_b32t196h12": "wkv5_bwd", "wkv6_bidir_fused_f32_b32t196h12": "wkv6_fwd_fused"}
+         "wkv5_bwd_f32_b32t196h12": "wkv5_bwd", "wkv6_bidir_fused_f32_b32t196h12": "wkv6_fwd_fused",
+         "wkv6_state_f32_b32t196h12": "wkv6_fwd_state", "wkv5_causal_f32_b32t196h12": "wkv5_fwd"}
 FLUSH_BYTES = 512 << 20   # an L2 flush write; working sets below this get one before every step
 
 LAUNCHES = {"wkv6_causal_f32_b1t196h4": 1, "wkv6_causal_f32_b32t196h12": 1, "wkv4_f32_b8t1024c768": 1, "wkv6_bidir_f32_b32t196h12": 1, "wkv6_causal_bf16_b8t4096h32": 1,
@@ -104,7 +105,7 @@ LAUNCHES = {"wkv6_causal_f32_b1t196h4": 1, "wkv6_causal_f32_b32t196h12": 1, "wkv
             "wkv6_decode_f32_b512h32": 1, "wkv6_bidir_bwd_bf16_b32t196h12": 3,
             "wkv4_bwd_f32_b8t1024c768": 2, "wkv5_causal_bf16_b8t4096h32": 1,
             "wkv5_bwd_f32_b32t196h12": 4,   # S and G kinds with the static decay, du reduction, dw total
-            "wkv6_bidir_fused_f32_b32t196h12": 1}
+            "wkv6_bidir_fused_f32_b32t196h12": 1, "wkv6_state_f32_b32t196h12": 1, "wkv5_causal_f32_b32t196h12": 1}
 
 
 def units_of(name: str, x) -> int:

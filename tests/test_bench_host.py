@@ -68,3 +68,11 @@ def test_every_workload_constructs_on_the_host(monkeypatch):
         two = bench.DeviceWorkload(name, 1, 2)
         assert one.units > 0 and one.tokens > 0 and one.footprint() > 0, name
         assert two.units == one.units and two.tokens == one.tokens, name   # weak scaling: B per rank fixed
+
+
+def test_every_workload_has_its_tables():
+    """Each workload bench.py can time has its algorithmic work, entry point and
+    launch count, and a synthetic recipe."""
+    for name in bench.STEP_WORKLOADS + bench.EXTRA_WORKLOADS:
+        assert name in bench.ALG and name in bench.ENTRY and name in bench.LAUNCHES, name
+        assert name in synth.WORKLOADS, name
