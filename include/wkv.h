@@ -135,8 +135,9 @@ int wkv6_bidir_fwd(int B, int T, int C, int H, const float *r, const float *k, c
  * call's sT as the second call's s0 gives the same y and final state as one call
  * on [0, T) (up to fp32 rounding).  Errors: as wkv6_fwd, plus WKV_ERR_ALIGN for a
  * misaligned s0 or sT and WKV_ERR_TOO_LARGE when B*H*N*N >= 2^31.
- * Algorithm (every build): the token-by-token recurrence, with the state held in
- * registers by four warps per (b, h) and the inputs staged by a fifth.
+ * Algorithm: the chunked tensor-core form of wkv6_fwd, with s0 loaded into tensor
+ * memory before the first chunk and the state stored after the last.  (In the test
+ * build, the token-by-token recurrence.)
  */
 int wkv6_fwd_state(int B, int T, int C, int H, const float *r, const float *k, const float *v,
                    const float *w, const float *u, const float *s0, float *y, float *sT,
@@ -265,7 +266,8 @@ int wkv6_fwd_fused(int B, int T, int C, int H, int bidirectional, const float *r
  *   r, k, v, y : [B,T,C] float, y overwritten;  w, u : [C] float, w >= 0
  *   (state row i of head h decays by exp(-w[h*N + i]) per token).
  * Same sizes, pointer rules, stream semantics and errors as wkv6_fwd.
- * Algorithm (every build): the register recurrence of wkv6_fwd_state with the
+ * Algorithm (every build): the token-by-token recurrence, the state held in
+ * registers by four warps per (b, h) and the inputs staged by a fifth, with the
  * constant log-decay; no w tensor is read.
  */
 int wkv5_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,

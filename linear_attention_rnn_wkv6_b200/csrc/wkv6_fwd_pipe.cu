@@ -43,9 +43,10 @@
 //   (made by the same lane): one addition per element, so the result is the
 //   same whatever the timing.
 // * RWKV-5 (static decay, FwdParams::w5): the transform warp uses -w5 for every
-//   token inside [0, T) and the w tile is not loaded.  Initial and final states
-//   (FwdParams::s0, sT, causal only): the scaled state equals the true state at
-//   every stage boundary.
+//   token inside [0, T) and the w tile is not loaded; this is wkv5_fwd in every
+//   build.  Initial and final states (FwdParams::s0, sT, causal only; wkv6_fwd_state
+//   in the test build): the scaled state equals the true state at every stage
+//   boundary.
 #include "wkv_launch.cuh"
 
 namespace wkv {

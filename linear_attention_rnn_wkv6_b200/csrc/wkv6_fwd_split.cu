@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
     uint32_t ph_m1 = 0, ph_p = 0;
     bool ok = true;
     constexpr int ndir = BIDIR ? 2 : 1;
+    const bool has_s0 = !BIDIR && !FUSED && prm.s0 != nullptr;   // wkv6_fwd_state
     load_chunk(BIDIR ? -1 : 1, 0);
 
     for (int di = 0; di < ndir && ok; ++di) {
@@ -247,8 +248,41 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
         const bool bonus = dir > 0;
         const bool accumulate_y = BIDIR && di == 1;    // the causal sweep adds to y
         const bool norm = FUSED && (!BIDIR || di == 1);  // the last sweep: norm/gate epilogue
-        // S = 0 at the start of every sweep
-        {
+        // S = 0 at the start of every sweep, or (causal, wkv6_fwd_state) the initial state:
+        // lanes 0..15 of every warp own row i = trow; S_in's three-term copy as the epilogue
+        // writes it
+        if (has_s0) {
+            float srow[64];
+            const float *src = prm.s0 + ((size_t)b * H + h) * kHead * kHead + (size_t)trow * kHead;
+#pragma unroll
+            for (int g = 0; g < 16; ++g) {
+                const float4 x4 = row_lane ? __ldg(reinterpret_cast<const float4 *>(src) + g)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                srow[4 * g] = x4.x;
+                srow[4 * g + 1] = x4.y;
+                srow[4 * g + 2] = x4.z;
+                srow[4 * g + 3] = x4.w;
+            }
+            float t32[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) t32[e] = srow[32 * half + e];
+                tmem_st32(tS + lane_off + 32 * half, t32);
+            }
+            tmem_wait_st();
+            if (row_lane) {
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    uint4 w0, w1, w2;
+                    split8(srow + 8 * g, w0, w1, w2);
+                    const uint32_t o = swz(trow, 8 * g);
+                    st_u128(sm.Sin[0], o, w0);
+                    st_u128(sm.Sin[1], o, w1);
+                    st_u128(sm.Sin[2], o, w2);
+                }
+            }
+        } else {
             float z[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) z[e] = 0.f;
@@ -399,7 +433,7 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                         for (int q = 0; q < kNP; ++q)
                             mma_bf16(tY, dadd(dA, prod_a(q) * kApB + 1024 * ks), dadd(dV, prod_b(q) * kTokB + 2048 * ks),
                                      kIdAV, ks > 0 || q > 0);
-                    if (c > 0) {
+                    if (c > 0 || has_s0) {
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
@@ -606,6 +640,27 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
             fence_before_sync();
             __syncthreads();
             fence_after_sync();
+        }
+    }
+    if (ok && !BIDIR && !FUSED && prm.sT != nullptr) {
+        // wkv6_fwd_state: every chunk's epilogue left S_out = diag(exp(Lam_L)) (S_in + Kt^T V)
+        // in TMEM, and tokens past T were zero (k = v = 0, log-decay 0): the state S_{T-1}
+        const size_t nstate = (size_t)prm.B * H * kHead * kHead;
+        float *dst = prm.sT + ((size_t)b * H + h) * kHead * kHead + (size_t)trow * kHead;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float t32[32];
+            tmem_ld32(tS + lane_off + 32 * half, t32);
+            tmem_wait_ld();
+            if (row_lane) {
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const size_t o = ((size_t)b * H + h) * kHead * kHead + (size_t)trow * kHead + 32 * half + 4 * g;
+                    if (in_range_vec(o, 4, nstate))
+                        *reinterpret_cast<float4 *>(dst + 32 * half + 4 * g) =
+                            make_float4(t32[4 * g], t32[4 * g + 1], t32[4 * g + 2], t32[4 * g + 3]);
+                }
+            }
         }
     }
     if (!ok && (tid == 0 || tid == 32)) {

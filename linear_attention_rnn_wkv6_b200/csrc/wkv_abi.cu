@@ -200,10 +200,13 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
                                                 static_cast<const float *>(v), static_cast<const float *>(w), prm,
                                                 reinterpret_cast<cudaStream_t>(stream)));
     }
-    if (!bf16 && s0 == nullptr && sT == nullptr && w5 == nullptr && kTensorCorePaths) {
+    if (!bf16 && w5 == nullptr && kTensorCorePaths) {
         // the chunked form (faster than the register recurrence at these sizes), with
-        // the decay prologue and norm/gate epilogue when fused
+        // the initial and final states of wkv6_fwd_state, or the decay prologue and
+        // norm/gate epilogue when fused
         FwdParams prm{B, T, C, H, u, y};
+        prm.s0 = s0;
+        prm.sT = sT;
         if (fused != nullptr) {
             prm.wb = fused->wb;
             prm.g = fused->g;
@@ -226,8 +229,8 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
     prm.w5 = w5;
     if (!bf16 && fused == nullptr)
         // fp32 without the fused prologue/epilogue: the register recurrence fed by a
-        // transform warp (in the product build only with an initial or final state or
-        // a static decay, which the chunked forms do not take)
+        // transform warp (in the product build only with a static decay, which the fp32
+        // chunked form does not take)
         return launched(wkv6_fwd_pipe_launch(bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)));
     if (fused != nullptr) {
         prm.wb = fused->wb;
