@@ -186,9 +186,7 @@ def uses_tensor_cores(name: str, library: str = "default") -> bool:
     """Whether the workload's entry point runs a chunked tensor-core form in that build
     (RWKV-4 and the decode step run on the CUDA cores in every build; the test build
     runs every RWKV-6 and RWKV-5 entry point on its recurrence kernels)."""
-    # the fp32 forward with a static decay runs the register recurrence in every build
-    register_recurrence = name.startswith("wkv5_causal_f32")
-    return library == "default" and not name.startswith("wkv4") and "decode" not in name and not register_recurrence
+    return library == "default" and not name.startswith("wkv4") and "decode" not in name
 
 
 def kernel_source_hash() -> str:

@@ -266,9 +266,9 @@ int wkv6_fwd_fused(int B, int T, int C, int H, int bidirectional, const float *r
  *   r, k, v, y : [B,T,C] float, y overwritten;  w, u : [C] float, w >= 0
  *   (state row i of head h decays by exp(-w[h*N + i]) per token).
  * Same sizes, pointer rules, stream semantics and errors as wkv6_fwd.
- * Algorithm (every build): the token-by-token recurrence, the state held in
- * registers by four warps per (b, h) and the inputs staged by a fifth, with the
- * constant log-decay; no w tensor is read.
+ * Algorithm: the chunked tensor-core form of wkv6_fwd with the constant log-decay
+ * in place of the loaded one (no w tensor is read).  (In the test build, the
+ * token-by-token recurrence.)
  */
 int wkv5_fwd(int B, int T, int C, int H, const float *r, const float *k, const float *v, const float *w,
              const float *u, float *y, wkv_stream_t stream);

@@ -42,11 +42,11 @@
 //   part; the causal sweep adds its part with one atomic add onto that store
 //   (made by the same lane): one addition per element, so the result is the
 //   same whatever the timing.
-// * RWKV-5 (static decay, FwdParams::w5): the transform warp uses -w5 for every
-//   token inside [0, T) and the w tile is not loaded; this is wkv5_fwd in every
-//   build.  Initial and final states (FwdParams::s0, sT, causal only; wkv6_fwd_state
-//   in the test build): the scaled state equals the true state at every stage
-//   boundary.
+// * The library built with WKV_RECURRENCE_PATHS runs every non-fused fp32 forward
+//   here.  RWKV-5 (static decay, FwdParams::w5, wkv5_fwd): the transform warp uses
+//   -w5 for every token inside [0, T) and the w tile is not loaded.  Initial and
+//   final states (FwdParams::s0, sT, causal only, wkv6_fwd_state): the scaled state
+//   equals the true state at every stage boundary.
 #include "wkv_launch.cuh"
 
 namespace wkv {

@@ -220,6 +220,11 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
 
     // ---- register prefetch of one chunk: tokens pq..pq+7, channels ch, ch+1
     float2 xr_[8], xk_[8], xv_[8], xw_[8];
+    // RWKV-5 (wkv5_fwd): the static log-decay -w5 of channels ch, ch + 1 at every token
+    // of [0, T); the w argument is then the [C] array w5 and is not read per token
+    const bool stat = !FUSED && prm.w5 != nullptr;
+    const float2 w5ew = stat ? make_float2(-__ldg(prm.w5 + cbase + ch), -__ldg(prm.w5 + cbase + ch + 1))
+                             : make_float2(0.f, 0.f);
     auto time_of = [&](int dir, int c, int p) { return dir > 0 ? c * kSL + p : T - 1 - (c * kSL + p); };
     auto load_chunk = [&](int dir, int c) {
 #pragma unroll
@@ -230,7 +235,7 @@ __global__ void __launch_bounds__(kThr, 3) wkv6_fwd_split_kernel(const float *__
                 xr_[e] = __ldg(reinterpret_cast<const float2 *>(r + o));
                 xk_[e] = __ldg(reinterpret_cast<const float2 *>(k + o));
                 xv_[e] = __ldg(reinterpret_cast<const float2 *>(v + o));
-                xw_[e] = __ldg(reinterpret_cast<const float2 *>(w + o));
+                xw_[e] = stat ? w5ew : __ldg(reinterpret_cast<const float2 *>(w + o));
             } else {
                 xr_[e] = xk_[e] = xv_[e] = xw_[e] = make_float2(0.f, 0.f);
             }

@@ -200,13 +200,14 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
                                                 static_cast<const float *>(v), static_cast<const float *>(w), prm,
                                                 reinterpret_cast<cudaStream_t>(stream)));
     }
-    if (!bf16 && w5 == nullptr && kTensorCorePaths) {
+    if (!bf16 && kTensorCorePaths) {
         // the chunked form (faster than the register recurrence at these sizes), with
-        // the initial and final states of wkv6_fwd_state, or the decay prologue and
-        // norm/gate epilogue when fused
+        // the initial and final states of wkv6_fwd_state, the static decay of wkv5_fwd,
+        // or the decay prologue and norm/gate epilogue when fused
         FwdParams prm{B, T, C, H, u, y};
         prm.s0 = s0;
         prm.sT = sT;
+        prm.w5 = w5;
         if (fused != nullptr) {
             prm.wb = fused->wb;
             prm.g = fused->g;
@@ -228,9 +229,8 @@ int fwd_common(bool bf16, bool bidir, int B, int T, int C, int H, const void *r,
     prm.sT = sT;
     prm.w5 = w5;
     if (!bf16 && fused == nullptr)
-        // fp32 without the fused prologue/epilogue: the register recurrence fed by a
-        // transform warp (in the product build only with a static decay, which the fp32
-        // chunked form does not take)
+        // the test build's fp32 forwards without the fused prologue/epilogue: the
+        // register recurrence fed by a transform warp
         return launched(wkv6_fwd_pipe_launch(bidir, mr, mk, mv, mw, prm, reinterpret_cast<cudaStream_t>(stream)));
     if (fused != nullptr) {
         prm.wb = fused->wb;

@@ -49,7 +49,8 @@ cudaError_t wkv6_fwd_tc_launch(const CUtensorMap &mr, const CUtensorMap &mk, con
                                cudaStream_t stream);
 // fp32 causal or bidirectional forward on the tensor cores (split-bf16 operands);
 // r, k, v, w are [B][T][C] fp32 device pointers, 8-byte aligned.  Causal and not
-// fused: prm.s0 / prm.sT, when set, are the initial and final states.
+// fused: prm.s0 / prm.sT, when set, are the initial and final states; prm.w5, when
+// set, is the static decay rate [C] (w is then not read).
 cudaError_t wkv6_fwd_split_launch(bool bidir, const float *r, const float *k, const float *v, const float *w,
                                   const FwdParams &prm, cudaStream_t stream);
 // fp32 causal or bidirectional forward for short sequences and few heads: one
