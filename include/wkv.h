@@ -27,9 +27,9 @@
  * forms where an entry point has one.  The same sources built with
  * -DWKV_RECURRENCE_PATHS=1 give libwkv_recurrence.so, a test and comparison
  * build with this same ABI in which wkv6_fwd, wkv6_fwd_bf16, wkv6_bidir_fwd,
- * wkv6_fwd_fused, wkv5_fwd_bf16, wkv6_bwd, wkv6_bwd_bf16 and wkv5_bwd run the
- * token-by-token recurrence kernels instead (the kernels wkv6_fwd_state,
- * wkv5_fwd and wkv6_bwd_noalloc use in both builds).  Results agree within the
+ * wkv6_fwd_fused, wkv6_fwd_state, wkv5_fwd, wkv5_fwd_bf16, wkv6_bwd,
+ * wkv6_bwd_bf16 and wkv5_bwd run the token-by-token recurrence kernels instead
+ * (the kernels wkv6_bwd_noalloc uses in both builds).  Results agree within the
  * tolerances stated below; nothing is selected at run time.  A third build,
  * libwkv_debug.so (-DWKV_DEVICE_CHECKS=1), is libwkv.so with an index check on
  * every global store of every kernel (and every L2 prefetch of an output row):
