@@ -35,6 +35,8 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kCh = 16;     // channels per CTA
 constexpr int kSeg = 32;    // segments of T per channel
+constexpr int kBat = 8;     // tokens whose loads are issued together (summary passes)
+constexpr int kBatR = 4;    // the same for the reruns, which load three or five arrays
 
 __device__ __forceinline__ float ex2(float x) {   // 2^x; -inf gives 0
     float y;
@@ -106,10 +108,22 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
     const float *kr = k + brow, *vr = v + brow, *gr = dy + brow;
     float *dkr = dk + brow, *dvr = dv + brow, *mr = mwork + brow;
 
-    // ---- F1: forward summary of the segment
+    // ---- F1: forward summary of the segment (the loads of kBat tokens issued before
+    // any of them is used; the updates stay in token order)
     Fwd st{0.f, 0.f, -INFINITY};
     if (live)
-        for (int t = t0, o = t0 * C + c; t < t1; ++t, o += C) fwd_update(st, kr[o] * kLog2e, vr[o], w2);
+        for (int t = t0; t < t1; t += kBat) {
+            float kk[kBat], vv[kBat];
+#pragma unroll
+            for (int e = 0; e < kBat; ++e) {
+                const int o = (t + e) * C + c;
+                kk[e] = t + e < t1 ? kr[o] : 0.f;
+                vv[e] = t + e < t1 ? vr[o] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < kBat; ++e)
+                if (t + e < t1) fwd_update(st, kk[e] * kLog2e, vv[e], w2);
+        }
     fsum[seg][ch] = st;
     __syncthreads();
 
@@ -130,24 +144,49 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
     // ---- F3: forward rerun; park y, the scaled g and the exponent m of every step
     st = in;
     if (live)
-        for (int t = t0, o = t0 * C + c; t < t1; ++t, o += C) {
-            if (!in_range((size_t)o, (size_t)T * C)) continue;   // y, g, m parked in this row of dv, dk, mwork
-            const float k2 = kr[o] * kLog2e, vt = vr[o];
-            const float uk = u2 + k2, d = st.p - uk;
-            const float ex = ex2(-fabsf(d));
-            const bool keep = d >= 0.f;
-            const float e1 = keep ? 1.f : ex, e2 = keep ? ex : 1.f;
-            const float den = fmaf(e1, st.b, e2);                 // >= 1
-            dvr[o] = __fdividef(fmaf(e1, st.a, e2 * vt), den);    // y_t
-            dkr[o] = __fdividef(gr[o], den);                      // g_t 2^{m_t}
-            mr[o] = fmaxf(st.p, uk);                              // m_t (log2)
-            fwd_update(st, k2, vt, w2);
+        for (int t = t0; t < t1; t += kBatR) {
+            float kk[kBatR], vv[kBatR], gg[kBatR];
+#pragma unroll
+            for (int e = 0; e < kBatR; ++e) {
+                const int o = (t + e) * C + c;
+                kk[e] = t + e < t1 ? kr[o] : 0.f;
+                vv[e] = t + e < t1 ? vr[o] : 0.f;
+                gg[e] = t + e < t1 ? gr[o] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < kBatR; ++e) {
+                const int o = (t + e) * C + c;
+                if (t + e >= t1) break;
+                if (!in_range((size_t)o, (size_t)T * C)) continue;   // y, g, m parked in this row of dv, dk, mwork
+                const float k2 = kk[e] * kLog2e, vt = vv[e];
+                const float uk = u2 + k2, d = st.p - uk;
+                const float ex = ex2(-fabsf(d));
+                const bool keep = d >= 0.f;
+                const float e1 = keep ? 1.f : ex, e2 = keep ? ex : 1.f;
+                const float den = fmaf(e1, st.b, e2);                 // >= 1
+                dvr[o] = __fdividef(fmaf(e1, st.a, e2 * vt), den);    // y_t
+                dkr[o] = __fdividef(gg[e], den);                      // g_t 2^{m_t}
+                mr[o] = fmaxf(st.p, uk);                              // m_t (log2)
+                fwd_update(st, k2, vt, w2);
+            }
         }
 
     // ---- R1: reverse summary of the segment (sums over its tokens, seen from t0 - 1)
     Rev rs{0.f, 0.f, 0.f, 0.f, -INFINITY};
     if (live)
-        for (int t = t1 - 1, o = (t1 - 1) * C + c; t >= t0; --t, o -= C) rev_update(rs, dkr[o], dvr[o], mr[o], w2);
+        for (int t = t1 - 1; t >= t0; t -= kBat) {
+            float gh[kBat], yy[kBat], mm[kBat];
+#pragma unroll
+            for (int e = 0; e < kBat; ++e) {
+                const int o = (t - e) * C + c;
+                gh[e] = t - e >= t0 ? dkr[o] : 0.f;
+                yy[e] = t - e >= t0 ? dvr[o] : 0.f;
+                mm[e] = t - e >= t0 ? mr[o] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < kBat; ++e)
+                if (t - e >= t0) rev_update(rs, gh[e], yy[e], mm[e], w2);
+        }
     rsum[seg][ch] = rs;
     __syncthreads();
 
@@ -163,18 +202,34 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
     // ---- R3: reverse rerun: dk, dv per token; dw, du per thread
     float dwa = 0.f, dua = 0.f;
     if (live)
-        for (int t = t1 - 1, o = (t1 - 1) * C + c; t >= t0; --t, o -= C) {
-            if (!in_range((size_t)o, (size_t)T * C)) continue;   // dk, dv: this batch row
-            const float gh = dkr[o], yt = dvr[o], m = mr[o];
-            const float k2 = kr[o] * kLog2e, vt = vr[o];
-            const float E = ex2(k2 + ri.q);            // e^{k_s} 2^q
-            const float F = ex2(u2 + k2 - m);          // bonus weight E_ss 2^{-m}
-            const float gb = gh * F;                   // g_s E_ss
-            dvr[o] = fmaf(E, ri.al, gb);
-            dkr[o] = fmaf(E, fmaf(vt, ri.al, -ri.be), gb * (vt - yt));
-            dwa = fmaf(-E, fmaf(vt, ri.al1, -ri.be1), dwa);
-            dua = fmaf(gb, vt - yt, dua);
-            rev_update(ri, gh, yt, m, w2);
+        for (int t = t1 - 1; t >= t0; t -= kBatR) {
+            float gg[kBatR], yy[kBatR], mm[kBatR], kk[kBatR], vv[kBatR];
+#pragma unroll
+            for (int e = 0; e < kBatR; ++e) {
+                const int o = (t - e) * C + c;
+                const bool in = t - e >= t0;
+                gg[e] = in ? dkr[o] : 0.f;
+                yy[e] = in ? dvr[o] : 0.f;
+                mm[e] = in ? mr[o] : 0.f;
+                kk[e] = in ? kr[o] : 0.f;
+                vv[e] = in ? vr[o] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < kBatR; ++e) {
+                const int o = (t - e) * C + c;
+                if (t - e < t0) break;
+                if (!in_range((size_t)o, (size_t)T * C)) continue;   // dk, dv: this batch row
+                const float gh = gg[e], yt = yy[e], m = mm[e];
+                const float k2 = kk[e] * kLog2e, vt = vv[e];
+                const float E = ex2(k2 + ri.q);            // e^{k_s} 2^q
+                const float F = ex2(u2 + k2 - m);          // bonus weight E_ss 2^{-m}
+                const float gb = gh * F;                   // g_s E_ss
+                dvr[o] = fmaf(E, ri.al, gb);
+                dkr[o] = fmaf(E, fmaf(vt, ri.al, -ri.be), gb * (vt - yt));
+                dwa = fmaf(-E, fmaf(vt, ri.al1, -ri.be1), dwa);
+                dua = fmaf(gb, vt - yt, dua);
+                rev_update(ri, gh, yt, m, w2);
+            }
         }
 
     // ---- per-(b, c) partials: sum over the segments in a fixed order
