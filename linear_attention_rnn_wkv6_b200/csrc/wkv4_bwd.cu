@@ -19,10 +19,12 @@
 // into 32 segments.  Phases per thread (segment):
 //   F1/F2  forward segment summary, then the forward state entering the segment
 //   F3     forward rerun: y_t, the scaled g_t and the step's exponent m_t are
-//          parked in dv, dk and the workspace (read back by the same thread)
-//   R1/R2  reverse segment summary of the four sums, then the sums entering the
-//          segment from the right (a segment of length L maps (a, a') to
-//          e^{-Lw} (a, a' + L a) before its own terms are added)
+//          parked in dv, dk and the workspace (read back by the same thread);
+//          the same pass sums the segment's own terms of the four future sums
+//          as seen from t0 - 1 (token t weighs e^{-(t - t0) w}, and (t - t0)
+//          times that in the primed sums), in time order
+//   R2     the sums entering the segment from the right (a segment of length L
+//          maps (a, a') to e^{-Lw} (a, a' + L a) before its own terms are added)
 //   R3     reverse rerun: dk, dv per token, dw and du accumulated per thread,
 //          reduced over the segments into per-(b, c) partials; a second kernel
 //          sums the partials over b in a fixed order (deterministic, no atomics).
@@ -35,7 +37,7 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kCh = 16;     // channels per CTA
 constexpr int kSeg = 32;    // segments of T per channel
-constexpr int kBat = 8;     // tokens whose loads are issued together (summary passes)
+constexpr int kBat = 8;     // tokens whose loads are issued together (the summary pass)
 constexpr int kBatR = 4;    // the same for the reruns, which load three or five arrays
 
 __device__ __forceinline__ float ex2(float x) {   // 2^x; -inf gives 0
@@ -62,6 +64,21 @@ __device__ __forceinline__ void fwd_update(Fwd &s, float k2, float v, float w2) 
     s.a = fmaf(e1, s.a, e2 * v);
     s.b = fmaf(e1, s.b, e2);
     s.p = fmaxf(pd, k2);
+}
+
+// Add a term of the segment summary: x gh 2^{e} (x gh y 2^{e} for beta), weighted by dt in
+// the primed sums, e = -m - dt w2 in log2 units for the token dt steps after the segment's
+// start.
+__device__ __forceinline__ void rev_term(Rev &r, float gh, float y, float m, float dt, float w2) {
+    const float e = fmaf(-dt, w2, -m);
+    const float qn = fmaxf(r.q, e);
+    const float eo = ex2(r.q - qn), en = ex2(e - qn);
+    const float g1 = en * gh, gy = g1 * y;
+    r.al = fmaf(eo, r.al, g1);
+    r.be = fmaf(eo, r.be, gy);
+    r.al1 = fmaf(eo, r.al1, dt * g1);
+    r.be1 = fmaf(eo, r.be1, dt * gy);
+    r.q = qn;
 }
 
 // Include token s (scaled g = gh 2^{-m}, output y) into the future sums.
@@ -141,8 +158,10 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
         in.p = q;
     }
 
-    // ---- F3: forward rerun; park y, the scaled g and the exponent m of every step
+    // ---- F3: forward rerun; park y, the scaled g and the exponent m of every step, and
+    // sum the segment's terms of the future sums (seen from t0 - 1)
     st = in;
+    Rev rs{0.f, 0.f, 0.f, 0.f, -INFINITY};
     if (live)
         for (int t = t0; t < t1; t += kBatR) {
             float kk[kBatR], vv[kBatR], gg[kBatR];
@@ -164,29 +183,17 @@ wkv4_bwd_kernel(int T, int C, const float *__restrict__ k, const float *__restri
                 const bool keep = d >= 0.f;
                 const float e1 = keep ? 1.f : ex, e2 = keep ? ex : 1.f;
                 const float den = fmaf(e1, st.b, e2);                 // >= 1
-                dvr[o] = __fdividef(fmaf(e1, st.a, e2 * vt), den);    // y_t
-                dkr[o] = __fdividef(gg[e], den);                      // g_t 2^{m_t}
-                mr[o] = fmaxf(st.p, uk);                              // m_t (log2)
+                const float yt = __fdividef(fmaf(e1, st.a, e2 * vt), den);   // y_t
+                const float gh = __fdividef(gg[e], den);                     // g_t 2^{m_t}
+                const float m = fmaxf(st.p, uk);                             // m_t (log2)
+                dvr[o] = yt;
+                dkr[o] = gh;
+                mr[o] = m;
+                rev_term(rs, gh, yt, m, (float)(t + e - t0), w2);
                 fwd_update(st, k2, vt, w2);
             }
         }
 
-    // ---- R1: reverse summary of the segment (sums over its tokens, seen from t0 - 1)
-    Rev rs{0.f, 0.f, 0.f, 0.f, -INFINITY};
-    if (live)
-        for (int t = t1 - 1; t >= t0; t -= kBat) {
-            float gh[kBat], yy[kBat], mm[kBat];
-#pragma unroll
-            for (int e = 0; e < kBat; ++e) {
-                const int o = (t - e) * C + c;
-                gh[e] = t - e >= t0 ? dkr[o] : 0.f;
-                yy[e] = t - e >= t0 ? dvr[o] : 0.f;
-                mm[e] = t - e >= t0 ? mr[o] : 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < kBat; ++e)
-                if (t - e >= t0) rev_update(rs, gh[e], yy[e], mm[e], w2);
-        }
     rsum[seg][ch] = rs;
     __syncthreads();
 
