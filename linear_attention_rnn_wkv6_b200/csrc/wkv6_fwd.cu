@@ -56,7 +56,7 @@
 
 namespace wkv {
 
-constexpr float kTheta = 40.0f;  // bound on |L| inside a run (exp(40) ~ 2.4e17)
+[[maybe_unused]] constexpr float kTheta = 40.0f;  // bound on |L| inside a run (exp(40) ~ 2.4e17)
 
 template <typename Tin, int WARPS, int TC>
 struct FwdSmem {
@@ -473,11 +473,11 @@ static cudaError_t launch_fwd(const CUtensorMap &mr, const CUtensorMap &mk, cons
 cudaError_t wkv6_fwd_launch(bool bf16, bool bidir, const CUtensorMap &mr, const CUtensorMap &mk,
                             const CUtensorMap &mv, const CUtensorMap &mw, const FwdParams &prm,
                             cudaStream_t stream) {
-    constexpr int TC = kFwdTC;
     // Reached only in the library built with WKV_RECURRENCE_PATHS: there the bf16
     // causal forward and the fused fp32 forwards run this kernel (the other fp32
-    // forwards run the pipelined recurrence in every build).
+    // forwards run the pipelined recurrence there).
 #if WKV_RECURRENCE_PATHS
+    constexpr int TC = kFwdTC;
     if (bf16) return bidir ? cudaErrorNotSupported : launch_fwd<__nv_bfloat16, 4, TC, false>(mr, mk, mv, mw, prm, stream);
     if (bidir) return launch_fwd<float, 4, TC, true>(mr, mk, mv, mw, prm, stream);
     return launch_fwd<float, 4, TC, false>(mr, mk, mv, mw, prm, stream);
