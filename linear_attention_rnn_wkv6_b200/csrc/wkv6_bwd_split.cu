@@ -699,11 +699,11 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
 
     if (tid == 0) {
-        mbar_init(&sm.bar_m1, 1);
+        mbar_init(&sm.bar_m1, 2);    // A^T and dA^T, committed by two threads
         mbar_init(&sm.bar_k, 1);
         mbar_init(&sm.bar_v, 1);
         mbar_init(&sm.bar_g, 1);
-        mbar_init(&sm.bar_fin, 2);
+        mbar_init(&sm.bar_fin, 3);   // the three issuing threads
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -838,6 +838,25 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
             fence_after_sync();
 
             if (!exact) {
+                // ===== A^T = Kt Q^T (warp 2) and dA^T = V dY^T (warp 3), one accumulator per
+                // issuing thread: issued first, they run while G is rescaled =====
+                if (tid == 64) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tA, bdadd(dKk, bprod_a(q) * kTokB + 32 * ks), bdadd(dQk, bprod_b(q) * kTokB + 32 * ks),
+                                     kIdAT, ks > 0 || q > 0);
+                    mma_commit(&sm.bar_m1);
+                } else if (tid == 96) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                        for (int q = 0; q < kBP; ++q)
+                            mma_bf16(tA + 32, bdadd(dVk, bprod_a(q) * kTokB + 32 * ks),
+                                     bdadd(dYk, bprod_b(q) * kTokB + 32 * ks), kIdAT, ks > 0 || q > 0);
+                    mma_commit(&sm.bar_m1);
+                }
                 // ===== Gt = diag(Gam) G_out in TMEM, and its two-term copy =====
                 if (!first) {
                     float gv[32];
@@ -862,23 +881,15 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                     tmem_st_16x256b_x8(tG + lane_off, gv);
                     tmem_wait_st();
                     fence_proxy_async_smem();
-                    fence_before_sync();
-                    __syncthreads();
-                    fence_after_sync();
                 }
-                // ===== A^T = Kt Q^T, dA^T = V dY^T (warp 0);  G += Q^T dY (warp 1) =====
-                if (tid == 0) {
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-                        for (int q = 0; q < kBP; ++q) {
-                            mma_bf16(tA, bdadd(dKk, bprod_a(q) * kTokB + 32 * ks), bdadd(dQk, bprod_b(q) * kTokB + 32 * ks),
-                                     kIdAT, ks > 0 || q > 0);
-                            mma_bf16(tA + 32, bdadd(dVk, bprod_a(q) * kTokB + 32 * ks),
-                                     bdadd(dYk, bprod_b(q) * kTokB + 32 * ks), kIdAT, ks > 0 || q > 0);
-                        }
-                    mma_commit(&sm.bar_m1);
-                } else if (tid == 32) {
+                ok = mbar_wait_bounded(&sm.bar_m1, ph);
+                fence_before_sync();
+                ok = __syncthreads_and(ok);
+                if (!ok) break;
+                fence_after_sync();
+                // ===== G += Q^T dY (warp 2, beside the masks of warps 0 and 1), onto the
+                // rescaled G; waited for with dV =====
+                if (tid == 64) {
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
@@ -887,10 +898,6 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                                      kIdG, true);
                     mma_commit(&sm.bar_g);
                 }
-                ok = mbar_wait_bounded(&sm.bar_m1, ph);
-                ok = __syncthreads_and(ok);
-                if (!ok) break;
-                fence_after_sync();
                 // ===== masks: A'^T, dA'^T = strict-upper (tau > s) of A^T, dA^T =====
                 if (warp < 2) {
                     float a[32];
@@ -1128,7 +1135,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
         if (tid < kHead && in_range((size_t)b * C + cbase + tid, (size_t)prm.B * C))
             prm.w5_part[((size_t)prm.B + b) * C + cbase + tid] = wx[tid] + wx[kHead + tid];
     }
-    if (!ok && (tid == 0 || tid == 32)) {
+    if (!ok && (tid == 0 || tid == 64 || tid == 96)) {
+        // a wait ran out: let every MMA issued so far (by the three issuing threads) finish
+        // before TMEM is released
         mma_commit(&sm.bar_fin);
         if (tid == 0) mbar_wait_bounded(&sm.bar_fin, 0);
     }
