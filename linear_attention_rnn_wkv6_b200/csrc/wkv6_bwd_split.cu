@@ -84,9 +84,18 @@ __device__ __forceinline__ uint64_t bdadd(uint64_t d, uint32_t bytes) { return d
 
 // Two consecutive inputs (channels ch, ch + 1) as fp32: one 8-byte load for fp32
 // inputs, one 4-byte load of a bf16 pair (exact widening) for bf16 inputs.
-__device__ __forceinline__ float2 ld_pair(const float *p) { return __ldg(reinterpret_cast<const float2 *>(p)); }
-__device__ __forceinline__ float2 ld_pair(const __nv_bfloat16 *p) {
-    const uint32_t x = __ldg(reinterpret_cast<const unsigned int *>(p));
+// Two adjacent channels of one token as loaded: an fp32 pair, or two bf16 values in
+// one word.  The prefetch registers hold them as loaded; they are widened to fp32 (exactly)
+// where the transform reads them, so that nothing waits for a load before then.
+template <typename T> struct RawPair;
+template <> struct RawPair<float> { using type = float2; };
+template <> struct RawPair<__nv_bfloat16> { using type = uint32_t; };
+__device__ __forceinline__ float2 ld_raw(const float *p) { return __ldg(reinterpret_cast<const float2 *>(p)); }
+__device__ __forceinline__ uint32_t ld_raw(const __nv_bfloat16 *p) {
+    return __ldg(reinterpret_cast<const unsigned int *>(p));
+}
+__device__ __forceinline__ float2 widen(float2 x) { return x; }
+__device__ __forceinline__ float2 widen(uint32_t x) {
     return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
 }
 
@@ -288,7 +297,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
     constexpr uint32_t kIdQ1 = idesc_bf16(64, 64, false, true);     // dA' (K) x Kt (MN)
     constexpr uint32_t kIdQ2 = idesc_bf16(64, 64, false, false);    // dY (K) x S_in (K-major, rows i)
 
-    float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    // the next chunk's inputs as loaded (tokens pq .. pq + 7, channels ch, ch + 1)
+    using Raw = typename RawPair<Tin>::type;
+    Raw lr_[8], lk_[8], lv_[8], lw_[8], ld_[8];
     // RWKV-5: the static log-decay of channels ch, ch + 1 at every token
     const float2 w5ew = STAT ? make_float2(-prm.w5[cbase + ch], -prm.w5[cbase + ch + 1]) : make_float2(0.f, 0.f);
     double w5acc = 0.0;   // RWKV-5: this thread's channel's decay-gradient total
@@ -299,14 +310,26 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
             const int p = pq + e;
             if (c * kBL + p < T) {
                 const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
-                xr_[e] = ld_pair(r + o);
-                xk_[e] = ld_pair(k + o);
-                xv_[e] = ld_pair(v + o);
-                xw_[e] = STAT ? w5ew : ld_pair(w + o);
-                xd_[e] = ld_pair(dy + o);
+                lr_[e] = ld_raw(r + o);
+                lk_[e] = ld_raw(k + o);
+                lv_[e] = ld_raw(v + o);
+                if (!STAT) lw_[e] = ld_raw(w + o);
+                ld_[e] = ld_raw(dy + o);
             } else {
-                xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
+                lr_[e] = lk_[e] = lv_[e] = lw_[e] = ld_[e] = Raw{};
             }
+        }
+    };
+    // the current chunk's inputs in fp32; past T every input and the log-decay are zero
+    float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    auto widen_chunk = [&](int c) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            xr_[e] = widen(lr_[e]);
+            xk_[e] = widen(lk_[e]);
+            xv_[e] = widen(lv_[e]);
+            xw_[e] = STAT ? (c * kBL + pq + e < T ? w5ew : make_float2(0.f, 0.f)) : widen(lw_[e]);
+            xd_[e] = widen(ld_[e]);
         }
     };
 
@@ -334,6 +357,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_s_kernel(const Tin *__restr
                 prefetch_rows(prm.dw, b, T, C, cbase, c, tid, dir, nBTC);
             }
             // ================= transform =================
+            widen_chunk(c);
             float s0, s1, a0, a1;
             decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
             // v.dy per token (the bonus scalar of dr, dk and du), reduced over the 64 channels;
@@ -726,7 +750,9 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
     constexpr uint32_t kIdKM = idesc_bf16(64, 64, false, true);    // dA'^T (K) x Q (MN);  A'^T (K) x dY (MN);  Kt (K) x Gt (MN)
     constexpr uint32_t kIdKK = idesc_bf16(64, 64, false, false);   // V (K) x Gt (K-major, rows i)
 
-    float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    // the next chunk's inputs as loaded (tokens pq .. pq + 7, channels ch, ch + 1)
+    using Raw = typename RawPair<Tin>::type;
+    Raw lr_[8], lk_[8], lv_[8], lw_[8], ld_[8];
     // RWKV-5: the static log-decay of channels ch, ch + 1 at every token
     const float2 w5ew = STAT ? make_float2(-prm.w5[cbase + ch], -prm.w5[cbase + ch + 1]) : make_float2(0.f, 0.f);
     double w5acc = 0.0;   // RWKV-5: this thread's channel's decay-gradient total
@@ -737,14 +763,26 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
             const int p = pq + e;
             if (c * kBL + p < T) {
                 const size_t o = ((size_t)b * T + time_of(dir, c, p)) * C + cbase + ch;
-                xr_[e] = ld_pair(r + o);
-                xk_[e] = ld_pair(k + o);
-                xv_[e] = ld_pair(v + o);
-                xw_[e] = STAT ? w5ew : ld_pair(w + o);
-                xd_[e] = ld_pair(dy + o);
+                lr_[e] = ld_raw(r + o);
+                lk_[e] = ld_raw(k + o);
+                lv_[e] = ld_raw(v + o);
+                if (!STAT) lw_[e] = ld_raw(w + o);
+                ld_[e] = ld_raw(dy + o);
             } else {
-                xr_[e] = xk_[e] = xv_[e] = xw_[e] = xd_[e] = make_float2(0.f, 0.f);
+                lr_[e] = lk_[e] = lv_[e] = lw_[e] = ld_[e] = Raw{};
             }
+        }
+    };
+    // the current chunk's inputs in fp32; past T every input and the log-decay are zero
+    float2 xr_[8], xk_[8], xv_[8], xw_[8], xd_[8];
+    auto widen_chunk = [&](int c) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            xr_[e] = widen(lr_[e]);
+            xk_[e] = widen(lk_[e]);
+            xv_[e] = widen(lv_[e]);
+            xw_[e] = STAT ? (c * kBL + pq + e < T ? w5ew : make_float2(0.f, 0.f)) : widen(lw_[e]);
+            xd_[e] = widen(ld_[e]);
         }
     };
 
@@ -775,6 +813,7 @@ __global__ void __launch_bounds__(kBThr, 3) wkv6_bwd_g_kernel(const Tin *__restr
                 prefetch_rows(prm.dv, b, T, C, cbase, c, tid, dir, nBTC);
             }
             // ================= transform =================
+            widen_chunk(c);
             float s0, s1, a0, a1;
             decay_sums(xw_, ds, warp, ch, s0, s1, a0, a1);
             {   // v.dy and sum r u k per token, reduced over the 64 channels
